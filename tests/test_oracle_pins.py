@@ -1,0 +1,358 @@
+"""Pins of the float64 oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: a library
+routine (scipy's Hadamard matrix, scipy's Beta law and quadrature, numpy's
+float16 rounding, torch's bf16/E4M3 conversions, numpy sorting), a closed
+form, a textbook table, the pages' printed numbers, or brute force.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.integrate
+import scipy.linalg
+import scipy.special
+import scipy.stats
+import torch
+
+from oracle import oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# random streams
+# --------------------------------------------------------------------------
+def test_splitmix64_published_first_output():
+    # SplitMix64 seeded with 0: first output is 0xE220A8397B1DCDAF (the
+    # generator's reference implementation, Steele/Lea/Flood 2014).
+    assert O.draw(0, 0, 0) == 0xE220A8397B1DCDAF
+
+
+def test_signs_and_gaussian_statistics():
+    P = O.make_params(128, 2, seed=123)
+    assert set(np.unique(P.signs)) <= {-1, 1}
+    big = O.make_params(1024, 2, seed=7)
+    s = big.S.astype(np.float64).ravel()
+    # bf16-exact entries
+    assert np.all(torch.tensor(s, dtype=torch.float32).to(torch.bfloat16).float().numpy() == s)
+    # iid N(0,1): moments and a Kolmogorov-Smirnov test against scipy's normal law
+    assert abs(s.mean()) < 5 / math.sqrt(s.size)
+    assert abs(s.var() - 1.0) < 5 * math.sqrt(2.0 / s.size) + 2e-5
+    ks = scipy.stats.kstest(s[:200000], "norm")
+    assert ks.pvalue > 1e-4
+    sg = np.concatenate([O.make_params(1024, 2, seed=k, with_S=False).signs for k in range(8)])
+    assert abs(sg.mean()) < 5 / math.sqrt(sg.size)
+
+
+# --------------------------------------------------------------------------
+# rounding to the storage formats
+# --------------------------------------------------------------------------
+def test_fp16_rounding_matches_numpy():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-8, 5, 2000),
+                           [0.0, 65504.0, 6.1e-5, 5.96e-8, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11]])
+    for v in vals:
+        assert O.round_fp16(v) == float(np.float16(v)), v
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(2)
+    vals = (rng.standard_normal(4000) * 10.0 ** rng.integers(-30, 30, 4000)).astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).double().numpy()
+    for v, r in zip(vals.astype(np.float64), ref):
+        assert O.round_bf16(v) == r, v
+
+
+def test_e4m3_rounding_matches_torch():
+    rng = np.random.default_rng(3)
+    vals = (rng.standard_normal(4000) * 10.0 ** rng.uniform(-3, 2.6, 4000)).astype(np.float32)
+    vals = vals[np.abs(vals) < 448.0]
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for v, r in zip(vals.astype(np.float64), ref):
+        assert O.e4m3(v) == int(r), v
+    # saturating beyond the largest finite value, signs kept
+    assert O.e4m3(1e6) == 0x7E and O.e4m3(-1e6) == 0xFE
+    assert O.e4m3_value(0x7E) == 448.0
+
+
+# --------------------------------------------------------------------------
+# rotation R = H D / sqrt(d)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [8, 128])
+def test_rotation_equals_sylvester_matrix(d):
+    P = O.make_params(d, 2, seed=5, with_S=False)
+    H = scipy.linalg.hadamard(d).astype(np.float64)   # natural-order Sylvester
+    R = H @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    rng = np.random.default_rng(d)
+    X = rng.standard_normal((16, d))
+    assert np.allclose(O.rotate(X, P.signs), X @ R.T, atol=1e-12, rtol=0)
+    assert np.allclose(O.rotate_t(X, P.signs), X @ R, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("d", [8, 128, 1024])
+def test_rotation_is_orthogonal(d):
+    P = O.make_params(d, 2, seed=9, with_S=False)
+    E = O.rotate(np.eye(d), P.signs)          # rows: R e_i -> columns of R
+    assert np.allclose(E @ E.T, np.eye(d), atol=1e-12)
+    x = np.random.default_rng(0).standard_normal((4, d))
+    assert np.allclose(np.linalg.norm(O.rotate(x, P.signs), axis=1), np.linalg.norm(x, axis=1),
+                       rtol=1e-13, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Lloyd-Max codebook for the coordinate law of a random unit vector
+# --------------------------------------------------------------------------
+def _coord_law(d):
+    # (T + 1) / 2 ~ Beta((d-1)/2, (d-1)/2) for one coordinate T of a uniform
+    # random unit vector in R^d: an independent library description of f_d.
+    a = (d - 1) / 2.0
+    return scipy.stats.beta(a, a, loc=-1.0, scale=2.0)
+
+
+@pytest.mark.parametrize("d,bits", [(8, 1), (8, 2), (8, 3), (128, 2), (128, 3), (128, 4),
+                                    (1024, 4)])
+def test_codebook_fixed_point_conditions(d, bits):
+    c64, c32, t32 = O.codebook(d, bits)
+    law = _coord_law(d)
+    L = 1 << bits
+    edges = np.concatenate([[-1.0], 0.5 * (c64[:-1] + c64[1:]), [1.0]])
+    for j in range(L):
+        lo, hi = edges[j], edges[j + 1]
+        mass = law.cdf(hi) - law.cdf(lo)
+        mom = scipy.integrate.quad(lambda t: t * law.pdf(t), lo, hi, epsabs=1e-15,
+                                   epsrel=1e-13, limit=400)[0]
+        assert abs(mom / mass - c64[j]) < 1e-10, (j, mom / mass, c64[j])
+    # symmetry, and fp32 boundaries are midpoints of the fp32 levels
+    assert np.all(c32 == -c32[::-1])
+    assert np.all(t32 == ((c32[:-1].astype(np.float64) + c32[1:]) / 2).astype(np.float32))
+    assert np.all(np.diff(c32) > 0)
+
+
+@pytest.mark.parametrize("d", [8, 16, 128, 1024])
+def test_codebook_one_bit_closed_form(d):
+    # b = 1: the levels are +-E|T| = +-Gamma(d/2) / (sqrt(pi) Gamma((d+1)/2))
+    c64, _, _ = O.codebook(d, 1)
+    ref = math.exp(scipy.special.gammaln(d / 2) - scipy.special.gammaln((d + 1) / 2)) / math.sqrt(math.pi)
+    assert abs(c64[1] - ref) < 1e-12 and abs(c64[0] + ref) < 1e-12
+    if d == 8:
+        assert abs(c64[1] - 0.29103) < 5e-6
+
+
+def test_codebook_tends_to_gaussian_lloyd_max():
+    table = _gold("gaussian_lloyd_max.json")["levels"]
+    for b in (1, 2, 3, 4):
+        ref = np.array(table[str(b)])
+        err = {}
+        for d in (128, 1024):
+            c64, _, _ = O.codebook(d, b)
+            pos = math.sqrt(d) * c64[(1 << (b - 1)):]
+            err[d] = np.max(np.abs(pos - ref) / ref)
+        assert err[1024] < 6e-3, (b, err)
+        assert err[1024] <= err[128] + 1e-4, (b, err)
+
+
+def test_codebook_parameter_count_matches_pages():
+    g = _gold("pages_numbers.json")
+    c64, c32, t32 = O.codebook(128, 3)
+    extra = g["turboquant_params_3bit_d128"]["value"] - g["dense_rotation_params_d128"]["value"]
+    assert len(c32) + len(t32) == extra == 15
+    assert 128 * 128 == g["dense_rotation_params_d128"]["value"]
+
+
+# --------------------------------------------------------------------------
+# quantizer: nearest codeword by brute force at d = 8
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [2, 3])
+def test_bucketize_is_nearest_codeword_bruteforce(bits):
+    d = 8
+    P = O.make_params(d, bits, seed=11)
+    L = 1 << bits
+    rng = np.random.default_rng(bits)
+    X = rng.standard_normal((4, d))
+    enc = O.encode(X, P, qjl=False)
+    U = O.rotate(X, P.signs) / np.linalg.norm(X, axis=1, keepdims=True)
+    c = P.c32.astype(np.float64)
+    total = L ** d
+    for v in range(X.shape[0]):
+        best, bestd = None, np.inf
+        for start in range(0, total, 1 << 20):
+            ids = np.arange(start, min(total, start + (1 << 20)), dtype=np.int64)
+            digits = (ids[:, None] // (L ** np.arange(d))[None, :]) % L
+            dist = ((U[v][None, :] - c[digits]) ** 2).sum(1)
+            k = int(np.argmin(dist))
+            if dist[k] < bestd:
+                bestd, best = dist[k], digits[k]
+        assert np.array_equal(best, enc.idx[v].astype(np.int64))
+
+
+# --------------------------------------------------------------------------
+# distortion: within 2.7x of 4^-b (pages), and equal to the law's integral
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_mse_within_pages_bound_and_matches_integral(bits):
+    d, n = 128, 100_000
+    P = O.make_params(d, bits, seed=21, with_S=False)
+    X = np.random.default_rng(100 + bits).standard_normal((n, d))
+    enc = O.encode(X, P, qjl=False, margins=False)
+    Y = O.rotate(X, P.signs)
+    rec = enc.nhat[:, None] * P.c32.astype(np.float64)[enc.idx]
+    nmse = np.mean(np.sum((Y - rec) ** 2, 1) / np.sum(X ** 2, 1))
+    bound = _gold("pages_numbers.json")["distortion_factor_vs_information_limit"]["value"] * 4.0 ** -bits
+    assert nmse <= bound, (nmse, bound)
+    # d * E[(T - Q(T))^2] under the coordinate law, by scipy quadrature
+    law = _coord_law(d)
+    c = P.c32.astype(np.float64)
+    t = np.concatenate([[-1.0], P.t32.astype(np.float64), [1.0]])
+    pred = d * sum(scipy.integrate.quad(lambda x, cj=c[j]: (x - cj) ** 2 * law.pdf(x), t[j], t[j + 1],
+                                        epsabs=1e-14, limit=400)[0] for j in range(len(c)))
+    assert abs(nmse - pred) / pred < 0.01, (nmse, pred)
+
+
+# --------------------------------------------------------------------------
+# QJL: the estimator is unbiased; without stage 2 it is biased
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [2, 3])
+def test_qjl_estimator_unbiased_over_seeds(bits):
+    d, n_seeds = 128, 10_000
+    rng = np.random.default_rng(7)
+    k = rng.standard_normal(d)
+    k[5] *= 20.0
+    q = rng.standard_normal(d)
+    q = q + 0.8 * k / np.linalg.norm(k) * np.linalg.norm(q)   # a sizeable <q, k>
+    truth = float(q @ k)
+    est_qjl = np.zeros(n_seeds)
+    est_mse = np.zeros(n_seeds)
+    for s in range(n_seeds):
+        P = O.make_params(d, bits, seed=1000 + s)
+        E = O.encode(k[None, :], P, qjl=True, margins=False)
+        est_qjl[s] = O.estimate(q, P, E)[0]
+        E0 = O.Encoded(bits, False, E.idx, E.nhat)
+        est_mse[s] = O.estimate(q, P, E0)[0]
+    se = est_qjl.std(ddof=1) / math.sqrt(n_seeds)
+    assert abs(est_qjl.mean() - truth) < 3 * se, (est_qjl.mean(), truth, se)
+    # the MSE-only estimate shrinks <q,k> (biased), as the pages state
+    se0 = est_mse.std(ddof=1) / math.sqrt(n_seeds)
+    assert abs(est_mse.mean() - truth) > 6 * se0, (est_mse.mean(), truth, se0)
+
+
+# --------------------------------------------------------------------------
+# attention and search
+# --------------------------------------------------------------------------
+def test_exact_attention_is_textbook_softmax():
+    rng = np.random.default_rng(4)
+    Q, K, V = rng.standard_normal((3, 5, 16)), rng.standard_normal((40, 16)), rng.standard_normal((40, 16))
+    Q = Q[0]
+    out = O.attend_exact(Q, K, V)
+    ref = scipy.special.softmax(Q @ K.T / 4.0, axis=1) @ V
+    assert np.allclose(out, ref, atol=1e-13)
+
+
+def test_attention_single_key_returns_dequantized_value():
+    d = 128
+    rng = np.random.default_rng(8)
+    Pk, Pv = O.make_params(d, 2, 1), O.make_params(d, 4, 2)
+    K, V = rng.standard_normal((1, d)), rng.standard_normal((1, d))
+    Ek, Ev = O.encode(K, Pk, qjl=True), O.encode(V, Pv, qjl=False)
+    out, lse, logits = O.attend(rng.standard_normal((3, d)), Pk, Ek, Pv, Ev, want_logits=True)
+    H = scipy.linalg.hadamard(d) / math.sqrt(d)
+    vhat = (np.diag(Pv.signs.astype(float)) @ H @ (Ev.nhat[0] * Pv.c32.astype(float)[Ev.idx[0]]))
+    assert np.allclose(out, vhat[None, :], atol=1e-12)
+    assert np.allclose(lse, logits[:, 0], atol=1e-12)
+
+
+def test_attention_weights_sum_to_one_and_causal_prefix():
+    d, L = 128, 300
+    rng = np.random.default_rng(9)
+    Pk, Pv = O.make_params(d, 2, 3), O.make_params(d, 3, 4)
+    K, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    Ek, Ev = O.encode(K, Pk, qjl=True), O.encode(V, Pv, qjl=False)
+    Q = rng.standard_normal((4, d))
+    out, lse, logits = O.attend(Q, Pk, Ek, Pv, Ev, want_logits=True)
+    # logits are the estimates scaled by 1/sqrt(d); weights exp(l - lse) sum to 1
+    for a in range(4):
+        assert np.allclose(logits[a], O.estimate(Q[a], Pk, Ek) / math.sqrt(d), atol=1e-12)
+        assert abs(np.exp(logits[a] - lse[a]).sum() - 1.0) < 1e-12
+    # a query that sees a prefix equals attention over the truncated sequence
+    nv = np.array([1, 57, 200, L], np.int32)
+    o2, _, _ = O.attend(Q, Pk, Ek, Pv, Ev, nvis=nv)
+    for a in range(4):
+        sub = lambda E: O.Encoded(E.bits, E.qjl, E.idx[:nv[a]], E.nhat[:nv[a]],
+                                  None if E.rho is None else E.rho[:nv[a]],
+                                  None if E.sbits is None else E.sbits[:nv[a]])
+        o3, _, _ = O.attend(Q[a:a + 1], Pk, sub(Ek), Pv, sub(Ev))
+        assert np.allclose(o2[a], o3[0], atol=1e-13)
+
+
+def test_search_topk_matches_sorting_with_ties():
+    d, n = 64, 500
+    rng = np.random.default_rng(10)
+    P = O.make_params(d, 4, 5)
+    X = rng.standard_normal((n, d))
+    X[123] = X[45]          # identical vectors -> identical scores (a tie)
+    X[400] = X[45]
+    E = O.encode(X, P, qjl=True, margins=False)
+    Q = rng.standard_normal((3, d))
+    Q[0] = X[45] * 3.0      # make the tied vectors the best matches
+    sc, ix = O.search(Q, P, E, 10)
+    for a in range(3):
+        est = O.estimate(Q[a], P, E)
+        order = np.lexsort((np.arange(n), -est))[:10]      # score desc, index asc
+        assert np.array_equal(ix[a], order)
+        assert np.array_equal(sc[a], est[order])
+    assert list(ix[0][:3]) == [45, 123, 400]
+
+
+# --------------------------------------------------------------------------
+# layout
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("kbits,kqjl,vbits,per_token", [(2, True, 4, 118), (2, True, 3, 102),
+                                                        (8, False, 4, 196), (4, True, 4, 150),
+                                                        (3, True, 3, 118)])
+def test_layout_byte_counts(kbits, kqjl, vbits, per_token):
+    lay = O.Layout(128, kbits, kqjl, vbits, page_tokens=64)
+    assert lay.page_bytes == 64 * per_token
+    # one fp16 norm per vector (plus rho for QJL keys): no per-block scales
+    scale_bytes = sum(b for n, (o, b) in lay.fields.items() if n in ("kn", "kr", "vn"))
+    assert scale_bytes == (6 if kqjl else 4)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_pack_roundtrip(bits):
+    rng = np.random.default_rng(bits)
+    idx = rng.integers(0, 1 << bits, (50, 128)).astype(np.uint8)
+    kap = O.to_kappa(idx, bits)
+    assert np.array_equal(O.from_kappa(kap, bits), idx)
+    for w in (1, 2, 4, 8):
+        v = rng.integers(0, 1 << w, (7, 64)).astype(np.uint8)
+        assert np.array_equal(O.unpack_fields(O.pack_fields(v, w), 64, w), v)
+    # field i sits at bit offset i*w, little-endian
+    v = np.zeros((1, 16), np.uint8)
+    v[0, 3] = 0b1011
+    assert O.pack_fields(v, 4)[0, 1] == 0b10110000
+
+
+def test_cache_write_read_roundtrip():
+    d = 128
+    rng = np.random.default_rng(12)
+    lay = O.Layout(d, 3, True, 3, page_tokens=16)
+    Pk, Pv = O.make_params(d, 3, 1), O.make_params(d, 3, 2)
+    X = rng.standard_normal((40, d))
+    Ek, Ev = O.encode(X, Pk, qjl=True), O.encode(X[::-1].copy(), Pv, qjl=False)
+    nheads = 2
+    cache = np.zeros((4 * nheads, lay.page_bytes), np.uint8)
+    slots = rng.permutation(64)[:40]
+    O.write_cache(lay, cache, slots, 1, nheads, Ek, Ev)
+    back = O.read_cache(lay, cache, slots, 1, nheads)
+    assert np.array_equal(back["kidx"], Ek.idx) and np.array_equal(back["vidx"], Ev.idx)
+    assert np.array_equal(back["ks"], Ek.sbits)
+    assert np.array_equal(back["kn"], Ek.nhat) and np.array_equal(back["kr"], Ek.rho)
+    assert np.array_equal(back["vn"], Ev.nhat)
+    assert not cache[0::2].any()          # head 0 pages untouched
