@@ -1,0 +1,418 @@
+// Attention computed directly over the compressed cache (decode and chunked
+// prefill), split over the key range and merged by log-sum-exp.
+//
+// Page "What is TurboQuant?", "Stage 2": the QJL bits make <q, k> estimates
+// unbiased; the attention-logit figure quoted there is computed from the
+// compressed keys.  Logit of key t for query q (R = H D / sqrt(d)):
+//   l_t = (nhat_t <Rq, c[code_t]> + rho_t sqrt(pi/2)/m <S R q, 2 s_t - 1>) / sqrt(d)
+// then softmax over the visible keys and o = R_v^T sum_t p_t nhat_v,t c_v[code_v,t].
+//
+// Kernels: prep (per query row: q_r = R q and w = S q_r), attention (one
+// block per (query group, key split): scores, online softmax, value
+// accumulation in the value rotation's basis), combine (merge the splits by
+// log-sum-exp, apply R_v^T with the Walsh-Hadamard butterflies, bf16 out).
+#include <cuda_runtime.h>
+
+#include "tq_dev.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int kChunk = 128;        // keys per inner step (one per thread)
+constexpr int kMaxG = 8;           // query heads per KV head handled per block
+
+struct PrepArgs {
+    const void *Q;          // [rows][D] bf16 or fp32
+    int in_f32;
+    int64_t rows;
+    DevParams kp;
+    float *qr;              // [rows][D]
+    float *w;               // [rows][D]
+};
+
+// One warp per query row; 4 rows per block.
+template <int D>
+__global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
+    constexpr int E = WarpVec<D>::E;
+    __shared__ float sq[4][D];
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    const int64_t row = int64_t(blockIdx.x) * 4 + wl;
+    if (row >= a.rows) return;
+    float x[E], sg[E];
+    if (a.in_f32) load_vec<D>(reinterpret_cast<const float *>(a.Q) + row * D, lane, x);
+    else load_vec<D>(reinterpret_cast<const __nv_bfloat16 *>(a.Q) + row * D, lane, x);
+    load_vec<D>(a.kp.signs, lane, sg);
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] *= sg[e];
+    fwht_warp<D>(x, lane);
+    const float rs = 1.0f / sqrtf(float(D));
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float v = x[e] * rs;
+            sq[wl][lane * E + e] = v;
+            a.qr[row * D + lane * E + e] = v;
+        }
+    }
+    __syncwarp();
+    for (int j = lane; j < D; j += 32) {
+        const uint16_t *srow = a.kp.S + size_t(j) * D;
+        float acc = 0.f;
+        for (int i = 0; i < D; ++i) acc = fmaf(__uint_as_float(uint32_t(srow[i]) << 16), sq[wl][i], acc);
+        a.w[row * D + j] = acc;
+    }
+}
+
+struct AttnArgs {
+    Layout L;
+    DevParams kp, vp;
+    const uint8_t *cache;
+    int64_t num_blocks;
+    int Hq, G, n_groups, n_splits, split_len;
+    const int32_t *block_table;
+    int bt_stride, max_blocks;
+    const int32_t *seq_lens;
+    int base_len;
+    const float *qr, *w;         // [rows][D]
+    float *part_o;               // [group][split][G][D]
+    float *part_ml;              // [group][split][G][2]
+    float *logits;               // optional
+    int64_t logits_stride;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ int visible_len(const AttnArgs &a, int b) {
+    return a.seq_lens ? a.seq_lens[b] : a.base_len + b + 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
+    constexpr int CPT = (D + kChunk - 1) / kChunk;     // coordinates per thread (value side)
+    __shared__ float sq[D][kMaxG];
+    __shared__ float sw[D][kMaxG];
+    __shared__ float lg[kMaxG][kChunk];
+    __shared__ float vn[kChunk];
+    __shared__ const uint8_t *pg[kChunk];
+    __shared__ float lvk[16], lvv[16];
+    __shared__ float s_m[kMaxG], s_l[kMaxG], s_alpha[kMaxG];
+
+    const Layout &L = a.L;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = blockIdx.x, split = blockIdx.y;
+    const int b = g / L.H, kvh = g - b * L.H;
+    const int G = a.G;
+    const int nv = visible_len(a, b);
+    const int t_begin = split * a.split_len;
+    const int t_end = min(nv, t_begin + a.split_len);
+    const int32_t *bt = a.block_table + int64_t(b) * a.bt_stride;
+    const int64_t row0 = int64_t(b) * a.Hq + int64_t(kvh) * G;
+
+    for (int i = tid; i < D * G; i += kChunk) {
+        const int h = i / D, c = i - h * D;
+        sq[c][h] = a.qr[(row0 + h) * D + c];
+        sw[c][h] = a.w[(row0 + h) * D + c];
+    }
+    if (tid < 16) {
+        lvk[tid] = tid < (1 << L.kbits) ? a.kp.lv[tid] : 0.f;
+        lvv[tid] = tid < (1 << L.vbits) ? a.vp.lv[tid] : 0.f;
+    }
+    if (tid < kMaxG) { s_m[tid] = -INFINITY; s_l[tid] = 0.f; }
+    float acc[kMaxG][CPT];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[h][c] = 0.f;
+    __syncthreads();
+
+    const float scale = 1.0f / sqrtf(float(D));
+    const float cq = 1.2533141373155003f / float(D);     // sqrt(pi/2) / m
+    const int kw = L.kc_w;
+
+    for (int c0 = t_begin; c0 < t_end; c0 += kChunk) {
+        // ---- scores: one key per thread
+        const int t = c0 + tid;
+        float lgt[kMaxG];
+        const uint8_t *page = nullptr;
+        if (t < t_end) {
+            const int bi = t / L.P;
+            const int blk = bi < a.max_blocks ? bt[bi] : -1;
+            if (blk >= 0 && blk < a.num_blocks) page = a.cache + (int64_t(blk) * L.H + kvh) * L.page_bytes;
+            else atomicOr(a.status, TQ_DEV_BLOCK_RANGE);
+        }
+        pg[tid] = page;
+        if (page) {
+            const int pos = t % L.P;
+            const uint8_t *kc = page + L.kc_off + pos * L.kc_bpt;
+            const uint8_t *kh = L.kbits == 3 ? page + L.kh_off + pos * L.kh_bpt : nullptr;
+            const uint8_t *ks = L.kqjl ? page + L.ks_off + pos * L.ks_bpt : nullptr;
+            float mse[kMaxG], qj[kMaxG];
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) { mse[h] = 0.f; qj[h] = 0.f; }
+            for (int i = 0; i < D; ++i) {
+                uint32_t kap = read_field(kc, i, kw);
+                if (kh) kap |= read_field(kh, i, 1) << 2;
+                const float cv = lvk[kap];
+                const bool pos_sign = ks ? (read_field(ks, i, 1) != 0) : true;
+#pragma unroll
+                for (int h = 0; h < kMaxG; ++h) {
+                    if (h < G) {
+                        mse[h] = fmaf(sq[i][h], cv, mse[h]);
+                        qj[h] += pos_sign ? sw[i][h] : -sw[i][h];
+                    }
+                }
+            }
+            const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2));
+            const float rk = L.kqjl ? h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2)) : 0.f;
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) {
+                float v = nk * mse[h];
+                if (L.kqjl) v = fmaf(rk * cq, qj[h], v);
+                lgt[h] = v * scale;
+            }
+            vn[tid] = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.vn_off + pos * 2));
+        } else {
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) lgt[h] = -INFINITY;
+            vn[tid] = 0.f;
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+            if (h < G) {
+                lg[h][tid] = lgt[h];
+                if (a.logits && t < t_end) a.logits[(row0 + h) * a.logits_stride + t] = lgt[h];
+            }
+        }
+        __syncthreads();
+
+        // ---- online softmax: warp w handles heads w, w + 4
+        for (int h = warp; h < G; h += 4) {
+            float mx = -INFINITY;
+            for (int j = lane; j < kChunk; j += 32) mx = fmaxf(mx, lg[h][j]);
+            mx = warp_max(mx);
+            const float m_old = s_m[h];
+            const float m_new = fmaxf(m_old, mx);
+            float sum = 0.f;
+            for (int j = lane; j < kChunk; j += 32) {
+                const float p = m_new == -INFINITY ? 0.f : expf(lg[h][j] - m_new);
+                lg[h][j] = p;
+                sum += p;
+            }
+            sum = warp_sum(sum);
+            if (lane == 0) {
+                const float alpha = m_old == -INFINITY ? 0.f : expf(m_old - m_new);
+                s_alpha[h] = alpha;
+                s_l[h] = s_l[h] * alpha + sum;
+                s_m[h] = m_new;
+            }
+        }
+        __syncthreads();
+
+        // ---- value accumulation: thread owns coordinates tid + kChunk * c
+        float al[kMaxG];
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) al[h] = h < G ? s_alpha[h] : 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) acc[h][c] *= al[h];
+        const int nloc = min(kChunk, t_end - c0);
+        for (int j = 0; j < nloc; ++j) {
+            const uint8_t *page = pg[j];
+            if (!page) continue;
+            const int pos = (c0 + j) % L.P;
+            const uint8_t *vc = page + L.vc_off + pos * L.vc_bpt;
+            const uint8_t *vh = L.vbits == 3 ? page + L.vh_off + pos * L.vh_bpt : nullptr;
+            const float nvv = vn[j];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+                const int i = tid + c * kChunk;
+                if (i < D) {
+                    uint32_t kap = read_field(vc, i, L.vc_w);
+                    if (vh) kap |= read_field(vh, i, 1) << 2;
+                    const float val = lvv[kap] * nvv;
+#pragma unroll
+                    for (int h = 0; h < kMaxG; ++h)
+                        if (h < G) acc[h][c] = fmaf(lg[h][j], val, acc[h][c]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- partial results of this split
+    const int64_t pbase = (int64_t(g) * a.n_splits + split) * G;
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+        if (h < G) {
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+                const int i = tid + c * kChunk;
+                if (i < D) a.part_o[(pbase + h) * D + i] = acc[h][c];
+            }
+        }
+    }
+    if (tid < G) {
+        a.part_ml[(pbase + tid) * 2] = s_m[tid];
+        a.part_ml[(pbase + tid) * 2 + 1] = s_l[tid];
+    }
+}
+
+struct CombineArgs {
+    int n_groups, n_splits, G, Hq, H;
+    const float *part_o, *part_ml;
+    DevParams vp;
+    void *out;          // bf16 [n_seq][Hq][D]
+    float *lse;         // optional [n_seq][Hq]
+};
+
+// One warp per (group, head): merge splits by log-sum-exp, rotate back.
+template <int D>
+__global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+    constexpr int E = WarpVec<D>::E;
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (r >= int64_t(a.n_groups) * a.G) return;
+    const int g = int(r / a.G), h = int(r - int64_t(g) * a.G);
+    float M = -INFINITY;
+    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, a.part_ml[((int64_t(g) * a.n_splits + s) * a.G + h) * 2]);
+    float Lsum = 0.f;
+    float o[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = 0.f;
+    for (int s = 0; s < a.n_splits; ++s) {
+        const int64_t pb = (int64_t(g) * a.n_splits + s) * a.G + h;
+        const float m = a.part_ml[pb * 2];
+        if (m == -INFINITY) continue;
+        const float f = expf(m - M);
+        Lsum = fmaf(a.part_ml[pb * 2 + 1], f, Lsum);
+        if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[e] = fmaf(a.part_o[pb * D + lane * E + e], f, o[e]);
+        }
+    }
+    const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] *= inv;
+    fwht_warp<D>(o, lane);
+    float sg[E];
+    load_vec<D>(a.vp.signs, lane, sg);
+    const float rs = 1.0f / sqrtf(float(D));
+    const int b = g / a.H, kvh = g - b * a.H;
+    const int64_t orow = int64_t(b) * a.Hq + int64_t(kvh) * a.G + h;
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + orow * D;
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[lane * E + e] = __float2bfloat16_rn(o[e] * rs * sg[e]);
+    }
+    if (a.lse && lane == 0) a.lse[orow] = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
+}
+
+struct Plan {
+    int n_groups, G, n_splits, split_len;
+    size_t off_qr, off_w, off_po, off_pml, total;
+};
+
+Plan make_plan(const Layout &L, const AttnShape &s) {
+    Plan p;
+    p.G = s.Hq / L.H;
+    p.n_groups = s.n_seq * L.H;
+    int sms = 148;
+    const int maxlen = s.max_len > 0 ? s.max_len : 1;
+    const int64_t target = int64_t(sms) * 4;
+    int splits = int((target + p.n_groups - 1) / p.n_groups);
+    const int max_splits = (maxlen + kChunk - 1) / kChunk;
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+    int split_len = (maxlen + splits - 1) / splits;
+    split_len = (split_len + kChunk - 1) / kChunk * kChunk;
+    splits = (maxlen + split_len - 1) / split_len;
+    p.n_splits = splits;
+    p.split_len = split_len;
+    const int64_t rows = int64_t(s.n_seq) * s.Hq;
+    size_t off = kWsHeader;
+    auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) / 256 * 256; return o; };
+    p.off_qr = take(sizeof(float) * rows * L.d);
+    p.off_w = take(sizeof(float) * rows * L.d);
+    p.off_po = take(sizeof(float) * int64_t(p.n_groups) * splits * p.G * L.d);
+    p.off_pml = take(sizeof(float) * int64_t(p.n_groups) * splits * p.G * 2);
+    p.total = off;
+    return p;
+}
+
+template <int D>
+int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q, const AttnShape &s,
+                  const uint8_t *cache, int64_t num_blocks, void *out, float *lse, float *logits,
+                  int64_t logits_stride, uint8_t *ws, cudaStream_t st) {
+    const Plan p = make_plan(L, s);
+    const int64_t rows = int64_t(s.n_seq) * s.Hq;
+    PrepArgs pa;
+    pa.Q = Q;
+    pa.in_f32 = 0;
+    pa.rows = rows;
+    pa.kp = kp->dev;
+    pa.qr = reinterpret_cast<float *>(ws + p.off_qr);
+    pa.w = reinterpret_cast<float *>(ws + p.off_w);
+    prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
+
+    AttnArgs a;
+    a.L = L;
+    a.kp = kp->dev;
+    a.vp = vp->dev;
+    a.cache = cache;
+    a.num_blocks = num_blocks;
+    a.Hq = s.Hq;
+    a.G = p.G;
+    a.n_groups = p.n_groups;
+    a.n_splits = p.n_splits;
+    a.split_len = p.split_len;
+    a.block_table = s.block_table;
+    a.bt_stride = s.bt_stride;
+    a.max_blocks = s.max_blocks;
+    a.seq_lens = s.seq_lens;
+    a.base_len = s.base_len;
+    a.qr = pa.qr;
+    a.w = pa.w;
+    a.part_o = reinterpret_cast<float *>(ws + p.off_po);
+    a.part_ml = reinterpret_cast<float *>(ws + p.off_pml);
+    a.logits = logits;
+    a.logits_stride = logits_stride;
+    a.status = reinterpret_cast<uint32_t *>(ws);
+    attn_kernel<D><<<dim3(unsigned(p.n_groups), unsigned(p.n_splits)), kChunk, 0, st>>>(a);
+
+    CombineArgs c;
+    c.n_groups = p.n_groups;
+    c.n_splits = p.n_splits;
+    c.G = p.G;
+    c.Hq = s.Hq;
+    c.H = L.H;
+    c.part_o = a.part_o;
+    c.part_ml = a.part_ml;
+    c.vp = vp->dev;
+    c.out = out;
+    c.lse = lse;
+    const int64_t crow = int64_t(p.n_groups) * p.G;
+    combine_kernel<D><<<unsigned((crow + 3) / 4), 128, 0, st>>>(c);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_ws_bytes(const Layout &L, const AttnShape &s) { return make_plan(L, s).total; }
+
+int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q,
+                     const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out, float *lse,
+                     float *logits, int64_t logits_stride, uint8_t *ws, size_t ws_bytes, void *stream) {
+    (void)ws_bytes;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (L.d) {
+        case 8: return run_attention<8>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        case 16: return run_attention<16>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        case 32: return run_attention<32>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        case 64: return run_attention<64>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        case 128: return run_attention<128>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        case 256: return run_attention<256>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tq

@@ -1,0 +1,418 @@
+// Write path: compress K/V vectors into the paged cache.
+//
+// Page "What is TurboQuant?", "Stage 1: rotation and scalar quantization by
+// PolarQuant" (randomized Hadamard rotation, per-coordinate Lloyd-Max codes,
+// no per-block scale) and "Stage 2: removing inner-product bias with a 1-bit
+// QJL residual"; ai-work-lab overview, "QJL" (+1/-1 sign bits of a random
+// projection of the residual); vLLM preset k8v4 (FP8 keys).
+//
+// Kernel 1 (encode_kernel, one warp per vector): load, norm, sign flip,
+// Walsh-Hadamard butterflies with __shfl_xor_sync, bucketize against the
+// Lloyd-Max boundaries in registers, sign-magnitude codes packed into the
+// page, fp16 norm; for QJL keys also the residual r = y - nhat c[idx] (kept
+// in fp32 scratch) and its fp16 norm rho.
+// Kernel 2 (qjl_gemm_kernel): z = S r on the tensor cores (tcgen05.mma,
+// accumulator in TMEM).  r is split into three bf16 terms (hi + mid + lo,
+// together the full fp32 mantissa) against the bf16-exact S, so the sign of
+// every z_j is that of the fp32-accurate product; the epilogue packs sign
+// bits straight into the page.
+#include <cuda_runtime.h>
+#include <cuda_fp8.h>
+
+#include "tc05.cuh"
+#include "tq_dev.cuh"
+
+namespace tq {
+namespace {
+
+struct EncodeArgs {
+    Layout L;
+    DevParams kp, vp;
+    const void *K, *V;
+    int64_t n_tokens;
+    const int32_t *slots;
+    int64_t num_slots;
+    uint8_t *cache;
+    float *resid;        // [n_tokens * H][D] (QJL keys) or nullptr
+    uint32_t *status;
+    int do_v;
+};
+
+template <int D, int W>
+__device__ __forceinline__ void store_codes(uint8_t *dst, int lane, const uint32_t (&f)[WarpVec<D>::E]) {
+    store_fields<D, W>(dst, lane, f);
+}
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+    constexpr int E = WarpVec<D>::E;
+    const int lane = threadIdx.x & 31;
+    const Layout &L = a.L;
+    const int64_t nvec = a.n_tokens * L.H;
+    const int64_t total = a.do_v ? 2 * nvec : nvec;
+    const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    const float rs = 1.0f / sqrtf(float(D));
+    const float sqrt_d = sqrtf(float(D));
+
+    for (int64_t vid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; vid < total; vid += nwarps) {
+        const bool is_v = vid >= nvec;
+        const int64_t v = is_v ? vid - nvec : vid;
+        const int64_t t = v / L.H;
+        const int h = int(v - t * L.H);
+        const int slot = a.slots[t];
+        if (slot < 0) continue;
+        if (slot >= a.num_slots) {
+            if (lane == 0) atomicOr(a.status, TQ_DEV_SLOT_RANGE);
+            continue;
+        }
+        const DevParams &P = is_v ? a.vp : a.kp;
+        const int bits = is_v ? L.vbits : L.kbits;
+
+        float x[E], sg[E];
+        load_vec<D>(reinterpret_cast<const TIn *>(is_v ? a.V : a.K) + v * D, lane, x);
+        load_vec<D>(P.signs, lane, sg);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            ss = fmaf(x[e], x[e], ss);
+            x[e] *= sg[e];
+        }
+        const float n = sqrtf(warp_sum(ss));
+        fwht_warp<D>(x, lane);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] *= rs;          // y = R x
+        const float inv = n > 0.f ? 1.0f / n : 0.f;
+        const uint16_t nh = f2h_bits(n);
+        const float nhf = h2f_bits(nh);
+
+        uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
+        const int pos = slot % L.P;
+
+        if (!is_v && L.kbits == 8) {
+            uint32_t f[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                f[e] = uint32_t(__nv_cvt_float_to_fp8(sqrt_d * (x[e] * inv), __NV_SATFINITE, __NV_E4M3));
+            store_codes<D, 8>(page + L.kc_off + pos * L.kc_bpt, lane, f);
+            if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kn_off + pos * 2) = nh;
+            continue;
+        }
+
+        const int nb = (1 << bits) - 1;
+        uint32_t kap[E];
+        float cval[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float u = x[e] * inv;
+            uint32_t idx = 0;
+            for (int j = 0; j < nb; ++j) idx += (P.bounds[j] <= u) ? 1u : 0u;
+            kap[e] = kappa_of(idx, bits);
+            cval[e] = P.lv[kap[e]];
+        }
+        const int code_off = is_v ? L.vc_off : L.kc_off;
+        const int code_bpt = is_v ? L.vc_bpt : L.kc_bpt;
+        uint8_t *cdst = page + code_off + pos * code_bpt;
+        if (bits == 1) {
+            store_codes<D, 1>(cdst, lane, kap);
+        } else if (bits == 2) {
+            store_codes<D, 2>(cdst, lane, kap);
+        } else if (bits == 4) {
+            store_codes<D, 4>(cdst, lane, kap);
+        } else {   // 3 bits: 2-bit magnitude array + 1-bit sign array
+            uint32_t lo[E], hi[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) { lo[e] = kap[e] & 3u; hi[e] = kap[e] >> 2; }
+            store_codes<D, 2>(cdst, lane, lo);
+            const int hoff = is_v ? L.vh_off : L.kh_off;
+            const int hbpt = is_v ? L.vh_bpt : L.kh_bpt;
+            store_codes<D, 1>(page + hoff + pos * hbpt, lane, hi);
+        }
+        if (lane == 0) *reinterpret_cast<uint16_t *>(page + (is_v ? L.vn_off : L.kn_off) + pos * 2) = nh;
+
+        if (!is_v && L.kqjl) {
+            float r[E], rr = 0.f;
+            const bool active = lane < WarpVec<D>::LANES;    // lanes past d hold no coordinate
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                r[e] = active ? fmaf(-nhf, cval[e], x[e]) : 0.f;
+                rr = fmaf(r[e], r[e], rr);
+            }
+            const float rho = sqrtf(warp_sum(rr));
+            if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kr_off + pos * 2) = f2h_bits(rho);
+            if (lane < WarpVec<D>::LANES) {
+                float *dst = a.resid + v * D + lane * E;
+#pragma unroll
+                for (int e = 0; e < E; ++e) dst[e] = r[e];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// QJL projection on the tensor cores.
+// ---------------------------------------------------------------------------
+struct QjlArgs {
+    Layout L;
+    const uint16_t *S;      // [m][D] bf16 bits, m = D
+    const float *resid;     // [nK][D]
+    int64_t nK;             // n_tokens * H
+    const int32_t *slots;
+    int64_t num_slots;
+    uint8_t *cache;
+    uint32_t *status;
+};
+
+constexpr int kBM = 128;       // vectors per tile (MMA M)
+constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
+constexpr uint32_t kMaxPolls = 1u << 24;
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+    __nv_bfloat16 b = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&b);
+}
+__device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
+    return __uint_as_float(uint32_t(b) << 16);
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
+    constexpr int M = D;                                   // projection rows
+    constexpr int NK = (D + kBK - 1) / kBK;
+    constexpr uint32_t TCOLS = BN < 32 ? 32 : BN;
+    constexpr int A_BYTES = kBM * 128;                     // one split tile
+    constexpr int B_BYTES = BN * 128;
+    constexpr int STAGE_BYTES = 3 * A_BYTES + B_BYTES;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar[2];
+    __shared__ uint32_t tmem_holder;
+    __shared__ int timed_out;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t row0 = int64_t(blockIdx.x) * kBM;
+    const int n0 = blockIdx.y * BN;
+
+    if (warp == 0) {
+        tc05::tmem_alloc(&tmem_holder, TCOLS);
+        tc05::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc05::mbar_init(&bar[0], 1);
+        tc05::mbar_init(&bar[1], 1);
+        tc05::fence_mbar_init();
+        timed_out = 0;
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    tc05::fence_after_sync();
+    const uint32_t tmem = tmem_holder;
+    constexpr uint32_t idesc = tc05::idesc_bf16_f32(kBM, BN < 16 ? 16 : BN);
+
+    for (int kc = 0; kc < NK; ++kc) {
+        const int st = kc & 1;
+        uint8_t *sA = smem + st * STAGE_BYTES;
+        uint8_t *sB = sA + 3 * A_BYTES;
+        if (kc >= 2) {
+            if (!tc05::mbar_wait_bounded(&bar[st], ((kc - 2) >> 1) & 1, kMaxPolls)) timed_out = 1;
+        }
+        // A: row tid of this tile, columns [kc*64, kc*64+64) of r, split in 3
+        {
+            const int64_t g = row0 + tid;
+            float rv[kBK];
+            const int c0 = kc * kBK;
+            if (g < a.nK && c0 + kBK <= D) {
+                const float4 *src = reinterpret_cast<const float4 *>(a.resid + g * D + c0);
+#pragma unroll
+                for (int q = 0; q < kBK / 4; ++q) {
+                    float4 f = src[q];
+                    rv[4 * q] = f.x; rv[4 * q + 1] = f.y; rv[4 * q + 2] = f.z; rv[4 * q + 3] = f.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < kBK; ++q) rv[q] = (g < a.nK && c0 + q < D) ? a.resid[g * D + c0 + q] : 0.f;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint16_t h2[2], m2[2], l2[2];
+#pragma unroll
+                    for (int z = 0; z < 2; ++z) {
+                        const float x = rv[ch * 8 + 2 * k + z];
+                        h2[z] = bf16_bits_rn(x);
+                        const float r1 = x - bf16_bits_to_f(h2[z]);
+                        m2[z] = bf16_bits_rn(r1);
+                        const float r2 = r1 - bf16_bits_to_f(m2[z]);
+                        l2[z] = bf16_bits_rn(r2);
+                    }
+                    hi[k] = uint32_t(h2[0]) | (uint32_t(h2[1]) << 16);
+                    mid[k] = uint32_t(m2[0]) | (uint32_t(m2[1]) << 16);
+                    lo[k] = uint32_t(l2[0]) | (uint32_t(l2[1]) << 16);
+                }
+                const uint32_t o = tc05::sw128_offset(tid, ch);
+                *reinterpret_cast<uint4 *>(sA + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sA + A_BYTES + o) = make_uint4(mid[0], mid[1], mid[2], mid[3]);
+                *reinterpret_cast<uint4 *>(sA + 2 * A_BYTES + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        // B: BN rows of S, same 64 columns
+        for (int q = tid; q < BN * 8; q += 128) {
+            const int row = q >> 3, ch = q & 7;
+            const int j = n0 + row, c = kc * kBK + ch * 8;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (j < M && c + 8 <= D) {
+                val = *reinterpret_cast<const uint4 *>(a.S + size_t(j) * D + c);
+            } else if (j < M && c < D) {
+                uint16_t tmp[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) tmp[z] = (c + z < D) ? a.S[size_t(j) * D + c + z] : 0;
+                val = make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
+                                 tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
+            }
+            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(row, ch)) = val;
+        }
+        tc05::fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc05::fence_after_sync();
+            const uint32_t aBase = tc05::smem_u32(sA), bBase = tc05::smem_u32(sB);
+#pragma unroll
+            for (int ks = 0; ks < kBK / 16; ++ks) {
+                const uint64_t bdesc = tc05::desc_kmajor_sw128(bBase + ks * 32);
+#pragma unroll
+                for (int sp = 0; sp < 3; ++sp) {
+                    const uint64_t adesc = tc05::desc_kmajor_sw128(aBase + sp * A_BYTES + ks * 32);
+                    tc05::mma_bf16(tmem, adesc, bdesc, idesc, (kc | ks | sp) != 0);
+                }
+            }
+            tc05::mma_commit(&bar[st]);
+        }
+    }
+    if (!tc05::mbar_wait_bounded(&bar[(NK - 1) & 1], ((NK - 1) >> 1) & 1, kMaxPolls)) timed_out = 1;
+    tc05::fence_after_sync();
+
+    // Epilogue: thread = tile row (vector); TMEM lanes 32*warp .. +31.
+    const int64_t g = row0 + warp * 32 + lane;
+    uint8_t *ks_dst = nullptr;
+    if (g < a.nK) {
+        const int64_t t = g / a.L.H;
+        const int h = int(g - t * a.L.H);
+        const int slot = a.slots[t];
+        if (slot >= 0 && slot < a.num_slots) {
+            uint8_t *page = a.cache + (int64_t(slot / a.L.P) * a.L.H + h) * int64_t(a.L.page_bytes);
+            ks_dst = page + a.L.ks_off + (slot % a.L.P) * a.L.ks_bpt;
+        }
+    }
+#pragma unroll 1
+    for (int c = 0; c < (BN + 31) / 32; ++c) {
+        uint32_t r[32];
+        tc05::tmem_ld_32x32b_x32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c * 32), r);
+        tc05::tmem_wait_ld();
+        uint32_t bits = 0;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) bits |= (__uint_as_float(r[k]) >= 0.f ? 1u : 0u) << k;
+        const int j0 = n0 + c * 32;
+        if (ks_dst && !timed_out) {
+            if (M >= 32) {
+                if (j0 < M) reinterpret_cast<uint32_t *>(ks_dst)[j0 >> 5] = bits;
+            } else {
+                for (int b = 0; b < M / 8; ++b) ks_dst[b] = uint8_t(bits >> (8 * b));
+            }
+        }
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc05::fence_after_sync();
+        tc05::tmem_dealloc(tmem, TCOLS);
+    }
+    if (tid == 0 && timed_out) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
+}
+
+template <int D>
+constexpr int qjl_bn() { return D >= 256 ? 256 : (D < 16 ? 16 : D); }
+
+template <int D>
+int launch_qjl(const QjlArgs &q, cudaStream_t st) {
+    constexpr int BN = qjl_bn<D>();
+    constexpr size_t smem = 2 * (3 * kBM * 128 + BN * 128) + 1024;
+    auto kern = qjl_gemm_kernel<D, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(unsigned((q.nK + kBM - 1) / kBM), unsigned((D + BN - 1) / BN));
+    kern<<<grid, 128, smem, st>>>(q);
+    return cudaGetLastError();
+}
+
+template <int D>
+int launch_encode_d(const EncodeArgs &a, int in_dtype, const tq_params *kp, cudaStream_t st) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t nvec = a.n_tokens * a.L.H * (a.do_v ? 2 : 1);
+    int64_t blocks = (nvec + 7) / 8;
+    const int64_t cap = int64_t(sms) * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    if (in_dtype == TQ_DTYPE_BF16) encode_kernel<D, __nv_bfloat16><<<unsigned(blocks), 256, 0, st>>>(a);
+    else encode_kernel<D, float><<<unsigned(blocks), 256, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (a.L.kqjl && a.n_tokens > 0) {
+        QjlArgs q;
+        q.L = a.L;
+        q.S = kp->dev.S;
+        q.resid = a.resid;
+        q.nK = a.n_tokens * a.L.H;
+        q.slots = a.slots;
+        q.num_slots = a.num_slots;
+        q.cache = a.cache;
+        q.status = a.status;
+        return launch_qjl<D>(q, st);
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t encode_ws_bytes(const Layout &L, int64_t n_tokens) {
+    size_t b = kWsHeader;
+    if (L.kqjl) b += size_t(n_tokens) * L.H * L.d * sizeof(float);
+    return b;
+}
+
+int launch_encode(const tq_params *kp, const tq_params *vp, const Layout &L, const void *K, const void *V,
+                  int in_dtype, int64_t n_tokens, const int32_t *slots, uint8_t *cache, int64_t num_blocks,
+                  uint8_t *ws, size_t ws_bytes, void *stream) {
+    (void)ws_bytes;
+    EncodeArgs a;
+    a.L = L;
+    a.kp = kp->dev;
+    if (vp) a.vp = vp->dev;
+    else a.vp = kp->dev;
+    a.K = K;
+    a.V = V;
+    a.n_tokens = n_tokens;
+    a.slots = slots;
+    a.num_slots = num_blocks * L.P;
+    a.cache = cache;
+    a.resid = L.kqjl ? reinterpret_cast<float *>(ws + kWsHeader) : nullptr;
+    a.status = reinterpret_cast<uint32_t *>(ws);
+    a.do_v = L.vbits > 0 ? 1 : 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (L.d) {
+        case 8: return launch_encode_d<8>(a, in_dtype, kp, st);
+        case 16: return launch_encode_d<16>(a, in_dtype, kp, st);
+        case 32: return launch_encode_d<32>(a, in_dtype, kp, st);
+        case 64: return launch_encode_d<64>(a, in_dtype, kp, st);
+        case 128: return launch_encode_d<128>(a, in_dtype, kp, st);
+        case 256: return launch_encode_d<256>(a, in_dtype, kp, st);
+        case 512: return launch_encode_d<512>(a, in_dtype, kp, st);
+        case 1024: return launch_encode_d<1024>(a, in_dtype, kp, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tq

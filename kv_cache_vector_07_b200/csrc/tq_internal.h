@@ -1,0 +1,116 @@
+// Internal declarations shared by the libtqkv translation units.
+// Host + device.  Nothing here is part of the C ABI (see include/tqkv.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "tqkv.h"
+
+#if defined(__CUDACC__)
+#define TQ_HD __host__ __device__
+#else
+#define TQ_HD
+#endif
+
+namespace tq {
+
+// Byte layout of one page (page_tokens slots of one KV head).  Offsets are
+// within the page; *_bpt are bytes per token of that field; -1 = absent.
+// Field order and sizes follow the description in tqkv.h.
+struct Layout {
+    int d, kbits, kqjl, vbits, P, H;
+    int kc_off, kc_bpt, kc_w;   // main K code array and its field width
+    int kh_off, kh_bpt;         // K sign-bit array (kbits == 3 only)
+    int ks_off, ks_bpt;         // QJL sign bits
+    int kn_off, kr_off;         // fp16 norms
+    int vc_off, vc_bpt, vc_w;
+    int vh_off, vh_bpt;
+    int vn_off;
+    int page_bytes;
+};
+
+inline int pad16(int x) { return (x + 15) & ~15; }
+
+// Returns false if the description is invalid.
+inline bool make_layout(const tq_cache_desc &c, Layout *L) {
+    L->d = c.d; L->kbits = c.kbits; L->kqjl = c.kqjl; L->vbits = c.vbits;
+    L->P = c.page_tokens; L->H = c.n_kv_heads;
+    const int d = c.d, P = c.page_tokens;
+    int off = 0;
+    auto add = [&](int bpt, int *o, int *b) { *o = off; *b = bpt; off += pad16(P * bpt); };
+    int dummy;
+    L->kh_off = L->kh_bpt = L->ks_off = L->ks_bpt = L->kr_off = -1;
+    L->vc_off = L->vc_bpt = L->vh_off = L->vh_bpt = L->vn_off = -1;
+    L->vc_w = 0;
+    if (c.kbits == 8) { add(d, &L->kc_off, &L->kc_bpt); L->kc_w = 8; }
+    else if (c.kbits == 3) { add(d * 2 / 8, &L->kc_off, &L->kc_bpt); L->kc_w = 2; add(d / 8, &L->kh_off, &L->kh_bpt); }
+    else { add(d * c.kbits / 8, &L->kc_off, &L->kc_bpt); L->kc_w = c.kbits; }
+    if (c.kqjl) add(d / 8, &L->ks_off, &L->ks_bpt);
+    add(2, &L->kn_off, &dummy);
+    if (c.kqjl) add(2, &L->kr_off, &dummy);
+    if (c.vbits > 0) {
+        if (c.vbits == 3) { add(d * 2 / 8, &L->vc_off, &L->vc_bpt); L->vc_w = 2; add(d / 8, &L->vh_off, &L->vh_bpt); }
+        else { add(d * c.vbits / 8, &L->vc_off, &L->vc_bpt); L->vc_w = c.vbits; }
+        add(2, &L->vn_off, &dummy);
+    }
+    L->page_bytes = off;
+    return true;
+}
+
+// Library-owned parameters.  Device arrays live in one allocation.
+struct DevParams {
+    int d, bits;
+    const float *signs;      // [d] +1/-1
+    const uint16_t *S;       // [d][d] bf16 bits, row-major (row j = projection j)
+    const float *lv;         // [2^bits] levels indexed by the stored sign-magnitude code
+    const float *bounds;     // [2^bits - 1] ascending decision boundaries
+};
+
+}  // namespace tq
+
+struct tq_params {
+    int d, bits;
+    uint64_t seed;
+    int device;
+    int8_t *h_signs;         // host copies
+    float *h_S;
+    float *h_levels;         // ascending bucket order
+    float *h_bounds;
+    void *d_block;           // device allocation
+    tq::DevParams dev;
+};
+
+namespace tq {
+
+// Workspace header: the first 256 bytes of every workspace.
+constexpr size_t kWsHeader = 256;
+
+// Launchers (defined in the .cu files).  Return cudaError_t as int.
+int launch_encode(const tq_params *kp, const tq_params *vp, const Layout &L, const void *K,
+                  const void *V, int in_dtype, int64_t n_tokens, const int32_t *slots,
+                  uint8_t *cache, int64_t num_blocks, uint8_t *ws, size_t ws_bytes, void *stream);
+size_t encode_ws_bytes(const Layout &L, int64_t n_tokens);
+
+struct AttnShape {
+    int n_seq;            // decode: batch; prefill: chunk length C
+    int Hq;
+    const int32_t *block_table;
+    int bt_stride;        // decode: max_blocks; prefill: 0 (all rows share one table)
+    int max_blocks;
+    const int32_t *seq_lens;   // decode: [B]; prefill: nullptr
+    int base_len;         // prefill: seq_len - C (query j sees base_len + j + 1)
+    int max_len;          // longest visible length
+};
+size_t attn_ws_bytes(const Layout &L, const AttnShape &s);
+int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q,
+                     const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out,
+                     float *lse, float *logits, int64_t logits_stride, uint8_t *ws,
+                     size_t ws_bytes, void *stream);
+
+size_t score_ws_bytes(const Layout &L, int64_t n_db, int n_q, int k);
+int launch_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
+                 const float *Q, int n_q, int k, float *top_scores, int64_t *top_idx,
+                 uint8_t *ws, size_t ws_bytes, void *stream);
+
+}  // namespace tq

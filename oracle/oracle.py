@@ -70,8 +70,8 @@ def _load():
     lib.orc_codebook.argtypes = [i32, i32, vp, vp, vp]
     lib.orc_rotate.argtypes = [i32, vp, vp, vp]
     lib.orc_rotate_t.argtypes = [i32, vp, vp, vp]
-    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-    lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp]
+    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp, vp]
     lib.orc_estimate.argtypes = [vp, i32, vp, vp]
     lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_attend_exact.argtypes = [i32, i32, i32, vp, vp, vp, vp]
@@ -204,6 +204,8 @@ class Encoded:
     sbits: np.ndarray | None = None
     umargin: np.ndarray | None = None
     zmargin: np.ndarray | None = None
+    nraw: np.ndarray | None = None      # unrounded ||x||
+    rraw: np.ndarray | None = None      # unrounded ||r||
 
 
 def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded:
@@ -215,8 +217,9 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
         code = np.zeros((n, d), np.uint8)
         nhat = np.zeros(n, np.float64)
         mg = np.zeros((n, d), np.float64) if margins else None
-        lib.orc_encode_fp8(n, d, _p(X), _p(P.signs), _p(code), _p(nhat), _p(mg))
-        return Encoded(8, False, code, nhat, umargin=mg)
+        nraw = np.zeros(n, np.float64)
+        lib.orc_encode_fp8(n, d, _p(X), _p(P.signs), _p(code), _p(nhat), _p(mg), _p(nraw))
+        return Encoded(8, False, code, nhat, umargin=mg, nraw=nraw)
     idx = np.zeros((n, d), np.uint8)
     nhat = np.zeros(n, np.float64)
     rho = np.zeros(n, np.float64) if qjl else None
@@ -225,9 +228,11 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
     zm = np.zeros((n, d), np.float64) if (margins and qjl) else None
     if qjl:
         assert P.S is not None
+    nraw = np.zeros(n, np.float64)
+    rraw = np.zeros(n, np.float64) if qjl else None
     lib.orc_encode(n, d, P.bits, 1 if qjl else 0, _p(X), _p(P.signs), _p(P.S), _p(P.c32),
-                   _p(P.t32), _p(idx), _p(nhat), _p(rho), _p(sb), _p(um), _p(zm))
-    return Encoded(P.bits, qjl, idx, nhat, rho, sb, um, zm)
+                   _p(P.t32), _p(idx), _p(nhat), _p(rho), _p(sb), _p(um), _p(zm), _p(nraw), _p(rraw))
+    return Encoded(P.bits, qjl, idx, nhat, rho, sb, um, zm, nraw, rraw)
 
 
 # ---------------------------------------------------------------------------
@@ -318,7 +323,7 @@ class Layout:
     """Structure-of-arrays page of ``page_tokens`` tokens of one KV head.
 
     kbits: 1..4 Lloyd-Max bits or 8 for FP8 keys; kqjl: QJL sign bits + rho;
-    vbits: 1..4.  Fields in order, each padded to 16 bytes:
+    vbits: 1..4, or 0 for no value fields (a search database).  Fields in order, each padded to 16 bytes:
       K codes  ("kc" for w in {1,2,4}; "kc_lo" (2-bit) + "kc_hi" (1-bit) for 3
                bits; "k8" bytes for FP8), "ks" QJL sign bits, "kn" fp16 norm,
       "kr" fp16 residual norm, V codes ("vc" or "vc_lo" + "vc_hi"), "vn".
@@ -355,8 +360,9 @@ class Layout:
         add("kn", 2)
         if self.kqjl:
             add("kr", 2)
-        codes("vc", self.vbits)
-        add("vn", 2)
+        if self.vbits > 0:
+            codes("vc", self.vbits)
+            add("vn", 2)
         self.page_bytes = off
 
 
@@ -422,9 +428,19 @@ def token_records(lay: Layout, Ek: Encoded, Ev: Encoded) -> dict:
     rec["kn"] = _fp16_bytes(Ek.nhat)
     if lay.kqjl:
         rec["kr"] = _fp16_bytes(Ek.rho)
-    rec.update(_code_arrays("vc", lay.vbits, Ev.idx))
-    rec["vn"] = _fp16_bytes(Ev.nhat)
+    if lay.vbits > 0:
+        rec.update(_code_arrays("vc", lay.vbits, Ev.idx))
+        rec["vn"] = _fp16_bytes(Ev.nhat)
     return rec
+
+
+def _field_index(lay: Layout, slots: np.ndarray, head: int, n_heads: int, off: int, bpt: int):
+    """(page rows, byte columns) of one field for each slot."""
+    P = lay.page_tokens
+    s = np.asarray(slots, np.int64)
+    page = (s // P) * n_heads + head
+    cols = off + (s % P)[:, None] * bpt + np.arange(bpt)[None, :]
+    return page[:, None], cols
 
 
 def write_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_heads: int,
@@ -432,27 +448,19 @@ def write_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_
     """Store the records of tokens with the given slots for one KV head into a
     cache array viewed as [num_blocks * n_heads, page_bytes] bytes."""
     rec = token_records(lay, Ek, Ev)
-    P = lay.page_tokens
     for name, (off, bpt) in lay.fields.items():
-        data = rec[name]
-        for t, s in enumerate(slots):
-            page = (int(s) // P) * n_heads + head
-            o = off + (int(s) % P) * bpt
-            cache[page, o:o + bpt] = data[t]
+        r, c = _field_index(lay, slots, head, n_heads, off, bpt)
+        cache[r, c] = rec[name]
 
 
 def read_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_heads: int) -> dict:
     """Decode the stored fields of the given slots of one KV head back into
     bucket indices / codes, sign bits and float64 norms."""
-    P, d = lay.page_tokens, lay.d
+    d = lay.d
     raw = {}
     for name, (off, bpt) in lay.fields.items():
-        buf = np.zeros((len(slots), bpt), np.uint8)
-        for t, s in enumerate(slots):
-            page = (int(s) // P) * n_heads + head
-            o = off + (int(s) % P) * bpt
-            buf[t] = cache[page, o:o + bpt]
-        raw[name] = buf
+        r, c = _field_index(lay, slots, head, n_heads, off, bpt)
+        raw[name] = np.ascontiguousarray(cache[r, c])
 
     def codes(prefix, bits):
         if bits == 8:
@@ -463,9 +471,11 @@ def read_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_h
             kap = unpack_fields(raw[prefix], d, bits)
         return from_kappa(kap, bits)
 
-    out = {"kidx": codes("kc", lay.kbits), "vidx": codes("vc", lay.vbits),
-           "kn": raw["kn"].copy().view(np.float16).reshape(-1).astype(np.float64),
-           "vn": raw["vn"].copy().view(np.float16).reshape(-1).astype(np.float64)}
+    out = {"kidx": codes("kc", lay.kbits),
+           "kn": raw["kn"].copy().view(np.float16).reshape(-1).astype(np.float64)}
+    if lay.vbits > 0:
+        out["vidx"] = codes("vc", lay.vbits)
+        out["vn"] = raw["vn"].copy().view(np.float16).reshape(-1).astype(np.float64)
     if lay.kqjl:
         out["ks"] = unpack_fields(raw["ks"], d, 1)
         out["kr"] = raw["kr"].copy().view(np.float16).reshape(-1).astype(np.float64)

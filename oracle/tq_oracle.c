@@ -297,12 +297,13 @@ void orc_rotate_t(int d, const int8_t *signs, const double *y, double *x)
  * idx_i = #{j : t_j <= u_i}, nhat = fp16(n), r = y - nhat * c[idx],
  * rho = fp16(||r||), s_j = [ (S r)_j >= 0 ].
  * Diagnostics for the parity exemptions: umargin[i] = min_j |u_i - t_j|
- * (unit-vector units) and zmargin[j] = |(S r)_j| / (||r|| ||S_j||).
+ * (unit-vector units), zmargin[j] = |(S r)_j| / (||r|| ||S_j||), and the
+ * unrounded norms nraw = ||x||, rraw = ||r||.
  * sbits / rho / zmargin are only written when qjl != 0. */
 void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *signs,
                 const float *S, const float *c32, const float *t32, uint8_t *idx,
                 double *nhat, double *rho, uint8_t *sbits, double *umargin,
-                double *zmargin)
+                double *zmargin, double *nraw, double *rraw)
 {
     int L = 1 << bits;
     #pragma omp parallel
@@ -318,6 +319,7 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
         orc_rotate(d, signs, x, y);
         double nh = orc_round_fp16(nn);
         nhat[v] = nh;
+        if (nraw) nraw[v] = nn;
         for (int i = 0; i < d; ++i) {
             double u = nn > 0.0 ? y[i] / nn : 0.0;
             int k = 0;
@@ -336,6 +338,7 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
         for (int i = 0; i < d; ++i) rn += r[i] * r[i];
         rn = sqrt(rn);
         rho[v] = orc_round_fp16(rn);
+        if (rraw) rraw[v] = rn;
         int m = d;
         for (int j = 0; j < m; ++j) {
             double z = 0.0, sn = 0.0;
@@ -356,7 +359,7 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
  * margin[i] = distance (unit-vector units) from u_i to the nearest E4M3
  * rounding midpoint. */
 void orc_encode_fp8(int n, int d, const double *X, const int8_t *signs, uint8_t *code,
-                    double *nhat, double *margin)
+                    double *nhat, double *margin, double *nraw)
 {
     double sd = sqrt((double)d);
     #pragma omp parallel
@@ -370,6 +373,7 @@ void orc_encode_fp8(int n, int d, const double *X, const int8_t *signs, uint8_t 
         nn = sqrt(nn);
         orc_rotate(d, signs, x, y);
         nhat[v] = orc_round_fp16(nn);
+        if (nraw) nraw[v] = nn;
         for (int i = 0; i < d; ++i) {
             double u = nn > 0.0 ? y[i] / nn : 0.0;
             double a = sd * u;

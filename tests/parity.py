@@ -1,0 +1,108 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+Codes and sign bits must match bit for bit, except:
+  * a code whose oracle coordinate u_i lies within 1e-6 (unit-vector units)
+    of a decision boundary (or an E4M3 rounding midpoint) - then the GPU code
+    may be either neighbour;
+  * a QJL sign whose |(S r)_j| / (||r|| ||S_j||) < 1e-6, and every sign of a
+    vector with an exempt code or norm (its residual legitimately differs).
+Norms (fp16) must be equal, or one fp16 ulp apart when the oracle's unrounded
+value lies within 1e-5 relative of the rounding midpoint between them (the
+GPU rounds from fp32); such a key's logits are exempt too.  Logits: |d| <= 1e-3 * max(|l_oracle|, rms of the
+row's logits), on keys without exemptions.  Outputs (bf16): |d| <= 2e-3 +
+half a bf16 ulp of the oracle value (the output rounding itself).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import oracle as O
+
+CODE_MARGIN = 1e-6
+SIGN_MARGIN = 1e-6
+NORM_TIE_REL = 1e-5
+LOGIT_REL = 1e-3
+OUT_ABS = 2e-3
+
+
+def fp16_match(gpu: np.ndarray, orc: np.ndarray, raw: np.ndarray):
+    """(ok mask, tie mask) for fp16-valued norms."""
+    g = np.asarray(gpu, np.float64)
+    o = np.asarray(orc, np.float64)
+    eq = g == o
+    gb = g.astype(np.float16).view(np.int16).astype(np.int64)
+    ob = o.astype(np.float16).view(np.int16).astype(np.int64)
+    adj = (np.abs(gb - ob) == 1) & (np.sign(g) == np.sign(o))
+    mid = 0.5 * (g + o)
+    tie = (~eq) & adj & (np.abs(np.asarray(raw) - mid) <= NORM_TIE_REL * np.abs(raw))
+    return eq | tie, tie
+
+
+def compare_vectors(gpu: dict, Ek: O.Encoded, key: bool, bits: int):
+    """Compare one head's decoded GPU fields with the oracle encoding.
+
+    Returns (report dict, exempt_vector mask).  Raises AssertionError on a
+    mismatch outside the exemptions."""
+    rep = {}
+    codes = gpu["kidx"] if key else gpu["vidx"]
+    norms = gpu["kn"] if key else gpu["vn"]
+    diff = codes != Ek.idx
+    margin_ok = Ek.umargin < CODE_MARGIN
+    bad = diff & ~margin_ok
+    rep["code_exempt"] = int((diff & margin_ok).sum())
+    assert not bad.any(), f"{int(bad.sum())} codes differ outside the boundary exemption " \
+                          f"(first at {np.argwhere(bad)[0].tolist()})"
+    if bits != 8:
+        # an exempt code may only move to the neighbouring bucket
+        assert np.all(np.abs(codes[diff].astype(int) - Ek.idx[diff].astype(int)) == 1)
+    ok, tie = fp16_match(norms, Ek.nhat, Ek.nraw)
+    assert ok.all(), f"{int((~ok).sum())} norms differ (first {np.argwhere(~ok)[0].tolist()})"
+    rep["norm_tie"] = int(tie.sum())
+    vec_exempt = diff.any(1) | tie
+    if key and Ek.qjl:
+        ok, rtie = fp16_match(gpu["kr"], Ek.rho, Ek.rraw)
+        bad_r = ~ok & ~vec_exempt
+        assert not bad_r.any(), f"{int(bad_r.sum())} residual norms differ"
+        rep["rho_tie"] = int(rtie.sum())
+        sdiff = gpu["ks"] != Ek.sbits
+        sex = (Ek.zmargin < SIGN_MARGIN) | vec_exempt[:, None]
+        bad_s = sdiff & ~sex
+        rep["sign_exempt"] = int((sdiff & sex).sum())
+        assert not bad_s.any(), f"{int(bad_s.sum())} QJL sign bits differ outside the exemption " \
+                                f"(first {np.argwhere(bad_s)[0].tolist()})"
+        # a residual norm rounded one ulp apart (a tie) changes that key's logit
+        vec_exempt = vec_exempt | sdiff.any(1) | ~ok | rtie
+    rep["vectors_exempt"] = int(vec_exempt.sum())
+    return rep, vec_exempt
+
+
+def check_logits(gpu: np.ndarray, orc: np.ndarray, exempt_keys: np.ndarray | None = None):
+    """gpu, orc: [rows, L] over the visible keys."""
+    rms = np.sqrt(np.mean(orc ** 2, axis=1, keepdims=True))
+    tol = LOGIT_REL * np.maximum(np.abs(orc), rms)
+    err = np.abs(gpu.astype(np.float64) - orc)
+    bad = err > tol
+    if exempt_keys is not None:
+        bad &= ~exempt_keys[None, :]
+    if bad.any():
+        where = np.argwhere(bad)[:8]
+        detail = [(int(r), int(t), float(gpu[r, t]), float(orc[r, t]), float(rms[r, 0])) for r, t in where]
+        raise AssertionError(f"{int(bad.sum())} logits outside tolerance; worst rel "
+                             f"{float(np.max(err / np.maximum(tol, 1e-30)) * LOGIT_REL):.3e}; "
+                             f"(row, key, gpu, oracle, rms): {detail}")
+    return float(np.max(err / np.maximum(np.maximum(np.abs(orc), rms), 1e-30)))
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.abs(np.asarray(x, np.float64))
+    a = np.where(a == 0, 2.0 ** -133, a)
+    e = np.floor(np.log2(a))
+    return 0.5 * 2.0 ** (np.maximum(e, -126) - 7)
+
+
+def check_outputs(gpu_bf16: np.ndarray, orc: np.ndarray):
+    err = np.abs(gpu_bf16.astype(np.float64) - orc)
+    tol = OUT_ABS + bf16_half_ulp(orc)
+    bad = err > tol
+    assert not bad.any(), f"{int(bad.sum())} outputs outside tolerance; max err {float(err.max()):.3e}"
+    return float(err.max())

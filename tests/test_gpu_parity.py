@@ -1,0 +1,350 @@
+"""CUDA path vs the float64 oracle, through the C ABI, on seeded inputs.
+
+Small cases compare every output; the full-size workloads (the 8B-layer
+write path, the GQA decode over 32 x 32K tokens, the 262K-token decode and
+2,048-query prefill, the 1M x 1024 search) compare sampled rows the oracle
+recomputes one by one.  Exemptions and tolerances are in parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import parity
+from kv_cache_vector_07_b200 import synth, tqkv
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+class Codec:
+    """Library and oracle parameters for one cache configuration."""
+
+    def __init__(self, d, kbits, kqjl, vbits, seed, page_tokens=64, H=1):
+        self.desc = tqkv.cache_desc(d, kbits, kqjl, vbits, page_tokens=page_tokens, n_kv_heads=H)
+        self.lay = O.Layout(d, kbits, kqjl, vbits, page_tokens=page_tokens)
+        self.kp = tqkv.make_params(d, kbits, 1000 + seed)
+        self.Pk = O.make_params(d, kbits, 1000 + seed)
+        self.vp = tqkv.make_params(d, vbits, 2000 + seed) if vbits else None
+        self.Pv = O.make_params(d, vbits, 2000 + seed, with_S=False) if vbits else None
+        self.d, self.kbits, self.kqjl, self.vbits, self.H, self.P = d, kbits, kqjl, vbits, H, page_tokens
+
+    def encode(self, K, V, slots, num_blocks):
+        cache = tqkv.alloc_cache(self.desc, num_blocks)
+        ws = tqkv.encode(self.kp, self.vp, self.desc, K, V, slots, cache)
+        torch.cuda.synchronize()
+        return cache, tqkv.read_status(ws)
+
+    def check_tokens(self, cache_np, slots_np, Kx, Vx, head):
+        """Compare the stored fields of the given tokens of one head."""
+        gpu = O.read_cache(self.lay, cache_np, slots_np, head, self.H)
+        Ek = O.encode(Kx, self.Pk, qjl=self.kqjl)
+        repk, exk = parity.compare_vectors(gpu, Ek, key=True, bits=self.kbits)
+        Ev = repv = None
+        if self.vbits:
+            Ev = O.encode(Vx, self.Pv, qjl=False)
+            repv, _ = parity.compare_vectors(gpu, Ev, key=False, bits=self.vbits)
+        return Ek, Ev, exk, repk, repv
+
+
+def cache_np(cache):
+    return cache.view(cache.shape[0] * cache.shape[1], -1).cpu().numpy()
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# single-head check: 1,024 keys/values (fp32, channels 5 and 77 x20), 16 queries
+# ---------------------------------------------------------------------------
+def test_single_head_small_check_every_output():
+    d, L = 128, 1024
+    Kh, Vh, Qh = synth.small_check(seed=0)
+    cd = Codec(d, 3, True, 3, seed=0, page_tokens=64, H=1)
+    bt, slots, nblk = synth.contiguous_block_table(1, L, 64, device=DEV, shuffle_seed=5)
+    K = torch.from_numpy(Kh).to(DEV).view(L, 1, d)
+    V = torch.from_numpy(Vh).to(DEV).view(L, 1, d)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    cn = cache_np(cache)
+    Ek, Ev, exk, repk, repv = cd.check_tokens(cn, slots.cpu().numpy(), Kh.astype(np.float64),
+                                              Vh.astype(np.float64), 0)
+    # every query attends the whole cache: 16 sequences sharing one block table
+    nq = Qh.shape[0]
+    Qb = torch.from_numpy(Qh).to(DEV).to(torch.bfloat16).view(nq, 1, d)
+    btq = bt.expand(nq, -1).contiguous()
+    seq = torch.full((nq,), L, dtype=torch.int32, device=DEV)
+    logits = torch.full((nq, 1, L), float("nan"), device=DEV)
+    lse = torch.empty((nq, 1), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Qb, btq, seq, L, cache, lse=lse, logits=logits)
+    torch.cuda.synchronize()
+    Qx = f64(Qb.view(nq, d))
+    o_ref, lse_ref, lg_ref = O.attend(Qx, cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+    parity.check_logits(f64(logits.view(nq, L)), lg_ref, exk)
+    parity.check_outputs(f64(out.view(nq, d)), o_ref)
+    assert np.allclose(f64(lse.view(nq)), lse_ref, rtol=1e-3, atol=1e-3)
+    # the same 16 queries as the last 16 positions of a prefill chunk
+    C = nq
+    outp = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qb, bt.view(-1), L, cache)
+    torch.cuda.synchronize()
+    nvis = np.arange(L - C + 1, L + 1, dtype=np.int32)
+    o_p, _, _ = O.attend(Qx, cd.Pk, Ek, cd.Pv, Ev, nvis=nvis)
+    parity.check_outputs(f64(outp.view(C, d)), o_p)
+
+
+# ---------------------------------------------------------------------------
+# write path of an 8B-dense-shaped layer: B=8, Hkv=8, d=128, 32,768 tokens
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("preset", ["k8v4", "k4qjl_v4"])
+def test_write_path_full_size_sampled(preset):
+    B, L, H, d, P = 8, 32768, 8, 128, 64
+    n = B * L
+    K = synth.lognormal_channels(n, H, d, seed=1, device=DEV)
+    V = synth.lognormal_channels(n, H, d, seed=10001, device=DEV)
+    cd = Codec(d, 8, False, 4, seed=1, H=H) if preset == "k8v4" else Codec(d, 4, True, 4, seed=1, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=11)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    cn = cache_np(cache)
+    rng = np.random.default_rng(3)
+    toks = np.sort(rng.choice(n, 2048, replace=False))
+    toks[0], toks[-1] = 0, n - 1
+    sl = slots.cpu().numpy()[toks]
+    Kt, Vt = f64(K[toks]), f64(V[toks])
+    reports = []
+    for h in range(H):
+        _, _, _, repk, repv = cd.check_tokens(cn, sl, Kt[:, h], Vt[:, h], h)
+        reports.append((repk, repv))
+    print(preset, reports[0])
+    if preset != "k8v4":
+        # one GQA decode step (32 query heads) over the freshly written cache
+        Q = synth.normal((B, 32, d), seed=12, device=DEV)
+        seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+        logits = torch.full((B, 32, L), float("nan"), device=DEV)
+        out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, logits=logits)
+        torch.cuda.synchronize()
+        for b, kvh in [(0, 0), (7, 5)]:
+            idx = np.arange(b * L, (b + 1) * L)
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, slots.cpu().numpy()[idx], f64(K[idx, kvh]), f64(V[idx, kvh]),
+                                                kvh)
+            rows = list(range(kvh * 4, kvh * 4 + 4))
+            o_ref, _, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref)
+
+
+# ---------------------------------------------------------------------------
+# GQA decode: B=32, Hq=32 over Hkv=8, L=32,768, K 2-bit + QJL, V 4-bit
+# ---------------------------------------------------------------------------
+def test_decode_gqa_32x32k_sampled_rows():
+    B, L, H, Hq, d, P = 32, 32768, 8, 32, 128, 64
+    n = B * L
+    K = synth.outlier_normal((n, H, d), seed=2, device=DEV)
+    V = synth.outlier_normal((n, H, d), seed=20002, device=DEV)
+    Q = synth.normal((B, Hq, d), seed=21, device=DEV)
+    cd = Codec(d, 2, True, 4, seed=2, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=22)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    lse = torch.empty((B, Hq), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, lse=lse, logits=logits)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b, kvh in [(0, 0), (31, 7), (13, 3)]:
+        idx = np.arange(b * L, (b + 1) * L)
+        Ek, Ev, exk, repk, _ = cd.check_tokens(cn, sl[idx], f64(K[idx, kvh]), f64(V[idx, kvh]), kvh)
+        rows = list(range(kvh * G, kvh * G + G))
+        o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+        parity.check_logits(f64(logits[b, rows]), lg_ref, exk)
+        parity.check_outputs(f64(out[b, rows]), o_ref)
+        assert np.allclose(f64(lse[b, rows]), lse_ref, rtol=1e-3, atol=1e-3)
+
+
+# ---------------------------------------------------------------------------
+# long context: B=1, Hq=32 over Hkv=4, L=262,144, 3-bit keys incl. QJL, 3-bit
+# values; one decode step and one 2,048-query prefill chunk (causal inside)
+# ---------------------------------------------------------------------------
+def test_long_context_decode_and_prefill_sampled():
+    L, H, Hq, d, P, C = 262144, 4, 32, 128, 64, 2048
+    K = synth.outlier_normal((L, H, d), seed=3, device=DEV)
+    V = synth.outlier_normal((L, H, d), seed=30003, device=DEV)
+    cd = Codec(d, 2, True, 3, seed=3, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(1, L, P, device=DEV, shuffle_seed=33)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    Qd = synth.normal((1, Hq, d), seed=31, device=DEV)
+    seq = torch.full((1,), L, dtype=torch.int32, device=DEV)
+    logits = torch.full((1, Hq, L), float("nan"), device=DEV)
+    out_d = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Qd, bt, seq, L, cache, logits=logits)
+    Qp = synth.normal((C, Hq, d), seed=32, device=DEV)
+    out_p = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qp, bt.view(-1), L, cache)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for kvh in (0, 3):
+        Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl, f64(K[:, kvh]), f64(V[:, kvh]), kvh)
+        rows = list(range(kvh * G, kvh * G + G))
+        o_ref, _, lg_ref = O.attend(f64(Qd[0, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+        parity.check_logits(f64(logits[0, rows]), lg_ref, exk)
+        parity.check_outputs(f64(out_d[0, rows]), o_ref)
+        for j in (0, 1, 777, C - 1):
+            nvis = np.full(G, L - C + j + 1, np.int32)
+            o_p, _, _ = O.attend(f64(Qp[j, rows]), cd.Pk, Ek, cd.Pv, Ev, nvis=nvis)
+            parity.check_outputs(f64(out_p[j, rows]), o_p)
+
+
+# ---------------------------------------------------------------------------
+# search
+# ---------------------------------------------------------------------------
+def _search_case(n_db, n_q, seed, d=1024):
+    X = synth.unit_normal(n_db, d, seed=seed, device=DEV)
+    Qs = synth.unit_normal(n_q, d, seed=seed + 1, device=DEV)
+    cd = Codec(d, 4, True, 0, seed=seed, H=1)
+    nblk = -(-n_db // 64)
+    slots = torch.arange(n_db, dtype=torch.int32, device=DEV)
+    cache, flags = cd.encode(X, None, slots, nblk)
+    assert flags == 0
+    return X, Qs, cd, cache
+
+
+def test_search_reduced_every_output():
+    n_db, n_q, k = 20000, 16, 10
+    X, Qs, cd, cache = _search_case(n_db, n_q, seed=4)
+    sc, ix = tqkv.score(cd.kp, cd.desc, cache, n_db, Qs, k)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    Ek, _, exk, _, _ = cd.check_tokens(cn, np.arange(n_db), f64(X), None, 0)
+    ref_sc, ref_ix = O.search(f64(Qs), cd.Pk, Ek, k + 1)
+    gs, gi = f64(sc), ix.cpu().numpy()
+    for a in range(n_q):
+        est = O.estimate(f64(Qs[a]), cd.Pk, Ek)
+        # GPU scores equal the oracle estimates of the returned vectors
+        tol = 1e-3 * np.maximum(np.abs(est[gi[a]]), np.sqrt(np.mean(est ** 2)))
+        ok = (np.abs(gs[a] - est[gi[a]]) <= tol) | exk[gi[a]]
+        assert ok.all()
+        # the returned set is the oracle's top-k unless the k-th/(k+1)-th gap is within tolerance
+        if ref_sc[a, k - 1] - ref_sc[a, k] > 2e-3 * abs(ref_sc[a, k - 1]):
+            assert set(gi[a]) == set(ref_ix[a, :k]) or exk[ref_ix[a, :k]].any()
+        assert np.all(np.diff(gs[a]) <= 0)
+
+
+def test_search_million_vectors_properties():
+    n_db, n_q, k = 1_000_000, 1024, 10
+    X, Qs, cd, cache = _search_case(n_db, n_q, seed=4)
+    sc, ix = tqkv.score(cd.kp, cd.desc, cache, n_db, Qs, k)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    rng = np.random.default_rng(44)
+    sample = np.sort(rng.choice(n_db, 1000, replace=False))
+    cd.check_tokens(cn, sample, f64(X[sample]), None, 0)
+    gs, gi = f64(sc), ix.cpu().numpy()
+    for a in rng.choice(n_q, 8, replace=False):
+        cand = np.unique(np.concatenate([gi[a], sample]))
+        Ek, _, exk, _, _ = cd.check_tokens(cn, cand, f64(X[cand]), None, 0)
+        est = O.estimate(f64(Qs[a]), cd.Pk, Ek)
+        pos = {int(t): i for i, t in enumerate(cand)}
+        mine = np.array([est[pos[int(t)]] for t in gi[a]])
+        rms = np.sqrt(np.mean(est ** 2))
+        assert np.all(np.abs(gs[a] - mine) <= 1e-3 * np.maximum(np.abs(mine), rms))
+        others = np.array([est[pos[int(t)]] for t in sample if int(t) not in set(gi[a].tolist())])
+        assert gs[a, k - 1] >= others.max() - 1e-3 * rms
+    exact = torch.topk(Qs @ X.T, k, dim=1).indices.cpu().numpy()
+    recall = np.mean([len(set(gi[a]) & set(exact[a])) / k for a in range(n_q)])
+    print(f"recall@10 vs exact fp32: {recall:.4f}")
+    assert recall > 0.3
+
+
+# ---------------------------------------------------------------------------
+# edge cases: small and large head dims, ragged and empty sequences, skipped
+# slots, zero vectors, out-of-range slots, G = 1 and 8
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,kbits,kqjl,vbits,P,Hq,H", [(8, 2, True, 1, 8, 2, 1), (16, 1, True, 2, 16, 8, 1),
+                                                       (64, 3, True, 2, 16, 4, 2), (256, 4, False, 3, 32, 1, 1),
+                                                       (128, 4, True, 4, 16, 8, 1), (32, 2, True, 4, 8, 6, 3)])
+def test_small_dims_ragged_sequences(d, kbits, kqjl, vbits, P, Hq, H):
+    seqs = [0, 1, 37, 3 * P + 5]
+    B, Lmax = len(seqs), max(seqs)
+    cd = Codec(d, kbits, kqjl, vbits, seed=d + kbits, page_tokens=P, H=H)
+    bps = -(-Lmax // P)
+    g = torch.Generator().manual_seed(d)
+    phys = torch.randperm(B * bps + 3, generator=g)[:B * bps].view(B, bps).to(torch.int32)
+    nblk = B * bps + 3
+    toks, slot_list = [], []
+    for b, Lb in enumerate(seqs):
+        for t in range(Lb):
+            toks.append((b, t))
+            slot_list.append(int(phys[b, t // P]) * P + t % P)
+    n = len(toks)
+    # append two skipped tokens (slot -1): their inputs must not reach the cache
+    slot_list += [-1, -1]
+    K = synth.outlier_normal((n + 2, H, d), seed=d, device=DEV, dtype=torch.float32)
+    V = synth.outlier_normal((n + 2, H, d), seed=d + 1, device=DEV, dtype=torch.float32)
+    K[0].zero_()            # a zero vector
+    slots = torch.tensor(slot_list, dtype=torch.int32, device=DEV)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    cn = cache_np(cache)
+    sl = np.array(slot_list[:n])
+    for h in range(H):
+        cd.check_tokens(cn, sl, f64(K[:n, h]), f64(V[:n, h]), h)
+    # bytes of pages no token was written to stay zero
+    used = set(int(s) // P for s in slot_list[:n])
+    unused = [blk for blk in range(nblk) if blk not in used]
+    assert not cache[unused].any()
+    Q = synth.normal((B, Hq, d), seed=d + 2, device=DEV)
+    bt = phys.to(DEV)
+    seq = torch.tensor(seqs, dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, Lmax), float("nan"), device=DEV)
+    lse = torch.empty((B, Hq), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, Lmax, cache, lse=lse, logits=logits)
+    torch.cuda.synchronize()
+    G = Hq // H
+    start = 0
+    for b, Lb in enumerate(seqs):
+        for kvh in range(H):
+            rows = list(range(kvh * G, kvh * G + G))
+            if Lb == 0:
+                assert torch.all(out[b, rows] == 0)
+                assert torch.all(torch.isneginf(lse[b, rows]))
+                continue
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl[start:start + Lb], f64(K[start:start + Lb, kvh]),
+                                                f64(V[start:start + Lb, kvh]), kvh)
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :Lb]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref)
+        start += Lb
+
+
+def test_out_of_range_slot_is_flagged_and_skipped():
+    cd = Codec(128, 2, True, 4, seed=9, page_tokens=16, H=1)
+    K = synth.normal((4, 1, 128), seed=1, device=DEV)
+    slots = torch.tensor([0, 1, 10_000, 2], dtype=torch.int32, device=DEV)
+    cache, flags = cd.encode(K, K, slots, 1)
+    assert flags & tqkv.TQ_DEV_SLOT_RANGE
+    cn = cache_np(cache)
+    Kx = f64(K[[0, 1, 3], 0])
+    cd.check_tokens(cn, np.array([0, 1, 2]), Kx, Kx, 0)
+
+
+def test_block_table_out_of_range_is_flagged():
+    cd = Codec(128, 2, True, 4, seed=9, page_tokens=16, H=1)
+    K = synth.normal((16, 1, 128), seed=1, device=DEV)
+    slots = torch.arange(16, dtype=torch.int32, device=DEV)
+    cache, _ = cd.encode(K, K, slots, 1)
+    Q = synth.normal((1, 1, 128), seed=2, device=DEV)
+    bt = torch.tensor([[0, 5]], dtype=torch.int32, device=DEV)     # block 5 does not exist
+    seq = torch.tensor([20], dtype=torch.int32, device=DEV)
+    ws = torch.zeros(tqkv.decode_workspace_bytes(cd.desc, 1, 1, 20), dtype=torch.uint8, device=DEV)
+    tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, 20, cache, workspace=ws)
+    assert tqkv.read_status(ws) & tqkv.TQ_DEV_BLOCK_RANGE
