@@ -50,7 +50,9 @@ enum tq_status {
     TQ_EUNSUPPORTED = 2,  /* valid but unsupported (e.g. d not a power of 2) */
     TQ_ECUDA = 3,         /* a CUDA runtime call or launch failed            */
     TQ_EDEVICE = 4,       /* a kernel reported an error in the status word   */
-    TQ_ENOMEM = 5         /* tq_make_params could not allocate               */
+    TQ_ENOMEM = 5,        /* tq_make_params could not allocate               */
+    TQ_ESCRATCH = 6       /* problem needs more scratch than
+                             tq_decode_attn_noalloc's static array holds     */
 };
 
 /* Bits of the device status word written by kernels (see tq_read_status). */
@@ -172,6 +174,32 @@ int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq_cache_desc
                    int64_t num_blocks, void *out, float *lse, float *logits,
                    int64_t logits_stride, void *workspace, size_t workspace_bytes,
                    void *stream);
+
+/* Decode attention without any device allocation, for callers that cannot
+ * allocate device memory (an engine that keeps all device memory in its own
+ * pool and forbids other allocations, a plug-in handed only one call's
+ * tensors, a latency-critical path that cannot afford a blocking cudaMalloc).
+ * The paper has no counterpart: this is a library convenience.  Same
+ * arguments and results as tq_decode_attn minus the workspace, which is
+ * replaced by a file-scope device array of TQ_NOALLOC_SCRATCH_BYTES bytes
+ * that every GPU loading the library holds until the process exits.
+ * - Sizes whose tq_decode_workspace_bytes exceeds TQ_NOALLOC_SCRATCH_BYTES
+ *   are rejected with TQ_ESCRATCH before anything is launched.
+ * - No cudaMalloc, cudaFree or allocating library routine is called.
+ * - The first call on a device looks up the array's device address with that
+ *   device current (cudaGetSymbolAddress) and caches it; make that first call
+ *   before any stream capture.
+ * - All calls on a device share the array, which keeps the last call's
+ *   contents; the status word at its start is cleared on every call (its
+ *   flags cannot be read back through this entry point).  Calls whose
+ *   execution overlaps on the GPU (different streams, or streams without an
+ *   ordering between them) race on the array and give undefined results. */
+#define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+int tq_decode_attn_noalloc(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc,
+                           const void *Q, int B, int Hq, const int32_t *block_table, int max_blocks,
+                           const int32_t *seq_lens, int max_seq_len, const void *cache,
+                           int64_t num_blocks, void *out, float *lse, float *logits,
+                           int64_t logits_stride, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Chunked prefill over the compressed cache (one sequence)                 */

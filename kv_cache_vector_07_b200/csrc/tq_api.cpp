@@ -207,6 +207,7 @@ extern "C" const char *tq_status_string(int status) {
         case TQ_ECUDA: return "CUDA error";
         case TQ_EDEVICE: return "device-side error flagged in the workspace status word";
         case TQ_ENOMEM: return "out of memory";
+        case TQ_ESCRATCH: return "problem needs more scratch than the no-allocation entry point's static array";
     }
     return "unknown status";
 }

@@ -26,7 +26,8 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"libtqkv.so is not built ({LIB_PATH}); run `python -m kv_cache_vector_07_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_EDEVICE, TQ_ENOMEM = range(6)
+TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_EDEVICE, TQ_ENOMEM, TQ_ESCRATCH = range(7)
+TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 TQ_DEV_SLOT_RANGE, TQ_DEV_BLOCK_RANGE, TQ_DEV_WAIT_TIMEOUT = 0x1, 0x2, 0x4
 TQ_DTYPE_BF16, TQ_DTYPE_F32 = 0, 1
 
@@ -61,6 +62,8 @@ _sig("tq_encode", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _vp, _i32, _i
 _sig("tq_decode_workspace_bytes", _sz, [ctypes.POINTER(CacheDesc), _i32, _i32, _i32])
 _sig("tq_decode_attn", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i32, _vp, _i32, _vp, _i32, _vp,
                               _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("tq_decode_attn_noalloc", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i32, _vp, _i32, _vp, _i32,
+                                      _vp, _i64, _vp, _vp, _vp, _i64, _vp])
 _sig("tq_prefill_workspace_bytes", _sz, [ctypes.POINTER(CacheDesc), _i32, _i32, _i32])
 _sig("tq_prefill_attn", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
                                _vp, _vp, _vp, _sz, _vp])
@@ -239,6 +242,24 @@ def decode_attn(kp: Params, vp: Params, desc: CacheDesc, Q: torch.Tensor, block_
                                block_table.shape[1], _ptr(seq_lens), max_seq_len, _ptr(cache), cache.shape[0],
                                _ptr(out), _ptr(lse), _ptr(logits), stride, _ptr(workspace), workspace.numel(),
                                _stream(stream)), "tq_decode_attn")
+    return out
+
+
+def decode_attn_noalloc(kp: Params, vp: Params, desc: CacheDesc, Q: torch.Tensor, block_table: torch.Tensor,
+                        seq_lens: torch.Tensor, max_seq_len: int, cache: torch.Tensor, out: torch.Tensor | None = None,
+                        lse: torch.Tensor | None = None, logits: torch.Tensor | None = None, stream=None):
+    """tq_decode_attn_noalloc: tq_decode_attn for callers that cannot allocate
+    device memory; the scratch is the library's static device array, shared
+    by all calls on the device (calls that overlap on the GPU race)."""
+    _dev_check(Q, block_table, seq_lens, cache, out, lse, logits)
+    B, Hq, d = Q.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    stride = logits.shape[-1] if logits is not None else 0
+    _check(_lib.tq_decode_attn_noalloc(kp.handle, vp.handle, ctypes.byref(desc), _ptr(Q), B, Hq, _ptr(block_table),
+                                       block_table.shape[1], _ptr(seq_lens), max_seq_len, _ptr(cache),
+                                       cache.shape[0], _ptr(out), _ptr(lse), _ptr(logits), stride, _stream(stream)),
+           "tq_decode_attn_noalloc")
     return out
 
 
