@@ -174,7 +174,7 @@ class StepWorkload:
         per_tok = page // P
         self.enc_bytes = 2 * n * H * d * 2 + n * H * per_tok
         self.dec_bytes = B * H * L * per_tok + 2 * self.Q.numel() * 2
-        self.launches = {"encode": 2, "decode": 3}
+        self.launches = {"encode": 1, "decode": 3}
 
     def ops(self):
         tq = self.tq
@@ -209,7 +209,7 @@ class StepWorkload:
         dec_gbs = self.dec_bytes / (op_ms["decode"] * 1e-3) / 1e9
         return ({"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                  "frac": round(enc_gbs / hbm_peak, 4), "traffic": traffic_for("encode"),
-                 "kernel": "tq_encode (encode_kernel + qjl_gemm_kernel)",
+                 "kernel": "tq_encode (encode128_kernel: TMA + tcgen05 rotation + quantize + tcgen05 QJL)",
                  "algorithmic_bytes": self.enc_bytes},
                 {"encode": {"vectors_per_s": self.n_vec / (op_ms["encode"] * 1e-3), "ms": op_ms["encode"],
                             "gbs": enc_gbs, "frac": enc_gbs / hbm_peak, "algorithmic_bytes": self.enc_bytes},

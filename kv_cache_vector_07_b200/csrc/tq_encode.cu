@@ -164,7 +164,7 @@ struct QjlArgs {
 
 constexpr int kBM = 128;       // vectors per tile (MMA M)
 constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
-constexpr uint32_t kMaxPolls = 1u << 24;
+constexpr uint32_t kMaxPolls = 1u << 20;   // about a second of polling, then give up
 
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
     __nv_bfloat16 b = __float2bfloat16_rn(x);
@@ -402,6 +402,10 @@ int launch_encode(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.status = reinterpret_cast<uint32_t *>(ws);
     a.do_v = L.vbits > 0 ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (in_dtype == TQ_DTYPE_BF16) {
+        const int r = launch_encode128(kp, vp, L, K, V, n_tokens, slots, cache, num_blocks, ws, stream);
+        if (r >= 0) return r;
+    }
     switch (L.d) {
         case 8: return launch_encode_d<8>(a, in_dtype, kp, st);
         case 16: return launch_encode_d<16>(a, in_dtype, kp, st);

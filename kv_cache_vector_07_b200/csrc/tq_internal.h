@@ -65,7 +65,21 @@ struct DevParams {
     const uint16_t *S;       // [d][d] bf16 bits, row-major (row j = projection j)
     const float *lv;         // [2^bits] levels indexed by the stored sign-magnitude code
     const float *bounds;     // [2^bits - 1] ascending decision boundaries
+    // d == 128 only (else null): 32 KB images of 128 x 128 operand tiles laid
+    // out exactly as the tensor cores read them from shared memory (K-major,
+    // 128-byte swizzle, two 64-column halves), so one bulk copy stages them.
+    const uint8_t *rot_img;  // bf16 (H D)[n][k] = (-1)^popcount(n & k) * D[k]
+    const uint8_t *s16_img;  // fp16 S[n][k] (exact for |S| >= 2^-17)
 };
+
+// Byte offset of element (row, col) of a 128 x 128 16-bit tile in the
+// 128-byte-swizzled K-major image: column half col / 64 at 16 KB, rows of 128
+// bytes, the 16-byte piece index XORed with row % 8.
+inline size_t sw128_image_offset(int row, int col) {
+    const int half = col >> 6, c = col & 63;
+    const int piece = c >> 3, e = c & 7;
+    return size_t(half) * 16384 + size_t(row) * 128 + size_t(((piece ^ (row & 7)) << 4) + e * 2);
+}
 
 }  // namespace tq
 
@@ -91,6 +105,10 @@ int launch_encode(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   const void *V, int in_dtype, int64_t n_tokens, const int32_t *slots,
                   uint8_t *cache, int64_t num_blocks, uint8_t *ws, size_t ws_bytes, void *stream);
 size_t encode_ws_bytes(const Layout &L, int64_t n_tokens);
+// Fused d = 128 bf16 encoder; returns -1 when the configuration is not covered.
+int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, const void *K, const void *V,
+                     int64_t n_tokens, const int32_t *slots, uint8_t *cache, int64_t num_blocks, uint8_t *ws,
+                     void *stream);
 
 struct AttnShape {
     int n_seq;            // decode: batch; prefill: chunk length C

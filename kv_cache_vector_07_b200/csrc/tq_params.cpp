@@ -10,6 +10,7 @@
 #include <new>
 #include <vector>
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "tq_internal.h"
@@ -261,12 +262,31 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
         }
     }
 
-    // one device block: signs | S (bf16) | levels by code | bounds
+    // Operand images for the d = 128 tensor-core encoder.
+    const bool imgs = d == 128;
+    std::vector<uint16_t> rot_img, s16_img;
+    if (imgs) {
+        rot_img.assign(128 * 128, 0);
+        s16_img.assign(128 * 128, 0);
+        for (int n = 0; n < 128; ++n)
+            for (int k = 0; k < 128; ++k) {
+                const bool neg = (__builtin_popcount(unsigned(n & k)) & 1) != (sg[k] < 0);
+                rot_img[tq::sw128_image_offset(n, k) / 2] = neg ? 0xBF80 : 0x3F80;       // bf16 -1 / +1
+                const __half h = __float2half_rn(bf16_to_float(S_bits[size_t(n) * 128 + k]));
+                uint16_t hb;
+                std::memcpy(&hb, &h, 2);
+                s16_img[tq::sw128_image_offset(n, k) / 2] = hb;
+            }
+    }
+
+    // one device block: signs | S (bf16) | levels by code | bounds | images
     const size_t off_signs = 0;
     const size_t off_S = 256 * ((sizeof(float) * d + 255) / 256);
     const size_t off_lv = off_S + 256 * ((sizeof(uint16_t) * dd + 255) / 256);
     const size_t off_bd = off_lv + 256;
-    const size_t total = off_bd + 256;
+    const size_t off_rot = off_bd + 256;
+    const size_t off_s16 = off_rot + (imgs ? 32768 : 0);
+    const size_t total = off_s16 + (imgs ? 32768 : 0);
     if (cudaMalloc(&p->d_block, total) != cudaSuccess) { p->d_block = nullptr; tq_free_params(p); return TQ_ENOMEM; }
     uint8_t *base = static_cast<uint8_t *>(p->d_block);
     std::vector<float> bd(L > 1 ? L - 1 : 1, 0.0f);
@@ -274,7 +294,9 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
     if (cudaMemcpy(base + off_signs, signs_f.data(), sizeof(float) * d, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(base + off_S, S_bits.data(), sizeof(uint16_t) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(base + off_lv, lv_code.data(), sizeof(float) * lv_code.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(base + off_bd, bd.data(), sizeof(float) * bd.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaMemcpy(base + off_bd, bd.data(), sizeof(float) * bd.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+        (imgs && (cudaMemcpy(base + off_rot, rot_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess ||
+                  cudaMemcpy(base + off_s16, s16_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess))) {
         tq_free_params(p);
         return TQ_ECUDA;
     }
@@ -284,6 +306,8 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
     p->dev.S = reinterpret_cast<const uint16_t *>(base + off_S);
     p->dev.lv = reinterpret_cast<const float *>(base + off_lv);
     p->dev.bounds = reinterpret_cast<const float *>(base + off_bd);
+    p->dev.rot_img = imgs ? base + off_rot : nullptr;
+    p->dev.s16_img = imgs ? base + off_s16 : nullptr;
     *out = p;
     return TQ_OK;
 }

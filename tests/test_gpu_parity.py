@@ -46,10 +46,16 @@ class Codec:
         Ek = O.encode(Kx, self.Pk, qjl=self.kqjl)
         repk, exk = parity.compare_vectors(gpu, Ek, key=True, bits=self.kbits)
         Ev = repv = None
+        self.last_exempt = exk
         if self.vbits:
             Ev = O.encode(Vx, self.Pv, qjl=False)
-            repv, _ = parity.compare_vectors(gpu, Ev, key=False, bits=self.vbits)
+            repv, exv = parity.compare_vectors(gpu, Ev, key=False, bits=self.vbits)
+            self.last_exempt = exk | exv
         return Ek, Ev, exk, repk, repv
+
+    def slack(self, Ev, logits, lse, out):
+        """Per-row output allowance from the keys exempt in the last check."""
+        return parity.exempt_slack(self.Pv, Ev, self.last_exempt, logits, lse, out)
 
 
 def cache_np(cache):
@@ -87,15 +93,15 @@ def test_single_head_small_check_every_output():
     Qx = f64(Qb.view(nq, d))
     o_ref, lse_ref, lg_ref = O.attend(Qx, cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
     parity.check_logits(f64(logits.view(nq, L)), lg_ref, exk)
-    parity.check_outputs(f64(out.view(nq, d)), o_ref)
+    parity.check_outputs(f64(out.view(nq, d)), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
     assert np.allclose(f64(lse.view(nq)), lse_ref, rtol=1e-3, atol=1e-3)
     # the same 16 queries as the last 16 positions of a prefill chunk
     C = nq
     outp = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qb, bt.view(-1), L, cache)
     torch.cuda.synchronize()
     nvis = np.arange(L - C + 1, L + 1, dtype=np.int32)
-    o_p, _, _ = O.attend(Qx, cd.Pk, Ek, cd.Pv, Ev, nvis=nvis)
-    parity.check_outputs(f64(outp.view(C, d)), o_p)
+    o_p, lse_p, lg_p = O.attend(Qx, cd.Pk, Ek, cd.Pv, Ev, nvis=nvis, want_logits=True)
+    parity.check_outputs(f64(outp.view(C, d)), o_p, cd.slack(Ev, lg_p, lse_p, o_p))
 
 
 # ---------------------------------------------------------------------------
@@ -134,9 +140,9 @@ def test_write_path_full_size_sampled(preset):
             Ek, Ev, exk, _, _ = cd.check_tokens(cn, slots.cpu().numpy()[idx], f64(K[idx, kvh]), f64(V[idx, kvh]),
                                                 kvh)
             rows = list(range(kvh * 4, kvh * 4 + 4))
-            o_ref, _, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
             parity.check_logits(f64(logits[b, rows]), lg_ref, exk)
-            parity.check_outputs(f64(out[b, rows]), o_ref)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
 
 
 # ---------------------------------------------------------------------------
@@ -166,7 +172,7 @@ def test_decode_gqa_32x32k_sampled_rows():
         rows = list(range(kvh * G, kvh * G + G))
         o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
         parity.check_logits(f64(logits[b, rows]), lg_ref, exk)
-        parity.check_outputs(f64(out[b, rows]), o_ref)
+        parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
         assert np.allclose(f64(lse[b, rows]), lse_ref, rtol=1e-3, atol=1e-3)
 
 
@@ -195,13 +201,13 @@ def test_long_context_decode_and_prefill_sampled():
     for kvh in (0, 3):
         Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl, f64(K[:, kvh]), f64(V[:, kvh]), kvh)
         rows = list(range(kvh * G, kvh * G + G))
-        o_ref, _, lg_ref = O.attend(f64(Qd[0, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+        o_ref, lse_ref, lg_ref = O.attend(f64(Qd[0, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
         parity.check_logits(f64(logits[0, rows]), lg_ref, exk)
-        parity.check_outputs(f64(out_d[0, rows]), o_ref)
+        parity.check_outputs(f64(out_d[0, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
         for j in (0, 1, 777, C - 1):
             nvis = np.full(G, L - C + j + 1, np.int32)
-            o_p, _, _ = O.attend(f64(Qp[j, rows]), cd.Pk, Ek, cd.Pv, Ev, nvis=nvis)
-            parity.check_outputs(f64(out_p[j, rows]), o_p)
+            o_p, lse_p, lg_p = O.attend(f64(Qp[j, rows]), cd.Pk, Ek, cd.Pv, Ev, nvis=nvis, want_logits=True)
+            parity.check_outputs(f64(out_p[j, rows]), o_p, cd.slack(Ev, lg_p, lse_p, o_p))
 
 
 # ---------------------------------------------------------------------------
@@ -322,7 +328,7 @@ def test_small_dims_ragged_sequences(d, kbits, kqjl, vbits, P, Hq, H):
                                                 f64(V[start:start + Lb, kvh]), kvh)
             o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
             parity.check_logits(f64(logits[b, rows, :Lb]), lg_ref, exk)
-            parity.check_outputs(f64(out[b, rows]), o_ref)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
         start += Lb
 
 
@@ -348,3 +354,32 @@ def test_block_table_out_of_range_is_flagged():
     ws = torch.zeros(tqkv.decode_workspace_bytes(cd.desc, 1, 1, 20), dtype=torch.uint8, device=DEV)
     tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, 20, cache, workspace=ws)
     assert tqkv.read_status(ws) & tqkv.TQ_DEV_BLOCK_RANGE
+
+
+# ---------------------------------------------------------------------------
+# every configuration of the fused d = 128 bf16 encoder: ragged tail tiles,
+# skipped slots, a zero vector, three KV heads
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kbits,kqjl,vbits", [(4, True, 4), (2, True, 4), (2, True, 3), (3, True, 3), (3, True, 4),
+                                              (8, False, 4), (4, False, 4), (3, False, 3), (4, True, 0)])
+def test_fused_encoder_configurations(kbits, kqjl, vbits):
+    d, H, P = 128, 3, 16
+    n = 1000                                  # 3,000 vectors: 23 full tiles and a ragged one
+    cd = Codec(d, kbits, kqjl, vbits, seed=40 + kbits + vbits, page_tokens=P, H=H)
+    K = synth.lognormal_channels(n, H, d, seed=41, device=DEV)
+    V = synth.lognormal_channels(n, H, d, seed=42, device=DEV) if vbits else None
+    K[7].zero_()
+    if V is not None:
+        V[9].zero_()
+    g = torch.Generator().manual_seed(43)
+    nblk = -(-n // P) + 2
+    perm = torch.randperm(nblk * P, generator=g)[:n].to(torch.int32)
+    perm[[5, 500]] = -1                       # skipped tokens
+    slots = perm.to(DEV)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    cn = cache_np(cache)
+    keep = np.flatnonzero(perm.numpy() >= 0)
+    sl = perm.numpy()[keep]
+    for h in range(H):
+        cd.check_tokens(cn, sl, f64(K[keep, h]), f64(V[keep, h]) if vbits else None, h)
