@@ -151,7 +151,7 @@ class Params:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
+        if h is not None and h.value and _lib is not None:
             _lib.tq_free_params(h)
             self._h = _vp()
 
