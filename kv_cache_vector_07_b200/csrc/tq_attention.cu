@@ -354,6 +354,12 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
     pa.w = reinterpret_cast<float *>(ws + p.off_w);
     prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
 
+    const int fast = launch_dec128(kp, vp, L, pa.qr, pa.w, s, p.G, p.n_groups, p.n_splits, p.split_len, cache,
+                                   num_blocks, reinterpret_cast<float *>(ws + p.off_po),
+                                   reinterpret_cast<float *>(ws + p.off_pml), logits, logits_stride,
+                                   reinterpret_cast<uint32_t *>(ws), st);
+    if (fast > 0) return fast;
+
     AttnArgs a;
     a.L = L;
     a.kp = kp->dev;
@@ -377,7 +383,7 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.logits = logits;
     a.logits_stride = logits_stride;
     a.status = reinterpret_cast<uint32_t *>(ws);
-    attn_kernel<D><<<dim3(unsigned(p.n_groups), unsigned(p.n_splits)), kChunk, 0, st>>>(a);
+    if (fast < 0) attn_kernel<D><<<dim3(unsigned(p.n_groups), unsigned(p.n_splits)), kChunk, 0, st>>>(a);
 
     CombineArgs c;
     c.n_groups = p.n_groups;

@@ -5,6 +5,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "tqkv.h"
 
 #if defined(__CUDACC__)
@@ -125,6 +127,13 @@ int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, 
                      const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out,
                      float *lse, float *logits, int64_t logits_stride, uint8_t *ws,
                      size_t ws_bytes, void *stream);
+
+// Tensor-core attention for d = 128 (decode and prefill query groups);
+// returns -1 when the configuration is not covered.
+int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, const float *qr, const float *w,
+                  const AttnShape &s, int G, int n_groups, int n_splits, int split_len, const uint8_t *cache,
+                  int64_t num_blocks, float *part_o, float *part_ml, float *logits, int64_t logits_stride,
+                  uint32_t *status, cudaStream_t st);
 
 size_t score_ws_bytes(const Layout &L, int64_t n_db, int n_q, int k);
 int launch_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,

@@ -86,7 +86,9 @@ def check_logits(gpu: np.ndarray, orc: np.ndarray, exempt_keys: np.ndarray | Non
     if exempt_keys is not None:
         bad &= ~exempt_keys[None, :]
     if bad.any():
-        where = np.argwhere(bad)[:8]
+        ratio = np.where(bad, err / np.maximum(tol, 1e-30), 0.0)
+        order = np.argsort(ratio, axis=None)[::-1][:8]
+        where = np.stack(np.unravel_index(order, ratio.shape), 1)
         detail = [(int(r), int(t), float(gpu[r, t]), float(orc[r, t]), float(rms[r, 0])) for r, t in where]
         raise AssertionError(f"{int(bad.sum())} logits outside tolerance; worst rel "
                              f"{float(np.max(err / np.maximum(tol, 1e-30)) * LOGIT_REL):.3e}; "

@@ -42,7 +42,9 @@ def _run(fn, desc, kp, vp, bt, lens, cache, Q, L):
 
 def _same(a, b):
     (o1, l1, g1), (o2, l2, g2) = a, b
-    assert np.all(np.abs(o1 - o2) <= 2e-3), np.abs(o1 - o2).max()        # output tolerance of the parity tests
+    # output tolerance of the parity tests, for two bf16-rounded results
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(o2), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(o1 - o2) <= 2e-3 + ulp), np.abs(o1 - o2).max()
     rms = np.sqrt(np.mean(g2 ** 2, axis=-1, keepdims=True))
     assert np.all(np.abs(g1 - g2) <= 1e-3 * np.maximum(np.abs(g2), rms))  # logit tolerance of the parity tests
     assert np.allclose(l1, l2, rtol=1e-3, atol=1e-3)
