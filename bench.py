@@ -32,6 +32,12 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "KV vectors encoded/s + decode-attn keys scored/s; % HBM roofline (1 B200)"
+EXTRA_METRICS = {"decode32k": "decode-attn keys scored/s", "longctx": "decode + prefill (query-head, key) pairs/s",
+                 "search": "database vectors scored per query per second (top-10 search)"}
+UNIT_NOTES = {"step": "units = KV vectors encoded + (query-head, key) pairs scored",
+              "decode32k": "units = (query-head, key) pairs scored",
+              "longctx": "units = (query-head, key) pairs scored in the decode step and the prefill chunk",
+              "search": "units = (query, database vector) pairs scored"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -149,10 +155,12 @@ class StepWorkload:
     name = ("write path B=8 x Hkv=8 x 32768 tokens x d=128 bf16 (K 4-bit Lloyd-Max + 1-bit QJL, V 4-bit) "
             "+ one GQA decode step Hq=32 over the written cache")
 
-    def __init__(self, dev):
+    def __init__(self, dev, batch=8, **_):
         from kv_cache_vector_07_b200 import synth, tqkv
         self.tq = tqkv
-        B, L, H, Hq, d, P = 8, 32768, 8, 32, 128, 64
+        B, L, H, Hq, d, P = batch, 32768, 8, 32, 128, 64
+        if batch != 8:
+            self.name = self.name.replace("B=8", f"B={batch}")
         self.B, self.L, self.H, self.Hq, self.d, self.P = B, L, H, Hq, d, P
         n = B * L
         self.n_vec = 2 * n * H
@@ -226,10 +234,12 @@ class Decode32kWorkload:
     """One GQA decode step: B=32, Hq=32 over Hkv=8, L=32,768, K 2-bit + QJL, V 4-bit."""
     name = "decode B=32 x Hq=32/Hkv=8 x 32768 tokens x d=128, K 2-bit Lloyd-Max + 1-bit QJL, V 4-bit (k3v4)"
 
-    def __init__(self, dev):
+    def __init__(self, dev, batch=32, seq_len=32768, **_):
         from kv_cache_vector_07_b200 import synth, tqkv
         self.tq = tqkv
-        B, L, H, Hq, d, P = 32, 32768, 8, 32, 128, 64
+        B, L, H, Hq, d, P = batch, seq_len, 8, 32, 128, 64
+        if (batch, seq_len) != (32, 32768):
+            self.name = self.name.replace("B=32", f"B={batch}").replace("32768 tokens", f"{seq_len} tokens")
         self.B, self.L, self.H, self.Hq, self.d, self.P = B, L, H, Hq, d, P
         n = B * L
         self.desc = tqkv.cache_desc(d, 2, True, 4, page_tokens=P, n_kv_heads=H)
@@ -282,7 +292,148 @@ class Decode32kWorkload:
                 "l2": "cache (0.99 GB) larger than L2", "parallelism": "replicas"}
 
 
-WORKLOADS = {"step": StepWorkload, "decode32k": Decode32kWorkload}
+class LongCtxWorkload:
+    """Long-context GQA: B=1, Hq=32 over Hkv=4, L=262,144, K 2-bit + QJL, V
+    3-bit; one decode step plus one 2,048-query prefill chunk (causal inside)."""
+    name = ("long context B=1 x Hq=32/Hkv=4 x 262144 tokens x d=128 (K 2-bit + QJL, V 3-bit): "
+            "one decode step + one 2048-query prefill chunk")
+
+    def __init__(self, dev, seq_len=262144, chunk=2048, **_):
+        from kv_cache_vector_07_b200 import synth, tqkv
+        self.tq = tqkv
+        L, H, Hq, d, P, C = seq_len, 4, 32, 128, 64, chunk
+        self.L, self.H, self.Hq, self.d, self.P, self.C = L, H, Hq, d, P, C
+        self.desc = tqkv.cache_desc(d, 2, True, 3, page_tokens=P, n_kv_heads=H)
+        self.kp = tqkv.make_params(d, 2, 1003)
+        self.vp = tqkv.make_params(d, 3, 2003)
+        self.bt, slots, nblk = synth.contiguous_block_table(1, L, P, device=dev, shuffle_seed=33)
+        self.cache = tqkv.alloc_cache(self.desc, nblk, device=dev)
+        step = 1 << 16
+        for t0 in range(0, L, step):
+            K = synth.outlier_normal((min(step, L - t0), H, d), seed=3 + t0, device=dev)
+            V = synth.outlier_normal((min(step, L - t0), H, d), seed=30003 + t0, device=dev)
+            tqkv.encode(self.kp, self.vp, self.desc, K, V, slots[t0:t0 + step].contiguous(), self.cache)
+        torch.cuda.synchronize()
+        self.Qd = synth.normal((1, Hq, d), seed=31, device=dev)
+        self.Qp = synth.normal((C, Hq, d), seed=32, device=dev)
+        self.seq = torch.full((1,), L, dtype=torch.int32, device=dev)
+        self.out_d = torch.empty_like(self.Qd)
+        self.out_p = torch.empty_like(self.Qp)
+        self.ws_d = torch.zeros(tqkv.decode_workspace_bytes(self.desc, 1, Hq, L), dtype=torch.uint8, device=dev)
+        self.ws_p = torch.zeros(tqkv.prefill_workspace_bytes(self.desc, C, Hq, L), dtype=torch.uint8, device=dev)
+        per_tok = tqkv.cache_bytes(self.desc) // P
+        self.dec_pairs = Hq * L
+        self.pre_pairs = Hq * sum(L - C + j + 1 for j in range(C))
+        self.units = self.dec_pairs + self.pre_pairs
+        self.dec_bytes = H * L * per_tok
+        self.pre_flops = self.pre_pairs * 2 * (2 * d + d)       # QK^T over 256 features + PV over 128
+        self.launches = {"decode": 3, "prefill": 3}
+
+    def ops(self):
+        tq = self.tq
+        return [("decode", lambda: tq.decode_attn(self.kp, self.vp, self.desc, self.Qd, self.bt, self.seq, self.L,
+                                                  self.cache, out=self.out_d, workspace=self.ws_d)),
+                ("prefill", lambda: tq.prefill_attn(self.kp, self.vp, self.desc, self.Qp, self.bt.view(-1), self.L,
+                                                    self.cache, out=self.out_p, workspace=self.ws_p))]
+
+    def host_io(self):
+        h = {"Qd": self.Qd.cpu().pin_memory(), "Qp": self.Qp.cpu().pin_memory()}
+        od = torch.empty(self.out_d.shape, dtype=self.out_d.dtype).pin_memory()
+        op = torch.empty(self.out_p.shape, dtype=self.out_p.dtype).pin_memory()
+
+        def step():
+            self.Qd.copy_(h["Qd"], non_blocking=True)
+            self.Qp.copy_(h["Qp"], non_blocking=True)
+            for _, f in self.ops():
+                f()
+            od.copy_(self.out_d, non_blocking=True)
+            op.copy_(self.out_p, non_blocking=True)
+        return step, sum(t.numel() * t.element_size() for t in h.values()), (od.numel() + op.numel()) * 2
+
+    def roofline(self, op_ms, hbm_peak):
+        _, tfl, tfl_s, _ = _peaks()
+        tf = self.pre_flops / (op_ms["prefill"] * 1e-3) / 1e12
+        gbs = self.dec_bytes / (op_ms["decode"] * 1e-3) / 1e9
+        return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl_s, "unit": "TFLOP/s",
+                 "frac": round(tf / tfl_s, 4), "traffic": traffic_for("prefill"),
+                 "kernel": "tq_prefill_attn", "algorithmic_flops": self.pre_flops,
+                 "peak_note": "sustained fp16/bf16 dense (MEASURED_PEAKS.json bf16_tflops_sustained)"},
+                {"decode": {"keys_scored_per_s": self.dec_pairs / (op_ms["decode"] * 1e-3), "ms": op_ms["decode"],
+                            "gbs": gbs, "frac": gbs / hbm_peak, "algorithmic_bytes": self.dec_bytes},
+                 "prefill": {"pairs_per_s": self.pre_pairs / (op_ms["prefill"] * 1e-3), "ms": op_ms["prefill"],
+                             "tflops": tf, "frac": tf / tfl_s}})
+
+    def config(self):
+        return {"workload": self.name, "batch": 1, "seq_len": self.L, "n_kv_heads": self.H, "n_q_heads": self.Hq,
+                "head_dim": self.d, "chunk": self.C, "preset": "K2+QJL/V3", "parallelism": "replicas",
+                "l2": "cache (107 MB) read once per decode; prefill re-reads it per query tile"}
+
+
+class SearchWorkload:
+    """Top-10 inner-product search: 1,000,000 x 1024 unit vectors (4-bit +
+    QJL), 1,024 queries."""
+    name = "search 1,000,000 x d=1024 (4-bit Lloyd-Max + 1-bit QJL) x 1024 queries, top-10"
+
+    def __init__(self, dev, n_db=1_000_000, n_q=1024, **_):
+        from kv_cache_vector_07_b200 import synth, tqkv
+        self.tq = tqkv
+        d = 1024
+        self.n_db, self.n_q, self.k, self.d = n_db, n_q, 10, d
+        self.desc = tqkv.cache_desc(d, 4, True, 0, page_tokens=64, n_kv_heads=1)
+        self.p = tqkv.make_params(d, 4, 1004)
+        X = synth.unit_normal(n_db, d, seed=4, device=dev)
+        self.cache = tqkv.alloc_cache(self.desc, -(-n_db // 64), device=dev)
+        slots = torch.arange(n_db, dtype=torch.int32, device=dev)
+        ws = torch.zeros(tqkv.encode_workspace_bytes(self.desc, n_db), dtype=torch.uint8, device=dev)
+        s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tqkv.encode(self.p, None, self.desc, X, None, slots, self.cache, workspace=ws)
+        s0.record()
+        tqkv.encode(self.p, None, self.desc, X, None, slots, self.cache, workspace=ws)
+        e0.record()
+        torch.cuda.synchronize()
+        self.db_encode_ms = s0.elapsed_time(e0)
+        del X, ws
+        self.Q = synth.unit_normal(n_q, d, seed=5, device=dev)
+        self.ws = torch.zeros(tqkv.score_workspace_bytes(self.desc, n_db, n_q, 10), dtype=torch.uint8, device=dev)
+        self.sc = torch.empty((n_q, 10), device=dev)
+        self.ix = torch.empty((n_q, 10), dtype=torch.int64, device=dev)
+        self.units = n_db * n_q
+        self.flops = 2 * n_q * n_db * 2 * d
+        self.launches = {"score": 3}
+
+    def ops(self):
+        tq = self.tq
+        return [("score", lambda: tq.score(self.p, self.desc, self.cache, self.n_db, self.Q, self.k,
+                                           top_scores=self.sc, top_idx=self.ix, workspace=self.ws))]
+
+    def host_io(self):
+        h = self.Q.cpu().pin_memory()
+        o1 = torch.empty(self.sc.shape).pin_memory()
+        o2 = torch.empty(self.ix.shape, dtype=torch.int64).pin_memory()
+
+        def step():
+            self.Q.copy_(h, non_blocking=True)
+            self.ops()[0][1]()
+            o1.copy_(self.sc, non_blocking=True)
+            o2.copy_(self.ix, non_blocking=True)
+        return step, h.numel() * 4, o1.numel() * 4 + o2.numel() * 8
+
+    def roofline(self, op_ms, hbm_peak):
+        _, tfl, tfl_s, _ = _peaks()
+        tf = self.flops / (op_ms["score"] * 1e-3) / 1e12
+        return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl_s, "unit": "TFLOP/s",
+                 "frac": round(tf / tfl_s, 4), "traffic": traffic_for("score"), "kernel": "tq_score",
+                 "algorithmic_flops": self.flops},
+                {"score": {"scores_per_s": self.units / (op_ms["score"] * 1e-3), "ms": op_ms["score"], "tflops": tf},
+                 "db_encode": {"ms": self.db_encode_ms, "vectors_per_s": self.n_db / (self.db_encode_ms * 1e-3)}})
+
+    def config(self):
+        return {"workload": self.name, "n_db": self.n_db, "n_queries": self.n_q, "head_dim": self.d, "k": self.k,
+                "preset": "4-bit + QJL", "parallelism": "replicas"}
+
+
+WORKLOADS = {"step": StepWorkload, "decode32k": Decode32kWorkload, "longctx": LongCtxWorkload,
+             "search": SearchWorkload}
 
 
 def traffic_for(op: str):
@@ -311,7 +462,8 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     from kv_cache_vector_07_b200 import build as b
     b.build()
-    wl = WORKLOADS[args.workload](dev)
+    sizes = {k: v for k, v in (("batch", args.batch), ("seq_len", args.seq_len)) if v}
+    wl = WORKLOADS[args.workload](dev, **sizes)
     ops = wl.ops()
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -366,8 +518,8 @@ def run_ours(args):
     hbm, bf16, bf16s, src = _peaks()
     roof, parts = wl.roofline(op_ms, hbm)
     roof["peak_source"] = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"
-    line = {"metric": METRIC, "value": value, "unit": "units/s",
-            "unit_note": "units = KV vectors encoded + (query-head, key) pairs scored",
+    line = {"metric": METRIC if args.workload == "step" else EXTRA_METRICS[args.workload], "value": value,
+            "unit": "units/s", "unit_note": UNIT_NOTES[args.workload],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_max * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)", "config": wl.config(),
@@ -401,22 +553,60 @@ def _oracle_slice(seed_slice: int, L: int = 32768, d: int = 128, G: int = 4, kbi
     return 2 * L + G * L
 
 
+def _attend_slice(kind: str, n: int):
+    """Oracle attention or search on an oracle-encoded slice; returns
+    (seconds spent in the timed part, units)."""
+    from kv_cache_vector_07_b200 import synth
+    from oracle import oracle as O
+    d = 1024 if kind == "search" else 128
+    if kind == "search":
+        n_db, n_q = 20000, 4
+        X = synth.unit_normal(n_db, d, seed=40 + n).numpy().astype(np.float64)
+        Q = synth.unit_normal(n_q, d, seed=50 + n).numpy().astype(np.float64)
+        P = O.make_params(d, 4, 1004)
+        E = O.encode(X, P, qjl=True, margins=False)
+        t0 = time.perf_counter()
+        O.search(Q, P, E, 10)
+        return time.perf_counter() - t0, n_db * n_q
+    L, G, kb, vb = (32768, 4, 2, 4) if kind == "decode32k" else (65536, 8, 2, 3)
+    K = synth.outlier_normal((L, d), seed=60 + n, dtype=torch.float32).numpy().astype(np.float64)
+    V = synth.outlier_normal((L, d), seed=70 + n, dtype=torch.float32).numpy().astype(np.float64)
+    Q = synth.normal((G, d), seed=80 + n, dtype=torch.float32).numpy().astype(np.float64)
+    Pk, Pv = O.make_params(d, kb, 1002), O.make_params(d, vb, 2002, with_S=False)
+    Ek, Ev = O.encode(K, Pk, qjl=True, margins=False), O.encode(V, Pv, qjl=False, margins=False)
+    t0 = time.perf_counter()
+    O.attend(Q, Pk, Ek, Pv, Ev)
+    return time.perf_counter() - t0, G * L
+
+
 def cpu_baseline(workload: str, budget_s: float = 15.0):
     from oracle import oracle as O
     O.build()
-    O.codebook(128, 4)
     cores = len(os.sched_getaffinity(0))
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-    units, t0, n = 0, time.perf_counter(), 0
-    while time.perf_counter() - t0 < budget_s or n == 0:
-        units += _oracle_slice(n)
-        n += 1
-    dt = time.perf_counter() - t0
-    return {"value": units / dt, "unit": "units/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} (sequence, KV head) slices of the step workload: each encodes 32,768 keys "
-                      f"(4-bit + QJL) and 32,768 values (4-bit) and scores them for 4 query heads "
-                      f"(float64 oracle, OpenMP); workload: {workload}",
-            "seconds": dt}
+    units, spent, n = 0, 0.0, 0
+    wall0 = time.perf_counter()
+    if workload == "step":
+        O.codebook(128, 4)
+        while spent < budget_s or n == 0:
+            t0 = time.perf_counter()
+            units += _oracle_slice(n)
+            spent += time.perf_counter() - t0
+            n += 1
+        sample = (f"{n} (sequence, KV head) slices of the step workload: each encodes 32,768 keys (4-bit + QJL) "
+                  f"and 32,768 values (4-bit) and scores them for 4 query heads (float64 oracle, OpenMP)")
+    else:
+        while (spent < budget_s and time.perf_counter() - wall0 < 4 * budget_s) or n == 0:
+            dt, u = _attend_slice(workload, n)
+            spent += dt
+            units += u
+            n += 1
+        what = {"decode32k": "one KV head (4 query heads) over 32,768 oracle-encoded tokens",
+                "longctx": "one KV head (8 query heads) over 65,536 oracle-encoded tokens",
+                "search": "4 queries over 20,000 oracle-encoded d=1024 vectors"}[workload]
+        sample = f"{n} slices, each {what}; only the scoring is timed (float64 oracle, OpenMP)"
+    return {"value": units / spent, "unit": "units/s", "cores": cores, "kind": "oracle", "sample": sample,
+            "seconds": spent}
 
 
 def run_reference(args):
@@ -436,8 +626,8 @@ def run_reference(args):
     dt = time.perf_counter() - t0
     value = units / dt
     wl_name = StepWorkload.name
-    line = {"metric": METRIC, "value": value, "unit": "units/s",
-            "unit_note": "units = KV vectors encoded + (query-head, key) pairs scored",
+    line = {"metric": METRIC if args.workload == "step" else EXTRA_METRICS[args.workload], "value": value,
+            "unit": "units/s", "unit_note": UNIT_NOTES[args.workload],
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
@@ -459,6 +649,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the workload's sequence length")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
