@@ -399,7 +399,7 @@ class SearchWorkload:
         self.ix = torch.empty((n_q, 10), dtype=torch.int64, device=dev)
         self.units = n_db * n_q
         self.flops = 2 * n_q * n_db * 2 * d
-        self.launches = {"score": 3}
+        self.launches = {"score": 4}
 
     def ops(self):
         tq = self.tq
@@ -421,9 +421,11 @@ class SearchWorkload:
     def roofline(self, op_ms, hbm_peak):
         _, tfl, tfl_s, _ = _peaks()
         tf = self.flops / (op_ms["score"] * 1e-3) / 1e12
-        return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl_s, "unit": "TFLOP/s",
-                 "frac": round(tf / tfl_s, 4), "traffic": traffic_for("score"), "kernel": "tq_score",
-                 "algorithmic_flops": self.flops},
+        # a search of tens of milliseconds timed on its own: the burst figure
+        return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl, "unit": "TFLOP/s",
+                 "frac": round(tf / tfl, 4), "traffic": traffic_for("score"), "kernel": "tq_score",
+                 "algorithmic_flops": self.flops,
+                 "peak_note": "burst fp16/bf16 dense (MEASURED_PEAKS.json bf16_tflops; fp16 nominal = bf16 nominal)"},
                 {"score": {"scores_per_s": self.units / (op_ms["score"] * 1e-3), "ms": op_ms["score"], "tflops": tf},
                  "db_encode": {"ms": self.db_encode_ms, "vectors_per_s": self.n_db / (self.db_encode_ms * 1e-3)}})
 
@@ -517,7 +519,10 @@ def run_ours(args):
 
     hbm, bf16, bf16s, src = _peaks()
     roof, parts = wl.roofline(op_ms, hbm)
-    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"
+    if src != "measured":
+        roof["peak_source"] = "fallback"
+    else:
+        roof["peak_source"] = "measured" + ("" if "peak_note" in roof else " (MEASURED_PEAKS.json hbm_gbs)")
     line = {"metric": METRIC if args.workload == "step" else EXTRA_METRICS[args.workload], "value": value,
             "unit": "units/s", "unit_note": UNIT_NOTES[args.workload],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -136,6 +136,16 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   uint32_t *status, cudaStream_t st);
 
 size_t score_ws_bytes(const Layout &L, int64_t n_db, int n_q, int k);
+// Tensor-core search (4-bit + QJL database, d in {128, 256, 512, 1024},
+// k <= 16): blocks per query tile, or 0 when not covered; workspace pieces;
+// launcher of the query-feature and scoring kernels (writes 2 * n_groups
+// candidate lists per query into pv / pi).
+int search_tc_groups(const Layout &L, int64_t n_db, int n_q, int k);
+size_t search_tc_qf_bytes(const Layout &L, int n_q);
+size_t search_tc_qscale_bytes(int n_q);
+int launch_search_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db, int n_q, int k,
+                     const float *qr, const float *w, uint8_t *qf, float *qscale, float *pv, int64_t *pi,
+                     int n_groups, uint32_t *status, cudaStream_t st);
 int launch_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
                  const float *Q, int n_q, int k, float *top_scores, int64_t *top_idx,
                  uint8_t *ws, size_t ws_bytes, void *stream);

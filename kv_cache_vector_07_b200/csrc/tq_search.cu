@@ -206,29 +206,38 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *pv, const int64
 }
 
 struct SPlan {
-    int n_splits;
+    int n_splits;               // candidate lists per query
+    int tc_groups;              // > 0: tensor-core path with this many blocks per query tile
     int64_t split_len;
-    size_t off_qr, off_w, off_pv, off_pi, total;
+    size_t off_qr, off_w, off_pv, off_pi, off_qf, off_qs, total;
 };
 
 SPlan splan(const Layout &L, int64_t n_db, int n_q, int k) {
     SPlan s;
-    const int tiles = (n_q + kQT - 1) / kQT;
-    const int64_t target = 148 * 6;
-    int64_t splits = (target + tiles - 1) / tiles;
-    const int64_t maxs = (n_db + kTile - 1) / kTile;
-    if (splits > maxs) splits = maxs;
-    if (splits < 1) splits = 1;
-    s.split_len = ((n_db + splits - 1) / splits + kTile - 1) / kTile * kTile;
-    if (s.split_len < kTile) s.split_len = kTile;
-    s.n_splits = int((n_db + s.split_len - 1) / s.split_len);
-    if (s.n_splits < 1) s.n_splits = 1;
+    s.tc_groups = search_tc_groups(L, n_db, n_q, k);
+    if (s.tc_groups > 0) {
+        s.n_splits = 2 * s.tc_groups;
+        s.split_len = 0;
+    } else {
+        const int tiles = (n_q + kQT - 1) / kQT;
+        const int64_t target = 148 * 6;
+        int64_t splits = (target + tiles - 1) / tiles;
+        const int64_t maxs = (n_db + kTile - 1) / kTile;
+        if (splits > maxs) splits = maxs;
+        if (splits < 1) splits = 1;
+        s.split_len = ((n_db + splits - 1) / splits + kTile - 1) / kTile * kTile;
+        if (s.split_len < kTile) s.split_len = kTile;
+        s.n_splits = int((n_db + s.split_len - 1) / s.split_len);
+        if (s.n_splits < 1) s.n_splits = 1;
+    }
     size_t off = kWsHeader;
     auto take = [&](size_t b) { size_t o = off; off += (b + 255) / 256 * 256; return o; };
     s.off_qr = take(sizeof(float) * size_t(n_q) * L.d);
     s.off_w = take(sizeof(float) * size_t(n_q) * L.d);
     s.off_pv = take(sizeof(float) * size_t(n_q) * s.n_splits * k);
     s.off_pi = take(sizeof(int64_t) * size_t(n_q) * s.n_splits * k);
+    s.off_qf = s.tc_groups > 0 ? take(search_tc_qf_bytes(L, n_q)) : 0;
+    s.off_qs = s.tc_groups > 0 ? take(search_tc_qscale_bytes(n_q)) : 0;
     s.total = off;
     return s;
 }
@@ -245,6 +254,16 @@ int run_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_
         if (e != cudaSuccess) return e;
     }
     prep_f32_kernel<D><<<unsigned((n_q + 3) / 4), 128, psm, st>>>(Q, n_q, p->dev, qr, w);
+    float *pv = reinterpret_cast<float *>(ws + s.off_pv);
+    int64_t *pi = reinterpret_cast<int64_t *>(ws + s.off_pi);
+    if (s.tc_groups > 0) {
+        const int e = launch_search_tc(p, L, db, n_db, n_q, k, qr, w, ws + s.off_qf,
+                                       reinterpret_cast<float *>(ws + s.off_qs), pv, pi, s.tc_groups,
+                                       reinterpret_cast<uint32_t *>(ws), st);
+        if (e != cudaSuccess) return e;
+        merge_kernel<<<unsigned((n_q + 3) / 4), 128, 0, st>>>(pv, pi, n_q, s.n_splits, k, top_v, top_i);
+        return cudaGetLastError();
+    }
     ScoreArgs a;
     a.L = L;
     a.p = p->dev;
@@ -256,8 +275,8 @@ int run_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_
     a.split_len = s.split_len;
     a.qr = qr;
     a.w = w;
-    a.part_v = reinterpret_cast<float *>(ws + s.off_pv);
-    a.part_i = reinterpret_cast<int64_t *>(ws + s.off_pi);
+    a.part_v = pv;
+    a.part_i = pi;
     const size_t ssm = sizeof(float) * 2 * D * kQT;
     if (ssm > 16 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ssm));

@@ -1,0 +1,450 @@
+// Compressed inner-product search on the tensor cores (4-bit Lloyd-Max +
+// QJL database; head dimension 128, 256, 512 or 1024; k <= 16).
+//
+// ai-work-lab overview, "QJL" and the vector-search paragraphs: the codec
+// used for keys also scores database vectors, with no index preprocessing.
+// Estimate of <q, x_t>:
+//   nhat_t <Rq, c[code_t]> + rho_t sqrt(pi/2)/m <S R q, 2 s_t - 1>.
+//
+// As a GEMM: D[128 queries x 512 vectors] = Qf[128 x 2d] Xf[512 x 2d]^T on
+// tcgen05 (fp16 operands, fp32 accumulator in TMEM, all 512 columns):
+//   Qf = 2^-e [R q | S R q] per query (fp16, prepared once, TMA-loaded one
+//        64-feature chunk at a time; e makes the largest feature 1 <= |f| < 2
+//        and the scores are multiplied back by 2^e);
+//   Xf = [nhat c[code] | rho sqrt(pi/2)/m (2 s - 1)] per database vector,
+//        dequantized by the block's threads into shared memory (128-byte
+//        swizzled K-major tiles) while the previous chunk's MMAs run.
+// Epilogue: thread (query, half) reads its 256 estimates from TMEM and keeps
+// a running top-k (ties to the lower index); a merge kernel combines the
+// blocks' lists.
+//
+// Inside every 32-coordinate group the QJL features are in the order
+// (p, p + 16) for feature positions (2p, 2p + 1), so a pair of sign bits
+// becomes an fp16 pair with one shift and one mask.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "tc05.cuh"
+#include "tq_dev.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int kQ = 128;                 // queries per block (MMA M, TMEM lanes)
+constexpr int kN = 512;                 // database vectors per tile (two MMAs of N = 256)
+constexpr int kThreads = 256;
+constexpr int kTopK = 16;               // largest k this path takes
+constexpr int kSMs = 148;               // grid sizing (fixed, so workspace sizes do not depend on the device)
+constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
+
+// shared layout (offsets from a 1024-aligned base)
+constexpr uint32_t SA = 0;                       // 2 stages x [128 x 64] fp16 (16 KB each)
+constexpr uint32_t SB = 32768;                   // 2 stages x 2 halves x [256 x 64] fp16 (64 KB per stage)
+constexpr uint32_t SLUT = SB + 131072;           // [256 code bytes][32 lane copies] half2 (32 KB)
+constexpr uint32_t STOPV = SLUT + 32768;         // [256 threads][k] scores
+constexpr uint32_t STOPI = STOPV + kThreads * kTopK * 4;   // [256 threads][k] indices (n_db < 2^31)
+constexpr uint32_t SBAR = STOPI + kThreads * kTopK * 4;
+constexpr uint32_t SM_TOTAL = SBAR + 64 + 1024;  // + slack for aligning the base
+static_assert(SM_TOTAL <= 232448, "shared memory");
+
+struct SearchTcArgs {
+    Layout L;
+    const float *lv;               // levels by stored code (16)
+    const uint8_t *db;
+    int64_t n_db;
+    int n_q, k;
+    int64_t n_tiles;               // ceil(n_db / 512)
+    int n_groups;                  // blocks per query tile
+    const float *qscale;           // [n_q_pad] 2^e
+    float *part_v;                 // [n_q][2 n_groups][k]
+    int64_t *part_i;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ uint32_t h2pack(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// The two database rows a thread dequantizes: tile rows tid and tid + 256.
+struct Rows {
+    const uint8_t *page[2];
+    int pos[2];
+    uint32_t nh2[2], rh2[2];        // nhat and -rho sqrt(pi/2)/m as fp16 pairs
+};
+
+template <int D>
+__device__ __forceinline__ void rows_for(const SearchTcArgs &a, int64_t tile, int tid, Rows &r) {
+    const Layout &L = a.L;
+    const float cq = 1.2533141373155003f / float(D);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int64_t v = tile * kN + tid + 256 * j;
+        if (tile < a.n_tiles && v < a.n_db) {
+            r.page[j] = a.db + (v / L.P) * int64_t(L.page_bytes);
+            r.pos[j] = int(v % L.P);
+            const float nh = h2f_bits(*reinterpret_cast<const uint16_t *>(r.page[j] + L.kn_off + r.pos[j] * 2));
+            const float rh = h2f_bits(*reinterpret_cast<const uint16_t *>(r.page[j] + L.kr_off + r.pos[j] * 2)) * cq;
+            r.nh2[j] = h2pack(nh, nh);
+            r.rh2[j] = h2pack(-rh, -rh);
+        } else {
+            r.page[j] = nullptr;
+            r.pos[j] = 0;
+            r.nh2[j] = r.rh2[j] = 0;
+        }
+    }
+}
+
+// Raw code bytes of chunk kc for both rows: 32 code bytes (MSE chunk) or 8
+// sign bytes (QJL chunk, in raw[j][0].x/.y).
+template <int D>
+__device__ __forceinline__ void load_raw(const Layout &L, const Rows &r, int kc, uint4 (&raw)[2][2]) {
+    constexpr int MSE_KC = D / 64;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        raw[j][0] = raw[j][1] = make_uint4(0, 0, 0, 0);
+        if (!r.page[j]) continue;
+        if (kc < MSE_KC) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(r.page[j] + L.kc_off + r.pos[j] * (D / 2) + kc * 32);
+            raw[j][0] = __ldg(src);
+            raw[j][1] = __ldg(src + 1);
+        } else {
+            const uint2 s = __ldg(reinterpret_cast<const uint2 *>(r.page[j] + L.ks_off + r.pos[j] * (D / 8) +
+                                                                  (kc - MSE_KC) * 8));
+            raw[j][0].x = s.x;
+            raw[j][0].y = s.y;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
+    constexpr int NKC = 2 * D / 64;             // feature chunks per tile
+    constexpr int MSE_KC = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(sm + SLUT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
+    uint64_t *bar_a = bars, *bar_m = bars + 2;   // A loaded / MMAs done, per stage
+    __shared__ uint32_t tmem_holder;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qt = blockIdx.x, grp = blockIdx.y;
+    const int K = a.k;
+    const Layout &L = a.L;
+    float *tv = reinterpret_cast<float *>(sm + STOPV) + tid * kTopK;
+    int32_t *ti = reinterpret_cast<int32_t *>(sm + STOPI) + tid * kTopK;
+
+    for (int i = tid; i < 256 * 32; i += kThreads) {
+        const int e = i >> 5;
+        lut[i] = h2pack(a.lv[e & 15], a.lv[e >> 4]);
+    }
+    for (int r = 0; r < K; ++r) {
+        tv[r] = -INFINITY;
+        ti[r] = -1;
+    }
+    if (warp == 0) {
+        tc05::tmem_alloc(&tmem_holder, 512);
+        tc05::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) tc05::mbar_init(&bars[i], 1);
+        tc05::fence_mbar_init();
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    tc05::fence_after_sync();
+    const uint32_t tmem = tmem_holder;
+    constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
+
+    const int q = qt * kQ + (tid & 127);
+    const int half = tid >> 7;
+    const float qsc = a.qscale[q];
+    const uint32_t *lut_lane = lut + lane;
+
+    // per-stage mbarrier phases and "MMAs outstanding" flags, bit st of each
+    uint32_t phase_a = 0, phase_m = 0, used_m = 0;
+    bool timeout = false;
+    int a_pending = -1;              // thread 0: stage whose A load is not yet waited for
+
+    int64_t tile = grp;
+    int kc = 0;
+    Rows cur;
+    rows_for<D>(a, tile, tid, cur);
+    uint4 raw[2][2];
+    load_raw<D>(L, cur, 0, raw);
+
+    while (tile < a.n_tiles) {
+        // prefetch the next step's bytes (next chunk, or the next tile's first)
+        int64_t ntile = tile;
+        int nkc = kc + 1;
+        Rows nxt = cur;
+        if (nkc == NKC) {
+            nkc = 0;
+            ntile += a.n_groups;
+            rows_for<D>(a, ntile, tid, nxt);
+        }
+        uint4 nraw[2][2];
+        load_raw<D>(L, nxt, nkc, nraw);
+
+        const int st = kc & 1;
+        uint8_t *sA = sm + SA + st * 16384;
+        uint8_t *sB = sm + SB + st * 65536;
+        // the stage is free once the MMAs that read it have completed
+        if ((used_m >> st) & 1u) {
+            if (!tc05::mbar_wait_bounded(&bar_m[st], (phase_m >> st) & 1u, kPolls)) timeout = true;
+            phase_m ^= 1u << st;
+            used_m &= ~(1u << st);
+        }
+        if (tid == 0) {
+            tc05::mbar_expect_tx(&bar_a[st], 16384);
+            tc05::tma_load_2d(sA, &tmQ, kc * 64, qt * kQ, &bar_a[st]);
+            a_pending = st;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint8_t *brow = sB + j * 32768;
+            uint32_t w[32];
+            if (kc < MSE_KC) {
+                const uint32_t cw[8] = {raw[j][0].x, raw[j][0].y, raw[j][0].z, raw[j][0].w,
+                                        raw[j][1].x, raw[j][1].y, raw[j][1].z, raw[j][1].w};
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
+                    w[i] = hmul2u(lut_lane[byte * 32], cur.nh2[j]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t word = (i < 16) ? raw[j][0].x : raw[j][0].y;
+                    const int p = i & 15;
+                    w[i] = cur.rh2[j] ^ ((word << (15 - p)) & 0x80008000u);
+                }
+            }
+#pragma unroll
+            for (int pc = 0; pc < 8; ++pc)
+                *reinterpret_cast<uint4 *>(brow + tc05::sw128_offset(uint32_t(tid), uint32_t(pc))) =
+                    make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
+        }
+        tc05::fence_proxy_async_smem();
+        tc05::fence_before_sync();
+        if (__syncthreads_or(timeout)) break;
+        if (tid == 0) {
+            if (!tc05::mbar_wait_bounded(&bar_a[st], (phase_a >> st) & 1u, kPolls)) timeout = true;
+            a_pending = -1;
+            tc05::fence_after_sync();
+            const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sB);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = tc05::desc_kmajor_sw128(aa + ks * 32);
+                const bool acc = (kc | ks) != 0;
+                tc05::mma_f16(tmem, ad, tc05::desc_kmajor_sw128(bb + ks * 32), idesc, acc);
+                tc05::mma_f16(tmem + 256, ad, tc05::desc_kmajor_sw128(bb + 32768 + ks * 32), idesc, acc);
+            }
+            tc05::mma_commit(&bar_m[st]);
+        }
+        phase_a ^= 1u << st;
+        used_m |= 1u << st;
+
+        if (kc == NKC - 1) {
+            // the last commit covers every earlier MMA; consume both stages' phases
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int o = st ^ s2;
+                if ((used_m >> o) & 1u) {
+                    if (!tc05::mbar_wait_bounded(&bar_m[o], (phase_m >> o) & 1u, kPolls)) timeout = true;
+                    phase_m ^= 1u << o;
+                    used_m &= ~(1u << o);
+                }
+            }
+            tc05::fence_after_sync();
+            const int64_t v0 = tile * kN + half * 256;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                uint32_t r[32];
+                tc05::tmem_ld_32x32b_x32(tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(half * 256 + c * 32),
+                                         r);
+                tc05::tmem_wait_ld();
+                if (q < a.n_q) {
+                    float kth = tv[K - 1];
+                    bool full = ti[K - 1] >= 0;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float s = __uint_as_float(r[e]) * qsc;
+                        const int32_t id = int32_t(v0 + c * 32 + e);
+                        if (id < a.n_db && (!full || s > kth)) {
+                            int p = K - 1;
+                            while (p > 0 && (ti[p - 1] < 0 || s > tv[p - 1])) {
+                                tv[p] = tv[p - 1];
+                                ti[p] = ti[p - 1];
+                                --p;
+                            }
+                            tv[p] = s;
+                            ti[p] = id;
+                            kth = tv[K - 1];
+                            full = ti[K - 1] >= 0;
+                        }
+                    }
+                }
+            }
+            tc05::fence_before_sync();
+            if (__syncthreads_or(timeout)) break;
+            tc05::fence_after_sync();
+        }
+        tile = ntile;
+        kc = nkc;
+        cur = nxt;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            raw[j][0] = nraw[j][0];
+            raw[j][1] = nraw[j][1];
+        }
+    }
+    // after an early exit, let the copy and the MMAs still in flight finish
+    // before shared memory and TMEM are given back
+    if (a_pending >= 0 && !tc05::mbar_wait_bounded(&bar_a[a_pending], (phase_a >> a_pending) & 1u, kPolls))
+        timeout = true;
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+        if (((used_m >> s) & 1u) && !tc05::mbar_wait_bounded(&bar_m[s], (phase_m >> s) & 1u, kPolls)) timeout = true;
+    if (q < a.n_q) {
+        for (int r = 0; r < K; ++r) {
+            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + half) * K + r;
+            a.part_v[o] = tv[r];
+            a.part_i[o] = ti[r];
+        }
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc05::fence_after_sync();
+        tc05::tmem_dealloc(tmem, 512);
+    }
+    if (timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
+}
+
+// Query features [n_q_pad][2d] fp16 = 2^-e [R q | S R q] (QJL half in the
+// pair order described above) and qscale = 2^e.  One warp per query.
+template <int D>
+__global__ void __launch_bounds__(128) qfeat_kernel(const float *qr, const float *w, int n_q, int n_q_pad,
+                                                    __half *out, float *qscale) {
+    const int lane = threadIdx.x & 31;
+    const int q = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (q >= n_q_pad) return;
+    float m = 0.f;
+    if (q < n_q)
+        for (int i = lane; i < D; i += 32)
+            m = fmaxf(m, fmaxf(fabsf(qr[int64_t(q) * D + i]), fabsf(w[int64_t(q) * D + i])));
+    m = warp_max(m);
+    int ex = 0;
+    if (m > 0.f) frexpf(m, &ex);                 // m < 2^ex
+    const float down = m > 0.f ? ldexpf(1.f, 1 - ex) : 1.f;
+    if (lane == 0) qscale[q] = m > 0.f ? ldexpf(1.f, ex - 1) : 1.f;
+    for (int i = lane; i < 2 * D; i += 32) {
+        float v = 0.f;
+        if (q < n_q) {
+            if (i < D) {
+                v = qr[int64_t(q) * D + i];
+            } else {
+                const int k = i - D, pp = k & 31;
+                const int coord = (k & ~31) + ((pp & 1) ? (pp >> 1) + 16 : (pp >> 1));
+                v = w[int64_t(q) * D + coord];
+            }
+        }
+        out[int64_t(q) * 2 * D + i] = __float2half_rn(v * down);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult qr;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+template <int D>
+int run_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db, int n_q, int k, const float *qr,
+           const float *w, uint8_t *qf_bytes, float *qscale, float *pv, int64_t *pi, int n_groups, uint32_t *status,
+           cudaStream_t st) {
+    const int n_qt = (n_q + kQ - 1) / kQ;
+    const int n_q_pad = n_qt * kQ;
+    __half *qf = reinterpret_cast<__half *>(qf_bytes);
+    qfeat_kernel<D><<<unsigned(n_q_pad / 4), 128, 0, st>>>(qr, w, n_q, n_q_pad, qf, qscale);
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    CUtensorMap tm;
+    cuuint64_t dims[2] = {cuuint64_t(2 * D), cuuint64_t(n_q_pad)};
+    cuuint64_t strides[1] = {cuuint64_t(2 * D * 2)};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, qf, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    SearchTcArgs a;
+    a.L = L;
+    a.lv = p->dev.lv;
+    a.db = db;
+    a.n_db = n_db;
+    a.n_q = n_q;
+    a.k = k;
+    a.n_tiles = (n_db + kN - 1) / kN;
+    a.n_groups = n_groups;
+    a.qscale = qscale;
+    a.part_v = pv;
+    a.part_i = pi;
+    a.status = status;
+    auto kern = score_tc_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SM_TOTAL));
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(unsigned(n_qt), unsigned(n_groups)), kThreads, SM_TOTAL, st>>>(tm, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Database groups (blocks per query tile) of the tensor-core search, 0 when
+// the configuration is not covered.  Each group yields two candidate lists
+// per query.
+int search_tc_groups(const Layout &L, int64_t n_db, int n_q, int k) {
+    if (!(L.kbits == 4 && L.kqjl && L.vbits == 0) || k > kTopK || n_db > INT32_MAX) return 0;
+    if (!(L.d == 128 || L.d == 256 || L.d == 512 || L.d == 1024)) return 0;
+    const int n_qt = (n_q + kQ - 1) / kQ;
+    const int64_t n_tiles = (n_db + kN - 1) / kN;
+    int64_t g = kSMs / n_qt;
+    if (g < 1) g = 1;
+    if (g > n_tiles) g = n_tiles;
+    return int(g);
+}
+
+size_t search_tc_qf_bytes(const Layout &L, int n_q) {
+    const size_t n_q_pad = size_t((n_q + kQ - 1) / kQ) * kQ;
+    return n_q_pad * 2 * size_t(L.d) * sizeof(__half);
+}
+
+size_t search_tc_qscale_bytes(int n_q) { return size_t((n_q + kQ - 1) / kQ) * kQ * sizeof(float); }
+
+int launch_search_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db, int n_q, int k,
+                     const float *qr, const float *w, uint8_t *qf, float *qscale, float *pv, int64_t *pi,
+                     int n_groups, uint32_t *status, cudaStream_t st) {
+    switch (L.d) {
+        case 128: return run_tc<128>(p, L, db, n_db, n_q, k, qr, w, qf, qscale, pv, pi, n_groups, status, st);
+        case 256: return run_tc<256>(p, L, db, n_db, n_q, k, qr, w, qf, qscale, pv, pi, n_groups, status, st);
+        case 512: return run_tc<512>(p, L, db, n_db, n_q, k, qr, w, qf, qscale, pv, pi, n_groups, status, st);
+        case 1024: return run_tc<1024>(p, L, db, n_db, n_q, k, qr, w, qf, qscale, pv, pi, n_groups, status, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tq

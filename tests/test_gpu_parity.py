@@ -271,6 +271,36 @@ def test_search_million_vectors_properties():
     assert recall > 0.3
 
 
+@pytest.mark.parametrize("d,kbits,kqjl,n_db,n_q,k,qscale", [
+    (128, 4, True, 3001, 130, 16, 1.0),      # tensor cores: two query tiles, ragged tails, largest k
+    (256, 4, True, 1500, 5, 1, 1e5),         # tensor cores: k = 1, queries far beyond the fp16 range
+    (512, 4, True, 777, 1, 3, 1e-6),         # tensor cores: one short tile, tiny query
+    (64, 3, True, 2000, 9, 7, 1.0),          # general kernel (head dim below the tensor-core tile)
+    (128, 2, False, 999, 3, 20, 1.0),        # general kernel (MSE-only codes, k above 16)
+])
+def test_search_configurations_every_output(d, kbits, kqjl, n_db, n_q, k, qscale):
+    X = synth.unit_normal(n_db, d, seed=d + n_db, device=DEV)
+    Qs = synth.unit_normal(n_q, d, seed=d + n_db + 1, device=DEV) * qscale
+    cd = Codec(d, kbits, kqjl, 0, seed=d + k, H=1)
+    nblk = -(-n_db // 64)
+    slots = torch.arange(n_db, dtype=torch.int32, device=DEV)
+    cache, flags = cd.encode(X, None, slots, nblk)
+    assert flags == 0
+    sc, ix = tqkv.score(cd.kp, cd.desc, cache, n_db, Qs, k)
+    torch.cuda.synchronize()
+    Ek, _, exk, _, _ = cd.check_tokens(cache_np(cache), np.arange(n_db), f64(X), None, 0)
+    ref_sc, ref_ix = O.search(f64(Qs), cd.Pk, Ek, min(k + 1, n_db))
+    gs, gi = f64(sc), ix.cpu().numpy()
+    for a in range(n_q):
+        assert len(set(gi[a].tolist())) == k and gi[a].min() >= 0 and gi[a].max() < n_db
+        est = O.estimate(f64(Qs[a]), cd.Pk, Ek)
+        tol = 1e-3 * np.maximum(np.abs(est[gi[a]]), np.sqrt(np.mean(est ** 2)))
+        assert ((np.abs(gs[a] - est[gi[a]]) <= tol) | exk[gi[a]]).all()
+        if k < n_db and ref_sc[a, k - 1] - ref_sc[a, k] > 2e-3 * abs(ref_sc[a, k - 1]):
+            assert set(gi[a]) == set(ref_ix[a, :k]) or exk[ref_ix[a, :k]].any()
+        assert np.all(np.diff(gs[a]) <= 0)
+
+
 # ---------------------------------------------------------------------------
 # edge cases: small and large head dims, ragged and empty sequences, skipped
 # slots, zero vectors, out-of-range slots, G = 1 and 8
