@@ -182,7 +182,7 @@ class StepWorkload:
         per_tok = page // P
         self.enc_bytes = 2 * n * H * d * 2 + n * H * per_tok
         self.dec_bytes = B * H * L * per_tok + 2 * self.Q.numel() * 2
-        self.launches = {"encode": 1, "decode": 3}
+        self.launches = {"encode": 1, "decode": 4}
 
     def ops(self):
         tq = self.tq
@@ -259,7 +259,7 @@ class Decode32kWorkload:
         self.ws_d = torch.zeros(tqkv.decode_workspace_bytes(self.desc, B, Hq, L), dtype=torch.uint8, device=dev)
         self.units = B * Hq * L
         self.dec_bytes = B * H * L * (tqkv.cache_bytes(self.desc) // P) + 2 * self.Q.numel() * 2
-        self.launches = {"decode": 3}
+        self.launches = {"decode": 4}
 
     def ops(self):
         tq = self.tq
@@ -327,7 +327,7 @@ class LongCtxWorkload:
         self.units = self.dec_pairs + self.pre_pairs
         self.dec_bytes = H * L * per_tok
         self.pre_flops = self.pre_pairs * 2 * (2 * d + d)       # QK^T over 256 features + PV over 128
-        self.launches = {"decode": 3, "prefill": 3}
+        self.launches = {"decode": 4, "prefill": 4}
 
     def ops(self):
         tq = self.tq
@@ -399,7 +399,7 @@ class SearchWorkload:
         self.ix = torch.empty((n_q, 10), dtype=torch.int64, device=dev)
         self.units = n_db * n_q
         self.flops = 2 * n_q * n_db * 2 * d
-        self.launches = {"score": 4}
+        self.launches = {"score": 5}
 
     def ops(self):
         tq = self.tq
@@ -464,7 +464,8 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     from kv_cache_vector_07_b200 import build as b
     b.build()
-    sizes = {k: v for k, v in (("batch", args.batch), ("seq_len", args.seq_len)) if v}
+    sizes = {k: v for k, v in (("batch", args.batch), ("seq_len", args.seq_len), ("n_db", args.n_db),
+                               ("n_q", args.n_q)) if v}
     wl = WORKLOADS[args.workload](dev, **sizes)
     ops = wl.ops()
     stream = torch.cuda.current_stream()
@@ -656,6 +657,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's sequence length")
+    ap.add_argument("--n-db", type=int, default=0, help="override the search database size")
+    ap.add_argument("--n-q", type=int, default=0, help="override the number of search queries")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -30,11 +30,11 @@ struct PrepArgs {
     float *w;               // [rows][D]
 };
 
-// One warp per query row; 4 rows per block.
+// q_r = R q, one warp per query row, 4 rows per block (w = S q_r follows
+// in the projection kernel).
 template <int D>
 __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
     constexpr int E = WarpVec<D>::E;
-    __shared__ float sq[4][D];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int64_t row = int64_t(blockIdx.x) * 4 + wl;
     if (row >= a.rows) return;
@@ -48,18 +48,7 @@ __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
     const float rs = 1.0f / sqrtf(float(D));
     if (lane < WarpVec<D>::LANES) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const float v = x[e] * rs;
-            sq[wl][lane * E + e] = v;
-            a.qr[row * D + lane * E + e] = v;
-        }
-    }
-    __syncwarp();
-    for (int j = lane; j < D; j += 32) {
-        const uint16_t *srow = a.kp.S + size_t(j) * D;
-        float acc = 0.f;
-        for (int i = 0; i < D; ++i) acc = fmaf(__uint_as_float(uint32_t(srow[i]) << 16), sq[wl][i], acc);
-        a.w[row * D + j] = acc;
+        for (int e = 0; e < E; ++e) a.qr[row * D + lane * E + e] = x[e] * rs;
     }
 }
 
@@ -353,6 +342,10 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
     pa.qr = reinterpret_cast<float *>(ws + p.off_qr);
     pa.w = reinterpret_cast<float *>(ws + p.off_w);
     prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
+    if (L.kqjl) {
+        const int e = launch_qproj(pa.qr, rows, D, kp->dev.S, pa.w, st);
+        if (e != cudaSuccess) return e;
+    }
 
     const int fast = launch_dec128(kp, vp, L, pa.qr, pa.w, s, p.G, p.n_groups, p.n_splits, p.split_len, cache,
                                    num_blocks, reinterpret_cast<float *>(ws + p.off_po),

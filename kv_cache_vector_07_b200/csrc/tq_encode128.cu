@@ -22,6 +22,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
+#include <cfloat>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -52,23 +53,23 @@ struct Enc128Args {
     uint32_t *status;
 };
 
-// Magnitude rank mu = #{k < 2^(B-1) - 1 : aa >= T[k]} of sorted thresholds,
-// by binary search.
+// Magnitude rank mu = #{k < 2^(B-1) - 1 : a >= T[k]} of the sorted positive
+// thresholds, by binary search on the float magnitude a = |Y|.
 template <int B>
-__device__ __forceinline__ int mag_rank(int aa, const int (&T)[7]) {
+__device__ __forceinline__ int mag_rank(float a, const float (&T)[7]) {
     if constexpr (B == 1) {
         return 0;
     } else if constexpr (B == 2) {
-        return aa >= T[0] ? 1 : 0;
+        return a >= T[0] ? 1 : 0;
     } else if constexpr (B == 3) {
-        const int b1 = aa >= T[1] ? 1 : 0;
-        const int b0 = aa >= (b1 ? T[2] : T[0]) ? 1 : 0;
+        const int b1 = a >= T[1] ? 1 : 0;
+        const int b0 = a >= (b1 ? T[2] : T[0]) ? 1 : 0;
         return (b1 << 1) | b0;
     } else {
-        const int b2 = aa >= T[3] ? 1 : 0;
-        const int b1 = aa >= (b2 ? T[5] : T[1]) ? 1 : 0;
-        const int t0 = b2 ? (b1 ? T[6] : T[4]) : (b1 ? T[2] : T[0]);
-        const int b0 = aa >= t0 ? 1 : 0;
+        const int b2 = a >= T[3] ? 1 : 0;
+        const int b1 = a >= (b2 ? T[5] : T[1]) ? 1 : 0;
+        const float t0 = b2 ? (b1 ? T[6] : T[4]) : (b1 ? T[2] : T[0]);
+        const int b0 = a >= t0 ? 1 : 0;
         return (b2 << 2) | (b1 << 1) | b0;
     }
 }
@@ -76,21 +77,20 @@ __device__ __forceinline__ int mag_rank(int aa, const int (&T)[7]) {
 // Bucketize this thread's 32 coordinates (Y = sqrt(128) y from the rotation
 // MMA) into sign-magnitude codes packed into words (B in {1,2,4}: one array
 // of B words; B = 3: words 0..1 hold the 2-bit magnitudes, word 2 the sign
-// bits).  T: positive boundaries scaled by sqrt(128) n, as float bits.  A
-// negative coordinate equal to a boundary belongs to the lower bucket (the
-// "- s"); -0.0 counts as non-negative.  With RESID, y is overwritten by the
-// residual y - nhat c[code] and rr receives its squared norm.
+// bits).  T: positive boundaries scaled by ||Y||.  -0.0 counts as
+// non-negative; a coordinate exactly on a boundary takes the upper magnitude
+// whatever its sign.  With RESID, y is overwritten by the residual in the Y
+// scale, Y - sqrt(128) nhat c[code], and rr receives its squared norm.
 template <int B, bool RESID>
-__device__ __forceinline__ void quantize32(float (&y)[32], const int (&T)[7], const float *lvs, float nhf, float rs,
+__device__ __forceinline__ void quantize32(float (&y)[32], const float (&T)[7], const float *lvs, float nhs,
                                            uint32_t (&cw)[4], float &rr) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) cw[k] = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const float Y = y[i];
-        const int s = Y < 0.f ? 1 : 0;
-        const int aa = (__float_as_int(Y) & 0x7fffffff) - s;
-        const uint32_t kap = uint32_t((s << (B - 1)) | mag_rank<B>(aa, T));
+        const uint32_t s = Y < 0.f ? 1u : 0u;
+        const uint32_t kap = (s << (B - 1)) | uint32_t(mag_rank<B>(fabsf(Y), T));
         if constexpr (B == 3) {
             cw[i >> 4] |= (kap & 3u) << (2 * (i & 15));
             cw[2] |= (kap >> 2) << i;
@@ -98,7 +98,7 @@ __device__ __forceinline__ void quantize32(float (&y)[32], const int (&T)[7], co
             cw[(i * B) >> 5] |= kap << ((i * B) & 31);
         }
         if constexpr (RESID) {
-            const float r = fmaf(-nhf, lvs[kap], Y * rs);
+            const float r = fmaf(-nhs, lvs[kap], Y);
             y[i] = r;
             rr = fmaf(r, r, rr);
         }
@@ -233,7 +233,11 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (tid == 0 && j + 1 < n_items) issue_mma1(j + 1);
         if (!tc05::mbar_wait_bounded(&bar_y[yb], uint32_t((j >> 1) & 1), kPolls)) timeout = true;
         tc05::fence_after_sync();
+        // MMA 1 of this item has read its x stage: refill it
+        if (tid == 0 && j + 2 < n_items) issue_x(j + 2);
 
+        // this thread's quarter of Y, and ||Y||^2 summed over the four
+        // quarters in a fixed order, so the four threads of a row agree
         float y[32];
         {
             uint32_t r[32];
@@ -242,19 +246,24 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
         }
-        float ss = 0.f;
+        float part[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ss = fmaf(y[i], y[i], ss);
-        // norm partials go to this item's x stage, free since MMA 1 read it
-        float *xs = reinterpret_cast<float *>(sm + SM_X + yb * kTile);
-        xs[q * 128 + row] = ss;
-        __syncthreads();
-        const float n = sqrtf(((xs[row] + xs[128 + row]) + xs[256 + row]) + xs[384 + row]) * rs;   // = ||x||
-        __syncthreads();
-        if (tid == 0 && j + 2 < n_items) {
-            tc05::fence_proxy_async_smem();
-            issue_x(j + 2);
+        for (int c = 0; c < 4; ++c) {
+            float ps = 0.f;
+            if (c == q) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ps = fmaf(y[i], y[i], ps);
+            } else {
+                uint32_t r[32];
+                tc05::tmem_ld_32x32b_x32(tmem + lane_base + uint32_t(yb * 128 + c * 32), r);
+                tc05::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ps = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ps);
+            }
+            part[c] = ps;
         }
+        const float ns = sqrtf(((part[0] + part[1]) + part[2]) + part[3]);   // ||Y|| = sqrt(128) ||x||
+        const float n = ns * rs;                                               // ||x||
         const uint16_t nh = f2h_bits(n);
         const float nhf = h2f_bits(nh);
         int pos = 0;
@@ -282,22 +291,20 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             }
         } else {
             const int nt = (1 << (bits - 1)) - 1;
-            const float scale = sq * n;
             const float *bnd = is_v ? a.v_bnd : a.k_bnd;
-            int T[7];
+            float T[7];
 #pragma unroll
-            for (int k = 0; k < 7; ++k)
-                T[k] = (k < nt && n > 0.f) ? __float_as_int(bnd[(1 << (bits - 1)) + k] * scale) : 0x7f7fffff;
+            for (int k = 0; k < 7; ++k) T[k] = (k < nt && ns > 0.f) ? bnd[(1 << (bits - 1)) + k] * ns : FLT_MAX;
             uint32_t cw[4];
             if (is_v) {
                 if constexpr (DO_V) {
-                    quantize32<DO_V ? VB : 1, false>(y, T, s_vlv, nhf, rs, cw, rr);
+                    quantize32<DO_V ? VB : 1, false>(y, T, s_vlv, 0.f, cw, rr);
                     if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
                                                             a.L.vh_bpt, cw);
                 }
             } else {
                 constexpr int KQ = KB == 8 ? 1 : KB;
-                quantize32<KQ, QJL>(y, T, s_klv, nhf, rs, cw, rr);
+                quantize32<KQ, QJL>(y, T, s_klv, sq * nhf, cw, rr);
                 if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
             }
             if (page && q == 0)
@@ -305,14 +312,12 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         }
 
         if (!is_v && QJL) {
-            // rho, then r scaled by 2^k (|r| < 2^14) split into fp16 hi + lo
-            xr[q * 128 + row] = rr;
-            __syncthreads();
-            const float rho = sqrtf(((xr[row] + xr[128 + row]) + xr[256 + row]) + xr[384 + row]);
-            if (page && q == 0) *reinterpret_cast<uint16_t *>(page + a.L.kr_off + pos * 2) = f2h_bits(rho);
+            // the residual (Y scale) times 2^(12 - e), ||Y|| < 2^(e + 1), so
+            // |.| < 2^14, split into fp16 hi + lo; the signs of S r do not
+            // depend on the positive scale
             int e = 0;
-            if (rho > 0.f) e = ((__float_as_int(rho) >> 23) & 0xff) - 127;
-            const int ebits = min(254, max(1, 127 + 13 - e));
+            if (ns > 0.f) e = ((__float_as_int(ns) >> 23) & 0xff) - 127;
+            const int ebits = min(254, max(1, 127 + 12 - e));
             const float sc = __int_as_float(ebits << 23);
             const int c = q >> 1;                          // 64-column half of the operand tile
             uint8_t *ahi = sm + SM_AHI + c * 16384, *alo = sm + SM_ALO + c * 16384;
@@ -332,6 +337,7 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 *reinterpret_cast<uint4 *>(ahi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
                 *reinterpret_cast<uint4 *>(alo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
             }
+            xr[q * 128 + row] = rr;
             tc05::fence_proxy_async_smem();
             tc05::fence_before_sync();
             __syncthreads();
@@ -351,6 +357,11 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                                           (sp | cc | ks) != 0);
                 tc05::mma_commit(bar_z);
             }
+            if (page && q == 0) {
+                // rho = ||r|| = ||Y-scale residual|| / sqrt(128)
+                const float rho = sqrtf(((xr[row] + xr[128 + row]) + xr[256 + row]) + xr[384 + row]) * rs;
+                *reinterpret_cast<uint16_t *>(page + a.L.kr_off + pos * 2) = f2h_bits(rho);
+            }
             pending_k = tile;
         }
 
@@ -364,10 +375,13 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             uint32_t r[32];
             tc05::tmem_ld_32x32b_x32(tmem + lane_base + uint32_t(256 + q * 32), r);
             tc05::tmem_wait_ld();
-            uint32_t b = 0;
+            // bit k = [z_k >= 0]: the complement of the float sign bit (z = -0.0
+            // lies inside the zero-tolerance of the sign comparison)
+            uint32_t neg = 0;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) b |= (__uint_as_float(r[k]) >= 0.f ? 1u : 0u) << k;
-            if (kpage && !timeout) *reinterpret_cast<uint32_t *>(kpage + a.L.ks_off + kpos * a.L.ks_bpt + q * 4) = b;
+            for (int k = 0; k < 32; ++k) neg |= (r[k] >> (31 - k)) & (1u << k);
+            if (kpage && !timeout)
+                *reinterpret_cast<uint32_t *>(kpage + a.L.ks_off + kpos * a.L.ks_bpt + q * 4) = ~neg;
             pending_k = -1;
         }
         tc05::fence_before_sync();

@@ -135,6 +135,9 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   int64_t num_blocks, float *part_o, float *part_ml, float *logits, int64_t logits_stride,
                   uint32_t *status, cudaStream_t st);
 
+// w[r] = S q_r[r] for rows x D fp32 rows (S as bf16 bits, row j = projection j).
+int launch_qproj(const float *qr, int64_t rows, int D, const uint16_t *S, float *w, cudaStream_t st);
+
 size_t score_ws_bytes(const Layout &L, int64_t n_db, int n_q, int k);
 // Tensor-core search (4-bit + QJL database, d in {128, 256, 512, 1024},
 // k <= 16): blocks per query tile, or 0 when not covered; workspace pieces;

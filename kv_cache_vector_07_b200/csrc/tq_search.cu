@@ -18,15 +18,14 @@ constexpr int kQT = 8;          // queries per block
 constexpr int kTile = 128;      // database vectors per inner step
 constexpr int kMaxK = 64;
 
+// q_r = R q, one warp per query, 4 per block (w = S q_r follows in the
+// projection kernel).
 template <int D>
-__global__ void __launch_bounds__(128) prep_f32_kernel(const float *Q, int64_t rows, DevParams p, float *qr,
-                                                       float *w) {
+__global__ void __launch_bounds__(128) prep_f32_kernel(const float *Q, int64_t rows, DevParams p, float *qr) {
     constexpr int E = WarpVec<D>::E;
-    extern __shared__ float sq_dyn[];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int64_t row = int64_t(blockIdx.x) * 4 + wl;
     if (row >= rows) return;
-    float *sq = sq_dyn + wl * D;
     float x[E], sg[E];
     load_vec<D>(Q + row * D, lane, x);
     load_vec<D>(p.signs, lane, sg);
@@ -36,18 +35,7 @@ __global__ void __launch_bounds__(128) prep_f32_kernel(const float *Q, int64_t r
     const float rs = 1.0f / sqrtf(float(D));
     if (lane < WarpVec<D>::LANES) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const float v = x[e] * rs;
-            sq[lane * E + e] = v;
-            qr[row * D + lane * E + e] = v;
-        }
-    }
-    __syncwarp();
-    for (int j = lane; j < D; j += 32) {
-        const uint16_t *srow = p.S + size_t(j) * D;
-        float acc = 0.f;
-        for (int i = 0; i < D; ++i) acc = fmaf(__uint_as_float(uint32_t(srow[i]) << 16), sq[i], acc);
-        w[row * D + j] = acc;
+        for (int e = 0; e < E; ++e) qr[row * D + lane * E + e] = x[e] * rs;
     }
 }
 
@@ -248,12 +236,11 @@ int run_score(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_
     const SPlan s = splan(L, n_db, n_q, k);
     float *qr = reinterpret_cast<float *>(ws + s.off_qr);
     float *w = reinterpret_cast<float *>(ws + s.off_w);
-    const size_t psm = sizeof(float) * 4 * D;
-    if (psm > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(prep_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(psm));
+    prep_f32_kernel<D><<<unsigned((n_q + 3) / 4), 128, 0, st>>>(Q, n_q, p->dev, qr);
+    if (L.kqjl) {
+        const int e = launch_qproj(qr, n_q, D, p->dev.S, w, st);
         if (e != cudaSuccess) return e;
     }
-    prep_f32_kernel<D><<<unsigned((n_q + 3) / 4), 128, psm, st>>>(Q, n_q, p->dev, qr, w);
     float *pv = reinterpret_cast<float *>(ws + s.off_pv);
     int64_t *pi = reinterpret_cast<int64_t *>(ws + s.off_pi);
     if (s.tc_groups > 0) {

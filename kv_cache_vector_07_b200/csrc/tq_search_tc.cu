@@ -73,260 +73,289 @@ __device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
 }
 
 // The two database rows a thread dequantizes: tile rows tid and tid + 256.
+// Rows past the end point at vector 0 with zero scales, so loads and
+// dequantization need no branches.
 struct Rows {
-    const uint8_t *page[2];
-    int pos[2];
+    const uint8_t *kc[2], *ks[2];   // this row's code bytes and sign bytes
+    uint32_t nbits[2];              // fp16 bits: nhat | rho << 16 (loaded a chunk ahead)
     uint32_t nh2[2], rh2[2];        // nhat and -rho sqrt(pi/2)/m as fp16 pairs
 };
 
 template <int D>
 __device__ __forceinline__ void rows_for(const SearchTcArgs &a, int64_t tile, int tid, Rows &r) {
     const Layout &L = a.L;
-    const float cq = 1.2533141373155003f / float(D);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const int64_t v = tile * kN + tid + 256 * j;
-        if (tile < a.n_tiles && v < a.n_db) {
-            r.page[j] = a.db + (v / L.P) * int64_t(L.page_bytes);
-            r.pos[j] = int(v % L.P);
-            const float nh = h2f_bits(*reinterpret_cast<const uint16_t *>(r.page[j] + L.kn_off + r.pos[j] * 2));
-            const float rh = h2f_bits(*reinterpret_cast<const uint16_t *>(r.page[j] + L.kr_off + r.pos[j] * 2)) * cq;
-            r.nh2[j] = h2pack(nh, nh);
-            r.rh2[j] = h2pack(-rh, -rh);
+        const bool ok = v < a.n_db;
+        const int64_t vv = ok ? v : 0;
+        const uint8_t *page = a.db + (vv / L.P) * int64_t(L.page_bytes);
+        const int pos = int(vv % L.P);
+        r.kc[j] = page + L.kc_off + pos * (D / 2);
+        r.ks[j] = page + L.ks_off + pos * (D / 8);
+        uint32_t nb = 0;
+        if (ok)
+            nb = uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2))) |
+                 (uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2))) << 16);
+        r.nbits[j] = nb;
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void rows_scales(Rows &r) {
+    const float cq = 1.2533141373155003f / float(D);     // sqrt(pi/2) / m
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t nb = r.nbits[j];
+        r.nh2[j] = (nb & 0xFFFFu) * 0x10001u;
+        const float rh = h2f_bits(uint16_t(nb >> 16)) * cq;
+        r.rh2[j] = h2pack(-rh, -rh);
+    }
+}
+
+// Raw bytes of chunk kc for both rows: 32 code bytes (MSE chunk) or 8 sign
+// bytes (QJL chunk, in raw[j][0].x / .y).
+template <int D>
+__device__ __forceinline__ void load_raw(const Rows &r, int kc, uint4 (&raw)[2][2]) {
+    constexpr int MSE_KC = D / 64;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (kc < MSE_KC) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(r.kc[j] + kc * 32);
+            raw[j][0] = __ldg(src);
+            raw[j][1] = __ldg(src + 1);
         } else {
-            r.page[j] = nullptr;
-            r.pos[j] = 0;
-            r.nh2[j] = r.rh2[j] = 0;
+            const uint2 sg = __ldg(reinterpret_cast<const uint2 *>(r.ks[j] + (kc - MSE_KC) * 8));
+            raw[j][0].x = sg.x;
+            raw[j][0].y = sg.y;
         }
     }
 }
 
-// Raw code bytes of chunk kc for both rows: 32 code bytes (MSE chunk) or 8
-// sign bytes (QJL chunk, in raw[j][0].x/.y).
-template <int D>
-__device__ __forceinline__ void load_raw(const Layout &L, const Rows &r, int kc, uint4 (&raw)[2][2]) {
+// Per-block state of the scoring loop.
+struct Ctx {
+    uint8_t *sm;
+    uint64_t *bar_a, *bar_m;
+    const CUtensorMap *tmQ;
+    uint32_t tmem;
+    int tid, warp, qt, half;
+    float *tv;                      // top-k scores, entry r of thread t at [r * 256 + t]
+    int32_t *ti;
+    const uint32_t *lut_lane;
+    uint32_t phase_a, phase_m, used_m;   // bit st: stage st's phase / MMAs outstanding
+    int a_pending;                  // thread 0: stage whose A load is not yet waited for
+    bool timeout;
+    int64_t tile;
+    int kc;
+    Rows cur, nxt;
+};
+
+// One 64-feature chunk on stage ST: prefetch the next chunk's bytes into
+// `nraw`, dequantize `raw` into shared memory, issue the MMAs, and after the
+// tile's last chunk scan its estimates.  Returns false to leave the loop.
+template <int D, int ST>
+__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 (&raw)[2][2],
+                                           uint4 (&nraw)[2][2]) {
+    constexpr int NKC = 2 * D / 64;
     constexpr int MSE_KC = D / 64;
+    const int kc = c.kc;
+    const bool last = (ST == 1) && kc == NKC - 1;     // NKC is even: tiles end on stage 1
+    if (kc == 0) rows_scales<D>(c.cur);
+    if (last) {
+        rows_for<D>(a, c.tile + a.n_groups, c.tid, c.nxt);
+        load_raw<D>(c.nxt, 0, nraw);
+    } else {
+        load_raw<D>(c.cur, kc + 1, nraw);
+    }
+
+    uint8_t *sA = c.sm + SA + ST * 16384;
+    uint8_t *sB = c.sm + SB + ST * 65536;
+    if ((c.used_m >> ST) & 1u) {        // the stage is free once the MMAs that read it completed
+        if (!tc05::mbar_wait_bounded(&c.bar_m[ST], (c.phase_m >> ST) & 1u, kPolls)) c.timeout = true;
+        c.phase_m ^= 1u << ST;
+        c.used_m &= ~(1u << ST);
+    }
+    if (c.tid == 0) {
+        tc05::mbar_expect_tx(&c.bar_a[ST], 16384);
+        tc05::tma_load_2d(sA, c.tmQ, kc * 64, c.qt * kQ, &c.bar_a[ST]);
+        c.a_pending = ST;
+    }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        raw[j][0] = raw[j][1] = make_uint4(0, 0, 0, 0);
-        if (!r.page[j]) continue;
+        uint8_t *brow = sB + j * 32768;
+        uint32_t w[32];
         if (kc < MSE_KC) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(r.page[j] + L.kc_off + r.pos[j] * (D / 2) + kc * 32);
-            raw[j][0] = __ldg(src);
-            raw[j][1] = __ldg(src + 1);
+            const uint32_t cw[8] = {raw[j][0].x, raw[j][0].y, raw[j][0].z, raw[j][0].w,
+                                    raw[j][1].x, raw[j][1].y, raw[j][1].z, raw[j][1].w};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
+                w[i] = hmul2u(c.lut_lane[byte * 32], c.cur.nh2[j]);
+            }
         } else {
-            const uint2 s = __ldg(reinterpret_cast<const uint2 *>(r.page[j] + L.ks_off + r.pos[j] * (D / 8) +
-                                                                  (kc - MSE_KC) * 8));
-            raw[j][0].x = s.x;
-            raw[j][0].y = s.y;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t word = (i < 16) ? raw[j][0].x : raw[j][0].y;
+                w[i] = c.cur.rh2[j] ^ ((word << (15 - (i & 15))) & 0x80008000u);
+            }
         }
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc)
+            *reinterpret_cast<uint4 *>(brow + tc05::sw128_offset(uint32_t(c.tid), uint32_t(pc))) =
+                make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
     }
+    tc05::fence_proxy_async_smem();
+    tc05::fence_before_sync();
+    if (__syncthreads_or(c.timeout)) return false;
+    if (c.tid == 0) {
+        if (!tc05::mbar_wait_bounded(&c.bar_a[ST], (c.phase_a >> ST) & 1u, kPolls)) c.timeout = true;
+        c.a_pending = -1;
+        tc05::fence_after_sync();
+        const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sB);
+        constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = tc05::desc_kmajor_sw128(aa + ks * 32);
+            const bool acc = (kc | ks) != 0;
+            tc05::mma_f16(c.tmem, ad, tc05::desc_kmajor_sw128(bb + ks * 32), idesc, acc);
+            tc05::mma_f16(c.tmem + 256, ad, tc05::desc_kmajor_sw128(bb + 32768 + ks * 32), idesc, acc);
+        }
+        tc05::mma_commit(&c.bar_m[ST]);
+    }
+    c.phase_a ^= 1u << ST;
+    c.used_m |= 1u << ST;
+
+    if (last) {
+        // the last commit covers every earlier MMA; consume both stages' phases
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+            const int o = ST ^ s2;
+            if ((c.used_m >> o) & 1u) {
+                if (!tc05::mbar_wait_bounded(&c.bar_m[o], (c.phase_m >> o) & 1u, kPolls)) c.timeout = true;
+                c.phase_m ^= 1u << o;
+                c.used_m &= ~(1u << o);
+            }
+        }
+        tc05::fence_after_sync();
+        // estimates stay in accumulator units (2^-e of the true value) until the end
+        const int64_t rem = a.n_db - (c.tile * kN + c.half * 256);
+        const int lim = rem < 256 ? int(rem) : 256;
+        const int32_t id0 = int32_t(c.tile * kN + c.half * 256);
+        const int K = a.k;
+        float kth = c.tv[(K - 1) * kThreads + c.tid];
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t r[32];
+            tc05::tmem_ld_32x32b_x32(c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.half * 256 + cc * 32),
+                                     r);
+            tc05::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float sv = __uint_as_float(r[e]);
+                if (sv > kth && cc * 32 + e < lim) {
+                    int p = K - 1;
+                    while (p > 0 && sv > c.tv[(p - 1) * kThreads + c.tid]) {
+                        c.tv[p * kThreads + c.tid] = c.tv[(p - 1) * kThreads + c.tid];
+                        c.ti[p * kThreads + c.tid] = c.ti[(p - 1) * kThreads + c.tid];
+                        --p;
+                    }
+                    c.tv[p * kThreads + c.tid] = sv;
+                    c.ti[p * kThreads + c.tid] = id0 + cc * 32 + e;
+                    kth = c.tv[(K - 1) * kThreads + c.tid];
+                }
+            }
+        }
+        tc05::fence_before_sync();
+        if (__syncthreads_or(c.timeout)) return false;
+        tc05::fence_after_sync();
+        c.tile += a.n_groups;
+        c.kc = 0;
+        c.cur = c.nxt;
+    } else {
+        c.kc = kc + 1;
+    }
+    return true;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
-    constexpr int NKC = 2 * D / 64;             // feature chunks per tile
-    constexpr int MSE_KC = D / 64;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint32_t *lut = reinterpret_cast<uint32_t *>(sm + SLUT);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
-    uint64_t *bar_a = bars, *bar_m = bars + 2;   // A loaded / MMAs done, per stage
     __shared__ uint32_t tmem_holder;
+    Ctx c;
+    c.sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(c.sm + SLUT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(c.sm + SBAR);
+    c.bar_a = bars;
+    c.bar_m = bars + 2;
+    c.tmQ = &tmQ;
+    c.tid = threadIdx.x;
+    c.warp = c.tid >> 5;
+    c.qt = blockIdx.x;
+    c.half = c.tid >> 7;
+    const int grp = blockIdx.y, K = a.k;
+    c.tv = reinterpret_cast<float *>(c.sm + STOPV);
+    c.ti = reinterpret_cast<int32_t *>(c.sm + STOPI);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = blockIdx.x, grp = blockIdx.y;
-    const int K = a.k;
-    const Layout &L = a.L;
-    float *tv = reinterpret_cast<float *>(sm + STOPV) + tid * kTopK;
-    int32_t *ti = reinterpret_cast<int32_t *>(sm + STOPI) + tid * kTopK;
-
-    for (int i = tid; i < 256 * 32; i += kThreads) {
+    for (int i = c.tid; i < 256 * 32; i += kThreads) {
         const int e = i >> 5;
         lut[i] = h2pack(a.lv[e & 15], a.lv[e >> 4]);
     }
     for (int r = 0; r < K; ++r) {
-        tv[r] = -INFINITY;
-        ti[r] = -1;
+        c.tv[r * kThreads + c.tid] = -INFINITY;
+        c.ti[r * kThreads + c.tid] = -1;
     }
-    if (warp == 0) {
+    if (c.warp == 0) {
         tc05::tmem_alloc(&tmem_holder, 512);
         tc05::tmem_relinquish();
     }
-    if (tid == 0) {
+    if (c.tid == 0) {
         for (int i = 0; i < 4; ++i) tc05::mbar_init(&bars[i], 1);
         tc05::fence_mbar_init();
     }
     tc05::fence_before_sync();
     __syncthreads();
     tc05::fence_after_sync();
-    const uint32_t tmem = tmem_holder;
-    constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
+    c.tmem = tmem_holder;
+    c.lut_lane = lut + (c.tid & 31);
+    c.phase_a = c.phase_m = c.used_m = 0;
+    c.a_pending = -1;
+    c.timeout = false;
+    c.tile = grp;
+    c.kc = 0;
 
-    const int q = qt * kQ + (tid & 127);
-    const int half = tid >> 7;
-    const float qsc = a.qscale[q];
-    const uint32_t *lut_lane = lut + lane;
-
-    // per-stage mbarrier phases and "MMAs outstanding" flags, bit st of each
-    uint32_t phase_a = 0, phase_m = 0, used_m = 0;
-    bool timeout = false;
-    int a_pending = -1;              // thread 0: stage whose A load is not yet waited for
-
-    int64_t tile = grp;
-    int kc = 0;
-    Rows cur;
-    rows_for<D>(a, tile, tid, cur);
-    uint4 raw[2][2];
-    load_raw<D>(L, cur, 0, raw);
-
-    while (tile < a.n_tiles) {
-        // prefetch the next step's bytes (next chunk, or the next tile's first)
-        int64_t ntile = tile;
-        int nkc = kc + 1;
-        Rows nxt = cur;
-        if (nkc == NKC) {
-            nkc = 0;
-            ntile += a.n_groups;
-            rows_for<D>(a, ntile, tid, nxt);
-        }
-        uint4 nraw[2][2];
-        load_raw<D>(L, nxt, nkc, nraw);
-
-        const int st = kc & 1;
-        uint8_t *sA = sm + SA + st * 16384;
-        uint8_t *sB = sm + SB + st * 65536;
-        // the stage is free once the MMAs that read it have completed
-        if ((used_m >> st) & 1u) {
-            if (!tc05::mbar_wait_bounded(&bar_m[st], (phase_m >> st) & 1u, kPolls)) timeout = true;
-            phase_m ^= 1u << st;
-            used_m &= ~(1u << st);
-        }
-        if (tid == 0) {
-            tc05::mbar_expect_tx(&bar_a[st], 16384);
-            tc05::tma_load_2d(sA, &tmQ, kc * 64, qt * kQ, &bar_a[st]);
-            a_pending = st;
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            uint8_t *brow = sB + j * 32768;
-            uint32_t w[32];
-            if (kc < MSE_KC) {
-                const uint32_t cw[8] = {raw[j][0].x, raw[j][0].y, raw[j][0].z, raw[j][0].w,
-                                        raw[j][1].x, raw[j][1].y, raw[j][1].z, raw[j][1].w};
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
-                    w[i] = hmul2u(lut_lane[byte * 32], cur.nh2[j]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const uint32_t word = (i < 16) ? raw[j][0].x : raw[j][0].y;
-                    const int p = i & 15;
-                    w[i] = cur.rh2[j] ^ ((word << (15 - p)) & 0x80008000u);
-                }
-            }
-#pragma unroll
-            for (int pc = 0; pc < 8; ++pc)
-                *reinterpret_cast<uint4 *>(brow + tc05::sw128_offset(uint32_t(tid), uint32_t(pc))) =
-                    make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
-        }
-        tc05::fence_proxy_async_smem();
-        tc05::fence_before_sync();
-        if (__syncthreads_or(timeout)) break;
-        if (tid == 0) {
-            if (!tc05::mbar_wait_bounded(&bar_a[st], (phase_a >> st) & 1u, kPolls)) timeout = true;
-            a_pending = -1;
-            tc05::fence_after_sync();
-            const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sB);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = tc05::desc_kmajor_sw128(aa + ks * 32);
-                const bool acc = (kc | ks) != 0;
-                tc05::mma_f16(tmem, ad, tc05::desc_kmajor_sw128(bb + ks * 32), idesc, acc);
-                tc05::mma_f16(tmem + 256, ad, tc05::desc_kmajor_sw128(bb + 32768 + ks * 32), idesc, acc);
-            }
-            tc05::mma_commit(&bar_m[st]);
-        }
-        phase_a ^= 1u << st;
-        used_m |= 1u << st;
-
-        if (kc == NKC - 1) {
-            // the last commit covers every earlier MMA; consume both stages' phases
-            for (int s2 = 0; s2 < 2; ++s2) {
-                const int o = st ^ s2;
-                if ((used_m >> o) & 1u) {
-                    if (!tc05::mbar_wait_bounded(&bar_m[o], (phase_m >> o) & 1u, kPolls)) timeout = true;
-                    phase_m ^= 1u << o;
-                    used_m &= ~(1u << o);
-                }
-            }
-            tc05::fence_after_sync();
-            const int64_t v0 = tile * kN + half * 256;
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                uint32_t r[32];
-                tc05::tmem_ld_32x32b_x32(tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(half * 256 + c * 32),
-                                         r);
-                tc05::tmem_wait_ld();
-                if (q < a.n_q) {
-                    float kth = tv[K - 1];
-                    bool full = ti[K - 1] >= 0;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float s = __uint_as_float(r[e]) * qsc;
-                        const int32_t id = int32_t(v0 + c * 32 + e);
-                        if (id < a.n_db && (!full || s > kth)) {
-                            int p = K - 1;
-                            while (p > 0 && (ti[p - 1] < 0 || s > tv[p - 1])) {
-                                tv[p] = tv[p - 1];
-                                ti[p] = ti[p - 1];
-                                --p;
-                            }
-                            tv[p] = s;
-                            ti[p] = id;
-                            kth = tv[K - 1];
-                            full = ti[K - 1] >= 0;
-                        }
-                    }
-                }
-            }
-            tc05::fence_before_sync();
-            if (__syncthreads_or(timeout)) break;
-            tc05::fence_after_sync();
-        }
-        tile = ntile;
-        kc = nkc;
-        cur = nxt;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            raw[j][0] = nraw[j][0];
-            raw[j][1] = nraw[j][1];
-        }
+    uint4 rawA[2][2], rawB[2][2];
+    rows_for<D>(a, c.tile, c.tid, c.cur);
+    load_raw<D>(c.cur, 0, rawA);
+    while (c.tile < a.n_tiles) {
+        if (!chunk_step<D, 0>(c, a, rawA, rawB)) break;
+        if (!chunk_step<D, 1>(c, a, rawB, rawA)) break;
     }
     // after an early exit, let the copy and the MMAs still in flight finish
     // before shared memory and TMEM are given back
-    if (a_pending >= 0 && !tc05::mbar_wait_bounded(&bar_a[a_pending], (phase_a >> a_pending) & 1u, kPolls))
-        timeout = true;
+    if (c.a_pending >= 0 && !tc05::mbar_wait_bounded(&c.bar_a[c.a_pending], (c.phase_a >> c.a_pending) & 1u, kPolls))
+        c.timeout = true;
 #pragma unroll
-    for (int s = 0; s < 2; ++s)
-        if (((used_m >> s) & 1u) && !tc05::mbar_wait_bounded(&bar_m[s], (phase_m >> s) & 1u, kPolls)) timeout = true;
+    for (int s2 = 0; s2 < 2; ++s2)
+        if (((c.used_m >> s2) & 1u) && !tc05::mbar_wait_bounded(&c.bar_m[s2], (c.phase_m >> s2) & 1u, kPolls))
+            c.timeout = true;
+    const int q = c.qt * kQ + (c.tid & 127);
     if (q < a.n_q) {
+        const float qsc = a.qscale[q];
         for (int r = 0; r < K; ++r) {
-            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + half) * K + r;
-            a.part_v[o] = tv[r];
-            a.part_i[o] = ti[r];
+            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + c.half) * K + r;
+            const int32_t id = c.ti[r * kThreads + c.tid];
+            a.part_v[o] = id >= 0 ? c.tv[r * kThreads + c.tid] * qsc : -INFINITY;
+            a.part_i[o] = id;
         }
     }
     tc05::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (c.warp == 0) {
         tc05::fence_after_sync();
-        tc05::tmem_dealloc(tmem, 512);
+        tc05::tmem_dealloc(c.tmem, 512);
     }
-    if (timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
+    if (c.timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
 }
 
 // Query features [n_q_pad][2d] fp16 = 2^-e [R q | S R q] (QJL half in the
