@@ -315,6 +315,7 @@ Plan make_plan(const Layout &L, const AttnShape &s) {
     int split_len = (maxlen + splits - 1) / splits;
     split_len = (split_len + kChunk - 1) / kChunk * kChunk;
     splits = (maxlen + split_len - 1) / split_len;
+    if (pf128_covers(L, s)) splits = pf128_splits(L, s, &split_len);
     p.n_splits = splits;
     p.split_len = split_len;
     const int64_t rows = int64_t(s.n_seq) * s.Hq;
@@ -347,10 +348,16 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
         if (e != cudaSuccess) return e;
     }
 
-    const int fast = launch_dec128(kp, vp, L, pa.qr, pa.w, s, p.G, p.n_groups, p.n_splits, p.split_len, cache,
-                                   num_blocks, reinterpret_cast<float *>(ws + p.off_po),
-                                   reinterpret_cast<float *>(ws + p.off_pml), logits, logits_stride,
-                                   reinterpret_cast<uint32_t *>(ws), st);
+    int fast;
+    if (pf128_covers(L, s))
+        fast = launch_pf128(kp, vp, L, pa.qr, pa.w, s, p.n_splits, p.split_len, cache, num_blocks,
+                            reinterpret_cast<float *>(ws + p.off_po), reinterpret_cast<float *>(ws + p.off_pml),
+                            reinterpret_cast<uint32_t *>(ws), st);
+    else
+        fast = launch_dec128(kp, vp, L, pa.qr, pa.w, s, p.G, p.n_groups, p.n_splits, p.split_len, cache,
+                             num_blocks, reinterpret_cast<float *>(ws + p.off_po),
+                             reinterpret_cast<float *>(ws + p.off_pml), logits, logits_stride,
+                             reinterpret_cast<uint32_t *>(ws), st);
     if (fast > 0) return fast;
 
     AttnArgs a;

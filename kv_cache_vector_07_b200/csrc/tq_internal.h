@@ -138,6 +138,15 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
 // w[r] = S q_r[r] for rows x D fp32 rows (S as bf16 bits, row j = projection j).
 int launch_qproj(const float *qr, int64_t rows, int D, const uint16_t *S, float *w, cudaStream_t st);
 
+// Tensor-core chunked prefill for d = 128, 64-token pages, b-bit + QJL keys
+// and b-bit values (b in 2..4), 128 % G == 0: whether it applies, its key
+// split (count, length in keys), and the launcher writing combine partials.
+bool pf128_covers(const Layout &L, const AttnShape &s);
+int pf128_splits(const Layout &L, const AttnShape &s, int *split_len);
+int launch_pf128(const tq_params *kp, const tq_params *vp, const Layout &L, const float *qr, const float *w,
+                 const AttnShape &s, int n_splits, int split_len, const uint8_t *cache, int64_t num_blocks,
+                 float *part_o, float *part_ml, uint32_t *status, cudaStream_t st);
+
 size_t score_ws_bytes(const Layout &L, int64_t n_db, int n_q, int k);
 // Tensor-core search (4-bit + QJL database, d in {128, 256, 512, 1024},
 // k <= 16): blocks per query tile, or 0 when not covered; workspace pieces;

@@ -211,6 +211,43 @@ def test_long_context_decode_and_prefill_sampled():
 
 
 # ---------------------------------------------------------------------------
+# tensor-core prefill: every output and lse, ragged query tiles, ragged last
+# page, several key splits, G = 1 .. 8
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kbits,vbits,Hq,H,C,L", [
+    (2, 3, 32, 4, 100, 5000),     # G = 8: 16 positions per block, last block ragged, four key splits
+    (3, 3, 8, 8, 64, 3100),       # G = 1: 128 positions per block, half used
+    (4, 4, 16, 2, 40, 2600),      # G = 8, two KV heads
+    (2, 2, 2, 1, 70, 1500),       # G = 2: 64 positions per block
+    (3, 4, 8, 2, 33, 4096),       # G = 4, one position in the last block
+])
+def test_prefill_tensor_core_every_output(kbits, vbits, Hq, H, C, L):
+    d, P = 128, 64
+    seed = 40 + kbits * 10 + vbits
+    K = synth.outlier_normal((L, H, d), seed=seed, device=DEV)
+    V = synth.outlier_normal((L, H, d), seed=seed + 1, device=DEV)
+    cd = Codec(d, kbits, True, vbits, seed=seed, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(1, L, P, device=DEV, shuffle_seed=seed)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    Qp = synth.normal((C, Hq, d), seed=seed + 2, device=DEV)
+    lse = torch.empty((C, Hq), device=DEV)
+    out = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qp, bt.view(-1), L, cache, lse=lse)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for kvh in range(H):
+        Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl, f64(K[:, kvh]), f64(V[:, kvh]), kvh)
+        rows = list(range(kvh * G, kvh * G + G))
+        Qr = f64(Qp[:, rows]).reshape(C * G, d)
+        nvis = np.repeat(np.arange(L - C + 1, L + 1, dtype=np.int32), G)
+        o_p, lse_p, lg_p = O.attend(Qr, cd.Pk, Ek, cd.Pv, Ev, nvis=nvis, want_logits=True)
+        parity.check_outputs(f64(out[:, rows]).reshape(C * G, d), o_p, cd.slack(Ev, lg_p, lse_p, o_p))
+        assert np.allclose(f64(lse[:, rows]).reshape(C * G), lse_p, rtol=1e-3, atol=1e-3)
+
+
+# ---------------------------------------------------------------------------
 # search
 # ---------------------------------------------------------------------------
 def _search_case(n_db, n_q, seed, d=1024):
