@@ -216,13 +216,14 @@ class StepWorkload:
         enc_gbs = self.enc_bytes / (op_ms["encode"] * 1e-3) / 1e9
         dec_gbs = self.dec_bytes / (op_ms["decode"] * 1e-3) / 1e9
         return ({"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                 "frac": round(enc_gbs / hbm_peak, 4), "traffic": traffic_for("encode"),
+                 "frac": round(enc_gbs / hbm_peak, 4), "traffic": traffic_for("step/encode") if self.default_size else None,
                  "kernel": "tq_encode (encode128_kernel: TMA + tcgen05 rotation + quantize + tcgen05 QJL)",
                  "algorithmic_bytes": self.enc_bytes},
                 {"encode": {"vectors_per_s": self.n_vec / (op_ms["encode"] * 1e-3), "ms": op_ms["encode"],
                             "gbs": enc_gbs, "frac": enc_gbs / hbm_peak, "algorithmic_bytes": self.enc_bytes},
                  "decode": {"keys_scored_per_s": self.n_pairs / (op_ms["decode"] * 1e-3), "ms": op_ms["decode"],
-                            "gbs": dec_gbs, "frac": dec_gbs / hbm_peak, "algorithmic_bytes": self.dec_bytes}})
+                            "gbs": dec_gbs, "frac": dec_gbs / hbm_peak, "algorithmic_bytes": self.dec_bytes,
+                            "traffic": traffic_for("step/decode") if self.default_size else None}})
 
     def config(self):
         return {"workload": self.name, "batch": self.B, "seq_len": self.L, "n_kv_heads": self.H,
@@ -281,7 +282,7 @@ class Decode32kWorkload:
     def roofline(self, op_ms, hbm_peak):
         gbs = self.dec_bytes / (op_ms["decode"] * 1e-3) / 1e9
         return ({"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                 "frac": round(gbs / hbm_peak, 4), "traffic": traffic_for("decode"),
+                 "frac": round(gbs / hbm_peak, 4), "traffic": traffic_for("decode32k/decode") if self.default_size else None,
                  "kernel": "tq_decode_attn (prep + attn + combine)", "algorithmic_bytes": self.dec_bytes},
                 {"decode": {"keys_scored_per_s": self.units / (op_ms["decode"] * 1e-3), "ms": op_ms["decode"],
                             "gbs": gbs, "frac": gbs / hbm_peak}})
@@ -355,7 +356,7 @@ class LongCtxWorkload:
         tf = self.pre_flops / (op_ms["prefill"] * 1e-3) / 1e12
         gbs = self.dec_bytes / (op_ms["decode"] * 1e-3) / 1e9
         return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl_s, "unit": "TFLOP/s",
-                 "frac": round(tf / tfl_s, 4), "traffic": traffic_for("prefill"),
+                 "frac": round(tf / tfl_s, 4), "traffic": traffic_for("longctx/prefill") if self.default_size else None,
                  "kernel": "tq_prefill_attn", "algorithmic_flops": self.pre_flops,
                  "peak_note": "sustained fp16/bf16 dense (MEASURED_PEAKS.json bf16_tflops_sustained)"},
                 {"decode": {"keys_scored_per_s": self.dec_pairs / (op_ms["decode"] * 1e-3), "ms": op_ms["decode"],
@@ -423,7 +424,7 @@ class SearchWorkload:
         tf = self.flops / (op_ms["score"] * 1e-3) / 1e12
         # a search of tens of milliseconds timed on its own: the burst figure
         return ({"bound": "tensor", "achieved": round(tf, 2), "peak": tfl, "unit": "TFLOP/s",
-                 "frac": round(tf / tfl, 4), "traffic": traffic_for("score"), "kernel": "tq_score",
+                 "frac": round(tf / tfl, 4), "traffic": traffic_for("search/score") if self.default_size else None, "kernel": "tq_score",
                  "algorithmic_flops": self.flops,
                  "peak_note": "burst fp16/bf16 dense (MEASURED_PEAKS.json bf16_tflops; fp16 nominal = bf16 nominal)"},
                 {"score": {"scores_per_s": self.units / (op_ms["score"] * 1e-3), "ms": op_ms["score"], "tflops": tf},
@@ -438,20 +439,23 @@ WORKLOADS = {"step": StepWorkload, "decode32k": Decode32kWorkload, "longctx": Lo
              "search": SearchWorkload}
 
 
-def traffic_for(op: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the kernels as currently built (matching source digest)."""
+def traffic_for(key: str):
+    """DRAM bytes per launch ("workload/op") from the committed ncu summary,
+    scaled to the workload; None unless the kernel's source is unchanged
+    since the capture (matching sha256)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
-            j = json.load(f)
-        from kv_cache_vector_07_b200 import build as b
-        if j.get("source_digest") != b._digest():
+            e = json.load(f).get("entries", {}).get(key)
+        if not e:
             return None
-        v = j.get("ops", {}).get(op)
-        return v
+        with open(os.path.join(ROOT, e["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != e["sha256"]:
+                return None
+        return int(e["bytes_per_launch"])
     except Exception:
         return None
 
@@ -467,6 +471,7 @@ def run_ours(args):
     sizes = {k: v for k, v in (("batch", args.batch), ("seq_len", args.seq_len), ("n_db", args.n_db),
                                ("n_q", args.n_q)) if v}
     wl = WORKLOADS[args.workload](dev, **sizes)
+    wl.default_size = not sizes           # committed traffic counts refer to the default sizes
     ops = wl.ops()
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
