@@ -7,24 +7,24 @@
 //   ( nhat_t <Rq, c[code_t]> + rho_t sqrt(pi/2)/m <S R q, 2 s_t - 1> ) / sqrt(d),
 // then softmax and the sum of dequantized values nhat_v c_v[code] (rotated
 // back by the combine kernel).  A block takes 128 query rows (positions x
-// GQA heads of one KV head) and walks one key split a page at a time:
-//   dequantize   all 256 threads: centroids of the page's 64 keys as fp16
-//                hi + lo tiles, the QJL signs as a +-1 tile, per-key scales;
-//   MMA  QK      S_mse = q_hi C_hi + q_lo C_hi + q_hi C_lo and
-//                S_qjl = w_hi Sigma + w_lo Sigma on tcgen05 (TMEM
-//                accumulators): the hi/lo splits keep both terms at
-//                fp32-level accuracy, which large logits need;
-//   softmax      one thread per row (TMEM lane): logits, causal mask, online
-//                max / sum, P' = p nhat_v as fp16 hi + lo into shared memory
-//                (lo over the C_lo tile, dead once QK completed), O rescaled
-//                in TMEM when the row maximum grows;
-//                meanwhile warps 4-7 dequantize the values as fp16 hi + lo
-//                tiles (MN-major; lo over the C_hi tile);
-//   MMA  PV      O += P'_hi V_hi + P'_lo V_hi + P'_hi V_lo on tcgen05: with
-//                outlier value channels, fp16 weights or fp16 centroids alone
-//                move outputs by more than the output tolerance.
-// The split's partial (O, max, sum) goes to the workspace in the layout the
-// log-sum-exp combine kernel reads.
+// GQA heads of one KV head) and walks one key split a page (64 keys) at a
+// time, with three warp roles synchronized by mbarriers:
+//   producers (warps 8-11)  dequantize page t into stage t % 2: centroids as
+//                fp16 hi + lo tiles, QJL signs as a +-1 tile, value
+//                centroids as fp16 hi + lo tiles (MN-major), per-key scales;
+//   MMA issuer (warp 12)    QK(t): S_mse = q_hi C_hi + q_lo C_hi + q_hi C_lo,
+//                S_qjl = w_hi Sigma + w_lo Sigma, with the query tiles as the
+//                A operand in tensor memory; then PV(t - 1):
+//                O += P_hi V_hi + P_lo V_hi + P_hi V_lo;
+//   softmax (warps 0-7)     two threads per row (TMEM lane), one per half of
+//                the page's keys: logits, causal mask, online max / sum (both
+//                threads of a row compute the page maximum from all 64
+//                columns, so they agree without exchanging), O rescaled in
+//                TMEM when the maximum grows, P' = p nhat_v as fp16 hi + lo.
+// QK(t + 1) runs while the softmax of page t works and the producers fill
+// page t + 2.  The hi/lo splits keep logits and outputs within tolerance
+// with outlier channels.  The split's partial (O, max, sum) goes to the
+// workspace in the layout the log-sum-exp combine kernel reads.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -35,19 +35,27 @@ namespace tq {
 namespace {
 
 constexpr int kKeys = 64;               // keys per tile (one page)
+constexpr int kThreads = 416;           // 8 softmax + 4 producer warps + 1 MMA warp
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 // shared layout (offsets from a 1024-aligned base)
-constexpr uint32_t SQH = 0, SQL = 32768, SQW = 65536, SQWL = 98304;   // [128 x 128] fp16, K-major, halves at +16 KB
-constexpr uint32_t SKH = 131072, SKL = SKH + 16384, SKS = SKL + 16384;  // [64 x 128], halves at +8 KB
-constexpr uint32_t SV = SKS + 16384;                              // [64 keys x 128 dims], MN-major (V_hi; V_lo at SKH)
-constexpr uint32_t SP = SV + 16384;                               // [128 x 64] fp16, K-major (P'_hi; P'_lo at SKL)
-constexpr uint32_t SKLUT = SP + 16384;                            // K pair table, <= 8 KB
-constexpr uint32_t SVLUT = SKLUT + 8192;                          // V pair table, <= 8 KB
-constexpr uint32_t SMETA = SVLUT + 8192;                          // float4 [64]: a, b, nhat_v, 0
-constexpr uint32_t SBAR = SMETA + 1024;
-constexpr uint32_t SM_TOTAL = SBAR + 64 + 1024;
-static_assert(SM_TOTAL <= 232448, "shared memory");
+constexpr uint32_t kStage = 81920;                       // one page's operand tiles
+constexpr uint32_t OKH = 0, OKL = 16384, OKS = 32768;    // [64 keys x 128] K-major, halves at +8 KB
+constexpr uint32_t OVH = 49152, OVL = 65536;             // [64 keys x 128 dims] MN-major, halves at +8 KB
+// P' hi / lo [128 rows x 64 keys] K-major go over the stage's C_hi / C_lo
+// tiles, dead once QK of the page has completed
+constexpr uint32_t SKLUT = 2 * kStage;                   // K pair table, 8 KB
+constexpr uint32_t SVLUT = SKLUT + 8192;                 // V pair table, 8 KB
+constexpr uint32_t SMETA = SVLUT + 8192;                 // float4 [2][64]: a, b, nhat_v, 0
+constexpr uint32_t SQS = SMETA + 2048;                   // float [128] query scales
+constexpr uint32_t SLSUM = SQS + 512;                    // float [2][128] per-half row sums
+constexpr uint32_t SFLAG = SLSUM + 1024;                 // abort flag
+constexpr uint32_t SBAR = SFLAG + 128;                   // mbarriers, page-valid flags
+constexpr uint32_t SRAW = SBAR + 256;                    // two raw pages (bulk copies), page_bytes each
+constexpr uint32_t smem_bytes(int page_bytes) { return SRAW + 2u * uint32_t((page_bytes + 127) & ~127) + 1024u; }
+
+// TMEM columns
+constexpr uint32_t TQH = 0, TQL = 64, TWH = 128, TWL = 192, TSM = 256, TSQ = 320, TO = 384;
 
 struct Pf128Args {
     Layout L;
@@ -122,8 +130,18 @@ __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// Bounded wait that also gives up once another thread has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag) {
+    for (uint32_t i = 0; i < kPolls; ++i) {
+        if (tc05::mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u && *abort_flag) return false;
+    }
+    *abort_flag = 1u;
+    return false;
+}
+
 template <int KB, int VB>
-__global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
+__global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
     constexpr int NCK = pair_copies<KB, 8, 8192>(), NCV = pair_copies<VB, 8, 8192>();
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_holder;
@@ -131,8 +149,20 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
     uint2 *lutk = reinterpret_cast<uint2 *>(sm + SKLUT);
     uint2 *lutv = reinterpret_cast<uint2 *>(sm + SVLUT);
     float4 *meta = reinterpret_cast<float4 *>(sm + SMETA);
+    float *qs_arr = reinterpret_cast<float *>(sm + SQS);
+    float *lsum = reinterpret_cast<float *>(sm + SLSUM);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + SFLAG);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
-    uint64_t *bar_qk = bars, *bar_pv = bars + 1;
+    uint64_t *full = bars;          // [2] producers -> MMA (count 128)
+    uint64_t *pv_done = bars + 2;   // [2] PV of a stage's page completed (commit)
+    uint64_t *qk_full = bars + 4;   // QK completed (commit)
+    uint64_t *s_free = bars + 5;    // softmax read S (count 256)
+    uint64_t *p_full = bars + 6;    // softmax wrote P and rescaled O (count 256)
+    uint64_t *raw_full = bars + 7;  // [2] raw page landed (bulk copy, or plain arrive for a missing page)
+    uint64_t *raw_empty = bars + 9; // [2] producers finished reading a raw page (count 128)
+    int *pvalid = reinterpret_cast<int *>(sm + SBAR + 128);   // [2] raw page present
+    const uint32_t raw_stride = uint32_t((a.L.page_bytes + 127) & ~127);
+    uint8_t *raw = sm + SRAW;
 
     const Layout &L = a.L;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,23 +173,25 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
     const int vis_max = a.base_len + j_hi;                 // keys the tile's last row sees
     const int k_begin = split * a.split_len;
     const int k_end = min(k_begin + a.split_len, vis_max);
-    // row of this thread (warps 0-3 own the 128 TMEM lanes)
-    const int r = tid & 127;
+    // softmax rows: warps w and w + 4 share lanes 32 (w % 4) ..
+    const int r = (warp & 3) * 32 + lane;
+    const int half = (warp >> 2) & 1;
     const int jr = j_lo + r / G, hr = r - (r / G) * G;
     const bool row_ok = jr < a.C;
     const int vis_r = row_ok ? a.base_len + jr + 1 : 0;
     const int64_t pbase = ((int64_t(jr) * L.H + kvh) * a.n_splits + split) * G + hr;
 
     if (k_begin >= k_end) {                                // nothing visible in this split
-        if (tid < 128 && row_ok) {
+        if (warp < 4 && row_ok) {
             a.part_ml[pbase * 2] = -INFINITY;
             a.part_ml[pbase * 2 + 1] = 0.f;
         }
         return;
     }
+    const int n_tiles = (k_end - k_begin + kKeys - 1) / kKeys;
 
     // ---- tables
-    for (int i = tid; i < pair_entries<KB>() * NCK; i += 256) {
+    for (int i = tid; i < pair_entries<KB>() * NCK; i += kThreads) {
         int k0, k1;
         pair_codes<KB>(i / NCK, k0, k1);
         const float c0 = a.k_lv[k0], c1 = a.k_lv[k1];
@@ -167,7 +199,7 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
         const float2 hf = __half22float2(h);
         lutk[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&h), h2u(c0 - hf.x, c1 - hf.y));
     }
-    for (int i = tid; i < pair_entries<VB>() * NCV; i += 256) {
+    for (int i = tid; i < pair_entries<VB>() * NCV; i += kThreads) {
         int k0, k1;
         pair_codes<VB>(i / NCV, k0, k1);
         const float c0 = a.v_lv[k0], c1 = a.v_lv[k1];
@@ -175,9 +207,34 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
         const float2 hf = __half22float2(h);
         lutv[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&h), h2u(c0 - hf.x, c1 - hf.y));
     }
-    // ---- query tiles: row r = 2^-e [q_r hi | q_r lo | w hi | w lo], 1 <= max |.| < 2
-    float qs = 1.f;                                        // 2^e
-    if (tid < 128) {
+    if (warp == 12) {
+        tc05::tmem_alloc(&tmem_holder, 512);
+        tc05::tmem_relinquish();
+        if (lane == 0) {
+            tc05::mbar_init(&full[0], 128);
+            tc05::mbar_init(&full[1], 128);
+            tc05::mbar_init(&pv_done[0], 1);
+            tc05::mbar_init(&pv_done[1], 1);
+            tc05::mbar_init(qk_full, 1);
+            tc05::mbar_init(s_free, 256);
+            tc05::mbar_init(p_full, 256);
+            tc05::mbar_init(&raw_full[0], 1);
+            tc05::mbar_init(&raw_full[1], 1);
+            tc05::mbar_init(&raw_empty[0], 128);
+            tc05::mbar_init(&raw_empty[1], 128);
+            *abort_flag = 0u;
+            tc05::fence_mbar_init();
+        }
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    tc05::fence_after_sync();
+    const uint32_t tmem = tmem_holder;
+    const uint32_t lrow = uint32_t((warp & 3) * 32) << 16;
+
+    // ---- query tiles into TMEM: row r = 2^-e [q_r hi | q_r lo | w hi | w lo],
+    // 1 <= max |.| < 2, 64 columns each (two fp16 per column)
+    if (warp < 4) {
         const float *qp = a.qr + (int64_t(jr) * a.Hq + int64_t(kvh) * G + hr) * 128;
         const float *wp = a.w + (int64_t(jr) * a.Hq + int64_t(kvh) * G + hr) * 128;
         float mx = 0.f;
@@ -191,116 +248,137 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
         int ex = 0;
         if (mx > 0.f) frexpf(mx, &ex);
         const float down = mx > 0.f ? ldexpf(1.f, 1 - ex) : 1.f;
-        qs = mx > 0.f ? ldexpf(1.f, ex - 1) : 1.f;
+        qs_arr[r] = mx > 0.f ? ldexpf(1.f, ex - 1) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
-            float x[8], y[8];
-            if (row_ok) {
-                const float4 x0 = *reinterpret_cast<const float4 *>(qp + 8 * c);
-                const float4 x1 = *reinterpret_cast<const float4 *>(qp + 8 * c + 4);
-                const float4 y0 = *reinterpret_cast<const float4 *>(wp + 8 * c);
-                const float4 y1 = *reinterpret_cast<const float4 *>(wp + 8 * c + 4);
-                x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w; x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
-                y[0] = y0.x; y[1] = y0.y; y[2] = y0.z; y[3] = y0.w; y[4] = y1.x; y[5] = y1.y; y[6] = y1.z; y[7] = y1.w;
-            } else {
+        for (int c = 0; c < 4; ++c) {                      // 32 coordinates -> 16 columns per tile
+            uint32_t qh[16], ql[16], wh[16], wl[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = y[e] = 0.f;
-            }
-            uint32_t wh[4], wl[4], ww[4], wwl[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a0 = x[2 * e] * down, a1 = x[2 * e + 1] * down;
-                const __half2 h = __floats2half2_rn(a0, a1);
+            for (int e = 0; e < 16; ++e) {
+                float x0 = 0.f, x1 = 0.f, y0 = 0.f, y1 = 0.f;
+                if (row_ok) {
+                    const float2 x = *reinterpret_cast<const float2 *>(qp + 32 * c + 2 * e);
+                    const float2 y = *reinterpret_cast<const float2 *>(wp + 32 * c + 2 * e);
+                    x0 = x.x * down; x1 = x.y * down; y0 = y.x * down; y1 = y.y * down;
+                }
+                const __half2 h = __floats2half2_rn(x0, x1);
                 const float2 hf = __half22float2(h);
-                wh[e] = *reinterpret_cast<const uint32_t *>(&h);
-                wl[e] = h2u(a0 - hf.x, a1 - hf.y);
-                const float b0 = y[2 * e] * down, b1 = y[2 * e + 1] * down;
-                const __half2 g = __floats2half2_rn(b0, b1);
+                qh[e] = *reinterpret_cast<const uint32_t *>(&h);
+                ql[e] = h2u(x0 - hf.x, x1 - hf.y);
+                const __half2 g = __floats2half2_rn(y0, y1);
                 const float2 gf = __half22float2(g);
-                ww[e] = *reinterpret_cast<const uint32_t *>(&g);
-                wwl[e] = h2u(b0 - gf.x, b1 - gf.y);
+                wh[e] = *reinterpret_cast<const uint32_t *>(&g);
+                wl[e] = h2u(y0 - gf.x, y1 - gf.y);
             }
-            const uint32_t off = uint32_t(c >> 3) * 16384u + tc05::sw128_offset(uint32_t(r), uint32_t(c & 7));
-            *reinterpret_cast<uint4 *>(sm + SQH + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            *reinterpret_cast<uint4 *>(sm + SQL + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            *reinterpret_cast<uint4 *>(sm + SQW + off) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
-            *reinterpret_cast<uint4 *>(sm + SQWL + off) = make_uint4(wwl[0], wwl[1], wwl[2], wwl[3]);
+            tc05::tmem_st_32x32b_x16(tmem + lrow + TQH + uint32_t(16 * c), qh);
+            tc05::tmem_st_32x32b_x16(tmem + lrow + TQL + uint32_t(16 * c), ql);
+            tc05::tmem_st_32x32b_x16(tmem + lrow + TWH + uint32_t(16 * c), wh);
+            tc05::tmem_st_32x32b_x16(tmem + lrow + TWL + uint32_t(16 * c), wl);
         }
+        tc05::tmem_wait_st();
     }
-    if (warp == 0) {
-        tc05::tmem_alloc(&tmem_holder, 256);
-        tc05::tmem_relinquish();
-    }
-    if (tid == 0) {
-        tc05::mbar_init(bar_qk, 1);
-        tc05::mbar_init(bar_pv, 1);
-        tc05::fence_mbar_init();
-    }
-    tc05::fence_proxy_async_smem();
     tc05::fence_before_sync();
     __syncthreads();
     tc05::fence_after_sync();
-    const uint32_t tmem = tmem_holder;
-    const uint32_t t_smse = tmem, t_sqjl = tmem + 64, t_o = tmem + 128;
-    const uint32_t lrow = uint32_t((warp & 3) * 32) << 16;
 
     const float sl = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
     const float cq = 1.2533141373155003f / 128.f;                    // sqrt(pi/2) / m
-    float m_run = -INFINITY, l_run = 0.f;                            // log2 units
-    uint32_t ph_qk = 0, ph_pv = 0;
     bool timeout = false;
-    const int n_tiles = (k_end - k_begin + kKeys - 1) / kKeys;
 
-    for (int t = 0; t < n_tiles; ++t) {
-        const int k0 = k_begin + t * kKeys;
-        if (t > 0) {                                   // PV of the previous tile read V and P
-            if (!tc05::mbar_wait_bounded(bar_pv, ph_pv, kPolls)) timeout = true;
-            ph_pv ^= 1u;
-            tc05::fence_after_sync();
-        }
-        // ---- dequantize: key kk, coordinates [32 qq, 32 qq + 32)
-        {
-            const int kk = tid >> 2, qq = tid & 3;
-            const int kidx = k0 + kk;
-            const uint8_t *page = nullptr;
-            if (kidx < k_end) {
-                const int blk = a.block_table[kidx >> 6];
-                if (blk >= 0 && blk < a.num_blocks)
-                    page = a.cache + (int64_t(blk) * L.H + kvh) * int64_t(L.page_bytes);
-                else
-                    atomicOr(a.status, TQ_DEV_BLOCK_RANGE);
-            }
-            const int pos = kidx & 63;
-            uint32_t kh[16], kl[16], ks[16];
-            if (page) {
-                uint32_t lo[4], hi;
-                load_codes<KB>(page + L.kc_off, L.kc_bpt, page + L.kh_off, L.kh_bpt, pos, qq, lo, hi);
-                const uint2 *lk = lutk + (lane & (NCK - 1));
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const uint2 e = lk[pair_index<KB>(lo, hi, p) * NCK];
-                    kh[p] = e.x;
-                    kl[p] = e.y;
-                }
-                const uint32_t sg = *reinterpret_cast<const uint32_t *>(page + L.ks_off + pos * L.ks_bpt + qq * 4);
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const uint32_t b = sg >> (2 * p);          // bit 0: coordinate 2p, bit 1: 2p + 1
-                    ks[p] = 0xBC00BC00u ^ (((b << 15) & 0x8000u) | ((b << 30) & 0x80000000u));
-                }
+    if (warp >= 8 && warp < 12) {
+        // ================= producers: key kk (one per lane), dims [64 hh, 64 hh + 64);
+        // pages arrive by bulk copy two pages ahead into a raw ring
+        const int t4 = tid - 256, kk = t4 & 63, hh = t4 >> 6;
+        const uint2 *lk = lutk + (lane & (NCK - 1));
+        const uint2 *lv = lutv + (lane & (NCV - 1));
+        auto issue_raw = [&](int t) {                       // thread 256 only
+            const int rs = t & 1;
+            const int kp = k_begin + t * kKeys;
+            int blk = -1;
+            if (kp < k_end) blk = a.block_table[kp >> 6];
+            if (blk >= 0 && blk < a.num_blocks) {
+                pvalid[rs] = 1;
+                tc05::mbar_expect_tx(&raw_full[rs], uint32_t(L.page_bytes));
+                tc05::bulk_g2s(raw + rs * raw_stride, a.cache + (int64_t(blk) * L.H + kvh) * int64_t(L.page_bytes),
+                               uint32_t(L.page_bytes), &raw_full[rs]);
             } else {
-#pragma unroll
-                for (int p = 0; p < 16; ++p) kh[p] = kl[p] = ks[p] = 0u;
+                if (kp < k_end) atomicOr(a.status, TQ_DEV_BLOCK_RANGE);
+                pvalid[rs] = 0;
+                tc05::mbar_arrive(&raw_full[rs]);
             }
-            const uint32_t half = uint32_t(qq >> 1) * 8192u;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t off = half + tc05::sw128_offset(uint32_t(kk), uint32_t((qq & 1) * 4 + c));
-                *reinterpret_cast<uint4 *>(sm + SKH + off) = make_uint4(kh[4 * c], kh[4 * c + 1], kh[4 * c + 2], kh[4 * c + 3]);
-                *reinterpret_cast<uint4 *>(sm + SKL + off) = make_uint4(kl[4 * c], kl[4 * c + 1], kl[4 * c + 2], kl[4 * c + 3]);
-                *reinterpret_cast<uint4 *>(sm + SKS + off) = make_uint4(ks[4 * c], ks[4 * c + 1], ks[4 * c + 2], ks[4 * c + 3]);
+        };
+        int issued = 0, landed = 0;                          // thread 256: raw pages requested / seen landed
+        if (tid == 256) {
+            issue_raw(0);
+            if (n_tiles > 1) issue_raw(1);
+            issued = min(2, n_tiles);
+        }
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t & 1;
+            uint8_t *sb = sm + uint32_t(st) * kStage;
+            if (t >= 2 && !wait_or_abort(&pv_done[st], uint32_t((t - 2) >> 1) & 1u, abort_flag)) {
+                timeout = true;
+                break;
             }
-            if (qq == 0) {
+            if (!wait_or_abort(&raw_full[st], uint32_t(t >> 1) & 1u, abort_flag)) {
+                timeout = true;
+                break;
+            }
+            landed = t + 1;
+            const int kidx = k_begin + t * kKeys + kk;
+            const uint8_t *page = (pvalid[st] && kidx < k_end) ? raw + st * raw_stride : nullptr;
+            const int pos = kk;
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                const int qq = 2 * hh + sub;
+                uint32_t x0[16], x1[16], x2[16];
+                if (page) {
+                    uint32_t lo[4], hi;
+                    load_codes<KB>(page + L.kc_off, L.kc_bpt, page + L.kh_off, L.kh_bpt, pos, qq, lo, hi);
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const uint2 e = lk[pair_index<KB>(lo, hi, p) * NCK];
+                        x0[p] = e.x;
+                        x1[p] = e.y;
+                    }
+                    const uint32_t sg = *reinterpret_cast<const uint32_t *>(page + L.ks_off + pos * L.ks_bpt + qq * 4);
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const uint32_t b = sg >> (2 * p);      // bit 0: coordinate 2p, bit 1: 2p + 1
+                        x2[p] = 0xBC00BC00u ^ (((b << 15) & 0x8000u) | ((b << 30) & 0x80000000u));
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) x0[p] = x1[p] = x2[p] = 0u;
+                }
+                const uint32_t hoff = uint32_t(hh) * 8192u;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
+                    *reinterpret_cast<uint4 *>(sb + OKH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(sb + OKL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(sb + OKS + off) = make_uint4(x2[4 * c], x2[4 * c + 1], x2[4 * c + 2], x2[4 * c + 3]);
+                }
+                if (page) {
+                    uint32_t lo[4], hi;
+                    load_codes<VB>(page + L.vc_off, L.vc_bpt, page + L.vh_off, L.vh_bpt, pos, qq, lo, hi);
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const uint2 e = lv[pair_index<VB>(lo, hi, p) * NCV];
+                        x0[p] = e.x;
+                        x1[p] = e.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) x0[p] = x1[p] = 0u;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
+                    *reinterpret_cast<uint4 *>(sb + OVH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(sb + OVL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
+                }
+            }
+            if (hh == 0) {
                 float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (page) {
                     const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2));
@@ -308,109 +386,145 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
                     const float nv = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.vn_off + pos * 2));
                     m4 = make_float4(nk * sl, rk * cq * sl, nv, 0.f);
                 }
-                meta[kk] = m4;
+                meta[st * 64 + kk] = m4;
             }
-        }
-        tc05::fence_proxy_async_smem();
-        tc05::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tc05::fence_after_sync();
-            constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 64);
-            const uint32_t qh = tc05::smem_u32(sm + SQH), ql = tc05::smem_u32(sm + SQL);
-            const uint32_t qw = tc05::smem_u32(sm + SQW), qwl = tc05::smem_u32(sm + SQWL);
-            const uint32_t bh = tc05::smem_u32(sm + SKH), bl = tc05::smem_u32(sm + SKL), bs = tc05::smem_u32(sm + SKS);
-            // passes: q_hi C_hi, q_lo C_hi, q_hi C_lo -> S_mse; w_hi Sigma, w_lo Sigma -> S_qjl
-#pragma unroll
-            for (int pass = 0; pass < 5; ++pass) {
-                const uint32_t A = pass == 1 ? ql : pass == 3 ? qw : pass == 4 ? qwl : qh;
-                const uint32_t B = pass == 2 ? bl : pass >= 3 ? bs : bh;
-                const uint32_t D = pass >= 3 ? t_sqjl : t_smse;
-                const bool first = pass == 0 || pass == 3;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t ad = tc05::desc_kmajor_sw128(A + uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u);
-                    const uint64_t bd = tc05::desc_kmajor_sw128(B + uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u);
-                    tc05::mma_f16(D, ad, bd, idesc, !first || ks > 0);
-                }
-            }
-            tc05::mma_commit(bar_qk);
-        }
-        // ---- values: warps 4-7, key kk, dims [64 hh, 64 hh + 64), once QK has
-        // read the C_hi tile that V_lo overwrites
-        if (warp >= 4) {
-            const int t4 = tid - 128, kk = t4 >> 1, hh = t4 & 1;
-            const int kidx = k0 + kk;
-            const uint8_t *page = nullptr;
-            if (kidx < k_end) {
-                const int blk = a.block_table[kidx >> 6];
-                if (blk >= 0 && blk < a.num_blocks) page = a.cache + (int64_t(blk) * L.H + kvh) * int64_t(L.page_bytes);
-            }
-            const int pos = kidx & 63;
-            if (!tc05::mbar_wait_bounded(bar_qk, ph_qk, kPolls)) timeout = true;
-            tc05::fence_after_sync();
-            const uint2 *lv = lutv + (lane & (NCV - 1));
-#pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {
-                const int qq = 2 * hh + sub;
-                uint32_t vh[16], vl[16];
-                if (page) {
-                    uint32_t lo[4], hi;
-                    load_codes<VB>(page + L.vc_off, L.vc_bpt, page + L.vh_off, L.vh_bpt, pos, qq, lo, hi);
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) {
-                        const uint2 e = lv[pair_index<VB>(lo, hi, p) * NCV];
-                        vh[p] = e.x;
-                        vl[p] = e.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) vh[p] = vl[p] = 0u;
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = uint32_t(hh) * 8192u + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
-                    *reinterpret_cast<uint4 *>(sm + SV + off) = make_uint4(vh[4 * c], vh[4 * c + 1], vh[4 * c + 2], vh[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(sm + SKH + off) = make_uint4(vl[4 * c], vl[4 * c + 1], vl[4 * c + 2], vl[4 * c + 3]);
-                }
-            }
+            tc05::mbar_arrive(&raw_empty[st]);                  // raw page read
             tc05::fence_proxy_async_smem();
+            tc05::mbar_arrive(&full[st]);
+            if (tid == 256 && t + 2 < n_tiles) {
+                // the raw slot is refilled once every producer has read it
+                if (!wait_or_abort(&raw_empty[st], uint32_t(t >> 1) & 1u, abort_flag)) {
+                    timeout = true;
+                    break;
+                }
+                issue_raw(t + 2);
+                issued = t + 3;
+            }
         }
-        // ---- softmax: warps 0-3, thread = row
-        if (warp < 4) {
-            if (!tc05::mbar_wait_bounded(bar_qk, ph_qk, kPolls)) timeout = true;
+        // after an early exit, copies still in flight land before shared memory is given back
+        if (tid == 256)
+            for (int j = landed; j < issued; ++j)
+                if (!tc05::mbar_wait_bounded(&raw_full[j & 1], uint32_t(j >> 1) & 1u, kPolls)) timeout = true;
+    } else if (warp == 12) {
+        // ================= MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = tc05::idesc_f16_f32(128, 64);
+            constexpr uint32_t idesc_pv = tc05::idesc_f16_f32(128, 128) | tc05::kIdescBMajorMN;
+            auto issue_pv = [&](int t) {
+                const uint32_t sb = tc05::smem_u32(sm + uint32_t(t & 1) * kStage);
+                const uint32_t ph = sb + OKH, pl = sb + OKL;     // P' over the dead C tiles
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc05::mma_f16(tmem + TO, tc05::desc_kmajor_sw128((part == 1 ? pl : ph) + uint32_t(ks) * 32u),
+                                      tc05::desc_mnmajor_sw128(sb + (part == 2 ? OVL : OVH) + uint32_t(ks) * 2048u,
+                                                               8192u, 1024u),
+                                      idesc_pv, t > 0 || part > 0 || ks > 0);
+                tc05::mma_commit(&pv_done[t & 1]);
+            };
+            int issued_pv = 0;
+            for (int t = 0; t < n_tiles && !timeout; ++t) {
+                const int st = t & 1;
+                if (!wait_or_abort(&full[st], uint32_t(t >> 1) & 1u, abort_flag)) { timeout = true; break; }
+                if (t >= 1 && !wait_or_abort(s_free, uint32_t(t - 1) & 1u, abort_flag)) { timeout = true; break; }
+                tc05::fence_after_sync();
+                const uint32_t sb = tc05::smem_u32(sm + uint32_t(st) * kStage);
+                // passes: q_hi C_hi, q_lo C_hi, q_hi C_lo -> S_mse; w_hi Sigma, w_lo Sigma -> S_qjl
+#pragma unroll
+                for (int pass = 0; pass < 5; ++pass) {
+                    const uint32_t A = tmem + (pass == 1 ? TQL : pass == 3 ? TWH : pass == 4 ? TWL : TQH);
+                    const uint32_t B = sb + (pass == 2 ? OKL : pass >= 3 ? OKS : OKH);
+                    const uint32_t D = tmem + (pass >= 3 ? TSQ : TSM);
+                    const bool first = pass == 0 || pass == 3;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc05::mma_f16_ts(D, A + uint32_t(ks) * 8u,
+                                         tc05::desc_kmajor_sw128(B + uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u),
+                                         idesc_qk, !first || ks > 0);
+                }
+                tc05::mma_commit(qk_full);
+                if (t >= 1) {
+                    if (!wait_or_abort(p_full, uint32_t(t - 1) & 1u, abort_flag)) { timeout = true; break; }
+                    tc05::fence_after_sync();
+                    issue_pv(t - 1);
+                    issued_pv = t;
+                }
+            }
+            if (!timeout) {
+                if (wait_or_abort(p_full, uint32_t(n_tiles - 1) & 1u, abort_flag)) {
+                    tc05::fence_after_sync();
+                    issue_pv(n_tiles - 1);
+                    issued_pv = n_tiles;
+                } else {
+                    timeout = true;
+                }
+            }
+            // everything this thread issued completes before TMEM is given back
+            if (issued_pv > 0 &&
+                !wait_or_abort(&pv_done[(issued_pv - 1) & 1], uint32_t((issued_pv - 1) >> 1) & 1u, abort_flag))
+                timeout = true;
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax: row r, keys [32 half, 32 half + 32) of each page
+        const float qs = qs_arr[r];
+        float m_run = -INFINITY, l_run = 0.f;                    // log2 units
+        // waits decided per warp, so the warp-wide TMEM accesses stay converged
+        auto wait_w = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(kFull, wait_or_abort(bar, parity, abort_flag));
+        };
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t & 1;
+            const int k0 = k_begin + t * kKeys;
+            // QK(t) done; the page's scales were published with its operand tiles
+            if (!wait_w(qk_full, uint32_t(t) & 1u) || !wait_w(&full[st], uint32_t(t >> 1) & 1u)) {
+                timeout = true;
+                break;
+            }
             tc05::fence_after_sync();
-            const int lim = min(k_end, vis_r) - k0;            // keys [0, lim) of the tile are visible
-            float lp[64];
+            const int lim = min(k_end, vis_r) - k0;            // keys [0, lim) of the page are visible
+            const float4 *mt = meta + st * 64;
+            float lp[32];
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
+                const int cc = c ^ half ^ 1;                    // the other half first, then this thread's
                 uint32_t ra[32], rb[32];
-                tc05::tmem_ld_32x32b_x32(t_smse + lrow + uint32_t(c * 32), ra);
-                tc05::tmem_ld_32x32b_x32(t_sqjl + lrow + uint32_t(c * 32), rb);
+                tc05::tmem_ld_32x32b_x32(tmem + lrow + TSM + uint32_t(cc * 32), ra);
+                tc05::tmem_ld_32x32b_x32(tmem + lrow + TSQ + uint32_t(cc * 32), rb);
                 tc05::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float4 mk = meta[c * 32 + e];
+                    const float4 mk = mt[cc * 32 + e];
                     float v = fmaf(mk.y, __uint_as_float(rb[e]), mk.x * __uint_as_float(ra[e]));
-                    if (c * 32 + e >= lim) v = -INFINITY;
-                    lp[c * 32 + e] = v;
+                    if (cc * 32 + e >= lim) v = -INFINITY;
+                    if (c == 1) lp[e] = v;
                     mx = fmaxf(mx, v);
                 }
             }
+            tc05::fence_before_sync();
+            tc05::mbar_arrive(s_free);                          // S may be overwritten by QK(t + 1)
             const float m_new = fmaxf(m_run, qs * mx);
             const bool grow = m_new > m_run && m_run != -INFINITY && t > 0;
             const float alpha = grow ? exp2f(m_run - m_new) : 1.f;
+            if (t > 0) {                                        // PV(t - 1) done: O stable, P free
+                if (!wait_w(&pv_done[(t - 1) & 1], uint32_t((t - 1) >> 1) & 1u)) {
+                    timeout = true;
+                    break;
+                }
+                tc05::fence_after_sync();
+            }
             if (__any_sync(kFull, grow)) {
-                // O rows scaled by alpha (1 for rows whose maximum did not grow)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {                   // this thread's 64 columns of O
                     uint32_t ro[32];
-                    tc05::tmem_ld_32x32b_x32(t_o + lrow + uint32_t(c * 32), ro);
+                    const uint32_t col = TO + uint32_t(half * 64 + c * 32);
+                    tc05::tmem_ld_32x32b_x32(tmem + lrow + col, ro);
                     tc05::tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-                    tc05::tmem_st_32x32b_x32(t_o + lrow + uint32_t(c * 32), ro);
+                    tc05::tmem_st_32x32b_x32(tmem + lrow + col, ro);
                 }
                 tc05::tmem_wait_st();
             }
@@ -418,87 +532,71 @@ __global__ void __launch_bounds__(256, 1) pf128_kernel(Pf128Args a) {
             m_run = m_new;
             float psum = 0.f;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t pw[4], pl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int k = c * 8 + 2 * e;
+                    const int k = c * 8 + 2 * e;                // within this half
                     float p0 = 0.f, p1 = 0.f;
                     if (m_run != -INFINITY) {
                         p0 = exp2f(fmaf(qs, lp[k], -m_run));
                         p1 = exp2f(fmaf(qs, lp[k + 1], -m_run));
                     }
                     psum += p0 + p1;
-                    const float q0 = p0 * meta[k].z, q1 = p1 * meta[k + 1].z;
+                    const float q0 = p0 * mt[half * 32 + k].z, q1 = p1 * mt[half * 32 + k + 1].z;
                     const __half2 h = __floats2half2_rn(q0, q1);
                     const float2 hf = __half22float2(h);
                     pw[e] = *reinterpret_cast<const uint32_t *>(&h);
                     pl[e] = h2u(q0 - hf.x, q1 - hf.y);
                 }
-                const uint32_t off = tc05::sw128_offset(uint32_t(r), uint32_t(c));
-                *reinterpret_cast<uint4 *>(sm + SP + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-                *reinterpret_cast<uint4 *>(sm + SKL + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+                const uint32_t off = tc05::sw128_offset(uint32_t(r), uint32_t(half * 4 + c));
+                uint8_t *sb = sm + uint32_t(st) * kStage;       // QK(t) has completed: C tiles are dead
+                *reinterpret_cast<uint4 *>(sb + OKH + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                *reinterpret_cast<uint4 *>(sb + OKL + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
             }
             l_run += psum;
             tc05::fence_proxy_async_smem();
+            tc05::fence_before_sync();
+            tc05::mbar_arrive(p_full);
         }
-        ph_qk ^= 1u;
-        tc05::fence_before_sync();
-        if (__syncthreads_or(timeout)) break;
-        if (tid == 0) {
-            tc05::fence_after_sync();
-            constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 128) | tc05::kIdescBMajorMN;
-            const uint32_t ph = tc05::smem_u32(sm + SP), pl = tc05::smem_u32(sm + SKL);
-            const uint32_t vh = tc05::smem_u32(sm + SV), vl = tc05::smem_u32(sm + SKH);
-            // P'_hi V_hi, P'_lo V_hi, P'_hi V_lo
-#pragma unroll
-            for (int part = 0; part < 3; ++part)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc05::mma_f16(t_o, tc05::desc_kmajor_sw128((part == 1 ? pl : ph) + uint32_t(ks) * 32u),
-                                  tc05::desc_mnmajor_sw128((part == 2 ? vl : vh) + uint32_t(ks) * 2048u, 8192u, 1024u),
-                                  idesc, t > 0 || part > 0 || ks > 0);
-            tc05::mma_commit(bar_pv);
-        }
-    }
-    // the last PV (or, after an early exit, whatever is in flight)
-    if (!tc05::mbar_wait_bounded(bar_pv, ph_pv, kPolls)) timeout = true;
-    tc05::fence_after_sync();
-    if (warp < 4) {
+        // ---- partial result of this split: this thread's 64 columns of O
+        if (!timeout && !wait_w(&pv_done[(n_tiles - 1) & 1], uint32_t((n_tiles - 1) >> 1) & 1u)) timeout = true;
+        tc05::fence_after_sync();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             uint32_t ro[32];
-            tc05::tmem_ld_32x32b_x32(t_o + lrow + uint32_t(c * 32), ro);
+            tc05::tmem_ld_32x32b_x32(tmem + lrow + TO + uint32_t(half * 64 + c * 32), ro);
             tc05::tmem_wait_ld();
             if (row_ok) {
-                float4 *dst = reinterpret_cast<float4 *>(a.part_o + pbase * 128 + c * 32);
+                float4 *dst = reinterpret_cast<float4 *>(a.part_o + pbase * 128 + half * 64 + c * 32);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     dst[e] = make_float4(__uint_as_float(ro[4 * e]), __uint_as_float(ro[4 * e + 1]),
                                          __uint_as_float(ro[4 * e + 2]), __uint_as_float(ro[4 * e + 3]));
             }
         }
-        if (row_ok) {
-            a.part_ml[pbase * 2] = m_run == -INFINITY ? -INFINITY : m_run * 0.6931471805599453f;
-            a.part_ml[pbase * 2 + 1] = l_run;
-        }
+        lsum[half * 128 + r] = l_run;                  // the two halves' sums meet after the barrier
+        if (half == 0 && row_ok) a.part_ml[pbase * 2] = m_run == -INFINITY ? -INFINITY : m_run * 0.6931471805599453f;
     }
     tc05::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp < 4 && row_ok) a.part_ml[pbase * 2 + 1] = lsum[r] + lsum[128 + r];
+    if (warp == 12) {
         tc05::fence_after_sync();
-        tc05::tmem_dealloc(tmem, 256);
+        tc05::tmem_dealloc(tmem, 512);
     }
-    if (timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
+    if (timeout || *abort_flag) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
 }
 
 template <int KB, int VB>
 int run(const Pf128Args &a, cudaStream_t st) {
     auto kern = pf128_kernel<KB, VB>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SM_TOTAL));
+    const uint32_t smem = smem_bytes(a.L.page_bytes);
+    if (smem > 232448u) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     const dim3 grid(unsigned((a.C + a.PT - 1) / a.PT), unsigned(a.L.H), unsigned(a.n_splits));
-    kern<<<grid, 256, SM_TOTAL, st>>>(a);
+    kern<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 

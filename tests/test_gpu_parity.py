@@ -211,6 +211,45 @@ def test_long_context_decode_and_prefill_sampled():
 
 
 # ---------------------------------------------------------------------------
+# tensor-core decode: every logit, output and lse on outlier-channel data
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kbits,vbits,B,Hq,H,L", [
+    (2, 4, 3, 32, 8, 3000),       # k3v4 preset, G = 4, ragged lengths
+    (4, 3, 2, 16, 2, 2500),       # G = 8
+    (2, 3, 2, 8, 4, 4100),        # G = 2
+])
+def test_decode_tensor_core_every_output(kbits, vbits, B, Hq, H, L):
+    d, P = 128, 64
+    seed = 60 + kbits * 10 + vbits
+    K = synth.outlier_normal((B * L, H, d), seed=seed, device=DEV)
+    V = synth.outlier_normal((B * L, H, d), seed=seed + 1, device=DEV)
+    cd = Codec(d, kbits, True, vbits, seed=seed, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    lens = [L - 37 * b for b in range(B)]
+    seq = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    Q = synth.normal((B, Hq, d), seed=seed + 2, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    lse = torch.empty((B, Hq), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, lse=lse, logits=logits)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b in range(B):
+        n = lens[b]
+        idx = np.arange(b * L, b * L + n)
+        for kvh in range(H):
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl[idx], f64(K[idx, kvh]), f64(V[idx, kvh]), kvh)
+            rows = list(range(kvh * G, kvh * G + G))
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
+            assert np.allclose(f64(lse[b, rows]), lse_ref, rtol=1e-3, atol=1e-3)
+
+
+# ---------------------------------------------------------------------------
 # tensor-core prefill: every output and lse, ragged query tiles, ragged last
 # page, several key splits, G = 1 .. 8
 # ---------------------------------------------------------------------------
