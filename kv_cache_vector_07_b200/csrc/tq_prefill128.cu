@@ -9,22 +9,26 @@
 // back by the combine kernel).  A block takes 128 query rows (positions x
 // GQA heads of one KV head) and walks one key split a page (64 keys) at a
 // time, with three warp roles synchronized by mbarriers:
-//   producers (warps 8-11)  dequantize page t into stage t % 2: centroids as
-//                fp16 hi + lo tiles, QJL signs as a +-1 tile, value
-//                centroids as fp16 hi + lo tiles (MN-major), per-key scales;
+//   producers (warps 8-11)  for page t: the key operands (centroids as fp16
+//                hi + lo tiles, QJL signs as a +-1 tile, per-key logit
+//                scales) into key stage t % 2 as soon as QK(t - 2) and its
+//                softmax read are done, then the value operands (centroids as
+//                fp16 hi + lo tiles, MN-major, and n_v) into value stage t % 2
+//                once PV(t - 2) is done; raw pages arrive by bulk copy ahead;
 //   MMA issuer (warp 12)    QK(t): S_mse = q_hi C_hi + q_lo C_hi + q_hi C_lo,
 //                S_qjl = w_hi Sigma + w_lo Sigma, with the query tiles as the
 //                A operand in tensor memory; then PV(t - 1):
 //                O += P_hi V_hi + P_lo V_hi + P_hi V_lo;
 //   softmax (warps 0-7)     two threads per row (TMEM lane), one per half of
-//                the page's keys: logits, causal mask, online max / sum (both
-//                threads of a row compute the page maximum from all 64
-//                columns, so they agree without exchanging), O rescaled in
-//                TMEM when the maximum grows, P' = p nhat_v as fp16 hi + lo.
-// QK(t + 1) runs while the softmax of page t works and the producers fill
-// page t + 2.  The hi/lo splits keep logits and outputs within tolerance
-// with outlier channels.  The split's partial (O, max, sum) goes to the
-// workspace in the layout the log-sum-exp combine kernel reads.
+//                the page's keys: read their half of S (releasing it to
+//                QK(t + 1)), logits, causal mask, the row maximum met through
+//                shared memory, online sum, O rescaled in TMEM when the
+//                maximum grows, P' = p nhat_v as fp16 hi + lo.
+// The tensor pipe alternates QK(t + 1) and PV(t) while the softmax of page t
+// and the producers of pages t + 1 / t + 2 run.  The hi/lo splits keep
+// logits and outputs within tolerance with outlier channels.  The split's
+// partial (O, max, sum) goes to the workspace in the layout the log-sum-exp
+// combine kernel reads.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -39,20 +43,31 @@ constexpr int kThreads = 416;           // 8 softmax + 4 producer warps + 1 MMA 
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 // shared layout (offsets from a 1024-aligned base)
-constexpr uint32_t kStage = 81920;                       // one page's operand tiles
-constexpr uint32_t OKH = 0, OKL = 16384, OKS = 32768;    // [64 keys x 128] K-major, halves at +8 KB
-constexpr uint32_t OVH = 49152, OVL = 65536;             // [64 keys x 128 dims] MN-major, halves at +8 KB
-// P' hi / lo [128 rows x 64 keys] K-major go over the stage's C_hi / C_lo
-// tiles, dead once QK of the page has completed
-constexpr uint32_t SKLUT = 2 * kStage;                   // K pair table, 8 KB
+constexpr uint32_t kKStage = 49152, kVStage = 32768;     // one page's key / value operand tiles
+constexpr uint32_t SK = 0;                               // [2] key stages: C_hi, C_lo, Sigma
+constexpr uint32_t OKH = 0, OKL = 16384, OKS = 32768;    //   [64 keys x 128] K-major, halves at +8 KB
+constexpr uint32_t SV = 2 * kKStage;                     // [2] value stages: V_hi, V_lo
+constexpr uint32_t OVH = 0, OVL = 16384;                 //   [64 keys x 128 dims] MN-major, halves at +8 KB
+constexpr uint32_t SPH = SV + 2 * kVStage, SPL = SPH + 16384;   // P' hi / lo [128 rows x 64 keys] K-major
+constexpr uint32_t SKLUT = SPL + 16384;                  // K pair table, 8 KB
 constexpr uint32_t SVLUT = SKLUT + 8192;                 // V pair table, 8 KB
-constexpr uint32_t SMETA = SVLUT + 8192;                 // float4 [2][64]: a, b, nhat_v, 0
-constexpr uint32_t SQS = SMETA + 2048;                   // float [128] query scales
+constexpr uint32_t SMK = SVLUT + 8192;                   // float2 [2][64]: logit scales a, b
+constexpr uint32_t SMV = SMK + 1024;                     // float [2][64]: nhat_v
+constexpr uint32_t SQS = SMV + 512;                      // float [128] query scales
 constexpr uint32_t SLSUM = SQS + 512;                    // float [2][128] per-half row sums
-constexpr uint32_t SFLAG = SLSUM + 1024;                 // abort flag
-constexpr uint32_t SBAR = SFLAG + 128;                   // mbarriers, page-valid flags
-constexpr uint32_t SRAW = SBAR + 256;                    // two raw pages (bulk copies), page_bytes each
-constexpr uint32_t smem_bytes(int page_bytes) { return SRAW + 2u * uint32_t((page_bytes + 127) & ~127) + 1024u; }
+constexpr uint32_t SXMAX = SLSUM + 1024;                 // float [2][2][128] half-row maxima
+constexpr uint32_t SFLAG = SXMAX + 2048;                 // abort flag
+constexpr uint32_t SBAR = SFLAG + 16;                    // 16 mbarriers, then 2 page-valid flags
+constexpr uint32_t SRAW = SBAR + 160;                    // raw pages (bulk copies)
+constexpr uint32_t kSmemMax = 232448;
+__host__ __device__ constexpr uint32_t raw_stride(int page_bytes) { return uint32_t((page_bytes + 127) & ~127); }
+// raw pages in flight: two when they fit, else one
+__host__ __device__ constexpr int raw_slots(int page_bytes) {
+    return SRAW + 2u * raw_stride(page_bytes) + 1024u <= kSmemMax ? 2 : 1;
+}
+__host__ __device__ constexpr uint32_t smem_bytes(int page_bytes) {
+    return SRAW + uint32_t(raw_slots(page_bytes)) * raw_stride(page_bytes) + 1024u;
+}
 
 // TMEM columns
 constexpr uint32_t TQH = 0, TQL = 64, TWH = 128, TWL = 192, TSM = 256, TSQ = 320, TO = 384;
@@ -130,14 +145,25 @@ __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Bounded wait that also gives up once another thread has given up.
+// Bounded wait that also gives up once another thread has given up: after a
+// few quick polls the thread naps between polls (so waiting warps leave the
+// issue slots to the working ones); about a second in all.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag) {
-    for (uint32_t i = 0; i < kPolls; ++i) {
+    for (uint32_t i = 0; i < 4u; ++i)
         if (tc05::mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 63u && *abort_flag) return false;
+    for (uint32_t i = 0; i < 4000000u; ++i) {
+        __nanosleep(64);
+        if (tc05::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
     }
     *abort_flag = 1u;
     return false;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 template <int KB, int VB>
@@ -148,21 +174,23 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint2 *lutk = reinterpret_cast<uint2 *>(sm + SKLUT);
     uint2 *lutv = reinterpret_cast<uint2 *>(sm + SVLUT);
-    float4 *meta = reinterpret_cast<float4 *>(sm + SMETA);
+    float2 *metak = reinterpret_cast<float2 *>(sm + SMK);
+    float *metav = reinterpret_cast<float *>(sm + SMV);
     float *qs_arr = reinterpret_cast<float *>(sm + SQS);
     float *lsum = reinterpret_cast<float *>(sm + SLSUM);
+    float *xmax = reinterpret_cast<float *>(sm + SXMAX);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + SFLAG);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
-    uint64_t *full = bars;          // [2] producers -> MMA (count 128)
-    uint64_t *pv_done = bars + 2;   // [2] PV of a stage's page completed (commit)
-    uint64_t *qk_full = bars + 4;   // QK completed (commit)
-    uint64_t *s_free = bars + 5;    // softmax read S (count 256)
-    uint64_t *p_full = bars + 6;    // softmax wrote P and rescaled O (count 256)
-    uint64_t *raw_full = bars + 7;  // [2] raw page landed (bulk copy, or plain arrive for a missing page)
-    uint64_t *raw_empty = bars + 9; // [2] producers finished reading a raw page (count 128)
+    uint64_t *kfull = bars;         // [2] key operands of a page written (count 128)
+    uint64_t *vfull = bars + 2;     // [2] value operands of a page written (count 128)
+    uint64_t *kfree = bars + 4;     // [2] QK of the page done (commit) and its S read (256): count 257
+    uint64_t *pv_done = bars + 6;   // [2] PV of the page done (commit)
+    uint64_t *qk_full = bars + 8;   // QK done (commit)
+    uint64_t *p_full = bars + 9;    // softmax wrote P and rescaled O (count 256)
+    uint64_t *raw_full = bars + 10; // [2] raw page landed (bulk copy, or plain arrive for a missing page)
+    uint64_t *raw_empty = bars + 12;// [2] producers finished reading a raw page (count 128)
+    uint64_t *xbar = bars + 14;     // [2] both halves of every row posted their maximum (count 256)
     int *pvalid = reinterpret_cast<int *>(sm + SBAR + 128);   // [2] raw page present
-    const uint32_t raw_stride = uint32_t((a.L.page_bytes + 127) & ~127);
-    uint8_t *raw = sm + SRAW;
 
     const Layout &L = a.L;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -173,6 +201,9 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
     const int vis_max = a.base_len + j_hi;                 // keys the tile's last row sees
     const int k_begin = split * a.split_len;
     const int k_end = min(k_begin + a.split_len, vis_max);
+    const uint32_t rstride = raw_stride(L.page_bytes);
+    const int n_raw = raw_slots(L.page_bytes);
+    uint8_t *raw = sm + SRAW;
     // softmax rows: warps w and w + 4 share lanes 32 (w % 4) ..
     const int r = (warp & 3) * 32 + lane;
     const int half = (warp >> 2) & 1;
@@ -211,17 +242,17 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
         tc05::tmem_alloc(&tmem_holder, 512);
         tc05::tmem_relinquish();
         if (lane == 0) {
-            tc05::mbar_init(&full[0], 128);
-            tc05::mbar_init(&full[1], 128);
-            tc05::mbar_init(&pv_done[0], 1);
-            tc05::mbar_init(&pv_done[1], 1);
+            for (int i = 0; i < 2; ++i) {
+                tc05::mbar_init(&kfull[i], 128);
+                tc05::mbar_init(&vfull[i], 128);
+                tc05::mbar_init(&kfree[i], 257);
+                tc05::mbar_init(&pv_done[i], 1);
+                tc05::mbar_init(&raw_full[i], 1);
+                tc05::mbar_init(&raw_empty[i], 128);
+                tc05::mbar_init(&xbar[i], 256);
+            }
             tc05::mbar_init(qk_full, 1);
-            tc05::mbar_init(s_free, 256);
             tc05::mbar_init(p_full, 256);
-            tc05::mbar_init(&raw_full[0], 1);
-            tc05::mbar_init(&raw_full[1], 1);
-            tc05::mbar_init(&raw_empty[0], 128);
-            tc05::mbar_init(&raw_empty[1], 128);
             *abort_flag = 0u;
             tc05::fence_mbar_init();
         }
@@ -285,20 +316,19 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
     bool timeout = false;
 
     if (warp >= 8 && warp < 12) {
-        // ================= producers: key kk (one per lane), dims [64 hh, 64 hh + 64);
-        // pages arrive by bulk copy two pages ahead into a raw ring
+        // ================= producers: key kk (one per lane), dims [64 hh, 64 hh + 64)
         const int t4 = tid - 256, kk = t4 & 63, hh = t4 >> 6;
         const uint2 *lk = lutk + (lane & (NCK - 1));
         const uint2 *lv = lutv + (lane & (NCV - 1));
         auto issue_raw = [&](int t) {                       // thread 256 only
-            const int rs = t & 1;
+            const int rs = t % n_raw;
             const int kp = k_begin + t * kKeys;
             int blk = -1;
             if (kp < k_end) blk = a.block_table[kp >> 6];
             if (blk >= 0 && blk < a.num_blocks) {
                 pvalid[rs] = 1;
                 tc05::mbar_expect_tx(&raw_full[rs], uint32_t(L.page_bytes));
-                tc05::bulk_g2s(raw + rs * raw_stride, a.cache + (int64_t(blk) * L.H + kvh) * int64_t(L.page_bytes),
+                tc05::bulk_g2s(raw + rs * rstride, a.cache + (int64_t(blk) * L.H + kvh) * int64_t(L.page_bytes),
                                uint32_t(L.page_bytes), &raw_full[rs]);
             } else {
                 if (kp < k_end) atomicOr(a.status, TQ_DEV_BLOCK_RANGE);
@@ -308,25 +338,24 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
         };
         int issued = 0, landed = 0;                          // thread 256: raw pages requested / seen landed
         if (tid == 256) {
-            issue_raw(0);
-            if (n_tiles > 1) issue_raw(1);
-            issued = min(2, n_tiles);
+            for (int j = 0; j < n_raw && j < n_tiles; ++j) issue_raw(j);
+            issued = min(n_raw, n_tiles);
         }
         for (int t = 0; t < n_tiles; ++t) {
             const int st = t & 1;
-            uint8_t *sb = sm + uint32_t(st) * kStage;
-            if (t >= 2 && !wait_or_abort(&pv_done[st], uint32_t((t - 2) >> 1) & 1u, abort_flag)) {
-                timeout = true;
-                break;
-            }
-            if (!wait_or_abort(&raw_full[st], uint32_t(t >> 1) & 1u, abort_flag)) {
-                timeout = true;
-                break;
-            }
+            const int rs = t % n_raw;
+            const uint32_t ruse = uint32_t(t / n_raw) & 1u;   // phase of this raw slot's use
+            if (!wait_or_abort(&raw_full[rs], ruse, abort_flag)) { timeout = true; break; }
             landed = t + 1;
             const int kidx = k_begin + t * kKeys + kk;
-            const uint8_t *page = (pvalid[st] && kidx < k_end) ? raw + st * raw_stride : nullptr;
+            const uint8_t *page = (pvalid[rs] && kidx < k_end) ? raw + rs * rstride : nullptr;
             const int pos = kk;
+            // -- key operands, once QK(t - 2) and the softmax's read of its S are done
+            if (t >= 2 && !wait_or_abort(&kfree[st], uint32_t((t - 2) >> 1) & 1u, abort_flag)) {
+                timeout = true;
+                break;
+            }
+            uint8_t *kb = sm + SK + uint32_t(st) * kKStage;
 #pragma unroll
             for (int sub = 0; sub < 2; ++sub) {
                 const int qq = 2 * hh + sub;
@@ -354,10 +383,32 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
-                    *reinterpret_cast<uint4 *>(sb + OKH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(sb + OKL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(sb + OKS + off) = make_uint4(x2[4 * c], x2[4 * c + 1], x2[4 * c + 2], x2[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(kb + OKH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(kb + OKL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(kb + OKS + off) = make_uint4(x2[4 * c], x2[4 * c + 1], x2[4 * c + 2], x2[4 * c + 3]);
                 }
+            }
+            if (hh == 0) {
+                float2 m2 = make_float2(0.f, 0.f);
+                if (page) {
+                    const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2));
+                    const float rk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2));
+                    m2 = make_float2(nk * sl, rk * cq * sl);
+                }
+                metak[st * 64 + kk] = m2;
+            }
+            tc05::fence_proxy_async_smem();
+            tc05::mbar_arrive(&kfull[st]);
+            // -- value operands, once PV(t - 2) is done
+            if (t >= 2 && !wait_or_abort(&pv_done[st], uint32_t((t - 2) >> 1) & 1u, abort_flag)) {
+                timeout = true;
+                break;
+            }
+            uint8_t *vb = sm + SV + uint32_t(st) * kVStage;
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                const int qq = 2 * hh + sub;
+                uint32_t x0[16], x1[16];
                 if (page) {
                     uint32_t lo[4], hi;
                     load_codes<VB>(page + L.vc_off, L.vc_bpt, page + L.vh_off, L.vh_bpt, pos, qq, lo, hi);
@@ -371,54 +422,45 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
 #pragma unroll
                     for (int p = 0; p < 16; ++p) x0[p] = x1[p] = 0u;
                 }
+                const uint32_t hoff = uint32_t(hh) * 8192u;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
-                    *reinterpret_cast<uint4 *>(sb + OVH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(sb + OVL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(vb + OVH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(vb + OVL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
                 }
             }
-            if (hh == 0) {
-                float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (page) {
-                    const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2));
-                    const float rk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2));
-                    const float nv = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.vn_off + pos * 2));
-                    m4 = make_float4(nk * sl, rk * cq * sl, nv, 0.f);
-                }
-                meta[st * 64 + kk] = m4;
-            }
-            tc05::mbar_arrive(&raw_empty[st]);                  // raw page read
+            if (hh == 0)
+                metav[st * 64 + kk] =
+                    page ? h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.vn_off + pos * 2)) : 0.f;
+            tc05::mbar_arrive(&raw_empty[rs]);                  // raw page read
             tc05::fence_proxy_async_smem();
-            tc05::mbar_arrive(&full[st]);
-            if (tid == 256 && t + 2 < n_tiles) {
+            tc05::mbar_arrive(&vfull[st]);
+            if (tid == 256 && t + n_raw < n_tiles) {
                 // the raw slot is refilled once every producer has read it
-                if (!wait_or_abort(&raw_empty[st], uint32_t(t >> 1) & 1u, abort_flag)) {
-                    timeout = true;
-                    break;
-                }
-                issue_raw(t + 2);
-                issued = t + 3;
+                if (!wait_or_abort(&raw_empty[rs], ruse, abort_flag)) { timeout = true; break; }
+                issue_raw(t + n_raw);
+                issued = t + n_raw + 1;
             }
         }
         // after an early exit, copies still in flight land before shared memory is given back
         if (tid == 256)
             for (int j = landed; j < issued; ++j)
-                if (!tc05::mbar_wait_bounded(&raw_full[j & 1], uint32_t(j >> 1) & 1u, kPolls)) timeout = true;
+                if (!tc05::mbar_wait_bounded(&raw_full[j % n_raw], uint32_t(j / n_raw) & 1u, kPolls)) timeout = true;
     } else if (warp == 12) {
         // ================= MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = tc05::idesc_f16_f32(128, 64);
             constexpr uint32_t idesc_pv = tc05::idesc_f16_f32(128, 128) | tc05::kIdescBMajorMN;
+            const uint32_t ph = tc05::smem_u32(sm + SPH), pl = tc05::smem_u32(sm + SPL);
             auto issue_pv = [&](int t) {
-                const uint32_t sb = tc05::smem_u32(sm + uint32_t(t & 1) * kStage);
-                const uint32_t ph = sb + OKH, pl = sb + OKL;     // P' over the dead C tiles
+                const uint32_t vb = tc05::smem_u32(sm + SV + uint32_t(t & 1) * kVStage);
 #pragma unroll
                 for (int part = 0; part < 3; ++part)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         tc05::mma_f16(tmem + TO, tc05::desc_kmajor_sw128((part == 1 ? pl : ph) + uint32_t(ks) * 32u),
-                                      tc05::desc_mnmajor_sw128(sb + (part == 2 ? OVL : OVH) + uint32_t(ks) * 2048u,
+                                      tc05::desc_mnmajor_sw128(vb + (part == 2 ? OVL : OVH) + uint32_t(ks) * 2048u,
                                                                8192u, 1024u),
                                       idesc_pv, t > 0 || part > 0 || ks > 0);
                 tc05::mma_commit(&pv_done[t & 1]);
@@ -426,15 +468,19 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
             int issued_pv = 0;
             for (int t = 0; t < n_tiles && !timeout; ++t) {
                 const int st = t & 1;
-                if (!wait_or_abort(&full[st], uint32_t(t >> 1) & 1u, abort_flag)) { timeout = true; break; }
-                if (t >= 1 && !wait_or_abort(s_free, uint32_t(t - 1) & 1u, abort_flag)) { timeout = true; break; }
+                if (!wait_or_abort(&kfull[st], uint32_t(t >> 1) & 1u, abort_flag)) { timeout = true; break; }
+                // S free: the softmax has read S(t - 1)
+                if (t >= 1 && !wait_or_abort(&kfree[(t - 1) & 1], uint32_t((t - 1) >> 1) & 1u, abort_flag)) {
+                    timeout = true;
+                    break;
+                }
                 tc05::fence_after_sync();
-                const uint32_t sb = tc05::smem_u32(sm + uint32_t(st) * kStage);
+                const uint32_t kb = tc05::smem_u32(sm + SK + uint32_t(st) * kKStage);
                 // passes: q_hi C_hi, q_lo C_hi, q_hi C_lo -> S_mse; w_hi Sigma, w_lo Sigma -> S_qjl
 #pragma unroll
                 for (int pass = 0; pass < 5; ++pass) {
                     const uint32_t A = tmem + (pass == 1 ? TQL : pass == 3 ? TWH : pass == 4 ? TWL : TQH);
-                    const uint32_t B = sb + (pass == 2 ? OKL : pass >= 3 ? OKS : OKH);
+                    const uint32_t B = kb + (pass == 2 ? OKL : pass >= 3 ? OKS : OKH);
                     const uint32_t D = tmem + (pass >= 3 ? TSQ : TSM);
                     const bool first = pass == 0 || pass == 3;
 #pragma unroll
@@ -444,17 +490,25 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
                                          idesc_qk, !first || ks > 0);
                 }
                 tc05::mma_commit(qk_full);
+                tc05::mma_commit(&kfree[st]);
                 if (t >= 1) {
-                    if (!wait_or_abort(p_full, uint32_t(t - 1) & 1u, abort_flag)) { timeout = true; break; }
+                    const int u = t - 1;
+                    if (!wait_or_abort(p_full, uint32_t(u) & 1u, abort_flag) ||
+                        !wait_or_abort(&vfull[u & 1], uint32_t(u >> 1) & 1u, abort_flag)) {
+                        timeout = true;
+                        break;
+                    }
                     tc05::fence_after_sync();
-                    issue_pv(t - 1);
+                    issue_pv(u);
                     issued_pv = t;
                 }
             }
             if (!timeout) {
-                if (wait_or_abort(p_full, uint32_t(n_tiles - 1) & 1u, abort_flag)) {
+                const int u = n_tiles - 1;
+                if (wait_or_abort(p_full, uint32_t(u) & 1u, abort_flag) &&
+                    wait_or_abort(&vfull[u & 1], uint32_t(u >> 1) & 1u, abort_flag)) {
                     tc05::fence_after_sync();
-                    issue_pv(n_tiles - 1);
+                    issue_pv(u);
                     issued_pv = n_tiles;
                 } else {
                     timeout = true;
@@ -477,44 +531,55 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
         for (int t = 0; t < n_tiles; ++t) {
             const int st = t & 1;
             const int k0 = k_begin + t * kKeys;
-            // QK(t) done; the page's scales were published with its operand tiles
-            if (!wait_w(qk_full, uint32_t(t) & 1u) || !wait_w(&full[st], uint32_t(t >> 1) & 1u)) {
+            // QK(t) done; its key scales were published with the key operands
+            if (!wait_w(qk_full, uint32_t(t) & 1u) || !wait_w(&kfull[st], uint32_t(t >> 1) & 1u)) {
                 timeout = true;
                 break;
             }
             tc05::fence_after_sync();
             const int lim = min(k_end, vis_r) - k0;            // keys [0, lim) of the page are visible
-            const float4 *mt = meta + st * 64;
+            // this thread's 32 columns of S, 16 at a time; then S (and the key
+            // scales) are released
             float lp[32];
             float mx = -INFINITY;
+            const bool all_visible = lim >= kKeys;
+            const float2 *mk = metak + st * 64 + half * 32;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const int cc = c ^ half ^ 1;                    // the other half first, then this thread's
-                uint32_t ra[32], rb[32];
-                tc05::tmem_ld_32x32b_x32(tmem + lrow + TSM + uint32_t(cc * 32), ra);
-                tc05::tmem_ld_32x32b_x32(tmem + lrow + TSQ + uint32_t(cc * 32), rb);
+                uint32_t ra[16], rb[16];
+                tc05::tmem_ld_32x32b_x16(tmem + lrow + TSM + uint32_t(half * 32 + c * 16), ra);
+                tc05::tmem_ld_32x32b_x16(tmem + lrow + TSQ + uint32_t(half * 32 + c * 16), rb);
                 tc05::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float4 mk = mt[cc * 32 + e];
-                    float v = fmaf(mk.y, __uint_as_float(rb[e]), mk.x * __uint_as_float(ra[e]));
-                    if (cc * 32 + e >= lim) v = -INFINITY;
-                    if (c == 1) lp[e] = v;
+                for (int e = 0; e < 16; ++e) {
+                    const float2 m2 = mk[c * 16 + e];
+                    float v = fmaf(m2.y, __uint_as_float(rb[e]), m2.x * __uint_as_float(ra[e]));
+                    if (!all_visible && half * 32 + c * 16 + e >= lim) v = -INFINITY;
+                    lp[c * 16 + e] = v;
                     mx = fmaxf(mx, v);
                 }
             }
             tc05::fence_before_sync();
-            tc05::mbar_arrive(s_free);                          // S may be overwritten by QK(t + 1)
+            tc05::mbar_arrive(&kfree[st]);
+            // the row maximum over both halves: post, meet, read the other half's
+            float *xm = xmax + st * 256;
+            xm[half * 128 + r] = mx;
+            tc05::mbar_arrive(&xbar[st]);
+            if (!wait_w(&xbar[st], uint32_t(t >> 1) & 1u)) {
+                timeout = true;
+                break;
+            }
+            mx = fmaxf(mx, xm[(half ^ 1) * 128 + r]);
             const float m_new = fmaxf(m_run, qs * mx);
             const bool grow = m_new > m_run && m_run != -INFINITY && t > 0;
             const float alpha = grow ? exp2f(m_run - m_new) : 1.f;
-            if (t > 0) {                                        // PV(t - 1) done: O stable, P free
-                if (!wait_w(&pv_done[(t - 1) & 1], uint32_t((t - 1) >> 1) & 1u)) {
-                    timeout = true;
-                    break;
-                }
-                tc05::fence_after_sync();
+            // PV(t - 1) done: P is free and O stable; then the page's n_v
+            if ((t > 0 && !wait_w(&pv_done[(t - 1) & 1], uint32_t((t - 1) >> 1) & 1u)) ||
+                !wait_w(&vfull[st], uint32_t(t >> 1) & 1u)) {
+                timeout = true;
+                break;
             }
+            tc05::fence_after_sync();
             if (__any_sync(kFull, grow)) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {                   // this thread's 64 columns of O
@@ -531,6 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
             l_run *= alpha;
             m_run = m_new;
             float psum = 0.f;
+            const float *nvp = metav + st * 64 + half * 32;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pw[4], pl[4];
@@ -539,20 +605,19 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
                     const int k = c * 8 + 2 * e;                // within this half
                     float p0 = 0.f, p1 = 0.f;
                     if (m_run != -INFINITY) {
-                        p0 = exp2f(fmaf(qs, lp[k], -m_run));
-                        p1 = exp2f(fmaf(qs, lp[k + 1], -m_run));
+                        p0 = ex2_approx(fmaf(qs, lp[k], -m_run));
+                        p1 = ex2_approx(fmaf(qs, lp[k + 1], -m_run));
                     }
                     psum += p0 + p1;
-                    const float q0 = p0 * mt[half * 32 + k].z, q1 = p1 * mt[half * 32 + k + 1].z;
+                    const float q0 = p0 * nvp[k], q1 = p1 * nvp[k + 1];
                     const __half2 h = __floats2half2_rn(q0, q1);
                     const float2 hf = __half22float2(h);
                     pw[e] = *reinterpret_cast<const uint32_t *>(&h);
                     pl[e] = h2u(q0 - hf.x, q1 - hf.y);
                 }
                 const uint32_t off = tc05::sw128_offset(uint32_t(r), uint32_t(half * 4 + c));
-                uint8_t *sb = sm + uint32_t(st) * kStage;       // QK(t) has completed: C tiles are dead
-                *reinterpret_cast<uint4 *>(sb + OKH + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-                *reinterpret_cast<uint4 *>(sb + OKL + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+                *reinterpret_cast<uint4 *>(sm + SPH + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                *reinterpret_cast<uint4 *>(sm + SPL + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
             }
             l_run += psum;
             tc05::fence_proxy_async_smem();
