@@ -356,36 +356,35 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
                 break;
             }
             uint8_t *kb = sm + SK + uint32_t(st) * kKStage;
-#pragma unroll
+#pragma unroll 1
             for (int sub = 0; sub < 2; ++sub) {
                 const int qq = 2 * hh + sub;
-                uint32_t x0[16], x1[16], x2[16];
+                uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi = 0u, sg = 0u;
                 if (page) {
-                    uint32_t lo[4], hi;
                     load_codes<KB>(page + L.kc_off, L.kc_bpt, page + L.kh_off, L.kh_bpt, pos, qq, lo, hi);
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) {
-                        const uint2 e = lk[pair_index<KB>(lo, hi, p) * NCK];
-                        x0[p] = e.x;
-                        x1[p] = e.y;
-                    }
-                    const uint32_t sg = *reinterpret_cast<const uint32_t *>(page + L.ks_off + pos * L.ks_bpt + qq * 4);
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) {
-                        const uint32_t b = sg >> (2 * p);      // bit 0: coordinate 2p, bit 1: 2p + 1
-                        x2[p] = 0xBC00BC00u ^ (((b << 15) & 0x8000u) | ((b << 30) & 0x80000000u));
-                    }
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) x0[p] = x1[p] = x2[p] = 0u;
+                    sg = *reinterpret_cast<const uint32_t *>(page + L.ks_off + pos * L.ks_bpt + qq * 4);
                 }
                 const uint32_t hoff = uint32_t(hh) * 8192u;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 4; ++c) {                   // 8 coordinates: one 16-byte chunk per tile
+                    uint32_t x0[4], x1[4], x2[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int p = 4 * c + q;
+                        if (page) {
+                            const uint2 e = lk[pair_index<KB>(lo, hi, p) * NCK];
+                            const uint32_t b = sg >> (2 * p);  // bit 0: coordinate 2p, bit 1: 2p + 1
+                            x0[q] = e.x;
+                            x1[q] = e.y;
+                            x2[q] = 0xBC00BC00u ^ (((b << 15) & 0x8000u) | ((b << 30) & 0x80000000u));
+                        } else {
+                            x0[q] = x1[q] = x2[q] = 0u;
+                        }
+                    }
                     const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
-                    *reinterpret_cast<uint4 *>(kb + OKH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(kb + OKL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(kb + OKS + off) = make_uint4(x2[4 * c], x2[4 * c + 1], x2[4 * c + 2], x2[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(kb + OKH + off) = make_uint4(x0[0], x0[1], x0[2], x0[3]);
+                    *reinterpret_cast<uint4 *>(kb + OKL + off) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
+                    *reinterpret_cast<uint4 *>(kb + OKS + off) = make_uint4(x2[0], x2[1], x2[2], x2[3]);
                 }
             }
             if (hh == 0) {
@@ -405,29 +404,28 @@ __global__ void __launch_bounds__(kThreads, 1) pf128_kernel(Pf128Args a) {
                 break;
             }
             uint8_t *vb = sm + SV + uint32_t(st) * kVStage;
-#pragma unroll
+#pragma unroll 1
             for (int sub = 0; sub < 2; ++sub) {
                 const int qq = 2 * hh + sub;
-                uint32_t x0[16], x1[16];
-                if (page) {
-                    uint32_t lo[4], hi;
-                    load_codes<VB>(page + L.vc_off, L.vc_bpt, page + L.vh_off, L.vh_bpt, pos, qq, lo, hi);
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) {
-                        const uint2 e = lv[pair_index<VB>(lo, hi, p) * NCV];
-                        x0[p] = e.x;
-                        x1[p] = e.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) x0[p] = x1[p] = 0u;
-                }
+                uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi = 0u;
+                if (page) load_codes<VB>(page + L.vc_off, L.vc_bpt, page + L.vh_off, L.vh_bpt, pos, qq, lo, hi);
                 const uint32_t hoff = uint32_t(hh) * 8192u;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    uint32_t x0[4], x1[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (page) {
+                            const uint2 e = lv[pair_index<VB>(lo, hi, 4 * c + q) * NCV];
+                            x0[q] = e.x;
+                            x1[q] = e.y;
+                        } else {
+                            x0[q] = x1[q] = 0u;
+                        }
+                    }
                     const uint32_t off = hoff + tc05::sw128_offset(uint32_t(kk), uint32_t(sub * 4 + c));
-                    *reinterpret_cast<uint4 *>(vb + OVH + off) = make_uint4(x0[4 * c], x0[4 * c + 1], x0[4 * c + 2], x0[4 * c + 3]);
-                    *reinterpret_cast<uint4 *>(vb + OVL + off) = make_uint4(x1[4 * c], x1[4 * c + 1], x1[4 * c + 2], x1[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(vb + OVH + off) = make_uint4(x0[0], x0[1], x0[2], x0[3]);
+                    *reinterpret_cast<uint4 *>(vb + OVL + off) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
                 }
             }
             if (hh == 0)
