@@ -84,6 +84,7 @@ extern "C" size_t tq_decode_workspace_bytes(const tq_cache_desc *desc, int B, in
     s.n_seq = B;
     s.Hq = Hq;
     s.max_len = max_seq_len;
+    s.is_decode = 1;
     return tq::attn_ws_bytes(L, s);
 }
 
@@ -113,6 +114,7 @@ extern "C" int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq
     s.bt_stride = max_blocks;
     s.max_blocks = max_blocks;
     s.seq_lens = seq_lens;
+    s.is_decode = 1;
     s.base_len = 0;
     s.max_len = max_seq_len;
     if (workspace_bytes < tq::attn_ws_bytes(L, s)) return TQ_EINVAL;

@@ -315,7 +315,28 @@ Plan make_plan(const Layout &L, const AttnShape &s) {
     int split_len = (maxlen + splits - 1) / splits;
     split_len = (split_len + kChunk - 1) / kChunk * kChunk;
     splits = (maxlen + split_len - 1) / split_len;
-    if (pf128_covers(L, s)) splits = pf128_splits(L, s, &split_len);
+    if (pf128_covers(L, s)) {
+        splits = pf128_splits(L, s, &split_len);
+    } else if (const int res = dec128_resident(L, p.G)) {
+        // tensor-core decode: whole waves of resident blocks, splits of at least 8 pages
+        const int64_t slots = int64_t(sms) * res;
+        const int max_sp = (maxlen + 511) / 512;
+        int best = 1;
+        double best_eff = 0.0;
+        for (int sp = 1; sp <= max_sp && sp <= 256; ++sp) {
+            const double waves = double(int64_t(p.n_groups) * sp) / double(slots);
+            const double eff = waves / double(int64_t(waves + 0.999999));
+            // prefer more blocks only while it buys efficiency or the first full wave
+            if (eff > best_eff + 0.02 || (best_eff < 0.5 && eff >= best_eff)) {
+                best_eff = eff;
+                best = sp;
+            }
+            if (waves >= 4.0) break;
+        }
+        split_len = (maxlen + best - 1) / best;
+        split_len = (split_len + kChunk - 1) / kChunk * kChunk;
+        splits = (maxlen + split_len - 1) / split_len;
+    }
     p.n_splits = splits;
     p.split_len = split_len;
     const int64_t rows = int64_t(s.n_seq) * s.Hq;

@@ -34,7 +34,7 @@ namespace tq {
 
 namespace {
 
-constexpr int kNS = 4;                  // page stages
+constexpr int kNS = 3;                  // page stages
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 struct Dec128Args {
@@ -83,9 +83,18 @@ __device__ __forceinline__ int visible(const Dec128Args &a, int b) {
     return a.seq_lens ? a.seq_lens[b] : a.base_len + b + 1;
 }
 
-// Table of fp16 pairs, replicated per lane: entry e for lane l at word
-// (e * 32 + l).  lookup(e) = half2(lv[e & mask], lv[e >> shift]).
-__device__ __forceinline__ uint32_t lut(const uint32_t *tab_lane, uint32_t e) { return tab_lane[e * 32]; }
+// Pair tables are replicated so that lanes spread over the banks: 16-entry
+// tables get 16 (key) / 32 (value) copies, 256-entry tables 8 copies (which
+// keeps four blocks' worth of shared memory per SM).  Lane l reads copy
+// l mod copies.
+template <int B>
+__host__ __device__ constexpr int key_copies() { return B == 4 ? 8 : 16; }
+template <int B>
+__host__ __device__ constexpr int val_copies() { return B == 4 ? 8 : 32; }
+
+// Value table entry e for this lane: half2(lv[e & mask], lv[e >> shift]).
+template <int VC>
+__device__ __forceinline__ uint32_t lut(const uint32_t *tab_lane, uint32_t e) { return tab_lane[e * VC]; }
 
 template <int KB, int VB, int NT>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
@@ -93,10 +102,11 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     static_assert(VB == 3 || VB == 4, "value bits");
     constexpr int KE = KB == 4 ? 256 : 16;          // key pair-table entries (two codes)
     constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
+    constexpr int KC = key_copies<KB>(), VC = val_copies<VB>();
     extern __shared__ __align__(16) uint8_t smem[];
-    uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][16 copies] {hi pair, lo pair}
-    uint32_t *lutV = reinterpret_cast<uint32_t *>(lutK + KE * 16);   // [VE][32 copies]
-    uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * 32);          // [NT][16][32]
+    uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][KC copies] {hi pair, lo pair}
+    uint32_t *lutV = reinterpret_cast<uint32_t *>(lutK + KE * KC);   // [VE][VC copies]
+    uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * VC);          // [NT][16][32]
     uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * 16 * 32);
     const Layout &L = a.L;
     const int pbytes = L.page_bytes;
@@ -119,17 +129,17 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     const int64_t row0 = int64_t(b) * a.Hq + int64_t(kvh) * G;
 
     // ---- tables: pair lookups (replicated per lane) and query fragments
-    for (int i = tid; i < KE * 16; i += 128) {
+    for (int i = tid; i < KE * KC; i += 128) {
         // centroid pair as fp16 hi + lo (the pair's fp32 values to ~22 bits)
-        const int e = i >> 4;
+        const int e = i / KC;
         float c0, c1;
         if (KB == 4) { c0 = a.k_lv[e & 15]; c1 = a.k_lv[e >> 4]; }
         else { c0 = a.k_lv[e & 3]; c1 = a.k_lv[(e >> 2) & 3]; }
         const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
         lutK[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
     }
-    for (int i = tid; i < VE * 32; i += 128) {
-        const int e = i >> 5;
+    for (int i = tid; i < VE * VC; i += 128) {
+        const int e = i / VC;
         float lo, hi;
         if (VB == 4) { lo = a.v_lv[e & 15]; hi = a.v_lv[e >> 4]; }
         else { lo = a.v_lv[e & 3]; hi = a.v_lv[(e >> 2) & 3]; }       // magnitudes (positive half)
@@ -191,8 +201,8 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     if (tid == 0)
         for (int i = 0; i < kNS - 1 && i < n_pages; ++i) issue_page(i);
 
-    const uint2 *lutK_l = lutK + (lane & 15);
-    const uint32_t *lutV_l = lutV + lane;
+    const uint2 *lutK_l = lutK + (lane & (KC - 1));
+    const uint32_t *lutV_l = lutV + (lane & (VC - 1));
     const float cq = 1.2533141373155003f / 128.0f;       // sqrt(pi/2) / m
     float m_run[NT], l_run[NT];
 #pragma unroll
@@ -261,7 +271,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     uint32_t Ah[4], Al[4];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
-                        const uint2 v = lutK_l[e[r] * 16];
+                        const uint2 v = lutK_l[e[r] * KC];
                         Ah[r] = v.x;
                         Al[r] = v.y;
                     }
@@ -372,10 +382,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                         for (int k = 0; k < 4; ++k) {
                             const int mt = 4 * wi + k;          // coordinates 16g + 2mt, +1
                             uint32_t A[4];
-                            A[0] = lut(lutV_l, (eAB >> (8 * k)) & 0xFF);
-                            A[1] = lut(lutV_l, (oAB >> (8 * k)) & 0xFF);
-                            A[2] = lut(lutV_l, (eCD >> (8 * k)) & 0xFF);
-                            A[3] = lut(lutV_l, (oCD >> (8 * k)) & 0xFF);
+                            A[0] = lut<VC>(lutV_l, (eAB >> (8 * k)) & 0xFF);
+                            A[1] = lut<VC>(lutV_l, (oAB >> (8 * k)) & 0xFF);
+                            A[2] = lut<VC>(lutV_l, (eCD >> (8 * k)) & 0xFF);
+                            A[3] = lut<VC>(lutV_l, (oCD >> (8 * k)) & 0xFF);
                             mma16816(O[mt], A, b0, b1);
                         }
                     }
@@ -399,10 +409,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     for (int mt = 0; mt < 8; ++mt) {
                         const int e0 = 2 * mt, e1 = 2 * mt + 1;     // coordinates 16g + e
                         uint32_t A[4];
-                        A[0] = lut(lutV_l, (eAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e0)) & 0x80008000u);
-                        A[1] = lut(lutV_l, (oAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e1)) & 0x80008000u);
-                        A[2] = lut(lutV_l, (eCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e0)) & 0x80008000u);
-                        A[3] = lut(lutV_l, (oCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e1)) & 0x80008000u);
+                        A[0] = lut<VC>(lutV_l, (eAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e0)) & 0x80008000u);
+                        A[1] = lut<VC>(lutV_l, (oAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e1)) & 0x80008000u);
+                        A[2] = lut<VC>(lutV_l, (eCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e0)) & 0x80008000u);
+                        A[3] = lut<VC>(lutV_l, (oCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e1)) & 0x80008000u);
                         mma16816(O[mt], A, b0, b1);
                     }
                 }
@@ -470,13 +480,26 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 }
 
 template <int KB, int VB, int NT>
-int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
+size_t dec_smem(int page_bytes) {
     constexpr int KE = KB == 4 ? 256 : 16, VE = VB == 4 ? 256 : 16;
     // the stage area also holds the final merge: 64 + 4 x 8 x 128 floats
-    size_t stages = size_t(kNS) * a.L.page_bytes;
+    size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
-    const size_t smem = size_t(KE) * 16 * 8 + size_t(VE) * 32 * 4 + size_t(NT) * 16 * 32 * 8 + stages +
-                        2 * kNS * 8 + kNS * 4 + 64;
+    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 + size_t(NT) * 16 * 32 * 8 +
+           stages + 2 * kNS * 8 + kNS * 4 + 64;
+}
+
+size_t dec_smem_for(const Layout &L, int G) {
+    const bool two = G > 4;
+    if (L.kbits == 2 && L.vbits == 4) return two ? dec_smem<2, 4, 2>(L.page_bytes) : dec_smem<2, 4, 1>(L.page_bytes);
+    if (L.kbits == 2 && L.vbits == 3) return two ? dec_smem<2, 3, 2>(L.page_bytes) : dec_smem<2, 3, 1>(L.page_bytes);
+    if (L.kbits == 4 && L.vbits == 4) return two ? dec_smem<4, 4, 2>(L.page_bytes) : dec_smem<4, 4, 1>(L.page_bytes);
+    return two ? dec_smem<4, 3, 2>(L.page_bytes) : dec_smem<4, 3, 1>(L.page_bytes);
+}
+
+template <int KB, int VB, int NT>
+int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
+    const size_t smem = dec_smem<KB, VB, NT>(a.L.page_bytes);
     auto kern = dec128_kernel<KB, VB, NT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
@@ -485,6 +508,18 @@ int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
 }
 
 }  // namespace
+
+// Blocks of the tensor-core decode kernel that fit on one SM (shared memory:
+// 228 KB per SM, 1 KB reserved per block; registers: at most 6 blocks for
+// one query-head tile, 4 for two), or 0 when the configuration is not covered.
+int dec128_resident(const Layout &L, int G) {
+    if (L.d != 128 || !L.kqjl || L.P != 64 || G > 8) return 0;
+    if (!((L.kbits == 2 || L.kbits == 4) && (L.vbits == 3 || L.vbits == 4))) return 0;
+    const size_t per = dec_smem_for(L, G) + 1024;
+    const int by_smem = int(233472 / per);
+    const int by_regs = G > 4 ? 4 : 6;
+    return by_smem < by_regs ? by_smem : by_regs;
+}
 
 // Tensor-core attention for d = 128; returns -1 when the configuration is not
 // covered (the caller then uses the general kernel).

@@ -121,12 +121,16 @@ struct AttnShape {
     const int32_t *seq_lens;   // decode: [B]; prefill: nullptr
     int base_len;         // prefill: seq_len - C (query j sees base_len + j + 1)
     int max_len;          // longest visible length
+    int is_decode;        // 1: decode (per-sequence lengths), 0: prefill chunk
 };
 size_t attn_ws_bytes(const Layout &L, const AttnShape &s);
 int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q,
                      const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out,
                      float *lse, float *logits, int64_t logits_stride, uint8_t *ws,
                      size_t ws_bytes, void *stream);
+
+// Blocks of the tensor-core decode kernel resident per SM (0: not covered).
+int dec128_resident(const Layout &L, int G);
 
 // Tensor-core attention for d = 128 (decode and prefill query groups);
 // returns -1 when the configuration is not covered.

@@ -666,7 +666,7 @@ int run(const Pf128Args &a, cudaStream_t st) {
 }  // namespace
 
 bool pf128_covers(const Layout &L, const AttnShape &s) {
-    if (L.d != 128 || L.P != kKeys || !L.kqjl || s.seq_lens != nullptr) return false;
+    if (L.d != 128 || L.P != kKeys || !L.kqjl || s.is_decode) return false;
     if (L.kbits < 2 || L.kbits > 4 || L.vbits < 2 || L.vbits > 4) return false;
     if (s.Hq % L.H) return false;
     const int G = s.Hq / L.H;
