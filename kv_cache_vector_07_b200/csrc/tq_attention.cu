@@ -52,6 +52,61 @@ __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
     }
 }
 
+// D = 128: q_r = R q and w = S q_r for 32 rows per block in one kernel: S
+// staged transposed in shared memory (fp32, 64 KB), the rotation by one warp
+// per row, the projection by thread (output j, 16 rows).
+constexpr int kPQRows = 32;
+constexpr size_t kPQSmem = sizeof(float) * (128 * 129 + kPQRows * 128);
+
+__global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
+    extern __shared__ float pq_smem[];
+    float *sT = pq_smem;                        // [k][j], row stride 129 (bank spread)
+    float *sq = pq_smem + 128 * 129;            // [32 rows][128]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t r0 = int64_t(blockIdx.x) * kPQRows;
+    for (int i = tid; i < 128 * 64; i += 256) {  // S[j][k] bf16 pairs -> sT[k][j]
+        const int j = i >> 6, k2 = (i & 63) * 2;
+        const uint32_t pr = *reinterpret_cast<const uint32_t *>(a.kp.S + size_t(j) * 128 + k2);
+        sT[k2 * 129 + j] = __uint_as_float(pr << 16);
+        sT[(k2 + 1) * 129 + j] = __uint_as_float(pr & 0xFFFF0000u);
+    }
+    float sg[4];
+    load_vec<128>(a.kp.signs, lane, sg);
+    for (int rr = warp; rr < kPQRows; rr += 8) {
+        const int64_t row = r0 + rr;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (row < a.rows) {
+            if (a.in_f32) load_vec<128>(reinterpret_cast<const float *>(a.Q) + row * 128, lane, x);
+            else load_vec<128>(reinterpret_cast<const __nv_bfloat16 *>(a.Q) + row * 128, lane, x);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] *= sg[e];
+        fwht_warp<128>(x, lane);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float v = x[e] * 0.08838834764831845f;
+            sq[rr * 128 + lane * 4 + e] = v;
+            if (row < a.rows) a.qr[row * 128 + lane * 4 + e] = v;
+        }
+    }
+    __syncthreads();
+    const int j = tid & 127, g = tid >> 7;      // output j, rows 16 g .. 16 g + 15
+    float acc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < 128; ++k) {
+        const float sv = sT[k * 129 + j];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = fmaf(sv, sq[(16 * g + r) * 128 + k], acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const int64_t row = r0 + 16 * g + r;
+        if (row < a.rows) a.w[row * 128 + j] = acc[r];
+    }
+}
+
 struct AttnArgs {
     Layout L;
     DevParams kp, vp;
@@ -254,7 +309,9 @@ struct CombineArgs {
     float *lse;         // optional [n_seq][Hq]
 };
 
-// One warp per (group, head): merge splits by log-sum-exp, rotate back.
+// One warp per (group, head): merge splits by log-sum-exp, rotate back.  The
+// split maxima and weights are reduced across lanes (lane s holds split s of a
+// 32-split chunk), so the partial-output loads of a chunk are independent.
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     constexpr int E = WarpVec<D>::E;
@@ -262,23 +319,36 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (r >= int64_t(a.n_groups) * a.G) return;
     const int g = int(r / a.G), h = int(r - int64_t(g) * a.G);
+    auto pb = [&](int s) { return (int64_t(g) * a.n_splits + s) * a.G + h; };
     float M = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, a.part_ml[((int64_t(g) * a.n_splits + s) * a.G + h) * 2]);
+    for (int s = lane; s < a.n_splits; s += 32) M = fmaxf(M, a.part_ml[pb(s) * 2]);
+    M = warp_max(M);
     float Lsum = 0.f;
     float o[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] = 0.f;
-    for (int s = 0; s < a.n_splits; ++s) {
-        const int64_t pb = (int64_t(g) * a.n_splits + s) * a.G + h;
-        const float m = a.part_ml[pb * 2];
-        if (m == -INFINITY) continue;
-        const float f = expf(m - M);
-        Lsum = fmaf(a.part_ml[pb * 2 + 1], f, Lsum);
-        if (lane < WarpVec<D>::LANES) {
+    for (int s0 = 0; s0 < a.n_splits; s0 += 32) {
+        const int s = s0 + lane;
+        float f = 0.f;
+        if (s < a.n_splits) {
+            const float m = a.part_ml[pb(s) * 2];
+            if (m != -INFINITY) {
+                f = expf(m - M);
+                Lsum = fmaf(a.part_ml[pb(s) * 2 + 1], f, Lsum);
+            }
+        }
+        const int n = min(32, a.n_splits - s0);
+        for (int i = 0; i < n; ++i) {
+            const float fi = __shfl_sync(kFull, f, i);
+            if (fi == 0.f) continue;
+            if (lane < WarpVec<D>::LANES) {
+                const float *src = a.part_o + pb(s0 + i) * D + lane * E;
 #pragma unroll
-            for (int e = 0; e < E; ++e) o[e] = fmaf(a.part_o[pb * D + lane * E + e], f, o[e]);
+                for (int e = 0; e < E; ++e) o[e] = fmaf(src[e], fi, o[e]);
+            }
         }
     }
+    Lsum = warp_sum(Lsum);
     const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] *= inv;
@@ -363,10 +433,17 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
     pa.kp = kp->dev;
     pa.qr = reinterpret_cast<float *>(ws + p.off_qr);
     pa.w = reinterpret_cast<float *>(ws + p.off_w);
-    prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
-    if (L.kqjl) {
-        const int e = launch_qproj(pa.qr, rows, D, kp->dev.S, pa.w, st);
+    if (D == 128 && L.kqjl) {
+        cudaError_t e = cudaFuncSetAttribute(prep_proj128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(kPQSmem));
         if (e != cudaSuccess) return e;
+        prep_proj128_kernel<<<unsigned((rows + kPQRows - 1) / kPQRows), 256, kPQSmem, st>>>(pa);
+    } else {
+        prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
+        if (L.kqjl) {
+            const int e = launch_qproj(pa.qr, rows, D, kp->dev.S, pa.w, st);
+            if (e != cudaSuccess) return e;
+        }
     }
 
     int fast;
