@@ -6,19 +6,23 @@
 // per-coordinate Lloyd-Max codes, no per-block scale) and "Stage 2" (1-bit
 // QJL projection of the residual); ai-work-lab overview, "QJL".
 //
-// Per tile of 128 vectors (one vector per TMEM lane / thread row):
+// Per tile of 128 vectors (one vector per TMEM lane):
 //   TMA     x tile [128 x 128 bf16] -> shared memory (128-byte swizzle)
 //   MMA 1   Y = X (H D)^T on tcgen05 (bf16, exact +-1 operand) -> TMEM;
 //           y = Y / sqrt(128) = R x
-//   threads (four per vector, 32 coordinates each) read Y from TMEM: norm,
-//           bucketize against the Lloyd-Max boundaries scaled by the norm,
-//           sign-magnitude codes packed into the page, fp16 norm; for QJL
-//           keys the residual r = y - nhat c[idx], rho = fp16 ||r||, and r
-//           (scaled by a power of two) split into fp16 hi + lo -> shared
-//   MMA 2   Z = (r_hi + r_lo) S^T on tcgen05 (fp16, S exact in fp16 except
-//           |S| < 2^-17) -> TMEM; the sign bits of Z go to the page.
-// Key and value tiles alternate so MMA 2 of a key tile overlaps the value
-// tile; MMA 1 of the next tile is issued before the current tile's epilogue.
+//   threads (two per vector, 64 coordinates each) read Y from TMEM: norm
+//           (each thread sums the whole row, so the pair agrees without
+//           exchanging), bucketize against the Lloyd-Max boundaries scaled by
+//           the norm, sign-magnitude codes packed into the page, fp16 norm; for
+//           QJL keys the residual r = y - nhat c[idx] (scaled by a power of
+//           two) split into fp16 hi + lo, written back over the tile's own Y
+//           columns, rho = fp16 ||r||
+//   MMA 2   Z = (r_hi + r_lo) S^T on tcgen05 with the residual as the A operand
+//           in tensor memory (fp16, S exact in fp16 except |S| < 2^-17); the
+//           sign bits of Z go to the page.
+// The block runs two independent groups of eight warps, each with its own
+// TMEM (Y, Z), x stage and named barrier, on alternate key/value tile pairs,
+// so one group's MMAs and loads overlap the other's arithmetic.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -35,9 +39,9 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr uint32_t kTile = 32768;          // one 128 x 128 16-bit tile
-constexpr uint32_t SM_ROT_K = 0, SM_ROT_V = 32768, SM_S16 = 65536, SM_X = 98304, SM_AHI = 163840,
-                   SM_ALO = 196608, SM_XCH = 229376;
-constexpr uint32_t SM_BAR = SM_XCH + 2048;
+constexpr uint32_t SM_ROT_K = 0, SM_ROT_V = 32768, SM_S16 = 65536, SM_X = 98304;   // x: one stage per group
+constexpr uint32_t SM_XR = SM_X + 2 * kTile;       // float [2 groups][2 halves][128] residual-norm partials
+constexpr uint32_t SM_BAR = SM_XR + 2048;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;        // barriers, TMEM address, level tables
 constexpr uint32_t kPolls = 1u << 20;    // about a second of polling, then give up
 
@@ -138,14 +142,17 @@ __device__ __forceinline__ uint8_t *row_page(const Enc128Args &a, int64_t v, int
     return a.cache + (int64_t(blk) * a.L.H + h) * int64_t(a.L.page_bytes);
 }
 
-// 16 warps: thread (row, q) owns vector row 32*(warp%4)+lane of the tile and
-// its coordinates [32q, 32q + 32), q = warp / 4 (TMEM lane slice warp % 4).
+// Two groups of 8 warps; in a group, thread (row, h) owns vector row
+// 32*(warp%4)+lane of the tile and its coordinates [64h, 64h + 64),
+// h = (warp%8)/4 (TMEM lane slice warp % 4).  Group g owns TMEM columns
+// [256g, 256g + 128) (Y, then the residual operand) and [256g + 128,
+// 256g + 256) (Z).
 template <int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(512, 1)
 encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Enc128Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = smem_raw;
-    float *xr = reinterpret_cast<float *>(sm + SM_XCH);              // [4][128] residual-norm partials
+    float *xr = reinterpret_cast<float *>(sm + SM_XR);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SM_BAR);
     uint64_t *bar_const = bars, *bar_x = bars + 1, *bar_y = bars + 3, *bar_z = bars + 5;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + SM_BAR + 64);
@@ -154,13 +161,16 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     constexpr bool DO_V = VB > 0;
     constexpr int PER = DO_V ? 2 : 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row = 32 * (warp & 3) + lane, q = warp >> 2;
+    const int grp = warp >> 3, gw = warp & 7, gtid = tid & 255;
+    const int row = 32 * (gw & 3) + lane, h = gw >> 2;
     if ((tc05::smem_u32(smem_raw) & 1023u) != 0) {       // the swizzled tiles need 1024-byte alignment
         if (tid == 0) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
         return;
     }
-    const int64_t n_pairs = a.n_tiles > blockIdx.x ? (a.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int64_t n_items = n_pairs * PER;
+    // tile pairs of this group: 2 blockIdx.x + grp + k * 2 gridDim.x
+    const int64_t first = 2 * int64_t(blockIdx.x) + grp, stride = 2 * int64_t(gridDim.x);
+    const int64_t n_my = a.n_tiles > first ? (a.n_tiles - 1 - first) / stride + 1 : 0;
+    const int64_t n_items = n_my * PER;
     bool timeout = false;
 
     if (warp == 0) {
@@ -171,53 +181,69 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         s_klv[tid] = (KB != 8 && tid < (1 << (KB == 8 ? 1 : KB))) ? a.k_lv[tid] : 0.f;
         s_vlv[tid] = (DO_V && tid < (1 << (VB > 0 ? VB : 1))) ? a.v_lv[tid] : 0.f;
     }
-    auto item_tile = [&](int64_t j) { return int64_t(blockIdx.x) + (j / PER) * int64_t(gridDim.x); };
+    auto item_tile = [&](int64_t j) { return first + (j / PER) * stride; };
     auto item_is_v = [&](int64_t j) { return DO_V && (j % PER) == 1; };
-    auto issue_x = [&](int64_t j) {
-        const int st = int(j & 1);
-        uint8_t *dst = sm + SM_X + st * kTile;
-        tc05::mbar_expect_tx(&bar_x[st], kTile);
+    uint8_t *xst = sm + SM_X + grp * kTile;
+    auto issue_x = [&](int64_t j) {                       // group issuer only
+        tc05::mbar_expect_tx(&bar_x[grp], kTile);
         const void *tm = item_is_v(j) ? static_cast<const void *>(&tmV) : static_cast<const void *>(&tmK);
         const int y = int(item_tile(j) * kRows);
-        tc05::tma_load_2d(dst, tm, 0, y, &bar_x[st]);
-        tc05::tma_load_2d(dst + 16384, tm, 64, y, &bar_x[st]);
+        tc05::tma_load_2d(xst, tm, 0, y, &bar_x[grp]);
+        tc05::tma_load_2d(xst + 16384, tm, 64, y, &bar_x[grp]);
     };
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) tc05::mbar_init(&bars[i], 1);
+        tc05::mbar_init(bar_const, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc05::mbar_init(&bar_x[i], 1);
+            tc05::mbar_init(&bar_y[i], 1);
+            tc05::mbar_init(&bar_z[i], 1);
+        }
         tc05::fence_mbar_init();
         tc05::mbar_expect_tx(bar_const, kTile * (1 + (DO_V ? 1 : 0) + (QJL ? 1 : 0)));
         tc05::bulk_g2s(sm + SM_ROT_K, a.k_rot, kTile, bar_const);
         if (DO_V) tc05::bulk_g2s(sm + SM_ROT_V, a.v_rot, kTile, bar_const);
         if (QJL) tc05::bulk_g2s(sm + SM_S16, a.s16, kTile, bar_const);
-        if (n_items > 0) issue_x(0);
-        if (n_items > 1) issue_x(1);
     }
     tc05::fence_before_sync();
     __syncthreads();
     tc05::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
-    const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+    const uint32_t ycol = tmem + uint32_t(grp * 256), zcol = ycol + 128u;
+    const uint32_t lane_base = uint32_t(32 * (gw & 3)) << 16;
     constexpr uint32_t idesc1 = tc05::idesc_bf16_f32(128, 128);
     constexpr uint32_t idesc2 = tc05::idesc_f16_f32(128, 128);
 
-    auto issue_mma1 = [&](int64_t j) {
-        const int st = int(j & 1);
-        if (!tc05::mbar_wait_bounded(&bar_x[st], uint32_t((j >> 1) & 1), kPolls)) timeout = true;
+    auto issue_mma1 = [&](int64_t j) {                    // group issuer only
+        if (!tc05::mbar_wait_bounded(&bar_x[grp], uint32_t(j & 1), kPolls)) timeout = true;
         tc05::fence_after_sync();
-        const uint32_t xa = tc05::smem_u32(sm + SM_X + st * kTile);
+        const uint32_t xa = tc05::smem_u32(xst);
         const uint32_t rb = tc05::smem_u32(sm + (item_is_v(j) ? SM_ROT_V : SM_ROT_K));
-        const uint32_t d = tmem + uint32_t(st * 128);
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc05::mma_bf16(d, tc05::desc_kmajor_sw128(xa + c * 16384 + ks * 32),
+                tc05::mma_bf16(ycol, tc05::desc_kmajor_sw128(xa + c * 16384 + ks * 32),
                                tc05::desc_kmajor_sw128(rb + c * 16384 + ks * 32), idesc1, (c | ks) != 0);
-        tc05::mma_commit(&bar_y[st]);
+        tc05::mma_commit(&bar_y[grp]);
     };
+    // Z = r S^T: k-step s reads the residual of quarter s / 2 (hi at +0, lo at
+    // +16 columns of the quarter, coordinates 16 (s % 2) .. at +8 (s % 2))
+    auto issue_mma2 = [&]() {                             // group issuer only
+        const uint32_t bs = tc05::smem_u32(sm + SM_S16);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int st = 0; st < 8; ++st)
+                tc05::mma_f16_ts(zcol, ycol + uint32_t(32 * (st >> 1) + 16 * part + 8 * (st & 1)),
+                                 tc05::desc_kmajor_sw128(bs + (st >> 2) * 16384 + (st & 3) * 32), idesc2,
+                                 (part | st) != 0);
+        tc05::mma_commit(&bar_z[grp]);
+    };
+    auto group_sync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(1 + grp) : "memory"); };
 
-    if (tid == 0 && n_items > 0) {
+    if (gtid == 0 && n_items > 0) {
         if (!tc05::mbar_wait_bounded(bar_const, 0, kPolls)) timeout = true;
+        issue_x(0);
         issue_mma1(0);
     }
 
@@ -226,154 +252,17 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     int64_t pending_k = -1;                             // key tile whose MMA 2 is in flight
     uint32_t z_phase = 0;
 
-    for (int64_t j = 0; j < n_items; ++j) {
-        const bool is_v = item_is_v(j);
-        const int64_t tile = item_tile(j);
-        const int yb = int(j & 1);
-        if (tid == 0 && j + 1 < n_items) issue_mma1(j + 1);
-        if (!tc05::mbar_wait_bounded(&bar_y[yb], uint32_t((j >> 1) & 1), kPolls)) timeout = true;
+    auto sign_pass = [&]() {
+        if (!tc05::mbar_wait_bounded(&bar_z[grp], z_phase, kPolls)) timeout = true;
+        z_phase ^= 1u;
         tc05::fence_after_sync();
-        // MMA 1 of this item has read its x stage: refill it
-        if (tid == 0 && j + 2 < n_items) issue_x(j + 2);
-
-        // this thread's quarter of Y, and ||Y||^2 summed over the four
-        // quarters in a fixed order, so the four threads of a row agree
-        float y[32];
-        {
+        int kpos = 0;
+        uint8_t *kpage = row_page(a, pending_k * kRows + row, &kpos);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int q = 2 * h + c;
             uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(tmem + lane_base + uint32_t(yb * 128 + q * 32), r);
-            tc05::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-        }
-        float part[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float ps = 0.f;
-            if (c == q) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) ps = fmaf(y[i], y[i], ps);
-            } else {
-                uint32_t r[32];
-                tc05::tmem_ld_32x32b_x32(tmem + lane_base + uint32_t(yb * 128 + c * 32), r);
-                tc05::tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) ps = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ps);
-            }
-            part[c] = ps;
-        }
-        const float ns = sqrtf(((part[0] + part[1]) + part[2]) + part[3]);   // ||Y|| = sqrt(128) ||x||
-        const float n = ns * rs;                                               // ||x||
-        const uint16_t nh = f2h_bits(n);
-        const float nhf = h2f_bits(nh);
-        int pos = 0;
-        uint8_t *page = row_page(a, tile * kRows + row, &pos);
-        const int bits = is_v ? VB : KB;
-        float rr = 0.f;
-
-        if (!is_v && KB == 8) {
-            // FP8 keys: e4m3(sqrt(d) y / n) = e4m3(Y / n)
-            const float inv = n > 0.f ? 1.0f / n : 0.f;
-            uint32_t w[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                uint32_t acc = 0;
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    acc |= uint32_t(__nv_cvt_float_to_fp8(y[4 * k + e] * inv, __NV_SATFINITE, __NV_E4M3)) << (8 * e);
-                w[k] = acc;
-            }
-            if (page) {
-                uint4 *dst = reinterpret_cast<uint4 *>(page + a.L.kc_off + pos * a.L.kc_bpt + q * 32);
-                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                if (q == 0) *reinterpret_cast<uint16_t *>(page + a.L.kn_off + pos * 2) = nh;
-            }
-        } else {
-            const int nt = (1 << (bits - 1)) - 1;
-            const float *bnd = is_v ? a.v_bnd : a.k_bnd;
-            float T[7];
-#pragma unroll
-            for (int k = 0; k < 7; ++k) T[k] = (k < nt && ns > 0.f) ? bnd[(1 << (bits - 1)) + k] * ns : FLT_MAX;
-            uint32_t cw[4];
-            if (is_v) {
-                if constexpr (DO_V) {
-                    quantize32<DO_V ? VB : 1, false>(y, T, s_vlv, 0.f, cw, rr);
-                    if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
-                                                            a.L.vh_bpt, cw);
-                }
-            } else {
-                constexpr int KQ = KB == 8 ? 1 : KB;
-                quantize32<KQ, QJL>(y, T, s_klv, sq * nhf, cw, rr);
-                if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
-            }
-            if (page && q == 0)
-                *reinterpret_cast<uint16_t *>(page + (is_v ? a.L.vn_off : a.L.kn_off) + pos * 2) = nh;
-        }
-
-        if (!is_v && QJL) {
-            // the residual (Y scale) times 2^(12 - e), ||Y|| < 2^(e + 1), so
-            // |.| < 2^14, split into fp16 hi + lo; the signs of S r do not
-            // depend on the positive scale
-            int e = 0;
-            if (ns > 0.f) e = ((__float_as_int(ns) >> 23) & 0xff) - 127;
-            const int ebits = min(254, max(1, 127 + 12 - e));
-            const float sc = __int_as_float(ebits << 23);
-            const int c = q >> 1;                          // 64-column half of the operand tile
-            uint8_t *ahi = sm + SM_AHI + c * 16384, *alo = sm + SM_ALO + c * 16384;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                uint32_t wh[4], wl[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float a0 = y[p * 8 + 2 * k] * sc, a1 = y[p * 8 + 2 * k + 1] * sc;
-                    const __half2 h = __floats2half2_rn(a0, a1);
-                    const float2 hf = __half22float2(h);
-                    const __half2 l = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
-                    wh[k] = *reinterpret_cast<const uint32_t *>(&h);
-                    wl[k] = *reinterpret_cast<const uint32_t *>(&l);
-                }
-                const uint32_t off = tc05::sw128_offset(uint32_t(row), uint32_t((q & 1) * 4 + p));
-                *reinterpret_cast<uint4 *>(ahi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                *reinterpret_cast<uint4 *>(alo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            }
-            xr[q * 128 + row] = rr;
-            tc05::fence_proxy_async_smem();
-            tc05::fence_before_sync();
-            __syncthreads();
-            if (tid == 0) {
-                tc05::fence_after_sync();
-                const uint32_t bh = tc05::smem_u32(sm + SM_AHI), bl = tc05::smem_u32(sm + SM_ALO);
-                const uint32_t bs = tc05::smem_u32(sm + SM_S16);
-                const uint32_t d = tmem + 256u;
-#pragma unroll
-                for (int sp = 0; sp < 2; ++sp)
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc05::mma_f16(d, tc05::desc_kmajor_sw128((sp ? bl : bh) + cc * 16384 + ks * 32),
-                                          tc05::desc_kmajor_sw128(bs + cc * 16384 + ks * 32), idesc2,
-                                          (sp | cc | ks) != 0);
-                tc05::mma_commit(bar_z);
-            }
-            if (page && q == 0) {
-                // rho = ||r|| = ||Y-scale residual|| / sqrt(128)
-                const float rho = sqrtf(((xr[row] + xr[128 + row]) + xr[256 + row]) + xr[384 + row]) * rs;
-                *reinterpret_cast<uint16_t *>(page + a.L.kr_off + pos * 2) = f2h_bits(rho);
-            }
-            pending_k = tile;
-        }
-
-        // sign bits of the key tile whose MMA 2 is in flight
-        if (QJL && pending_k >= 0 && (is_v || !DO_V)) {
-            if (!tc05::mbar_wait_bounded(bar_z, z_phase, kPolls)) timeout = true;
-            z_phase ^= 1u;
-            tc05::fence_after_sync();
-            int kpos = 0;
-            uint8_t *kpage = row_page(a, pending_k * kRows + row, &kpos);
-            uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(tmem + lane_base + uint32_t(256 + q * 32), r);
+            tc05::tmem_ld_32x32b_x32(zcol + lane_base + uint32_t(q * 32), r);
             tc05::tmem_wait_ld();
             // bit k = [z_k >= 0]: the complement of the float sign bit (z = -0.0
             // lies inside the zero-tolerance of the sign comparison)
@@ -382,10 +271,144 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             for (int k = 0; k < 32; ++k) neg |= (r[k] >> (31 - k)) & (1u << k);
             if (kpage && !timeout)
                 *reinterpret_cast<uint32_t *>(kpage + a.L.ks_off + kpos * a.L.ks_bpt + q * 4) = ~neg;
-            pending_k = -1;
         }
+        pending_k = -1;
+    };
+
+    for (int64_t j = 0; j < n_items; ++j) {
+        const bool is_v = item_is_v(j);
+        const int64_t tile = item_tile(j);
+        if (!tc05::mbar_wait_bounded(&bar_y[grp], uint32_t(j & 1), kPolls)) timeout = true;
+        tc05::fence_after_sync();
+        // MMA 1 of this item has read the group's x stage: refill it
+        if (gtid == 0 && j + 1 < n_items) issue_x(j + 1);
+
+        // ||Y||^2 over the whole row, quarters summed in a fixed order, so the
+        // two threads of a row agree
+        float part[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(c * 32), r);
+            tc05::tmem_wait_ld();
+            float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                p0 = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), p0);
+                p1 = fmaf(__uint_as_float(r[i + 1]), __uint_as_float(r[i + 1]), p1);
+            }
+            part[c] = p0 + p1;
+        }
+        const float ns = sqrtf(((part[0] + part[1]) + part[2]) + part[3]);   // ||Y|| = sqrt(128) ||x||
+        const float n = ns * rs;                                               // ||x||
+        const uint16_t nh = f2h_bits(n);
+        const float nhf = h2f_bits(nh);
+        int pos = 0;
+        uint8_t *page = row_page(a, tile * kRows + row, &pos);
+        const int bits = is_v ? VB : KB;
+        // residual scale 2^(12 - e), ||Y|| < 2^(e + 1): |r * scale| < 2^14
+        int e = 0;
+        if (ns > 0.f) e = ((__float_as_int(ns) >> 23) & 0xff) - 127;
+        const float sc = __int_as_float(min(254, max(1, 127 + 12 - e)) << 23);
+        float rr = 0.f;
+        float T[7];
+        {
+            const int nt = (1 << (bits - 1)) - 1;
+            const float *bnd = is_v ? a.v_bnd : a.k_bnd;
+#pragma unroll
+            for (int k = 0; k < 7; ++k)
+                T[k] = (k < nt && ns > 0.f && !(!is_v && KB == 8)) ? bnd[(1 << (bits - 1)) + k] * ns : FLT_MAX;
+        }
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+            const int q = 2 * h + c;
+            float y[32];
+            {
+                uint32_t r[32];
+                tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(q * 32), r);
+                tc05::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+            }
+            if (!is_v && KB == 8) {
+                // FP8 keys: e4m3(sqrt(d) y / n) = e4m3(Y / n)
+                const float inv = n > 0.f ? 1.0f / n : 0.f;
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2)
+                        acc |= uint32_t(__nv_cvt_float_to_fp8(y[4 * k + e2] * inv, __NV_SATFINITE, __NV_E4M3))
+                               << (8 * e2);
+                    w[k] = acc;
+                }
+                if (page) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(page + a.L.kc_off + pos * a.L.kc_bpt + q * 32);
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+            } else if (is_v) {
+                if constexpr (DO_V) {
+                    uint32_t cw[4];
+                    quantize32<DO_V ? VB : 1, false>(y, T, s_vlv, 0.f, cw, rr);
+                    if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
+                                                            a.L.vh_bpt, cw);
+                }
+            } else {
+                constexpr int KQ = KB == 8 ? 1 : KB;
+                uint32_t cw[4];
+                quantize32<KQ, QJL>(y, T, s_klv, sq * nhf, cw, rr);
+                if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
+                if constexpr (QJL) {
+                    // residual (Y scale) x 2^(12 - e) as fp16 hi + lo over this quarter's Y columns
+#pragma unroll
+                    for (int hf2 = 0; hf2 < 2; ++hf2) {
+                        uint32_t wh[8], wl[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float a0 = y[16 * hf2 + 2 * k] * sc, a1 = y[16 * hf2 + 2 * k + 1] * sc;
+                            const __half2 hh2 = __floats2half2_rn(a0, a1);
+                            const float2 hf = __half22float2(hh2);
+                            const __half2 ll2 = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
+                            wh[k] = *reinterpret_cast<const uint32_t *>(&hh2);
+                            wl[k] = *reinterpret_cast<const uint32_t *>(&ll2);
+                        }
+                        tc05::tmem_st_32x32b_x8(ycol + lane_base + uint32_t(q * 32 + 8 * hf2), wh);
+                        tc05::tmem_st_32x32b_x8(ycol + lane_base + uint32_t(q * 32 + 16 + 8 * hf2), wl);
+                    }
+                }
+            }
+        }
+        if (page && h == 0)
+            *reinterpret_cast<uint16_t *>(page + (is_v ? a.L.vn_off : a.L.kn_off) + pos * 2) = nh;
+        if (!is_v && QJL) {
+            tc05::tmem_wait_st();
+            xr[(grp * 2 + h) * 128 + row] = rr;
+        }
+        // sign bits of the key tile whose MMA 2 is in flight
+        if (QJL && DO_V && is_v && pending_k >= 0) sign_pass();
+
         tc05::fence_before_sync();
-        __syncthreads();
+        group_sync();                                   // Y read (and the residual written) by all
+        if (gtid == 0) {
+            tc05::fence_after_sync();
+            if (!is_v && QJL) issue_mma2();
+            if (j + 1 < n_items) {
+                // MMA 1 overwrites the residual MMA 2 reads
+                if (!is_v && QJL && !tc05::mbar_wait_bounded(&bar_z[grp], z_phase, kPolls)) timeout = true;
+                issue_mma1(j + 1);
+            }
+        }
+        if (!is_v && QJL) {
+            if (page && h == 0) {
+                // rho = ||r|| = ||Y-scale residual|| / sqrt(128)
+                const float rho = sqrtf(xr[(grp * 2) * 128 + row] + xr[(grp * 2 + 1) * 128 + row]) * rs;
+                *reinterpret_cast<uint16_t *>(page + a.L.kr_off + pos * 2) = f2h_bits(rho);
+            }
+            pending_k = tile;
+            if (!DO_V) sign_pass();
+        }
     }
 
     tc05::fence_before_sync();
@@ -430,7 +453,8 @@ int run(const CUtensorMap &mk, const CUtensorMap &mv, const Enc128Args &a, cudaS
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t grid = a.n_tiles < sms ? a.n_tiles : sms;
+    const int64_t want = (a.n_tiles + 1) / 2;          // two tile groups per block
+    const int64_t grid = want < sms ? want : sms;
     kern<<<unsigned(grid), 512, SM_TOTAL, st>>>(mk, mv, a);
     return cudaGetLastError();
 }
