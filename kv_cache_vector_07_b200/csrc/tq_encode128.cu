@@ -11,8 +11,10 @@
 //   MMA 1   Y = X (H D)^T on tcgen05 (bf16, exact +-1 operand) -> TMEM;
 //           y = Y / sqrt(128) = R x
 //   threads (two per vector, 64 coordinates each) read Y from TMEM: norm
-//           (each thread sums the whole row, so the pair agrees without
-//           exchanging), bucketize against the Lloyd-Max boundaries scaled by
+//           (each thread sums its own 64 coordinates by quarter; the pair
+//           swaps quarter sums through shared memory and adds all four in a
+//           fixed order, so both agree, and neither reads columns the other
+//           is about to overwrite with its residual), bucketize against the Lloyd-Max boundaries scaled by
 //           the norm, sign-magnitude codes packed into the page, fp16 norm; for
 //           QJL keys the residual r = y - nhat c[idx] (scaled by a power of
 //           two) split into fp16 hi + lo, written back over the tile's own Y
@@ -41,7 +43,8 @@ constexpr int kRows = 128;
 constexpr uint32_t kTile = 32768;          // one 128 x 128 16-bit tile
 constexpr uint32_t SM_ROT_K = 0, SM_ROT_V = 32768, SM_S16 = 65536, SM_X = 98304;   // x: one stage per group
 constexpr uint32_t SM_XR = SM_X + 2 * kTile;       // float [2 groups][2 halves][128] residual-norm partials
-constexpr uint32_t SM_BAR = SM_XR + 2048;
+constexpr uint32_t SM_YN = SM_XR + 2048;          // float [2 groups][4 quarters][128] ||Y||^2 partials
+constexpr uint32_t SM_BAR = SM_YN + 4096;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;        // barriers, TMEM address, level tables
 constexpr uint32_t kPolls = 1u << 20;    // about a second of polling, then give up
 
@@ -153,6 +156,7 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = smem_raw;
     float *xr = reinterpret_cast<float *>(sm + SM_XR);
+    float *yn = reinterpret_cast<float *>(sm + SM_YN);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SM_BAR);
     uint64_t *bar_const = bars, *bar_x = bars + 1, *bar_y = bars + 3, *bar_z = bars + 5;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + SM_BAR + 64);
@@ -283,13 +287,16 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         // MMA 1 of this item has read the group's x stage: refill it
         if (gtid == 0 && j + 1 < n_items) issue_x(j + 1);
 
-        // ||Y||^2 over the whole row, quarters summed in a fixed order, so the
-        // two threads of a row agree
-        float part[4];
+        // ||Y||^2 of the row: each thread sums its own two quarters (the
+        // partner overwrites its quarters with the residual as soon as it has
+        // its norm, so neither reads the other's columns); the quarter sums
+        // meet in shared memory and both threads add them in the same order
+        float *ynr = yn + grp * 512 + row;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+            const int q = 2 * h + c;
             uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(c * 32), r);
+            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(q * 32), r);
             tc05::tmem_wait_ld();
             float p0 = 0.f, p1 = 0.f;
 #pragma unroll
@@ -297,9 +304,11 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 p0 = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), p0);
                 p1 = fmaf(__uint_as_float(r[i + 1]), __uint_as_float(r[i + 1]), p1);
             }
-            part[c] = p0 + p1;
+            ynr[q * 128] = p0 + p1;
         }
-        const float ns = sqrtf(((part[0] + part[1]) + part[2]) + part[3]);   // ||Y|| = sqrt(128) ||x||
+        // warps gw and gw + 4 hold the two halves of the same 32 rows
+        asm volatile("bar.sync %0, 64;" ::"r"(3 + 4 * grp + (gw & 3)) : "memory");
+        const float ns = sqrtf(((ynr[0] + ynr[128]) + ynr[256]) + ynr[384]);   // ||Y|| = sqrt(128) ||x||
         const float n = ns * rs;                                               // ||x||
         const uint16_t nh = f2h_bits(n);
         const float nhf = h2f_bits(nh);
