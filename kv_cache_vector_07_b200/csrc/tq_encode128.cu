@@ -29,6 +29,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cfloat>
+#include <cstring>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -44,12 +45,25 @@ constexpr uint32_t kTile = 32768;          // one 128 x 128 16-bit tile
 constexpr uint32_t SM_ROT_K = 0, SM_ROT_V = 32768, SM_S16 = 65536, SM_X = 98304;   // x: one stage per group
 constexpr uint32_t SM_XR = SM_X + 2 * kTile;       // float [2 groups][2 halves][128] residual-norm partials
 constexpr uint32_t SM_YN = SM_XR + 2048;          // float [2 groups][4 quarters][128] ||Y||^2 partials
-constexpr uint32_t SM_BAR = SM_YN + 4096;
-constexpr uint32_t SM_TOTAL = SM_BAR + 256;        // barriers, TMEM address, level tables
+constexpr uint32_t SM_BAR = SM_YN + 4096;         // barriers, TMEM address, level tables
+constexpr uint32_t SM_TAB = SM_BAR + 256;          // magnitude-rank cell tables (keys, values)
+constexpr uint32_t SM_TOTAL = SM_TAB + 2 * 128;
+constexpr int kCells = 16;                         // cells of a rank table
 constexpr uint32_t kPolls = 1u << 20;    // about a second of polling, then give up
+
+// Magnitude-rank table of a 3- or 4-bit codebook.  With x = C |y| / ||y||
+// (C a power of two, so the scaled thresholds X_k = C t_k are exact) and the
+// unit cells [c, c + 1), c < 15, each cell holds at most one X_k: the rank
+// is mu_lo(c) + [x >= X in the cell], x clamped to 15, where no threshold
+// lies.  Entry c: {X in (c, c + 1) or a large value, mu_lo(c) = #{X_k <= c}}.
+struct RankTable {
+    float C;
+    float2 cell[kCells];
+};
 
 struct Enc128Args {
     Layout L;
+    RankTable k_tab, v_tab;
     const float *k_lv, *v_lv;          // levels by stored code
     const float *k_bnd, *v_bnd;        // ascending boundaries
     const uint8_t *k_rot, *v_rot, *s16;
@@ -88,16 +102,36 @@ __device__ __forceinline__ int mag_rank(float a, const float (&T)[7]) {
 // non-negative; a coordinate exactly on a boundary takes the upper magnitude
 // whatever its sign.  With RESID, y is overwritten by the residual in the Y
 // scale, Y - sqrt(128) nhat c[code], and rr receives its squared norm.
+//
+// For B >= 3 the rank comes from the cell table instead of the thresholds:
+// xs = C / ||Y|| (0 for a zero vector), tab = shared address of the table
+// minus (0x4B000000 << 3), so that the bits of 2^23 + floor(x), shifted by
+// three, index its 8-byte entries directly.
+template <int B>
+constexpr bool use_table() { return B == 3 || B == 4; }
+
 template <int B, bool RESID>
-__device__ __forceinline__ void quantize32(float (&y)[32], const float (&T)[7], const float *lvs, float nhs,
-                                           uint32_t (&cw)[4], float &rr) {
+__device__ __forceinline__ void quantize32(float (&y)[32], const float (&T)[7], float xs, uint32_t tab,
+                                           const float *lvs, float nhs, uint32_t (&cw)[4], float &rr) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) cw[k] = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const float Y = y[i];
-        const uint32_t s = Y < 0.f ? 1u : 0u;
-        const uint32_t kap = (s << (B - 1)) | uint32_t(mag_rank<B>(fabsf(Y), T));
+        uint32_t s, mu;
+        if constexpr (use_table<B>()) {
+            s = __float_as_uint(Y + 0.0f) >> 31;        // -0.0 + 0.0 = +0.0: zero is non-negative
+            const float x = fabsf(Y) * xs;
+            const uint32_t off = __float_as_uint(__fadd_rz(fminf(x, float(kCells - 1)), 8388608.0f)) << 3;
+            float tb;
+            uint32_t mlo;
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(tb), "=r"(mlo) : "r"(tab + off));
+            mu = mlo + (x >= tb ? 1u : 0u);
+        } else {
+            s = Y < 0.f ? 1u : 0u;
+            mu = uint32_t(mag_rank<B>(fabsf(Y), T));
+        }
+        const uint32_t kap = (s << (B - 1)) | mu;
         if constexpr (B == 3) {
             cw[i >> 4] |= (kap & 3u) << (2 * (i & 15));
             cw[2] |= (kap >> 2) << i;
@@ -152,7 +186,8 @@ __device__ __forceinline__ uint8_t *row_page(const Enc128Args &a, int64_t v, int
 // 256g + 256) (Z).
 template <int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(512, 1)
-encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Enc128Args a) {
+encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ Enc128Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = smem_raw;
     float *xr = reinterpret_cast<float *>(sm + SM_XR);
@@ -184,6 +219,9 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (tid < 16) {
         s_klv[tid] = (KB != 8 && tid < (1 << (KB == 8 ? 1 : KB))) ? a.k_lv[tid] : 0.f;
         s_vlv[tid] = (DO_V && tid < (1 << (VB > 0 ? VB : 1))) ? a.v_lv[tid] : 0.f;
+    } else if (tid < 16 + 2 * kCells) {
+        const int t = (tid - 16) / kCells, c = (tid - 16) % kCells;
+        reinterpret_cast<float2 *>(sm + SM_TAB)[t * kCells + c] = (t == 0 ? a.k_tab : a.v_tab).cell[c];
     }
     auto item_tile = [&](int64_t j) { return first + (j / PER) * stride; };
     auto item_is_v = [&](int64_t j) { return DO_V && (j % PER) == 1; };
@@ -270,9 +308,9 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             tc05::tmem_wait_ld();
             // bit k = [z_k >= 0]: the complement of the float sign bit (z = -0.0
             // lies inside the zero-tolerance of the sign comparison)
-            uint32_t neg = 0;
+            uint32_t neg = 0;                           // sign bits, coordinate k at bit k
 #pragma unroll
-            for (int k = 0; k < 32; ++k) neg |= (r[k] >> (31 - k)) & (1u << k);
+            for (int k = 31; k >= 0; --k) neg = __funnelshift_l(r[k], neg, 1);
             if (kpage && !timeout)
                 *reinterpret_cast<uint32_t *>(kpage + a.L.ks_off + kpos * a.L.ks_bpt + q * 4) = ~neg;
         }
@@ -321,13 +359,15 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const float sc = __int_as_float(min(254, max(1, 127 + 12 - e)) << 23);
         float rr = 0.f;
         float T[7];
-        {
+        if (!(is_v ? use_table<VB>() : use_table<KB>())) {
             const int nt = (1 << (bits - 1)) - 1;
             const float *bnd = is_v ? a.v_bnd : a.k_bnd;
 #pragma unroll
             for (int k = 0; k < 7; ++k)
                 T[k] = (k < nt && ns > 0.f && !(!is_v && KB == 8)) ? bnd[(1 << (bits - 1)) + k] * ns : FLT_MAX;
         }
+        const float xs = ns > 0.f ? (is_v ? a.v_tab.C : a.k_tab.C) / ns : 0.f;
+        const uint32_t tab = tc05::smem_u32(sm + SM_TAB + (is_v ? kCells * 8 : 0)) - (0x4B000000u << 3);
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
             const int q = 2 * h + c;
@@ -360,14 +400,14 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             } else if (is_v) {
                 if constexpr (DO_V) {
                     uint32_t cw[4];
-                    quantize32<DO_V ? VB : 1, false>(y, T, s_vlv, 0.f, cw, rr);
+                    quantize32<DO_V ? VB : 1, false>(y, T, xs, tab, s_vlv, 0.f, cw, rr);
                     if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
                                                             a.L.vh_bpt, cw);
                 }
             } else {
                 constexpr int KQ = KB == 8 ? 1 : KB;
                 uint32_t cw[4];
-                quantize32<KQ, QJL>(y, T, s_klv, sq * nhf, cw, rr);
+                quantize32<KQ, QJL>(y, T, xs, tab, s_klv, sq * nhf, cw, rr);
                 if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
                 if constexpr (QJL) {
                     // residual (Y scale) x 2^(12 - e) as fp16 hi + lo over this quarter's Y columns
@@ -468,6 +508,37 @@ int run(const CUtensorMap &mk, const CUtensorMap &mv, const Enc128Args &a, cudaS
     return cudaGetLastError();
 }
 
+// Rank table of a 3- or 4-bit codebook (see RankTable); false if no power of
+// two puts the largest threshold below the last cell with every gap between
+// scaled thresholds at least one cell wide.
+bool make_rank_table(const tq_params *p, RankTable *t) {
+    *t = RankTable{};
+    if (!p || (p->bits != 3 && p->bits != 4)) return true;
+    const int L = 1 << p->bits, nt = L / 2 - 1;
+    const float *th = p->h_bounds + L / 2;         // positive thresholds, ascending
+    if (!(th[0] > 0.f)) return false;
+    float C = 1.f;
+    for (int i = 0; i < 40 && C * th[nt - 1] >= float(kCells - 1); ++i) C *= 0.5f;
+    for (int i = 0; i < 40 && 2.f * C * th[nt - 1] < float(kCells - 1); ++i) C *= 2.f;
+    if (!(C * th[nt - 1] < float(kCells - 1))) return false;
+    for (int k = 0; k + 1 < nt; ++k)
+        if (double(C * th[k + 1]) - double(C * th[k]) < 1.0) return false;
+    t->C = C;
+    for (int c = 0; c < kCells; ++c) {
+        int mlo = 0;
+        float tb = 3.0e38f;
+        for (int k = 0; k < nt; ++k) {
+            const float X = C * th[k];
+            if (X <= float(c)) ++mlo;
+            else if (X < float(c + 1)) tb = X;
+        }
+        float mlo_bits;
+        std::memcpy(&mlo_bits, &mlo, sizeof mlo_bits);   // the rank rides in the float's bits
+        t->cell[c] = make_float2(tb, mlo_bits);
+    }
+    return true;
+}
+
 }  // namespace
 
 // Returns -1 if this configuration is not handled by the fused kernel.
@@ -486,6 +557,7 @@ int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, 
     a.v_lv = vp ? vp->dev.lv : nullptr;
     a.v_bnd = vp ? vp->dev.bounds : nullptr;
     a.v_rot = vp ? vp->dev.rot_img : nullptr;
+    if (!make_rank_table(kp, &a.k_tab) || !make_rank_table(vb > 0 ? vp : nullptr, &a.v_tab)) return -1;
     a.n_vec = n_tokens * L.H;
     a.n_tiles = (a.n_vec + kRows - 1) / kRows;
     a.slots = slots;
