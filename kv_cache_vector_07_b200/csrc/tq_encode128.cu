@@ -294,12 +294,11 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     int64_t pending_k = -1;                             // key tile whose MMA 2 is in flight
     uint32_t z_phase = 0;
 
-    auto sign_pass = [&]() {
+    // the pending key tile is the current tile: its page is this item's
+    auto sign_pass = [&](uint8_t *kpage, int kpos) {
         if (!tc05::mbar_wait_bounded(&bar_z[grp], z_phase, kPolls)) timeout = true;
         z_phase ^= 1u;
         tc05::fence_after_sync();
-        int kpos = 0;
-        uint8_t *kpage = row_page(a, pending_k * kRows + row, &kpos);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const int q = 2 * h + c;
@@ -317,9 +316,14 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         pending_k = -1;
     };
 
+    uint8_t *page = nullptr;
+    int pos = 0;
     for (int64_t j = 0; j < n_items; ++j) {
         const bool is_v = item_is_v(j);
         const int64_t tile = item_tile(j);
+        // a tile's key item finds the row's page (its value item and sign
+        // pass reuse it); the slot load overlaps the wait for Y
+        if (!is_v) page = row_page(a, tile * kRows + row, &pos);
         if (!tc05::mbar_wait_bounded(&bar_y[grp], uint32_t(j & 1), kPolls)) timeout = true;
         tc05::fence_after_sync();
         // MMA 1 of this item has read the group's x stage: refill it
@@ -330,19 +334,24 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         // its norm, so neither reads the other's columns); the quarter sums
         // meet in shared memory and both threads add them in the same order
         float *ynr = yn + grp * 512 + row;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int q = 2 * h + c;
-            uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(q * 32), r);
+        float y[32];                                    // the quarter being quantized: 2h first
+        {
+            uint32_t r0[32], r1[32];
+            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(2 * h * 32), r0);
+            tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(2 * h * 32 + 32), r1);
             tc05::tmem_wait_ld();
-            float p0 = 0.f, p1 = 0.f;
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                p0 = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), p0);
-                p1 = fmaf(__uint_as_float(r[i + 1]), __uint_as_float(r[i + 1]), p1);
+                p0 = fmaf(__uint_as_float(r0[i]), __uint_as_float(r0[i]), p0);
+                p1 = fmaf(__uint_as_float(r0[i + 1]), __uint_as_float(r0[i + 1]), p1);
+                p2 = fmaf(__uint_as_float(r1[i]), __uint_as_float(r1[i]), p2);
+                p3 = fmaf(__uint_as_float(r1[i + 1]), __uint_as_float(r1[i + 1]), p3);
             }
-            ynr[q * 128] = p0 + p1;
+            ynr[2 * h * 128] = p0 + p1;
+            ynr[(2 * h + 1) * 128] = p2 + p3;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r0[i]);
         }
         // warps gw and gw + 4 hold the two halves of the same 32 rows
         asm volatile("bar.sync %0, 64;" ::"r"(3 + 4 * grp + (gw & 3)) : "memory");
@@ -350,8 +359,6 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const float n = ns * rs;                                               // ||x||
         const uint16_t nh = f2h_bits(n);
         const float nhf = h2f_bits(nh);
-        int pos = 0;
-        uint8_t *page = row_page(a, tile * kRows + row, &pos);
         const int bits = is_v ? VB : KB;
         // residual scale 2^(12 - e), ||Y|| < 2^(e + 1): |r * scale| < 2^14
         int e = 0;
@@ -371,8 +378,7 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
             const int q = 2 * h + c;
-            float y[32];
-            {
+            if (c == 1) {                               // quarter 2h + 1, still unwritten by anyone
                 uint32_t r[32];
                 tc05::tmem_ld_32x32b_x32(ycol + lane_base + uint32_t(q * 32), r);
                 tc05::tmem_wait_ld();
@@ -436,7 +442,7 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             xr[(grp * 2 + h) * 128 + row] = rr;
         }
         // sign bits of the key tile whose MMA 2 is in flight
-        if (QJL && DO_V && is_v && pending_k >= 0) sign_pass();
+        if (QJL && DO_V && is_v && pending_k >= 0) sign_pass(page, pos);
 
         tc05::fence_before_sync();
         group_sync();                                   // Y read (and the residual written) by all
@@ -456,7 +462,7 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 *reinterpret_cast<uint16_t *>(page + a.L.kr_off + pos * 2) = f2h_bits(rho);
             }
             pending_k = tile;
-            if (!DO_V) sign_pass();
+            if (!DO_V) sign_pass(page, pos);
         }
     }
 
