@@ -6,16 +6,19 @@
 // Estimate of <q, x_t>:
 //   nhat_t <Rq, c[code_t]> + rho_t sqrt(pi/2)/m <S R q, 2 s_t - 1>.
 //
-// As a GEMM: D[128 queries x 512 vectors] = Qf[128 x 2d] Xf[512 x 2d]^T on
-// tcgen05 (fp16 operands, fp32 accumulator in TMEM, all 512 columns):
+// As a GEMM: D[256 queries x 256 vectors] = Qf[256 x 2d] Xf[256 x 2d]^T on
+// tcgen05 as two M = 128 products sharing each dequantized chunk of Xf
+// (fp16 operands, fp32 accumulators in TMEM, 256 columns per query half,
+// all 512 columns):
 //   Qf = 2^-e [R q | S R q] per query (fp16, prepared once, TMA-loaded one
 //        64-feature chunk at a time; e makes the largest feature 1 <= |f| < 2
 //        and the scores are multiplied back by 2^e);
 //   Xf = [nhat c[code] | rho sqrt(pi/2)/m (2 s - 1)] per database vector,
-//        dequantized by the block's threads into shared memory (128-byte
-//        swizzled K-major tiles) while the previous chunk's MMAs run.
-// Epilogue: thread (query, half) reads its 256 estimates from TMEM and keeps
-// a running top-k (ties to the lower index); a merge kernel combines the
+//        dequantized by the block's threads (one database row each) into
+//        shared memory (128-byte swizzled K-major tiles) while the previous
+//        chunk's MMAs run.
+// Epilogue: thread q reads its query's 256 estimates from TMEM and keeps a
+// running top-k (ties to the lower index); a merge kernel combines the
 // blocks' lists.
 //
 // Inside every 32-coordinate group the QJL features are in the order
@@ -32,17 +35,17 @@
 namespace tq {
 namespace {
 
-constexpr int kQ = 128;                 // queries per block (MMA M, TMEM lanes)
-constexpr int kN = 512;                 // database vectors per tile (two MMAs of N = 256)
+constexpr int kQ = 256;                 // queries per block (two MMAs of M = 128, TMEM lanes)
+constexpr int kN = 256;                 // database vectors per tile (MMA N)
 constexpr int kThreads = 256;
 constexpr int kTopK = 16;               // largest k this path takes
 constexpr int kSMs = 148;               // grid sizing (fixed, so workspace sizes do not depend on the device)
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 // shared layout (offsets from a 1024-aligned base)
-constexpr uint32_t SA = 0;                       // 2 stages x [128 x 64] fp16 (16 KB each)
-constexpr uint32_t SB = 32768;                   // 2 stages x 2 halves x [256 x 64] fp16 (64 KB per stage)
-constexpr uint32_t SLUT = SB + 131072;           // [256 code bytes][32 lane copies] half2 (32 KB)
+constexpr uint32_t SA = 0;                       // 2 stages x [256 x 64] fp16 (32 KB each)
+constexpr uint32_t SB = 65536;                   // 2 stages x [256 x 64] fp16 (32 KB each)
+constexpr uint32_t SLUT = SB + 65536;            // [256 code bytes][32 lane copies] half2 (32 KB)
 constexpr uint32_t STOPV = SLUT + 32768;         // [256 threads][k] scores
 constexpr uint32_t STOPI = STOPV + kThreads * kTopK * 4;   // [256 threads][k] indices (n_db < 2^31)
 constexpr uint32_t SBAR = STOPI + kThreads * kTopK * 4;
@@ -55,7 +58,7 @@ struct SearchTcArgs {
     const uint8_t *db;
     int64_t n_db;
     int n_q, k;
-    int64_t n_tiles;               // ceil(n_db / 512)
+    int64_t n_tiles;               // ceil(n_db / 256)
     int n_groups;                  // blocks per query tile
     const float *qscale;           // [n_q_pad] 2^e
     float *part_v;                 // [n_q][2 n_groups][k]
@@ -72,63 +75,54 @@ __device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
     return *reinterpret_cast<const uint32_t *>(&r);
 }
 
-// The two database rows a thread dequantizes: tile rows tid and tid + 256.
-// Rows past the end point at vector 0 with zero scales, so loads and
-// dequantization need no branches.
+// The database row a thread dequantizes: tile row tid.  A row past the end
+// points at vector 0 with zero scales, so loads and dequantization need no
+// branches.
 struct Rows {
-    const uint8_t *kc[2], *ks[2];   // this row's code bytes and sign bytes
-    uint32_t nbits[2];              // fp16 bits: nhat | rho << 16 (loaded a chunk ahead)
-    uint32_t nh2[2], rh2[2];        // nhat and -rho sqrt(pi/2)/m as fp16 pairs
+    const uint8_t *kc, *ks;         // this row's code bytes and sign bytes
+    uint32_t nbits;                 // fp16 bits: nhat | rho << 16 (loaded a chunk ahead)
+    uint32_t nh2, rh2;              // nhat and -rho sqrt(pi/2)/m as fp16 pairs
 };
 
 template <int D>
 __device__ __forceinline__ void rows_for(const SearchTcArgs &a, int64_t tile, int tid, Rows &r) {
     const Layout &L = a.L;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int64_t v = tile * kN + tid + 256 * j;
-        const bool ok = v < a.n_db;
-        const int64_t vv = ok ? v : 0;
-        const uint8_t *page = a.db + (vv / L.P) * int64_t(L.page_bytes);
-        const int pos = int(vv % L.P);
-        r.kc[j] = page + L.kc_off + pos * (D / 2);
-        r.ks[j] = page + L.ks_off + pos * (D / 8);
-        uint32_t nb = 0;
-        if (ok)
-            nb = uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2))) |
-                 (uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2))) << 16);
-        r.nbits[j] = nb;
-    }
+    const int64_t v = tile * kN + tid;
+    const bool ok = v < a.n_db;
+    const int64_t vv = ok ? v : 0;
+    const uint8_t *page = a.db + (vv / L.P) * int64_t(L.page_bytes);
+    const int pos = int(vv % L.P);
+    r.kc = page + L.kc_off + pos * (D / 2);
+    r.ks = page + L.ks_off + pos * (D / 8);
+    uint32_t nb = 0;
+    if (ok)
+        nb = uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2))) |
+             (uint32_t(__ldg(reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2))) << 16);
+    r.nbits = nb;
 }
 
 template <int D>
 __device__ __forceinline__ void rows_scales(Rows &r) {
     const float cq = 1.2533141373155003f / float(D);     // sqrt(pi/2) / m
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const uint32_t nb = r.nbits[j];
-        r.nh2[j] = (nb & 0xFFFFu) * 0x10001u;
-        const float rh = h2f_bits(uint16_t(nb >> 16)) * cq;
-        r.rh2[j] = h2pack(-rh, -rh);
-    }
+    const uint32_t nb = r.nbits;
+    r.nh2 = (nb & 0xFFFFu) * 0x10001u;
+    const float rh = h2f_bits(uint16_t(nb >> 16)) * cq;
+    r.rh2 = h2pack(-rh, -rh);
 }
 
-// Raw bytes of chunk kc for both rows: 32 code bytes (MSE chunk) or 8 sign
-// bytes (QJL chunk, in raw[j][0].x / .y).
+// Raw bytes of chunk kc of the row: 32 code bytes (MSE chunk) or 8 sign
+// bytes (QJL chunk, in raw[0].x / .y).
 template <int D>
-__device__ __forceinline__ void load_raw(const Rows &r, int kc, uint4 (&raw)[2][2]) {
+__device__ __forceinline__ void load_raw(const Rows &r, int kc, uint4 (&raw)[2]) {
     constexpr int MSE_KC = D / 64;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        if (kc < MSE_KC) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(r.kc[j] + kc * 32);
-            raw[j][0] = __ldg(src);
-            raw[j][1] = __ldg(src + 1);
-        } else {
-            const uint2 sg = __ldg(reinterpret_cast<const uint2 *>(r.ks[j] + (kc - MSE_KC) * 8));
-            raw[j][0].x = sg.x;
-            raw[j][0].y = sg.y;
-        }
+    if (kc < MSE_KC) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(r.kc + kc * 32);
+        raw[0] = __ldg(src);
+        raw[1] = __ldg(src + 1);
+    } else {
+        const uint2 sg = __ldg(reinterpret_cast<const uint2 *>(r.ks + (kc - MSE_KC) * 8));
+        raw[0].x = sg.x;
+        raw[0].y = sg.y;
     }
 }
 
@@ -138,7 +132,7 @@ struct Ctx {
     uint64_t *bar_a, *bar_m;
     const CUtensorMap *tmQ;
     uint32_t tmem;
-    int tid, warp, qt, half;
+    int tid, warp, qt, qh;          // qh: query half (M = 128 tile) of this thread's query
     float *tv;                      // top-k scores, entry r of thread t at [r * 256 + t]
     int32_t *ti;
     const uint32_t *lut_lane;
@@ -154,8 +148,7 @@ struct Ctx {
 // `nraw`, dequantize `raw` into shared memory, issue the MMAs, and after the
 // tile's last chunk scan its estimates.  Returns false to leave the loop.
 template <int D, int ST>
-__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 (&raw)[2][2],
-                                           uint4 (&nraw)[2][2]) {
+__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 (&raw)[2], uint4 (&nraw)[2]) {
     constexpr int NKC = 2 * D / 64;
     constexpr int MSE_KC = D / 64;
     const int kc = c.kc;
@@ -168,40 +161,37 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
         load_raw<D>(c.cur, kc + 1, nraw);
     }
 
-    uint8_t *sA = c.sm + SA + ST * 16384;
-    uint8_t *sB = c.sm + SB + ST * 65536;
+    uint8_t *sA = c.sm + SA + ST * 32768;
+    uint8_t *sB = c.sm + SB + ST * 32768;
     if ((c.used_m >> ST) & 1u) {        // the stage is free once the MMAs that read it completed
         if (!tc05::mbar_wait_bounded(&c.bar_m[ST], (c.phase_m >> ST) & 1u, kPolls)) c.timeout = true;
         c.phase_m ^= 1u << ST;
         c.used_m &= ~(1u << ST);
     }
     if (c.tid == 0) {
-        tc05::mbar_expect_tx(&c.bar_a[ST], 16384);
+        tc05::mbar_expect_tx(&c.bar_a[ST], 32768);
         tc05::tma_load_2d(sA, c.tmQ, kc * 64, c.qt * kQ, &c.bar_a[ST]);
         c.a_pending = ST;
     }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        uint8_t *brow = sB + j * 32768;
+    {
         uint32_t w[32];
         if (kc < MSE_KC) {
-            const uint32_t cw[8] = {raw[j][0].x, raw[j][0].y, raw[j][0].z, raw[j][0].w,
-                                    raw[j][1].x, raw[j][1].y, raw[j][1].z, raw[j][1].w};
+            const uint32_t cw[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y, raw[1].z, raw[1].w};
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
-                w[i] = hmul2u(c.lut_lane[byte * 32], c.cur.nh2[j]);
+                w[i] = hmul2u(c.lut_lane[byte * 32], c.cur.nh2);
             }
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const uint32_t word = (i < 16) ? raw[j][0].x : raw[j][0].y;
-                w[i] = c.cur.rh2[j] ^ ((word << (15 - (i & 15))) & 0x80008000u);
+                const uint32_t word = (i < 16) ? raw[0].x : raw[0].y;
+                w[i] = c.cur.rh2 ^ ((word << (15 - (i & 15))) & 0x80008000u);
             }
         }
 #pragma unroll
         for (int pc = 0; pc < 8; ++pc)
-            *reinterpret_cast<uint4 *>(brow + tc05::sw128_offset(uint32_t(c.tid), uint32_t(pc))) =
+            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(c.tid), uint32_t(pc))) =
                 make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
     }
     tc05::fence_proxy_async_smem();
@@ -213,12 +203,13 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
         tc05::fence_after_sync();
         const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sB);
         constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
+        // query half h: A rows [128 h, 128 h + 128) (16 KB apart), columns [256 h, 256 h + 256)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = tc05::desc_kmajor_sw128(aa + ks * 32);
+            const uint64_t bd = tc05::desc_kmajor_sw128(bb + ks * 32);
             const bool acc = (kc | ks) != 0;
-            tc05::mma_f16(c.tmem, ad, tc05::desc_kmajor_sw128(bb + ks * 32), idesc, acc);
-            tc05::mma_f16(c.tmem + 256, ad, tc05::desc_kmajor_sw128(bb + 32768 + ks * 32), idesc, acc);
+            tc05::mma_f16(c.tmem, tc05::desc_kmajor_sw128(aa + ks * 32), bd, idesc, acc);
+            tc05::mma_f16(c.tmem + 256, tc05::desc_kmajor_sw128(aa + 16384 + ks * 32), bd, idesc, acc);
         }
         tc05::mma_commit(&c.bar_m[ST]);
     }
@@ -238,15 +229,15 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
         }
         tc05::fence_after_sync();
         // estimates stay in accumulator units (2^-e of the true value) until the end
-        const int64_t rem = a.n_db - (c.tile * kN + c.half * 256);
-        const int lim = rem < 256 ? int(rem) : 256;
-        const int32_t id0 = int32_t(c.tile * kN + c.half * 256);
+        const int64_t rem = a.n_db - c.tile * kN;
+        const int lim = rem < kN ? int(rem) : kN;
+        const int32_t id0 = int32_t(c.tile * kN);
         const int K = a.k;
         float kth = c.tv[(K - 1) * kThreads + c.tid];
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
             uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.half * 256 + cc * 32),
+            tc05::tmem_ld_32x32b_x32(c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.qh * 256 + cc * 32),
                                      r);
             tc05::tmem_wait_ld();
 #pragma unroll
@@ -292,7 +283,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     c.tid = threadIdx.x;
     c.warp = c.tid >> 5;
     c.qt = blockIdx.x;
-    c.half = c.tid >> 7;
+    c.qh = c.tid >> 7;
     const int grp = blockIdx.y, K = a.k;
     c.tv = reinterpret_cast<float *>(c.sm + STOPV);
     c.ti = reinterpret_cast<int32_t *>(c.sm + STOPI);
@@ -324,7 +315,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     c.tile = grp;
     c.kc = 0;
 
-    uint4 rawA[2][2], rawB[2][2];
+    uint4 rawA[2], rawB[2];
     rows_for<D>(a, c.tile, c.tid, c.cur);
     load_raw<D>(c.cur, 0, rawA);
     while (c.tile < a.n_tiles) {
@@ -339,11 +330,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     for (int s2 = 0; s2 < 2; ++s2)
         if (((c.used_m >> s2) & 1u) && !tc05::mbar_wait_bounded(&c.bar_m[s2], (c.phase_m >> s2) & 1u, kPolls))
             c.timeout = true;
-    const int q = c.qt * kQ + (c.tid & 127);
+    const int q = c.qt * kQ + c.tid;                    // = 256 qt + 128 qh + TMEM lane
     if (q < a.n_q) {
         const float qsc = a.qscale[q];
         for (int r = 0; r < K; ++r) {
-            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + c.half) * K + r;
+            const int64_t o = (int64_t(q) * a.n_groups + grp) * K + r;
             const int32_t id = c.ti[r * kThreads + c.tid];
             a.part_v[o] = id >= 0 ? c.tv[r * kThreads + c.tid] * qsc : -INFINITY;
             a.part_i[o] = id;
@@ -415,7 +406,7 @@ int run_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
     CUtensorMap tm;
     cuuint64_t dims[2] = {cuuint64_t(2 * D), cuuint64_t(n_q_pad)};
     cuuint64_t strides[1] = {cuuint64_t(2 * D * 2)};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, uint32_t(kQ)};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, qf, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -444,7 +435,7 @@ int run_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
 }  // namespace
 
 // Database groups (blocks per query tile) of the tensor-core search, 0 when
-// the configuration is not covered.  Each group yields two candidate lists
+// the configuration is not covered.  Each group yields one candidate list
 // per query.
 int search_tc_groups(const Layout &L, int64_t n_db, int n_q, int k) {
     if (!(L.kbits == 4 && L.kqjl && L.vbits == 0) || k > kTopK || n_db > INT32_MAX) return 0;
