@@ -93,20 +93,67 @@ def aggregate(units_per_rank: float, times_s: list[float]) -> tuple[float, float
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and throttle reasons while the timed region runs.
+
+    NVML (read-only queries) is polled from a thread about every millisecond,
+    so even a region of a few milliseconds yields samples; without NVML,
+    nvidia-smi at its 200 ms rate.  Nothing here changes a GPU setting."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
         self.proc = None
         self.path = None
+        self.thread = None
+        self.nvml = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             self.sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
         except Exception:
             self.sel = str(device_index)
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.sel)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.handle = pynvml, h
+            self.bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while not self.done.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for n, b in self.bits.items():
+                    if r & b:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            self.done.wait(0.001)
 
     def start(self):
+        import threading
+        self.sm, self.power, self.reasons = [], [], set()
+        if self.nvml is not None:
+            try:
+                self.smax = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            except Exception:
+                self.smax = None
+            self.done = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -116,7 +163,16 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _result(self, sm, smax, power, source):
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(self.reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "source": source}
+
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.done.set()
+            self.thread.join(timeout=5)
+            return self._result(self.sm, self.smax, self.power, "nvml, 1 ms polling")
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -124,8 +180,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons, power = [], [], set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, power = [], [], []
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
@@ -137,13 +192,11 @@ class ClockSampler:
                     power.append(float(parts[3]))
                 except ValueError:
                     continue
-                for n, v in zip(names, parts[5:9]):
+                for n, v in zip(self.NAMES, parts[5:9]):
                     if v.lower().startswith("active"):
-                        reasons.add(n)
+                        self.reasons.add(n)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+        return self._result(sm, max(smax) if smax else None, power, "nvidia-smi, 200 ms")
 
 
 # --------------------------------------------------------------------------
@@ -483,7 +536,8 @@ def run_ours(args):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
     clocks.start()
-    time.sleep(0.3)
+    if clocks.thread is None:
+        time.sleep(0.3)                   # nvidia-smi needs a moment to start sampling
     torch.cuda.synchronize()
     barrier(world)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -204,7 +204,7 @@ SPlan splan(const Layout &L, int64_t n_db, int n_q, int k) {
     SPlan s;
     s.tc_groups = search_tc_groups(L, n_db, n_q, k);
     if (s.tc_groups > 0) {
-        s.n_splits = s.tc_groups;
+        s.n_splits = 2 * s.tc_groups;
         s.split_len = 0;
     } else {
         const int tiles = (n_q + kQT - 1) / kQT;

@@ -14,12 +14,12 @@
 //        64-feature chunk at a time; e makes the largest feature 1 <= |f| < 2
 //        and the scores are multiplied back by 2^e);
 //   Xf = [nhat c[code] | rho sqrt(pi/2)/m (2 s - 1)] per database vector,
-//        dequantized by the block's threads (one database row each) into
-//        shared memory (128-byte swizzled K-major tiles) while the previous
-//        chunk's MMAs run.
-// Epilogue: thread q reads its query's 256 estimates from TMEM and keeps a
-// running top-k (ties to the lower index); a merge kernel combines the
-// blocks' lists.
+//        dequantized by the block's threads (two per database row, 32
+//        features each) into shared memory (128-byte swizzled K-major
+//        tiles) while the previous chunk's MMAs run.
+// Epilogue: two threads per query each read half of its 256 estimates from
+// TMEM and keep a running top-k (ties to the lower index); a merge kernel
+// combines the blocks' lists.
 //
 // Inside every 32-coordinate group the QJL features are in the order
 // (p, p + 16) for feature positions (2p, 2p + 1), so a pair of sign bits
@@ -37,7 +37,7 @@ namespace {
 
 constexpr int kQ = 256;                 // queries per block (two MMAs of M = 128, TMEM lanes)
 constexpr int kN = 256;                 // database vectors per tile (MMA N)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kTopK = 16;               // largest k this path takes
 constexpr int kSMs = 148;               // grid sizing (fixed, so workspace sizes do not depend on the device)
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
@@ -75,9 +75,9 @@ __device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
     return *reinterpret_cast<const uint32_t *>(&r);
 }
 
-// The database row a thread dequantizes: tile row tid.  A row past the end
-// points at vector 0 with zero scales, so loads and dequantization need no
-// branches.
+// The database row a thread dequantizes: tile row tid % 256 (features
+// [32 p, 32 p + 32) of each chunk, p = tid / 256).  A row past the end points
+// at vector 0 with zero scales, so loads and dequantization need no branches.
 struct Rows {
     const uint8_t *kc, *ks;         // this row's code bytes and sign bytes
     uint32_t nbits;                 // fp16 bits: nhat | rho << 16 (loaded a chunk ahead)
@@ -87,7 +87,7 @@ struct Rows {
 template <int D>
 __device__ __forceinline__ void rows_for(const SearchTcArgs &a, int64_t tile, int tid, Rows &r) {
     const Layout &L = a.L;
-    const int64_t v = tile * kN + tid;
+    const int64_t v = tile * kN + (tid & 255);
     const bool ok = v < a.n_db;
     const int64_t vv = ok ? v : 0;
     const uint8_t *page = a.db + (vv / L.P) * int64_t(L.page_bytes);
@@ -110,20 +110,13 @@ __device__ __forceinline__ void rows_scales(Rows &r) {
     r.rh2 = h2pack(-rh, -rh);
 }
 
-// Raw bytes of chunk kc of the row: 32 code bytes (MSE chunk) or 8 sign
-// bytes (QJL chunk, in raw[0].x / .y).
+// Raw bytes of part p of chunk kc of the row: 16 code bytes (MSE chunk) or
+// 4 sign bytes (QJL chunk, in raw.x).
 template <int D>
-__device__ __forceinline__ void load_raw(const Rows &r, int kc, uint4 (&raw)[2]) {
+__device__ __forceinline__ void load_raw(const Rows &r, int kc, int p, uint4 &raw) {
     constexpr int MSE_KC = D / 64;
-    if (kc < MSE_KC) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(r.kc + kc * 32);
-        raw[0] = __ldg(src);
-        raw[1] = __ldg(src + 1);
-    } else {
-        const uint2 sg = __ldg(reinterpret_cast<const uint2 *>(r.ks + (kc - MSE_KC) * 8));
-        raw[0].x = sg.x;
-        raw[0].y = sg.y;
-    }
+    if (kc < MSE_KC) raw = __ldg(reinterpret_cast<const uint4 *>(r.kc + kc * 32 + 16 * p));
+    else raw.x = __ldg(reinterpret_cast<const uint32_t *>(r.ks + (kc - MSE_KC) * 8 + 4 * p));
 }
 
 // Per-block state of the scoring loop.
@@ -132,7 +125,8 @@ struct Ctx {
     uint64_t *bar_a, *bar_m;
     const CUtensorMap *tmQ;
     uint32_t tmem;
-    int tid, warp, qt, qh;          // qh: query half (M = 128 tile) of this thread's query
+    int tid, warp, qt, qh, part;    // qh: query half (M = 128 tile) of this thread's query;
+                                    // part: feature half it dequantizes, vector half it scans
     float *tv;                      // top-k scores, entry r of thread t at [r * 256 + t]
     int32_t *ti;
     const uint32_t *lut_lane;
@@ -148,7 +142,7 @@ struct Ctx {
 // `nraw`, dequantize `raw` into shared memory, issue the MMAs, and after the
 // tile's last chunk scan its estimates.  Returns false to leave the loop.
 template <int D, int ST>
-__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 (&raw)[2], uint4 (&nraw)[2]) {
+__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 &raw, uint4 &nraw) {
     constexpr int NKC = 2 * D / 64;
     constexpr int MSE_KC = D / 64;
     const int kc = c.kc;
@@ -156,9 +150,9 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
     if (kc == 0) rows_scales<D>(c.cur);
     if (last) {
         rows_for<D>(a, c.tile + a.n_groups, c.tid, c.nxt);
-        load_raw<D>(c.nxt, 0, nraw);
+        load_raw<D>(c.nxt, 0, c.part, nraw);
     } else {
-        load_raw<D>(c.cur, kc + 1, nraw);
+        load_raw<D>(c.cur, kc + 1, c.part, nraw);
     }
 
     uint8_t *sA = c.sm + SA + ST * 32768;
@@ -174,24 +168,22 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
         c.a_pending = ST;
     }
     {
-        uint32_t w[32];
+        // features [32 part, 32 part + 32) of row tid % 256: 16-byte chunks 4 part .. 4 part + 3
+        uint32_t w[16];
         if (kc < MSE_KC) {
-            const uint32_t cw[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+            const uint32_t cw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
                 const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
                 w[i] = hmul2u(c.lut_lane[byte * 32], c.cur.nh2);
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const uint32_t word = (i < 16) ? raw[0].x : raw[0].y;
-                w[i] = c.cur.rh2 ^ ((word << (15 - (i & 15))) & 0x80008000u);
-            }
+            for (int i = 0; i < 16; ++i) w[i] = c.cur.rh2 ^ ((raw.x << (15 - i)) & 0x80008000u);
         }
 #pragma unroll
-        for (int pc = 0; pc < 8; ++pc)
-            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(c.tid), uint32_t(pc))) =
+        for (int pc = 0; pc < 4; ++pc)
+            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(c.tid & 255), uint32_t(4 * c.part + pc))) =
                 make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
     }
     tc05::fence_proxy_async_smem();
@@ -229,16 +221,17 @@ __device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const 
         }
         tc05::fence_after_sync();
         // estimates stay in accumulator units (2^-e of the true value) until the end
-        const int64_t rem = a.n_db - c.tile * kN;
-        const int lim = rem < kN ? int(rem) : kN;
-        const int32_t id0 = int32_t(c.tile * kN);
+        // this thread's vector half: columns [128 part, 128 part + 128) of its query half
+        const int64_t rem = a.n_db - (c.tile * kN + 128 * c.part);
+        const int lim = rem < 128 ? int(rem) : 128;
+        const int32_t id0 = int32_t(c.tile * kN + 128 * c.part);
         const int K = a.k;
         float kth = c.tv[(K - 1) * kThreads + c.tid];
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
             uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.qh * 256 + cc * 32),
-                                     r);
+            tc05::tmem_ld_32x32b_x32(
+                c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.qh * 256 + 128 * c.part + cc * 32), r);
             tc05::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -283,7 +276,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     c.tid = threadIdx.x;
     c.warp = c.tid >> 5;
     c.qt = blockIdx.x;
-    c.qh = c.tid >> 7;
+    c.qh = (c.tid >> 7) & 1;
+    c.part = c.tid >> 8;
     const int grp = blockIdx.y, K = a.k;
     c.tv = reinterpret_cast<float *>(c.sm + STOPV);
     c.ti = reinterpret_cast<int32_t *>(c.sm + STOPI);
@@ -315,9 +309,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     c.tile = grp;
     c.kc = 0;
 
-    uint4 rawA[2], rawB[2];
+    uint4 rawA = make_uint4(0, 0, 0, 0), rawB = rawA;
     rows_for<D>(a, c.tile, c.tid, c.cur);
-    load_raw<D>(c.cur, 0, rawA);
+    load_raw<D>(c.cur, 0, c.part, rawA);
     while (c.tile < a.n_tiles) {
         if (!chunk_step<D, 0>(c, a, rawA, rawB)) break;
         if (!chunk_step<D, 1>(c, a, rawB, rawA)) break;
@@ -330,11 +324,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     for (int s2 = 0; s2 < 2; ++s2)
         if (((c.used_m >> s2) & 1u) && !tc05::mbar_wait_bounded(&c.bar_m[s2], (c.phase_m >> s2) & 1u, kPolls))
             c.timeout = true;
-    const int q = c.qt * kQ + c.tid;                    // = 256 qt + 128 qh + TMEM lane
+    const int q = c.qt * kQ + (c.tid & 255);            // = 256 qt + 128 qh + TMEM lane
     if (q < a.n_q) {
         const float qsc = a.qscale[q];
         for (int r = 0; r < K; ++r) {
-            const int64_t o = (int64_t(q) * a.n_groups + grp) * K + r;
+            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + c.part) * K + r;
             const int32_t id = c.ti[r * kThreads + c.tid];
             a.part_v[o] = id >= 0 ? c.tv[r * kThreads + c.tid] * qsc : -INFINITY;
             a.part_i[o] = id;
@@ -435,8 +429,8 @@ int run_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
 }  // namespace
 
 // Database groups (blocks per query tile) of the tensor-core search, 0 when
-// the configuration is not covered.  Each group yields one candidate list
-// per query.
+// the configuration is not covered.  Each group yields two candidate lists
+// per query (one per vector half of its tiles).
 int search_tc_groups(const Layout &L, int64_t n_db, int n_q, int k) {
     if (!(L.kbits == 4 && L.kqjl && L.vbits == 0) || k > kTopK || n_db > INT32_MAX) return 0;
     if (!(L.d == 128 || L.d == 256 || L.d == 512 || L.d == 1024)) return 0;
