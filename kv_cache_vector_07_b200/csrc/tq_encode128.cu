@@ -14,8 +14,10 @@
 //           (each thread sums its own 64 coordinates by quarter; the pair
 //           swaps quarter sums through shared memory and adds all four in a
 //           fixed order, so both agree, and neither reads columns the other
-//           is about to overwrite with its residual), bucketize against the Lloyd-Max boundaries scaled by
-//           the norm, sign-magnitude codes packed into the page, fp16 norm; for
+//           is about to overwrite with its residual), bucketize (3- and
+//           4-bit codebooks: a 16-cell rank table over C |y| / ||y||; 1- and
+//           2-bit: the boundaries scaled by the norm), sign-magnitude codes
+//           packed into the page, fp16 norm; for
 //           QJL keys the residual r = y - nhat c[idx] (scaled by a power of
 //           two) split into fp16 hi + lo, written back over the tile's own Y
 //           columns, rho = fp16 ||r||
