@@ -34,7 +34,11 @@ namespace tq {
 
 namespace {
 
-constexpr int kNS = 3;                  // page stages
+// Page stages: 4-bit-key pages (150 B per token) take two, so that four
+// blocks fit in an SM's shared memory next to the 256-entry pair tables;
+// smaller pages keep three.
+template <int KB>
+__host__ __device__ constexpr int page_stages() { return KB == 4 ? 2 : 3; }
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 struct Dec128Args {
@@ -100,6 +104,7 @@ template <int KB, int VB, int NT>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     static_assert(KB == 2 || KB == 4, "key bits");
     static_assert(VB == 3 || VB == 4, "value bits");
+    constexpr int kNS = page_stages<KB>();
     constexpr int KE = KB == 4 ? 256 : 16;          // key pair-table entries (two codes)
     constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
     constexpr int KC = key_copies<KB>(), VC = val_copies<VB>();
@@ -483,6 +488,7 @@ template <int KB, int VB, int NT>
 size_t dec_smem(int page_bytes) {
     constexpr int KE = KB == 4 ? 256 : 16, VE = VB == 4 ? 256 : 16;
     // the stage area also holds the final merge: 64 + 4 x 8 x 128 floats
+    constexpr int kNS = page_stages<KB>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
     return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 + size_t(NT) * 16 * 32 * 8 +
