@@ -179,7 +179,7 @@ int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq_cache_desc
  * allocate device memory (an engine that keeps all device memory in its own
  * pool and forbids other allocations, a plug-in handed only one call's
  * tensors, a latency-critical path that cannot afford a blocking cudaMalloc).
- * The paper has no counterpart: this is a library convenience.  Same
+ * The pages describe no counterpart: this is a library convenience.  Same
  * arguments and results as tq_decode_attn minus the workspace, which is
  * replaced by a file-scope device array of TQ_NOALLOC_SCRATCH_BYTES bytes
  * that every GPU loading the library holds until the process exits.

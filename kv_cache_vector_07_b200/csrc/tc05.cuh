@@ -261,7 +261,7 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
-// Two-dimensional tiled tensor copy global -> shared (no multicast),
+// Two-dimensional tiled tensor copy global -> this CTA's shared memory,
 // coordinates (x = innermost element index, y = row), completing on the
 // mbarrier.  x * element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
