@@ -236,7 +236,7 @@ class StepWorkload:
         per_tok = page // P
         self.enc_bytes = 2 * n * H * d * 2 + n * H * per_tok
         self.dec_bytes = B * H * L * per_tok + 2 * self.Q.numel() * 2
-        self.launches = {"encode": 1, "decode": 4}
+        self.launches = {"encode": 1, "decode": 3}       # decode: fused query prep, dec128, combine
 
     def ops(self):
         tq = self.tq
@@ -314,7 +314,7 @@ class Decode32kWorkload:
         self.ws_d = torch.zeros(tqkv.decode_workspace_bytes(self.desc, B, Hq, L), dtype=torch.uint8, device=dev)
         self.units = B * Hq * L
         self.dec_bytes = B * H * L * (tqkv.cache_bytes(self.desc) // P) + 2 * self.Q.numel() * 2
-        self.launches = {"decode": 4}
+        self.launches = {"decode": 3}                    # fused query prep, dec128, combine
 
     def ops(self):
         tq = self.tq
@@ -382,7 +382,7 @@ class LongCtxWorkload:
         self.units = self.dec_pairs + self.pre_pairs
         self.dec_bytes = H * L * per_tok
         self.pre_flops = self.pre_pairs * 2 * (2 * d + d)       # QK^T over 256 features + PV over 128
-        self.launches = {"decode": 4, "prefill": 4}
+        self.launches = {"decode": 3, "prefill": 3}      # each: fused query prep, dec128 / pf128, combine
 
     def ops(self):
         tq = self.tq
