@@ -356,3 +356,109 @@ def test_cache_write_read_roundtrip():
     assert np.array_equal(back["kn"], Ek.nhat) and np.array_equal(back["kr"], Ek.rho)
     assert np.array_equal(back["vn"], Ev.nhat)
     assert not cache[0::2].any()          # head 0 pages untouched
+
+
+# --------------------------------------------------------------------------
+# attention through the oracle's own compressed path, on keys and values
+# that its codes represent exactly (the identity quantizer in code form)
+# --------------------------------------------------------------------------
+def _exact_from_codes(P, idx, nhat):
+    """Vectors x_t = R^T (nhat_t c[idx_t]) built with scipy's Hadamard matrix,
+    so that the oracle's encoded form (idx, nhat) reconstructs them exactly."""
+    d = P.d
+    R = scipy.linalg.hadamard(d).astype(np.float64) @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    Y = nhat[:, None] * P.c32.astype(np.float64)[idx]
+    return Y @ R          # rows: (R^T y_t)^T
+
+
+@pytest.mark.parametrize("L,nq", [(300, 5), (777, 3)])
+def test_attend_equals_textbook_softmax_on_exactly_coded_kv(L, nq):
+    d = 128
+    rng = np.random.default_rng(L)
+    Pk, Pv = O.make_params(d, 4, 31, with_S=False), O.make_params(d, 3, 32, with_S=False)
+    kidx = rng.integers(0, 16, (L, d)).astype(np.uint8)
+    vidx = rng.integers(0, 8, (L, d)).astype(np.uint8)
+    kn = np.array([O.round_fp16(v) for v in rng.uniform(2.0, 30.0, L)])
+    vn = np.array([O.round_fp16(v) for v in rng.uniform(0.5, 8.0, L)])
+    Kx, Vx = _exact_from_codes(Pk, kidx, kn), _exact_from_codes(Pv, vidx, vn)
+    Ek, Ev = O.Encoded(4, False, kidx, kn), O.Encoded(3, False, vidx, vn)
+    Q = rng.standard_normal((nq, d)) * 1.5
+    nvis = np.array([L, 1, L // 2, L - 3, 64][:nq], np.int32)
+    out, lse, logits = O.attend(Q, Pk, Ek, Pv, Ev, nvis=nvis, want_logits=True)
+    for a in range(nq):
+        n = nvis[a]
+        lg = Q[a] @ Kx[:n].T / math.sqrt(d)
+        ref = scipy.special.softmax(lg) @ Vx[:n]
+        assert np.allclose(out[a], ref, atol=1e-11, rtol=0), a
+        assert abs(lse[a] - scipy.special.logsumexp(lg)) < 1e-11
+        assert np.allclose(logits[a, :n], lg, atol=1e-11, rtol=0)
+        assert np.all(np.isneginf(logits[a, n:]))
+
+
+# --------------------------------------------------------------------------
+# FP8 keys: code = torch's E4M3 cast of sqrt(d) R x / ||x||
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [8, 128, 1024])
+def test_fp8_encode_matches_torch_e4m3_of_rotated_unit_vector(d):
+    rng = np.random.default_rng(d + 5)
+    P = O.make_params(d, 8, 77, with_S=False)
+    X = rng.standard_normal((40, d)) * np.exp(rng.standard_normal(d))[None, :]
+    X[3] = 0.0
+    enc = O.encode(X, P, qjl=False)
+    R = scipy.linalg.hadamard(d).astype(np.float64) @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    n = np.linalg.norm(X, axis=1)
+    Y = X @ R.T
+    U = np.where(n[:, None] > 0, Y / np.where(n > 0, n, 1.0)[:, None], 0.0)
+    a = math.sqrt(d) * U
+    # compare only where the oracle's value is not within 1e-9 of a rounding midpoint
+    # (torch casts from fp32; the oracle rounds the float64 value)
+    ref = torch.from_numpy(a.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    clear = enc.umargin * math.sqrt(d) > 1e-6 * np.maximum(1.0, np.abs(a))
+    assert clear.mean() > 0.99
+    assert np.array_equal(enc.idx[clear], ref[clear])
+    assert np.array_equal(enc.nhat, n.astype(np.float16).astype(np.float64))
+    # reconstruction nhat e4m3(code) / sqrt(d) within half an E4M3 step of R x (plus the fp16 norm's rounding)
+    val = torch.from_numpy(enc.idx.copy()).view(torch.float8_e4m3fn).double().numpy()
+    rec = enc.nhat[:, None] * val / math.sqrt(d)
+    half_step = np.where(np.abs(a) >= 2.0 ** -6, np.exp2(np.floor(np.log2(np.maximum(np.abs(a), 1e-300))) - 4),
+                         2.0 ** -10)
+    bound = n[:, None] * half_step / math.sqrt(d) * (1 + 1e-9) + np.abs(Y) * 2.0 ** -11
+    assert np.all(np.abs(rec - Y) <= bound)
+    assert np.all(enc.idx[3] == 0) and enc.nhat[3] == 0.0
+
+
+# --------------------------------------------------------------------------
+# exemption margins against direct numpy distances
+# --------------------------------------------------------------------------
+def test_code_and_sign_margins_match_direct_distances():
+    d = 128
+    rng = np.random.default_rng(55)
+    P = O.make_params(d, 3, 91)
+    X = rng.standard_normal((12, d))
+    X[:, 5] *= 20.0
+    enc = O.encode(X, P, qjl=True)
+    R = scipy.linalg.hadamard(d).astype(np.float64) @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    n = np.linalg.norm(X, axis=1)
+    U = (X @ R.T) / n[:, None]
+    t = P.t32.astype(np.float64)
+    um = np.min(np.abs(U[:, :, None] - t[None, None, :]), axis=2)
+    assert np.allclose(enc.umargin, um, rtol=0, atol=1e-13)
+    r = X @ R.T - enc.nhat[:, None] * P.c32.astype(np.float64)[enc.idx]
+    Z = r @ P.S.astype(np.float64).T
+    zm = np.abs(Z) / (np.linalg.norm(r, axis=1)[:, None] * np.linalg.norm(P.S.astype(np.float64), axis=1)[None, :])
+    assert np.allclose(enc.zmargin, zm, rtol=1e-9, atol=1e-15)
+    assert np.array_equal(enc.sbits, (Z >= 0).astype(np.uint8))
+
+
+def test_fp8_margin_matches_direct_distance_to_rounding_midpoints():
+    d = 64
+    rng = np.random.default_rng(56)
+    P = O.make_params(d, 8, 92, with_S=False)
+    X = rng.standard_normal((6, d))
+    enc = O.encode(X, P, qjl=False)
+    vals = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()  # finite, >= 0
+    mids = 0.5 * (vals[:-1] + vals[1:])
+    R = scipy.linalg.hadamard(d).astype(np.float64) @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    a = math.sqrt(d) * (X @ R.T) / np.linalg.norm(X, axis=1)[:, None]
+    mg = np.min(np.abs(np.abs(a)[:, :, None] - mids[None, None, :]), axis=2) / math.sqrt(d)
+    assert np.allclose(enc.umargin, mg, rtol=0, atol=1e-13)
