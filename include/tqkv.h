@@ -242,6 +242,19 @@ int tq_read_status(void *workspace, void *stream, uint32_t *flags);
 /* Static description of a status code. */
 const char *tq_status_string(int status);
 
+/* ------------------------------------------------------------------------ */
+/* Testing aid                                                              */
+/* ------------------------------------------------------------------------ */
+/* Make the next tq_decode_attn launch of the tensor-core decode kernel
+ * (d = 128, 64-token pages, Lloyd-Max keys with QJL) start every block with a
+ * wait of `polls` polls on an on-chip barrier that nothing completes.  The
+ * wait runs out before any copy or tensor-core operation is issued, the
+ * blocks take their time-out path (no further copies, results written as
+ * empty) and the workspace status word gets TQ_DEV_WAIT_TIMEOUT.  It exists
+ * so that the time-out path can be exercised without a fault; polls = 0
+ * cancels a pending request.  The pages describe no counterpart. */
+int tq_test_stall_next_decode(uint32_t polls);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,7 +66,7 @@ namespace {
 bool attn_params_ok(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc, int Hq) {
     if (!valid_desc(desc) || !kp || !vp) return false;
     if (desc->d > 256) return false;
-    if (desc->kbits == 8 || desc->vbits == 0) return false;
+    if (desc->vbits == 0) return false;
     if (kp->d != desc->d || kp->bits != desc->kbits || vp->d != desc->d || vp->bits != desc->vbits) return false;
     if (Hq < 1 || Hq % desc->n_kv_heads) return false;
     const int G = Hq / desc->n_kv_heads;
@@ -94,8 +94,8 @@ extern "C" int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq
                               float *logits, int64_t logits_stride, void *workspace, size_t workspace_bytes,
                               void *stream) {
     if (!attn_params_ok(kp, vp, desc, Hq)) {
-        if (valid_desc(desc) && (desc->kbits == 8 || desc->d > 256 || (Hq >= 1 && Hq % desc->n_kv_heads == 0 &&
-                                                                     Hq / desc->n_kv_heads > 8)))
+        if (valid_desc(desc) && (desc->d > 256 || (Hq >= 1 && Hq % desc->n_kv_heads == 0 &&
+                                                   Hq / desc->n_kv_heads > 8)))
             return TQ_EUNSUPPORTED;
         return TQ_EINVAL;
     }
@@ -139,7 +139,7 @@ extern "C" int tq_prefill_attn(const tq_params *kp, const tq_params *vp, const t
                                const void *cache, int64_t num_blocks, void *out, float *lse, void *workspace,
                                size_t workspace_bytes, void *stream) {
     if (!attn_params_ok(kp, vp, desc, Hq)) {
-        if (valid_desc(desc) && (desc->kbits == 8 || desc->d > 256)) return TQ_EUNSUPPORTED;
+        if (valid_desc(desc) && desc->d > 256) return TQ_EUNSUPPORTED;
         return TQ_EINVAL;
     }
     if (C < 0 || seq_len < C || max_blocks < 0 || num_blocks < 0) return TQ_EINVAL;

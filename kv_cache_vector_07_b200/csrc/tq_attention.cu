@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
         sw[c][h] = a.w[(row0 + h) * D + c];
     }
     if (tid < 16) {
-        lvk[tid] = tid < (1 << L.kbits) ? a.kp.lv[tid] : 0.f;
+        lvk[tid] = (L.kbits <= 4 && tid < (1 << L.kbits)) ? a.kp.lv[tid] : 0.f;
         lvv[tid] = tid < (1 << L.vbits) ? a.vp.lv[tid] : 0.f;
     }
     if (tid < kMaxG) { s_m[tid] = -INFINITY; s_l[tid] = 0.f; }
@@ -193,9 +193,14 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) { mse[h] = 0.f; qj[h] = 0.f; }
             for (int i = 0; i < D; ++i) {
-                uint32_t kap = read_field(kc, i, kw);
-                if (kh) kap |= read_field(kh, i, 1) << 2;
-                const float cv = lvk[kap];
+                float cv;
+                if (kw == 8) {
+                    cv = e4m3_to_float(kc[i]);          // FP8 key: e4m3(sqrt(d) u_i)
+                } else {
+                    uint32_t kap = read_field(kc, i, kw);
+                    if (kh) kap |= read_field(kh, i, 1) << 2;
+                    cv = lvk[kap];
+                }
                 const bool pos_sign = ks ? (read_field(ks, i, 1) != 0) : true;
 #pragma unroll
                 for (int h = 0; h < kMaxG; ++h) {
@@ -205,7 +210,9 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
                     }
                 }
             }
-            const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2));
+            // FP8 keys store sqrt(d) u: the estimate is nhat <Rq, e4m3(code)> / sqrt(d)
+            const float nk = h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kn_off + pos * 2)) *
+                             (kw == 8 ? scale : 1.0f);
             const float rk = L.kqjl ? h2f_bits(*reinterpret_cast<const uint16_t *>(page + L.kr_off + pos * 2)) : 0.f;
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) {

@@ -24,6 +24,8 @@
 //           and one table lookup gives the fp16 pair.
 // Warps merge in shared memory; blocks leave (m, l, o) partials for the
 // log-sum-exp combine kernel.
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
@@ -39,6 +41,10 @@ namespace {
 // smaller pages keep three.
 template <int KB>
 __host__ __device__ constexpr int page_stages() { return KB == 4 ? 2 : 3; }
+// Key pair-table entries: two 4-bit codes (256), two 2-bit codes (16); FP8
+// keys need no table (each E4M3 byte converts to fp16 exactly).
+template <int KB>
+__host__ __device__ constexpr int key_entries() { return KB == 4 ? 256 : (KB == 2 ? 16 : 0); }
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 struct Dec128Args {
@@ -57,7 +63,21 @@ struct Dec128Args {
     float *logits;
     int64_t logits_stride;
     uint32_t *status;
+    uint32_t stall_polls;          // testing aid: > 0 makes every block first wait
+                                   // this many polls on a barrier nothing completes
 };
+
+// Bounded wait that also gives up once another thread of the block has given
+// up (checked every 256 polls); the first thread to give up raises the flag.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, uint32_t max_polls,
+                                              volatile int *abort_flag) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
+        if (tc05::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    return false;
+}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -92,7 +112,7 @@ __device__ __forceinline__ int visible(const Dec128Args &a, int b) {
 // keeps four blocks' worth of shared memory per SM).  Lane l reads copy
 // l mod copies.
 template <int B>
-__host__ __device__ constexpr int key_copies() { return B == 4 ? 8 : 16; }
+__host__ __device__ constexpr int key_copies() { return B == 4 ? 8 : (B == 2 ? 16 : 1); }
 template <int B>
 __host__ __device__ constexpr int val_copies() { return B == 4 ? 8 : 32; }
 
@@ -102,10 +122,11 @@ __device__ __forceinline__ uint32_t lut(const uint32_t *tab_lane, uint32_t e) { 
 
 template <int KB, int VB, int NT>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
-    static_assert(KB == 2 || KB == 4, "key bits");
+    static_assert(KB == 2 || KB == 4 || KB == 8, "key bits");
     static_assert(VB == 3 || VB == 4, "value bits");
+    constexpr bool FP8 = KB == 8;                   // E4M3 keys, no QJL part
     constexpr int kNS = page_stages<KB>();
-    constexpr int KE = KB == 4 ? 256 : 16;          // key pair-table entries (two codes)
+    constexpr int KE = key_entries<KB>();           // key pair-table entries (two codes)
     constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
     constexpr int KC = key_copies<KB>(), VC = val_copies<VB>();
     extern __shared__ __align__(16) uint8_t smem[];
@@ -118,7 +139,9 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     const int stage_area = max(kNS * pbytes, (64 + 4 * 8 * 128) * 4);
     uint64_t *full = reinterpret_cast<uint64_t *>(stage0 + stage_area);
     uint64_t *empty = full + kNS;
-    int *pvalid = reinterpret_cast<int *>(empty + kNS);
+    uint64_t *never = empty + kNS;                 // completed by nothing (stall_polls only)
+    int *pvalid = reinterpret_cast<int *>(never + 1);
+    volatile int *abort_flag = pvalid + kNS;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -140,6 +163,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
         float c0, c1;
         if (KB == 4) { c0 = a.k_lv[e & 15]; c1 = a.k_lv[e >> 4]; }
         else { c0 = a.k_lv[e & 3]; c1 = a.k_lv[(e >> 2) & 3]; }
+        if (FP8) continue;
         const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
         lutK[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
     }
@@ -158,7 +182,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             const int hd = 4 * nt + (gg >> 1);
             const bool lo_part = (gg & 1) != 0;
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            if (hd < G) {
+            if (hd < G && !(FP8 && ks >= 8)) {
                 const float *src = ks < 8 ? a.qr + (row0 + hd) * 128 : a.w + (row0 + hd) * 128;
                 int c[4];
                 if (ks < 8) {
@@ -183,8 +207,14 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             tc05::mbar_init(&full[s], 1);
             tc05::mbar_init(&empty[s], 4);
         }
+        tc05::mbar_init(never, 1);
+        *abort_flag = 0;
         tc05::fence_mbar_init();
     }
+    __syncthreads();
+    // Testing aid: a wait that runs out before any bulk copy is issued, so the
+    // block takes the abort path with nothing in flight.
+    if (a.stall_polls) wait_or_abort(never, 0, a.stall_polls, abort_flag);
     __syncthreads();
 
     auto issue_page = [&](int i) {          // thread 0 only
@@ -202,9 +232,13 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc05::smem_u32(&full[st])) : "memory");
         }
     };
-    bool timeout = false;
-    if (tid == 0)
-        for (int i = 0; i < kNS - 1 && i < n_pages; ++i) issue_page(i);
+    // Pages [0, issued) have been handed to the copy engine (thread 0's count).
+    // On the first wait that runs out, every warp leaves the page loop at its
+    // next check, no further copy is issued, and thread 0 drains the copies
+    // still in flight before the stage memory is reused for the merge.
+    int issued = 0;
+    if (tid == 0 && !*abort_flag)
+        for (int i = 0; i < kNS - 1 && i < n_pages; ++i) { issue_page(i); issued = i + 1; }
 
     const uint2 *lutK_l = lutK + (lane & (KC - 1));
     const uint32_t *lutV_l = lutV + (lane & (VC - 1));
@@ -218,16 +252,22 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) O[mt][k] = 0.f;
 
+    int i_stop = n_pages;                  // thread 0: first page not consumed
     for (int i = 0; i < n_pages; ++i) {
         const int st = i % kNS;
-        if (tid == 0 && i + kNS - 1 < n_pages) {
+        bool fail = *abort_flag != 0;
+        if (!fail && tid == 0 && i + kNS - 1 < n_pages) {
             const int j = i + kNS - 1;            // refill the stage page i-1 used
-            if (j >= kNS) {
-                if (!tc05::mbar_wait_bounded(&empty[j % kNS], uint32_t(((j / kNS) - 1) & 1), kPolls)) timeout = true;
-            }
-            issue_page(j);
+            if (j >= kNS && !wait_or_abort(&empty[j % kNS], uint32_t(((j / kNS) - 1) & 1), kPolls, abort_flag))
+                fail = true;
+            else { issue_page(j); issued = j + 1; }
         }
-        if (!tc05::mbar_wait_bounded(&full[st], uint32_t((i / kNS) & 1), kPolls)) timeout = true;
+        if (!fail) fail = !wait_or_abort(&full[st], uint32_t((i / kNS) & 1), kPolls, abort_flag);
+        if (__any_sync(kFull, fail || *abort_flag)) {
+            if (lane == 0) *abort_flag = 1;
+            i_stop = i;
+            break;
+        }
         const uint8_t *pg = stage0 + st * pbytes;
         const int tok0 = (p_begin + i) * L.P + warp * 16;     // token index of row 0 of this warp
         if (pvalid[st] && tok0 < nv && warp * 16 < L.P) {
@@ -238,9 +278,32 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) { accM[nt][k] = 0.f; accQ[nt][k] = 0.f; }
-            {
+            if constexpr (FP8) {
+                // E4M3 bytes [32t, 32t + 32) of tokens g and g + 8; bytes 4ks .. 4ks + 3
+                // hold the coordinates of k = 2t, 2t+1 (low pair) and 2t+8, 2t+9 (high pair)
+                const uint8_t *kcb = pg + L.kc_off;
+                const uint4 u0 = *reinterpret_cast<const uint4 *>(kcb + (pr + g) * 128 + 32 * t);
+                const uint4 u1 = *reinterpret_cast<const uint4 *>(kcb + (pr + g) * 128 + 32 * t + 16);
+                const uint4 u2 = *reinterpret_cast<const uint4 *>(kcb + (pr + g + 8) * 128 + 32 * t);
+                const uint4 u3 = *reinterpret_cast<const uint4 *>(kcb + (pr + g + 8) * 128 + 32 * t + 16);
+                const uint32_t w0[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                const uint32_t w1[8] = {u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    uint32_t A[4];
+                    A[0] = e4m3x2_to_half2_bits(w0[ks]);
+                    A[2] = e4m3x2_to_half2_bits(w0[ks] >> 16);
+                    A[1] = e4m3x2_to_half2_bits(w1[ks]);
+                    A[3] = e4m3x2_to_half2_bits(w1[ks] >> 16);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint2 bb = sB[(nt * 16 + ks) * 32 + lane];
+                        mma16816(accM[nt], A, bb.x, bb.y);
+                    }
+                }
+            } else {
                 // key codes of tokens g and g + 8 for coordinates [32t, 32t + 32)
-                uint32_t kc0[KB], kc1[KB];
+                uint32_t kc0[KB == 8 ? 1 : KB], kc1[KB == 8 ? 1 : KB];
                 const uint8_t *kcb = pg + L.kc_off;
                 if (KB == 4) {
                     const uint4 u0 = *reinterpret_cast<const uint4 *>(kcb + (pr + g) * 64 + 16 * t);
@@ -303,10 +366,12 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     }
                 }
             }
-            const float nk0 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g) * 2));
-            const float nk1 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g + 8) * 2));
-            const float rk0 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kr_off + (pr + g) * 2)) * cq;
-            const float rk1 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kr_off + (pr + g + 8) * 2)) * cq;
+            // FP8 keys store sqrt(d) u: their estimate carries an extra 1/sqrt(d)
+            const float nsc = FP8 ? 0.08838834764831845f : 1.0f;
+            const float nk0 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g) * 2)) * nsc;
+            const float nk1 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g + 8) * 2)) * nsc;
+            const float rk0 = FP8 ? 0.f : h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kr_off + (pr + g) * 2)) * cq;
+            const float rk1 = FP8 ? 0.f : h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kr_off + (pr + g + 8) * 2)) * cq;
             const float nv0 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.vn_off + (pr + g) * 2));
             const float nv1 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.vn_off + (pr + g + 8) * 2));
             const bool ok0 = tok0 + g < nv, ok1 = tok0 + g + 8 < nv;
@@ -429,6 +494,13 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 
     // ---- merge the four warps: m, l per head; O in the rotated basis
     __syncthreads();
+    const bool timeout = *abort_flag != 0;
+    if (timeout) {
+        if (tid == 0)                      // let copies in flight land before the stages are reused
+            for (int p = i_stop; p < issued; ++p)
+                tc05::mbar_wait_bounded(&full[p % kNS], uint32_t((p / kNS) & 1), kPolls);
+        __syncthreads();
+    }
     float *mm = reinterpret_cast<float *>(stage0);               // [4 warps][8 heads]
     float *ll = mm + 32;
     float *oo = ll + 32;                                         // [4 warps][8 heads][128]
@@ -486,17 +558,19 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 
 template <int KB, int VB, int NT>
 size_t dec_smem(int page_bytes) {
-    constexpr int KE = KB == 4 ? 256 : 16, VE = VB == 4 ? 256 : 16;
+    constexpr int KE = key_entries<KB>(), VE = VB == 4 ? 256 : 16;
     // the stage area also holds the final merge: 64 + 4 x 8 x 128 floats
     constexpr int kNS = page_stages<KB>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
     return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 + size_t(NT) * 16 * 32 * 8 +
-           stages + 2 * kNS * 8 + kNS * 4 + 64;
+           stages + (2 * kNS + 1) * 8 + kNS * 4 + 4 + 64;
 }
 
 size_t dec_smem_for(const Layout &L, int G) {
     const bool two = G > 4;
+    if (L.kbits == 8 && L.vbits == 4) return two ? dec_smem<8, 4, 2>(L.page_bytes) : dec_smem<8, 4, 1>(L.page_bytes);
+    if (L.kbits == 8 && L.vbits == 3) return two ? dec_smem<8, 3, 2>(L.page_bytes) : dec_smem<8, 3, 1>(L.page_bytes);
     if (L.kbits == 2 && L.vbits == 4) return two ? dec_smem<2, 4, 2>(L.page_bytes) : dec_smem<2, 4, 1>(L.page_bytes);
     if (L.kbits == 2 && L.vbits == 3) return two ? dec_smem<2, 3, 2>(L.page_bytes) : dec_smem<2, 3, 1>(L.page_bytes);
     if (L.kbits == 4 && L.vbits == 4) return two ? dec_smem<4, 4, 2>(L.page_bytes) : dec_smem<4, 4, 1>(L.page_bytes);
@@ -515,12 +589,22 @@ int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
 
 }  // namespace
 
+namespace {
+std::atomic<uint32_t> g_decode_stall{0};
+}
+
+uint32_t take_decode_stall() { return g_decode_stall.exchange(0); }
+
 // Blocks of the tensor-core decode kernel that fit on one SM (shared memory:
 // 228 KB per SM, 1 KB reserved per block; registers: at most 6 blocks for
 // one query-head tile, 4 for two), or 0 when the configuration is not covered.
+bool dec128_keys_ok(const Layout &L) {
+    return ((L.kbits == 2 || L.kbits == 4) && L.kqjl) || (L.kbits == 8 && !L.kqjl);
+}
+
 int dec128_resident(const Layout &L, int G) {
-    if (L.d != 128 || !L.kqjl || L.P != 64 || G > 8) return 0;
-    if (!((L.kbits == 2 || L.kbits == 4) && (L.vbits == 3 || L.vbits == 4))) return 0;
+    if (L.d != 128 || L.P != 64 || G > 8) return 0;
+    if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return 0;
     const size_t per = dec_smem_for(L, G) + 1024;
     const int by_smem = int(233472 / per);
     const int by_regs = G > 4 ? 4 : 6;
@@ -533,8 +617,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   const AttnShape &s, int G, int n_groups, int n_splits, int split_len, const uint8_t *cache,
                   int64_t num_blocks, float *part_o, float *part_ml, float *logits, int64_t logits_stride,
                   uint32_t *status, cudaStream_t st) {
-    if (L.d != 128 || !L.kqjl || L.P != 64 || G > 8) return -1;
-    if (!((L.kbits == 2 || L.kbits == 4) && (L.vbits == 3 || L.vbits == 4))) return -1;
+    if (L.d != 128 || L.P != 64 || G > 8) return -1;
+    if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return -1;
     if (split_len % L.P) return -1;
     Dec128Args a;
     a.L = L;
@@ -558,12 +642,22 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.logits = logits;
     a.logits_stride = logits_stride;
     a.status = status;
+    a.stall_polls = take_decode_stall();
     const bool two = G > 4;
     if (L.kbits == 2 && L.vbits == 4) return two ? run_dec<2, 4, 2>(a, n_groups, st) : run_dec<2, 4, 1>(a, n_groups, st);
     if (L.kbits == 2 && L.vbits == 3) return two ? run_dec<2, 3, 2>(a, n_groups, st) : run_dec<2, 3, 1>(a, n_groups, st);
     if (L.kbits == 4 && L.vbits == 4) return two ? run_dec<4, 4, 2>(a, n_groups, st) : run_dec<4, 4, 1>(a, n_groups, st);
     if (L.kbits == 4 && L.vbits == 3) return two ? run_dec<4, 3, 2>(a, n_groups, st) : run_dec<4, 3, 1>(a, n_groups, st);
+    if (L.kbits == 8 && L.vbits == 4) return two ? run_dec<8, 4, 2>(a, n_groups, st) : run_dec<8, 4, 1>(a, n_groups, st);
+    if (L.kbits == 8 && L.vbits == 3) return two ? run_dec<8, 3, 2>(a, n_groups, st) : run_dec<8, 3, 1>(a, n_groups, st);
     return -1;
 }
 
+void set_decode_stall(uint32_t polls) { g_decode_stall.store(polls); }
+
 }  // namespace tq
+
+extern "C" int tq_test_stall_next_decode(uint32_t polls) {
+    tq::set_decode_stall(polls);
+    return TQ_OK;
+}

@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "tq_internal.h"
@@ -178,6 +179,19 @@ __device__ __forceinline__ uint16_t f2h_bits(float x) {
 __device__ __forceinline__ float h2f_bits(uint16_t b) {
     __half h = *reinterpret_cast<__half *>(&b);
     return __half2float(h);
+}
+
+// Value of an OCP E4M3 byte (CUDA's fp8 conversion; exact in fp16).
+__device__ __forceinline__ float e4m3_to_float(uint8_t b) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+// Two E4M3 bytes (low byte -> low half) as an fp16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_half2_bits(uint32_t two_bytes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes & 0xFFFFu),
+                                                     __NV_E4M3);
+    return uint32_t(h.x) | (uint32_t(h.y) << 16);
 }
 
 // Read W-bit field i (W in {1, 2, 4, 8}) of a packed token array.

@@ -92,7 +92,9 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
             uint32_t f[E];
 #pragma unroll
             for (int e = 0; e < E; ++e)
-                f[e] = uint32_t(__nv_cvt_float_to_fp8(sqrt_d * (x[e] * inv), __NV_SATFINITE, __NV_E4M3));
+                // the zero vector has u = +0 (not the -0 a sign flip of a zero leaves)
+                f[e] = uint32_t(__nv_cvt_float_to_fp8(n > 0.f ? sqrt_d * (x[e] * inv) : 0.f, __NV_SATFINITE,
+                                                      __NV_E4M3));
             store_codes<D, 8>(page + L.kc_off + pos * L.kc_bpt, lane, f);
             if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kn_off + pos * 2) = nh;
             continue;

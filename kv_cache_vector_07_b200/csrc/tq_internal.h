@@ -129,6 +129,11 @@ int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, 
                      float *lse, float *logits, int64_t logits_stride, uint8_t *ws,
                      size_t ws_bytes, void *stream);
 
+// Testing aid of the tensor-core decode kernel: the poll budget of a wait
+// that nothing completes, taken (and reset to 0) by the next launch.
+uint32_t take_decode_stall();
+void set_decode_stall(uint32_t polls);
+
 // Blocks of the tensor-core decode kernel resident per SM (0: not covered).
 int dec128_resident(const Layout &L, int G);
 

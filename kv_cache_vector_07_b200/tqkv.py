@@ -71,6 +71,7 @@ _sig("tq_score_workspace_bytes", _sz, [ctypes.POINTER(CacheDesc), _i64, _i32, _i
 _sig("tq_score", _i32, [_vp, ctypes.POINTER(CacheDesc), _vp, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
 _sig("tq_read_status", _i32, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)])
 _sig("tq_status_string", ctypes.c_char_p, [_i32])
+_sig("tq_test_stall_next_decode", _i32, [ctypes.c_uint32])
 
 
 class TQError(RuntimeError):
@@ -308,3 +309,10 @@ def read_status(workspace: torch.Tensor, stream=None) -> int:
     flags = ctypes.c_uint32()
     _check(_lib.tq_read_status(_ptr(workspace), _stream(stream), ctypes.byref(flags)), "tq_read_status")
     return int(flags.value)
+
+
+def test_stall_next_decode(polls: int) -> None:
+    """tq_test_stall_next_decode: the next tensor-core decode launch waits
+    `polls` polls on a barrier nothing completes and takes its time-out path
+    (a testing aid for the TQ_DEV_WAIT_TIMEOUT flag; 0 cancels)."""
+    _check(_lib.tq_test_stall_next_decode(int(polls)), "tq_test_stall_next_decode")

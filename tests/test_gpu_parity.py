@@ -217,13 +217,15 @@ def test_long_context_decode_and_prefill_sampled():
     (2, 4, 3, 32, 8, 3000),       # k3v4 preset, G = 4, ragged lengths
     (4, 3, 2, 16, 2, 2500),       # G = 8
     (2, 3, 2, 8, 4, 4100),        # G = 2
+    (8, 4, 3, 32, 8, 2200),       # k8v4 preset (FP8 keys, 4-bit values), G = 4
+    (8, 3, 2, 16, 2, 1900),       # FP8 keys, G = 8
 ])
 def test_decode_tensor_core_every_output(kbits, vbits, B, Hq, H, L):
     d, P = 128, 64
     seed = 60 + kbits * 10 + vbits
     K = synth.outlier_normal((B * L, H, d), seed=seed, device=DEV)
     V = synth.outlier_normal((B * L, H, d), seed=seed + 1, device=DEV)
-    cd = Codec(d, kbits, True, vbits, seed=seed, H=H)
+    cd = Codec(d, kbits, kbits != 8, vbits, seed=seed, H=H)
     bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
     cache, flags = cd.encode(K, V, slots, nblk)
     assert flags == 0
@@ -259,13 +261,14 @@ def test_decode_tensor_core_every_output(kbits, vbits, B, Hq, H, L):
     (4, 4, 16, 2, 40, 2600),      # G = 8, two KV heads
     (2, 2, 2, 1, 70, 1500),       # G = 2: 64 positions per block
     (3, 4, 8, 2, 33, 4096),       # G = 4, one position in the last block
+    (8, 4, 16, 4, 24, 1500),      # k8v4: FP8 keys, each chunk position as a decode query group
 ])
 def test_prefill_tensor_core_every_output(kbits, vbits, Hq, H, C, L):
     d, P = 128, 64
     seed = 40 + kbits * 10 + vbits
     K = synth.outlier_normal((L, H, d), seed=seed, device=DEV)
     V = synth.outlier_normal((L, H, d), seed=seed + 1, device=DEV)
-    cd = Codec(d, kbits, True, vbits, seed=seed, H=H)
+    cd = Codec(d, kbits, kbits != 8, vbits, seed=seed, H=H)
     bt, slots, nblk = synth.contiguous_block_table(1, L, P, device=DEV, shuffle_seed=seed)
     cache, flags = cd.encode(K, V, slots, nblk)
     assert flags == 0
@@ -383,7 +386,9 @@ def test_search_configurations_every_output(d, kbits, kqjl, n_db, n_q, k, qscale
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("d,kbits,kqjl,vbits,P,Hq,H", [(8, 2, True, 1, 8, 2, 1), (16, 1, True, 2, 16, 8, 1),
                                                        (64, 3, True, 2, 16, 4, 2), (256, 4, False, 3, 32, 1, 1),
-                                                       (128, 4, True, 4, 16, 8, 1), (32, 2, True, 4, 8, 6, 3)])
+                                                       (128, 4, True, 4, 16, 8, 1), (32, 2, True, 4, 8, 6, 3),
+                                                       (64, 8, False, 4, 16, 4, 2), (256, 8, False, 2, 32, 8, 1),
+                                                       (128, 8, False, 4, 64, 3, 1)])
 def test_small_dims_ragged_sequences(d, kbits, kqjl, vbits, P, Hq, H):
     seqs = [0, 1, 37, 3 * P + 5]
     B, Lmax = len(seqs), max(seqs)
@@ -460,6 +465,35 @@ def test_block_table_out_of_range_is_flagged():
     ws = torch.zeros(tqkv.decode_workspace_bytes(cd.desc, 1, 1, 20), dtype=torch.uint8, device=DEV)
     tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, 20, cache, workspace=ws)
     assert tqkv.read_status(ws) & tqkv.TQ_DEV_BLOCK_RANGE
+
+
+def test_decode_wait_timeout_is_flagged_and_context_survives():
+    """A bounded on-chip wait that runs out (a barrier nothing completes, set
+    up through the testing aid) sets TQ_DEV_WAIT_TIMEOUT, returns promptly,
+    leaves nothing in flight, and the next call on the same context is exact."""
+    import time
+    cd = Codec(128, 2, True, 4, seed=19, H=2)
+    B, Hq, L = 2, 8, 700
+    K = synth.outlier_normal((B * L, 2, 128), seed=191, device=DEV)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, 64, device=DEV, shuffle_seed=19)
+    cache, flags = cd.encode(K, K, slots, nblk)
+    assert flags == 0
+    Q = synth.normal((B, Hq, 128), seed=192, device=DEV)
+    seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    ws = torch.zeros(tqkv.decode_workspace_bytes(cd.desc, B, Hq, L), dtype=torch.uint8, device=DEV)
+    ref = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, workspace=ws)
+    torch.cuda.synchronize()
+    assert tqkv.read_status(ws) == 0
+    tqkv.test_stall_next_decode(2000)
+    t0 = time.perf_counter()
+    tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, workspace=ws)
+    flags = tqkv.read_status(ws)
+    assert time.perf_counter() - t0 < 5.0
+    assert flags & tqkv.TQ_DEV_WAIT_TIMEOUT
+    again = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, workspace=ws)
+    torch.cuda.synchronize()
+    assert tqkv.read_status(ws) == 0
+    assert torch.equal(again, ref)
 
 
 # ---------------------------------------------------------------------------

@@ -462,3 +462,26 @@ def test_fp8_margin_matches_direct_distance_to_rounding_midpoints():
     a = math.sqrt(d) * (X @ R.T) / np.linalg.norm(X, axis=1)[:, None]
     mg = np.min(np.abs(np.abs(a)[:, :, None] - mids[None, None, :]), axis=2) / math.sqrt(d)
     assert np.allclose(enc.umargin, mg, rtol=0, atol=1e-13)
+
+
+def test_attend_with_fp8_keys_equals_textbook_softmax_on_exactly_coded_kv():
+    """The FP8-key estimator nhat <Rq, e4m3(code)> / sqrt(d) on keys that the
+    codes represent exactly: attention equals scipy's softmax(QK^T/sqrt(d))V."""
+    d, L, nq = 128, 400, 4
+    rng = np.random.default_rng(8)
+    Pk, Pv = O.make_params(d, 8, 33, with_S=False), O.make_params(d, 4, 34, with_S=False)
+    codes = rng.integers(0, 0x7F, (L, d)).astype(np.uint8) | (rng.integers(0, 2, (L, d)).astype(np.uint8) << 7)
+    kn = np.array([O.round_fp16(v) for v in rng.uniform(1.0, 40.0, L)])
+    vidx = rng.integers(0, 16, (L, d)).astype(np.uint8)
+    vn = np.array([O.round_fp16(v) for v in rng.uniform(0.5, 8.0, L)])
+    vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    R = scipy.linalg.hadamard(d).astype(np.float64) @ np.diag(Pk.signs.astype(np.float64)) / math.sqrt(d)
+    Kx = (kn[:, None] * vals / math.sqrt(d)) @ R
+    Vx = _exact_from_codes(Pv, vidx, vn)
+    Ek, Ev = O.Encoded(8, False, codes, kn), O.Encoded(4, False, vidx, vn)
+    Q = rng.standard_normal((nq, d))
+    out, lse, logits = O.attend(Q, Pk, Ek, Pv, Ev, want_logits=True)
+    lg = Q @ Kx.T / math.sqrt(d)
+    assert np.allclose(logits, lg, atol=1e-11, rtol=0)
+    assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-11, rtol=0)
+    assert np.allclose(lse, scipy.special.logsumexp(lg, axis=1), atol=1e-11, rtol=0)
