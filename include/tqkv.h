@@ -165,7 +165,8 @@ int tq_encode(const tq_params *kp, const tq_params *vp, const tq_cache_desc *des
  * then softmax and o = R_v^T sum_t p_t nhat_v,t c_v[code_v,t], bf16 (RNE).
  * Pages: "What is TurboQuant?" ("Stage 2": unbiased inner products; the 8x
  * attention-logit figure), ai-work-lab overview (attention on compressed
- * keys).  Requires kbits in 1..4 (FP8-key decode is not provided).
+ * keys).  FP8 keys (kbits = 8, preset k8v4) score nhat <Rq, e4m3(code)> / sqrt(d)
+ * ("What is TurboQuant?", vLLM presets: k8v4 = FP8 keys + 4-bit values).
  * workspace: >= tq_decode_workspace_bytes(desc, B, Hq, max_seq_len). */
 size_t tq_decode_workspace_bytes(const tq_cache_desc *desc, int B, int Hq, int max_seq_len);
 int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc,

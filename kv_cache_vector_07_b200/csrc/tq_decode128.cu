@@ -44,7 +44,13 @@ __host__ __device__ constexpr int page_stages() { return KB == 4 ? 2 : 3; }
 // Key pair-table entries: two 4-bit codes (256), two 2-bit codes (16); FP8
 // keys need no table (each E4M3 byte converts to fp16 exactly).
 template <int KB>
-__host__ __device__ constexpr int key_entries() { return KB == 4 ? 256 : (KB == 2 ? 16 : 0); }
+__host__ __device__ constexpr int key_entries() { return KB == 4 ? 256 : 0; }
+// Query-operand k-steps: 2-bit keys take a sign plane and a sign x magnitude
+// plane (8 each) plus 8 for the QJL signs; 4-bit keys 8 + 8; FP8 keys 8.
+template <int KB>
+__host__ __device__ constexpr int query_ksteps() { return KB == 2 ? 24 : (KB == 4 ? 16 : 8); }
+template <int KB>
+__host__ __device__ constexpr int qjl_kstep0() { return KB == 2 ? 16 : 8; }
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 struct Dec128Args {
@@ -116,9 +122,22 @@ __host__ __device__ constexpr int key_copies() { return B == 4 ? 8 : (B == 2 ? 1
 template <int B>
 __host__ __device__ constexpr int val_copies() { return B == 4 ? 8 : 32; }
 
-// Value table entry e for this lane: half2(lv[e & mask], lv[e >> shift]).
-template <int VC>
-__device__ __forceinline__ uint32_t lut(const uint32_t *tab_lane, uint32_t e) { return tab_lane[e * VC]; }
+// Table lookups with the index taken straight from a code word: field
+// `pos` (width W bits, at bit W * pos) of `w`, as a byte offset into a table
+// of STRIDE-byte entries (STRIDE = copies x entry size), ORed with the
+// lane's copy offset (which lies below STRIDE): one shift and one LOP3.
+template <int W, int STRIDE>
+__device__ __forceinline__ uint32_t field_offset(uint32_t w, int pos, uint32_t lane_off) {
+    constexpr int SH = __builtin_ctz(STRIDE);
+    constexpr uint32_t MASK = ((1u << W) - 1u) << SH;
+    const int r = W * pos - SH;
+    const uint32_t x = r >= 0 ? (w >> r) : (w << (-r));
+    return (x & MASK) | lane_off;
+}
+template <typename T>
+__device__ __forceinline__ T lds_at(const void *base, uint32_t byte_off) {
+    return *reinterpret_cast<const T *>(reinterpret_cast<const uint8_t *>(base) + byte_off);
+}
 
 template <int KB, int VB, int NT>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
@@ -129,11 +148,12 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     constexpr int KE = key_entries<KB>();           // key pair-table entries (two codes)
     constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
     constexpr int KC = key_copies<KB>(), VC = val_copies<VB>();
+    constexpr int NKS = query_ksteps<KB>(), QK0 = qjl_kstep0<KB>();
     extern __shared__ __align__(16) uint8_t smem[];
     uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][KC copies] {hi pair, lo pair}
     uint32_t *lutV = reinterpret_cast<uint32_t *>(lutK + KE * KC);   // [VE][VC copies]
-    uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * VC);          // [NT][16][32]
-    uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * 16 * 32);
+    uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * VC);          // [NT][NKS][32]
+    uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * NKS * 32);
     const Layout &L = a.L;
     const int pbytes = L.page_bytes;
     const int stage_area = max(kNS * pbytes, (64 + 4 * 8 * 128) * 4);
@@ -160,10 +180,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     for (int i = tid; i < KE * KC; i += 128) {
         // centroid pair as fp16 hi + lo (the pair's fp32 values to ~22 bits)
         const int e = i / KC;
-        float c0, c1;
-        if (KB == 4) { c0 = a.k_lv[e & 15]; c1 = a.k_lv[e >> 4]; }
-        else { c0 = a.k_lv[e & 3]; c1 = a.k_lv[(e >> 2) & 3]; }
-        if (FP8) continue;
+        const float c0 = a.k_lv[e & 15], c1 = a.k_lv[e >> 4];
         const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
         lutK[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
     }
@@ -174,27 +191,49 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
         else { lo = a.v_lv[e & 3]; hi = a.v_lv[(e >> 2) & 3]; }       // magnitudes (positive half)
         lutV[i] = h2bits(lo, hi);
     }
+    // 2-bit keys: stored code (n, m) = (negative, larger magnitude) has level
+    // (1 - 2n)(c_0 + m (c_1 - c_0)); the key side of the product is then two
+    // exact planes, s = +-1 and 2 s m in {0, +-2}, and the constants c_0 and
+    // (c_1 - c_0)/2 ride on the query operand, scaled by 2^kexp into [0.5, 1)
+    // so that their fp16 hi + lo split keeps its precision.
+    float plane_f[2] = {1.f, 1.f}, kscale = 1.f;
+    if (KB == 2) {
+        const float c0 = a.k_lv[0], c1 = a.k_lv[1];
+        int e2;
+        frexpf(fmaxf(fabsf(c0), fabsf(0.5f * (c1 - c0))), &e2);
+        plane_f[0] = ldexpf(c0, -e2);
+        plane_f[1] = ldexpf(0.5f * (c1 - c0), -e2);
+        kscale = ldexpf(1.f, e2);
+    }
     {
         const float qs = 0.08838834764831845f * 1.4426950408889634f;   // 1/sqrt(128) * log2(e)
-        for (int i = tid; i < NT * 16 * 32; i += 128) {
-            const int ln = i & 31, ks = (i >> 5) & 15, nt = i >> 9;
+        for (int i = tid; i < NT * NKS * 32; i += 128) {
+            const int ln = i & 31, ks = (i >> 5) % NKS, nt = (i >> 5) / NKS;
             const int gg = ln >> 2, tt = ln & 3;
             const int hd = 4 * nt + (gg >> 1);
             const bool lo_part = (gg & 1) != 0;
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            if (hd < G && !(FP8 && ks >= 8)) {
-                const float *src = ks < 8 ? a.qr + (row0 + hd) * 128 : a.w + (row0 + hd) * 128;
+            if (hd < G) {
+                const float *src = ks < QK0 ? a.qr + (row0 + hd) * 128 : a.w + (row0 + hd) * 128;
                 int c[4];
-                if (ks < 8) {
+                float f = 1.f;
+                if (ks >= QK0) {
+                    const int j = 2 * (ks - QK0);
+                    c[0] = 32 * tt + j; c[1] = 32 * tt + j + 16; c[2] = 32 * tt + j + 1; c[3] = 32 * tt + j + 17;
+                } else if (KB == 2) {
+                    // plane k-step kk: word kk / 4 of the thread's 32 coordinates, pair
+                    // i0 = 2 (kk % 4): coordinates (i0, i0 + 8) then (i0 + 1, i0 + 9)
+                    const int kk = ks & 7;
+                    const int base = 32 * tt + 16 * (kk >> 2) + 2 * (kk & 3);
+                    c[0] = base; c[1] = base + 8; c[2] = base + 1; c[3] = base + 9;
+                    f = plane_f[ks >> 3];
+                } else {
                     const int base = 32 * tt + 4 * ks;
                     c[0] = base; c[1] = base + 1; c[2] = base + 2; c[3] = base + 3;
-                } else {
-                    const int j = 2 * (ks - 8);
-                    c[0] = 32 * tt + j; c[1] = 32 * tt + j + 16; c[2] = 32 * tt + j + 1; c[3] = 32 * tt + j + 17;
                 }
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const float x = src[c[k]] * qs;
+                    const float x = src[c[k]] * qs * f;
                     const float h = __half2float(__float2half_rn(x));
                     v[k] = lo_part ? (x - h) : h;
                 }
@@ -240,8 +279,8 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     if (tid == 0 && !*abort_flag)
         for (int i = 0; i < kNS - 1 && i < n_pages; ++i) { issue_page(i); issued = i + 1; }
 
-    const uint2 *lutK_l = lutK + (lane & (KC - 1));
-    const uint32_t *lutV_l = lutV + (lane & (VC - 1));
+    const uint32_t vlane_off = uint32_t(lane & (VC - 1)) * 4u;     // this lane's value-table copy
+    const uint32_t klane_off = uint32_t(lane & (KC - 1)) * 8u;     // this lane's key-table copy
     const float cq = 1.2533141373155003f / 128.0f;       // sqrt(pi/2) / m
     float m_run[NT], l_run[NT];
 #pragma unroll
@@ -297,57 +336,67 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     A[3] = e4m3x2_to_half2_bits(w1[ks] >> 16);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bb = sB[(nt * 16 + ks) * 32 + lane];
+                        const uint2 bb = sB[(nt * NKS + ks) * 32 + lane];
                         mma16816(accM[nt], A, bb.x, bb.y);
                     }
                 }
             } else {
-                // key codes of tokens g and g + 8 for coordinates [32t, 32t + 32)
-                uint32_t kc0[KB == 8 ? 1 : KB], kc1[KB == 8 ? 1 : KB];
                 const uint8_t *kcb = pg + L.kc_off;
-                if (KB == 4) {
-                    const uint4 u0 = *reinterpret_cast<const uint4 *>(kcb + (pr + g) * 64 + 16 * t);
-                    const uint4 u1 = *reinterpret_cast<const uint4 *>(kcb + (pr + g + 8) * 64 + 16 * t);
-                    kc0[0] = u0.x; kc0[1] = u0.y; kc0[KB > 2 ? 2 : 0] = u0.z; kc0[KB > 2 ? 3 : 1] = u0.w;
-                    kc1[0] = u1.x; kc1[1] = u1.y; kc1[KB > 2 ? 2 : 0] = u1.z; kc1[KB > 2 ? 3 : 1] = u1.w;
-                } else {
+                if constexpr (KB == 2) {
+                    // 2-bit codes of tokens g and g + 8 for coordinates [32t, 32t + 32): two words
+                    // each; coordinate i of a word sits at bits 2i (magnitude) and 2i + 1 (sign)
                     const uint2 u0 = *reinterpret_cast<const uint2 *>(kcb + (pr + g) * 32 + 8 * t);
                     const uint2 u1 = *reinterpret_cast<const uint2 *>(kcb + (pr + g + 8) * 32 + 8 * t);
-                    kc0[0] = u0.x; kc0[1] = u0.y;
-                    kc1[0] = u1.x; kc1[1] = u1.y;
-                }
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    uint32_t e[4];
-                    if (KB == 4) {
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t w0 = (ks >> 2) ? u0.y : u0.x, w1 = (ks >> 2) ? u1.y : u1.x;
+                        const int sh = 14 - 4 * (ks & 3);       // coordinate i0 -> bits 14, 15 (and 30, 31)
+                        uint32_t x[4];
+                        x[0] = w0 << sh;
+                        x[1] = w1 << sh;
+                        x[2] = w0 << (sh - 2);
+                        x[3] = w1 << (sh - 2);
+                        uint32_t As[4], Am[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            As[r] = (x[r] & 0x80008000u) | 0x3C003C00u;   // +-1
+                            Am[r] = x[r] & 0xC000C000u;                    // 0 or +-2
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint2 bs = sB[(nt * NKS + ks) * 32 + lane];
+                            const uint2 bm = sB[(nt * NKS + 8 + ks) * 32 + lane];
+                            mma16816(accM[nt], As, bs.x, bs.y);
+                            mma16816(accM[nt], Am, bm.x, bm.y);
+                        }
+                    }
+                } else {
+                    // 4-bit codes of tokens g and g + 8 for coordinates [32t, 32t + 32)
+                    const uint4 u0 = *reinterpret_cast<const uint4 *>(kcb + (pr + g) * 64 + 16 * t);
+                    const uint4 u1 = *reinterpret_cast<const uint4 *>(kcb + (pr + g + 8) * 64 + 16 * t);
+                    const uint32_t kc0[4] = {u0.x, u0.y, u0.z, u0.w}, kc1[4] = {u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
                         // bytes 2ks, 2ks+1 of the thread's 16 code bytes: coordinate pairs
                         const uint32_t w0 = kc0[ks >> 1], w1 = kc1[ks >> 1];
-                        const int sh = 16 * (ks & 1);
-                        e[0] = (w0 >> sh) & 0xFF;
-                        e[2] = (w0 >> (sh + 8)) & 0xFF;
-                        e[1] = (w1 >> sh) & 0xFF;
-                        e[3] = (w1 >> (sh + 8)) & 0xFF;
-                    } else {
-                        // byte ks: two 4-bit pair indices
-                        const uint32_t w0 = kc0[ks >> 2], w1 = kc1[ks >> 2];
-                        const int sh = 8 * (ks & 3);
-                        e[0] = (w0 >> sh) & 0xF;
-                        e[2] = (w0 >> (sh + 4)) & 0xF;
-                        e[1] = (w1 >> sh) & 0xF;
-                        e[3] = (w1 >> (sh + 4)) & 0xF;
-                    }
-                    uint32_t Ah[4], Al[4];
+                        const int bp = 2 * (ks & 1);
+                        uint2 v[4];
+                        v[0] = lds_at<uint2>(lutK, field_offset<8, KC * 8>(w0, bp, klane_off));
+                        v[2] = lds_at<uint2>(lutK, field_offset<8, KC * 8>(w0, bp + 1, klane_off));
+                        v[1] = lds_at<uint2>(lutK, field_offset<8, KC * 8>(w1, bp, klane_off));
+                        v[3] = lds_at<uint2>(lutK, field_offset<8, KC * 8>(w1, bp + 1, klane_off));
+                        uint32_t Ah[4], Al[4];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const uint2 v = lutK_l[e[r] * KC];
-                        Ah[r] = v.x;
-                        Al[r] = v.y;
-                    }
+                        for (int r = 0; r < 4; ++r) {
+                            Ah[r] = v[r].x;
+                            Al[r] = v[r].y;
+                        }
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bb = sB[(nt * 16 + ks) * 32 + lane];
-                        mma16816(accM[nt], Ah, bb.x, bb.y);
-                        mma16816(accM[nt], Al, bb.x, bb.y);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint2 bb = sB[(nt * NKS + ks) * 32 + lane];
+                            mma16816(accM[nt], Ah, bb.x, bb.y);
+                            mma16816(accM[nt], Al, bb.x, bb.y);
+                        }
                     }
                 }
                 const uint32_t s0 = *reinterpret_cast<const uint32_t *>(pg + L.ks_off + (pr + g) * 16 + 4 * t);
@@ -361,13 +410,13 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     A[3] = sign_pair(s1, 2 * ks + 1);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bb = sB[(nt * 16 + 8 + ks) * 32 + lane];
+                        const uint2 bb = sB[(nt * NKS + QK0 + ks) * 32 + lane];
                         mma16816(accQ[nt], A, bb.x, bb.y);
                     }
                 }
             }
             // FP8 keys store sqrt(d) u: their estimate carries an extra 1/sqrt(d)
-            const float nsc = FP8 ? 0.08838834764831845f : 1.0f;
+            const float nsc = FP8 ? 0.08838834764831845f : kscale;
             const float nk0 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g) * 2)) * nsc;
             const float nk1 = h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kn_off + (pr + g + 8) * 2)) * nsc;
             const float rk0 = FP8 ? 0.f : h2f_bits(*reinterpret_cast<const uint16_t *>(pg + L.kr_off + (pr + g) * 2)) * cq;
@@ -425,9 +474,12 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     const float x1 = __shfl_sync(kFull, alpha[NT - 1], hd & 3);
                     ah[c] = hd < 4 ? x0 : x1;
                 }
+                // most tiles leave every running maximum unchanged: skip the rescale then
+                if (__any_sync(kFull, ah[0] != 1.f || ah[1] != 1.f)) {
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    O[mt][0] *= ah[0]; O[mt][1] *= ah[1]; O[mt][2] *= ah[0]; O[mt][3] *= ah[1];
+                    for (int mt = 0; mt < 8; ++mt) {
+                        O[mt][0] *= ah[0]; O[mt][1] *= ah[1]; O[mt][2] *= ah[0]; O[mt][3] *= ah[1];
+                    }
                 }
             }
             // ---------------- values: thread coordinates [16g, 16g + 16), tokens 2t, 2t+1, 2t+8, 2t+9
@@ -452,10 +504,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                         for (int k = 0; k < 4; ++k) {
                             const int mt = 4 * wi + k;          // coordinates 16g + 2mt, +1
                             uint32_t A[4];
-                            A[0] = lut<VC>(lutV_l, (eAB >> (8 * k)) & 0xFF);
-                            A[1] = lut<VC>(lutV_l, (oAB >> (8 * k)) & 0xFF);
-                            A[2] = lut<VC>(lutV_l, (eCD >> (8 * k)) & 0xFF);
-                            A[3] = lut<VC>(lutV_l, (oCD >> (8 * k)) & 0xFF);
+                            A[0] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(eAB, k, vlane_off));
+                            A[1] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(oAB, k, vlane_off));
+                            A[2] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(eCD, k, vlane_off));
+                            A[3] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(oCD, k, vlane_off));
                             mma16816(O[mt], A, b0, b1);
                         }
                     }
@@ -479,10 +531,14 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                     for (int mt = 0; mt < 8; ++mt) {
                         const int e0 = 2 * mt, e1 = 2 * mt + 1;     // coordinates 16g + e
                         uint32_t A[4];
-                        A[0] = lut<VC>(lutV_l, (eAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e0)) & 0x80008000u);
-                        A[1] = lut<VC>(lutV_l, (oAB >> (4 * mt)) & 0xF) ^ ((zAB << (15 - e1)) & 0x80008000u);
-                        A[2] = lut<VC>(lutV_l, (eCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e0)) & 0x80008000u);
-                        A[3] = lut<VC>(lutV_l, (oCD >> (4 * mt)) & 0xF) ^ ((zCD << (15 - e1)) & 0x80008000u);
+                        A[0] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(eAB, mt, vlane_off)) ^
+                               ((zAB << (15 - e0)) & 0x80008000u);
+                        A[1] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(oAB, mt, vlane_off)) ^
+                               ((zAB << (15 - e1)) & 0x80008000u);
+                        A[2] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(eCD, mt, vlane_off)) ^
+                               ((zCD << (15 - e0)) & 0x80008000u);
+                        A[3] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(oCD, mt, vlane_off)) ^
+                               ((zCD << (15 - e1)) & 0x80008000u);
                         mma16816(O[mt], A, b0, b1);
                     }
                 }
@@ -563,18 +619,28 @@ size_t dec_smem(int page_bytes) {
     constexpr int kNS = page_stages<KB>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
-    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 + size_t(NT) * 16 * 32 * 8 +
+    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 +
+           size_t(NT) * query_ksteps<KB>() * 32 * 8 +
            stages + (2 * kNS + 1) * 8 + kNS * 4 + 4 + 64;
 }
 
-size_t dec_smem_for(const Layout &L, int G) {
-    const bool two = G > 4;
-    if (L.kbits == 8 && L.vbits == 4) return two ? dec_smem<8, 4, 2>(L.page_bytes) : dec_smem<8, 4, 1>(L.page_bytes);
-    if (L.kbits == 8 && L.vbits == 3) return two ? dec_smem<8, 3, 2>(L.page_bytes) : dec_smem<8, 3, 1>(L.page_bytes);
-    if (L.kbits == 2 && L.vbits == 4) return two ? dec_smem<2, 4, 2>(L.page_bytes) : dec_smem<2, 4, 1>(L.page_bytes);
-    if (L.kbits == 2 && L.vbits == 3) return two ? dec_smem<2, 3, 2>(L.page_bytes) : dec_smem<2, 3, 1>(L.page_bytes);
-    if (L.kbits == 4 && L.vbits == 4) return two ? dec_smem<4, 4, 2>(L.page_bytes) : dec_smem<4, 4, 1>(L.page_bytes);
-    return two ? dec_smem<4, 3, 2>(L.page_bytes) : dec_smem<4, 3, 1>(L.page_bytes);
+
+// Blocks of one instantiation resident per SM, from the occupancy calculator
+// (registers, shared memory and the 128-thread block).
+// The kernel only covers d = 128 with 64-token pages, so the page size (and
+// the answer) is fixed per instantiation and computed once.
+template <int KB, int VB, int NT>
+int dec_resident(int page_bytes) {
+    static std::atomic<int> cached{-1};
+    const int c = cached.load();
+    if (c >= 0) return c;
+    const size_t smem = dec_smem<KB, VB, NT>(page_bytes);
+    auto kern = dec128_kernel<KB, VB, NT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, smem) != cudaSuccess) return 0;
+    cached.store(n);
+    return n;
 }
 
 template <int KB, int VB, int NT>
@@ -605,10 +671,13 @@ bool dec128_keys_ok(const Layout &L) {
 int dec128_resident(const Layout &L, int G) {
     if (L.d != 128 || L.P != 64 || G > 8) return 0;
     if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return 0;
-    const size_t per = dec_smem_for(L, G) + 1024;
-    const int by_smem = int(233472 / per);
-    const int by_regs = G > 4 ? 4 : 6;
-    return by_smem < by_regs ? by_smem : by_regs;
+    const bool two = G > 4;
+    const int pb = L.page_bytes;
+#define TQ_DEC_RES(K, V) \
+    if (L.kbits == K && L.vbits == V) return two ? dec_resident<K, V, 2>(pb) : dec_resident<K, V, 1>(pb);
+    TQ_DEC_RES(2, 4) TQ_DEC_RES(2, 3) TQ_DEC_RES(4, 4) TQ_DEC_RES(4, 3) TQ_DEC_RES(8, 4) TQ_DEC_RES(8, 3)
+#undef TQ_DEC_RES
+    return 0;
 }
 
 // Tensor-core attention for d = 128; returns -1 when the configuration is not
