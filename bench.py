@@ -41,13 +41,14 @@ import torch  # noqa: E402
 
 METRIC = "KV vectors encoded/s + decode-attn keys scored/s; % HBM roofline (1 B200)"
 WORKLOAD_METRICS = {"step": METRIC, "encode": "KV vectors encoded/s", "decode32k": "decode-attn keys scored/s",
-                    "decode_k8v4": "decode-attn keys scored/s",
+                    "decode_k8v4": "decode-attn keys scored/s", "decode_step": "decode-attn keys scored/s",
                     "longctx": "decode + prefill (query-head, key) pairs/s",
                     "search": "(query, database vector) pairs scored/s (top-10 search)"}
 UNIT_NOTES = {"step": "units = KV vectors encoded (two presets) + (query-head, key) pairs scored",
               "encode": "units = KV vectors encoded (two presets)",
               "decode32k": "units = (query-head, key) pairs scored",
               "decode_k8v4": "units = (query-head, key) pairs scored",
+              "decode_step": "units = (query-head, key) pairs scored (the new tokens' write included in the time)",
               "longctx": "units = (query-head, key) pairs scored in the decode step and the prefill chunk",
               "search": "units = (query, database vector) pairs scored"}
 FALLBACK_HBM_GBS = 6650.0
@@ -350,6 +351,36 @@ class Decode32kK8V4(Decode32k):
                                 "batch": batch, "seq_len": seq_len, "n_q_heads": 32, "n_kv_heads": 8}}
 
 
+class Decode32kStep(Decode32k):
+    """The k3v4 decode step with the new token's write fused in (tq_decode_step):
+    each sequence's token at position 32,767 is compressed into the cache and
+    all 32 query heads attend over the 32,768 tokens."""
+
+    def __init__(self, dev, batch=32, seq_len=32768, **kw):
+        super().__init__(dev, batch=batch, seq_len=seq_len, **kw)
+        from kv_cache_vector_07_b200 import synth
+        self.Kn = synth.outlier_normal((self.B, self.H, self.d), seed=23, device=dev)
+        self.Vn = synth.outlier_normal((self.B, self.H, self.d), seed=24, device=dev)
+        self.new_slots = (self.bt[:, -1].to(torch.int64) * self.P + (self.L - 1) % self.P).to(torch.int32)
+
+    def ops(self):
+        tq = self.tq
+
+        def f():
+            tq.decode_step(self.kp, self.vp, self.desc, self.Kn, self.Vn, self.new_slots, self.Q, self.bt, self.seq,
+                           self.L, self.cache, out=self.out, workspace=self.ws)
+        work = self.B * self.H * self.L * self.per_tok + 2 * self.Q.numel() * 2 + 2 * 2 * self.Kn.numel()
+        return [Op("decode_step_k3v4", f, self.B * self.Hq * self.L, "(query-head, key) pairs scored", "hbm", work,
+                   "tq_decode_step (new-token encode + query prep in one launch, dec128 tensor-core decode, combine)",
+                   3, extra={"new_tokens_written": self.B * self.H * 2})]
+
+    @staticmethod
+    def config(batch=32, seq_len=32768, **_):
+        return {"decode_step": {"what": f"B={batch} x Hq=32/Hkv=8 x {seq_len} tokens x d=128, k3v4: write the new "
+                                        "token's K/V, then attend (fused decode step)",
+                                "batch": batch, "seq_len": seq_len}}
+
+
 class LongCtx:
     """Config: B=1, Hq=32 over Hkv=4, 262,144 tokens, K 2-bit + QJL, V 3-bit;
     one decode step plus one 2,048-query prefill chunk (causal inside)."""
@@ -505,10 +536,11 @@ class Search:
 
 
 # workload -> (classes in the timed step, classes timed as parts)
-WORKLOADS = {"step": ((WritePath, Decode32k), (Decode32kK8V4, LongCtx, Search)),
+WORKLOADS = {"step": ((WritePath, Decode32k), (Decode32kK8V4, Decode32kStep, LongCtx, Search)),
              "encode": ((WritePath,), ()),
              "decode32k": ((Decode32k,), ()),
              "decode_k8v4": ((Decode32kK8V4,), ()),
+             "decode_step": ((Decode32kStep,), ()),
              "longctx": ((LongCtx,), ()),
              "search": ((Search,), ())}
 WORKLOAD_NAMES = {"step": "write path (k8v4 and K4+QJL/V4, 8 x 8 x 32768 x 128 bf16) + k3v4 GQA decode "
@@ -516,6 +548,7 @@ WORKLOAD_NAMES = {"step": "write path (k8v4 and K4+QJL/V4, 8 x 8 x 32768 x 128 b
                   "encode": "write path 8 x 8 x 32768 x 128 bf16, presets k8v4 and K4+QJL/V4",
                   "decode32k": "k3v4 GQA decode 32 x 32/8 heads x 32768 x 128",
                   "decode_k8v4": "k8v4 GQA decode 32 x 32/8 heads x 32768 x 128 (FP8 keys)",
+                  "decode_step": "fused k3v4 decode step (write the new token, attend) 32 x 32/8 heads x 32768",
                   "longctx": "long-context 1 x 32/4 heads x 262144: decode + 2048-query prefill",
                   "search": "search 1,000,000 x 1024, 1024 queries, top-10"}
 
@@ -803,8 +836,9 @@ def _oracle_sample(workload: str, n: int, small: bool):
         t1, u1 = _oracle_encode_slice(n, 4096 if small else 32768)
         t2, u2 = _oracle_attend_slice("decode32k", n, 4096 if small else 32768)
         return t1 + t2, u1 + u2
-    if workload in ("decode32k", "decode_k8v4"):
-        return _oracle_attend_slice(workload, n, 8192 if small else 32768)
+    if workload in ("decode32k", "decode_k8v4", "decode_step"):
+        return _oracle_attend_slice("decode32k" if workload == "decode_step" else workload, n,
+                                    8192 if small else 32768)
     if workload == "longctx":
         return _oracle_attend_slice("longctx", n, 8192 if small else 65536)
     return _oracle_attend_slice("search", n, 5000 if small else 20000)
@@ -817,11 +851,12 @@ SAMPLE_TEXT = {
             "presets) plus 4 query heads scored over {L} k3v4 keys (encode of the decode slice untimed)",
     "decode32k": "slices of one KV head: 4 query heads over {L} k3v4 keys (encode untimed)",
     "decode_k8v4": "slices of one KV head: 4 query heads over {L} k8v4 keys (encode untimed)",
+    "decode_step": "slices of one KV head: 4 query heads over {L} k3v4 keys (encode untimed)",
     "longctx": "slices of one KV head: 8 query heads over {L} keys (K 2-bit + QJL, V 3-bit; encode untimed)",
     "search": "slices: 4 queries over {L} oracle-encoded d=1024 vectors (encode untimed)",
 }
 SAMPLE_L = {"encode": (4096, 32768), "step": (4096, 32768), "decode32k": (8192, 32768),
-            "decode_k8v4": (8192, 32768), "longctx": (8192, 65536),
+            "decode_k8v4": (8192, 32768), "decode_step": (8192, 32768), "longctx": (8192, 65536),
             "search": (5000, 20000)}
 
 

@@ -176,6 +176,24 @@ int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq_cache_desc
                    int64_t logits_stride, void *workspace, size_t workspace_bytes,
                    void *stream);
 
+/* One decode step with the new token's write fused in: for every sequence b,
+ * K_new/V_new [B][n_kv_heads][d] (device, bf16) are compressed into cache
+ * slot slot_mapping[b] (< 0 skips the write; >= num_blocks * page_tokens
+ * skips it and sets TQ_DEV_SLOT_RANGE), exactly as tq_encode would, and then
+ * the queries Q attend over seq_lens[b] tokens that include it, exactly as
+ * tq_decode_attn.  The write shares the launch that prepares the queries
+ * (a warp per vector; QJL signs from an fp32 projection by S), so the step
+ * takes the same three launches as tq_decode_attn alone.  Pages: "What is
+ * TurboQuant?" (the cache dtype is chosen per vLLM preset and the serving
+ * engine writes each new token as it decodes; "vLLM: available by switching
+ * --kv-cache-dtype").  Workspace: tq_decode_workspace_bytes(desc, B, Hq,
+ * max_seq_len). */
+int tq_decode_step(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc, const void *K_new,
+                   const void *V_new, const int32_t *slot_mapping, const void *Q, int B, int Hq,
+                   const int32_t *block_table, int max_blocks, const int32_t *seq_lens, int max_seq_len,
+                   void *cache, int64_t num_blocks, void *out, float *lse, float *logits,
+                   int64_t logits_stride, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Decode attention without any device allocation, for callers that cannot
  * allocate device memory (an engine that keeps all device memory in its own
  * pool and forbids other allocations, a plug-in handed only one call's

@@ -123,6 +123,45 @@ extern "C" int tq_decode_attn(const tq_params *kp, const tq_params *vp, const tq
                                             workspace_bytes, stream));
 }
 
+extern "C" int tq_decode_step(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc, const void *K_new,
+                              const void *V_new, const int32_t *slot_mapping, const void *Q, int B, int Hq,
+                              const int32_t *block_table, int max_blocks, const int32_t *seq_lens, int max_seq_len,
+                              void *cache, int64_t num_blocks, void *out, float *lse, float *logits,
+                              int64_t logits_stride, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!attn_params_ok(kp, vp, desc, Hq)) {
+        if (valid_desc(desc) && (desc->d > 256 || (Hq >= 1 && Hq % desc->n_kv_heads == 0 &&
+                                                   Hq / desc->n_kv_heads > 8)))
+            return TQ_EUNSUPPORTED;
+        return TQ_EINVAL;
+    }
+    if (B < 0 || max_blocks < 0 || max_seq_len < 0 || num_blocks < 0) return TQ_EINVAL;
+    if (B == 0) return TQ_OK;
+    if (!K_new || !V_new || !slot_mapping || !Q || !block_table || !seq_lens || !cache || !out || !workspace)
+        return TQ_EINVAL;
+    if (!aligned(K_new, 16) || !aligned(V_new, 16) || !aligned(Q, 16) || !aligned(cache, 256) ||
+        !aligned(workspace, 256) || !aligned(out, 16))
+        return TQ_EINVAL;
+    if (logits && logits_stride < max_seq_len) return TQ_EINVAL;
+    if (int64_t(max_blocks) * desc->page_tokens < max_seq_len) return TQ_EINVAL;
+    tq::Layout L;
+    tq::make_layout(*desc, &L);
+    tq::AttnShape s{};
+    s.n_seq = B;
+    s.Hq = Hq;
+    s.block_table = block_table;
+    s.bt_stride = max_blocks;
+    s.max_blocks = max_blocks;
+    s.seq_lens = seq_lens;
+    s.is_decode = 1;
+    s.base_len = 0;
+    s.max_len = max_seq_len;
+    if (workspace_bytes < tq::attn_ws_bytes(L, s)) return TQ_EINVAL;
+    tq::StepTokens step{K_new, V_new, slot_mapping, static_cast<uint8_t *>(cache)};
+    return cuda_status(tq::launch_attention(kp, vp, L, Q, s, static_cast<const uint8_t *>(cache), num_blocks, out,
+                                            lse, logits, logits_stride, static_cast<uint8_t *>(workspace),
+                                            workspace_bytes, stream, &step));
+}
+
 extern "C" size_t tq_prefill_workspace_bytes(const tq_cache_desc *desc, int C, int Hq, int seq_len) {
     if (!valid_desc(desc) || C < 0 || Hq < 1 || seq_len < C) return 0;
     tq::Layout L;

@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "tq_dev.cuh"
+#include "tq_encode_vec.cuh"
 
 namespace tq {
 namespace {
@@ -104,6 +105,113 @@ __global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
     for (int r = 0; r < 16; ++r) {
         const int64_t row = r0 + 16 * g + r;
         if (row < a.rows) a.w[row * 128 + j] = acc[r];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fused decode step, first launch: the new token's K and V of every sequence
+// are compressed into the cache and the queries are prepared, one warp per
+// vector.  Both need a projection by S (QJL keys: z = S r; queries: w =
+// S q_r), done here from a per-warp shared copy of the vector, fp32
+// products: lane l owns outputs [l E, l E + E) and reads its rows of S.
+// ---------------------------------------------------------------------------
+struct StepArgs {
+    Layout L;
+    DevParams kp, vp;
+    const __nv_bfloat16 *K, *V;      // new tokens [B][H][D]
+    const int32_t *slots;            // [B], < 0 = skip
+    int64_t num_slots;
+    uint8_t *cache;
+    int B;
+    PrepArgs prep;                   // queries [rows][D] -> qr, w
+    uint32_t *status;
+};
+
+template <int D>
+__device__ __forceinline__ void project_rows(const uint16_t *S, const float *vs, int lane,
+                                             float (&z)[WarpVec<D>::E]) {
+    constexpr int E = WarpVec<D>::E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) z[e] = 0.f;
+    if (lane >= WarpVec<D>::LANES) return;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const uint16_t *row = S + size_t(lane * E + e) * D;
+        float acc = 0.f;
+        for (int i = 0; i < D; i += 8) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(row + i);
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc = fmaf(__uint_as_float(w4[k] << 16), vs[i + 2 * k], acc);
+                acc = fmaf(__uint_as_float(w4[k] & 0xFFFF0000u), vs[i + 2 * k + 1], acc);
+            }
+        }
+        z[e] = acc;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) step_prep_kernel(StepArgs a) {
+    constexpr int E = WarpVec<D>::E;
+    __shared__ float svec[8][D > 8 ? D : 8];
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    const Layout &L = a.L;
+    const int64_t n_enc = int64_t(a.B) * L.H * 2;
+    const int64_t job = int64_t(blockIdx.x) * 8 + wl;
+    float *vs = svec[wl];
+    if (job < n_enc) {
+        const bool is_v = job >= int64_t(a.B) * L.H;
+        const int64_t v = is_v ? job - int64_t(a.B) * L.H : job;
+        const int b = int(v / L.H), h = int(v - int64_t(b) * L.H);
+        const int slot = a.slots[b];
+        if (slot < 0) return;
+        if (slot >= a.num_slots) {
+            if (lane == 0) atomicOr(a.status, TQ_DEV_SLOT_RANGE);
+            return;
+        }
+        float x[E], r[E];
+        load_vec<D>((is_v ? a.V : a.K) + v * D, lane, x);
+        uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
+        const int pos = slot % L.P;
+        if (!encode_vector_warp<D>(L, is_v ? a.vp : a.kp, is_v, x, page, pos, lane, r)) return;
+        if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) vs[lane * E + e] = r[e];
+        }
+        __syncwarp();
+        float z[E];
+        project_rows<D>(a.kp.S, vs, lane, z);
+        uint32_t bit[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) bit[e] = z[e] >= 0.f ? 1u : 0u;     // s_j = [(S r)_j >= 0]
+        store_fields<D, 1>(page + L.ks_off + pos * L.ks_bpt, lane, bit);
+        return;
+    }
+    const int64_t row = job - n_enc;
+    if (row >= a.prep.rows) return;
+    float x[E], sg[E];
+    load_vec<D>(reinterpret_cast<const __nv_bfloat16 *>(a.prep.Q) + row * D, lane, x);
+    load_vec<D>(a.kp.signs, lane, sg);
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] *= sg[e];
+    fwht_warp<D>(x, lane);
+    const float rs = 1.0f / sqrtf(float(D));
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            x[e] *= rs;
+            a.prep.qr[row * D + lane * E + e] = x[e];
+            vs[lane * E + e] = x[e];
+        }
+    }
+    if (!L.kqjl) return;
+    __syncwarp();
+    float z[E];
+    project_rows<D>(a.kp.S, vs, lane, z);
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) a.prep.w[row * D + lane * E + e] = z[e];
     }
 }
 
@@ -430,7 +538,7 @@ Plan make_plan(const Layout &L, const AttnShape &s) {
 template <int D>
 int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q, const AttnShape &s,
                   const uint8_t *cache, int64_t num_blocks, void *out, float *lse, float *logits,
-                  int64_t logits_stride, uint8_t *ws, cudaStream_t st) {
+                  int64_t logits_stride, uint8_t *ws, cudaStream_t st, const StepTokens *step) {
     const Plan p = make_plan(L, s);
     const int64_t rows = int64_t(s.n_seq) * s.Hq;
     PrepArgs pa;
@@ -440,7 +548,23 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
     pa.kp = kp->dev;
     pa.qr = reinterpret_cast<float *>(ws + p.off_qr);
     pa.w = reinterpret_cast<float *>(ws + p.off_w);
-    if (D == 128 && L.kqjl) {
+    if (step) {
+        // decode step: the new tokens' encode shares the query-preparation launch
+        StepArgs sa;
+        sa.L = L;
+        sa.kp = kp->dev;
+        sa.vp = vp->dev;
+        sa.K = static_cast<const __nv_bfloat16 *>(step->K);
+        sa.V = static_cast<const __nv_bfloat16 *>(step->V);
+        sa.slots = step->slots;
+        sa.num_slots = num_blocks * L.P;
+        sa.cache = step->cache;
+        sa.B = s.n_seq;
+        sa.prep = pa;
+        sa.status = reinterpret_cast<uint32_t *>(ws);
+        const int64_t jobs = int64_t(s.n_seq) * L.H * 2 + rows;
+        step_prep_kernel<D><<<unsigned((jobs + 7) / 8), 256, 0, st>>>(sa);
+    } else if (D == 128 && L.kqjl) {
         cudaError_t e = cudaFuncSetAttribute(prep_proj128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(kPQSmem));
         if (e != cudaSuccess) return e;
@@ -512,17 +636,16 @@ size_t attn_ws_bytes(const Layout &L, const AttnShape &s) { return make_plan(L, 
 
 int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q,
                      const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out, float *lse,
-                     float *logits, int64_t logits_stride, uint8_t *ws, size_t ws_bytes, void *stream) {
+                     float *logits, int64_t logits_stride, uint8_t *ws, size_t ws_bytes, void *stream,
+                     const StepTokens *step) {
     (void)ws_bytes;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define TQ_RUN_ATT(DD) \
+    case DD: return run_attention<DD>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st, step);
     switch (L.d) {
-        case 8: return run_attention<8>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
-        case 16: return run_attention<16>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
-        case 32: return run_attention<32>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
-        case 64: return run_attention<64>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
-        case 128: return run_attention<128>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
-        case 256: return run_attention<256>(kp, vp, L, Q, s, cache, num_blocks, out, lse, logits, logits_stride, ws, st);
+        TQ_RUN_ATT(8) TQ_RUN_ATT(16) TQ_RUN_ATT(32) TQ_RUN_ATT(64) TQ_RUN_ATT(128) TQ_RUN_ATT(256)
     }
+#undef TQ_RUN_ATT
     return cudaErrorInvalidValue;
 }
 

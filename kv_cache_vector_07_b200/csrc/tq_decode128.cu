@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     constexpr int NKS = query_ksteps<KB>(), QK0 = qjl_kstep0<KB>();
     extern __shared__ __align__(16) uint8_t smem[];
     uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][KC copies] {hi pair, lo pair}
-    uint32_t *lutV = reinterpret_cast<uint32_t *>(lutK + KE * KC);   // [VE][VC copies]
+    uint2 *lutV = reinterpret_cast<uint2 *>(lutK + KE * KC);        // [VE][VC copies] {hi pair, lo pair}
     uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * VC);          // [NT][NKS][32]
     uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * NKS * 32);
     const Layout &L = a.L;
@@ -189,7 +189,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
         float lo, hi;
         if (VB == 4) { lo = a.v_lv[e & 15]; hi = a.v_lv[e >> 4]; }
         else { lo = a.v_lv[e & 3]; hi = a.v_lv[(e >> 2) & 3]; }       // magnitudes (positive half)
-        lutV[i] = h2bits(lo, hi);
+        // level pair as fp16 hi + lo: outputs of outlier channels (tens) need
+        // the levels' fp32 accuracy, not fp16's 2^-12
+        const float h0 = __half2float(__float2half_rn(lo)), h1 = __half2float(__float2half_rn(hi));
+        lutV[i] = make_uint2(h2bits(h0, h1), h2bits(lo - h0, hi - h1));
     }
     // 2-bit keys: stored code (n, m) = (negative, larger magnitude) has level
     // (1 - 2n)(c_0 + m (c_1 - c_0)); the key side of the product is then two
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     if (tid == 0 && !*abort_flag)
         for (int i = 0; i < kNS - 1 && i < n_pages; ++i) { issue_page(i); issued = i + 1; }
 
-    const uint32_t vlane_off = uint32_t(lane & (VC - 1)) * 4u;     // this lane's value-table copy
+    const uint32_t vlane_off = uint32_t(lane & (VC - 1)) * 8u;     // this lane's value-table copy
     const uint32_t klane_off = uint32_t(lane & (KC - 1)) * 8u;     // this lane's key-table copy
     const float cq = 1.2533141373155003f / 128.0f;       // sqrt(pi/2) / m
     float m_run[NT], l_run[NT];
@@ -426,6 +429,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             const bool ok0 = tok0 + g < nv, ok1 = tok0 + g + 8 < nv;
             // ---------------- online softmax (log2 units) for heads t and 4 + t
             uint32_t pk[NT];           // half2(P'[token g][h], P'[token g+8][h])
+            uint32_t pk_lo = 0;        // one head tile: P' - fp16(P') for the spare columns
             float alpha[NT];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -448,7 +452,12 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                 l_run[nt] = fmaf(l_run[nt], al, p0 + p1);
                 m_run[nt] = m_new;
                 alpha[nt] = al;
-                pk[nt] = h2bits(ok0 ? p0 * nv0 : 0.f, ok1 ? p1 * nv1 : 0.f);
+                const float q0 = ok0 ? p0 * nv0 : 0.f, q1 = ok1 ? p1 * nv1 : 0.f;
+                pk[nt] = h2bits(q0, q1);
+                if (NT == 1) {
+                    const float2 hq = __half22float2(*reinterpret_cast<const __half2 *>(&pk[nt]));
+                    pk_lo = h2bits(q0 - hq.x, q1 - hq.y);
+                }
             }
             // ---------------- P^T fragment: head column g, tokens 2t, 2t+1 (+8)
             uint32_t b0, b1;
@@ -458,8 +467,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                 if (NT > 1) {
                     const uint32_t u0 = __shfl_sync(kFull, pk[NT - 1], src0), u1 = __shfl_sync(kFull, pk[NT - 1], src1);
                     if (g >= 4) { v0 = u0; v1 = u1; }
-                } else if (g >= 4) {
-                    v0 = 0; v1 = 0;
+                } else {
+                    // one head tile: columns 4..7 carry the low parts of columns 0..3
+                    const uint32_t u0 = __shfl_sync(kFull, pk_lo, src0), u1 = __shfl_sync(kFull, pk_lo, src1);
+                    if (g >= 4) { v0 = u0; v1 = u1; }
                 }
                 b0 = prmt(v0, v1, 0x5410);         // tokens 2t, 2t+1
                 b1 = prmt(v0, v1, 0x7632);         // tokens 2t+8, 2t+9
@@ -503,12 +514,15 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int mt = 4 * wi + k;          // coordinates 16g + 2mt, +1
-                            uint32_t A[4];
-                            A[0] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(eAB, k, vlane_off));
-                            A[1] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(oAB, k, vlane_off));
-                            A[2] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(eCD, k, vlane_off));
-                            A[3] = lds_at<uint32_t>(lutV, field_offset<8, VC * 4>(oCD, k, vlane_off));
-                            mma16816(O[mt], A, b0, b1);
+                            uint2 v[4];
+                            v[0] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(eAB, k, vlane_off));
+                            v[1] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(oAB, k, vlane_off));
+                            v[2] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(eCD, k, vlane_off));
+                            v[3] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(oCD, k, vlane_off));
+                            const uint32_t Ah[4] = {v[0].x, v[1].x, v[2].x, v[3].x};
+                            const uint32_t Al[4] = {v[0].y, v[1].y, v[2].y, v[3].y};
+                            mma16816(O[mt], Ah, b0, b1);
+                            mma16816(O[mt], Al, b0, b1);
                         }
                     }
                 } else {
@@ -530,16 +544,18 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
                         const int e0 = 2 * mt, e1 = 2 * mt + 1;     // coordinates 16g + e
-                        uint32_t A[4];
-                        A[0] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(eAB, mt, vlane_off)) ^
-                               ((zAB << (15 - e0)) & 0x80008000u);
-                        A[1] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(oAB, mt, vlane_off)) ^
-                               ((zAB << (15 - e1)) & 0x80008000u);
-                        A[2] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(eCD, mt, vlane_off)) ^
-                               ((zCD << (15 - e0)) & 0x80008000u);
-                        A[3] = lds_at<uint32_t>(lutV, field_offset<4, VC * 4>(oCD, mt, vlane_off)) ^
-                               ((zCD << (15 - e1)) & 0x80008000u);
-                        mma16816(O[mt], A, b0, b1);
+                        const uint32_t z[4] = {(zAB << (15 - e0)) & 0x80008000u, (zAB << (15 - e1)) & 0x80008000u,
+                                               (zCD << (15 - e0)) & 0x80008000u, (zCD << (15 - e1)) & 0x80008000u};
+                        uint2 v[4];
+                        v[0] = lds_at<uint2>(lutV, field_offset<4, VC * 8>(eAB, mt, vlane_off));
+                        v[1] = lds_at<uint2>(lutV, field_offset<4, VC * 8>(oAB, mt, vlane_off));
+                        v[2] = lds_at<uint2>(lutV, field_offset<4, VC * 8>(eCD, mt, vlane_off));
+                        v[3] = lds_at<uint2>(lutV, field_offset<4, VC * 8>(oCD, mt, vlane_off));
+                        uint32_t Ah[4], Al[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) { Ah[r] = v[r].x ^ z[r]; Al[r] = v[r].y ^ z[r]; }
+                        mma16816(O[mt], Ah, b0, b1);
+                        mma16816(O[mt], Al, b0, b1);
                     }
                 }
             }
@@ -577,7 +593,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
         // this warp's factor for heads 2t, 2t+1: exp2(m_warp - M)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const int hd = 2 * t + c;
+            const int hd = NT == 1 ? ((2 * t + c) & 3) : 2 * t + c;   // one tile: column 4 + h is head h
             float M = -INFINITY;
             for (int w2 = 0; w2 < 4; ++w2) M = fmaxf(M, mm[w2 * 8 + hd]);
             const float mw = mm[warp * 8 + hd];
@@ -596,8 +612,11 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     }
     __syncthreads();
     const int64_t pbase = (int64_t(grp) * a.n_splits + split) * G;
-    for (int i = tid; i < G * 128; i += 128)
-        a.part_o[pbase * 128 + i] = ((oo[i] + oo[1024 + i]) + oo[2048 + i]) + oo[3072 + i];
+    for (int i = tid; i < G * 128; i += 128) {
+        float o = ((oo[i] + oo[1024 + i]) + oo[2048 + i]) + oo[3072 + i];
+        if (NT == 1) o += ((oo[512 + i] + oo[1536 + i]) + oo[2560 + i]) + oo[3584 + i];
+        a.part_o[pbase * 128 + i] = o;
+    }
     if (tid < G) {
         float M = -INFINITY;
         for (int w2 = 0; w2 < 4; ++w2) M = fmaxf(M, mm[w2 * 8 + tid]);
@@ -619,7 +638,7 @@ size_t dec_smem(int page_bytes) {
     constexpr int kNS = page_stages<KB>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
-    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 4 +
+    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 8 +
            size_t(NT) * query_ksteps<KB>() * 32 * 8 +
            stages + (2 * kNS + 1) * 8 + kNS * 4 + 4 + 64;
 }

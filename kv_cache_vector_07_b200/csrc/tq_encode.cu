@@ -21,6 +21,7 @@
 
 #include "tc05.cuh"
 #include "tq_dev.cuh"
+#include "tq_encode_vec.cuh"
 
 namespace tq {
 namespace {
@@ -38,11 +39,6 @@ struct EncodeArgs {
     int do_v;
 };
 
-template <int D, int W>
-__device__ __forceinline__ void store_codes(uint8_t *dst, int lane, const uint32_t (&f)[WarpVec<D>::E]) {
-    store_fields<D, W>(dst, lane, f);
-}
-
 template <int D, typename TIn>
 __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     constexpr int E = WarpVec<D>::E;
@@ -51,8 +47,6 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     const int64_t nvec = a.n_tokens * L.H;
     const int64_t total = a.do_v ? 2 * nvec : nvec;
     const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-    const float rs = 1.0f / sqrtf(float(D));
-    const float sqrt_d = sqrtf(float(D));
 
     for (int64_t vid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; vid < total; vid += nwarps) {
         const bool is_v = vid >= nvec;
@@ -66,86 +60,14 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
             continue;
         }
         const DevParams &P = is_v ? a.vp : a.kp;
-        const int bits = is_v ? L.vbits : L.kbits;
-
-        float x[E], sg[E];
+        float x[E], r[E];
         load_vec<D>(reinterpret_cast<const TIn *>(is_v ? a.V : a.K) + v * D, lane, x);
-        load_vec<D>(P.signs, lane, sg);
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            ss = fmaf(x[e], x[e], ss);
-            x[e] *= sg[e];
-        }
-        const float n = sqrtf(warp_sum(ss));
-        fwht_warp<D>(x, lane);
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[e] *= rs;          // y = R x
-        const float inv = n > 0.f ? 1.0f / n : 0.f;
-        const uint16_t nh = f2h_bits(n);
-        const float nhf = h2f_bits(nh);
-
         uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
         const int pos = slot % L.P;
-
-        if (!is_v && L.kbits == 8) {
-            uint32_t f[E];
+        if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r) && lane < WarpVec<D>::LANES) {
+            float *dst = a.resid + v * D + lane * E;
 #pragma unroll
-            for (int e = 0; e < E; ++e)
-                // the zero vector has u = +0 (not the -0 a sign flip of a zero leaves)
-                f[e] = uint32_t(__nv_cvt_float_to_fp8(n > 0.f ? sqrt_d * (x[e] * inv) : 0.f, __NV_SATFINITE,
-                                                      __NV_E4M3));
-            store_codes<D, 8>(page + L.kc_off + pos * L.kc_bpt, lane, f);
-            if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kn_off + pos * 2) = nh;
-            continue;
-        }
-
-        const int nb = (1 << bits) - 1;
-        uint32_t kap[E];
-        float cval[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const float u = x[e] * inv;
-            uint32_t idx = 0;
-            for (int j = 0; j < nb; ++j) idx += (P.bounds[j] <= u) ? 1u : 0u;
-            kap[e] = kappa_of(idx, bits);
-            cval[e] = P.lv[kap[e]];
-        }
-        const int code_off = is_v ? L.vc_off : L.kc_off;
-        const int code_bpt = is_v ? L.vc_bpt : L.kc_bpt;
-        uint8_t *cdst = page + code_off + pos * code_bpt;
-        if (bits == 1) {
-            store_codes<D, 1>(cdst, lane, kap);
-        } else if (bits == 2) {
-            store_codes<D, 2>(cdst, lane, kap);
-        } else if (bits == 4) {
-            store_codes<D, 4>(cdst, lane, kap);
-        } else {   // 3 bits: 2-bit magnitude array + 1-bit sign array
-            uint32_t lo[E], hi[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) { lo[e] = kap[e] & 3u; hi[e] = kap[e] >> 2; }
-            store_codes<D, 2>(cdst, lane, lo);
-            const int hoff = is_v ? L.vh_off : L.kh_off;
-            const int hbpt = is_v ? L.vh_bpt : L.kh_bpt;
-            store_codes<D, 1>(page + hoff + pos * hbpt, lane, hi);
-        }
-        if (lane == 0) *reinterpret_cast<uint16_t *>(page + (is_v ? L.vn_off : L.kn_off) + pos * 2) = nh;
-
-        if (!is_v && L.kqjl) {
-            float r[E], rr = 0.f;
-            const bool active = lane < WarpVec<D>::LANES;    // lanes past d hold no coordinate
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                r[e] = active ? fmaf(-nhf, cval[e], x[e]) : 0.f;
-                rr = fmaf(r[e], r[e], rr);
-            }
-            const float rho = sqrtf(warp_sum(rr));
-            if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kr_off + pos * 2) = f2h_bits(rho);
-            if (lane < WarpVec<D>::LANES) {
-                float *dst = a.resid + v * D + lane * E;
-#pragma unroll
-                for (int e = 0; e < E; ++e) dst[e] = r[e];
-            }
+            for (int e = 0; e < E; ++e) dst[e] = r[e];
         }
     }
 }

@@ -123,11 +123,18 @@ struct AttnShape {
     int max_len;          // longest visible length
     int is_decode;        // 1: decode (per-sequence lengths), 0: prefill chunk
 };
+// New tokens of a fused decode step (one per sequence): bf16 K and V
+// [B][H][d], their slots, and the cache they are written into.
+struct StepTokens {
+    const void *K, *V;
+    const int32_t *slots;
+    uint8_t *cache;
+};
 size_t attn_ws_bytes(const Layout &L, const AttnShape &s);
 int launch_attention(const tq_params *kp, const tq_params *vp, const Layout &L, const void *Q,
                      const AttnShape &s, const uint8_t *cache, int64_t num_blocks, void *out,
                      float *lse, float *logits, int64_t logits_stride, uint8_t *ws,
-                     size_t ws_bytes, void *stream);
+                     size_t ws_bytes, void *stream, const StepTokens *step = nullptr);
 
 // Testing aid of the tensor-core decode kernel: the poll budget of a wait
 // that nothing completes, taken (and reset to 0) by the next launch.

@@ -64,6 +64,8 @@ _sig("tq_decode_attn", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i
                               _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("tq_decode_attn_noalloc", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i32, _vp, _i32, _vp, _i32,
                                       _vp, _i64, _vp, _vp, _vp, _i64, _vp])
+_sig("tq_decode_step", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp,
+                              _i32, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("tq_prefill_workspace_bytes", _sz, [ctypes.POINTER(CacheDesc), _i32, _i32, _i32])
 _sig("tq_prefill_attn", _i32, [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
                                _vp, _vp, _vp, _sz, _vp])
@@ -243,6 +245,30 @@ def decode_attn(kp: Params, vp: Params, desc: CacheDesc, Q: torch.Tensor, block_
                                block_table.shape[1], _ptr(seq_lens), max_seq_len, _ptr(cache), cache.shape[0],
                                _ptr(out), _ptr(lse), _ptr(logits), stride, _ptr(workspace), workspace.numel(),
                                _stream(stream)), "tq_decode_attn")
+    return out
+
+
+def decode_step(kp: Params, vp: Params, desc: CacheDesc, K_new: torch.Tensor, V_new: torch.Tensor,
+                slot_mapping: torch.Tensor, Q: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                max_seq_len: int, cache: torch.Tensor, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None, logits: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None):
+    """tq_decode_step: write K_new/V_new bf16 [B, n_kv_heads, d] at slot_mapping
+    [B], then decode attention of Q bf16 [B, Hq, d] over seq_lens tokens."""
+    _dev_check(K_new, V_new, slot_mapping, Q, block_table, seq_lens, cache, out, lse, logits, workspace)
+    if K_new.dtype != torch.bfloat16 or V_new.dtype != torch.bfloat16 or slot_mapping.dtype != torch.int32:
+        raise ValueError("K_new/V_new must be bf16 and slot_mapping int32")
+    B, Hq, d = Q.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    if workspace is None:
+        workspace = _workspace(decode_workspace_bytes(desc, B, Hq, max_seq_len), Q.device)
+    stride = logits.shape[-1] if logits is not None else 0
+    _check(_lib.tq_decode_step(kp.handle, vp.handle, ctypes.byref(desc), _ptr(K_new), _ptr(V_new),
+                               _ptr(slot_mapping), _ptr(Q), B, Hq, _ptr(block_table), block_table.shape[1],
+                               _ptr(seq_lens), max_seq_len, _ptr(cache), cache.shape[0], _ptr(out), _ptr(lse),
+                               _ptr(logits), stride, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "tq_decode_step")
     return out
 
 

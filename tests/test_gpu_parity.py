@@ -467,6 +467,58 @@ def test_block_table_out_of_range_is_flagged():
     assert tqkv.read_status(ws) & tqkv.TQ_DEV_BLOCK_RANGE
 
 
+# ---------------------------------------------------------------------------
+# fused decode step: the new token's write shares the query-prep launch
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,kbits,kqjl,vbits,B,Hq,H,L", [
+    (128, 2, True, 4, 4, 32, 8, 777),      # k3v4, tensor-core decode
+    (128, 8, False, 4, 3, 16, 4, 500),     # k8v4, tensor-core decode
+    (128, 3, True, 3, 2, 8, 2, 300),       # 3-bit keys: general decode kernel
+    (64, 4, True, 2, 3, 4, 1, 130),        # d = 64, general kernels
+])
+def test_decode_step_writes_new_token_and_attends(d, kbits, kqjl, vbits, B, Hq, H, L):
+    P = 64 if d == 128 else 16
+    seed = 300 + kbits + d
+    cd = Codec(d, kbits, kqjl, vbits, seed=seed, page_tokens=P, H=H)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
+    K = synth.outlier_normal((B, L, H, d), seed=seed + 1, device=DEV)
+    V = synth.outlier_normal((B, L, H, d), seed=seed + 2, device=DEV)
+    sl = slots.view(B, L)
+    old = sl[:, :L - 1].reshape(-1).contiguous()
+    cache, flags = cd.encode(K[:, :L - 1].reshape(-1, H, d).contiguous(), V[:, :L - 1].reshape(-1, H, d).contiguous(),
+                             old, nblk)
+    assert flags == 0
+    new_slots = sl[:, L - 1].contiguous().clone()
+    new_slots[1] = -1                                   # sequence 1 writes nothing this step
+    lens = [L] * B
+    lens[1] = L - 1
+    seq = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    Q = synth.normal((B, Hq, d), seed=seed + 3, device=DEV)
+    ws = torch.zeros(tqkv.decode_workspace_bytes(cd.desc, B, Hq, L), dtype=torch.uint8, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    lse = torch.empty((B, Hq), device=DEV)
+    out = tqkv.decode_step(cd.kp, cd.vp, cd.desc, K[:, L - 1].contiguous(), V[:, L - 1].contiguous(), new_slots, Q,
+                           bt, seq, L, cache, lse=lse, logits=logits, workspace=ws)
+    torch.cuda.synchronize()
+    assert tqkv.read_status(ws) == 0
+    cn = cache_np(cache)
+    sln = sl.cpu().numpy()
+    # the skipped token's slot stays empty
+    lay = cd.lay
+    back = O.read_cache(lay, cn, sln[1, L - 1:L], 0, H)
+    assert np.all(back["kn"] == 0)
+    G = Hq // H
+    for b in range(B):
+        n = lens[b]
+        for kvh in range(H):
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, sln[b, :n], f64(K[b, :n, kvh]), f64(V[b, :n, kvh]), kvh)
+            rows = list(range(kvh * G, kvh * G + G))
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
+            assert np.allclose(f64(lse[b, rows]), lse_ref, rtol=1e-3, atol=1e-3)
+
+
 def test_decode_wait_timeout_is_flagged_and_context_survives():
     """A bounded on-chip wait that runs out (a barrier nothing completes, set
     up through the testing aid) sets TQ_DEV_WAIT_TIMEOUT, returns promptly,
