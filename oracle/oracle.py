@@ -68,12 +68,13 @@ def _load():
     lib.orc_gauss_bf16.argtypes = [i32, i32, u64, vp]
     lib.orc_codebook.restype = i32
     lib.orc_codebook.argtypes = [i32, i32, vp, vp, vp]
-    lib.orc_rotate.argtypes = [i32, vp, vp, vp]
-    lib.orc_rotate_t.argtypes = [i32, vp, vp, vp]
-    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-    lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.orc_rotate.argtypes = [i32, vp, vp, vp, vp]
+    lib.orc_rotate_t.argtypes = [i32, vp, vp, vp, vp]
+    lib.orc_dense_rotation.argtypes = [i32, u64, vp, vp, vp]
+    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_estimate.argtypes = [vp, i32, vp, vp]
-    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_attend_exact.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     lib.orc_search.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     _lib = lib
@@ -126,12 +127,14 @@ class Params:
     c32: np.ndarray | None       # float32 levels
     t32: np.ndarray | None       # float32 boundaries
     iters: int = 0
+    Rm: np.ndarray | None = None  # dense rotation [d, d] (None: H D / sqrt(d))
 
 
-def make_params(d: int, bits: int, seed: int, with_S: bool = True) -> Params:
+def make_params(d: int, bits: int, seed: int, with_S: bool = True, rotation: str = "hadamard") -> Params:
     """Signs, Gaussian S (m = d, bf16-exact) and, for bits in 1..4, the
     Lloyd-Max codebook of the coordinate law of a random unit vector in R^d.
-    bits = 8 denotes FP8 (E4M3) codes and has no codebook."""
+    bits = 8 denotes FP8 (E4M3) codes and has no codebook.  rotation =
+    "dense" replaces H D / sqrt(d) by the dense random rotation."""
     lib = _load()
     signs = np.zeros(d, np.int8)
     lib.orc_signs(d, seed, _p(signs))
@@ -145,7 +148,22 @@ def make_params(d: int, bits: int, seed: int, with_S: bool = True) -> Params:
         c64, c32, t32 = codebook(d, bits)
     elif bits != 8:
         raise ValueError("bits must be 1..4 or 8")
-    return Params(d, bits, seed, signs, S, c64, c32, t32, iters)
+    Rm = None
+    if rotation == "dense":
+        Rm = dense_rotation(d, seed)[2]
+    elif rotation != "hadamard":
+        raise ValueError("rotation must be 'hadamard' or 'dense'")
+    return Params(d, bits, seed, signs, S, c64, c32, t32, iters, Rm)
+
+
+def dense_rotation(d: int, seed: int):
+    """(G, Q, Rm): the Gaussian matrix, its row-orthonormalised float64 form
+    and the stored rotation (Q rounded to float32)."""
+    G = np.zeros((d, d), np.float64)
+    Q = np.zeros((d, d), np.float64)
+    Rm = np.zeros((d, d), np.float64)
+    _load().orc_dense_rotation(d, seed, _p(G), _p(Q), _p(Rm))
+    return G, Q, Rm
 
 
 _codebook_cache: dict = {}
@@ -167,25 +185,27 @@ def codebook(d: int, bits: int):
     return _codebook_cache[key]
 
 
-def rotate(x: np.ndarray, signs: np.ndarray) -> np.ndarray:
+def rotate(x: np.ndarray, signs: np.ndarray, Rm: np.ndarray | None = None) -> np.ndarray:
     x = np.ascontiguousarray(x, np.float64)
     d = x.shape[-1]
     flat = x.reshape(-1, d)
     out = np.zeros_like(flat)
     lib = _load()
+    Rm = None if Rm is None else np.ascontiguousarray(Rm, np.float64)
     for r in range(flat.shape[0]):
-        lib.orc_rotate(d, _p(signs), _p(flat[r]), _p(out[r]))
+        lib.orc_rotate(d, _p(signs), _p(Rm), _p(flat[r]), _p(out[r]))
     return out.reshape(x.shape)
 
 
-def rotate_t(y: np.ndarray, signs: np.ndarray) -> np.ndarray:
+def rotate_t(y: np.ndarray, signs: np.ndarray, Rm: np.ndarray | None = None) -> np.ndarray:
     y = np.ascontiguousarray(y, np.float64)
     d = y.shape[-1]
     flat = y.reshape(-1, d)
     out = np.zeros_like(flat)
     lib = _load()
+    Rm = None if Rm is None else np.ascontiguousarray(Rm, np.float64)
     for r in range(flat.shape[0]):
-        lib.orc_rotate_t(d, _p(signs), _p(flat[r]), _p(out[r]))
+        lib.orc_rotate_t(d, _p(signs), _p(Rm), _p(flat[r]), _p(out[r]))
     return out.reshape(y.shape)
 
 
@@ -218,7 +238,7 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
         nhat = np.zeros(n, np.float64)
         mg = np.zeros((n, d), np.float64) if margins else None
         nraw = np.zeros(n, np.float64)
-        lib.orc_encode_fp8(n, d, _p(X), _p(P.signs), _p(code), _p(nhat), _p(mg), _p(nraw))
+        lib.orc_encode_fp8(n, d, _p(X), _p(P.signs), _p(P.Rm), _p(code), _p(nhat), _p(mg), _p(nraw))
         return Encoded(8, False, code, nhat, umargin=mg, nraw=nraw)
     idx = np.zeros((n, d), np.uint8)
     nhat = np.zeros(n, np.float64)
@@ -230,7 +250,7 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
         assert P.S is not None
     nraw = np.zeros(n, np.float64)
     rraw = np.zeros(n, np.float64) if qjl else None
-    lib.orc_encode(n, d, P.bits, 1 if qjl else 0, _p(X), _p(P.signs), _p(P.S), _p(P.c32),
+    lib.orc_encode(n, d, P.bits, 1 if qjl else 0, _p(X), _p(P.signs), _p(P.Rm), _p(P.S), _p(P.c32),
                    _p(P.t32), _p(idx), _p(nhat), _p(rho), _p(sb), _p(um), _p(zm), _p(nraw), _p(rraw))
     return Encoded(P.bits, qjl, idx, nhat, rho, sb, um, zm, nraw, rraw)
 
@@ -242,14 +262,14 @@ class _Keys(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("qjl", ctypes.c_int), ("d", ctypes.c_int),
                 ("signs", ctypes.c_void_p), ("S", ctypes.c_void_p), ("c32", ctypes.c_void_p),
                 ("idx", ctypes.c_void_p), ("fp8", ctypes.c_void_p), ("nhat", ctypes.c_void_p),
-                ("rho", ctypes.c_void_p), ("sbits", ctypes.c_void_p)]
+                ("rho", ctypes.c_void_p), ("sbits", ctypes.c_void_p), ("Rm", ctypes.c_void_p)]
 
 
 def _keys(P: Params, E: Encoded, keep: list) -> _Keys:
     arrs = [np.ascontiguousarray(a) if a is not None else None
-            for a in (P.signs, P.S, P.c32, E.idx, E.nhat, E.rho, E.sbits)]
+            for a in (P.signs, P.S, P.c32, E.idx, E.nhat, E.rho, E.sbits, P.Rm)]
     keep.extend(arrs)
-    signs, S, c32, idx, nhat, rho, sb = arrs
+    signs, S, c32, idx, nhat, rho, sb, Rm = arrs
     k = _Keys()
     k.kind = 1 if E.bits == 8 else 0
     k.qjl = 1 if E.qjl else 0
@@ -262,6 +282,7 @@ def _keys(P: Params, E: Encoded, keep: list) -> _Keys:
     k.nhat = _p(nhat)
     k.rho = _p(rho)
     k.sbits = _p(sb)
+    k.Rm = _p(Rm)
     return k
 
 
@@ -290,7 +311,8 @@ def attend(Q: np.ndarray, Pk: Params, Ek: Encoded, Pv: Params, Ev: Encoded,
     logits = np.zeros((nq, L), np.float64) if want_logits else None
     nv = None if nvis is None else np.ascontiguousarray(nvis, np.int32)
     vs, vc, vi, vn = (np.ascontiguousarray(a) for a in (Pv.signs, Pv.c32, Ev.idx, Ev.nhat))
-    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vc), _p(vi),
+    vR = None if Pv.Rm is None else np.ascontiguousarray(Pv.Rm)
+    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), _p(vc), _p(vi),
                        _p(vn), _p(logits), _p(out), _p(lse))
     return out, lse, logits
 

@@ -149,6 +149,48 @@ void orc_gauss_bf16(int m, int d, uint64_t seed, float *S)
     }
 }
 
+/* Dense random rotation (the alternative to H D / sqrt(d)).  G is d x d iid
+ * N(0,1) by Box-Muller of draw(seed, 2, .) pairs, row-major, full float64.
+ * Its rows are orthonormalised in order by modified Gram-Schmidt (the Q of
+ * the QR factorisation of G^T with a positive diagonal, transposed), and the
+ * result is stored in float32 (round to nearest even), so that both sides of
+ * the computation hold the same matrix.  Outputs: G (optional), Q (float64,
+ * before rounding; optional) and Rm (the stored matrix, float32 values). */
+void orc_dense_rotation(int d, uint64_t seed, double *G, double *Q, double *Rm)
+{
+    size_t dd = (size_t)d * d;
+    double *g = (double *)malloc(sizeof(double) * dd);
+    for (size_t k = 0; k < dd; k += 2) {
+        uint64_t p = k / 2;
+        uint64_t a = orc_draw(seed, 2, 2 * p), b = orc_draw(seed, 2, 2 * p + 1);
+        double u1 = ((double)(a >> 11) + 1.0) * 0x1.0p-53;
+        double u2 = (double)(b >> 11) * 0x1.0p-53;
+        double rad = sqrt(-2.0 * log(u1));
+        g[k] = rad * cos(2.0 * M_PI * u2);
+        if (k + 1 < dd) g[k + 1] = rad * sin(2.0 * M_PI * u2);
+    }
+    if (G) memcpy(G, g, sizeof(double) * dd);
+    double *q = (double *)malloc(sizeof(double) * dd);
+    memcpy(q, g, sizeof(double) * dd);
+    for (int j = 0; j < d; ++j) {
+        double *v = q + (size_t)j * d;
+        for (int k = 0; k < j; ++k) {
+            const double *e = q + (size_t)k * d;
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i) dot += v[i] * e[i];
+            for (int i = 0; i < d; ++i) v[i] -= dot * e[i];
+        }
+        double nn = 0.0;
+        for (int i = 0; i < d; ++i) nn += v[i] * v[i];
+        nn = sqrt(nn);
+        for (int i = 0; i < d; ++i) v[i] /= nn;
+    }
+    if (Q) memcpy(Q, q, sizeof(double) * dd);
+    for (size_t k = 0; k < dd; ++k) Rm[k] = (double)(float)q[k];   /* float32, round to nearest even */
+    free(g);
+    free(q);
+}
+
 /* Density of one coordinate of a uniformly random unit vector in R^d:
  *   f_d(t) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) * (1 - t^2)^((d-3)/2). */
 typedef struct { double logk; double a; int moment; } dens_t;
@@ -270,18 +312,34 @@ static void fwht_inplace(int d, double *v)
             }
 }
 
-/* y = R x */
-void orc_rotate(int d, const int8_t *signs, const double *x, double *y)
+/* y = R x.  Rm != NULL selects the dense rotation: y = Rm x, Rm row-major. */
+void orc_rotate(int d, const int8_t *signs, const double *Rm, const double *x, double *y)
 {
+    if (Rm) {
+        for (int j = 0; j < d; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i) s += Rm[(size_t)j * d + i] * x[i];
+            y[j] = s;
+        }
+        return;
+    }
     for (int i = 0; i < d; ++i) y[i] = signs[i] * x[i];
     fwht_inplace(d, y);
     double s = 1.0 / sqrt((double)d);
     for (int i = 0; i < d; ++i) y[i] *= s;
 }
 
-/* x = R^T y = D H y / sqrt(d)  (H is symmetric) */
-void orc_rotate_t(int d, const int8_t *signs, const double *y, double *x)
+/* x = R^T y = D H y / sqrt(d)  (H is symmetric); dense: x = Rm^T y. */
+void orc_rotate_t(int d, const int8_t *signs, const double *Rm, const double *y, double *x)
 {
+    if (Rm) {
+        for (int i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j) s += Rm[(size_t)j * d + i] * y[j];
+            x[i] = s;
+        }
+        return;
+    }
     for (int i = 0; i < d; ++i) x[i] = y[i];
     fwht_inplace(d, x);
     double s = 1.0 / sqrt((double)d);
@@ -301,7 +359,7 @@ void orc_rotate_t(int d, const int8_t *signs, const double *y, double *x)
  * unrounded norms nraw = ||x||, rraw = ||r||.
  * sbits / rho / zmargin are only written when qjl != 0. */
 void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *signs,
-                const float *S, const float *c32, const float *t32, uint8_t *idx,
+                const double *Rm, const float *S, const float *c32, const float *t32, uint8_t *idx,
                 double *nhat, double *rho, uint8_t *sbits, double *umargin,
                 double *zmargin, double *nraw, double *rraw)
 {
@@ -313,10 +371,12 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
     #pragma omp for schedule(static)
     for (int v = 0; v < n; ++v) {
         const double *x = X + (size_t)v * d;
+        orc_rotate(d, signs, Rm, x, y);
+        /* n = ||x|| (= ||R x||; the dense rotation uses ||R x|| itself) */
+        const double *nsrc = Rm ? y : x;
         double nn = 0.0;
-        for (int i = 0; i < d; ++i) nn += x[i] * x[i];
+        for (int i = 0; i < d; ++i) nn += nsrc[i] * nsrc[i];
         nn = sqrt(nn);
-        orc_rotate(d, signs, x, y);
         double nh = orc_round_fp16(nn);
         nhat[v] = nh;
         if (nraw) nraw[v] = nn;
@@ -358,7 +418,7 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
 /* FP8 keys: code_i = e4m3_rne_satfinite(sqrt(d) * u_i), nhat = fp16(||x||).
  * margin[i] = distance (unit-vector units) from u_i to the nearest E4M3
  * rounding midpoint. */
-void orc_encode_fp8(int n, int d, const double *X, const int8_t *signs, uint8_t *code,
+void orc_encode_fp8(int n, int d, const double *X, const int8_t *signs, const double *Rm, uint8_t *code,
                     double *nhat, double *margin, double *nraw)
 {
     double sd = sqrt((double)d);
@@ -368,10 +428,11 @@ void orc_encode_fp8(int n, int d, const double *X, const int8_t *signs, uint8_t 
     #pragma omp for schedule(static)
     for (int v = 0; v < n; ++v) {
         const double *x = X + (size_t)v * d;
+        orc_rotate(d, signs, Rm, x, y);
+        const double *nsrc = Rm ? y : x;
         double nn = 0.0;
-        for (int i = 0; i < d; ++i) nn += x[i] * x[i];
+        for (int i = 0; i < d; ++i) nn += nsrc[i] * nsrc[i];
         nn = sqrt(nn);
-        orc_rotate(d, signs, x, y);
         nhat[v] = orc_round_fp16(nn);
         if (nraw) nraw[v] = nn;
         for (int i = 0; i < d; ++i) {
@@ -411,6 +472,7 @@ typedef struct {
     const double *nhat;     /* [L] */
     const double *rho;      /* [L] (QJL only) */
     const uint8_t *sbits;   /* [L][m] (QJL only) */
+    const double *Rm;       /* dense rotation (row-major d x d) or NULL */
 } orc_keys_t;
 
 /* Estimates of <q, k_t> for t in [0, L):
@@ -421,7 +483,7 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
     int d = K->d, m = d;
     double *qr = (double *)malloc(sizeof(double) * d);
     double *w = (double *)malloc(sizeof(double) * m);
-    orc_rotate(d, K->signs, q, qr);
+    orc_rotate(d, K->signs, K->Rm, q, qr);
     if (K->kind == 0 && K->qjl) {
         for (int j = 0; j < m; ++j) {
             double s = 0.0;
@@ -459,7 +521,7 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
  * logits [nq][L] (positions past nvis set to -inf) and lse [nq] (natural log
  * of the softmax denominator of the scaled logits). */
 void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const orc_keys_t *K,
-                const int8_t *v_signs, const float *v_c32, const uint8_t *v_idx,
+                const int8_t *v_signs, const double *v_Rm, const float *v_c32, const uint8_t *v_idx,
                 const double *v_nhat, double *logits, double *out, double *lse)
 {
     double *est = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
@@ -479,7 +541,7 @@ void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const or
             for (int i = 0; i < d; ++i) orot[i] += pv * (double)v_c32[v_idx[(size_t)t * d + i]];
         }
         for (int i = 0; i < d; ++i) orot[i] = den > 0.0 ? orot[i] / den : 0.0;
-        orc_rotate_t(d, v_signs, orot, out + (size_t)a * d);
+        orc_rotate_t(d, v_signs, v_Rm, orot, out + (size_t)a * d);
         if (logits) {
             for (int t = 0; t < L; ++t) logits[(size_t)a * L + t] = t < nv ? est[t] : -INFINITY;
         }

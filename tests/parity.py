@@ -117,7 +117,7 @@ def exempt_slack(Pv: O.Params, Ev: O.Encoded, exempt: np.ndarray, logits: np.nda
     ex = np.flatnonzero(exempt)
     if ex.size == 0:
         return slack
-    vhat = O.rotate_t(Ev.nhat[ex, None] * Pv.c32.astype(np.float64)[Ev.idx[ex]], Pv.signs)
+    vhat = O.rotate_t(Ev.nhat[ex, None] * Pv.c32.astype(np.float64)[Ev.idx[ex]], Pv.signs, Pv.Rm)
     vmax = np.abs(vhat).max(1)
     for r in range(rows):
         p = np.exp(logits[r, ex] - lse[r])

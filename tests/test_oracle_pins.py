@@ -485,3 +485,72 @@ def test_attend_with_fp8_keys_equals_textbook_softmax_on_exactly_coded_kv():
     assert np.allclose(logits, lg, atol=1e-11, rtol=0)
     assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-11, rtol=0)
     assert np.allclose(lse, scipy.special.logsumexp(lg, axis=1), atol=1e-11, rtol=0)
+
+
+# --------------------------------------------------------------------------
+# dense random rotation (the alternative to H D / sqrt(d))
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d,seed", [(8, 3), (128, 5), (256, 6)])
+def test_dense_rotation_is_numpy_qr_in_float32(d, seed):
+    G, Q, Rm = O.dense_rotation(d, seed)
+    # G: iid N(0,1) from its own stream (moments; a KS test against scipy's normal law)
+    g = G.ravel()
+    assert abs(g.mean()) < 5 / math.sqrt(g.size) and abs(g.var() - 1.0) < 5 * math.sqrt(2.0 / g.size)
+    if d >= 128:
+        assert scipy.stats.kstest(g, "norm").pvalue > 1e-4
+    # rows of Q = Gram-Schmidt of the rows of G = numpy's QR of G^T with a positive diagonal
+    q, r = np.linalg.qr(G.T)
+    q = q * np.sign(np.diag(r))[None, :]
+    assert np.allclose(Q, q.T, atol=1e-10, rtol=0)
+    # stored entries: numpy's float32 rounding of Q
+    assert np.array_equal(Rm, Q.astype(np.float32).astype(np.float64))
+    # orthogonal to float32 precision
+    assert np.max(np.abs(Rm @ Rm.T - np.eye(d))) < 1e-6
+    # the rotation routines use it (y = Rm x, x = Rm^T y)
+    P = O.make_params(d, 2, seed, with_S=False, rotation="dense")
+    X = np.random.default_rng(d).standard_normal((5, d))
+    assert np.allclose(O.rotate(X, P.signs, P.Rm), X @ Rm.T, atol=1e-12, rtol=0)
+    assert np.allclose(O.rotate_t(X, P.signs, P.Rm), X @ Rm, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_dense_rotation_bucketize_is_nearest_codeword_bruteforce(bits):
+    d = 8
+    P = O.make_params(d, bits, seed=12, rotation="dense")
+    L = 1 << bits
+    X = np.random.default_rng(20 + bits).standard_normal((4, d))
+    enc = O.encode(X, P, qjl=False)
+    Y = X @ P.Rm.T
+    U = Y / np.linalg.norm(Y, axis=1, keepdims=True)            # n = ||R x|| for the dense rotation
+    assert np.allclose(enc.nraw, np.linalg.norm(Y, axis=1), rtol=1e-14)
+    c = P.c32.astype(np.float64)
+    digits = (np.arange(L ** d)[:, None] // (L ** np.arange(d))[None, :]) % L
+    for v in range(X.shape[0]):
+        dist = ((U[v][None, :] - c[digits]) ** 2).sum(1)
+        assert np.array_equal(digits[int(np.argmin(dist))], enc.idx[v].astype(np.int64))
+
+
+def test_dense_rotation_mse_within_pages_bound_and_attention_textbook():
+    d, n, bits = 128, 20000, 3
+    P = O.make_params(d, bits, seed=31, with_S=False, rotation="dense")
+    X = np.random.default_rng(5).standard_normal((n, d)) * np.exp(np.random.default_rng(6).standard_normal(d))
+    enc = O.encode(X, P, qjl=False, margins=False)
+    Y = X @ P.Rm.T
+    rec = enc.nhat[:, None] * P.c32.astype(np.float64)[enc.idx]
+    nmse = np.mean(np.sum((Y - rec) ** 2, 1) / np.sum(Y ** 2, 1))
+    bound = _gold("pages_numbers.json")["distortion_factor_vs_information_limit"]["value"] * 4.0 ** -bits
+    assert nmse <= bound, (nmse, bound)
+    # attention with dense rotations, on K/V the codes represent exactly
+    rng = np.random.default_rng(7)
+    L = 200
+    Pk, Pv = O.make_params(d, 4, 41, with_S=False, rotation="dense"), O.make_params(d, 2, 42, with_S=False,
+                                                                                     rotation="dense")
+    kidx, vidx = rng.integers(0, 16, (L, d)).astype(np.uint8), rng.integers(0, 4, (L, d)).astype(np.uint8)
+    kn, vn = (np.array([O.round_fp16(v) for v in rng.uniform(1.0, 9.0, L)]) for _ in range(2))
+    Kx = (kn[:, None] * Pk.c32.astype(np.float64)[kidx]) @ Pk.Rm
+    Vx = (vn[:, None] * Pv.c32.astype(np.float64)[vidx]) @ Pv.Rm
+    Q = rng.standard_normal((3, d))
+    out, lse, _ = O.attend(Q, Pk, O.Encoded(4, False, kidx, kn), Pv, O.Encoded(2, False, vidx, vn))
+    lg = Q @ Kx.T / math.sqrt(d)               # <Rm q, nhat c> = <q, Rm^T nhat c>
+    assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-10, rtol=0)
+    assert np.allclose(lse, scipy.special.logsumexp(lg, axis=1), atol=1e-10, rtol=0)
