@@ -71,10 +71,11 @@ def _load():
     lib.orc_rotate.argtypes = [i32, vp, vp, vp, vp]
     lib.orc_rotate_t.argtypes = [i32, vp, vp, vp, vp]
     lib.orc_dense_rotation.argtypes = [i32, u64, vp, vp, vp]
-    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_encode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                               i32, vp, vp]
     lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_estimate.argtypes = [vp, i32, vp, vp]
-    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_attend_exact.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     lib.orc_search.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     _lib = lib
@@ -128,6 +129,17 @@ class Params:
     t32: np.ndarray | None       # float32 boundaries
     iters: int = 0
     Rm: np.ndarray | None = None  # dense rotation [d, d] (None: H D / sqrt(d))
+    # fractional rates (bits = b + 1/2): coordinates d/2 .. d-1 use b bits
+    # (bits2 = b) with their own codebook; coordinates 0 .. d/2-1 use b + 1
+    bits2: int = 0
+    c32b: np.ndarray | None = None
+    t32b: np.ndarray | None = None
+    c64b: np.ndarray | None = None
+
+    @property
+    def rate(self):
+        """Bits per coordinate: bits, or bits - 1/2 for a fractional rate."""
+        return self.bits - 0.5 if self.bits2 else self.bits
 
 
 def make_params(d: int, bits: int, seed: int, with_S: bool = True, rotation: str = "hadamard") -> Params:
@@ -144,16 +156,21 @@ def make_params(d: int, bits: int, seed: int, with_S: bool = True, rotation: str
         lib.orc_gauss_bf16(d, d, seed, _p(S))
     c64 = c32 = t32 = None
     iters = 0
+    bits2, cb = 0, (None, None, None)
+    if bits in (1.5, 2.5, 3.5):
+        bits2 = int(bits - 0.5)
+        bits = bits2 + 1
+        cb = codebook(d, bits2)
     if bits in (1, 2, 3, 4):
         c64, c32, t32 = codebook(d, bits)
     elif bits != 8:
-        raise ValueError("bits must be 1..4 or 8")
+        raise ValueError("bits must be 1..4, 8 or 1.5, 2.5, 3.5")
     Rm = None
     if rotation == "dense":
         Rm = dense_rotation(d, seed)[2]
     elif rotation != "hadamard":
         raise ValueError("rotation must be 'hadamard' or 'dense'")
-    return Params(d, bits, seed, signs, S, c64, c32, t32, iters, Rm)
+    return Params(d, bits, seed, signs, S, c64, c32, t32, iters, Rm, bits2, cb[1], cb[2], cb[0])
 
 
 def dense_rotation(d: int, seed: int):
@@ -251,8 +268,9 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
     nraw = np.zeros(n, np.float64)
     rraw = np.zeros(n, np.float64) if qjl else None
     lib.orc_encode(n, d, P.bits, 1 if qjl else 0, _p(X), _p(P.signs), _p(P.Rm), _p(P.S), _p(P.c32),
-                   _p(P.t32), _p(idx), _p(nhat), _p(rho), _p(sb), _p(um), _p(zm), _p(nraw), _p(rraw))
-    return Encoded(P.bits, qjl, idx, nhat, rho, sb, um, zm, nraw, rraw)
+                   _p(P.t32), _p(idx), _p(nhat), _p(rho), _p(sb), _p(um), _p(zm), _p(nraw), _p(rraw),
+                   P.bits2, _p(P.c32b), _p(P.t32b))
+    return Encoded(P.rate, qjl, idx, nhat, rho, sb, um, zm, nraw, rraw)
 
 
 # ---------------------------------------------------------------------------
@@ -262,14 +280,15 @@ class _Keys(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("qjl", ctypes.c_int), ("d", ctypes.c_int),
                 ("signs", ctypes.c_void_p), ("S", ctypes.c_void_p), ("c32", ctypes.c_void_p),
                 ("idx", ctypes.c_void_p), ("fp8", ctypes.c_void_p), ("nhat", ctypes.c_void_p),
-                ("rho", ctypes.c_void_p), ("sbits", ctypes.c_void_p), ("Rm", ctypes.c_void_p)]
+                ("rho", ctypes.c_void_p), ("sbits", ctypes.c_void_p), ("Rm", ctypes.c_void_p),
+                ("c32b", ctypes.c_void_p)]
 
 
 def _keys(P: Params, E: Encoded, keep: list) -> _Keys:
     arrs = [np.ascontiguousarray(a) if a is not None else None
-            for a in (P.signs, P.S, P.c32, E.idx, E.nhat, E.rho, E.sbits, P.Rm)]
+            for a in (P.signs, P.S, P.c32, E.idx, E.nhat, E.rho, E.sbits, P.Rm, P.c32b)]
     keep.extend(arrs)
-    signs, S, c32, idx, nhat, rho, sb, Rm = arrs
+    signs, S, c32, idx, nhat, rho, sb, Rm, c32b = arrs
     k = _Keys()
     k.kind = 1 if E.bits == 8 else 0
     k.qjl = 1 if E.qjl else 0
@@ -283,6 +302,7 @@ def _keys(P: Params, E: Encoded, keep: list) -> _Keys:
     k.rho = _p(rho)
     k.sbits = _p(sb)
     k.Rm = _p(Rm)
+    k.c32b = _p(c32b)
     return k
 
 
@@ -312,7 +332,8 @@ def attend(Q: np.ndarray, Pk: Params, Ek: Encoded, Pv: Params, Ev: Encoded,
     nv = None if nvis is None else np.ascontiguousarray(nvis, np.int32)
     vs, vc, vi, vn = (np.ascontiguousarray(a) for a in (Pv.signs, Pv.c32, Ev.idx, Ev.nhat))
     vR = None if Pv.Rm is None else np.ascontiguousarray(Pv.Rm)
-    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), _p(vc), _p(vi),
+    vcb = None if Pv.c32b is None else np.ascontiguousarray(Pv.c32b)
+    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), _p(vc), _p(vcb), _p(vi),
                        _p(vn), _p(logits), _p(out), _p(lse))
     return out, lse, logits
 
@@ -344,7 +365,8 @@ def search(Q: np.ndarray, P: Params, E: Encoded, k: int):
 class Layout:
     """Structure-of-arrays page of ``page_tokens`` tokens of one KV head.
 
-    kbits: 1..4 Lloyd-Max bits or 8 for FP8 keys; kqjl: QJL sign bits + rho;
+    kbits: 1..4 Lloyd-Max bits, 1.5 / 2.5 / 3.5 (fractional rates) or 8 for
+    FP8 keys; kqjl: QJL sign bits + rho;
     vbits: 1..4, or 0 for no value fields (a search database).  Fields in order, each padded to 16 bytes:
       K codes  ("kc" for w in {1,2,4}; "kc_lo" (2-bit) + "kc_hi" (1-bit) for 3
                bits; "k8" bytes for FP8), "ks" QJL sign bits, "kn" fp16 norm,
@@ -367,14 +389,18 @@ class Layout:
             self.fields[name] = (off, bytes_per_token)
             off += -(-(P * bytes_per_token) // 16) * 16
 
-        def codes(prefix, bits):
+        def codes(prefix, bits, n=d):
             if bits == 8:
-                add(prefix[0] + "8", d)
+                add(prefix[0] + "8", n)
+            elif bits != int(bits):
+                # fractional rate b + 1/2: coordinates 0 .. d/2-1 with b + 1 bits, then d/2 .. d-1 with b
+                codes(prefix + "A", int(bits + 0.5), d // 2)
+                codes(prefix + "B", int(bits - 0.5), d // 2)
             elif bits == 3:
-                add(prefix + "_lo", d * 2 // 8)
-                add(prefix + "_hi", d // 8)
+                add(prefix + "_lo", n * 2 // 8)
+                add(prefix + "_hi", n // 8)
             else:
-                add(prefix, d * bits // 8)
+                add(prefix, n * int(bits) // 8)
 
         codes("kc", self.kbits)
         if self.kqjl:
@@ -432,9 +458,15 @@ def _fp16_bytes(v: np.ndarray) -> np.ndarray:
     return np.asarray(v, np.float64).astype(np.float16).view(np.uint8).reshape(-1, 2)
 
 
-def _code_arrays(prefix: str, bits: int, codes: np.ndarray) -> dict:
+def _code_arrays(prefix: str, bits, codes: np.ndarray) -> dict:
     if bits == 8:
         return {prefix[0] + "8": codes.astype(np.uint8)}
+    if bits != int(bits):
+        h = codes.shape[1] // 2
+        out = _code_arrays(prefix + "A", int(bits + 0.5), codes[:, :h])
+        out.update(_code_arrays(prefix + "B", int(bits - 0.5), codes[:, h:]))
+        return out
+    bits = int(bits)
     kap = to_kappa(codes, bits)
     if bits == 3:
         return {prefix + "_lo": pack_fields(kap & 3, 2), prefix + "_hi": pack_fields(kap >> 2, 1)}
@@ -484,13 +516,17 @@ def read_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_h
         r, c = _field_index(lay, slots, head, n_heads, off, bpt)
         raw[name] = np.ascontiguousarray(cache[r, c])
 
-    def codes(prefix, bits):
+    def codes(prefix, bits, n=d):
         if bits == 8:
             return raw[prefix[0] + "8"].copy()
+        if bits != int(bits):
+            return np.concatenate([codes(prefix + "A", int(bits + 0.5), d // 2),
+                                   codes(prefix + "B", int(bits - 0.5), d // 2)], axis=1)
+        bits = int(bits)
         if bits == 3:
-            kap = unpack_fields(raw[prefix + "_lo"], d, 2) | (unpack_fields(raw[prefix + "_hi"], d, 1) << 2)
+            kap = unpack_fields(raw[prefix + "_lo"], n, 2) | (unpack_fields(raw[prefix + "_hi"], n, 1) << 2)
         else:
-            kap = unpack_fields(raw[prefix], d, bits)
+            kap = unpack_fields(raw[prefix], n, bits)
         return from_kappa(kap, bits)
 
     out = {"kidx": codes("kc", lay.kbits),

@@ -352,7 +352,8 @@ void orc_rotate_t(int d, const int8_t *signs, const double *Rm, const double *y,
 
 /* Stage 1 plus optional stage 2 for n vectors of dimension d (row-major X).
  * Per vector: n = ||x||, y = R x, u = y / n (u = 0 for the zero vector),
- * idx_i = #{j : t_j <= u_i}, nhat = fp16(n), r = y - nhat * c[idx],
+ * idx_i = #{j : t_j <= u_i} (fractional rates, bits2 > 0: coordinates
+ * d/2 .. d-1 take the bits2-bit codebook c32b / t32b instead), nhat = fp16(n), r = y - nhat * c[idx],
  * rho = fp16(||r||), s_j = [ (S r)_j >= 0 ].
  * Diagnostics for the parity exemptions: umargin[i] = min_j |u_i - t_j|
  * (unit-vector units), zmargin[j] = |(S r)_j| / (||r|| ||S_j||), and the
@@ -361,9 +362,9 @@ void orc_rotate_t(int d, const int8_t *signs, const double *Rm, const double *y,
 void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *signs,
                 const double *Rm, const float *S, const float *c32, const float *t32, uint8_t *idx,
                 double *nhat, double *rho, uint8_t *sbits, double *umargin,
-                double *zmargin, double *nraw, double *rraw)
+                double *zmargin, double *nraw, double *rraw,
+                int bits2, const float *c32b, const float *t32b)
 {
-    int L = 1 << bits;
     #pragma omp parallel
     {
     double *y = (double *)malloc(sizeof(double) * d);
@@ -381,17 +382,21 @@ void orc_encode(int n, int d, int bits, int qjl, const double *X, const int8_t *
         nhat[v] = nh;
         if (nraw) nraw[v] = nn;
         for (int i = 0; i < d; ++i) {
+            /* fractional rates: coordinates d/2 .. d-1 use the second codebook */
+            int second = bits2 > 0 && i >= d / 2;
+            const float *t = second ? t32b : t32, *c = second ? c32b : c32;
+            int L = 1 << (second ? bits2 : bits);
             double u = nn > 0.0 ? y[i] / nn : 0.0;
             int k = 0;
             double mg = INFINITY;
             for (int j = 0; j + 1 < L; ++j) {
-                if ((double)t32[j] <= u) ++k;
-                double dist = fabs(u - (double)t32[j]);
+                if ((double)t[j] <= u) ++k;
+                double dist = fabs(u - (double)t[j]);
                 if (dist < mg) mg = dist;
             }
             idx[(size_t)v * d + i] = (uint8_t)k;
             if (umargin) umargin[(size_t)v * d + i] = mg;
-            r[i] = y[i] - nh * (double)c32[k];
+            r[i] = y[i] - nh * (double)c[k];
         }
         if (!qjl) continue;
         double rn = 0.0;
@@ -473,6 +478,7 @@ typedef struct {
     const double *rho;      /* [L] (QJL only) */
     const uint8_t *sbits;   /* [L][m] (QJL only) */
     const double *Rm;       /* dense rotation (row-major d x d) or NULL */
+    const float *c32b;      /* fractional rates: levels of coordinates d/2 .. d-1, or NULL */
 } orc_keys_t;
 
 /* Estimates of <q, k_t> for t in [0, L):
@@ -499,7 +505,10 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
             for (int i = 0; i < d; ++i) e += qr[i] * orc_e4m3_value(K->fp8[(size_t)t * d + i]);
             e = K->nhat[t] * e / sqrt((double)d);
         } else {
-            for (int i = 0; i < d; ++i) e += qr[i] * (double)K->c32[K->idx[(size_t)t * d + i]];
+            for (int i = 0; i < d; ++i) {
+                const float *c = (K->c32b && i >= d / 2) ? K->c32b : K->c32;
+                e += qr[i] * (double)c[K->idx[(size_t)t * d + i]];
+            }
             e *= K->nhat[t];
             if (K->qjl) {
                 double s = 0.0;
@@ -521,7 +530,8 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
  * logits [nq][L] (positions past nvis set to -inf) and lse [nq] (natural log
  * of the softmax denominator of the scaled logits). */
 void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const orc_keys_t *K,
-                const int8_t *v_signs, const double *v_Rm, const float *v_c32, const uint8_t *v_idx,
+                const int8_t *v_signs, const double *v_Rm, const float *v_c32, const float *v_c32b,
+                const uint8_t *v_idx,
                 const double *v_nhat, double *logits, double *out, double *lse)
 {
     double *est = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
@@ -538,7 +548,10 @@ void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const or
             double p = exp(est[t] - mx);
             den += p;
             double pv = p * v_nhat[t];
-            for (int i = 0; i < d; ++i) orot[i] += pv * (double)v_c32[v_idx[(size_t)t * d + i]];
+            for (int i = 0; i < d; ++i) {
+                const float *c = (v_c32b && i >= d / 2) ? v_c32b : v_c32;
+                orot[i] += pv * (double)c[v_idx[(size_t)t * d + i]];
+            }
         }
         for (int i = 0; i < d; ++i) orot[i] = den > 0.0 ? orot[i] / den : 0.0;
         orc_rotate_t(d, v_signs, v_Rm, orot, out + (size_t)a * d);

@@ -103,6 +103,16 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     return 0.5 * 2.0 ** (np.maximum(e, -126) - 7)
 
 
+def levels_of(P: O.Params, idx: np.ndarray) -> np.ndarray:
+    """Float64 levels of bucket indices [n, d] (fractional rates: the second
+    codebook for coordinates d/2 .. d-1)."""
+    lv = P.c32.astype(np.float64)[idx]
+    if P.bits2:
+        h = idx.shape[1] // 2
+        lv[:, h:] = P.c32b.astype(np.float64)[idx[:, h:]]
+    return lv
+
+
 def exempt_slack(Pv: O.Params, Ev: O.Encoded, exempt: np.ndarray, logits: np.ndarray, lse: np.ndarray,
                  out: np.ndarray) -> np.ndarray:
     """Per-row bound on how far exempt keys can legitimately move an output.
@@ -117,7 +127,7 @@ def exempt_slack(Pv: O.Params, Ev: O.Encoded, exempt: np.ndarray, logits: np.nda
     ex = np.flatnonzero(exempt)
     if ex.size == 0:
         return slack
-    vhat = O.rotate_t(Ev.nhat[ex, None] * Pv.c32.astype(np.float64)[Ev.idx[ex]], Pv.signs, Pv.Rm)
+    vhat = O.rotate_t(Ev.nhat[ex, None] * levels_of(Pv, Ev.idx[ex]), Pv.signs, Pv.Rm)
     vmax = np.abs(vhat).max(1)
     for r in range(rows):
         p = np.exp(logits[r, ex] - lse[r])

@@ -554,3 +554,94 @@ def test_dense_rotation_mse_within_pages_bound_and_attention_textbook():
     lg = Q @ Kx.T / math.sqrt(d)               # <Rm q, nhat c> = <q, Rm^T nhat c>
     assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-10, rtol=0)
     assert np.allclose(lse, scipy.special.logsumexp(lg, axis=1), atol=1e-10, rtol=0)
+
+
+# --------------------------------------------------------------------------
+# fractional rates b + 1/2: coordinates 0 .. d/2-1 at b + 1 bits, the rest at b
+# --------------------------------------------------------------------------
+def test_fractional_rate_bucketize_is_nearest_codeword_bruteforce():
+    d, rate = 8, 2.5
+    P = O.make_params(d, rate, seed=13)
+    assert (P.bits, P.bits2) == (3, 2)
+    X = np.random.default_rng(25).standard_normal((3, d))
+    enc = O.encode(X, P, qjl=False)
+    U = O.rotate(X, P.signs) / np.linalg.norm(X, axis=1, keepdims=True)
+    ca, cb = P.c32.astype(np.float64), P.c32b.astype(np.float64)
+    da = (np.arange(8 ** 4)[:, None] // (8 ** np.arange(4))[None, :]) % 8
+    db = (np.arange(4 ** 4)[:, None] // (4 ** np.arange(4))[None, :]) % 4
+    for v in range(3):
+        # the squared error separates over the two halves: each half's nearest codeword independently
+        ea = ((U[v, :4][None, :] - ca[da]) ** 2).sum(1)
+        eb = ((U[v, 4:][None, :] - cb[db]) ** 2).sum(1)
+        best = np.concatenate([da[int(np.argmin(ea))], db[int(np.argmin(eb))]])
+        assert np.array_equal(best, enc.idx[v].astype(np.int64))
+        # and the joint search over all 8^4 x 4^4 code vectors agrees
+        tot = ea[:, None] + eb[None, :]
+        ia, ib = np.unravel_index(int(np.argmin(tot)), tot.shape)
+        assert np.array_equal(np.concatenate([da[ia], db[ib]]), enc.idx[v].astype(np.int64))
+
+
+@pytest.mark.parametrize("rate", [1.5, 2.5, 3.5])
+def test_fractional_rate_mse_is_the_mean_of_its_two_codebooks(rate):
+    d, n = 128, 40000
+    P = O.make_params(d, rate, seed=27, with_S=False)
+    X = np.random.default_rng(int(rate * 10)).standard_normal((n, d))
+    enc = O.encode(X, P, qjl=False, margins=False)
+    Y = O.rotate(X, P.signs)
+    lv = np.concatenate([P.c32.astype(np.float64)[enc.idx[:, :64]], P.c32b.astype(np.float64)[enc.idx[:, 64:]]], 1)
+    nmse = np.mean(np.sum((Y - enc.nhat[:, None] * lv) ** 2, 1) / np.sum(X ** 2, 1))
+    law = _coord_law(d)
+
+    def dist(c, t):
+        e = np.concatenate([[-1.0], t.astype(np.float64), [1.0]])
+        c = c.astype(np.float64)
+        return d * sum(scipy.integrate.quad(lambda x, cj=c[j]: (x - cj) ** 2 * law.pdf(x), e[j], e[j + 1],
+                                            epsabs=1e-14, limit=400)[0] for j in range(len(c)))
+    pred = 0.5 * (dist(P.c32, P.t32) + dist(P.c32b, P.t32b))
+    assert abs(nmse - pred) / pred < 0.02, (nmse, pred)
+    lo, hi = O.make_params(d, P.bits, 1, with_S=False), O.make_params(d, P.bits2, 1, with_S=False)
+    assert dist(lo.c32, lo.t32) < nmse < dist(hi.c32, hi.t32)
+
+
+@pytest.mark.parametrize("kbits,kqjl,vbits,per_token", [(2.5, True, 3.5, 40 + 16 + 4 + 56 + 2),
+                                                        (1.5, True, 2.5, 24 + 16 + 4 + 40 + 2),
+                                                        (3.5, False, 2.5, 56 + 2 + 40 + 2)])
+def test_fractional_layout_byte_counts_and_roundtrip(kbits, kqjl, vbits, per_token):
+    d = 128
+    lay = O.Layout(d, kbits, kqjl, vbits, page_tokens=16)
+    assert lay.page_bytes == 16 * per_token
+    rng = np.random.default_rng(3)
+    Pk, Pv = O.make_params(d, kbits, 1), O.make_params(d, vbits, 2, with_S=False)
+    X = rng.standard_normal((20, d))
+    Ek, Ev = O.encode(X, Pk, qjl=kqjl), O.encode(X[::-1].copy(), Pv, qjl=False)
+    cache = np.zeros((2 * 2, lay.page_bytes), np.uint8)
+    slots = rng.permutation(32)[:20]
+    O.write_cache(lay, cache, slots, 0, 2, Ek, Ev)
+    back = O.read_cache(lay, cache, slots, 0, 2)
+    assert np.array_equal(back["kidx"], Ek.idx) and np.array_equal(back["vidx"], Ev.idx)
+    assert int(Ek.idx[:, :64].max()) < (1 << Pk.bits) and int(Ek.idx[:, 64:].max()) < (1 << Pk.bits2)
+
+
+def test_fractional_rate_attention_and_qjl_unbiased():
+    d = 128
+    rng = np.random.default_rng(17)
+    Pk, Pv = O.make_params(d, 3.5, 51, with_S=False), O.make_params(d, 2.5, 52, with_S=False)
+    L = 150
+    kidx = np.concatenate([rng.integers(0, 16, (L, 64)), rng.integers(0, 8, (L, 64))], 1).astype(np.uint8)
+    vidx = np.concatenate([rng.integers(0, 8, (L, 64)), rng.integers(0, 4, (L, 64))], 1).astype(np.uint8)
+    kn, vn = (np.array([O.round_fp16(v) for v in rng.uniform(1.0, 9.0, L)]) for _ in range(2))
+    H = scipy.linalg.hadamard(d).astype(np.float64)
+    R = lambda P: H @ np.diag(P.signs.astype(np.float64)) / math.sqrt(d)
+    lvk = np.concatenate([Pk.c32.astype(np.float64)[kidx[:, :64]], Pk.c32b.astype(np.float64)[kidx[:, 64:]]], 1)
+    lvv = np.concatenate([Pv.c32.astype(np.float64)[vidx[:, :64]], Pv.c32b.astype(np.float64)[vidx[:, 64:]]], 1)
+    Kx, Vx = (kn[:, None] * lvk) @ R(Pk), (vn[:, None] * lvv) @ R(Pv)
+    Q = rng.standard_normal((3, d))
+    out, lse, _ = O.attend(Q, Pk, O.Encoded(3.5, False, kidx, kn), Pv, O.Encoded(2.5, False, vidx, vn))
+    lg = Q @ Kx.T / math.sqrt(d)
+    assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-10, rtol=0)
+    # stage 2 keeps the 2.5-bit estimate unbiased
+    k = rng.standard_normal(d)
+    q = rng.standard_normal(d) + 0.7 * k
+    est = np.array([O.estimate(q, P, O.encode(k[None, :], P, qjl=True, margins=False))[0]
+                    for P in (O.make_params(d, 2.5, 3000 + s) for s in range(3000))])
+    assert abs(est.mean() - q @ k) < 3 * est.std(ddof=1) / math.sqrt(len(est))
