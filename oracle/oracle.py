@@ -75,7 +75,12 @@ def _load():
                                i32, vp, vp]
     lib.orc_encode_fp8.argtypes = [i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_estimate.argtypes = [vp, i32, vp, vp]
-    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_attend.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_polar_codebook.restype = i32
+    lib.orc_polar_codebook.argtypes = [i32, i32, vp, vp, vp]
+    lib.orc_polar_decode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.orc_encode_polar.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                     vp, vp, vp, vp, vp, vp]
     lib.orc_attend_exact.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     lib.orc_search.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     _lib = lib
@@ -274,6 +279,105 @@ def encode(X: np.ndarray, P: Params, qjl: bool, margins: bool = True) -> Encoded
 
 
 # ---------------------------------------------------------------------------
+# PolarQuant: the polar-coordinate angle quantizer
+# ---------------------------------------------------------------------------
+@dataclass
+class PolarParams:
+    """Parameters of the polar quantizer: the rotation (signs / dense Rm), S
+    for QJL, level-1 angle codebook (b1 bits, uniform cells on [0, 2 pi)) and
+    one Lloyd-Max codebook of bh bits per level l = 2 .. log2 d."""
+    d: int
+    b1: int
+    bh: int
+    seed: int
+    signs: np.ndarray
+    S: np.ndarray | None
+    c1: np.ndarray          # float32 [2^b1] level-1 centroids
+    t1: np.ndarray          # float32 [2^b1 - 1] boundaries (midpoints of the fp32 centroids)
+    ch: np.ndarray          # float32 [log2 d - 1][2^bh]
+    th: np.ndarray          # float32 [log2 d - 1][2^bh - 1]
+    ch64: np.ndarray        # float64 levels
+    Rm: np.ndarray | None = None
+    bits: str = "polar"
+
+
+def polar_params(d: int, seed: int, b1: int = 4, bh: int = 2, with_S: bool = True,
+                 rotation: str = "hadamard") -> PolarParams:
+    base = make_params(d, 8, seed, with_S=with_S, rotation=rotation)
+    L1 = 1 << b1
+    c1_64 = (np.arange(L1) + 0.5) * (2.0 * np.pi / L1)      # the uniform law's Lloyd-Max levels: cell centres
+    c1 = c1_64.astype(np.float32)
+    t1 = ((c1[:-1].astype(np.float64) + c1[1:]) / 2).astype(np.float32)
+    levels = int(np.log2(d))
+    H = 1 << bh
+    ch = np.zeros((levels - 1, H), np.float32)
+    th = np.zeros((levels - 1, H - 1), np.float32)
+    ch64 = np.zeros((levels - 1, H), np.float64)
+    for l in range(2, levels + 1):
+        c64, c32, t32 = polar_codebook(1 << (l - 1), bh)
+        ch64[l - 2], ch[l - 2], th[l - 2] = c64, c32, t32
+    return PolarParams(d, b1, bh, seed, base.signs, base.S, c1, t1, ch, th, ch64, base.Rm)
+
+
+_polar_cache: dict = {}
+
+
+def polar_codebook(k: int, bits: int):
+    """(c64, c32, t32) of the level angle for sub-block dimension k."""
+    if (k, bits) not in _polar_cache:
+        L = 1 << bits
+        c64, c32, t32 = np.zeros(L), np.zeros(L, np.float32), np.zeros(L - 1, np.float32)
+        if _load().orc_polar_codebook(k, bits, _p(c64), _p(c32), _p(t32)) < 0:
+            raise RuntimeError("polar Lloyd-Max iteration did not converge")
+        _polar_cache[(k, bits)] = (c64, c32, t32)
+    return _polar_cache[(k, bits)]
+
+
+@dataclass
+class PolarEncoded:
+    qjl: bool
+    codes1: np.ndarray      # uint8 [n, d/2] level-1 angle codes
+    codesh: np.ndarray      # uint8 [n, d/2 - 1] higher-level codes (level 2 first)
+    nhat: np.ndarray
+    yhat: np.ndarray        # float64 [n, d] reconstruction in the rotated basis
+    rho: np.ndarray | None = None
+    sbits: np.ndarray | None = None
+    margin1: np.ndarray | None = None
+    marginh: np.ndarray | None = None
+    zmargin: np.ndarray | None = None
+    nraw: np.ndarray | None = None
+    rraw: np.ndarray | None = None
+    bits: str = "polar"
+
+
+def encode_polar(X: np.ndarray, P: PolarParams, qjl: bool) -> PolarEncoded:
+    X = np.ascontiguousarray(X, np.float64)
+    n, d = X.shape
+    h = d // 2
+    c1, cd = np.zeros((n, h), np.uint8), np.zeros((n, h - 1), np.uint8)
+    nhat, yhat, nraw = np.zeros(n), np.zeros((n, d)), np.zeros(n)
+    m1, mh = np.zeros((n, h)), np.zeros((n, h - 1))
+    rho = np.zeros(n) if qjl else None
+    sb = np.zeros((n, d), np.uint8) if qjl else None
+    zm = np.zeros((n, d)) if qjl else None
+    rr = np.zeros(n) if qjl else None
+    _load().orc_encode_polar(n, d, P.b1, P.bh, 1 if qjl else 0, _p(X), _p(P.signs), _p(P.Rm), _p(P.S), _p(P.c1),
+                             _p(P.t1), _p(np.ascontiguousarray(P.ch)), _p(np.ascontiguousarray(P.th)), _p(c1), _p(cd),
+                             _p(nhat), _p(yhat), _p(rho), _p(sb), _p(m1), _p(mh), _p(zm), _p(nraw), _p(rr))
+    return PolarEncoded(qjl, c1, cd, nhat, yhat, rho, sb, m1, mh, zm, nraw, rr)
+
+
+def polar_decode(codes1: np.ndarray, codesh: np.ndarray, nhat: np.ndarray, P: PolarParams) -> np.ndarray:
+    n, h = codes1.shape
+    d = 2 * h
+    yhat = np.zeros((n, d))
+    _load().orc_polar_decode(n, d, P.b1, P.bh, _p(np.ascontiguousarray(codes1, np.uint8)),
+                             _p(np.ascontiguousarray(codesh, np.uint8)), _p(np.ascontiguousarray(nhat, np.float64)),
+                             _p(P.c1), _p(np.ascontiguousarray(P.ch)), _p(yhat))
+    return yhat
+
+
+# ---------------------------------------------------------------------------
 # estimator, attention, search
 # ---------------------------------------------------------------------------
 class _Keys(ctypes.Structure):
@@ -281,10 +385,19 @@ class _Keys(ctypes.Structure):
                 ("signs", ctypes.c_void_p), ("S", ctypes.c_void_p), ("c32", ctypes.c_void_p),
                 ("idx", ctypes.c_void_p), ("fp8", ctypes.c_void_p), ("nhat", ctypes.c_void_p),
                 ("rho", ctypes.c_void_p), ("sbits", ctypes.c_void_p), ("Rm", ctypes.c_void_p),
-                ("c32b", ctypes.c_void_p)]
+                ("c32b", ctypes.c_void_p), ("yhat", ctypes.c_void_p)]
 
 
-def _keys(P: Params, E: Encoded, keep: list) -> _Keys:
+def _keys(P, E, keep: list) -> _Keys:
+    if isinstance(E, PolarEncoded):
+        arrs = [np.ascontiguousarray(a) if a is not None else None
+                for a in (P.signs, P.S, E.nhat, E.rho, E.sbits, P.Rm, E.yhat)]
+        keep.extend(arrs)
+        signs, S, nhat, rho, sb, Rm, yh = arrs
+        k = _Keys()
+        k.kind, k.qjl, k.d = 2, 1 if E.qjl else 0, P.d
+        k.signs, k.S, k.nhat, k.rho, k.sbits, k.Rm, k.yhat = (_p(a) for a in (signs, S, nhat, rho, sb, Rm, yh))
+        return k
     arrs = [np.ascontiguousarray(a) if a is not None else None
             for a in (P.signs, P.S, P.c32, E.idx, E.nhat, E.rho, E.sbits, P.Rm, P.c32b)]
     keep.extend(arrs)
@@ -330,10 +443,15 @@ def attend(Q: np.ndarray, Pk: Params, Ek: Encoded, Pv: Params, Ev: Encoded,
     lse = np.zeros(nq, np.float64)
     logits = np.zeros((nq, L), np.float64) if want_logits else None
     nv = None if nvis is None else np.ascontiguousarray(nvis, np.int32)
-    vs, vc, vi, vn = (np.ascontiguousarray(a) for a in (Pv.signs, Pv.c32, Ev.idx, Ev.nhat))
     vR = None if Pv.Rm is None else np.ascontiguousarray(Pv.Rm)
+    if isinstance(Ev, PolarEncoded):
+        vs, vn, vy = (np.ascontiguousarray(a) for a in (Pv.signs, Ev.nhat, Ev.yhat))
+        _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), None, None, _p(vy), None,
+                           _p(vn), _p(logits), _p(out), _p(lse))
+        return out, lse, logits
+    vs, vc, vi, vn = (np.ascontiguousarray(a) for a in (Pv.signs, Pv.c32, Ev.idx, Ev.nhat))
     vcb = None if Pv.c32b is None else np.ascontiguousarray(Pv.c32b)
-    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), _p(vc), _p(vcb), _p(vi),
+    _load().orc_attend(nq, L, d, _p(Q), _p(nv), ctypes.byref(K), _p(vs), _p(vR), _p(vc), _p(vcb), None, _p(vi),
                        _p(vn), _p(logits), _p(out), _p(lse))
     return out, lse, logits
 
@@ -390,7 +508,11 @@ class Layout:
             off += -(-(P * bytes_per_token) // 16) * 16
 
         def codes(prefix, bits, n=d):
-            if bits == 8:
+            if bits == "polar":
+                # level-1 angles: 4-bit fields, d/2 of them; higher levels: 2-bit, d/2 slots (last unused)
+                add(prefix[0] + "p1", d // 2 * 4 // 8)
+                add(prefix[0] + "ph", d // 2 * 2 // 8)
+            elif bits == 8:
                 add(prefix[0] + "8", n)
             elif bits != int(bits):
                 # fractional rate b + 1/2: coordinates 0 .. d/2-1 with b + 1 bits, then d/2 .. d-1 with b
@@ -458,7 +580,12 @@ def _fp16_bytes(v: np.ndarray) -> np.ndarray:
     return np.asarray(v, np.float64).astype(np.float16).view(np.uint8).reshape(-1, 2)
 
 
-def _code_arrays(prefix: str, bits, codes: np.ndarray) -> dict:
+def _code_arrays(prefix: str, bits, codes) -> dict:
+    if bits == "polar":
+        E = codes
+        ph = np.zeros((E.codesh.shape[0], E.codesh.shape[1] + 1), np.uint8)
+        ph[:, :-1] = E.codesh
+        return {prefix[0] + "p1": pack_fields(E.codes1, 4), prefix[0] + "ph": pack_fields(ph, 2)}
     if bits == 8:
         return {prefix[0] + "8": codes.astype(np.uint8)}
     if bits != int(bits):
@@ -476,14 +603,14 @@ def _code_arrays(prefix: str, bits, codes: np.ndarray) -> dict:
 def token_records(lay: Layout, Ek: Encoded, Ev: Encoded) -> dict:
     """Per-token bytes of every field (name -> [n, bytes_per_token])."""
     rec = {}
-    rec.update(_code_arrays("kc", lay.kbits, Ek.idx))
+    rec.update(_code_arrays("kc", lay.kbits, Ek if lay.kbits == "polar" else Ek.idx))
     if lay.kqjl:
         rec["ks"] = pack_fields(Ek.sbits, 1)
     rec["kn"] = _fp16_bytes(Ek.nhat)
     if lay.kqjl:
         rec["kr"] = _fp16_bytes(Ek.rho)
     if lay.vbits > 0:
-        rec.update(_code_arrays("vc", lay.vbits, Ev.idx))
+        rec.update(_code_arrays("vc", lay.vbits, Ev if lay.vbits == "polar" else Ev.idx))
         rec["vn"] = _fp16_bytes(Ev.nhat)
     return rec
 
@@ -517,6 +644,9 @@ def read_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_h
         raw[name] = np.ascontiguousarray(cache[r, c])
 
     def codes(prefix, bits, n=d):
+        if bits == "polar":
+            return (unpack_fields(raw[prefix[0] + "p1"], d // 2, 4),
+                    unpack_fields(raw[prefix[0] + "ph"], d // 2, 2)[:, :-1].copy())
         if bits == 8:
             return raw[prefix[0] + "8"].copy()
         if bits != int(bits):

@@ -479,6 +479,7 @@ typedef struct {
     const uint8_t *sbits;   /* [L][m] (QJL only) */
     const double *Rm;       /* dense rotation (row-major d x d) or NULL */
     const float *c32b;      /* fractional rates: levels of coordinates d/2 .. d-1, or NULL */
+    const double *yhat;     /* kind 2 (polar codes): reconstruction y_hat [L][d] in the rotated basis */
 } orc_keys_t;
 
 /* Estimates of <q, k_t> for t in [0, L):
@@ -490,7 +491,7 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
     double *qr = (double *)malloc(sizeof(double) * d);
     double *w = (double *)malloc(sizeof(double) * m);
     orc_rotate(d, K->signs, K->Rm, q, qr);
-    if (K->kind == 0 && K->qjl) {
+    if (K->kind != 1 && K->qjl) {
         for (int j = 0; j < m; ++j) {
             double s = 0.0;
             for (int i = 0; i < d; ++i) s += (double)K->S[(size_t)j * d + i] * qr[i];
@@ -501,7 +502,15 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
     #pragma omp parallel for schedule(static)
     for (int t = 0; t < L; ++t) {
         double e = 0.0;
-        if (K->kind == 1) {
+        if (K->kind == 2) {
+            for (int i = 0; i < d; ++i) e += qr[i] * K->yhat[(size_t)t * d + i];
+            if (K->qjl) {
+                double s = 0.0;
+                for (int j = 0; j < m; ++j)
+                    s += (K->sbits[(size_t)t * m + j] ? 1.0 : -1.0) * w[j];
+                e += K->rho[t] * cq * s;
+            }
+        } else if (K->kind == 1) {
             for (int i = 0; i < d; ++i) e += qr[i] * orc_e4m3_value(K->fp8[(size_t)t * d + i]);
             e = K->nhat[t] * e / sqrt((double)d);
         } else {
@@ -531,7 +540,7 @@ void orc_estimate(const orc_keys_t *K, int L, const double *q, double *est)
  * of the softmax denominator of the scaled logits). */
 void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const orc_keys_t *K,
                 const int8_t *v_signs, const double *v_Rm, const float *v_c32, const float *v_c32b,
-                const uint8_t *v_idx,
+                const double *v_yhat, const uint8_t *v_idx,
                 const double *v_nhat, double *logits, double *out, double *lse)
 {
     double *est = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
@@ -548,6 +557,10 @@ void orc_attend(int nq, int L, int d, const double *Q, const int *nvis, const or
             double p = exp(est[t] - mx);
             den += p;
             double pv = p * v_nhat[t];
+            if (v_yhat) {               /* polar values: y_hat already carries nhat */
+                for (int i = 0; i < d; ++i) orot[i] += p * v_yhat[(size_t)t * d + i];
+                continue;
+            }
             for (int i = 0; i < d; ++i) {
                 const float *c = (v_c32b && i >= d / 2) ? v_c32b : v_c32;
                 orot[i] += pv * (double)c[v_idx[(size_t)t * d + i]];
@@ -617,4 +630,220 @@ void orc_search(int nq, int n_db, int k, const double *Q, const orc_keys_t *K,
         }
     }
     free(est);
+}
+
+/* ------------------------------------------------------------------------ */
+/* PolarQuant: the polar-coordinate angle quantizer ("What is TurboQuant?",  */
+/* "Stage 1": the standalone PolarQuant maps the rotated vector to polar     */
+/* coordinates and quantizes the angles, so that no per-vector scale other   */
+/* than the final radius is stored).                                         */
+/*                                                                           */
+/* Transform of y in R^d (d = 2^L): level 1 takes the pairs (y_2p, y_2p+1)   */
+/* to radii r1_p and angles theta_p = atan2(y_2p+1, y_2p) in [0, 2 pi);      */
+/* level l = 2 .. L takes pairs of level-(l-1) radii (a, b) to sqrt(a^2+b^2) */
+/* and psi = atan2(b, a) in [0, pi/2].  The level-L radius is ||y||.         */
+/* Codes: theta on 2^b1 uniform cells of [0, 2 pi) (the Lloyd-Max quantizer  */
+/* of the uniform law: cell centres); psi of level l by the Lloyd-Max        */
+/* quantizer, 2^bh levels, of its law for a uniformly random direction:      */
+/* density proportional to (sin psi cos psi)^(k-1), k = 2^(l-1).             */
+/* ------------------------------------------------------------------------ */
+typedef struct { double km1; int moment; } angle_dens_t;
+
+static double angle_dens(const angle_dens_t *D, double p)
+{
+    double s = sin(p) * cos(p);
+    if (s <= 0.0) return 0.0;
+    double f = exp(D->km1 * log(s));
+    return D->moment ? p * f : f;
+}
+
+static double angle_simpson(const angle_dens_t *D, double a, double b, double fa, double fm, double fb,
+                            double whole, int depth)
+{
+    double m = 0.5 * (a + b), lm = 0.5 * (a + m), rm = 0.5 * (m + b);
+    double flm = angle_dens(D, lm), frm = angle_dens(D, rm);
+    double left = (m - a) / 6.0 * (fa + 4.0 * flm + fm);
+    double right = (b - m) / 6.0 * (fm + 4.0 * frm + fb);
+    double delta = left + right - whole;
+    if (depth <= 0 || fabs(delta) <= 15.0 * 1e-17 + 3e-16 * fabs(left + right))
+        return left + right + delta / 15.0;
+    return angle_simpson(D, a, m, fa, flm, fm, left, depth - 1) + angle_simpson(D, m, b, fm, frm, fb, right, depth - 1);
+}
+
+static double angle_integrate(double km1, int moment, double a, double b)
+{
+    angle_dens_t D = {km1, moment};
+    double sum = 0.0;
+    const int panels = 64;
+    for (int p = 0; p < panels; ++p) {
+        double lo = a + (b - a) * p / panels, hi = a + (b - a) * (p + 1) / panels;
+        double fa = angle_dens(&D, lo), fb = angle_dens(&D, hi), fm = angle_dens(&D, 0.5 * (lo + hi));
+        sum += angle_simpson(&D, lo, hi, fa, fm, fb, (hi - lo) / 6.0 * (fa + 4.0 * fm + fb), 50);
+    }
+    return sum;
+}
+
+/* Lloyd-Max levels (c64, ascending) of psi for sub-block dimension k, with
+ * fp32 copies c32 and fp32 midpoint boundaries t32.  Start: pi/4 plus the
+ * normal quantiles scaled by 1 / (2 sqrt(k + 1)), clamped inside (0, pi/2);
+ * iterate midpoints / conditional means to 1e-13; symmetrise about pi/4.
+ * Returns the iteration count or -1. */
+int orc_polar_codebook(int k, int bits, double *c64, float *c32, float *t32)
+{
+    int L = 1 << bits;
+    double *c = (double *)malloc(sizeof(double) * L), *t = (double *)malloc(sizeof(double) * (L + 1));
+    const double q = M_PI / 4.0, sd = 0.5 / sqrt(k + 1.0);
+    for (int j = 0; j < L; ++j) {
+        double v = q + sd * normal_quantile((j + 0.5) / L);
+        c[j] = fmin(fmax(v, 1e-3), M_PI / 2.0 - 1e-3);
+    }
+    int it, ok = 0;
+    for (it = 1; it <= 100000; ++it) {
+        t[0] = 0.0;
+        t[L] = M_PI / 2.0;
+        for (int j = 1; j < L; ++j) t[j] = 0.5 * (c[j - 1] + c[j]);
+        double md = 0.0;
+        for (int j = 0; j < L; ++j) {
+            double nc = angle_integrate(k - 1.0, 1, t[j], t[j + 1]) / angle_integrate(k - 1.0, 0, t[j], t[j + 1]);
+            md = fmax(md, fabs(nc - c[j]));
+            c[j] = nc;
+        }
+        if (md < 1e-13) { ok = 1; break; }
+    }
+    for (int j = 0; j < L / 2; ++j) {
+        double s = 0.5 * (c[j] + (M_PI / 2.0 - c[L - 1 - j]));
+        c[j] = s;
+        c[L - 1 - j] = M_PI / 2.0 - s;
+    }
+    for (int j = 0; j < L; ++j) { c64[j] = c[j]; c32[j] = (float)c[j]; }
+    for (int j = 0; j + 1 < L; ++j) t32[j] = (float)(0.5 * ((double)c32[j] + (double)c32[j + 1]));
+    free(c);
+    free(t);
+    return ok ? it : -1;
+}
+
+/* Angle node order of the higher-level codes: level 2's d/4 angles, then
+ * level 3's d/8, ..., level L's one (d/2 - 1 in all). */
+static int polar_node(int d, int level, int i)
+{
+    int off = 0;
+    for (int l = 2; l < level; ++l) off += d >> l;
+    return off + i;
+}
+
+/* Reconstruction y_hat of polar codes: the level-L radius nhat, split top
+ * down by the centroid angles (fp32-stored values), level 1 by theta.
+ * c1: 2^b1 level-1 centroids; ch: per level l = 2 .. L (row l - 2) 2^bh
+ * centroids. */
+void orc_polar_decode(int n, int d, int b1, int bh, const uint8_t *codes1, const uint8_t *codesh,
+                      const double *nhat, const float *c1, const float *ch, double *yhat)
+{
+    int Lv = 0;
+    while ((1 << Lv) < d) ++Lv;
+    int H = 1 << bh;
+    double *r = (double *)malloc(sizeof(double) * d), *r2 = (double *)malloc(sizeof(double) * d);
+    for (int v = 0; v < n; ++v) {
+        r[0] = nhat[v];
+        for (int l = Lv; l >= 2; --l) {
+            int nodes = d >> l;
+            for (int i = 0; i < nodes; ++i) {
+                double psi = (double)ch[(size_t)(l - 2) * H + codesh[(size_t)v * (d / 2 - 1) + polar_node(d, l, i)]];
+                r2[2 * i] = r[i] * cos(psi);
+                r2[2 * i + 1] = r[i] * sin(psi);
+            }
+            memcpy(r, r2, sizeof(double) * 2 * nodes);
+        }
+        for (int p = 0; p < d / 2; ++p) {
+            double th = (double)c1[codes1[(size_t)v * (d / 2) + p]];
+            yhat[(size_t)v * d + 2 * p] = r[p] * cos(th);
+            yhat[(size_t)v * d + 2 * p + 1] = r[p] * sin(th);
+        }
+    }
+    free(r);
+    free(r2);
+}
+
+/* Encode with the polar quantizer: y = R x, n = ||x|| (||R x|| for the
+ * dense rotation), the angles of the transform, their codes, nhat = fp16(n);
+ * for QJL keys the residual r = y - y_hat(codes, nhat), rho = fp16(||r||) and
+ * s_j = [(S r)_j >= 0].  Margins (unit-vector units): |angle - nearest
+ * boundary| x (radius being split) / n, for level 1 the boundaries 0 and
+ * 2 pi included. */
+void orc_encode_polar(int n, int d, int b1, int bh, int qjl, const double *X, const int8_t *signs, const double *Rm,
+                      const float *S, const float *c1, const float *t1, const float *ch, const float *th,
+                      uint8_t *codes1, uint8_t *codesh, double *nhat, double *yhat, double *rho, uint8_t *sbits,
+                      double *margin1, double *marginh, double *zmargin, double *nraw, double *rraw)
+{
+    int Lv = 0;
+    while ((1 << Lv) < d) ++Lv;
+    int L1 = 1 << b1, H = 1 << bh;
+    #pragma omp parallel
+    {
+    double *y = (double *)malloc(sizeof(double) * d), *r = (double *)malloc(sizeof(double) * d);
+    double *r2 = (double *)malloc(sizeof(double) * d);
+    #pragma omp for schedule(static)
+    for (int v = 0; v < n; ++v) {
+        const double *x = X + (size_t)v * d;
+        orc_rotate(d, signs, Rm, x, y);
+        const double *nsrc = Rm ? y : x;
+        double nn = 0.0;
+        for (int i = 0; i < d; ++i) nn += nsrc[i] * nsrc[i];
+        nn = sqrt(nn);
+        nhat[v] = orc_round_fp16(nn);
+        if (nraw) nraw[v] = nn;
+        for (int p = 0; p < d / 2; ++p) {
+            double a = y[2 * p], b = y[2 * p + 1];
+            double t = atan2(b, a);
+            if (t < 0.0) t += 2.0 * M_PI;
+            int k = 0;
+            double mg = fmin(t, 2.0 * M_PI - t);
+            for (int j = 0; j + 1 < L1; ++j) {
+                if ((double)t1[j] <= t) ++k;
+                mg = fmin(mg, fabs(t - (double)t1[j]));
+            }
+            codes1[(size_t)v * (d / 2) + p] = (uint8_t)k;
+            r[p] = sqrt(a * a + b * b);
+            if (margin1) margin1[(size_t)v * (d / 2) + p] = nn > 0.0 ? mg * r[p] / nn : INFINITY;
+        }
+        for (int l = 2; l <= Lv; ++l) {
+            int nodes = d >> l;
+            for (int i = 0; i < nodes; ++i) {
+                double a = r[2 * i], b = r[2 * i + 1];
+                double psi = atan2(b, a), rr = sqrt(a * a + b * b);
+                const float *tl = th + (size_t)(l - 2) * (H - 1);
+                int k = 0;
+                double mg = INFINITY;
+                for (int j = 0; j + 1 < H; ++j) {
+                    if ((double)tl[j] <= psi) ++k;
+                    mg = fmin(mg, fabs(psi - (double)tl[j]));
+                }
+                codesh[(size_t)v * (d / 2 - 1) + polar_node(d, l, i)] = (uint8_t)k;
+                if (marginh) marginh[(size_t)v * (d / 2 - 1) + polar_node(d, l, i)] = nn > 0.0 ? mg * rr / nn : INFINITY;
+                r2[i] = rr;
+            }
+            memcpy(r, r2, sizeof(double) * nodes);
+        }
+        double *yh = yhat + (size_t)v * d;
+        orc_polar_decode(1, d, b1, bh, codes1 + (size_t)v * (d / 2), codesh + (size_t)v * (d / 2 - 1), nhat + v,
+                         c1, ch, yh);
+        if (!qjl) continue;
+        double rn = 0.0;
+        for (int i = 0; i < d; ++i) { r[i] = y[i] - yh[i]; rn += r[i] * r[i]; }
+        rn = sqrt(rn);
+        rho[v] = orc_round_fp16(rn);
+        if (rraw) rraw[v] = rn;
+        for (int j = 0; j < d; ++j) {
+            double z = 0.0, sn = 0.0;
+            for (int i = 0; i < d; ++i) {
+                z += (double)S[(size_t)j * d + i] * r[i];
+                sn += (double)S[(size_t)j * d + i] * (double)S[(size_t)j * d + i];
+            }
+            sbits[(size_t)v * d + j] = z >= 0.0 ? 1 : 0;
+            if (zmargin) zmargin[(size_t)v * d + j] = rn > 0.0 ? fabs(z) / (rn * sqrt(sn)) : INFINITY;
+        }
+    }
+    free(y);
+    free(r);
+    free(r2);
+    }
 }

@@ -645,3 +645,101 @@ def test_fractional_rate_attention_and_qjl_unbiased():
     est = np.array([O.estimate(q, P, O.encode(k[None, :], P, qjl=True, margins=False))[0]
                     for P in (O.make_params(d, 2.5, 3000 + s) for s in range(3000))])
     assert abs(est.mean() - q @ k) < 3 * est.std(ddof=1) / math.sqrt(len(est))
+
+
+# --------------------------------------------------------------------------
+# PolarQuant: the polar-coordinate angle quantizer
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("k", [2, 4, 16, 64])
+def test_polar_angle_codebook_fixed_point_under_beta_law(k):
+    # for a random direction, the angle psi between two k-dimensional
+    # sub-block radii has sin^2 psi ~ Beta(k/2, k/2) (ratio of chi-squares)
+    c64, c32, t32 = O.polar_codebook(k, 2)
+    law = scipy.stats.beta(k / 2, k / 2)
+    pdf = lambda p: law.pdf(math.sin(p) ** 2) * 2 * math.sin(p) * math.cos(p)
+    edges = np.concatenate([[0.0], 0.5 * (c64[:-1] + c64[1:]), [math.pi / 2]])
+    for j in range(4):
+        mass = scipy.integrate.quad(pdf, edges[j], edges[j + 1], epsabs=1e-14, limit=400)[0]
+        mom = scipy.integrate.quad(lambda p: p * pdf(p), edges[j], edges[j + 1], epsabs=1e-14, limit=400)[0]
+        assert abs(mom / mass - c64[j]) < 1e-9, (k, j)
+    assert np.allclose(c64 + c64[::-1], math.pi / 2, atol=1e-14)
+    assert np.all(t32 == ((c32[:-1].astype(np.float64) + c32[1:]) / 2).astype(np.float32))
+    # and the law itself: angles of Gaussian sub-blocks (numpy) pass a KS test against it
+    g = np.random.default_rng(k).standard_normal((20000, 2 * k))
+    psi = np.arctan2(np.linalg.norm(g[:, k:], axis=1), np.linalg.norm(g[:, :k], axis=1))
+    assert scipy.stats.kstest(np.sin(psi) ** 2, law.cdf).pvalue > 1e-4
+
+
+def test_polar_d2_and_d4_against_numpy():
+    P2 = O.polar_params(2, 3, with_S=False)
+    X = np.random.default_rng(1).standard_normal((200, 2))
+    E = O.encode_polar(X, P2, qjl=False)
+    Y = O.rotate(X, P2.signs)
+    th = np.mod(np.arctan2(Y[:, 1], Y[:, 0]), 2 * np.pi)
+    code = np.floor(th / (2 * np.pi / 16)).astype(int)
+    clear = E.margin1[:, 0] > 1e-9
+    assert np.array_equal(E.codes1[clear, 0], code[clear])
+    c = P2.c1.astype(np.float64)[E.codes1[:, 0]]
+    assert np.allclose(E.yhat, E.nhat[:, None] * np.stack([np.cos(c), np.sin(c)], 1), atol=1e-14)
+    P4 = O.polar_params(4, 4, with_S=False)
+    X = np.random.default_rng(2).standard_normal((200, 4))
+    E = O.encode_polar(X, P4, qjl=False)
+    Y = O.rotate(X, P4.signs)
+    psi = np.arctan2(np.hypot(Y[:, 2], Y[:, 3]), np.hypot(Y[:, 0], Y[:, 1]))
+    ref = np.searchsorted(P4.th[0].astype(np.float64), psi, side="right")
+    clear = E.marginh[:, 0] > 1e-9
+    assert np.array_equal(E.codesh[clear, 0], ref[clear])
+    ps = P4.ch[0].astype(np.float64)[E.codesh[:, 0]]
+    t1, t2 = (P4.c1.astype(np.float64)[E.codes1[:, j]] for j in (0, 1))
+    yh = E.nhat[:, None] * np.stack([np.cos(ps) * np.cos(t1), np.cos(ps) * np.sin(t1),
+                                     np.sin(ps) * np.cos(t2), np.sin(ps) * np.sin(t2)], 1)
+    assert np.allclose(E.yhat, yh, atol=1e-13)
+
+
+def test_polar_decode_encode_idempotent_and_scale_free():
+    d = 128
+    P = O.polar_params(d, 6, with_S=False)
+    X = np.random.default_rng(3).standard_normal((30, d)) * np.exp(np.random.default_rng(4).standard_normal(d))
+    E = O.encode_polar(X, P, qjl=False)
+    assert np.allclose(np.linalg.norm(E.yhat, axis=1), E.nhat, rtol=1e-13)     # only the radius is stored
+    E2 = O.encode_polar(O.rotate_t(E.yhat, P.signs), P, qjl=False)              # the decoded vector re-encodes to itself
+    assert np.array_equal(E2.codes1, E.codes1) and np.array_equal(E2.codesh, E.codesh)
+    assert np.allclose(E2.yhat, E.yhat, atol=1e-12)
+    E3 = O.encode_polar(4.0 * X, P, qjl=False)                                 # no scale besides the norm
+    assert np.array_equal(E3.codes1, E.codes1) and np.array_equal(E3.codesh, E.codesh)
+    assert np.array_equal(E3.nhat, 4.0 * E.nhat)
+    # distortion: better than the 2-bit Lloyd-Max coordinate quantizer at ~3 bits per coordinate
+    Xb = np.random.default_rng(5).standard_normal((5000, d))
+    Eb = O.encode_polar(Xb, P, qjl=False)
+    nm = np.mean(np.sum((O.rotate(Xb, P.signs) - Eb.yhat) ** 2, 1) / np.sum(Xb ** 2, 1))
+    P2 = O.make_params(d, 2, 6, with_S=False)
+    E2b = O.encode(Xb, P2, qjl=False, margins=False)
+    n2 = np.mean(np.sum((O.rotate(Xb, P2.signs) - E2b.nhat[:, None] * P2.c32.astype(np.float64)[E2b.idx]) ** 2, 1)
+                 / np.sum(Xb ** 2, 1))
+    assert nm < n2
+
+
+def test_polar_attention_textbook_and_qjl_unbiased():
+    d, L = 64, 120
+    rng = np.random.default_rng(8)
+    Pk, Pv = O.polar_params(d, 61, with_S=False), O.polar_params(d, 62, with_S=False)
+
+    def coded(P):
+        c1 = rng.integers(0, 16, (L, d // 2)).astype(np.uint8)
+        ch = rng.integers(0, 4, (L, d // 2 - 1)).astype(np.uint8)
+        nh = np.array([O.round_fp16(v) for v in rng.uniform(1.0, 9.0, L)])
+        yh = O.polar_decode(c1, ch, nh, P)
+        return O.PolarEncoded(False, c1, ch, nh, yh), O.rotate_t(yh, P.signs)
+    Ek, Kx = coded(Pk)
+    Ev, Vx = coded(Pv)
+    Q = rng.standard_normal((3, d))
+    out, lse, logits = O.attend(Q, Pk, Ek, Pv, Ev, want_logits=True)
+    lg = Q @ Kx.T / math.sqrt(d)
+    assert np.allclose(logits, lg, atol=1e-11, rtol=0)
+    assert np.allclose(out, scipy.special.softmax(lg, axis=1) @ Vx, atol=1e-11, rtol=0)
+    # QJL on the polar residual keeps inner products unbiased
+    k = rng.standard_normal(d)
+    q = rng.standard_normal(d) + 0.6 * k
+    est = np.array([O.estimate(q, P, O.encode_polar(k[None, :], P, qjl=True))[0]
+                    for P in (O.polar_params(d, 4000 + s) for s in range(3000))])
+    assert abs(est.mean() - q @ k) < 3 * est.std(ddof=1) / math.sqrt(len(est))
