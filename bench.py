@@ -42,6 +42,9 @@ import torch  # noqa: E402
 METRIC = "KV vectors encoded/s + decode-attn keys scored/s; % HBM roofline (1 B200)"
 WORKLOAD_METRICS = {"step": METRIC, "encode": "KV vectors encoded/s", "decode32k": "decode-attn keys scored/s",
                     "decode_k8v4": "decode-attn keys scored/s", "decode_step": "decode-attn keys scored/s",
+                    "dense": "KV vectors encoded/s + decode-attn keys scored/s",
+                    "frac35": "KV vectors encoded/s + decode-attn keys scored/s",
+                    "polar": "KV vectors encoded/s + decode-attn keys scored/s",
                     "longctx": "decode + prefill (query-head, key) pairs/s",
                     "search": "(query, database vector) pairs scored/s (top-10 search)"}
 UNIT_NOTES = {"step": "units = KV vectors encoded (two presets) + (query-head, key) pairs scored",
@@ -49,6 +52,9 @@ UNIT_NOTES = {"step": "units = KV vectors encoded (two presets) + (query-head, k
               "decode32k": "units = (query-head, key) pairs scored",
               "decode_k8v4": "units = (query-head, key) pairs scored",
               "decode_step": "units = (query-head, key) pairs scored (the new tokens' write included in the time)",
+              "dense": "units = KV vectors encoded + (query-head, key) pairs scored",
+              "frac35": "units = KV vectors encoded + (query-head, key) pairs scored",
+              "polar": "units = KV vectors encoded + (query-head, key) pairs scored",
               "longctx": "units = (query-head, key) pairs scored in the decode step and the prefill chunk",
               "search": "units = (query, database vector) pairs scored"}
 FALLBACK_HBM_GBS = 6650.0
@@ -381,6 +387,73 @@ class Decode32kStep(Decode32k):
                                 "batch": batch, "seq_len": seq_len}}
 
 
+class PresetPart:
+    """A write path and a GQA decode over it under an alternative codec: B=8
+    sequences x 8 KV heads x 8,192 tokens x d=128 bf16 (N(0,1), channels 5
+    and 77 x20), 32 query heads."""
+    kbits, kqjl, vbits, rotation, tag, what = 2, True, 4, 0, "", ""
+
+    def __init__(self, dev, batch=8, seq_len=8192, **_):
+        from kv_cache_vector_07_b200 import synth, tqkv
+        self.tq = tqkv
+        B, L, H, Hq, d, P = batch, seq_len, 8, 32, 128, 64
+        self.B, self.L, self.H, self.Hq, self.d, self.P = B, L, H, Hq, d, P
+        n = B * L
+        self.n = n
+        self.desc = tqkv.cache_desc(d, self.kbits, self.kqjl, self.vbits, page_tokens=P, n_kv_heads=H)
+        self.kp = tqkv.make_params(d, self.kbits, 1005, self.rotation)
+        self.vp = tqkv.make_params(d, self.vbits, 2005, self.rotation)
+        self.K = synth.outlier_normal((n, H, d), seed=51, device=dev)
+        self.V = synth.outlier_normal((n, H, d), seed=52, device=dev)
+        self.bt, self.slots, nblk = synth.contiguous_block_table(B, L, P, device=dev, shuffle_seed=53)
+        self.cache = tqkv.alloc_cache(self.desc, nblk, device=dev)
+        self.ws_e = torch.zeros(tqkv.encode_workspace_bytes(self.desc, n), dtype=torch.uint8, device=dev)
+        tqkv.encode(self.kp, self.vp, self.desc, self.K, self.V, self.slots, self.cache, workspace=self.ws_e)
+        self.Q = synth.normal((B, Hq, d), seed=54, device=dev)
+        self.seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.Q)
+        self.ws_d = torch.zeros(tqkv.decode_workspace_bytes(self.desc, B, Hq, L), dtype=torch.uint8, device=dev)
+        self.per_tok = tqkv.cache_bytes(self.desc) // P
+        torch.cuda.synchronize()
+
+    def ops(self):
+        tq = self.tq
+
+        def fe():
+            tq.encode(self.kp, self.vp, self.desc, self.K, self.V, self.slots, self.cache, workspace=self.ws_e)
+
+        def fd():
+            tq.decode_attn(self.kp, self.vp, self.desc, self.Q, self.bt, self.seq, self.L, self.cache, out=self.out,
+                           workspace=self.ws_d)
+        ex = {"bytes_per_token_and_head": self.per_tok, "codec": self.what}
+        return [Op(f"{self.tag}_encode", fe, 2 * self.n * self.H, "vectors encoded", "hbm",
+                   2 * self.n * self.H * self.d * 2 + self.n * self.H * self.per_tok,
+                   "tq_encode (general encoder: warp per vector)", 2 if self.kqjl else 1, flush=True, extra=ex),
+                Op(f"{self.tag}_decode", fd, self.B * self.Hq * self.L, "(query-head, key) pairs scored", "hbm",
+                   self.B * self.H * self.L * self.per_tok, "tq_decode_attn", 3, flush=True, extra=ex)]
+
+    @classmethod
+    def config(cls, batch=8, seq_len=8192, **_):
+        return {cls.tag: {"what": f"B={batch} x Hkv=8 x {seq_len} tokens x d=128 bf16, 32 query heads: " + cls.what,
+                          "batch": batch, "seq_len": seq_len}}
+
+
+class DenseRotation(PresetPart):
+    kbits, kqjl, vbits, rotation, tag = 2, True, 4, 1, "dense_k3v4"
+    what = "k3v4 under the dense random rotation (encode: dense 128 x 128 product per vector)"
+
+
+class Fractional35(PresetPart):
+    kbits, kqjl, vbits, rotation, tag = 16 | 2, True, 16 | 3, 0, "frac35"
+    what = "3.5-bit keys incl. QJL (2.5-bit Lloyd-Max + QJL) and 3.5-bit values (fractional rates, general kernels)"
+
+
+class PolarCodes(PresetPart):
+    kbits, kqjl, vbits, rotation, tag = 32, True, 32, 0, "polar"
+    what = ("PolarQuant angle codes (4-bit level-1 angles, 2-bit higher levels) for keys with QJL and for values "
+            "(general kernels)")
+
+
 class LongCtx:
     """Config: B=1, Hq=32 over Hkv=4, 262,144 tokens, K 2-bit + QJL, V 3-bit;
     one decode step plus one 2,048-query prefill chunk (causal inside)."""
@@ -536,11 +609,15 @@ class Search:
 
 
 # workload -> (classes in the timed step, classes timed as parts)
-WORKLOADS = {"step": ((WritePath, Decode32k), (Decode32kK8V4, Decode32kStep, LongCtx, Search)),
+WORKLOADS = {"step": ((WritePath, Decode32k), (Decode32kK8V4, Decode32kStep, LongCtx, Search, DenseRotation,
+                                                Fractional35, PolarCodes)),
              "encode": ((WritePath,), ()),
              "decode32k": ((Decode32k,), ()),
              "decode_k8v4": ((Decode32kK8V4,), ()),
              "decode_step": ((Decode32kStep,), ()),
+             "dense": ((DenseRotation,), ()),
+             "frac35": ((Fractional35,), ()),
+             "polar": ((PolarCodes,), ()),
              "longctx": ((LongCtx,), ()),
              "search": ((Search,), ())}
 WORKLOAD_NAMES = {"step": "write path (k8v4 and K4+QJL/V4, 8 x 8 x 32768 x 128 bf16) + k3v4 GQA decode "
@@ -549,6 +626,9 @@ WORKLOAD_NAMES = {"step": "write path (k8v4 and K4+QJL/V4, 8 x 8 x 32768 x 128 b
                   "decode32k": "k3v4 GQA decode 32 x 32/8 heads x 32768 x 128",
                   "decode_k8v4": "k8v4 GQA decode 32 x 32/8 heads x 32768 x 128 (FP8 keys)",
                   "decode_step": "fused k3v4 decode step (write the new token, attend) 32 x 32/8 heads x 32768",
+                  "dense": "k3v4 write path + decode under the dense rotation, 8 x 8 x 8192",
+                  "frac35": "3.5-bit fractional-rate write path + decode, 8 x 8 x 8192",
+                  "polar": "PolarQuant-coded write path + decode, 8 x 8 x 8192",
                   "longctx": "long-context 1 x 32/4 heads x 262144: decode + 2048-query prefill",
                   "search": "search 1,000,000 x 1024, 1024 queries, top-10"}
 
@@ -761,7 +841,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
         if part_cls:
-            for name in ("decode_k8v4", "longctx", "search"):
+            for name in ("decode_k8v4", "longctx", "search", "dense", "frac35", "polar"):
                 cb = cpu_baseline(name, budget_s=min(4.0, args.cpu_budget))
                 for k in [k for k in parts if k.startswith(name)]:
                     parts[k]["cpu_baseline"] = cb
@@ -828,8 +908,34 @@ def _oracle_attend_slice(kind: str, n: int, L: int | None = None):
     return time.perf_counter() - t0, G * L
 
 
+def _oracle_codec_slice(kind: str, n: int, L: int):
+    """One KV head of the alternative-codec parts on the oracle: encode L keys
+    and L values, then score them for 4 query heads.  (seconds, units)."""
+    from kv_cache_vector_07_b200 import synth
+    from oracle import oracle as O
+    d = 128
+    K = synth.outlier_normal((L, d), seed=90 + n, dtype=torch.float32).numpy().astype(np.float64)
+    V = synth.outlier_normal((L, d), seed=91 + n, dtype=torch.float32).numpy().astype(np.float64)
+    Q = synth.normal((4, d), seed=92 + n, dtype=torch.float32).numpy().astype(np.float64)
+    if kind == "dense":
+        Pk, Pv = O.make_params(d, 2, 1005, rotation="dense"), O.make_params(d, 4, 2005, False, rotation="dense")
+    elif kind == "polar":
+        Pk, Pv = O.polar_params(d, 1005), O.polar_params(d, 2005, with_S=False)
+    else:
+        Pk, Pv = O.make_params(d, 2.5, 1005), O.make_params(d, 3.5, 2005, with_S=False)
+    t0 = time.perf_counter()
+    if kind == "polar":
+        Ek, Ev = O.encode_polar(K, Pk, qjl=True), O.encode_polar(V, Pv, qjl=False)
+    else:
+        Ek, Ev = O.encode(K, Pk, qjl=True, margins=False), O.encode(V, Pv, qjl=False, margins=False)
+    O.attend(Q, Pk, Ek, Pv, Ev)
+    return time.perf_counter() - t0, 2 * L + 4 * L
+
+
 def _oracle_sample(workload: str, n: int, small: bool):
     """One bounded sample of the workload on the oracle: (seconds, units)."""
+    if workload in ("dense", "frac35", "polar"):
+        return _oracle_codec_slice(workload, n, 2048 if small else 8192)
     if workload == "encode":
         return _oracle_encode_slice(n, 4096 if small else 32768)
     if workload == "step":
@@ -852,11 +958,15 @@ SAMPLE_TEXT = {
     "decode32k": "slices of one KV head: 4 query heads over {L} k3v4 keys (encode untimed)",
     "decode_k8v4": "slices of one KV head: 4 query heads over {L} k8v4 keys (encode untimed)",
     "decode_step": "slices of one KV head: 4 query heads over {L} k3v4 keys (encode untimed)",
+    "dense": "slices of one KV head: encode {L} keys and {L} values (k3v4, dense rotation), score 4 query heads",
+    "frac35": "slices of one KV head: encode {L} keys and {L} values (3.5-bit rates), score 4 query heads",
+    "polar": "slices of one KV head: encode {L} keys and {L} values (PolarQuant codes), score 4 query heads",
     "longctx": "slices of one KV head: 8 query heads over {L} keys (K 2-bit + QJL, V 3-bit; encode untimed)",
     "search": "slices: 4 queries over {L} oracle-encoded d=1024 vectors (encode untimed)",
 }
 SAMPLE_L = {"encode": (4096, 32768), "step": (4096, 32768), "decode32k": (8192, 32768),
             "decode_k8v4": (8192, 32768), "decode_step": (8192, 32768), "longctx": (8192, 65536),
+            "dense": (2048, 8192), "frac35": (2048, 8192), "polar": (2048, 8192),
             "search": (5000, 20000)}
 
 

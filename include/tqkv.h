@@ -64,8 +64,34 @@ enum tq_status {
 #define TQ_DTYPE_BF16 0
 #define TQ_DTYPE_F32  1
 
-/* Code widths: 1..4 = Lloyd-Max bits per coordinate; 8 = FP8 E4M3 (keys). */
+/* Code widths: 1..4 = Lloyd-Max bits per coordinate; 8 = FP8 E4M3 (keys);
+ * TQ_BITS_HALF | b (b in 1..3) = the fractional rate b + 1/2: coordinates
+ * 0 .. d/2-1 of the rotated vector take b + 1 bits and coordinates
+ * d/2 .. d-1 take b bits, each half with the Lloyd-Max codebook of its width
+ * for the same coordinate law (the rotation makes every coordinate follow
+ * that law, so the split needs no calibration).  Rates 1.5, 2.5 and 3.5
+ * ("What is TurboQuant?": quality-neutral at 3.5 bits per channel, a minor
+ * loss at 2.5; community forks ship turboquant25 / turboquant35 presets);
+ * the split rule is not on the pages.  16 <= d <= 256; the general kernels
+ * serve these rates. */
 #define TQ_BITS_FP8 8
+#define TQ_BITS_HALF 16
+/* TQ_BITS_POLAR: the polar-coordinate angle quantizer of the standalone
+ * PolarQuant ("What is TurboQuant?", "Stage 1": vectors mapped to polar
+ * coordinates, the angles quantized, no per-vector scale beyond one radius;
+ * ai-work-lab overview, PolarQuant section).  After the rotation, level 1
+ * turns coordinate pairs (y_2p, y_2p+1) into radii and angles atan2 in
+ * [0, 2 pi); each level l = 2 .. log2 d turns pairs of radii (a, b) into
+ * sqrt(a^2 + b^2) and psi = atan2(b, a) in [0, pi/2]; the last radius is the
+ * stored norm.  Level-1 angles take 4 bits on 16 uniform cells (centres as
+ * levels); level-l angles take 2 bits from the Lloyd-Max quantizer of their
+ * law for a random direction, density proportional to (sin psi cos psi)^(k-1)
+ * with k = 2^(l-1).  The bit allocation (4, 2) is our reading.  Layout: the
+ * d/2 level-1 codes as 4-bit fields, then d/2 slots of 2-bit fields holding
+ * level 2's d/4 codes, level 3's d/8, ..., level log2 d's one (last slot
+ * zero): 3d/8 bytes.  Keys may add QJL on the residual y - y_hat.
+ * 8 <= d <= 256; the general kernels serve it (no vector search). */
+#define TQ_BITS_POLAR 32
 
 /* ------------------------------------------------------------------------ */
 /* Parameters                                                               */
@@ -79,7 +105,9 @@ typedef struct tq_params tq_params;   /* opaque, library-owned */
  * decision boundaries (fp32).  Page: "What is TurboQuant?", "Stage 1" and
  * "Where calibration-free pays off" (the parameters depend on nothing but
  * (d, bits, seed)).
- * d: power of two in [8, 1024]; bits in {1,2,3,4,8}.  *out receives the
+ * d: power of two in [8, 1024]; bits in {1,2,3,4,8} or TQ_BITS_HALF | b
+ * (b in 1..3, then 16 <= d <= 256; levels and bounds of the (b + 1)-bit
+ * codebook come first, then those of the b-bit one).  *out receives the
  * handle.  Returns TQ_EINVAL / TQ_EUNSUPPORTED on bad arguments, TQ_ENOMEM /
  * TQ_ECUDA on allocation or copy failure.  Synchronous. */
 int tq_make_params(int d, int bits, uint64_t seed, tq_params **out);
@@ -90,6 +118,30 @@ int tq_make_params(int d, int bits, uint64_t seed, tq_params **out);
  * output pointer may be NULL.  Returns TQ_EUNSUPPORTED for bad (d, bits). */
 int tq_compute_params_host(int d, int bits, uint64_t seed, int8_t *signs, float *S, float *levels,
                            float *bounds);
+
+/* Rotations.  TQ_ROT_HADAMARD: R = H D / sqrt(d) (tq_make_params).
+ * TQ_ROT_DENSE: the dense random rotation ("TurboQuant and RotorQuant on DGX
+ * Spark", section on compression quality: TurboQuant's 128 x 128 = 16,384
+ * rotation parameters): the d x d matrix of iid N(0,1) entries (Box-Muller of
+ * SplitMix64 draws, stream 2) with its rows orthonormalised in order (the Q
+ * of the QR factorisation of its transpose with a positive diagonal,
+ * transposed), stored in float32 (round to nearest even); under it the norm
+ * is n = ||R x|| and the inverse applied to outputs is R^T.  d <= 256.  The
+ * cache layout is the same for both. */
+#define TQ_ROT_HADAMARD 0
+#define TQ_ROT_DENSE 1
+
+/* tq_make_params with a choice of rotation (TQ_ROT_*).  TQ_EUNSUPPORTED for
+ * an unknown rotation or TQ_ROT_DENSE with d > 256. */
+int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, tq_params **out);
+
+/* The same matrix computed on the host only (no CUDA call). */
+int tq_compute_rotation_host(int d, uint64_t seed, int rotation, float *R);
+
+/* Copy the rotation matrix R (row-major d x d, y = R x) of a handle to R:
+ * H D / sqrt(d) in float32 for TQ_ROT_HADAMARD, the stored matrix for
+ * TQ_ROT_DENSE. */
+int tq_params_export_rotation(const tq_params *p, float *R);
 
 /* Release a handle (NULL is a no-op).  Synchronous. */
 void tq_free_params(tq_params *p);
@@ -112,7 +164,9 @@ int tq_params_export(const tq_params *p, int8_t *signs, float *S, float *levels,
  *   V codes   as K codes with vbits (absent if vbits = 0)
  *   V norm    fp16 ||v|| (absent if vbits = 0)
  * Code fields of one token: coordinate i at bit offset i*w of the token's
- * little-endian byte string.  A Lloyd-Max code is stored sign-magnitude:
+ * little-endian byte string.  A fractional rate stores the first half of
+ * the coordinates as a (b + 1)-bit code of d/2 coordinates, then the second
+ * half as a b-bit code of d/2 coordinates (each by the rules above).  A Lloyd-Max code is stored sign-magnitude:
  * top bit set for the negative half of the levels, low bits the rank of the
  * level's magnitude (0 = smallest).  QJL bit j is 1 iff (S r)_j >= 0.
  * The cache is an array [num_blocks][n_kv_heads] of pages; token slot s lives
@@ -121,9 +175,9 @@ int tq_params_export(const tq_params *p, int8_t *signs, float *S, float *levels,
  * (no per-block scales); the byte layout itself is not on the pages. */
 typedef struct {
     int d;            /* head dim, power of two in [8, 1024]              */
-    int kbits;        /* 1..4 Lloyd-Max, or 8 = FP8 E4M3                   */
-    int kqjl;         /* 1: QJL sign bits + residual norm (kbits 1..4)     */
-    int vbits;        /* 1..4, or 0 = no value fields (vector search)      */
+    int kbits;        /* 1..4 Lloyd-Max, 8 = FP8 E4M3, or TQ_BITS_HALF|b   */
+    int kqjl;         /* 1: QJL sign bits + residual norm (not FP8 keys)   */
+    int vbits;        /* 1..4, TQ_BITS_HALF|b, or 0 = no value fields      */
     int page_tokens;  /* multiple of 8, 8..256                             */
     int n_kv_heads;   /* >= 1                                              */
 } tq_cache_desc;

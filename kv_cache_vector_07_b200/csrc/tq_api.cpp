@@ -12,10 +12,17 @@ bool valid_desc(const tq_cache_desc *c) {
     if (!c) return false;
     const int d = c->d;
     if (d < 8 || d > 1024 || (d & (d - 1))) return false;
-    if (!(c->kbits == 1 || c->kbits == 2 || c->kbits == 3 || c->kbits == 4 || c->kbits == 8)) return false;
+    auto half_ok = [&](int b) { return (b & ~TQ_BITS_HALF) >= 1 && (b & ~TQ_BITS_HALF) <= 3 && d >= 16 && d <= 256; };
+    const bool kh = (c->kbits & TQ_BITS_HALF) != 0, vh = (c->vbits & TQ_BITS_HALF) != 0;
+    const bool polar_ok = d >= 8 && d <= 256;
+    if (c->kbits == TQ_BITS_POLAR ? !polar_ok
+        : (kh ? !half_ok(c->kbits) : !(c->kbits == 1 || c->kbits == 2 || c->kbits == 3 || c->kbits == 4 ||
+                                       c->kbits == 8)))
+        return false;
     if (c->kqjl != 0 && c->kqjl != 1) return false;
     if (c->kbits == 8 && c->kqjl) return false;
-    if (c->vbits < 0 || c->vbits > 4) return false;
+    if (c->vbits == TQ_BITS_POLAR ? !polar_ok : (vh ? !half_ok(c->vbits) : (c->vbits < 0 || c->vbits > 4)))
+        return false;
     if (c->page_tokens < 8 || c->page_tokens > 256 || (c->page_tokens % 8)) return false;
     if (c->n_kv_heads < 1) return false;
     return true;
@@ -215,7 +222,7 @@ extern "C" int tq_score(const tq_params *p, const tq_cache_desc *desc, const voi
                         size_t workspace_bytes, void *stream) {
     if (!valid_desc(desc) || !p) return TQ_EINVAL;
     if (desc->n_kv_heads != 1 || desc->vbits != 0) return TQ_EINVAL;
-    if (desc->kbits == 8) return TQ_EUNSUPPORTED;
+    if (desc->kbits == 8 || desc->kbits == TQ_BITS_POLAR) return TQ_EUNSUPPORTED;
     if (p->d != desc->d || p->bits != desc->kbits) return TQ_EINVAL;
     if (n_db < 1 || n_q < 0 || k < 1 || k > 64 || k > n_db) return TQ_EINVAL;
     if (n_q == 0) return TQ_OK;

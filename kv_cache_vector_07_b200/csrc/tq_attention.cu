@@ -36,20 +36,17 @@ struct PrepArgs {
 template <int D>
 __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
     constexpr int E = WarpVec<D>::E;
+    __shared__ float wbuf[4][D <= 256 ? D : 4];          // dense rotation only (d <= 256)
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int64_t row = int64_t(blockIdx.x) * 4 + wl;
     if (row >= a.rows) return;
-    float x[E], sg[E];
+    float x[E];
     if (a.in_f32) load_vec<D>(reinterpret_cast<const float *>(a.Q) + row * D, lane, x);
     else load_vec<D>(reinterpret_cast<const __nv_bfloat16 *>(a.Q) + row * D, lane, x);
-    load_vec<D>(a.kp.signs, lane, sg);
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] *= sg[e];
-    fwht_warp<D>(x, lane);
-    const float rs = 1.0f / sqrtf(float(D));
+    rotate_warp<D>(a.kp, x, wbuf[wl], lane);
     if (lane < WarpVec<D>::LANES) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) a.qr[row * D + lane * E + e] = x[e] * rs;
+        for (int e = 0; e < E; ++e) a.qr[row * D + lane * E + e] = x[e];
     }
 }
 
@@ -154,7 +151,7 @@ __device__ __forceinline__ void project_rows(const uint16_t *S, const float *vs,
 template <int D>
 __global__ void __launch_bounds__(256) step_prep_kernel(StepArgs a) {
     constexpr int E = WarpVec<D>::E;
-    __shared__ float svec[8][D > 8 ? D : 8];
+    __shared__ float svec[8][warp_buf_floats<D>()];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const Layout &L = a.L;
     const int64_t n_enc = int64_t(a.B) * L.H * 2;
@@ -174,7 +171,7 @@ __global__ void __launch_bounds__(256) step_prep_kernel(StepArgs a) {
         load_vec<D>((is_v ? a.V : a.K) + v * D, lane, x);
         uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
         const int pos = slot % L.P;
-        if (!encode_vector_warp<D>(L, is_v ? a.vp : a.kp, is_v, x, page, pos, lane, r)) return;
+        if (!encode_vector_warp<D>(L, is_v ? a.vp : a.kp, is_v, x, page, pos, lane, r, vs)) return;
         if (lane < WarpVec<D>::LANES) {
 #pragma unroll
             for (int e = 0; e < E; ++e) vs[lane * E + e] = r[e];
@@ -190,17 +187,12 @@ __global__ void __launch_bounds__(256) step_prep_kernel(StepArgs a) {
     }
     const int64_t row = job - n_enc;
     if (row >= a.prep.rows) return;
-    float x[E], sg[E];
+    float x[E];
     load_vec<D>(reinterpret_cast<const __nv_bfloat16 *>(a.prep.Q) + row * D, lane, x);
-    load_vec<D>(a.kp.signs, lane, sg);
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] *= sg[e];
-    fwht_warp<D>(x, lane);
-    const float rs = 1.0f / sqrtf(float(D));
+    rotate_warp<D>(a.kp, x, vs, lane);
     if (lane < WarpVec<D>::LANES) {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            x[e] *= rs;
             a.prep.qr[row * D + lane * E + e] = x[e];
             vs[lane * E + e] = x[e];
         }
@@ -245,7 +237,8 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
     __shared__ float lg[kMaxG][kChunk];
     __shared__ float vn[kChunk];
     __shared__ const uint8_t *pg[kChunk];
-    __shared__ float lvk[16], lvv[16];
+    __shared__ float lvk[16], lvv[16], lvk2[8], lvv2[8];
+    __shared__ float ptk[132], ptv[132];                  // polar tables of keys / values
     __shared__ float s_m[kMaxG], s_l[kMaxG], s_alpha[kMaxG];
 
     const Layout &L = a.L;
@@ -265,8 +258,17 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
         sw[c][h] = a.w[(row0 + h) * D + c];
     }
     if (tid < 16) {
-        lvk[tid] = (L.kbits <= 4 && tid < (1 << L.kbits)) ? a.kp.lv[tid] : 0.f;
-        lvv[tid] = tid < (1 << L.vbits) ? a.vp.lv[tid] : 0.f;
+        // first (or only) codebook of each; fractional rates add a second
+        lvk[tid] = (L.ka_bits <= 4 && tid < (1 << L.ka_bits)) ? a.kp.lv[tid] : 0.f;
+        lvv[tid] = tid < (1 << L.va_bits) ? a.vp.lv[tid] : 0.f;
+        if (tid < 8) {
+            lvk2[tid] = (L.khalf && tid < (1 << L.kb_bits)) ? a.kp.lv2[tid] : 0.f;
+            lvv2[tid] = (L.vhalf && tid < (1 << L.vb_bits)) ? a.vp.lv2[tid] : 0.f;
+        }
+    }
+    for (int i = tid; i < 132; i += kChunk) {
+        ptk[i] = L.kpolar ? a.kp.polar[i] : 0.f;
+        ptv[i] = L.vpolar ? a.vp.polar[i] : 0.f;
     }
     if (tid < kMaxG) { s_m[tid] = -INFINITY; s_l[tid] = 0.f; }
     float acc[kMaxG][CPT];
@@ -295,19 +297,40 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
         if (page) {
             const int pos = t % L.P;
             const uint8_t *kc = page + L.kc_off + pos * L.kc_bpt;
-            const uint8_t *kh = L.kbits == 3 ? page + L.kh_off + pos * L.kh_bpt : nullptr;
+            const uint8_t *kh = L.ka_bits == 3 ? page + L.kh_off + pos * L.kh_bpt : nullptr;
+            // fractional rates: coordinates nA .. D-1 in the second code arrays
+            const int nA = L.khalf ? D / 2 : D;
+            const uint8_t *kc2 = L.khalf ? page + L.kc2_off + pos * L.kc2_bpt : nullptr;
+            const uint8_t *kh2 = (L.khalf && L.kb_bits == 3) ? page + L.kh2_off + pos * L.kh2_bpt : nullptr;
             const uint8_t *ks = L.kqjl ? page + L.ks_off + pos * L.ks_bpt : nullptr;
             float mse[kMaxG], qj[kMaxG];
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) { mse[h] = 0.f; qj[h] = 0.f; }
-            for (int i = 0; i < D; ++i) {
+            // polar keys: pairs of the unit-radius reconstruction (the norm is applied below)
+            for (int p = 0; L.kpolar && p < D / 2; ++p) {
+                const float2 yv = polar_pair<D>(kc, page + L.kc2_off + pos * L.kc2_bpt, ptk, p);
+                const bool s0 = ks ? (read_field(ks, 2 * p, 1) != 0) : true;
+                const bool s1 = ks ? (read_field(ks, 2 * p + 1, 1) != 0) : true;
+#pragma unroll
+                for (int h = 0; h < kMaxG; ++h) {
+                    if (h < G) {
+                        mse[h] = fmaf(sq[2 * p][h], yv.x, fmaf(sq[2 * p + 1][h], yv.y, mse[h]));
+                        qj[h] += (s0 ? sw[2 * p][h] : -sw[2 * p][h]) + (s1 ? sw[2 * p + 1][h] : -sw[2 * p + 1][h]);
+                    }
+                }
+            }
+            for (int i = 0; !L.kpolar && i < D; ++i) {
                 float cv;
                 if (kw == 8) {
                     cv = e4m3_to_float(kc[i]);          // FP8 key: e4m3(sqrt(d) u_i)
-                } else {
+                } else if (i < nA) {
                     uint32_t kap = read_field(kc, i, kw);
                     if (kh) kap |= read_field(kh, i, 1) << 2;
                     cv = lvk[kap];
+                } else {
+                    uint32_t kap = read_field(kc2, i - nA, L.kc2_w);
+                    if (kh2) kap |= read_field(kh2, i - nA, 1) << 2;
+                    cv = lvk2[kap];
                 }
                 const bool pos_sign = ks ? (read_field(ks, i, 1) != 0) : true;
 #pragma unroll
@@ -380,15 +403,28 @@ __global__ void __launch_bounds__(kChunk) attn_kernel(AttnArgs a) {
             if (!page) continue;
             const int pos = (c0 + j) % L.P;
             const uint8_t *vc = page + L.vc_off + pos * L.vc_bpt;
-            const uint8_t *vh = L.vbits == 3 ? page + L.vh_off + pos * L.vh_bpt : nullptr;
+            const uint8_t *vh = L.va_bits == 3 ? page + L.vh_off + pos * L.vh_bpt : nullptr;
+            const int vA = L.vhalf ? D / 2 : D;
             const float nvv = vn[j];
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {
                 const int i = tid + c * kChunk;
                 if (i < D) {
-                    uint32_t kap = read_field(vc, i, L.vc_w);
-                    if (vh) kap |= read_field(vh, i, 1) << 2;
-                    const float val = lvv[kap] * nvv;
+                    float lvl;
+                    if (L.vpolar) {
+                        const float2 yv = polar_pair<D>(vc, page + L.vc2_off + pos * L.vc2_bpt, ptv, i >> 1);
+                        lvl = (i & 1) ? yv.y : yv.x;
+                    } else if (i < vA) {
+                        uint32_t kap = read_field(vc, i, L.vc_w);
+                        if (vh) kap |= read_field(vh, i, 1) << 2;
+                        lvl = lvv[kap];
+                    } else {
+                        const int i2 = i - vA;
+                        uint32_t kap = read_field(page + L.vc2_off + pos * L.vc2_bpt, i2, L.vc2_w);
+                        if (L.vb_bits == 3) kap |= read_field(page + L.vh2_off + pos * L.vh2_bpt, i2, 1) << 2;
+                        lvl = lvv2[kap];
+                    }
+                    const float val = lvl * nvv;
 #pragma unroll
                     for (int h = 0; h < kMaxG; ++h)
                         if (h < G) acc[h][c] = fmaf(lg[h][j], val, acc[h][c]);
@@ -430,6 +466,7 @@ struct CombineArgs {
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     constexpr int E = WarpVec<D>::E;
+    __shared__ float wbuf[4][D <= 256 ? D : 4];          // dense rotation only (d <= 256)
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (r >= int64_t(a.n_groups) * a.G) return;
@@ -467,16 +504,31 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] *= inv;
-    fwht_warp<D>(o, lane);
-    float sg[E];
-    load_vec<D>(a.vp.signs, lane, sg);
-    const float rs = 1.0f / sqrtf(float(D));
     const int b = g / a.H, kvh = g - b * a.H;
     const int64_t orow = int64_t(b) * a.Hq + int64_t(kvh) * a.G + h;
     __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + orow * D;
-    if (lane < WarpVec<D>::LANES) {
+    if (a.vp.rot) {
+        // o = R^T o_r with the dense rotation: rows of its transpose
+        float *vs = wbuf[(threadIdx.x >> 5) & 3];
+        if (lane < WarpVec<D>::LANES) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) out[lane * E + e] = __float2bfloat16_rn(o[e] * rs * sg[e]);
+            for (int e = 0; e < E; ++e) vs[lane * E + e] = o[e];
+        }
+        __syncwarp();
+        dense_rows<D>(a.vp.RdT, vs, lane, o);
+        if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) out[lane * E + e] = __float2bfloat16_rn(o[e]);
+        }
+    } else {
+        fwht_warp<D>(o, lane);
+        float sg[E];
+        load_vec<D>(a.vp.signs, lane, sg);
+        const float rs = 1.0f / sqrtf(float(D));
+        if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) out[lane * E + e] = __float2bfloat16_rn(o[e] * rs * sg[e]);
+        }
     }
     if (a.lse && lane == 0) a.lse[orow] = Lsum > 0.f ? M + logf(Lsum) : -INFINITY;
 }
@@ -564,7 +616,7 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
         sa.status = reinterpret_cast<uint32_t *>(ws);
         const int64_t jobs = int64_t(s.n_seq) * L.H * 2 + rows;
         step_prep_kernel<D><<<unsigned((jobs + 7) / 8), 256, 0, st>>>(sa);
-    } else if (D == 128 && L.kqjl) {
+    } else if (D == 128 && L.kqjl && !kp->dev.rot) {
         cudaError_t e = cudaFuncSetAttribute(prep_proj128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(kPQSmem));
         if (e != cudaSuccess) return e;

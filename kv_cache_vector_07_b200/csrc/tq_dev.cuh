@@ -181,6 +181,56 @@ __device__ __forceinline__ float h2f_bits(uint16_t b) {
     return __half2float(h);
 }
 
+// z = M v for a dense fp32 matrix M [D][D] (row-major) and a vector v held
+// in shared memory, lane l producing outputs [l E, l E + E) (the warp
+// mapping of WarpVec); fp32 products in index order.
+template <int D>
+__device__ __forceinline__ void dense_rows(const float *M, const float *vs, int lane, float (&z)[WarpVec<D>::E]) {
+    constexpr int E = WarpVec<D>::E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) z[e] = 0.f;
+    if (lane >= WarpVec<D>::LANES) return;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float4 *row = reinterpret_cast<const float4 *>(M + size_t(lane * E + e) * D);
+        float acc = 0.f;
+        for (int i = 0; i < D / 4; ++i) {
+            const float4 m = row[i];
+            acc = fmaf(m.x, vs[4 * i], acc);
+            acc = fmaf(m.y, vs[4 * i + 1], acc);
+            acc = fmaf(m.z, vs[4 * i + 2], acc);
+            acc = fmaf(m.w, vs[4 * i + 3], acc);
+        }
+        z[e] = acc;
+    }
+}
+
+// y = R x for the warp-held vector x (lane mapping of WarpVec): the dense
+// rotation through the shared buffer wbuf (D floats of this warp), else
+// H D / sqrt(D) by sign flip and butterflies.
+template <int D>
+__device__ __forceinline__ void rotate_warp(const DevParams &P, float (&x)[WarpVec<D>::E], float *wbuf, int lane) {
+    constexpr int E = WarpVec<D>::E;
+    if (P.rot) {
+        if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) wbuf[lane * E + e] = x[e];
+        }
+        __syncwarp();
+        dense_rows<D>(P.Rd, wbuf, lane, x);
+        __syncwarp();
+        return;
+    }
+    float sg[E];
+    load_vec<D>(P.signs, lane, sg);
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] *= sg[e];
+    fwht_warp<D>(x, lane);
+    const float rs = 1.0f / sqrtf(float(D));
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] *= rs;
+}
+
 // Value of an OCP E4M3 byte (CUDA's fp8 conversion; exact in fp16).
 __device__ __forceinline__ float e4m3_to_float(uint8_t b) {
     const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
@@ -198,6 +248,29 @@ __device__ __forceinline__ uint32_t e4m3x2_to_half2_bits(uint32_t two_bytes) {
 __device__ __forceinline__ uint32_t read_field(const uint8_t *arr, int i, int W) {
     const int bit = i * W;
     return (uint32_t(arr[bit >> 3]) >> (bit & 7)) & ((1u << W) - 1u);
+}
+
+// Coordinates (2p, 2p + 1) of the unit-radius reconstruction of a polar
+// code: the cos / sin factors of the centre angles on the path from the top
+// level down to pair p, then the level-1 angle.  c1: the token's 4-bit
+// level-1 codes; ch: its 2-bit higher-level slots (level 2 first); tab: the
+// polar table (bounds, cos, sin per level; see DevParams::polar).
+template <int D>
+__device__ __forceinline__ float2 polar_pair(const uint8_t *c1, const uint8_t *ch, const float *tab, int p) {
+    constexpr int H = D / 2;
+    int level = 0;
+    while ((1 << level) < D) ++level;
+    float r = 1.f;
+    int slot = H - 1;
+#pragma unroll 1
+    for (int nodes = 1; nodes < H; nodes <<= 1, --level) {
+        slot -= nodes;
+        const uint32_t k = read_field(ch, slot + (p >> (level - 1)), 2);
+        const float *tl = tab + 48 + 12 * (level - 2);
+        r *= ((p >> (level - 2)) & 1) ? tl[8 + k] : tl[4 + k];
+    }
+    const uint32_t k1 = read_field(c1, p, 4);
+    return make_float2(r * tab[16 + k1], r * tab[32 + k1]);
 }
 
 }  // namespace tq

@@ -12,10 +12,10 @@
 // page, fp16 norm; for QJL keys also the residual r = y - nhat c[idx] (kept
 // in fp32 scratch) and its fp16 norm rho.
 // Kernel 2 (qjl_gemm_kernel): z = S r on the tensor cores (tcgen05.mma,
-// accumulator in TMEM).  r is split into three bf16 terms (hi + mid + lo,
-// together the full fp32 mantissa) against the bf16-exact S, so the sign of
-// every z_j is that of the fp32-accurate product; the epilogue packs sign
-// bits straight into the page.
+// accumulator in TMEM).  r (kept scaled by a power of two per vector) is
+// split into fp16 hi + lo against the fp16 copy of S, 22 bits of r, so every
+// z_j whose sign could differ from the exact product's lies within 2^-22
+// ||r|| ||S_j|| of zero; the epilogue packs sign bits straight into the page.
 #include <cuda_runtime.h>
 #include <cuda_fp8.h>
 
@@ -42,6 +42,7 @@ struct EncodeArgs {
 template <int D, typename TIn>
 __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     constexpr int E = WarpVec<D>::E;
+    __shared__ float wbuf[8][warp_buf_floats<D>()];
     const int lane = threadIdx.x & 31;
     const Layout &L = a.L;
     const int64_t nvec = a.n_tokens * L.H;
@@ -64,10 +65,24 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         load_vec<D>(reinterpret_cast<const TIn *>(is_v ? a.V : a.K) + v * D, lane, x);
         uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
         const int pos = slot % L.P;
-        if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r) && lane < WarpVec<D>::LANES) {
-            float *dst = a.resid + v * D + lane * E;
+        if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r, wbuf[threadIdx.x >> 5])) {
+            // the residual is stored times 2^e with ||r|| 2^e in [2^10, 2^11): the
+            // projection's fp16 hi + lo parts then stay normal, and its signs do
+            // not depend on a positive scale
+            float rr = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) dst[e] = r[e];
+            for (int e = 0; e < E; ++e) rr = fmaf(r[e], r[e], rr);
+            rr = warp_sum(rr);
+            float sc = 1.f;
+            if (rr > 0.f) {
+                const int ex = ((__float_as_int(sqrtf(rr)) >> 23) & 0xff) - 127;
+                sc = __int_as_float(min(254, max(1, 127 + 10 - ex)) << 23);
+            }
+            if (lane < WarpVec<D>::LANES) {
+                float *dst = a.resid + v * D + lane * E;
+#pragma unroll
+                for (int e = 0; e < E; ++e) dst[e] = r[e] * sc;
+            }
         }
     }
 }
@@ -77,8 +92,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 // ---------------------------------------------------------------------------
 struct QjlArgs {
     Layout L;
-    const uint16_t *S;      // [m][D] bf16 bits, m = D
-    const float *resid;     // [nK][D]
+    const uint16_t *S16;    // [m][D] fp16 bits, m = D
+    const float *resid;     // [nK][D], each row scaled by a power of two
     int64_t nK;             // n_tokens * H
     const int32_t *slots;
     int64_t num_slots;
@@ -90,22 +105,23 @@ constexpr int kBM = 128;       // vectors per tile (MMA M)
 constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
 constexpr uint32_t kMaxPolls = 1u << 20;   // about a second of polling, then give up
 
-__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
-    __nv_bfloat16 b = __float2bfloat16_rn(x);
-    return *reinterpret_cast<uint16_t *>(&b);
-}
-__device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
-    return __uint_as_float(uint32_t(b) << 16);
-}
-
+// z = S r for a tile of 128 residuals against BN projection rows, on the
+// tensor cores.  r (fp32, scaled per row by a power of two) is split into
+// fp16 hi + lo (22 bits; the scale keeps both parts normal) against the
+// fp16 copy of S (exact for |S| >= 2^-14); two MMAs per k-step and per 256
+// output columns, fp32 accumulators in TMEM (BN = 512 fills all of it).  The
+// epilogue packs the sign bits [z_j >= 0] into the page.  The grid runs the
+// N tiles of one residual tile next to each other, so the tile's rows are
+// read from DRAM once and served to the others from L2.
 template <int D, int BN>
 __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
     constexpr int M = D;                                   // projection rows
     constexpr int NK = (D + kBK - 1) / kBK;
+    constexpr int NI = BN < 256 ? BN : 256;                // N of one MMA
     constexpr uint32_t TCOLS = BN < 32 ? 32 : BN;
     constexpr int A_BYTES = kBM * 128;                     // one split tile
     constexpr int B_BYTES = BN * 128;
-    constexpr int STAGE_BYTES = 3 * A_BYTES + B_BYTES;
+    constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar[2];
@@ -114,8 +130,8 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t row0 = int64_t(blockIdx.x) * kBM;
-    const int n0 = blockIdx.y * BN;
+    const int n0 = blockIdx.x * BN;
+    const int64_t row0 = int64_t(blockIdx.y) * kBM;
 
     if (warp == 0) {
         tc05::tmem_alloc(&tmem_holder, TCOLS);
@@ -131,16 +147,16 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
     __syncthreads();
     tc05::fence_after_sync();
     const uint32_t tmem = tmem_holder;
-    constexpr uint32_t idesc = tc05::idesc_bf16_f32(kBM, BN < 16 ? 16 : BN);
+    constexpr uint32_t idesc = tc05::idesc_f16_f32(kBM, NI < 16 ? 16 : NI);
 
     for (int kc = 0; kc < NK; ++kc) {
         const int st = kc & 1;
         uint8_t *sA = smem + st * STAGE_BYTES;
-        uint8_t *sB = sA + 3 * A_BYTES;
+        uint8_t *sB = sA + 2 * A_BYTES;
         if (kc >= 2) {
             if (!tc05::mbar_wait_bounded(&bar[st], ((kc - 2) >> 1) & 1, kMaxPolls)) timed_out = 1;
         }
-        // A: row tid of this tile, columns [kc*64, kc*64+64) of r, split in 3
+        // A: row tid of this tile, columns [kc*64, kc*64+64) of r as fp16 hi + lo
         {
             const int64_t g = row0 + tid;
             float rv[kBK];
@@ -158,40 +174,32 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
             }
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                uint32_t hi[4], mid[4], lo[4];
+                uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    uint16_t h2[2], m2[2], l2[2];
-#pragma unroll
-                    for (int z = 0; z < 2; ++z) {
-                        const float x = rv[ch * 8 + 2 * k + z];
-                        h2[z] = bf16_bits_rn(x);
-                        const float r1 = x - bf16_bits_to_f(h2[z]);
-                        m2[z] = bf16_bits_rn(r1);
-                        const float r2 = r1 - bf16_bits_to_f(m2[z]);
-                        l2[z] = bf16_bits_rn(r2);
-                    }
-                    hi[k] = uint32_t(h2[0]) | (uint32_t(h2[1]) << 16);
-                    mid[k] = uint32_t(m2[0]) | (uint32_t(m2[1]) << 16);
-                    lo[k] = uint32_t(l2[0]) | (uint32_t(l2[1]) << 16);
+                    const float x0 = rv[ch * 8 + 2 * k], x1 = rv[ch * 8 + 2 * k + 1];
+                    const __half2 h = __floats2half2_rn(x0, x1);
+                    const float2 hf = __half22float2(h);
+                    const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+                    hi[k] = *reinterpret_cast<const uint32_t *>(&h);
+                    lo[k] = *reinterpret_cast<const uint32_t *>(&l);
                 }
                 const uint32_t o = tc05::sw128_offset(tid, ch);
                 *reinterpret_cast<uint4 *>(sA + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sA + A_BYTES + o) = make_uint4(mid[0], mid[1], mid[2], mid[3]);
-                *reinterpret_cast<uint4 *>(sA + 2 * A_BYTES + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                *reinterpret_cast<uint4 *>(sA + A_BYTES + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
         }
-        // B: BN rows of S, same 64 columns
+        // B: BN rows of S (fp16), same 64 columns
         for (int q = tid; q < BN * 8; q += 128) {
             const int row = q >> 3, ch = q & 7;
             const int j = n0 + row, c = kc * kBK + ch * 8;
             uint4 val = make_uint4(0, 0, 0, 0);
             if (j < M && c + 8 <= D) {
-                val = *reinterpret_cast<const uint4 *>(a.S + size_t(j) * D + c);
+                val = *reinterpret_cast<const uint4 *>(a.S16 + size_t(j) * D + c);
             } else if (j < M && c < D) {
                 uint16_t tmp[8];
 #pragma unroll
-                for (int z = 0; z < 8; ++z) tmp[z] = (c + z < D) ? a.S[size_t(j) * D + c + z] : 0;
+                for (int z = 0; z < 8; ++z) tmp[z] = (c + z < D) ? a.S16[size_t(j) * D + c + z] : 0;
                 val = make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
                                  tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
             }
@@ -204,11 +212,15 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
             const uint32_t aBase = tc05::smem_u32(sA), bBase = tc05::smem_u32(sB);
 #pragma unroll
             for (int ks = 0; ks < kBK / 16; ++ks) {
-                const uint64_t bdesc = tc05::desc_kmajor_sw128(bBase + ks * 32);
 #pragma unroll
-                for (int sp = 0; sp < 3; ++sp) {
-                    const uint64_t adesc = tc05::desc_kmajor_sw128(aBase + sp * A_BYTES + ks * 32);
-                    tc05::mma_bf16(tmem, adesc, bdesc, idesc, (kc | ks | sp) != 0);
+                for (int nb = 0; nb < BN / NI; ++nb) {
+                    // rows nb*NI .. of the B tile: 8-row groups are 1024 bytes apart
+                    const uint64_t bdesc = tc05::desc_kmajor_sw128(bBase + nb * NI * 128 + ks * 32);
+#pragma unroll
+                    for (int sp = 0; sp < 2; ++sp) {
+                        const uint64_t adesc = tc05::desc_kmajor_sw128(aBase + sp * A_BYTES + ks * 32);
+                        tc05::mma_f16(tmem + uint32_t(nb * NI), adesc, bdesc, idesc, (kc | ks | sp) != 0);
+                    }
                 }
             }
             tc05::mma_commit(&bar[st]);
@@ -256,16 +268,16 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
 }
 
 template <int D>
-constexpr int qjl_bn() { return D >= 256 ? 256 : (D < 16 ? 16 : D); }
+constexpr int qjl_bn() { return D >= 512 ? 512 : (D < 16 ? 16 : D); }
 
 template <int D>
 int launch_qjl(const QjlArgs &q, cudaStream_t st) {
     constexpr int BN = qjl_bn<D>();
-    constexpr size_t smem = 2 * (3 * kBM * 128 + BN * 128) + 1024;
+    constexpr size_t smem = 2 * (2 * kBM * 128 + BN * 128) + 1024;
     auto kern = qjl_gemm_kernel<D, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    dim3 grid(unsigned((q.nK + kBM - 1) / kBM), unsigned((D + BN - 1) / BN));
+    dim3 grid(unsigned((D + BN - 1) / BN), unsigned((q.nK + kBM - 1) / kBM));
     kern<<<grid, 128, smem, st>>>(q);
     return cudaGetLastError();
 }
@@ -287,7 +299,7 @@ int launch_encode_d(const EncodeArgs &a, int in_dtype, const tq_params *kp, cuda
     if (a.L.kqjl && a.n_tokens > 0) {
         QjlArgs q;
         q.L = a.L;
-        q.S = kp->dev.S;
+        q.S16 = kp->dev.S16;
         q.resid = a.resid;
         q.nK = a.n_tokens * a.L.H;
         q.slots = a.slots;

@@ -553,7 +553,7 @@ bool make_rank_table(const tq_params *p, RankTable *t) {
 int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, const void *K, const void *V,
                      int64_t n_tokens, const int32_t *slots, uint8_t *cache, int64_t num_blocks, uint8_t *ws,
                      void *stream) {
-    if (L.d != 128 || !kp->dev.rot_img) return -1;
+    if (L.d != 128 || !kp->dev.rot_img || L.khalf || L.vhalf) return -1;
     if (L.vbits > 0 && (!vp || !vp->dev.rot_img)) return -1;
     const int kb = L.kbits, vb = L.vbits, q = L.kqjl;
     Enc128Args a;

@@ -13,31 +13,180 @@
 
 namespace tq {
 
+// Shared-memory floats the per-vector encoder needs per warp: the dense
+// rotation's staging (D), the polar transform (3 D) and two codebook copies
+// (64 floats at codebook_offset) for d <= 256; the codebooks alone above.
+template <int D>
+__host__ __device__ constexpr int warp_buf_floats() { return D <= 256 ? (3 * D > 2 * D + 64 ? 3 * D : 2 * D + 64) : 64; }
+template <int D>
+__host__ __device__ constexpr int codebook_offset() { return D <= 256 ? 2 * D : 0; }
+
+// Store a fractional-rate code (coordinates 0 .. D/2-1 at wa bits, the rest
+// at wb = wa - 1) of one token: the lanes' sign-magnitude codes are staged in
+// shared memory (cb, D bytes of this warp), then each lane assembles whole
+// bytes of the packed arrays (coordinate i at bit i * w; a 3-bit code as a
+// 2-bit array and a 1-bit array).
+template <int D>
+__device__ __forceinline__ void store_half_codes(uint8_t *page, int pos, int lane, const uint32_t (&kap)[WarpVec<D>::E],
+                                                 uint8_t *cb, int wa, int c_off, int c_bpt, int h_off, int h_bpt,
+                                                 int c2_off, int c2_bpt, int h2_off, int h2_bpt) {
+    constexpr int E = WarpVec<D>::E;
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) cb[lane * E + e] = uint8_t(kap[e]);
+    }
+    __syncwarp();
+    constexpr int n = D / 2;
+    for (int seg = 0; seg < 2; ++seg) {
+        const int w = seg ? wa - 1 : wa, base = seg * n;
+        const int mw = w == 3 ? 2 : w, per = 8 / mw;
+        uint8_t *dst = page + (seg ? c2_off + pos * c2_bpt : c_off + pos * c_bpt);
+        for (int j = lane; j < n * mw / 8; j += 32) {
+            uint32_t byte = 0;
+            for (int k = 0; k < per; ++k) byte |= (uint32_t(cb[base + j * per + k]) & ((1u << mw) - 1u)) << (k * mw);
+            dst[j] = uint8_t(byte);
+        }
+        if (w == 3) {
+            uint8_t *hd = page + (seg ? h2_off + pos * h2_bpt : h_off + pos * h_bpt);
+            for (int j = lane; j < n / 8; j += 32) {
+                uint32_t byte = 0;
+                for (int k = 0; k < 8; ++k) byte |= ((uint32_t(cb[base + 8 * j + k]) >> 2) & 1u) << k;
+                hd[j] = uint8_t(byte);
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// Polar codes of the warp-held rotated vector y (lane l holds coordinates
+// [l E, l E + E)), n = its norm and nh = fp16(n): the transform level by
+// level through shared memory (wbuf: 3 D floats of this warp: y, two radius
+// buffers, code bytes), angle codes by the bounds of P.polar, the packed
+// arrays, the fp16 norm; then y_hat top down from the centres' cos / sin and
+// r = y - y_hat into r.  Angles from atan2f; an angle within ~1e-7 (relative
+// to the radius it splits) of a bound may take either neighbour.
+template <int D>
+__device__ __forceinline__ bool polar_encode_warp(const Layout &L, const DevParams &P, bool is_v,
+                                                  const float (&y)[WarpVec<D>::E], float n, uint16_t nh,
+                                                  uint8_t *page, int pos, int lane, float (&r)[WarpVec<D>::E],
+                                                  float *wbuf) {
+    constexpr int E = WarpVec<D>::E;
+    constexpr int H = D / 2;
+    (void)n;
+    float *ys = wbuf, *ra = wbuf + D, *rb = wbuf + D + H;
+    uint8_t *cb = reinterpret_cast<uint8_t *>(wbuf + 2 * D);   // [H] level-1 codes, then [H] higher-level slots
+    const float *tab = P.polar;
+    if (lane < WarpVec<D>::LANES) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) ys[lane * E + e] = y[e];
+    }
+    __syncwarp();
+    const float two_pi = 6.283185307179586f;
+    for (int p = lane; p < H; p += 32) {
+        const float a = ys[2 * p], b = ys[2 * p + 1];
+        float t = atan2f(b, a);
+        if (t < 0.f) t += two_pi;
+        uint32_t k = 0;
+        for (int j = 0; j < 15; ++j) k += tab[j] <= t ? 1u : 0u;
+        cb[p] = uint8_t(k);
+        ra[p] = sqrtf(a * a + b * b);
+    }
+    __syncwarp();
+    float *src = ra, *dst = rb;
+    int slot = 0;
+    for (int l = 2, nodes = H / 2; nodes >= 1; ++l, nodes >>= 1) {
+        const float *tl = tab + 48 + 12 * (l - 2);
+        for (int i = lane; i < nodes; i += 32) {
+            const float a = src[2 * i], b = src[2 * i + 1];
+            const float psi = atan2f(b, a);
+            uint32_t k = 0;
+            for (int j = 0; j < 3; ++j) k += tl[j] <= psi ? 1u : 0u;
+            cb[H + slot + i] = uint8_t(k);
+            dst[i] = sqrtf(a * a + b * b);
+        }
+        slot += nodes;
+        __syncwarp();
+        float *t2 = src; src = dst; dst = t2;
+    }
+    if (lane == 0) cb[H + H - 1] = 0;                          // the unused last slot
+    __syncwarp();
+    // packed arrays: 4-bit level-1 fields, 2-bit higher-level fields
+    const int c_off = is_v ? L.vc_off : L.kc_off, c_bpt = is_v ? L.vc_bpt : L.kc_bpt;
+    const int c2_off = is_v ? L.vc2_off : L.kc2_off, c2_bpt = is_v ? L.vc2_bpt : L.kc2_bpt;
+    for (int j = lane; j < H / 2; j += 32)
+        page[c_off + pos * c_bpt + j] = uint8_t(cb[2 * j] | (cb[2 * j + 1] << 4));
+    for (int j = lane; j < H / 4; j += 32)
+        page[c2_off + pos * c2_bpt + j] =
+            uint8_t(cb[H + 4 * j] | (cb[H + 4 * j + 1] << 2) | (cb[H + 4 * j + 2] << 4) | (cb[H + 4 * j + 3] << 6));
+    if (lane == 0) *reinterpret_cast<uint16_t *>(page + (is_v ? L.vn_off : L.kn_off) + pos * 2) = nh;
+    if (is_v || !L.kqjl) return false;
+    // y_hat: the stored radius split top down by the centre angles
+    const float nhf = h2f_bits(nh);
+    src = ra; dst = rb;
+    if (lane == 0) src[0] = nhf;
+    __syncwarp();
+    // levels log2 D .. 2 top down; level l has D >> l angles, stored from
+    // slot H - 1 - (its count and those of the levels above) upward
+    slot = H - 1;
+    int level = 0;
+    while ((1 << level) < D) ++level;
+    for (int nodes = 1; nodes < H; nodes <<= 1, --level) {
+        slot -= nodes;
+        const float *tl = tab + 48 + 12 * (level - 2);
+        for (int i = lane; i < nodes; i += 32) {
+            const uint32_t k = cb[H + slot + i];
+            dst[2 * i] = src[i] * tl[4 + k];
+            dst[2 * i + 1] = src[i] * tl[8 + k];
+        }
+        __syncwarp();
+        float *t2 = src; src = dst; dst = t2;
+    }
+    for (int p = lane; p < H; p += 32) {
+        const uint32_t k = cb[p];
+        ys[2 * p] = src[p] * tab[16 + k];                          // y_hat over y's staging area
+        ys[2 * p + 1] = src[p] * tab[32 + k];
+    }
+    __syncwarp();
+    float rr = 0.f;
+    const bool active = lane < WarpVec<D>::LANES;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        r[e] = active ? y[e] - ys[lane * E + e] : 0.f;
+        rr = fmaf(r[e], r[e], rr);
+    }
+    const float rho = sqrtf(warp_sum(rr));
+    if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kr_off + pos * 2) = f2h_bits(rho);
+    __syncwarp();
+    return true;
+}
+
 // Compress the warp-held vector x (lane l holds coordinates [l E, l E + E)
 // of the input, E = WarpVec<D>::E) into slot `pos` of `page`: n = ||x||,
 // y = R x, codes = bucket(y / n) stored sign-magnitude, fp16 norm; FP8 keys
 // store e4m3(sqrt(d) y / n).  For QJL keys the residual r = y - nhat c[code]
 // is left in r (fp32, rotated basis), rho = fp16 ||r|| is stored, and the
 // function returns true (the caller projects r by S).  x is overwritten.
+//
+// The dense rotation (P.rot) takes y = R x through wbuf (D floats of shared
+// memory for this warp) and the norm of y; H D / sqrt(d) the norm of x.
 template <int D>
 __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevParams &P, bool is_v, float (&x)[WarpVec<D>::E],
-                                                   uint8_t *page, int pos, int lane, float (&r)[WarpVec<D>::E]) {
+                                                   uint8_t *page, int pos, int lane, float (&r)[WarpVec<D>::E],
+                                                   float *wbuf) {
     constexpr int E = WarpVec<D>::E;
-    const float rs = 1.0f / sqrtf(float(D));
     const float sqrt_d = sqrtf(float(D));
     const int bits = is_v ? L.vbits : L.kbits;
-    float sg[E];
-    load_vec<D>(P.signs, lane, sg);
     float ss = 0.f;
+    if (!P.rot) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        ss = fmaf(x[e], x[e], ss);
-        x[e] *= sg[e];
+        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+    }
+    rotate_warp<D>(P, x, wbuf, lane);                   // y = R x
+    if (P.rot) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
     }
     const float n = sqrtf(warp_sum(ss));
-    fwht_warp<D>(x, lane);
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] *= rs;          // y = R x
     const float inv = n > 0.f ? 1.0f / n : 0.f;
     const uint16_t nh = f2h_bits(n);
     const float nhf = h2f_bits(nh);
@@ -53,21 +202,52 @@ __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevPar
         return false;
     }
 
-    const int nb = (1 << bits) - 1;
+    if (is_v ? L.vpolar : L.kpolar) {
+        // polar codes: transform, codes and (keys with QJL) the residual y - y_hat
+        const bool res = polar_encode_warp<D>(L, P, is_v, x, n, nh, page, pos, lane, r, wbuf);
+        return res && !is_v && L.kqjl;
+    }
+    // fractional rates: lanes holding coordinates d/2 .. d-1 use the second codebook
+    const bool half = is_v ? L.vhalf : L.khalf;
+    const bool second = half && lane >= WarpVec<D>::LANES / 2;
+    const int wbits = half ? (second ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
+    // bucket = #{j : t_j <= u} by a binary search over this lane's codebook,
+    // staged in the warp's buffer (lanes of the second half of a fractional
+    // rate use their own copy): 2^W - 1 ascending bounds, then 2^W levels
+    float *tbase = wbuf + codebook_offset<D>();
+    __syncwarp();
+    for (int j = lane; j < 64; j += 32) {            // both codebooks, by all lanes
+        const int seg = j >> 5, o = j & 31;
+        if (seg == 1 && !half) continue;
+        const int w = half ? (seg ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
+        if (o < (1 << w) - 1) tbase[j] = (seg ? P.bounds2 : P.bounds)[o];
+        else if (o >= 16 && o < 16 + (1 << w)) tbase[j] = (seg ? P.lv2 : P.lv)[o - 16];
+    }
+    __syncwarp();
+    const float *tb = tbase + (second ? 32 : 0);
     uint32_t kap[E];
     float cval[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const float u = x[e] * inv;
         uint32_t idx = 0;
-        for (int j = 0; j < nb; ++j) idx += (P.bounds[j] <= u) ? 1u : 0u;
-        kap[e] = kappa_of(idx, bits);
-        cval[e] = P.lv[kap[e]];
+        for (int step = 1 << (wbits - 1); step >= 1; step >>= 1)
+            idx += (tb[idx + step - 1] <= u) ? uint32_t(step) : 0u;
+        kap[e] = kappa_of(idx, wbits);
+        cval[e] = tb[16 + kap[e]];
     }
+    __syncwarp();
     const int code_off = is_v ? L.vc_off : L.kc_off;
     const int code_bpt = is_v ? L.vc_bpt : L.kc_bpt;
     uint8_t *cdst = page + code_off + pos * code_bpt;
-    if (bits == 1) {
+    if (half) {
+        if (is_v)
+            store_half_codes<D>(page, pos, lane, kap, reinterpret_cast<uint8_t *>(wbuf), L.va_bits, L.vc_off, L.vc_bpt,
+                                L.vh_off, L.vh_bpt, L.vc2_off, L.vc2_bpt, L.vh2_off, L.vh2_bpt);
+        else
+            store_half_codes<D>(page, pos, lane, kap, reinterpret_cast<uint8_t *>(wbuf), L.ka_bits, L.kc_off, L.kc_bpt,
+                                L.kh_off, L.kh_bpt, L.kc2_off, L.kc2_bpt, L.kh2_off, L.kh2_bpt);
+    } else if (bits == 1) {
         store_fields<D, 1>(cdst, lane, kap);
     } else if (bits == 2) {
         store_fields<D, 2>(cdst, lane, kap);

@@ -23,14 +23,24 @@ namespace tq {
 struct Layout {
     int d, kbits, kqjl, vbits, P, H;
     int kc_off, kc_bpt, kc_w;   // main K code array and its field width
-    int kh_off, kh_bpt;         // K sign-bit array (kbits == 3 only)
+    int kh_off, kh_bpt;         // K sign-bit array (3-bit codes only)
     int ks_off, ks_bpt;         // QJL sign bits
     int kn_off, kr_off;         // fp16 norms
     int vc_off, vc_bpt, vc_w;
     int vh_off, vh_bpt;
     int vn_off;
     int page_bytes;
+    // Fractional rates (TQ_BITS_HALF | b): kc/kh above hold coordinates
+    // 0 .. d/2-1 at ka_bits = b + 1 bits, kc2/kh2 coordinates d/2 .. d-1 at
+    // kb_bits = b (likewise for values); ka_bits = kb_bits = kbits otherwise.
+    int khalf, ka_bits, kb_bits, kc2_off, kc2_bpt, kc2_w, kh2_off, kh2_bpt;
+    int vhalf, va_bits, vb_bits, vc2_off, vc2_bpt, vc2_w, vh2_off, vh2_bpt;
+    // Polar codes (TQ_BITS_POLAR): kc holds the d/2 level-1 angle codes
+    // (4 bits), kc2 the d/2 - 1 higher-level codes (2 bits, d/2 slots).
+    int kpolar, vpolar;
 };
+
+inline bool is_half(int bits) { return (bits & TQ_BITS_HALF) != 0; }
 
 inline int pad16(int x) { return (x + 15) & ~15; }
 
@@ -45,15 +55,46 @@ inline bool make_layout(const tq_cache_desc &c, Layout *L) {
     L->kh_off = L->kh_bpt = L->ks_off = L->ks_bpt = L->kr_off = -1;
     L->vc_off = L->vc_bpt = L->vh_off = L->vh_bpt = L->vn_off = -1;
     L->vc_w = 0;
-    if (c.kbits == 8) { add(d, &L->kc_off, &L->kc_bpt); L->kc_w = 8; }
-    else if (c.kbits == 3) { add(d * 2 / 8, &L->kc_off, &L->kc_bpt); L->kc_w = 2; add(d / 8, &L->kh_off, &L->kh_bpt); }
-    else { add(d * c.kbits / 8, &L->kc_off, &L->kc_bpt); L->kc_w = c.kbits; }
+    L->kc2_off = L->kc2_bpt = L->kh2_off = L->kh2_bpt = -1;
+    L->vc2_off = L->vc2_bpt = L->vh2_off = L->vh2_bpt = -1;
+    L->kc2_w = L->vc2_w = 0;
+    // one code of `bits` bits over n coordinates: a main array (w bits) and,
+    // for 3 bits, a 2-bit array followed by a 1-bit sign array
+    auto code = [&](int bits, int n, int *co, int *cb, int *cw, int *ho, int *hb) {
+        if (bits == 8) { add(n, co, cb); *cw = 8; }
+        else if (bits == 3) { add(n * 2 / 8, co, cb); *cw = 2; add(n / 8, ho, hb); }
+        else { add(n * bits / 8, co, cb); *cw = bits; }
+    };
+    L->kpolar = c.kbits == TQ_BITS_POLAR ? 1 : 0;
+    L->vpolar = c.vbits == TQ_BITS_POLAR ? 1 : 0;
+    auto polar_codes = [&](int *co, int *cb, int *cw, int *c2o, int *c2b, int *c2w) {
+        add(d / 2 * 4 / 8, co, cb); *cw = 4;
+        add(d / 2 * 2 / 8, c2o, c2b); *c2w = 2;
+    };
+    L->khalf = is_half(c.kbits) ? 1 : 0;
+    L->ka_bits = L->khalf ? (c.kbits & 7) + 1 : c.kbits;
+    L->kb_bits = L->khalf ? (c.kbits & 7) : c.kbits;
+    const int kn = L->khalf ? d / 2 : d;
+    if (L->kpolar) {
+        polar_codes(&L->kc_off, &L->kc_bpt, &L->kc_w, &L->kc2_off, &L->kc2_bpt, &L->kc2_w);
+    } else {
+        code(L->ka_bits, kn, &L->kc_off, &L->kc_bpt, &L->kc_w, &L->kh_off, &L->kh_bpt);
+        if (L->khalf) code(L->kb_bits, d / 2, &L->kc2_off, &L->kc2_bpt, &L->kc2_w, &L->kh2_off, &L->kh2_bpt);
+    }
     if (c.kqjl) add(d / 8, &L->ks_off, &L->ks_bpt);
     add(2, &L->kn_off, &dummy);
     if (c.kqjl) add(2, &L->kr_off, &dummy);
+    L->vhalf = is_half(c.vbits) ? 1 : 0;
+    L->va_bits = L->vhalf ? (c.vbits & 7) + 1 : c.vbits;
+    L->vb_bits = L->vhalf ? (c.vbits & 7) : c.vbits;
     if (c.vbits > 0) {
-        if (c.vbits == 3) { add(d * 2 / 8, &L->vc_off, &L->vc_bpt); L->vc_w = 2; add(d / 8, &L->vh_off, &L->vh_bpt); }
-        else { add(d * c.vbits / 8, &L->vc_off, &L->vc_bpt); L->vc_w = c.vbits; }
+        const int vn = L->vhalf ? d / 2 : d;
+        if (L->vpolar) {
+            polar_codes(&L->vc_off, &L->vc_bpt, &L->vc_w, &L->vc2_off, &L->vc2_bpt, &L->vc2_w);
+        } else {
+            code(L->va_bits, vn, &L->vc_off, &L->vc_bpt, &L->vc_w, &L->vh_off, &L->vh_bpt);
+            if (L->vhalf) code(L->vb_bits, d / 2, &L->vc2_off, &L->vc2_bpt, &L->vc2_w, &L->vh2_off, &L->vh2_bpt);
+        }
         add(2, &L->vn_off, &dummy);
     }
     L->page_bytes = off;
@@ -65,13 +106,25 @@ struct DevParams {
     int d, bits;
     const float *signs;      // [d] +1/-1
     const uint16_t *S;       // [d][d] bf16 bits, row-major (row j = projection j)
+    const uint16_t *S16;     // the same matrix as fp16 bits (exact for |S| >= 2^-14)
     const float *lv;         // [2^bits] levels indexed by the stored sign-magnitude code
     const float *bounds;     // [2^bits - 1] ascending decision boundaries
+    // fractional rates: lv / bounds belong to the (b + 1)-bit codebook of
+    // coordinates 0 .. d/2-1, lv2 / bounds2 to the b-bit one of the rest
+    const float *lv2, *bounds2;
+    // polar codes (TQ_BITS_POLAR): level-1 bounds [0, 16), cos / sin of the
+    // level-1 centres [16, 32) / [32, 48), level l >= 2 at 48 + 12 (l - 2):
+    // 3 bounds, 4 cos, 4 sin of its centres
+    const float *polar;
     // d == 128 only (else null): 32 KB images of 128 x 128 operand tiles laid
     // out exactly as the tensor cores read them from shared memory (K-major,
     // 128-byte swizzle, two 64-column halves), so one bulk copy stages them.
     const uint8_t *rot_img;  // bf16 (H D)[n][k] = (-1)^popcount(n & k) * D[k]
     const uint8_t *s16_img;  // fp16 S[n][k] (exact for |S| >= 2^-17)
+    // Dense random rotation (rot = 1, d <= 256) instead of H D / sqrt(d):
+    // Rd[j][i] (y = Rd x) and its transpose RdT (x = Rd^T y), fp32.
+    int rot;
+    const float *Rd, *RdT;
 };
 
 // Byte offset of element (row, col) of a 128 x 128 16-bit tile in the
@@ -93,6 +146,7 @@ struct tq_params {
     float *h_S;
     float *h_levels;         // ascending bucket order
     float *h_bounds;
+    float *h_R;              // dense rotation [d][d] (nullptr: H D / sqrt(d))
     void *d_block;           // device allocation
     tq::DevParams dev;
 };

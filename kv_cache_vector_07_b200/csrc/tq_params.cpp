@@ -158,6 +158,65 @@ bool lloyd_max_positive(int d, int bits, std::vector<double> &pos) {
     return false;
 }
 
+// Law of the polar transform's angle between two k-dimensional sub-block
+// radii of a random direction: density proportional to (sin p cos p)^(k-1)
+// on [0, pi/2].  Cell mass and first moment by composite Gauss-Legendre.
+struct AngleLaw {
+    double km1;
+    std::vector<double> gx, gw;
+    explicit AngleLaw(int k) : km1(k - 1.0) { gauss_legendre(24, gx, gw); }
+    double pdf(double p) const {
+        const double s = std::sin(p) * std::cos(p);
+        return s > 0.0 ? std::exp(km1 * std::log(s)) : 0.0;
+    }
+    template <typename F>
+    double integral(double lo, double hi, F f) const {
+        const int panels = 256;
+        double sum = 0.0, h = (hi - lo) / panels;
+        for (int q = 0; q < panels; ++q) {
+            const double c = lo + (q + 0.5) * h;
+            for (size_t j = 0; j < gx.size(); ++j) {
+                const double x = c + 0.5 * h * gx[j];
+                sum += gw[j] * f(x) * pdf(x);
+            }
+        }
+        return sum * 0.5 * h;
+    }
+};
+
+// Lloyd-Max levels of the angle law with 2^bits levels (ascending).  The law
+// is symmetric about pi/4: the lower half of the levels is iterated with
+// pi/4 as its last edge and mirrored.
+bool lloyd_max_angle(int k, int bits, std::vector<double> &lv) {
+    const int L = 1 << bits, h = L / 2;
+    AngleLaw law(k);
+    const double q = M_PI / 4.0;
+    std::vector<double> c(h), edge(h + 1);
+    for (int j = 0; j < h; ++j) c[j] = q * (j + 0.5) / h;          // any ordered start in (0, pi/4)
+    bool ok = false;
+    for (int it = 0; it < 200000 && !ok; ++it) {
+        edge[0] = 0.0;
+        edge[h] = q;
+        for (int j = 1; j < h; ++j) edge[j] = 0.5 * (c[j - 1] + c[j]);
+        double change = 0.0;
+        for (int j = 0; j < h; ++j) {
+            const double m0 = law.integral(edge[j], edge[j + 1], [](double) { return 1.0; });
+            const double m1 = law.integral(edge[j], edge[j + 1], [](double x) { return x; });
+            const double nc = m1 / m0;
+            change = std::fmax(change, std::fabs(nc - c[j]));
+            c[j] = nc;
+        }
+        ok = change < 1e-15;
+    }
+    if (!ok) return false;
+    lv.assign(L, 0.0);
+    for (int j = 0; j < h; ++j) {
+        lv[j] = c[j];
+        lv[L - 1 - j] = 2.0 * q - c[j];
+    }
+    return true;
+}
+
 }  // namespace
 
 namespace {
@@ -183,22 +242,125 @@ bool host_params(int d, int bits, uint64_t seed, std::vector<int8_t> &signs, std
     levels.clear();
     bounds.clear();
     if (bits == 8) return true;
-    const int L = 1 << bits, h = L / 2;
-    std::vector<double> pos;
-    if (!lloyd_max_positive(d, bits, pos)) return false;
-    levels.assign(L, 0.0f);
-    for (int k = 0; k < h; ++k) {
-        const float c = float(pos[k]);
-        levels[h + k] = c;
-        levels[h - 1 - k] = -c;
+    if (bits == TQ_BITS_POLAR) {
+        // level-1 angles: uniform cells of [0, 2 pi), centres as levels; then
+        // 2-bit Lloyd-Max levels of the angle law for levels 2 .. log2 d
+        const int L1 = 16;
+        for (int j = 0; j < L1; ++j) levels.push_back(float((j + 0.5) * (2.0 * M_PI / L1)));
+        for (int j = 0; j + 1 < L1; ++j) bounds.push_back(float(0.5 * (double(levels[j]) + double(levels[j + 1]))));
+        for (int l = 2; (1 << l) <= d; ++l) {
+            std::vector<double> lv;
+            if (!lloyd_max_angle(1 << (l - 1), 2, lv)) return false;
+            const size_t b0 = levels.size();
+            for (double v : lv) levels.push_back(float(v));
+            for (int j = 0; j + 1 < 4; ++j)
+                bounds.push_back(float(0.5 * (double(levels[b0 + j]) + double(levels[b0 + j + 1]))));
+        }
+        return true;
     }
-    bounds.assign(L - 1, 0.0f);
-    for (int j = 0; j + 1 < L; ++j) bounds[j] = float(0.5 * (double(levels[j]) + double(levels[j + 1])));
+    // a fractional rate concatenates the (b + 1)-bit codebook and the b-bit one
+    const int widths[2] = {(bits & TQ_BITS_HALF) ? (bits & 7) + 1 : bits, (bits & TQ_BITS_HALF) ? (bits & 7) : 0};
+    for (int part = 0; part < 2 && widths[part] > 0; ++part) {
+        const int L = 1 << widths[part], h = L / 2;
+        std::vector<double> pos;
+        if (!lloyd_max_positive(d, widths[part], pos)) return false;
+        std::vector<float> lv(L, 0.0f);
+        for (int k = 0; k < h; ++k) {
+            const float c = float(pos[k]);
+            lv[h + k] = c;
+            lv[h - 1 - k] = -c;
+        }
+        for (int j = 0; j < L; ++j) levels.push_back(lv[j]);
+        for (int j = 0; j + 1 < L; ++j) bounds.push_back(float(0.5 * (double(lv[j]) + double(lv[j + 1]))));
+    }
     return true;
+}
+
+// Levels and bounds per code width: the first (or only) codebook, and for a
+// fractional rate the second.
+int log2i(int d) {
+    int l = 0;
+    while ((1 << l) < d) ++l;
+    return l;
+}
+int n_levels(int bits, int d) {
+    if (bits == 8) return 0;
+    if (bits == TQ_BITS_POLAR) return 16 + 4 * (log2i(d) - 1);
+    if (bits & TQ_BITS_HALF) return (2 << (bits & 7)) + (1 << (bits & 7));
+    return 1 << bits;
+}
+int n_bounds(int bits, int d) {
+    if (bits == 8) return 0;
+    if (bits == TQ_BITS_POLAR) return 15 + 3 * (log2i(d) - 1);
+    if (bits & TQ_BITS_HALF) return n_levels(bits, d) - 2;
+    return (1 << bits) - 1;
+}
+
+// Dense rotation: rows of the d x d Gaussian matrix (SplitMix64 stream 2,
+// Box-Muller, float64) orthonormalised in order, computed here as the
+// Householder QR factorisation of its transpose with the columns of Q
+// signed so that the triangular factor has a positive diagonal; stored in
+// float32 (round to nearest even).
+void dense_rotation_host(int d, uint64_t seed, std::vector<float> &R) {
+    const size_t dd = size_t(d) * d;
+    std::vector<double> g(dd);
+    for (size_t k = 0; k < dd; k += 2) {
+        const uint64_t pr = k / 2;
+        const uint64_t a = splitmix_at(seed, 2, 2 * pr), b = splitmix_at(seed, 2, 2 * pr + 1);
+        const double u1 = (double(a >> 11) + 1.0) * 0x1.0p-53;
+        const double u2 = double(b >> 11) * 0x1.0p-53;
+        const double rad = std::sqrt(-2.0 * std::log(u1));
+        g[k] = rad * std::cos(2.0 * M_PI * u2);
+        if (k + 1 < dd) g[k + 1] = rad * std::sin(2.0 * M_PI * u2);
+    }
+    // A = G^T (A[i][j] = G[j][i]); reflect columns k = 0 .. d-1 in turn
+    std::vector<double> A(dd), vs(dd, 0.0), vn(d, 0.0);
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) A[size_t(i) * d + j] = g[size_t(j) * d + i];
+    for (int k = 0; k < d; ++k) {
+        double xn = 0.0;
+        for (int i = k; i < d; ++i) xn += A[size_t(i) * d + k] * A[size_t(i) * d + k];
+        xn = std::sqrt(xn);
+        const double x0 = A[size_t(k) * d + k];
+        const double alpha = x0 >= 0.0 ? -xn : xn;
+        double *v = &vs[size_t(k) * d];
+        for (int i = k; i < d; ++i) v[i] = A[size_t(i) * d + k];
+        v[k] -= alpha;
+        double v2 = 0.0;
+        for (int i = k; i < d; ++i) v2 += v[i] * v[i];
+        vn[k] = v2;
+        if (v2 == 0.0) continue;
+        for (int j = k; j < d; ++j) {
+            double t = 0.0;
+            for (int i = k; i < d; ++i) t += v[i] * A[size_t(i) * d + j];
+            const double f = 2.0 * t / v2;
+            for (int i = k; i < d; ++i) A[size_t(i) * d + j] -= f * v[i];
+        }
+    }
+    // Q = H_0 H_1 ... H_{d-1} I
+    std::vector<double> Q(dd, 0.0);
+    for (int i = 0; i < d; ++i) Q[size_t(i) * d + i] = 1.0;
+    for (int k = d - 1; k >= 0; --k) {
+        if (vn[k] == 0.0) continue;
+        const double *v = &vs[size_t(k) * d];
+        for (int j = 0; j < d; ++j) {
+            double t = 0.0;
+            for (int i = k; i < d; ++i) t += v[i] * Q[size_t(i) * d + j];
+            const double f = 2.0 * t / vn[k];
+            for (int i = k; i < d; ++i) Q[size_t(i) * d + j] -= f * v[i];
+        }
+    }
+    R.assign(dd, 0.0f);
+    for (int j = 0; j < d; ++j) {
+        const double sg = A[size_t(j) * d + j] < 0.0 ? -1.0 : 1.0;     // sign of the triangular diagonal
+        for (int i = 0; i < d; ++i) R[size_t(j) * d + i] = float(sg * Q[size_t(i) * d + j]);
+    }
 }
 
 bool args_ok(int d, int bits) {
     if (d < 8 || d > 1024 || (d & (d - 1))) return false;
+    if (bits == TQ_BITS_POLAR) return d >= 8 && d <= 256;
+    if (bits & TQ_BITS_HALF) return (bits & ~TQ_BITS_HALF) >= 1 && (bits & ~TQ_BITS_HALF) <= 3 && d >= 16 && d <= 256;
     return bits == 1 || bits == 2 || bits == 3 || bits == 4 || bits == 8;
 }
 
@@ -222,9 +384,18 @@ extern "C" int tq_compute_params_host(int d, int bits, uint64_t seed, int8_t *si
 }
 
 extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
+    return tq_make_params_rot(d, bits, seed, TQ_ROT_HADAMARD, out);
+}
+
+extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, tq_params **out) {
     if (!out) return TQ_EINVAL;
     *out = nullptr;
     if (!args_ok(d, bits)) return TQ_EUNSUPPORTED;
+    if (rotation != TQ_ROT_HADAMARD && rotation != TQ_ROT_DENSE) return TQ_EUNSUPPORTED;
+    const bool dense = rotation == TQ_ROT_DENSE;
+    if (dense && d > 256) return TQ_EUNSUPPORTED;
+    std::vector<float> Rd;
+    if (dense) dense_rotation_host(d, seed, Rd);
 
     std::vector<int8_t> sg;
     std::vector<uint16_t> S_bits;
@@ -238,11 +409,11 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
     p->seed = seed;
     cudaGetDevice(&p->device);
     const size_t dd = size_t(d) * d;
-    const int L = bits == 8 ? 0 : (1 << bits);
+    const int L = n_levels(bits, d), NB = n_bounds(bits, d);
     p->h_signs = new int8_t[d];
     p->h_S = new float[dd];
     p->h_levels = L ? new float[L] : nullptr;
-    p->h_bounds = L ? new float[L - 1] : nullptr;
+    p->h_bounds = L ? new float[NB] : nullptr;
     std::vector<float> signs_f(d);
     for (int i = 0; i < d; ++i) {
         p->h_signs[i] = sg[i];
@@ -250,20 +421,60 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
     }
     for (size_t k = 0; k < dd; ++k) p->h_S[k] = bf16_to_float(S_bits[k]);
     // Device levels are indexed by the stored sign-magnitude code:
-    // code = (neg << (bits-1)) | rank.
-    std::vector<float> lv_code(L > 0 ? L : 1, 0.0f);
-    if (L) {
-        const int h = L / 2;
+    // code = (neg << (w-1)) | rank.  Each codebook takes 32 floats of the
+    // level area and 32 of the bound area (the second one: fractional rates).
+    std::vector<float> lv_code(64, 0.0f), bd_dev(64, 0.0f);
+    // polar tables: level-1 bounds [0, 16), cos / sin of the level-1 centres
+    // [16, 32) / [32, 48); level l >= 2 at 48 + 12 (l - 2): 3 bounds, 4 cos, 4 sin
+    std::vector<float> polar_tab(256, 0.0f);
+    const bool polar = bits == TQ_BITS_POLAR;
+    if (polar) {
         for (int j = 0; j < L; ++j) p->h_levels[j] = lv[j];
-        for (int j = 0; j + 1 < L; ++j) p->h_bounds[j] = bd0[j];
-        for (int k = 0; k < h; ++k) {
-            lv_code[k] = lv[h + k];
-            lv_code[h + k] = lv[h - 1 - k];
+        for (int j = 0; j < NB; ++j) p->h_bounds[j] = bd0[j];
+        for (int j = 0; j < 15; ++j) polar_tab[j] = bd0[j];
+        for (int j = 0; j < 16; ++j) {
+            polar_tab[16 + j] = float(std::cos(double(lv[j])));
+            polar_tab[32 + j] = float(std::sin(double(lv[j])));
+        }
+        for (int l = 2; (1 << l) <= d; ++l) {
+            const int b = 48 + 12 * (l - 2), li = 16 + 4 * (l - 2), bi = 15 + 3 * (l - 2);
+            for (int j = 0; j < 3; ++j) polar_tab[b + j] = bd0[bi + j];
+            for (int j = 0; j < 4; ++j) {
+                polar_tab[b + 4 + j] = float(std::cos(double(lv[li + j])));
+                polar_tab[b + 8 + j] = float(std::sin(double(lv[li + j])));
+            }
+        }
+    }
+    if (L && !polar) {
+        for (int j = 0; j < L; ++j) p->h_levels[j] = lv[j];
+        for (int j = 0; j < NB; ++j) p->h_bounds[j] = bd0[j];
+        const bool half = (bits & TQ_BITS_HALF) != 0;
+        const int wa = half ? (bits & 7) + 1 : bits;
+        int lbase = 0, bbase = 0;
+        for (int part = 0; part < (half ? 2 : 1); ++part) {
+            const int w = part == 0 ? wa : wa - 1, Lw = 1 << w, h = Lw / 2;
+            for (int k = 0; k < h; ++k) {
+                lv_code[32 * part + k] = lv[lbase + h + k];
+                lv_code[32 * part + h + k] = lv[lbase + h - 1 - k];
+            }
+            for (int j = 0; j + 1 < Lw; ++j) bd_dev[32 * part + j] = bd0[bbase + j];
+            lbase += Lw;
+            bbase += Lw - 1;
         }
     }
 
-    // Operand images for the d = 128 tensor-core encoder.
-    const bool imgs = d == 128;
+    p->h_R = nullptr;
+    std::vector<float> RdT;
+    if (dense) {
+        p->h_R = new float[dd];
+        std::memcpy(p->h_R, Rd.data(), sizeof(float) * dd);
+        RdT.assign(dd, 0.0f);
+        for (int j = 0; j < d; ++j)
+            for (int i = 0; i < d; ++i) RdT[size_t(i) * d + j] = Rd[size_t(j) * d + i];
+    }
+
+    // Operand images for the d = 128 tensor-core encoder (Hadamard rotation only).
+    const bool imgs = d == 128 && !dense && bits != TQ_BITS_POLAR && !(bits & TQ_BITS_HALF);
     std::vector<uint16_t> rot_img, s16_img;
     if (imgs) {
         rot_img.assign(128 * 128, 0);
@@ -279,24 +490,35 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
             }
     }
 
-    // one device block: signs | S (bf16) | levels by code | bounds | images
+    std::vector<uint16_t> S16(dd);
+    for (size_t k = 0; k < dd; ++k) {
+        const __half h = __float2half_rn(bf16_to_float(S_bits[k]));
+        std::memcpy(&S16[k], &h, 2);
+    }
+    // one device block: signs | S (bf16) | levels by code | bounds | images | S (fp16) | polar | dense
     const size_t off_signs = 0;
     const size_t off_S = 256 * ((sizeof(float) * d + 255) / 256);
     const size_t off_lv = off_S + 256 * ((sizeof(uint16_t) * dd + 255) / 256);
     const size_t off_bd = off_lv + 256;
     const size_t off_rot = off_bd + 256;
     const size_t off_s16 = off_rot + (imgs ? 32768 : 0);
-    const size_t total = off_s16 + (imgs ? 32768 : 0);
+    const size_t off_S16 = off_s16 + (imgs ? 32768 : 0);
+    const size_t off_polar = off_S16 + 256 * ((sizeof(uint16_t) * dd + 255) / 256);
+    const size_t off_R = off_polar + (polar ? 1024 : 0);
+    const size_t off_RT = off_R + (dense ? sizeof(float) * dd : 0);
+    const size_t total = off_RT + (dense ? sizeof(float) * dd : 0);
     if (cudaMalloc(&p->d_block, total) != cudaSuccess) { p->d_block = nullptr; tq_free_params(p); return TQ_ENOMEM; }
     uint8_t *base = static_cast<uint8_t *>(p->d_block);
-    std::vector<float> bd(L > 1 ? L - 1 : 1, 0.0f);
-    for (int j = 0; j + 1 < L; ++j) bd[j] = p->h_bounds[j];
     if (cudaMemcpy(base + off_signs, signs_f.data(), sizeof(float) * d, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(base + off_S, S_bits.data(), sizeof(uint16_t) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(base + off_lv, lv_code.data(), sizeof(float) * lv_code.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(base + off_bd, bd.data(), sizeof(float) * bd.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base + off_lv, lv_code.data(), 256, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base + off_bd, bd_dev.data(), 256, cudaMemcpyHostToDevice) != cudaSuccess ||
         (imgs && (cudaMemcpy(base + off_rot, rot_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess ||
-                  cudaMemcpy(base + off_s16, s16_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess))) {
+                  cudaMemcpy(base + off_s16, s16_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess)) ||
+        cudaMemcpy(base + off_S16, S16.data(), sizeof(uint16_t) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
+        (polar && cudaMemcpy(base + off_polar, polar_tab.data(), 1024, cudaMemcpyHostToDevice) != cudaSuccess) ||
+        (dense && (cudaMemcpy(base + off_R, Rd.data(), sizeof(float) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
+                   cudaMemcpy(base + off_RT, RdT.data(), sizeof(float) * dd, cudaMemcpyHostToDevice) != cudaSuccess))) {
         tq_free_params(p);
         return TQ_ECUDA;
     }
@@ -306,8 +528,15 @@ extern "C" int tq_make_params(int d, int bits, uint64_t seed, tq_params **out) {
     p->dev.S = reinterpret_cast<const uint16_t *>(base + off_S);
     p->dev.lv = reinterpret_cast<const float *>(base + off_lv);
     p->dev.bounds = reinterpret_cast<const float *>(base + off_bd);
+    p->dev.lv2 = reinterpret_cast<const float *>(base + off_lv + 128);
+    p->dev.bounds2 = reinterpret_cast<const float *>(base + off_bd + 128);
     p->dev.rot_img = imgs ? base + off_rot : nullptr;
     p->dev.s16_img = imgs ? base + off_s16 : nullptr;
+    p->dev.S16 = reinterpret_cast<const uint16_t *>(base + off_S16);
+    p->dev.polar = polar ? reinterpret_cast<const float *>(base + off_polar) : nullptr;
+    p->dev.rot = dense ? 1 : 0;
+    p->dev.Rd = dense ? reinterpret_cast<const float *>(base + off_R) : nullptr;
+    p->dev.RdT = dense ? reinterpret_cast<const float *>(base + off_RT) : nullptr;
     *out = p;
     return TQ_OK;
 }
@@ -319,7 +548,43 @@ extern "C" void tq_free_params(tq_params *p) {
     delete[] p->h_S;
     delete[] p->h_levels;
     delete[] p->h_bounds;
+    delete[] p->h_R;
     delete p;
+}
+
+extern "C" int tq_compute_rotation_host(int d, uint64_t seed, int rotation, float *R) {
+    if (!R || d < 8 || d > 1024 || (d & (d - 1))) return TQ_EINVAL;
+    if (rotation == TQ_ROT_DENSE) {
+        if (d > 256) return TQ_EUNSUPPORTED;
+        std::vector<float> Rd;
+        dense_rotation_host(d, seed, Rd);
+        std::memcpy(R, Rd.data(), sizeof(float) * Rd.size());
+        return TQ_OK;
+    }
+    if (rotation != TQ_ROT_HADAMARD) return TQ_EUNSUPPORTED;
+    std::vector<int8_t> sg;
+    std::vector<uint16_t> sb;
+    std::vector<float> lv, bd;
+    if (!host_params(d, 8, seed, sg, sb, lv, bd)) return TQ_EUNSUPPORTED;
+    const double s = 1.0 / std::sqrt(double(d));
+    for (int j = 0; j < d; ++j)
+        for (int i = 0; i < d; ++i)
+            R[size_t(j) * d + i] = float(((__builtin_popcount(unsigned(j & i)) & 1) ? -s : s) * sg[i]);
+    return TQ_OK;
+}
+
+extern "C" int tq_params_export_rotation(const tq_params *p, float *R) {
+    if (!p || !R) return TQ_EINVAL;
+    const int d = p->d;
+    if (p->h_R) {
+        std::memcpy(R, p->h_R, sizeof(float) * size_t(d) * d);
+        return TQ_OK;
+    }
+    const double s = 1.0 / std::sqrt(double(d));
+    for (int j = 0; j < d; ++j)
+        for (int i = 0; i < d; ++i)
+            R[size_t(j) * d + i] = float(((__builtin_popcount(unsigned(j & i)) & 1) ? -s : s) * p->h_signs[i]);
+    return TQ_OK;
 }
 
 extern "C" int tq_params_export(const tq_params *p, int8_t *signs, float *S, float *levels,
@@ -329,9 +594,8 @@ extern "C" int tq_params_export(const tq_params *p, int8_t *signs, float *S, flo
     if (signs) std::memcpy(signs, p->h_signs, d);
     if (S) std::memcpy(S, p->h_S, sizeof(float) * d * d);
     if (p->bits != 8) {
-        const int L = 1 << p->bits;
-        if (levels) std::memcpy(levels, p->h_levels, sizeof(float) * L);
-        if (bounds) std::memcpy(bounds, p->h_bounds, sizeof(float) * (L - 1));
+        if (levels) std::memcpy(levels, p->h_levels, sizeof(float) * n_levels(p->bits, p->d));
+        if (bounds) std::memcpy(bounds, p->h_bounds, sizeof(float) * n_bounds(p->bits, p->d));
     }
     return TQ_OK;
 }

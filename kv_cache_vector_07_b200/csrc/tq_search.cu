@@ -23,19 +23,16 @@ constexpr int kMaxK = 64;
 template <int D>
 __global__ void __launch_bounds__(128) prep_f32_kernel(const float *Q, int64_t rows, DevParams p, float *qr) {
     constexpr int E = WarpVec<D>::E;
+    __shared__ float wbuf[4][D <= 256 ? D : 4];          // dense rotation only (d <= 256)
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int64_t row = int64_t(blockIdx.x) * 4 + wl;
     if (row >= rows) return;
-    float x[E], sg[E];
+    float x[E];
     load_vec<D>(Q + row * D, lane, x);
-    load_vec<D>(p.signs, lane, sg);
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] *= sg[e];
-    fwht_warp<D>(x, lane);
-    const float rs = 1.0f / sqrtf(float(D));
+    rotate_warp<D>(p, x, wbuf[wl], lane);
     if (lane < WarpVec<D>::LANES) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) qr[row * D + lane * E + e] = x[e] * rs;
+        for (int e = 0; e < E; ++e) qr[row * D + lane * E + e] = x[e];
     }
 }
 
@@ -59,7 +56,7 @@ __global__ void __launch_bounds__(128) score_kernel(ScoreArgs a) {
     __shared__ float sc[kQT][kTile];
     __shared__ float topv[kQT][kMaxK];
     __shared__ int64_t topi[kQT][kMaxK];
-    __shared__ float lv[16];
+    __shared__ float lv[16], lv2[8];
 
     const Layout &L = a.L;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -75,7 +72,8 @@ __global__ void __launch_bounds__(128) score_kernel(ScoreArgs a) {
         sq[c * kQT + q] = q < nq ? a.qr[int64_t(q0 + q) * D + c] : 0.f;
         sw[c * kQT + q] = q < nq ? a.w[int64_t(q0 + q) * D + c] : 0.f;
     }
-    if (tid < 16) lv[tid] = tid < (1 << L.kbits) ? a.p.lv[tid] : 0.f;
+    if (tid < 16) lv[tid] = tid < (1 << L.ka_bits) ? a.p.lv[tid] : 0.f;
+    if (tid < 8) lv2[tid] = (L.khalf && tid < (1 << L.kb_bits)) ? a.p.lv2[tid] : 0.f;   // fractional rates
     for (int i = tid; i < kQT * kMaxK; i += 128) {
         topv[i / kMaxK][i % kMaxK] = -INFINITY;
         topi[i / kMaxK][i % kMaxK] = -1;
@@ -90,15 +88,23 @@ __global__ void __launch_bounds__(128) score_kernel(ScoreArgs a) {
             const uint8_t *page = a.db + (t / L.P) * int64_t(L.page_bytes);
             const int pos = int(t % L.P);
             const uint8_t *kc = page + L.kc_off + pos * L.kc_bpt;
-            const uint8_t *kh = L.kbits == 3 ? page + L.kh_off + pos * L.kh_bpt : nullptr;
+            const uint8_t *kh = L.ka_bits == 3 ? page + L.kh_off + pos * L.kh_bpt : nullptr;
             const uint8_t *ks = L.kqjl ? page + L.ks_off + pos * L.ks_bpt : nullptr;
+            const int nA = L.khalf ? D / 2 : D;
             float mse[kQT], qj[kQT];
 #pragma unroll
             for (int q = 0; q < kQT; ++q) { mse[q] = 0.f; qj[q] = 0.f; }
             for (int i = 0; i < D; ++i) {
-                uint32_t kap = read_field(kc, i, L.kc_w);
-                if (kh) kap |= read_field(kh, i, 1) << 2;
-                const float cv = lv[kap];
+                float cv;
+                if (i < nA) {
+                    uint32_t kap = read_field(kc, i, L.kc_w);
+                    if (kh) kap |= read_field(kh, i, 1) << 2;
+                    cv = lv[kap];
+                } else {
+                    uint32_t kap = read_field(page + L.kc2_off + pos * L.kc2_bpt, i - nA, L.kc2_w);
+                    if (L.kb_bits == 3) kap |= read_field(page + L.kh2_off + pos * L.kh2_bpt, i - nA, 1) << 2;
+                    cv = lv2[kap];
+                }
                 const bool ps = ks ? (read_field(ks, i, 1) != 0) : true;
 #pragma unroll
                 for (int q = 0; q < kQT; ++q) {

@@ -30,6 +30,29 @@ TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_EDEVICE, TQ_ENOMEM, TQ_ESCRATCH 
 TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 TQ_DEV_SLOT_RANGE, TQ_DEV_BLOCK_RANGE, TQ_DEV_WAIT_TIMEOUT = 0x1, 0x2, 0x4
 TQ_DTYPE_BF16, TQ_DTYPE_F32 = 0, 1
+TQ_ROT_HADAMARD, TQ_ROT_DENSE = 0, 1
+TQ_BITS_HALF = 16
+TQ_BITS_POLAR = 32
+
+
+def half_bits(rate: float) -> int:
+    """Code width of a fractional rate (1.5, 2.5, 3.5): TQ_BITS_HALF | b."""
+    b = int(rate - 0.5)
+    if rate - 0.5 != b or not 1 <= b <= 3:
+        raise ValueError("fractional rates are 1.5, 2.5 and 3.5")
+    return TQ_BITS_HALF | b
+
+
+def _n_levels(bits: int, d: int) -> tuple[int, int]:
+    if bits == 8:
+        return 0, 0
+    if bits == TQ_BITS_POLAR:
+        lv = int(np.log2(d))
+        return 16 + 4 * (lv - 1), 15 + 3 * (lv - 1)
+    if bits & TQ_BITS_HALF:
+        b = bits & 7
+        return (2 << b) + (1 << b), (2 << b) + (1 << b) - 2
+    return 1 << bits, (1 << bits) - 1
 
 _vp, _i32, _i64, _u64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
 
@@ -52,6 +75,9 @@ def _sig(name, res, args):
 
 
 _sig("tq_make_params", _i32, [_i32, _i32, _u64, ctypes.POINTER(_vp)])
+_sig("tq_make_params_rot", _i32, [_i32, _i32, _u64, _i32, ctypes.POINTER(_vp)])
+_sig("tq_compute_rotation_host", _i32, [_i32, _u64, _i32, _vp])
+_sig("tq_params_export_rotation", _i32, [_vp, _vp])
 _sig("tq_compute_params_host", _i32, [_i32, _i32, _u64, _vp, _vp, _vp, _vp])
 _sig("tq_free_params", None, [_vp])
 _sig("tq_params_export", _i32, [_vp, _vp, _vp, _vp, _vp])
@@ -131,11 +157,17 @@ def _dev_check(*tensors):
 class Params:
     """Handle of library-owned parameters (tq_make_params)."""
 
-    def __init__(self, d: int, bits: int, seed: int):
+    def __init__(self, d: int, bits: int, seed: int, rotation: int = TQ_ROT_HADAMARD):
         h = _vp()
-        _check(_lib.tq_make_params(d, bits, seed, ctypes.byref(h)), "tq_make_params")
+        _check(_lib.tq_make_params_rot(d, bits, seed, rotation, ctypes.byref(h)), "tq_make_params_rot")
         self._h = h
-        self.d, self.bits, self.seed = d, bits, seed
+        self.d, self.bits, self.seed, self.rotation = d, bits, seed, rotation
+
+    def rotation_matrix(self) -> np.ndarray:
+        """tq_params_export_rotation: R [d, d] (y = R x), float32."""
+        R = np.zeros((self.d, self.d), np.float32)
+        _check(_lib.tq_params_export_rotation(self._h, R.ctypes.data), "tq_params_export_rotation")
+        return R
 
     @property
     def handle(self):
@@ -145,9 +177,9 @@ class Params:
         d = self.d
         signs = np.zeros(d, np.int8)
         S = np.zeros((d, d), np.float32)
-        L = 1 << self.bits if self.bits != 8 else 0
+        L, NB = _n_levels(self.bits, d)
         lv = np.zeros(max(L, 1), np.float32)
-        bd = np.zeros(max(L - 1, 1), np.float32)
+        bd = np.zeros(max(NB, 1), np.float32)
         _check(_lib.tq_params_export(self._h, signs.ctypes.data, S.ctypes.data, lv.ctypes.data, bd.ctypes.data),
                "tq_params_export")
         return signs, S, (lv if L else None), (bd if L else None)
@@ -159,16 +191,23 @@ class Params:
             self._h = _vp()
 
 
-def make_params(d: int, bits: int, seed: int) -> Params:
-    return Params(d, bits, seed)
+def make_params(d: int, bits: int, seed: int, rotation: int = TQ_ROT_HADAMARD) -> Params:
+    return Params(d, bits, seed, rotation)
+
+
+def compute_rotation_host(d: int, seed: int, rotation: int = TQ_ROT_DENSE) -> np.ndarray:
+    """tq_compute_rotation_host: the rotation matrix of (d, seed) on the host."""
+    R = np.zeros((d, d), np.float32)
+    _check(_lib.tq_compute_rotation_host(d, seed, rotation, R.ctypes.data), "tq_compute_rotation_host")
+    return R
 
 
 def compute_params_host(d: int, bits: int, seed: int):
     signs = np.zeros(d, np.int8)
     S = np.zeros((d, d), np.float32)
-    L = 1 << bits if bits != 8 else 0
+    L, NB = _n_levels(bits, d)
     lv = np.zeros(max(L, 1), np.float32)
-    bd = np.zeros(max(L - 1, 1), np.float32)
+    bd = np.zeros(max(NB, 1), np.float32)
     _check(_lib.tq_compute_params_host(d, bits, seed, signs.ctypes.data, S.ctypes.data, lv.ctypes.data,
                                        bd.ctypes.data), "tq_compute_params_host")
     return signs, S, (lv if L else None), (bd if L else None)

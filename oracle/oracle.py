@@ -530,7 +530,7 @@ class Layout:
         add("kn", 2)
         if self.kqjl:
             add("kr", 2)
-        if self.vbits > 0:
+        if self.vbits == "polar" or self.vbits > 0:
             codes("vc", self.vbits)
             add("vn", 2)
         self.page_bytes = off
@@ -609,7 +609,7 @@ def token_records(lay: Layout, Ek: Encoded, Ev: Encoded) -> dict:
     rec["kn"] = _fp16_bytes(Ek.nhat)
     if lay.kqjl:
         rec["kr"] = _fp16_bytes(Ek.rho)
-    if lay.vbits > 0:
+    if lay.vbits == "polar" or lay.vbits > 0:
         rec.update(_code_arrays("vc", lay.vbits, Ev if lay.vbits == "polar" else Ev.idx))
         rec["vn"] = _fp16_bytes(Ev.nhat)
     return rec
@@ -661,7 +661,7 @@ def read_cache(lay: Layout, cache: np.ndarray, slots: np.ndarray, head: int, n_h
 
     out = {"kidx": codes("kc", lay.kbits),
            "kn": raw["kn"].copy().view(np.float16).reshape(-1).astype(np.float64)}
-    if lay.vbits > 0:
+    if lay.vbits == "polar" or lay.vbits > 0:
         out["vidx"] = codes("vc", lay.vbits)
         out["vn"] = raw["vn"].copy().view(np.float16).reshape(-1).astype(np.float64)
     if lay.kqjl:

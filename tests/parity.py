@@ -151,3 +151,47 @@ def check_outputs(gpu_bf16: np.ndarray, orc: np.ndarray, slack: np.ndarray | Non
         raise AssertionError(f"{int(bad.sum())} outputs outside tolerance; max err {float(err.max()):.3e}; "
                              f"(row, col, gpu, oracle, slack): {detail}")
     return float(err.max())
+
+
+def compare_polar(gpu: dict, E: O.PolarEncoded, key: bool):
+    """Polar codes: level-1 and higher-level angle codes bit-exact except
+    where the oracle's angle lies within CODE_MARGIN (unit-vector units) of a
+    bound (then either neighbour, and the vector's reconstruction is exempt);
+    norms as compare_vectors; QJL signs and rho as compare_vectors.  Returns
+    (report, exempt_vector mask)."""
+    c1, ch = gpu["kidx"] if key else gpu["vidx"]
+    norms = gpu["kn"] if key else gpu["vn"]
+    d1, dh = c1 != E.codes1, ch != E.codesh
+    bad = (d1 & ~(E.margin1 < CODE_MARGIN)) | np.zeros_like(d1)
+    badh = dh & ~(E.marginh < CODE_MARGIN)
+    assert not bad.any(), f"{int(bad.sum())} level-1 angle codes differ outside the exemption"
+    assert not badh.any(), f"{int(badh.sum())} higher-level angle codes differ outside the exemption"
+    ok, tie = fp16_match(norms, E.nhat, E.nraw)
+    assert ok.all(), f"{int((~ok).sum())} norms differ"
+    vec_exempt = d1.any(1) | dh.any(1) | tie
+    rep = {"code_exempt": int(d1.sum() + dh.sum()), "norm_tie": int(tie.sum())}
+    if key and E.qjl:
+        okr, rtie = fp16_match(gpu["kr"], E.rho, E.rraw)
+        assert not (~okr & ~vec_exempt).any(), "residual norms differ"
+        sdiff = gpu["ks"] != E.sbits
+        sex = (E.zmargin < SIGN_MARGIN) | vec_exempt[:, None]
+        assert not (sdiff & ~sex).any(), f"{int((sdiff & ~sex).sum())} QJL sign bits differ outside the exemption"
+        vec_exempt = vec_exempt | sdiff.any(1) | ~okr | rtie
+    rep["vectors_exempt"] = int(vec_exempt.sum())
+    return rep, vec_exempt
+
+
+def exempt_slack_polar(Pv, Ev: O.PolarEncoded, exempt: np.ndarray, logits: np.ndarray, lse: np.ndarray,
+                       out: np.ndarray) -> np.ndarray:
+    """exempt_slack for polar-coded values (reconstruction y_hat)."""
+    slack = np.zeros(logits.shape[0])
+    ex = np.flatnonzero(exempt)
+    if ex.size == 0:
+        return slack
+    vmax = np.abs(O.rotate_t(Ev.yhat[ex], Pv.signs, Pv.Rm)).max(1)
+    for r in range(logits.shape[0]):
+        p = np.exp(logits[r, ex] - lse[r])
+        p = np.where(np.isfinite(p), p, 0.0)
+        slack[r] = 2.0 * np.sum(p * (vmax + np.abs(out[r]).max()))
+    return slack
+

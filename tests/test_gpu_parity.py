@@ -25,13 +25,15 @@ DEV = "cuda"
 class Codec:
     """Library and oracle parameters for one cache configuration."""
 
-    def __init__(self, d, kbits, kqjl, vbits, seed, page_tokens=64, H=1):
-        self.desc = tqkv.cache_desc(d, kbits, kqjl, vbits, page_tokens=page_tokens, n_kv_heads=H)
+    def __init__(self, d, kbits, kqjl, vbits, seed, page_tokens=64, H=1, dense=False):
+        lib = lambda b: tqkv.half_bits(b) if b != int(b) else int(b)      # fractional rates: TQ_BITS_HALF | b
+        self.desc = tqkv.cache_desc(d, lib(kbits), kqjl, lib(vbits), page_tokens=page_tokens, n_kv_heads=H)
         self.lay = O.Layout(d, kbits, kqjl, vbits, page_tokens=page_tokens)
-        self.kp = tqkv.make_params(d, kbits, 1000 + seed)
-        self.Pk = O.make_params(d, kbits, 1000 + seed)
-        self.vp = tqkv.make_params(d, vbits, 2000 + seed) if vbits else None
-        self.Pv = O.make_params(d, vbits, 2000 + seed, with_S=False) if vbits else None
+        rot, orot = (tqkv.TQ_ROT_DENSE, "dense") if dense else (tqkv.TQ_ROT_HADAMARD, "hadamard")
+        self.kp = tqkv.make_params(d, lib(kbits), 1000 + seed, rot)
+        self.Pk = O.make_params(d, kbits, 1000 + seed, rotation=orot)
+        self.vp = tqkv.make_params(d, lib(vbits), 2000 + seed, rot) if vbits else None
+        self.Pv = O.make_params(d, vbits, 2000 + seed, with_S=False, rotation=orot) if vbits else None
         self.d, self.kbits, self.kqjl, self.vbits, self.H, self.P = d, kbits, kqjl, vbits, H, page_tokens
 
     def encode(self, K, V, slots, num_blocks):
@@ -517,6 +519,207 @@ def test_decode_step_writes_new_token_and_attends(d, kbits, kqjl, vbits, B, Hq, 
             parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
             parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
             assert np.allclose(f64(lse[b, rows]), lse_ref, rtol=1e-3, atol=1e-3)
+
+
+# ---------------------------------------------------------------------------
+# dense random rotation: every path that rotates (encode, query preparation,
+# the output's inverse rotation), with the tensor-core kernels downstream
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,kbits,kqjl,vbits,Hq,H,L,C", [
+    (128, 2, True, 4, 32, 8, 700, 16),     # k3v4: tensor-core decode; prefill 16 x 4 heads
+    (128, 8, False, 4, 16, 4, 500, 8),     # k8v4
+    (64, 3, True, 3, 8, 2, 300, 4),        # general kernels
+    (256, 4, True, 2, 4, 1, 200, 3),
+])
+def test_dense_rotation_encode_decode_prefill(d, kbits, kqjl, vbits, Hq, H, L, C):
+    P = 64 if d == 128 else 16
+    seed = 500 + d + kbits
+    cd = Codec(d, kbits, kqjl, vbits, seed=seed, page_tokens=P, H=H, dense=True)
+    assert np.array_equal(cd.kp.rotation_matrix().astype(np.float64), cd.Pk.Rm)
+    B = 2
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
+    K = synth.outlier_normal((B * L, H, d), seed=seed + 1, device=DEV)
+    V = synth.outlier_normal((B * L, H, d), seed=seed + 2, device=DEV)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    Q = synth.normal((B, Hq, d), seed=seed + 3, device=DEV)
+    seq = torch.tensor([L, L - 50], dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, logits=logits)
+    Qp = synth.normal((C, Hq, d), seed=seed + 4, device=DEV)
+    out_p = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qp, bt[0].contiguous(), L, cache)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b in range(B):
+        n = int(seq[b])
+        idx = np.arange(b * L, b * L + n)
+        for kvh in range(H):
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl[idx], f64(K[idx, kvh]), f64(V[idx, kvh]), kvh)
+            rows = list(range(kvh * G, kvh * G + G))
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
+            if b == 0:
+                for j in range(C):
+                    nvis = np.full(G, L - C + j + 1, np.int32)
+                    o_p, lse_p, lg_p = O.attend(f64(Qp[j, rows]), cd.Pk, Ek, cd.Pv, Ev, nvis=nvis, want_logits=True)
+                    parity.check_outputs(f64(out_p[j, rows]), o_p, cd.slack(Ev, lg_p, lse_p, o_p))
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_dense_rotation_search(d):
+    n_db, n_q, k = 3000, 130, 10
+    X = synth.unit_normal(n_db, d, seed=60 + d, device=DEV)
+    Qs = synth.unit_normal(n_q, d, seed=61 + d, device=DEV)
+    cd = Codec(d, 4, True, 0, seed=62 + d, H=1, dense=True)
+    cache, flags = cd.encode(X, None, torch.arange(n_db, dtype=torch.int32, device=DEV), -(-n_db // 64))
+    assert flags == 0
+    sc, ix = tqkv.score(cd.kp, cd.desc, cache, n_db, Qs, k)
+    torch.cuda.synchronize()
+    E = O.encode(f64(X), cd.Pk, qjl=True)
+    gpu = O.read_cache(cd.lay, cache_np(cache), np.arange(n_db), 0, 1)
+    _, ex = parity.compare_vectors(gpu, E, key=True, bits=4)
+    for q in range(0, n_q, 13):
+        est = O.estimate(f64(Qs[q]), cd.Pk, E)
+        rms = float(np.sqrt(np.mean(est ** 2)))
+        got = ix[q].cpu().numpy()
+        ok = ~ex[got]
+        assert np.all(np.abs(sc[q].cpu().numpy()[ok] - est[got][ok]) <= 1e-3 * np.maximum(np.abs(est[got][ok]), rms))
+        assert np.all(est[got] >= np.sort(est)[::-1][k - 1] - 2e-3 * rms)
+
+
+# ---------------------------------------------------------------------------
+# fractional rates (b + 1/2 bits per coordinate) through the general kernels
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,kbits,kqjl,vbits,Hq,H,L,P", [
+    (128, 2.5, True, 3.5, 16, 4, 600, 64),     # 3.5-bit keys incl. QJL, 3.5-bit values
+    (128, 1.5, True, 2.5, 8, 2, 400, 16),      # 2.5-bit keys incl. QJL, 2.5-bit values
+    (64, 3.5, False, 1.5, 4, 1, 300, 16),
+    (256, 2.5, True, 2.5, 8, 8, 150, 32),
+    (16, 1.5, False, 3.5, 2, 2, 90, 8),
+])
+def test_fractional_rates_encode_decode_prefill(d, kbits, kqjl, vbits, Hq, H, L, P):
+    seed = 700 + d + int(10 * kbits)
+    cd = Codec(d, kbits, kqjl, vbits, seed=seed, page_tokens=P, H=H)
+    B = 2
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
+    K = synth.outlier_normal((B * L, H, d), seed=seed + 1, device=DEV, dtype=torch.float32)
+    V = synth.outlier_normal((B * L, H, d), seed=seed + 2, device=DEV, dtype=torch.float32)
+    K[3].zero_()
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    Q = synth.normal((B, Hq, d), seed=seed + 3, device=DEV)
+    seq = torch.tensor([L, L - 21], dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, logits=logits)
+    C = 5
+    Qp = synth.normal((C, Hq, d), seed=seed + 4, device=DEV)
+    out_p = tqkv.prefill_attn(cd.kp, cd.vp, cd.desc, Qp, bt[0].contiguous(), L, cache)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b in range(B):
+        n = int(seq[b])
+        idx = np.arange(b * L, b * L + n)
+        for kvh in range(H):
+            Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl[idx], f64(K[idx, kvh]), f64(V[idx, kvh]), kvh)
+            rows = list(range(kvh * G, kvh * G + G))
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
+            if b == 0:
+                for j in range(C):
+                    nvis = np.full(G, L - C + j + 1, np.int32)
+                    o_p, lse_p, lg_p = O.attend(f64(Qp[j, rows]), cd.Pk, Ek, cd.Pv, Ev, nvis=nvis, want_logits=True)
+                    parity.check_outputs(f64(out_p[j, rows]), o_p, cd.slack(Ev, lg_p, lse_p, o_p))
+
+
+@pytest.mark.parametrize("d,rate", [(128, 3.5), (256, 2.5)])
+def test_fractional_rate_search(d, rate):
+    n_db, n_q, k = 2500, 20, 10
+    X = synth.unit_normal(n_db, d, seed=80 + d, device=DEV)
+    Qs = synth.unit_normal(n_q, d, seed=81 + d, device=DEV)
+    cd = Codec(d, rate, True, 0, seed=82 + d, H=1)
+    cache, flags = cd.encode(X, None, torch.arange(n_db, dtype=torch.int32, device=DEV), -(-n_db // 64))
+    assert flags == 0
+    sc, ix = tqkv.score(cd.kp, cd.desc, cache, n_db, Qs, k)
+    torch.cuda.synchronize()
+    E = O.encode(f64(X), cd.Pk, qjl=True)
+    gpu = O.read_cache(cd.lay, cache_np(cache), np.arange(n_db), 0, 1)
+    _, ex = parity.compare_vectors(gpu, E, key=True, bits=rate)
+    for q in range(n_q):
+        est = O.estimate(f64(Qs[q]), cd.Pk, E)
+        rms = float(np.sqrt(np.mean(est ** 2)))
+        got = ix[q].cpu().numpy()
+        ok = ~ex[got]
+        assert np.all(np.abs(sc[q].cpu().numpy()[ok] - est[got][ok]) <= 1e-3 * np.maximum(np.abs(est[got][ok]), rms))
+        assert np.all(est[got] >= np.sort(est)[::-1][k - 1] - 2e-3 * rms)
+
+
+# ---------------------------------------------------------------------------
+# PolarQuant codes (polar-coordinate angle quantizer) through the general kernels
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,kqjl,vpolar,Hq,H,L,P", [
+    (128, True, True, 16, 4, 500, 64),       # polar keys + QJL, polar values
+    (64, False, False, 8, 2, 300, 16),       # polar keys, 4-bit values
+    (256, True, True, 4, 1, 160, 32),
+    (8, True, True, 2, 1, 70, 8),
+])
+def test_polar_codes_encode_decode_prefill(d, kqjl, vpolar, Hq, H, L, P):
+    seed = 900 + d
+    vb = tqkv.TQ_BITS_POLAR if vpolar else 4
+    desc = tqkv.cache_desc(d, tqkv.TQ_BITS_POLAR, kqjl, vb, page_tokens=P, n_kv_heads=H)
+    kp, vp = tqkv.make_params(d, tqkv.TQ_BITS_POLAR, 1000 + seed), tqkv.make_params(d, vb, 2000 + seed)
+    Pk = O.polar_params(d, 1000 + seed)
+    Pv = O.polar_params(d, 2000 + seed, with_S=False) if vpolar else O.make_params(d, 4, 2000 + seed, with_S=False)
+    lay = O.Layout(d, "polar", kqjl, "polar" if vpolar else 4, page_tokens=P)
+    B = 2
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
+    K = synth.outlier_normal((B * L, H, d), seed=seed + 1, device=DEV, dtype=torch.float32)
+    V = synth.outlier_normal((B * L, H, d), seed=seed + 2, device=DEV, dtype=torch.float32)
+    K[5].zero_()
+    cache = tqkv.alloc_cache(desc, nblk)
+    ws = tqkv.encode(kp, vp, desc, K, V, slots, cache)
+    torch.cuda.synchronize()
+    assert tqkv.read_status(ws) == 0
+    Q = synth.normal((B, Hq, d), seed=seed + 3, device=DEV)
+    seq = torch.tensor([L, L - 13], dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    out = tqkv.decode_attn(kp, vp, desc, Q, bt, seq, L, cache, logits=logits)
+    C = 4
+    Qp = synth.normal((C, Hq, d), seed=seed + 4, device=DEV)
+    out_p = tqkv.prefill_attn(kp, vp, desc, Qp, bt[0].contiguous(), L, cache)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b in range(B):
+        n = int(seq[b])
+        idx = np.arange(b * L, b * L + n)
+        for kvh in range(H):
+            gpu = O.read_cache(lay, cn, sl[idx], kvh, H)
+            Ek = O.encode_polar(f64(K[idx, kvh]), Pk, qjl=kqjl)
+            _, exk = parity.compare_polar(gpu, Ek, key=True)
+            if vpolar:
+                Ev = O.encode_polar(f64(V[idx, kvh]), Pv, qjl=False)
+                _, exv = parity.compare_polar(gpu, Ev, key=False)
+                slack = lambda lg, ls, o: parity.exempt_slack_polar(Pv, Ev, exk | exv, lg, ls, o)
+            else:
+                Ev = O.encode(f64(V[idx, kvh]), Pv, qjl=False)
+                _, exv = parity.compare_vectors(gpu, Ev, key=False, bits=4)
+                slack = lambda lg, ls, o: parity.exempt_slack(Pv, Ev, exk | exv, lg, ls, o)
+            rows = list(range(kvh * G, kvh * G + G))
+            o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), Pk, Ek, Pv, Ev, want_logits=True)
+            parity.check_logits(f64(logits[b, rows, :n]), lg_ref, exk)
+            parity.check_outputs(f64(out[b, rows]), o_ref, slack(lg_ref, lse_ref, o_ref))
+            if b == 0:
+                for j in range(C):
+                    nvis = np.full(G, L - C + j + 1, np.int32)
+                    o_p, lse_p, lg_p = O.attend(f64(Qp[j, rows]), Pk, Ek, Pv, Ev, nvis=nvis, want_logits=True)
+                    parity.check_outputs(f64(out_p[j, rows]), o_p, slack(lg_p, lse_p, o_p))
 
 
 def test_decode_wait_timeout_is_flagged_and_context_survives():
