@@ -263,16 +263,24 @@ int tq_decode_step(const tq_params *kp, const tq_params *vp, const tq_cache_desc
  *   device current (cudaGetSymbolAddress) and caches it; make that first call
  *   before any stream capture.
  * - All calls on a device share the array, which keeps the last call's
- *   contents; the status word at its start is cleared on every call (its
- *   flags cannot be read back through this entry point).  Calls whose
- *   execution overlaps on the GPU (different streams, or streams without an
- *   ordering between them) race on the array and give undefined results. */
+ *   contents; the status word at its start is cleared at the start of every
+ *   call and read back by tq_noalloc_read_status.  Calls whose execution
+ *   overlaps on the GPU (different streams, or streams without an ordering
+ *   between them) race on the array and give undefined results. */
 #define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 int tq_decode_attn_noalloc(const tq_params *kp, const tq_params *vp, const tq_cache_desc *desc,
                            const void *Q, int B, int Hq, const int32_t *block_table, int max_blocks,
                            const int32_t *seq_lens, int max_seq_len, const void *cache,
                            int64_t num_blocks, void *out, float *lse, float *logits,
                            int64_t logits_stride, void *stream);
+
+/* The device status word (TQ_DEV_* bits) left by the last
+ * tq_decode_attn_noalloc on the current device, copied to *flags and
+ * cleared, as tq_read_status does for a workspace (a slot or block out of
+ * range, a wait that timed out: results invalid).  Orders after the work on
+ * `stream` and synchronizes it.  Allocates nothing; like the entry point it
+ * follows, it looks up the array's device address on first use. */
+int tq_noalloc_read_status(void *stream, uint32_t *flags);
 
 /* ------------------------------------------------------------------------ */
 /* Chunked prefill over the compressed cache (one sequence)                 */

@@ -59,3 +59,12 @@ extern "C" int tq_decode_attn_noalloc(const tq_params *kp, const tq_params *vp, 
     return tq_decode_attn(kp, vp, desc, Q, B, Hq, block_table, max_blocks, seq_lens, max_seq_len, cache,
                           num_blocks, out, lse, logits, logits_stride, ws, size_t(TQ_NOALLOC_SCRATCH_BYTES), stream);
 }
+
+extern "C" int tq_noalloc_read_status(void *stream, uint32_t *flags) {
+    if (!flags) return TQ_EINVAL;
+    void *ws = nullptr;
+    const int st = scratch_of_current_device(&ws);
+    if (st != TQ_OK) return st;
+    // the status word sits at the start of the static array's header
+    return tq_read_status(ws, stream, flags);
+}

@@ -100,6 +100,7 @@ _sig("tq_score", _i32, [_vp, ctypes.POINTER(CacheDesc), _vp, _i64, _vp, _i32, _i
 _sig("tq_read_status", _i32, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)])
 _sig("tq_status_string", ctypes.c_char_p, [_i32])
 _sig("tq_test_stall_next_decode", _i32, [ctypes.c_uint32])
+_sig("tq_noalloc_read_status", _i32, [_vp, ctypes.POINTER(ctypes.c_uint32)])
 
 
 class TQError(RuntimeError):
@@ -327,6 +328,14 @@ def decode_attn_noalloc(kp: Params, vp: Params, desc: CacheDesc, Q: torch.Tensor
                                        cache.shape[0], _ptr(out), _ptr(lse), _ptr(logits), stride, _stream(stream)),
            "tq_decode_attn_noalloc")
     return out
+
+
+def noalloc_read_status(stream=None) -> int:
+    """tq_noalloc_read_status: status flags of the last no-allocation decode
+    on the current device (cleared by the read)."""
+    flags = ctypes.c_uint32()
+    _check(_lib.tq_noalloc_read_status(_stream(stream), ctypes.byref(flags)), "tq_noalloc_read_status")
+    return int(flags.value)
 
 
 def prefill_workspace_bytes(desc: CacheDesc, C: int, Hq: int, seq_len: int) -> int:

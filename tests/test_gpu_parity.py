@@ -26,14 +26,17 @@ class Codec:
     """Library and oracle parameters for one cache configuration."""
 
     def __init__(self, d, kbits, kqjl, vbits, seed, page_tokens=64, H=1, dense=False):
-        lib = lambda b: tqkv.half_bits(b) if b != int(b) else int(b)      # fractional rates: TQ_BITS_HALF | b
+        # fractional rates: TQ_BITS_HALF | b; "polar": the polar angle codes
+        lib = lambda b: tqkv.TQ_BITS_POLAR if b == "polar" else (tqkv.half_bits(b) if b != int(b) else int(b))
         self.desc = tqkv.cache_desc(d, lib(kbits), kqjl, lib(vbits), page_tokens=page_tokens, n_kv_heads=H)
         self.lay = O.Layout(d, kbits, kqjl, vbits, page_tokens=page_tokens)
         rot, orot = (tqkv.TQ_ROT_DENSE, "dense") if dense else (tqkv.TQ_ROT_HADAMARD, "hadamard")
+        op = lambda b, seed, **kw: (O.polar_params(d, seed, rotation=orot, **kw) if b == "polar"
+                                    else O.make_params(d, b, seed, rotation=orot, **kw))
         self.kp = tqkv.make_params(d, lib(kbits), 1000 + seed, rot)
-        self.Pk = O.make_params(d, kbits, 1000 + seed, rotation=orot)
+        self.Pk = op(kbits, 1000 + seed)
         self.vp = tqkv.make_params(d, lib(vbits), 2000 + seed, rot) if vbits else None
-        self.Pv = O.make_params(d, vbits, 2000 + seed, with_S=False, rotation=orot) if vbits else None
+        self.Pv = op(vbits, 2000 + seed, with_S=False) if vbits else None
         self.d, self.kbits, self.kqjl, self.vbits, self.H, self.P = d, kbits, kqjl, vbits, H, page_tokens
 
     def encode(self, K, V, slots, num_blocks):
@@ -45,18 +48,28 @@ class Codec:
     def check_tokens(self, cache_np, slots_np, Kx, Vx, head):
         """Compare the stored fields of the given tokens of one head."""
         gpu = O.read_cache(self.lay, cache_np, slots_np, head, self.H)
-        Ek = O.encode(Kx, self.Pk, qjl=self.kqjl)
-        repk, exk = parity.compare_vectors(gpu, Ek, key=True, bits=self.kbits)
+        if self.kbits == "polar":
+            Ek = O.encode_polar(Kx, self.Pk, qjl=self.kqjl)
+            repk, exk = parity.compare_polar(gpu, Ek, key=True)
+        else:
+            Ek = O.encode(Kx, self.Pk, qjl=self.kqjl)
+            repk, exk = parity.compare_vectors(gpu, Ek, key=True, bits=self.kbits)
         Ev = repv = None
         self.last_exempt = exk
         if self.vbits:
-            Ev = O.encode(Vx, self.Pv, qjl=False)
-            repv, exv = parity.compare_vectors(gpu, Ev, key=False, bits=self.vbits)
+            if self.vbits == "polar":
+                Ev = O.encode_polar(Vx, self.Pv, qjl=False)
+                repv, exv = parity.compare_polar(gpu, Ev, key=False)
+            else:
+                Ev = O.encode(Vx, self.Pv, qjl=False)
+                repv, exv = parity.compare_vectors(gpu, Ev, key=False, bits=self.vbits)
             self.last_exempt = exk | exv
         return Ek, Ev, exk, repk, repv
 
     def slack(self, Ev, logits, lse, out):
         """Per-row output allowance from the keys exempt in the last check."""
+        if self.vbits == "polar":
+            return parity.exempt_slack_polar(self.Pv, Ev, self.last_exempt, logits, lse, out)
         return parity.exempt_slack(self.Pv, Ev, self.last_exempt, logits, lse, out)
 
 
@@ -477,10 +490,12 @@ def test_block_table_out_of_range_is_flagged():
     (128, 8, False, 4, 3, 16, 4, 500),     # k8v4, tensor-core decode
     (128, 3, True, 3, 2, 8, 2, 300),       # 3-bit keys: general decode kernel
     (64, 4, True, 2, 3, 4, 1, 130),        # d = 64, general kernels
+    (128, 2.5, True, 3.5, 2, 8, 2, 200),   # fractional rates
+    (128, "polar", True, "polar", 2, 8, 4, 150),   # polar codes
 ])
 def test_decode_step_writes_new_token_and_attends(d, kbits, kqjl, vbits, B, Hq, H, L):
     P = 64 if d == 128 else 16
-    seed = 300 + kbits + d
+    seed = 300 + d + (9 if kbits == "polar" else int(2 * kbits))
     cd = Codec(d, kbits, kqjl, vbits, seed=seed, page_tokens=P, H=H)
     bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=seed)
     K = synth.outlier_normal((B, L, H, d), seed=seed + 1, device=DEV)

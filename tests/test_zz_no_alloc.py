@@ -75,3 +75,19 @@ def test_noalloc_rejects_problems_beyond_its_static_scratch():
     with pytest.raises(tqkv.TQError) as e:
         tqkv.decode_attn_noalloc(kp, vp, desc, Q, bt, lens, L, cache)
     assert e.value.code == tqkv.TQ_ESCRATCH
+
+
+def test_noalloc_status_word_reports_a_block_out_of_range():
+    # the no-allocation entry point's flags are readable: a block-table entry
+    # beyond the cache sets TQ_DEV_BLOCK_RANGE; the next clean call reports 0
+    desc, kp, vp, bt, lens, cache, Q = _case(B=2, Hq=8, H=2, L=500, seed=73)
+    good = _run(tqkv.decode_attn_noalloc, desc, kp, vp, bt, lens, cache, Q, 500)
+    assert tqkv.noalloc_read_status() == 0
+    bad = bt.clone()
+    bad[1, 3] = cache.shape[0] + 5
+    _run(tqkv.decode_attn_noalloc, desc, kp, vp, bad, lens, cache, Q, 500)
+    assert tqkv.noalloc_read_status() & tqkv.TQ_DEV_BLOCK_RANGE
+    again = _run(tqkv.decode_attn_noalloc, desc, kp, vp, bt, lens, cache, Q, 500)
+    assert tqkv.noalloc_read_status() == 0
+    _same(again, good)
+
