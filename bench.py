@@ -432,6 +432,12 @@ class PresetPart:
                 Op(f"{self.tag}_decode", fd, self.B * self.Hq * self.L, "(query-head, key) pairs scored", "hbm",
                    self.B * self.H * self.L * self.per_tok, "tq_decode_attn", 3, flush=True, extra=ex)]
 
+    def host_inputs(self):
+        return {"K": self.K, "V": self.V, "Q": self.Q}
+
+    def host_outputs(self):
+        return {"out": self.out}
+
     @classmethod
     def config(cls, batch=8, seq_len=8192, **_):
         return {cls.tag: {"what": f"B={batch} x Hkv=8 x {seq_len} tokens x d=128 bf16, 32 query heads: " + cls.what,

@@ -56,14 +56,18 @@ __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
 constexpr int kPQRows = 32;
 constexpr size_t kPQSmem = sizeof(float) * (128 * 129 + kPQRows * 128);
 
+// blockIdx.y selects which outputs j this block projects: all 128, or (with
+// few rows, so that more blocks share the work) a quarter of them, staging
+// only those rows of S; every block rotates its own rows.
 __global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
     extern __shared__ float pq_smem[];
     float *sT = pq_smem;                        // [k][j], row stride 129 (bank spread)
     float *sq = pq_smem + 128 * 129;            // [32 rows][128]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = int64_t(blockIdx.x) * kPQRows;
-    for (int i = tid; i < 128 * 64; i += 256) {  // S[j][k] bf16 pairs -> sT[k][j]
-        const int j = i >> 6, k2 = (i & 63) * 2;
+    const int jn = 128 / int(gridDim.y), j0 = int(blockIdx.y) * jn;
+    for (int i = tid; i < jn * 64; i += 256) {  // S[j][k] bf16 pairs -> sT[k][j]
+        const int j = j0 + (i >> 6), k2 = (i & 63) * 2;
         const uint32_t pr = *reinterpret_cast<const uint32_t *>(a.kp.S + size_t(j) * 128 + k2);
         sT[k2 * 129 + j] = __uint_as_float(pr << 16);
         sT[(k2 + 1) * 129 + j] = __uint_as_float(pr & 0xFFFF0000u);
@@ -84,11 +88,12 @@ __global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
         for (int e = 0; e < 4; ++e) {
             const float v = x[e] * 0.08838834764831845f;
             sq[rr * 128 + lane * 4 + e] = v;
-            if (row < a.rows) a.qr[row * 128 + lane * 4 + e] = v;
+            if (row < a.rows && blockIdx.y == 0) a.qr[row * 128 + lane * 4 + e] = v;
         }
     }
     __syncthreads();
     const int j = tid & 127, g = tid >> 7;      // output j, rows 16 g .. 16 g + 15
+    if (j < j0 || j >= j0 + jn) return;
     float acc[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) acc[r] = 0.f;
@@ -490,7 +495,24 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
             }
         }
         const int n = min(32, a.n_splits - s0);
-        for (int i = 0; i < n; ++i) {
+        int i = 0;
+        // eight splits' partials are loaded before they are added, so the
+        // loads overlap (long contexts have a hundred or more splits per row)
+        for (; i + 8 <= n; i += 8) {
+            float v[8][E], fi[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                fi[u] = __shfl_sync(kFull, f, i + u);
+                const float *src = a.part_o + pb(s0 + i + u) * D + lane * E;
+#pragma unroll
+                for (int e = 0; e < E; ++e) v[u][e] = (lane < WarpVec<D>::LANES && fi[u] != 0.f) ? src[e] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int e = 0; e < E; ++e) o[e] = fmaf(v[u][e], fi[u], o[e]);
+        }
+        for (; i < n; ++i) {
             const float fi = __shfl_sync(kFull, f, i);
             if (fi == 0.f) continue;
             if (lane < WarpVec<D>::LANES) {
@@ -515,7 +537,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
             for (int e = 0; e < E; ++e) vs[lane * E + e] = o[e];
         }
         __syncwarp();
-        dense_rows<D>(a.vp.RdT, vs, lane, o);
+        dense_cols<D>(a.vp.Rd, vs, lane, o);           // o_i = sum_j R[j][i] (o_r)_j
         if (lane < WarpVec<D>::LANES) {
 #pragma unroll
             for (int e = 0; e < E; ++e) out[lane * E + e] = __float2bfloat16_rn(o[e]);
@@ -620,7 +642,9 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
         cudaError_t e = cudaFuncSetAttribute(prep_proj128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(kPQSmem));
         if (e != cudaSuccess) return e;
-        prep_proj128_kernel<<<unsigned((rows + kPQRows - 1) / kPQRows), 256, kPQSmem, st>>>(pa);
+        const unsigned rblocks = unsigned((rows + kPQRows - 1) / kPQRows);
+        const unsigned jsplit = rblocks < 64 ? 4u : 1u;      // few rows: four blocks per row tile
+        prep_proj128_kernel<<<dim3(rblocks, jsplit), 256, kPQSmem, st>>>(pa);
     } else {
         prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
         if (L.kqjl) {

@@ -181,27 +181,33 @@ __device__ __forceinline__ float h2f_bits(uint16_t b) {
     return __half2float(h);
 }
 
-// z = M v for a dense fp32 matrix M [D][D] (row-major) and a vector v held
-// in shared memory, lane l producing outputs [l E, l E + E) (the warp
-// mapping of WarpVec); fp32 products in index order.
+// z = M^T v for a dense fp32 matrix M [D][D] (row-major) and v in shared
+// memory: z_j = sum_i M[i][j] v_i, lane l producing outputs [l E, l E + E).
+// Row i is read as one coalesced run across the warp (lane l takes its E
+// entries), v_i is a shared-memory broadcast.
 template <int D>
-__device__ __forceinline__ void dense_rows(const float *M, const float *vs, int lane, float (&z)[WarpVec<D>::E]) {
+__device__ __forceinline__ void dense_cols(const float *M, const float *vs, int lane, float (&z)[WarpVec<D>::E]) {
     constexpr int E = WarpVec<D>::E;
 #pragma unroll
     for (int e = 0; e < E; ++e) z[e] = 0.f;
     if (lane >= WarpVec<D>::LANES) return;
+    const float *col = M + lane * E;
+#pragma unroll 4
+    for (int i = 0; i < D; ++i) {
+        const float v = vs[i];
+        if constexpr (E % 4 == 0) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const float4 *row = reinterpret_cast<const float4 *>(M + size_t(lane * E + e) * D);
-        float acc = 0.f;
-        for (int i = 0; i < D / 4; ++i) {
-            const float4 m = row[i];
-            acc = fmaf(m.x, vs[4 * i], acc);
-            acc = fmaf(m.y, vs[4 * i + 1], acc);
-            acc = fmaf(m.z, vs[4 * i + 2], acc);
-            acc = fmaf(m.w, vs[4 * i + 3], acc);
+            for (int c = 0; c < E / 4; ++c) {
+                const float4 m = reinterpret_cast<const float4 *>(col + size_t(i) * D)[c];
+                z[4 * c] = fmaf(m.x, v, z[4 * c]);
+                z[4 * c + 1] = fmaf(m.y, v, z[4 * c + 1]);
+                z[4 * c + 2] = fmaf(m.z, v, z[4 * c + 2]);
+                z[4 * c + 3] = fmaf(m.w, v, z[4 * c + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) z[e] = fmaf(col[size_t(i) * D + e], v, z[e]);
         }
-        z[e] = acc;
     }
 }
 
@@ -217,7 +223,7 @@ __device__ __forceinline__ void rotate_warp(const DevParams &P, float (&x)[WarpV
             for (int e = 0; e < E; ++e) wbuf[lane * E + e] = x[e];
         }
         __syncwarp();
-        dense_rows<D>(P.Rd, wbuf, lane, x);
+        dense_cols<D>(P.RdT, wbuf, lane, x);           // y_j = sum_i R[j][i] x_i = sum_i R^T[i][j] x_i
         __syncwarp();
         return;
     }

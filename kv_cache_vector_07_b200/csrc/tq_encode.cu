@@ -16,7 +16,11 @@
 // split into fp16 hi + lo against the fp16 copy of S, 22 bits of r, so every
 // z_j whose sign could differ from the exact product's lies within 2^-22
 // ||r|| ||S_j|| of zero; the epilogue packs sign bits straight into the page.
+#include <cstring>
+
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp8.h>
 
 #include "tc05.cuh"
@@ -92,7 +96,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 // ---------------------------------------------------------------------------
 struct QjlArgs {
     Layout L;
-    const uint16_t *S16;    // [m][D] fp16 bits, m = D
+    const uint16_t *S16;    // [m][D] fp16 bits (the tile fill when D < 64)
     const float *resid;     // [nK][D], each row scaled by a power of two
     int64_t nK;             // n_tokens * H
     const int32_t *slots;
@@ -103,43 +107,53 @@ struct QjlArgs {
 
 constexpr int kBM = 128;       // vectors per tile (MMA M)
 constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
+constexpr int kQThreads = 256; // two per residual row
 constexpr uint32_t kMaxPolls = 1u << 20;   // about a second of polling, then give up
 
 // z = S r for a tile of 128 residuals against BN projection rows, on the
 // tensor cores.  r (fp32, scaled per row by a power of two) is split into
 // fp16 hi + lo (22 bits; the scale keeps both parts normal) against the
 // fp16 copy of S (exact for |S| >= 2^-14); two MMAs per k-step and per 256
-// output columns, fp32 accumulators in TMEM (BN = 512 fills all of it).  The
-// epilogue packs the sign bits [z_j >= 0] into the page.  The grid runs the
-// N tiles of one residual tile next to each other, so the tile's rows are
-// read from DRAM once and served to the others from L2.
+// output columns, fp32 accumulators in TMEM (BN = 512 fills all of it).
+// Per 64-column chunk: S arrives by TMA (128-byte swizzle, the layout the
+// MMA reads), two threads per residual row convert their halves while the
+// next chunk's residual is already loading into registers, and one thread
+// issues the MMAs.  The epilogue packs the sign bits [z_j >= 0] into the
+// page.  The grid runs the N tiles of one residual tile next to each other,
+// so the tile's rows are read from DRAM once and served to the others from L2.
 template <int D, int BN>
-__global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
+__global__ void __launch_bounds__(kQThreads, 1)
+qjl_gemm_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ QjlArgs a) {
     constexpr int M = D;                                   // projection rows
     constexpr int NK = (D + kBK - 1) / kBK;
-    constexpr int NI = BN < 256 ? BN : 256;                // N of one MMA
+    constexpr int NI = BN < 256 ? BN : 256;                // N of one MMA (and one TMA box)
     constexpr uint32_t TCOLS = BN < 32 ? 32 : BN;
     constexpr int A_BYTES = kBM * 128;                     // one split tile
     constexpr int B_BYTES = BN * 128;
     constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+    constexpr int CW = kBK / 2;                            // columns per thread and chunk
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar[2];
+    __shared__ uint64_t bar_mma[2], bar_b[2];
     __shared__ uint32_t tmem_holder;
     __shared__ int timed_out;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = tid & (kBM - 1), hlf = tid >> 7;
     const int n0 = blockIdx.x * BN;
     const int64_t row0 = int64_t(blockIdx.y) * kBM;
+    const int64_t g = row0 + row;
 
     if (warp == 0) {
         tc05::tmem_alloc(&tmem_holder, TCOLS);
         tc05::tmem_relinquish();
     }
-    if (tid == 0) {
-        tc05::mbar_init(&bar[0], 1);
-        tc05::mbar_init(&bar[1], 1);
+    if (tid == 32) {
+        for (int i = 0; i < 2; ++i) {
+            tc05::mbar_init(&bar_mma[i], 1);
+            tc05::mbar_init(&bar_b[i], 1);
+        }
         tc05::fence_mbar_init();
         timed_out = 0;
     }
@@ -149,72 +163,79 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
     const uint32_t tmem = tmem_holder;
     constexpr uint32_t idesc = tc05::idesc_f16_f32(kBM, NI < 16 ? 16 : NI);
 
+    // this thread's columns [hlf * 32, hlf * 32 + 32) of chunk kc, zero past the data
+    auto load_chunk = [&](int kc, float (&rv)[CW]) {
+        const int c0 = kc * kBK + hlf * CW;
+        if (g < a.nK && c0 + CW <= D) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.resid + g * D + c0);
+#pragma unroll
+            for (int q = 0; q < CW / 4; ++q) {
+                const float4 f = src[q];
+                rv[4 * q] = f.x; rv[4 * q + 1] = f.y; rv[4 * q + 2] = f.z; rv[4 * q + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < CW; ++q) rv[q] = (g < a.nK && c0 + q < D) ? a.resid[g * D + c0 + q] : 0.f;
+        }
+    };
+    float rnext[CW];
+    load_chunk(0, rnext);
+
     for (int kc = 0; kc < NK; ++kc) {
         const int st = kc & 1;
         uint8_t *sA = smem + st * STAGE_BYTES;
         uint8_t *sB = sA + 2 * A_BYTES;
-        if (kc >= 2) {
-            if (!tc05::mbar_wait_bounded(&bar[st], ((kc - 2) >> 1) & 1, kMaxPolls)) timed_out = 1;
-        }
-        // A: row tid of this tile, columns [kc*64, kc*64+64) of r as fp16 hi + lo
-        {
-            const int64_t g = row0 + tid;
-            float rv[kBK];
-            const int c0 = kc * kBK;
-            if (g < a.nK && c0 + kBK <= D) {
-                const float4 *src = reinterpret_cast<const float4 *>(a.resid + g * D + c0);
+        if (kc >= 2 && !tc05::mbar_wait_bounded(&bar_mma[st], ((kc - 2) >> 1) & 1, kMaxPolls)) timed_out = 1;
+        if constexpr (D >= 64) {
+            if (tid == 0) {                                // S rows [n0, n0 + BN), columns of chunk kc
+                tc05::mbar_expect_tx(&bar_b[st], uint32_t(B_BYTES));
 #pragma unroll
-                for (int q = 0; q < kBK / 4; ++q) {
-                    float4 f = src[q];
-                    rv[4 * q] = f.x; rv[4 * q + 1] = f.y; rv[4 * q + 2] = f.z; rv[4 * q + 3] = f.w;
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < kBK; ++q) rv[q] = (g < a.nK && c0 + q < D) ? a.resid[g * D + c0 + q] : 0.f;
+                for (int nb = 0; nb < BN / NI; ++nb)
+                    tc05::tma_load_2d(sB + nb * NI * 128, &tmS, kc * kBK, n0 + nb * NI, &bar_b[st]);
             }
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float x0 = rv[ch * 8 + 2 * k], x1 = rv[ch * 8 + 2 * k + 1];
-                    const __half2 h = __floats2half2_rn(x0, x1);
-                    const float2 hf = __half22float2(h);
-                    const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-                    hi[k] = *reinterpret_cast<const uint32_t *>(&h);
-                    lo[k] = *reinterpret_cast<const uint32_t *>(&l);
-                }
-                const uint32_t o = tc05::sw128_offset(tid, ch);
-                *reinterpret_cast<uint4 *>(sA + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sA + A_BYTES + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-        }
-        // B: BN rows of S (fp16), same 64 columns
-        for (int q = tid; q < BN * 8; q += 128) {
-            const int row = q >> 3, ch = q & 7;
-            const int j = n0 + row, c = kc * kBK + ch * 8;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (j < M && c + 8 <= D) {
-                val = *reinterpret_cast<const uint4 *>(a.S16 + size_t(j) * D + c);
-            } else if (j < M && c < D) {
+        } else {
+            // rows of fewer than 64 columns: the threads fill the swizzled tile, zero-padded
+            for (int q = tid; q < BN * 8; q += kQThreads) {
+                const int r = q >> 3, ch = q & 7;
+                const int j = n0 + r, c = ch * 8;
                 uint16_t tmp[8];
 #pragma unroll
-                for (int z = 0; z < 8; ++z) tmp[z] = (c + z < D) ? a.S16[size_t(j) * D + c + z] : 0;
-                val = make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
-                                 tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
+                for (int z = 0; z < 8; ++z) tmp[z] = (j < M && c + z < D) ? a.S16[size_t(j) * D + c + z] : 0;
+                *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(r), uint32_t(ch))) =
+                    make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
+                               tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
             }
-            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(row, ch)) = val;
+        }
+        float rv[CW];
+#pragma unroll
+        for (int q = 0; q < CW; ++q) rv[q] = rnext[q];
+        if (kc + 1 < NK) load_chunk(kc + 1, rnext);       // in flight while this chunk is converted
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {                   // four 16-byte pieces of hi and of lo
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float x0 = rv[ch * 8 + 2 * k], x1 = rv[ch * 8 + 2 * k + 1];
+                const __half2 h = __floats2half2_rn(x0, x1);
+                const float2 hf = __half22float2(h);
+                const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+                hi[k] = *reinterpret_cast<const uint32_t *>(&h);
+                lo[k] = *reinterpret_cast<const uint32_t *>(&l);
+            }
+            const uint32_t o = tc05::sw128_offset(uint32_t(row), uint32_t(hlf * 4 + ch));
+            *reinterpret_cast<uint4 *>(sA + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sA + A_BYTES + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
         tc05::fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
+            if (D >= 64 && !tc05::mbar_wait_bounded(&bar_b[st], uint32_t(kc >> 1) & 1u, kMaxPolls)) timed_out = 1;
             tc05::fence_after_sync();
             const uint32_t aBase = tc05::smem_u32(sA), bBase = tc05::smem_u32(sB);
 #pragma unroll
             for (int ks = 0; ks < kBK / 16; ++ks) {
 #pragma unroll
                 for (int nb = 0; nb < BN / NI; ++nb) {
-                    // rows nb*NI .. of the B tile: 8-row groups are 1024 bytes apart
                     const uint64_t bdesc = tc05::desc_kmajor_sw128(bBase + nb * NI * 128 + ks * 32);
 #pragma unroll
                     for (int sp = 0; sp < 2; ++sp) {
@@ -223,38 +244,42 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
                     }
                 }
             }
-            tc05::mma_commit(&bar[st]);
+            tc05::mma_commit(&bar_mma[st]);
         }
     }
-    if (!tc05::mbar_wait_bounded(&bar[(NK - 1) & 1], ((NK - 1) >> 1) & 1, kMaxPolls)) timed_out = 1;
+    if (!tc05::mbar_wait_bounded(&bar_mma[(NK - 1) & 1], ((NK - 1) >> 1) & 1, kMaxPolls)) timed_out = 1;
+    // a chunk's B copy that was issued is always waited for above before its MMA,
+    // so no copy is in flight here
     tc05::fence_after_sync();
 
-    // Epilogue: thread = tile row (vector); TMEM lanes 32*warp .. +31.
-    const int64_t g = row0 + warp * 32 + lane;
-    uint8_t *ks_dst = nullptr;
-    if (g < a.nK) {
-        const int64_t t = g / a.L.H;
-        const int h = int(g - t * a.L.H);
-        const int slot = a.slots[t];
-        if (slot >= 0 && slot < a.num_slots) {
-            uint8_t *page = a.cache + (int64_t(slot / a.L.P) * a.L.H + h) * int64_t(a.L.page_bytes);
-            ks_dst = page + a.L.ks_off + (slot % a.L.P) * a.L.ks_bpt;
+    // Epilogue: warps 0-3, thread = tile row (vector); TMEM lanes 32*warp .. +31.
+    if (warp < 4) {
+        const int64_t ge = row0 + warp * 32 + lane;
+        uint8_t *ks_dst = nullptr;
+        if (ge < a.nK) {
+            const int64_t t = ge / a.L.H;
+            const int h = int(ge - t * a.L.H);
+            const int slot = a.slots[t];
+            if (slot >= 0 && slot < a.num_slots) {
+                uint8_t *page = a.cache + (int64_t(slot / a.L.P) * a.L.H + h) * int64_t(a.L.page_bytes);
+                ks_dst = page + a.L.ks_off + (slot % a.L.P) * a.L.ks_bpt;
+            }
         }
-    }
 #pragma unroll 1
-    for (int c = 0; c < (BN + 31) / 32; ++c) {
-        uint32_t r[32];
-        tc05::tmem_ld_32x32b_x32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c * 32), r);
-        tc05::tmem_wait_ld();
-        uint32_t bits = 0;
+        for (int c = 0; c < (BN + 31) / 32; ++c) {
+            uint32_t r[32];
+            tc05::tmem_ld_32x32b_x32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c * 32), r);
+            tc05::tmem_wait_ld();
+            uint32_t bits = 0;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) bits |= (__uint_as_float(r[k]) >= 0.f ? 1u : 0u) << k;
-        const int j0 = n0 + c * 32;
-        if (ks_dst && !timed_out) {
-            if (M >= 32) {
-                if (j0 < M) reinterpret_cast<uint32_t *>(ks_dst)[j0 >> 5] = bits;
-            } else {
-                for (int b = 0; b < M / 8; ++b) ks_dst[b] = uint8_t(bits >> (8 * b));
+            for (int k = 0; k < 32; ++k) bits |= (__uint_as_float(r[k]) >= 0.f ? 1u : 0u) << k;
+            const int j0 = n0 + c * 32;
+            if (ks_dst && !timed_out) {
+                if (M >= 32) {
+                    if (j0 < M) reinterpret_cast<uint32_t *>(ks_dst)[j0 >> 5] = bits;
+                } else {
+                    for (int b = 0; b < M / 8; ++b) ks_dst[b] = uint8_t(bits >> (8 * b));
+                }
             }
         }
     }
@@ -270,15 +295,44 @@ __global__ void __launch_bounds__(128, 1) qjl_gemm_kernel(QjlArgs a) {
 template <int D>
 constexpr int qjl_bn() { return D >= 512 ? 512 : (D < 16 ? 16 : D); }
 
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D map over S (fp16 [D][D], row-major): boxes of 64 columns x box_rows
+// rows with the 128-byte swizzle; rows past D (D < 16) read as zero.
+bool make_s_map(CUtensorMap *m, const uint16_t *S16, int D, int box_rows) {
+    auto fn = tmap_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(D)};
+    cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+    cuuint32_t box[2] = {cuuint32_t(D < 64 ? D : 64), cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(S16), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, D < 64 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
-int launch_qjl(const QjlArgs &q, cudaStream_t st) {
+int launch_qjl(const QjlArgs &q, const uint16_t *S16, cudaStream_t st) {
     constexpr int BN = qjl_bn<D>();
     constexpr size_t smem = 2 * (2 * kBM * 128 + BN * 128) + 1024;
+    CUtensorMap tm;
+    std::memset(&tm, 0, sizeof(tm));
+    if (D >= 64 && !make_s_map(&tm, S16, D, BN < 256 ? BN : 256)) return cudaErrorInvalidValue;
     auto kern = qjl_gemm_kernel<D, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     dim3 grid(unsigned((D + BN - 1) / BN), unsigned((q.nK + kBM - 1) / kBM));
-    kern<<<grid, 128, smem, st>>>(q);
+    kern<<<grid, kQThreads, smem, st>>>(tm, q);
     return cudaGetLastError();
 }
 
@@ -299,14 +353,14 @@ int launch_encode_d(const EncodeArgs &a, int in_dtype, const tq_params *kp, cuda
     if (a.L.kqjl && a.n_tokens > 0) {
         QjlArgs q;
         q.L = a.L;
-        q.S16 = kp->dev.S16;
         q.resid = a.resid;
+        q.S16 = kp->dev.S16;
         q.nK = a.n_tokens * a.L.H;
         q.slots = a.slots;
         q.num_slots = a.num_slots;
         q.cache = a.cache;
         q.status = a.status;
-        return launch_qjl<D>(q, st);
+        return launch_qjl<D>(q, kp->dev.S16, st);
     }
     return cudaSuccess;
 }

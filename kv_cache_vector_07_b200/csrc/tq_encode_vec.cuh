@@ -21,6 +21,26 @@ __host__ __device__ constexpr int warp_buf_floats() { return D <= 256 ? (3 * D >
 template <int D>
 __host__ __device__ constexpr int codebook_offset() { return D <= 256 ? 2 * D : 0; }
 
+// Sign-magnitude codes and levels of the lane's E coordinates u = x inv for a
+// W-bit codebook staged at tb (2^W - 1 ascending bounds, levels by code at
+// +16): bucket = #{j : t_j <= u} by a binary search with compile-time steps.
+template <int D, int W>
+__device__ __forceinline__ void bucketize_lane(const float (&x)[WarpVec<D>::E], float inv, const float *tb,
+                                               uint32_t (&kap)[WarpVec<D>::E], float (&cval)[WarpVec<D>::E]) {
+    constexpr uint32_t half = 1u << (W - 1);
+#pragma unroll
+    for (int e = 0; e < WarpVec<D>::E; ++e) {
+        const float u = x[e] * inv;
+        uint32_t idx = 0;
+#pragma unroll
+        for (uint32_t step = half; step >= 1; step >>= 1)
+            idx += (tb[idx + step - 1] <= u) ? step : 0u;
+        const uint32_t k = idx < half ? (half | (half - 1u - idx)) : (idx - half);
+        kap[e] = k;
+        cval[e] = tb[16 + k];
+    }
+}
+
 // Store a fractional-rate code (coordinates 0 .. D/2-1 at wa bits, the rest
 // at wb = wa - 1) of one token: the lanes' sign-magnitude codes are staged in
 // shared memory (cb, D bytes of this warp), then each lane assembles whole
@@ -227,14 +247,11 @@ __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevPar
     const float *tb = tbase + (second ? 32 : 0);
     uint32_t kap[E];
     float cval[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const float u = x[e] * inv;
-        uint32_t idx = 0;
-        for (int step = 1 << (wbits - 1); step >= 1; step >>= 1)
-            idx += (tb[idx + step - 1] <= u) ? uint32_t(step) : 0u;
-        kap[e] = kappa_of(idx, wbits);
-        cval[e] = tb[16 + kap[e]];
+    switch (wbits) {                                  // the search unrolled per width
+        case 1: bucketize_lane<D, 1>(x, inv, tb, kap, cval); break;
+        case 2: bucketize_lane<D, 2>(x, inv, tb, kap, cval); break;
+        case 3: bucketize_lane<D, 3>(x, inv, tb, kap, cval); break;
+        default: bucketize_lane<D, 4>(x, inv, tb, kap, cval); break;
     }
     __syncwarp();
     const int code_off = is_v ? L.vc_off : L.kc_off;
