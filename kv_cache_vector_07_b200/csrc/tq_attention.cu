@@ -156,7 +156,7 @@ __device__ __forceinline__ void project_rows(const uint16_t *S, const float *vs,
 template <int D>
 __global__ void __launch_bounds__(256) step_prep_kernel(StepArgs a) {
     constexpr int E = WarpVec<D>::E;
-    __shared__ float svec[8][warp_buf_floats<D>()];
+    __shared__ __align__(16) float svec[8][warp_buf_floats<D>()];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const Layout &L = a.L;
     const int64_t n_enc = int64_t(a.B) * L.H * 2;

@@ -46,7 +46,9 @@ struct EncodeArgs {
 template <int D, typename TIn>
 __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     constexpr int E = WarpVec<D>::E;
-    __shared__ float wbuf[8][warp_buf_floats<D>()];
+    __shared__ __align__(16) float wbuf[8][warp_buf_floats<D>()];
+    // d = 1024: the transpose buffer of encode1024_t
+    __shared__ __align__(16) float tbuf[D == 1024 ? 8 : 1][D == 1024 ? 1024 : 1];
     const int lane = threadIdx.x & 31;
     const Layout &L = a.L;
     const int64_t nvec = a.n_tokens * L.H;
@@ -69,6 +71,18 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         load_vec<D>(reinterpret_cast<const TIn *>(is_v ? a.V : a.K) + v * D, lane, x);
         uint8_t *page = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
         const int pos = slot % L.P;
+        if constexpr (D == 1024) {
+            const int bits = is_v ? L.vbits : L.kbits;
+            if (P.cells && !P.rot && bits <= 4 && !(is_v ? (L.vhalf || L.vpolar) : (L.khalf || L.kpolar))) {
+                float4 *cs = reinterpret_cast<float4 *>(wbuf[threadIdx.x >> 5]);
+                __syncwarp();
+                if (lane < 16) cs[lane] = P.cells[lane];
+                __syncwarp();
+                encode1024_t(L, P, is_v, x, page, pos, lane, tbuf[(threadIdx.x >> 5) & 7], cs,
+                             a.resid ? a.resid + v * D : nullptr);
+                continue;
+            }
+        }
         if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r, wbuf[threadIdx.x >> 5])) {
             // the residual is stored times 2^e with ||r|| 2^e in [2^10, 2^11): the
             // projection's fp16 hi + lo parts then stay normal, and its signs do

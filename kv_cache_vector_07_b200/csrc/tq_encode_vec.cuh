@@ -41,6 +41,23 @@ __device__ __forceinline__ void bucketize_lane(const float (&x)[WarpVec<D>::E], 
     }
 }
 
+// Sign-magnitude code and level of one coordinate y (u = y inv) from the
+// magnitude cells of DevParams staged at cs: the rank is the cell's count
+// plus [x >= its threshold], x = cellC |u| (xs = cellC inv).  -0.0 counts as
+// non-negative; a magnitude exactly on a threshold takes the upper rank.
+__device__ __forceinline__ uint32_t cell_code(float y, float xs, const float4 *cs, int bits, float &level) {
+    const uint32_t s = __float_as_uint(y + 0.0f) >> 31;
+    const float x = fabsf(y) * xs;
+    // floor(min(x, 15)) from the low mantissa bits of 2^23 + x (round toward zero)
+    const uint32_t c = __float_as_uint(__fadd_rz(fminf(x, 15.0f), 8388608.0f)) & 15u;
+    const float4 e = cs[c];
+    const bool up = x >= e.x;
+    const uint32_t mu = uint32_t(__float_as_int(e.y)) + (up ? 1u : 0u);
+    const float a = up ? e.w : e.z;
+    level = s ? -a : a;
+    return (s << (bits - 1)) | mu;
+}
+
 // Store a fractional-rate code (coordinates 0 .. D/2-1 at wa bits, the rest
 // at wb = wa - 1) of one token: the lanes' sign-magnitude codes are staged in
 // shared memory (cb, D bytes of this warp), then each lane assembles whole
@@ -229,31 +246,42 @@ __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevPar
     }
     // fractional rates: lanes holding coordinates d/2 .. d-1 use the second codebook
     const bool half = is_v ? L.vhalf : L.khalf;
-    const bool second = half && lane >= WarpVec<D>::LANES / 2;
-    const int wbits = half ? (second ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
-    // bucket = #{j : t_j <= u} by a binary search over this lane's codebook,
-    // staged in the warp's buffer (lanes of the second half of a fractional
-    // rate use their own copy): 2^W - 1 ascending bounds, then 2^W levels
-    float *tbase = wbuf + codebook_offset<D>();
-    __syncwarp();
-    for (int j = lane; j < 64; j += 32) {            // both codebooks, by all lanes
-        const int seg = j >> 5, o = j & 31;
-        if (seg == 1 && !half) continue;
-        const int w = half ? (seg ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
-        if (o < (1 << w) - 1) tbase[j] = (seg ? P.bounds2 : P.bounds)[o];
-        else if (o >= 16 && o < 16 + (1 << w)) tbase[j] = (seg ? P.lv2 : P.lv)[o - 16];
-    }
-    __syncwarp();
-    const float *tb = tbase + (second ? 32 : 0);
     uint32_t kap[E];
     float cval[E];
-    switch (wbits) {                                  // the search unrolled per width
-        case 1: bucketize_lane<D, 1>(x, inv, tb, kap, cval); break;
-        case 2: bucketize_lane<D, 2>(x, inv, tb, kap, cval); break;
-        case 3: bucketize_lane<D, 3>(x, inv, tb, kap, cval); break;
-        default: bucketize_lane<D, 4>(x, inv, tb, kap, cval); break;
+    float *tbase = wbuf + codebook_offset<D>();
+    if (P.cells && !half) {
+        // one magnitude-cell lookup per coordinate
+        __syncwarp();
+        if (lane < 16) reinterpret_cast<float4 *>(tbase)[lane] = P.cells[lane];
+        __syncwarp();
+        const float xs = P.cellC * inv;
+#pragma unroll
+        for (int e = 0; e < E; ++e) kap[e] = cell_code(x[e], xs, reinterpret_cast<const float4 *>(tbase), bits, cval[e]);
+        __syncwarp();
+    } else {
+        const bool second = half && lane >= WarpVec<D>::LANES / 2;
+        const int wbits = half ? (second ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
+        // bucket = #{j : t_j <= u} by a binary search over this lane's codebook,
+        // staged in the warp's buffer (lanes of the second half of a fractional
+        // rate use their own copy): 2^W - 1 ascending bounds, then 2^W levels
+        __syncwarp();
+        for (int j = lane; j < 64; j += 32) {            // both codebooks, by all lanes
+            const int seg = j >> 5, o = j & 31;
+            if (seg == 1 && !half) continue;
+            const int w = half ? (seg ? (is_v ? L.vb_bits : L.kb_bits) : (is_v ? L.va_bits : L.ka_bits)) : bits;
+            if (o < (1 << w) - 1) tbase[j] = (seg ? P.bounds2 : P.bounds)[o];
+            else if (o >= 16 && o < 16 + (1 << w)) tbase[j] = (seg ? P.lv2 : P.lv)[o - 16];
+        }
+        __syncwarp();
+        const float *tb = tbase + (second ? 32 : 0);
+        switch (wbits) {                                  // the search unrolled per width
+            case 1: bucketize_lane<D, 1>(x, inv, tb, kap, cval); break;
+            case 2: bucketize_lane<D, 2>(x, inv, tb, kap, cval); break;
+            case 3: bucketize_lane<D, 3>(x, inv, tb, kap, cval); break;
+            default: bucketize_lane<D, 4>(x, inv, tb, kap, cval); break;
+        }
+        __syncwarp();
     }
-    __syncwarp();
     const int code_off = is_v ? L.vc_off : L.kc_off;
     const int code_bpt = is_v ? L.vc_bpt : L.kc_bpt;
     uint8_t *cdst = page + code_off + pos * code_bpt;
@@ -291,6 +319,111 @@ __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevPar
     }
     const float rho = sqrtf(warp_sum(rr));
     if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kr_off + pos * 2) = f2h_bits(rho);
+    return true;
+}
+
+// d = 1024 under H D / 32 with magnitude cells (the general encoder's
+// search-database shape): the same butterflies as fwht_warp, but the five
+// lane-crossing strides run in registers after a transpose through shared
+// memory, so lane l ends with coordinates 32 j + l (j < 32).  Each of the
+// lane's residual stores is then one coalesced 128-byte row of the warp, and
+// the codes return to coordinate order through the same buffer (tbuf: 1024
+// floats of this warp; cs: the staged cells).  Returns whether the residual
+// (times 2^e, ||r|| 2^e in [2^10, 2^11)) was written to resid.
+__device__ __forceinline__ bool encode1024_t(const Layout &L, const DevParams &P, bool is_v, float (&x)[32],
+                                             uint8_t *page, int pos, int lane, float *tbuf, const float4 *cs,
+                                             float *resid) {
+    const int bits = is_v ? L.vbits : L.kbits;
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
+    const float n = sqrtf(warp_sum(ss));
+    {
+        float sg[32];
+        load_vec<1024>(P.signs, lane, sg);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] *= sg[e];
+    }
+    // strides 1 .. 16 (coordinate bits 0 .. 4) inside the lane
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1)
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if ((e & s) == 0) {
+                const float a = x[e], b = x[e + s];
+                x[e] = a + b;
+                x[e + s] = a - b;
+            }
+    // transpose: element e of lane l at row e, column l ^ e (no bank conflicts
+    // either way); afterwards x[j] is coordinate 32 j + lane
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) tbuf[e * 32 + (lane ^ e)] = x[e];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = tbuf[lane * 32 + (j ^ lane)];
+    // strides 32 .. 512 (coordinate bits 5 .. 9), now inside the lane
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1)
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if ((e & s) == 0) {
+                const float a = x[e], b = x[e + s];
+                x[e] = a + b;
+                x[e + s] = a - b;
+            }
+    const float inv = n > 0.f ? 1.0f / n : 0.f;
+    const uint16_t nh = f2h_bits(n);
+    const float nhf = h2f_bits(nh);
+    const float xs = P.cellC * inv;
+    const bool qjl = !is_v && L.kqjl;
+    uint8_t *cb = reinterpret_cast<uint8_t *>(tbuf);
+    float rr = 0.f;
+    __syncwarp();                                     // every lane has read its column
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float y = x[j] * 0.03125f;              // 1 / sqrt(1024)
+        float c;
+        cb[32 * j + lane] = uint8_t(cell_code(y, xs, cs, bits, c));
+        x[j] = fmaf(-nhf, c, y);                      // residual (used for QJL keys only)
+        rr = fmaf(x[j], x[j], rr);
+    }
+    __syncwarp();
+    // codes in coordinate order: lane l packs coordinates [32 l, 32 l + 32)
+    {
+        uint32_t kap[32];
+        const uint4 *src = reinterpret_cast<const uint4 *>(cb + 32 * lane);
+        const uint4 q0 = src[0], q1 = src[1];
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int e = 0; e < 32; ++e) kap[e] = (w[e >> 2] >> (8 * (e & 3))) & 0xFFu;
+        uint8_t *cdst = page + (is_v ? L.vc_off : L.kc_off) + pos * (is_v ? L.vc_bpt : L.kc_bpt);
+        if (bits == 1) {
+            store_fields<1024, 1>(cdst, lane, kap);
+        } else if (bits == 2) {
+            store_fields<1024, 2>(cdst, lane, kap);
+        } else if (bits == 4) {
+            store_fields<1024, 4>(cdst, lane, kap);
+        } else {   // 3 bits: 2-bit magnitude array + 1-bit sign array
+            uint32_t hi[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) { hi[e] = kap[e] >> 2; kap[e] &= 3u; }
+            store_fields<1024, 2>(cdst, lane, kap);
+            store_fields<1024, 1>(page + (is_v ? L.vh_off : L.kh_off) + pos * (is_v ? L.vh_bpt : L.kh_bpt), lane, hi);
+        }
+    }
+    __syncwarp();                                     // the buffer is free again
+    if (lane == 0) *reinterpret_cast<uint16_t *>(page + (is_v ? L.vn_off : L.kn_off) + pos * 2) = nh;
+    if (!qjl) return false;
+    rr = warp_sum(rr);
+    if (lane == 0) *reinterpret_cast<uint16_t *>(page + L.kr_off + pos * 2) = f2h_bits(sqrtf(rr));
+    float sc = 1.f;
+    if (rr > 0.f) {
+        const int ex = ((__float_as_int(sqrtf(rr)) >> 23) & 0xff) - 127;
+        sc = __int_as_float(min(254, max(1, 127 + 10 - ex)) << 23);
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) resid[32 * j + lane] = x[j] * sc;
     return true;
 }
 

@@ -125,6 +125,14 @@ struct DevParams {
     // Rd[j][i] (y = Rd x) and its transpose RdT (x = Rd^T y), fp32.
     int rot;
     const float *Rd, *RdT;
+    // Magnitude cells of a 1- to 4-bit codebook (null for fractional rates,
+    // polar codes, or when the thresholds are too close): with x = cellC |u|
+    // (cellC a power of two, so the scaled thresholds X_k are exact), cell
+    // c = min(floor(x), 15) holds at most one X_k; entry c is {X in the cell
+    // (else 3e38), #{X_k <= c} as int bits, |level| of that rank, |level| of
+    // the next}.  The magnitude rank is #{X_k <= x}.
+    const float4 *cells;
+    float cellC;
 };
 
 // Byte offset of element (row, col) of a 128 x 128 16-bit tile in the

@@ -463,6 +463,42 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
         }
     }
 
+    // magnitude cells (see DevParams::cells) of a single 1- to 4-bit codebook
+    std::vector<float> cells(64, 0.0f);
+    float cellC = 0.0f;
+    if (L && !polar && !(bits & TQ_BITS_HALF) && bits >= 1 && bits <= 4) {
+        const int h = 1 << (bits - 1), nt = h - 1;
+        std::vector<float> pos_t(static_cast<size_t>(nt)), pos_l(static_cast<size_t>(h));
+        for (int k = 0; k < nt; ++k) pos_t[k] = bd0[h + k];          // positive thresholds, ascending
+        for (int k = 0; k < h; ++k) pos_l[k] = lv_code[k];          // |level| by magnitude rank
+        bool ok = nt == 0 || pos_t[0] > 0.0f;
+        float C = 1.0f;
+        if (ok && nt > 0) {
+            for (int i = 0; i < 60 && C * pos_t[nt - 1] >= 15.0f; ++i) C *= 0.5f;
+            for (int i = 0; i < 60 && 2.0f * C * pos_t[nt - 1] < 15.0f; ++i) C *= 2.0f;
+            ok = C * pos_t[nt - 1] < 15.0f;
+            for (int k = 0; ok && k + 1 < nt; ++k) ok = double(C * pos_t[k + 1]) - double(C * pos_t[k]) >= 1.0;
+        }
+        if (ok) {
+            cellC = C;
+            for (int c = 0; c < 16; ++c) {
+                int mlo = 0;
+                float X = 3.0e38f;
+                for (int k = 0; k < nt; ++k) {
+                    const float Xk = C * pos_t[k];
+                    if (Xk <= float(c)) ++mlo;
+                    else if (Xk < float(c + 1)) X = Xk;
+                }
+                float mlo_bits;
+                std::memcpy(&mlo_bits, &mlo, sizeof mlo_bits);
+                cells[4 * c] = X;
+                cells[4 * c + 1] = mlo_bits;
+                cells[4 * c + 2] = pos_l[mlo];
+                cells[4 * c + 3] = pos_l[mlo + 1 < h ? mlo + 1 : mlo];
+            }
+        }
+    }
+
     p->h_R = nullptr;
     std::vector<float> RdT;
     if (dense) {
@@ -495,7 +531,7 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
         const __half h = __float2half_rn(bf16_to_float(S_bits[k]));
         std::memcpy(&S16[k], &h, 2);
     }
-    // one device block: signs | S (bf16) | levels by code | bounds | images | S (fp16) | polar | dense
+    // one device block: signs | S (bf16) | levels by code | bounds | images | S (fp16) | polar | cells | dense
     const size_t off_signs = 0;
     const size_t off_S = 256 * ((sizeof(float) * d + 255) / 256);
     const size_t off_lv = off_S + 256 * ((sizeof(uint16_t) * dd + 255) / 256);
@@ -504,7 +540,8 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
     const size_t off_s16 = off_rot + (imgs ? 32768 : 0);
     const size_t off_S16 = off_s16 + (imgs ? 32768 : 0);
     const size_t off_polar = off_S16 + 256 * ((sizeof(uint16_t) * dd + 255) / 256);
-    const size_t off_R = off_polar + (polar ? 1024 : 0);
+    const size_t off_cells = off_polar + (polar ? 1024 : 0);
+    const size_t off_R = off_cells + 256;
     const size_t off_RT = off_R + (dense ? sizeof(float) * dd : 0);
     const size_t total = off_RT + (dense ? sizeof(float) * dd : 0);
     if (cudaMalloc(&p->d_block, total) != cudaSuccess) { p->d_block = nullptr; tq_free_params(p); return TQ_ENOMEM; }
@@ -517,6 +554,7 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
                   cudaMemcpy(base + off_s16, s16_img.data(), 32768, cudaMemcpyHostToDevice) != cudaSuccess)) ||
         cudaMemcpy(base + off_S16, S16.data(), sizeof(uint16_t) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
         (polar && cudaMemcpy(base + off_polar, polar_tab.data(), 1024, cudaMemcpyHostToDevice) != cudaSuccess) ||
+        cudaMemcpy(base + off_cells, cells.data(), 256, cudaMemcpyHostToDevice) != cudaSuccess ||
         (dense && (cudaMemcpy(base + off_R, Rd.data(), sizeof(float) * dd, cudaMemcpyHostToDevice) != cudaSuccess ||
                    cudaMemcpy(base + off_RT, RdT.data(), sizeof(float) * dd, cudaMemcpyHostToDevice) != cudaSuccess))) {
         tq_free_params(p);
@@ -537,6 +575,8 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
     p->dev.rot = dense ? 1 : 0;
     p->dev.Rd = dense ? reinterpret_cast<const float *>(base + off_R) : nullptr;
     p->dev.RdT = dense ? reinterpret_cast<const float *>(base + off_RT) : nullptr;
+    p->dev.cells = cellC > 0.0f ? reinterpret_cast<const float4 *>(base + off_cells) : nullptr;
+    p->dev.cellC = cellC;
     *out = p;
     return TQ_OK;
 }
