@@ -49,7 +49,8 @@ constexpr uint32_t SM_XR = SM_X + 2 * kTile;       // float [2 groups][2 halves]
 constexpr uint32_t SM_YN = SM_XR + 2048;          // float [2 groups][4 quarters][128] ||Y||^2 partials
 constexpr uint32_t SM_BAR = SM_YN + 4096;         // barriers, TMEM address, level tables
 constexpr uint32_t SM_TAB = SM_BAR + 256;          // magnitude-rank cell tables (keys, values)
-constexpr uint32_t SM_TOTAL = SM_TAB + 2 * 128;
+constexpr uint32_t SM_LV2 = SM_TAB + 4 * 128;        // second-half level tables (fractional rates)
+constexpr uint32_t SM_TOTAL = SM_LV2 + 64;
 constexpr int kCells = 16;                         // cells of a rank table
 constexpr uint32_t kPolls = 1u << 20;    // about a second of polling, then give up
 
@@ -65,9 +66,11 @@ struct RankTable {
 
 struct Enc128Args {
     Layout L;
-    RankTable k_tab, v_tab;
+    RankTable k_tab, v_tab;            // first (or only) codebooks
+    RankTable k_tab2, v_tab2;          // fractional rates: codebooks of coordinates 64 .. 127
     const float *k_lv, *v_lv;          // levels by stored code
     const float *k_bnd, *v_bnd;        // ascending boundaries
+    const float *k_lv2, *v_lv2, *k_bnd2, *v_bnd2;   // fractional rates: second codebooks
     const uint8_t *k_rot, *v_rot, *s16;
     int64_t n_vec, n_tiles;
     const int32_t *slots;
@@ -186,7 +189,10 @@ __device__ __forceinline__ uint8_t *row_page(const Enc128Args &a, int64_t v, int
 // h = (warp%8)/4 (TMEM lane slice warp % 4).  Group g owns TMEM columns
 // [256g, 256g + 128) (Y, then the residual operand) and [256g + 128,
 // 256g + 256) (Z).
-template <int KB, int VB, bool QJL>
+// Fractional rates (KB2 != KB or VB2 != VB): coordinates 64 .. 127, which
+// are exactly the quarters of the threads with h = 1, take the second
+// codebook of KB2 (VB2) bits and the second code arrays of the page.
+template <int KB, int VB, bool QJL, int KB2 = KB, int VB2 = VB>
 __global__ void __launch_bounds__(512, 1)
 encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ Enc128Args a) {
@@ -198,6 +204,8 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     uint64_t *bar_const = bars, *bar_x = bars + 1, *bar_y = bars + 3, *bar_z = bars + 5;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + SM_BAR + 64);
     float *s_klv = reinterpret_cast<float *>(sm + SM_BAR + 128), *s_vlv = s_klv + 16;
+    float *s_klv2 = reinterpret_cast<float *>(sm + SM_LV2), *s_vlv2 = s_klv2 + 8;
+    constexpr bool FRAC_K = KB2 != KB, FRAC_V = VB2 != VB;
 
     constexpr bool DO_V = VB > 0;
     constexpr int PER = DO_V ? 2 : 1;
@@ -221,9 +229,14 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (tid < 16) {
         s_klv[tid] = (KB != 8 && tid < (1 << (KB == 8 ? 1 : KB))) ? a.k_lv[tid] : 0.f;
         s_vlv[tid] = (DO_V && tid < (1 << (VB > 0 ? VB : 1))) ? a.v_lv[tid] : 0.f;
-    } else if (tid < 16 + 2 * kCells) {
+    } else if (tid < 16 + 4 * kCells) {
         const int t = (tid - 16) / kCells, c = (tid - 16) % kCells;
-        reinterpret_cast<float2 *>(sm + SM_TAB)[t * kCells + c] = (t == 0 ? a.k_tab : a.v_tab).cell[c];
+        const RankTable &rt = t == 0 ? a.k_tab : t == 1 ? a.v_tab : t == 2 ? a.k_tab2 : a.v_tab2;
+        reinterpret_cast<float2 *>(sm + SM_TAB)[t * kCells + c] = rt.cell[c];
+    } else if (tid < 16 + 4 * kCells + 16) {
+        const int i = tid - 16 - 4 * kCells;
+        if (i < 8) s_klv2[i] = (FRAC_K && i < (1 << KB2)) ? a.k_lv2[i] : 0.f;
+        else s_vlv2[i - 8] = (FRAC_V && i - 8 < (1 << (VB2 > 0 ? VB2 : 1))) ? a.v_lv2[i - 8] : 0.f;
     }
     auto item_tile = [&](int64_t j) { return first + (j / PER) * stride; };
     auto item_is_v = [&](int64_t j) { return DO_V && (j % PER) == 1; };
@@ -361,22 +374,26 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const float n = ns * rs;                                               // ||x||
         const uint16_t nh = f2h_bits(n);
         const float nhf = h2f_bits(nh);
-        const int bits = is_v ? VB : KB;
+        // this thread's quarters 2h, 2h + 1 use the second codebook of a fractional rate
+        const bool second = h == 1 && (is_v ? FRAC_V : FRAC_K);
+        const int bits = is_v ? (h ? VB2 : VB) : (h ? KB2 : KB);
         // residual scale 2^(12 - e), ||Y|| < 2^(e + 1): |r * scale| < 2^14
         int e = 0;
         if (ns > 0.f) e = ((__float_as_int(ns) >> 23) & 0xff) - 127;
         const float sc = __int_as_float(min(254, max(1, 127 + 12 - e)) << 23);
         float rr = 0.f;
         float T[7];
-        if (!(is_v ? use_table<VB>() : use_table<KB>())) {
+        if (!(is_v ? (h ? use_table<VB2>() : use_table<VB>()) : (h ? use_table<KB2>() : use_table<KB>()))) {
             const int nt = (1 << (bits - 1)) - 1;
-            const float *bnd = is_v ? a.v_bnd : a.k_bnd;
+            const float *bnd = second ? (is_v ? a.v_bnd2 : a.k_bnd2) : (is_v ? a.v_bnd : a.k_bnd);
 #pragma unroll
             for (int k = 0; k < 7; ++k)
                 T[k] = (k < nt && ns > 0.f && !(!is_v && KB == 8)) ? bnd[(1 << (bits - 1)) + k] * ns : FLT_MAX;
         }
-        const float xs = ns > 0.f ? (is_v ? a.v_tab.C : a.k_tab.C) / ns : 0.f;
-        const uint32_t tab = tc05::smem_u32(sm + SM_TAB + (is_v ? kCells * 8 : 0)) - (0x4B000000u << 3);
+        const RankTable &rtab = second ? (is_v ? a.v_tab2 : a.k_tab2) : (is_v ? a.v_tab : a.k_tab);
+        const float xs = ns > 0.f ? rtab.C / ns : 0.f;
+        const uint32_t tab = tc05::smem_u32(sm + SM_TAB + ((is_v ? 1 : 0) + (second ? 2 : 0)) * kCells * 8) -
+                             (0x4B000000u << 3);
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
             const int q = 2 * h + c;
@@ -408,15 +425,38 @@ encode128_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             } else if (is_v) {
                 if constexpr (DO_V) {
                     uint32_t cw[4];
-                    quantize32<DO_V ? VB : 1, false>(y, T, xs, tab, s_vlv, 0.f, cw, rr);
-                    if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
-                                                            a.L.vh_bpt, cw);
+                    bool done = false;
+                    if constexpr (FRAC_V) {
+                        if (second) {
+                            quantize32<VB2, false>(y, T, xs, tab, s_vlv2, 0.f, cw, rr);
+                            if (page) store_codes32<VB2>(page, pos, q - 2, a.L.vc2_off, a.L.vc2_bpt, a.L.vh2_off,
+                                                         a.L.vh2_bpt, cw);
+                            done = true;
+                        }
+                    }
+                    if (!done) {
+                        quantize32<DO_V ? VB : 1, false>(y, T, xs, tab, s_vlv, 0.f, cw, rr);
+                        if (page) store_codes32<DO_V ? VB : 1>(page, pos, q, a.L.vc_off, a.L.vc_bpt, a.L.vh_off,
+                                                                a.L.vh_bpt, cw);
+                    }
                 }
             } else {
                 constexpr int KQ = KB == 8 ? 1 : KB;
                 uint32_t cw[4];
-                quantize32<KQ, QJL>(y, T, xs, tab, s_klv, sq * nhf, cw, rr);
-                if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
+                bool done = false;
+                if constexpr (FRAC_K) {
+                    if (second) {
+                        quantize32<KB2, QJL>(y, T, xs, tab, s_klv2, sq * nhf, cw, rr);
+                        if (page)
+                            store_codes32<KB2>(page, pos, q - 2, a.L.kc2_off, a.L.kc2_bpt, a.L.kh2_off, a.L.kh2_bpt,
+                                               cw);
+                        done = true;
+                    }
+                }
+                if (!done) {
+                    quantize32<KQ, QJL>(y, T, xs, tab, s_klv, sq * nhf, cw, rr);
+                    if (page) store_codes32<KQ>(page, pos, q, a.L.kc_off, a.L.kc_bpt, a.L.kh_off, a.L.kh_bpt, cw);
+                }
                 if constexpr (QJL) {
                     // residual (Y scale) x 2^(12 - e) as fp16 hi + lo over this quarter's Y columns
 #pragma unroll
@@ -502,9 +542,9 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KB, int VB, bool QJL>
+template <int KB, int VB, bool QJL, int KB2 = KB, int VB2 = VB>
 int run(const CUtensorMap &mk, const CUtensorMap &mv, const Enc128Args &a, cudaStream_t st) {
-    auto kern = encode128_kernel<KB, VB, QJL>;
+    auto kern = encode128_kernel<KB, VB, QJL, KB2, VB2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SM_TOTAL));
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -516,14 +556,15 @@ int run(const CUtensorMap &mk, const CUtensorMap &mv, const Enc128Args &a, cudaS
     return cudaGetLastError();
 }
 
-// Rank table of a 3- or 4-bit codebook (see RankTable); false if no power of
-// two puts the largest threshold below the last cell with every gap between
-// scaled thresholds at least one cell wide.
-bool make_rank_table(const tq_params *p, RankTable *t) {
+// Rank table of a 3- or 4-bit codebook (see RankTable) from its ascending
+// boundaries; false if no power of two puts the largest threshold below the
+// last cell with every gap between scaled thresholds at least one cell wide.
+// Other widths need no table (an empty one is returned).
+bool make_rank_table(int bits, const float *bounds, RankTable *t) {
     *t = RankTable{};
-    if (!p || (p->bits != 3 && p->bits != 4)) return true;
-    const int L = 1 << p->bits, nt = L / 2 - 1;
-    const float *th = p->h_bounds + L / 2;         // positive thresholds, ascending
+    if (bits != 3 && bits != 4) return true;
+    const int L = 1 << bits, nt = L / 2 - 1;
+    const float *th = bounds + L / 2;              // positive thresholds, ascending
     if (!(th[0] > 0.f)) return false;
     float C = 1.f;
     for (int i = 0; i < 40 && C * th[nt - 1] >= float(kCells - 1); ++i) C *= 0.5f;
@@ -547,15 +588,30 @@ bool make_rank_table(const tq_params *p, RankTable *t) {
     return true;
 }
 
+// Widths of the two halves of a codebook (equal unless the rate is
+// fractional) and the host boundaries of each.
+struct Halves {
+    int b1, b2;
+    const float *bnd1, *bnd2;
+};
+Halves halves_of(const tq_params *p, bool half, int ka, int kb) {
+    if (!p) return Halves{0, 0, nullptr, nullptr};
+    if (!half) return Halves{p->bits, p->bits, p->h_bounds, p->h_bounds};
+    return Halves{ka, kb, p->h_bounds, p->h_bounds + ((1 << ka) - 1)};
+}
+
 }  // namespace
 
 // Returns -1 if this configuration is not handled by the fused kernel.
 int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, const void *K, const void *V,
                      int64_t n_tokens, const int32_t *slots, uint8_t *cache, int64_t num_blocks, uint8_t *ws,
                      void *stream) {
-    if (L.d != 128 || !kp->dev.rot_img || L.khalf || L.vhalf) return -1;
+    if (L.d != 128 || !kp->dev.rot_img) return -1;
     if (L.vbits > 0 && (!vp || !vp->dev.rot_img)) return -1;
-    const int kb = L.kbits, vb = L.vbits, q = L.kqjl;
+    const int q = L.kqjl;
+    const Halves hk = halves_of(kp, L.khalf, L.ka_bits, L.kb_bits);
+    const Halves hv = halves_of(L.vbits > 0 ? vp : nullptr, L.vhalf, L.va_bits, L.vb_bits);
+    const int kb = hk.b1, kb2 = hk.b2, vb = hv.b1, vb2 = hv.b2;
     Enc128Args a;
     a.L = L;
     a.k_lv = kp->dev.lv;
@@ -565,7 +621,13 @@ int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, 
     a.v_lv = vp ? vp->dev.lv : nullptr;
     a.v_bnd = vp ? vp->dev.bounds : nullptr;
     a.v_rot = vp ? vp->dev.rot_img : nullptr;
-    if (!make_rank_table(kp, &a.k_tab) || !make_rank_table(vb > 0 ? vp : nullptr, &a.v_tab)) return -1;
+    a.k_lv2 = kp->dev.lv2;
+    a.k_bnd2 = kp->dev.bounds2;
+    a.v_lv2 = vp ? vp->dev.lv2 : nullptr;
+    a.v_bnd2 = vp ? vp->dev.bounds2 : nullptr;
+    if (!make_rank_table(kb, hk.bnd1, &a.k_tab) || !make_rank_table(kb2, hk.bnd2, &a.k_tab2) ||
+        !make_rank_table(vb, hv.bnd1, &a.v_tab) || !make_rank_table(vb2, hv.bnd2, &a.v_tab2))
+        return -1;
     a.n_vec = n_tokens * L.H;
     a.n_tiles = (a.n_vec + kRows - 1) / kRows;
     a.slots = slots;
@@ -580,6 +642,15 @@ int launch_encode128(const tq_params *kp, const tq_params *vp, const Layout &L, 
         mv = mk;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (L.khalf || L.vhalf) {
+        // fractional rates (both halves of keys and values): b + 1 bits, then b
+        if (!L.khalf || !L.vhalf || !q) return -1;
+        if (kb == 3 && vb == 4) return run<3, 4, true, 2, 3>(mk, mv, a, st);
+        if (kb == 2 && vb == 3) return run<2, 3, true, 1, 2>(mk, mv, a, st);
+        if (kb == 4 && vb == 4) return run<4, 4, true, 3, 3>(mk, mv, a, st);
+        if (kb == 3 && vb == 3) return run<3, 3, true, 2, 2>(mk, mv, a, st);
+        return -1;
+    }
     if (q) {
         if (kb == 4 && vb == 4) return run<4, 4, true>(mk, mv, a, st);
         if (kb == 2 && vb == 4) return run<2, 4, true>(mk, mv, a, st);

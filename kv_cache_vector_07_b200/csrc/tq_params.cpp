@@ -510,7 +510,7 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
     }
 
     // Operand images for the d = 128 tensor-core encoder (Hadamard rotation only).
-    const bool imgs = d == 128 && !dense && bits != TQ_BITS_POLAR && !(bits & TQ_BITS_HALF);
+    const bool imgs = d == 128 && !dense && bits != TQ_BITS_POLAR;
     std::vector<uint16_t> rot_img, s16_img;
     if (imgs) {
         rot_img.assign(128 * 128, 0);

@@ -767,15 +767,17 @@ def test_decode_wait_timeout_is_flagged_and_context_survives():
 
 
 # ---------------------------------------------------------------------------
-# every configuration of the fused d = 128 bf16 encoder: ragged tail tiles,
-# skipped slots, a zero vector, three KV heads
+# every configuration of the fused d = 128 bf16 encoder (fractional rates
+# included): ragged tail tiles, skipped slots, a zero vector, three KV heads
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("kbits,kqjl,vbits", [(4, True, 4), (2, True, 4), (2, True, 3), (3, True, 3), (3, True, 4),
-                                              (8, False, 4), (4, False, 4), (3, False, 3), (4, True, 0)])
+                                              (8, False, 4), (4, False, 4), (3, False, 3), (4, True, 0),
+                                              (2.5, True, 3.5), (1.5, True, 2.5), (3.5, True, 3.5),
+                                              (2.5, True, 2.5)])
 def test_fused_encoder_configurations(kbits, kqjl, vbits):
     d, H, P = 128, 3, 16
     n = 1000                                  # 3,000 vectors: 23 full tiles and a ragged one
-    cd = Codec(d, kbits, kqjl, vbits, seed=40 + kbits + vbits, page_tokens=P, H=H)
+    cd = Codec(d, kbits, kqjl, vbits, seed=int(40 + 2 * (kbits + vbits)), page_tokens=P, H=H)
     K = synth.lognormal_channels(n, H, d, seed=41, device=DEV)
     V = synth.lognormal_channels(n, H, d, seed=42, device=DEV) if vbits else None
     K[7].zero_()
