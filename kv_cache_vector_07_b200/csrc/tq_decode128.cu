@@ -36,21 +36,42 @@ namespace tq {
 
 namespace {
 
+// Fractional rates (FR): keys of KB bits on coordinates 0 .. 63 and KB - 1
+// on 64 .. 127 (KB in {2, 3}), both halves through fp16 hi + lo pair tables;
+// values of 4 bits, then 3.  K-steps 0 .. 3 cover the first half, 4 .. 7 the
+// second, so no k-step mixes the two codebooks.
+//
 // Page stages: 4-bit-key pages (150 B per token) take two, so that four
 // blocks fit in an SM's shared memory next to the 256-entry pair tables;
 // smaller pages keep three.
-template <int KB>
-__host__ __device__ constexpr int page_stages() { return KB == 4 ? 2 : 3; }
+template <int KB, bool FR = false>
+__host__ __device__ constexpr int page_stages() { return KB == 4 || FR ? 2 : 3; }
 // Key pair-table entries: two 4-bit codes (256), two 2-bit codes (16); FP8
-// keys need no table (each E4M3 byte converts to fp16 exactly).
-template <int KB>
-__host__ __device__ constexpr int key_entries() { return KB == 4 ? 256 : 0; }
+// keys need no table (each E4M3 byte converts to fp16 exactly).  FR: two
+// KB-bit codes (3 bits: two 2-bit magnitudes and two signs, 64), and the
+// second half's two (KB - 1)-bit codes.
+template <int KB, bool FR = false>
+__host__ __device__ constexpr int key_entries() { return FR ? (KB == 3 ? 64 : 16) : (KB == 4 ? 256 : 0); }
+template <int KB, bool FR = false>
+__host__ __device__ constexpr int key_entries2() { return FR ? (KB == 3 ? 16 : 4) : 0; }
 // Query-operand k-steps: 2-bit keys take a sign plane and a sign x magnitude
-// plane (8 each) plus 8 for the QJL signs; 4-bit keys 8 + 8; FP8 keys 8.
-template <int KB>
-__host__ __device__ constexpr int query_ksteps() { return KB == 2 ? 24 : (KB == 4 ? 16 : 8); }
-template <int KB>
-__host__ __device__ constexpr int qjl_kstep0() { return KB == 2 ? 16 : 8; }
+// plane (8 each) plus 8 for the QJL signs; 4-bit (and FR) keys 8 + 8; FP8 keys 8.
+template <int KB, bool FR = false>
+__host__ __device__ constexpr int query_ksteps() { return FR ? 16 : (KB == 2 ? 24 : (KB == 4 ? 16 : 8)); }
+template <int KB, bool FR = false>
+__host__ __device__ constexpr int qjl_kstep0() { return FR ? 8 : (KB == 2 ? 16 : 8); }
+// Levels of the two codes of pair-table entry e for codes of W bits (W = 3:
+// magnitudes at bits 0-1 / 2-3, signs at bits 4 / 5; else W-bit fields).
+template <int W>
+__device__ __forceinline__ void pair_codes_of(int e, int &k0, int &k1) {
+    if constexpr (W == 3) {
+        k0 = (e & 3) | (((e >> 4) & 1) << 2);
+        k1 = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+    } else {
+        k0 = e & ((1 << W) - 1);
+        k1 = (e >> W) & ((1 << W) - 1);
+    }
+}
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
 struct Dec128Args {
@@ -64,6 +85,7 @@ struct Dec128Args {
     int base_len;
     const float *qr, *w;           // [rows][128] from the prep kernel
     const float *k_lv, *v_lv;      // levels by stored code
+    const float *k_lv2, *v_lv2;    // fractional rates: the second codebooks
     float *part_o;                 // [group][split][G][128]
     float *part_ml;                // [group][split][G][2]  (natural-log max, sum)
     float *logits;
@@ -119,6 +141,7 @@ __device__ __forceinline__ int visible(const Dec128Args &a, int b) {
 // l mod copies.
 template <int B>
 __host__ __device__ constexpr int key_copies() { return B == 4 ? 8 : (B == 2 ? 16 : 1); }
+constexpr int kFrKC = 8, kFrKC2 = 16, kFrVC2 = 32;   // FR copies: key tables, value magnitude table
 template <int B>
 __host__ __device__ constexpr int val_copies() { return B == 4 ? 8 : 32; }
 
@@ -139,20 +162,25 @@ __device__ __forceinline__ T lds_at(const void *base, uint32_t byte_off) {
     return *reinterpret_cast<const T *>(reinterpret_cast<const uint8_t *>(base) + byte_off);
 }
 
-template <int KB, int VB, int NT>
+template <int KB, int VB, int NT, bool FR = false>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
-    static_assert(KB == 2 || KB == 4 || KB == 8, "key bits");
+    static_assert(KB == 2 || KB == 4 || KB == 8 || (FR && KB == 3), "key bits");
     static_assert(VB == 3 || VB == 4, "value bits");
+    static_assert(!FR || ((KB == 2 || KB == 3) && VB == 4), "fractional rates: keys 1.5 / 2.5 bits, values 3.5");
     constexpr bool FP8 = KB == 8;                   // E4M3 keys, no QJL part
-    constexpr int kNS = page_stages<KB>();
-    constexpr int KE = key_entries<KB>();           // key pair-table entries (two codes)
+    constexpr int kNS = page_stages<KB, FR>();
+    constexpr int KE = key_entries<KB, FR>();       // key pair-table entries (two codes)
+    constexpr int KE2 = key_entries2<KB, FR>();     // FR: second-half key pair table
     constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
-    constexpr int KC = key_copies<KB>(), VC = val_copies<VB>();
-    constexpr int NKS = query_ksteps<KB>(), QK0 = qjl_kstep0<KB>();
+    constexpr int VE2 = FR ? 16 : 0;                // FR: second-half value magnitude pairs
+    constexpr int KC = FR ? kFrKC : key_copies<KB>(), VC = val_copies<VB>();
+    constexpr int NKS = query_ksteps<KB, FR>(), QK0 = qjl_kstep0<KB, FR>();
     extern __shared__ __align__(16) uint8_t smem[];
     uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][KC copies] {hi pair, lo pair}
-    uint2 *lutV = reinterpret_cast<uint2 *>(lutK + KE * KC);        // [VE][VC copies] {hi pair, lo pair}
-    uint2 *sB = reinterpret_cast<uint2 *>(lutV + VE * VC);          // [NT][NKS][32]
+    uint2 *lutK2 = lutK + KE * KC;                                  // FR: [KE2][kFrKC2]
+    uint2 *lutV = lutK2 + KE2 * kFrKC2;                             // [VE][VC copies] {hi pair, lo pair}
+    uint2 *lutV2 = lutV + VE * VC;                                  // FR: [VE2][kFrVC2]
+    uint2 *sB = lutV2 + VE2 * kFrVC2;                               // [NT][NKS][32]
     uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * NKS * 32);
     const Layout &L = a.L;
     const int pbytes = L.page_bytes;
@@ -180,9 +208,26 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     for (int i = tid; i < KE * KC; i += 128) {
         // centroid pair as fp16 hi + lo (the pair's fp32 values to ~22 bits)
         const int e = i / KC;
-        const float c0 = a.k_lv[e & 15], c1 = a.k_lv[e >> 4];
+        int k0 = e & 15, k1 = e >> 4;
+        if constexpr (FR) pair_codes_of<KB == 8 ? 1 : KB>(e, k0, k1);
+        const float c0 = a.k_lv[k0], c1 = a.k_lv[k1];
         const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
         lutK[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
+    }
+    if constexpr (FR) {
+        for (int i = tid; i < KE2 * kFrKC2; i += 128) {
+            int k0, k1;
+            pair_codes_of<(KB > 1 ? KB - 1 : 1)>(i / kFrKC2, k0, k1);
+            const float c0 = a.k_lv2[k0], c1 = a.k_lv2[k1];
+            const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
+            lutK2[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
+        }
+        for (int i = tid; i < VE2 * kFrVC2; i += 128) {
+            const int e = i / kFrVC2;
+            const float lo = a.v_lv2[e & 3], hi = a.v_lv2[(e >> 2) & 3];   // 3-bit magnitudes
+            const float h0 = __half2float(__float2half_rn(lo)), h1 = __half2float(__float2half_rn(hi));
+            lutV2[i] = make_uint2(h2bits(h0, h1), h2bits(lo - h0, hi - h1));
+        }
     }
     for (int i = tid; i < VE * VC; i += 128) {
         const int e = i / VC;
@@ -200,7 +245,7 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     // (c_1 - c_0)/2 ride on the query operand, scaled by 2^kexp into [0.5, 1)
     // so that their fp16 hi + lo split keeps its precision.
     float plane_f[2] = {1.f, 1.f}, kscale = 1.f;
-    if (KB == 2) {
+    if (KB == 2 && !FR) {
         const float c0 = a.k_lv[0], c1 = a.k_lv[1];
         int e2;
         frexpf(fmaxf(fabsf(c0), fabsf(0.5f * (c1 - c0))), &e2);
@@ -223,6 +268,10 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                 if (ks >= QK0) {
                     const int j = 2 * (ks - QK0);
                     c[0] = 32 * tt + j; c[1] = 32 * tt + j + 16; c[2] = 32 * tt + j + 1; c[3] = 32 * tt + j + 17;
+                } else if (FR) {
+                    // half ks / 4, coordinates 16 (ks % 4) + 4 tt .. + 3 of that half
+                    const int base = 64 * (ks >> 2) + 16 * (ks & 3) + 4 * tt;
+                    c[0] = base; c[1] = base + 1; c[2] = base + 2; c[3] = base + 3;
                 } else if (KB == 2) {
                     // plane k-step kk: word kk / 4 of the thread's 32 coordinates, pair
                     // i0 = 2 (kk % 4): coordinates (i0, i0 + 8) then (i0 + 1, i0 + 9)
@@ -345,7 +394,88 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                 }
             } else {
                 const uint8_t *kcb = pg + L.kc_off;
-                if constexpr (KB == 2) {
+                if constexpr (FR) {
+                    // first half: KB-bit codes of coordinates 0 .. 63 (3 bits: a 2-bit magnitude
+                    // array and a sign array); second half: (KB - 1)-bit codes of 64 .. 127.
+                    // K-step ks covers coordinates 16 (ks % 4) + 4t .. + 3 of half ks / 4: pair
+                    // (4t, 4t + 1) for a0 / a1, (4t + 2, 4t + 3) for a2 / a3.
+                    const int ta = pr + g, tb2 = pr + g + 8;
+                    const uint4 m0 = *reinterpret_cast<const uint4 *>(kcb + ta * L.kc_bpt);
+                    const uint4 m1 = *reinterpret_cast<const uint4 *>(kcb + tb2 * L.kc_bpt);
+                    uint2 h0 = make_uint2(0u, 0u), h1 = make_uint2(0u, 0u);
+                    if constexpr (KB == 3) {
+                        h0 = *reinterpret_cast<const uint2 *>(pg + L.kh_off + ta * L.kh_bpt);
+                        h1 = *reinterpret_cast<const uint2 *>(pg + L.kh_off + tb2 * L.kh_bpt);
+                    }
+                    const uint8_t *kc2 = pg + L.kc2_off;
+                    uint4 n0, n1;                              // second half: 2-bit (16 B) or 1-bit (8 B)
+                    if constexpr (KB == 3) {
+                        n0 = *reinterpret_cast<const uint4 *>(kc2 + ta * L.kc2_bpt);
+                        n1 = *reinterpret_cast<const uint4 *>(kc2 + tb2 * L.kc2_bpt);
+                    } else {
+                        const uint2 x0 = *reinterpret_cast<const uint2 *>(kc2 + ta * L.kc2_bpt);
+                        const uint2 x1 = *reinterpret_cast<const uint2 *>(kc2 + tb2 * L.kc2_bpt);
+                        n0 = make_uint4(x0.x, x0.y, 0u, 0u);
+                        n1 = make_uint4(x1.x, x1.y, 0u, 0u);
+                    }
+                    const uint32_t mw0[4] = {m0.x, m0.y, m0.z, m0.w}, mw1[4] = {m1.x, m1.y, m1.z, m1.w};
+                    const uint32_t hw0[2] = {h0.x, h0.y}, hw1[2] = {h1.x, h1.y};
+                    const uint32_t nw0[4] = {n0.x, n0.y, n0.z, n0.w}, nw1[4] = {n1.x, n1.y, n1.z, n1.w};
+                    // pair-table indices of pairs a0 (low) and a2 (high) of one token
+                    auto idx2 = [&](uint32_t byte, uint32_t &lo, uint32_t &hi) { lo = byte & 15u; hi = byte >> 4; };
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const int kq = ks & 3;
+                        uint32_t i0, i2, j0, j2;                 // tokens g, g + 8
+                        uint2 v[4];
+                        if (ks < 4) {
+                            // 2-bit fields (KB = 3: magnitudes; KB = 2: the codes): byte 4 kq + t
+                            const uint32_t b0 = (mw0[kq] >> (8 * t)) & 0xFFu, b1 = (mw1[kq] >> (8 * t)) & 0xFFu;
+                            idx2(b0, i0, i2);
+                            idx2(b1, j0, j2);
+                            if constexpr (KB == 3) {
+                                // sign bits 16 kq + 4t .. + 3: word kq / 2, bit 16 (kq % 2) + 4t
+                                const int sh = 16 * (kq & 1) + 4 * t;
+                                const uint32_t s0 = (hw0[kq >> 1] >> sh) & 15u, s1 = (hw1[kq >> 1] >> sh) & 15u;
+                                i0 |= (s0 & 3u) << 4; i2 |= (s0 >> 2) << 4;
+                                j0 |= (s1 & 3u) << 4; j2 |= (s1 >> 2) << 4;
+                            }
+                            v[0] = lutK[i0 * KC + (lane & (KC - 1))];
+                            v[2] = lutK[i2 * KC + (lane & (KC - 1))];
+                            v[1] = lutK[j0 * KC + (lane & (KC - 1))];
+                            v[3] = lutK[j2 * KC + (lane & (KC - 1))];
+                        } else {
+                            if constexpr (KB == 3) {
+                                // 2-bit codes: byte 4 kq + t
+                                const uint32_t b0 = (nw0[kq] >> (8 * t)) & 0xFFu, b1 = (nw1[kq] >> (8 * t)) & 0xFFu;
+                                idx2(b0, i0, i2);
+                                idx2(b1, j0, j2);
+                            } else {
+                                // 1-bit codes: bits 16 kq + 4t .. + 3
+                                const int sh = 16 * (kq & 1) + 4 * t;
+                                const uint32_t b0 = (nw0[kq >> 1] >> sh) & 15u, b1 = (nw1[kq >> 1] >> sh) & 15u;
+                                i0 = b0 & 3u; i2 = b0 >> 2;
+                                j0 = b1 & 3u; j2 = b1 >> 2;
+                            }
+                            v[0] = lutK2[i0 * kFrKC2 + (lane & (kFrKC2 - 1))];
+                            v[2] = lutK2[i2 * kFrKC2 + (lane & (kFrKC2 - 1))];
+                            v[1] = lutK2[j0 * kFrKC2 + (lane & (kFrKC2 - 1))];
+                            v[3] = lutK2[j2 * kFrKC2 + (lane & (kFrKC2 - 1))];
+                        }
+                        uint32_t Ah[4], Al[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            Ah[r] = v[r].x;
+                            Al[r] = v[r].y;
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint2 bb = sB[(nt * NKS + ks) * 32 + lane];
+                            mma16816(accM[nt], Ah, bb.x, bb.y);
+                            mma16816(accM[nt], Al, bb.x, bb.y);
+                        }
+                    }
+                } else if constexpr (KB == 2) {
                     // 2-bit codes of tokens g and g + 8 for coordinates [32t, 32t + 32): two words
                     // each; coordinate i of a word sits at bits 2i (magnitude) and 2i + 1 (sign)
                     const uint2 u0 = *reinterpret_cast<const uint2 *>(kcb + (pr + g) * 32 + 8 * t);
@@ -496,7 +626,61 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             // ---------------- values: thread coordinates [16g, 16g + 16), tokens 2t, 2t+1, 2t+8, 2t+9
             {
                 const int ta = pr + 2 * t, tb = ta + 1, tc = ta + 8, td = ta + 9;
-                if (VB == 4) {
+                if constexpr (FR) {
+                    // first half: 4-bit codes of coordinates [8g, 8g + 8), word g of each token's
+                    // first-half array; MMAs 0 .. 3 (rows g / g + 8: coordinates 8g + 2mt, + 1)
+                    const uint8_t *vc = pg + L.vc_off;
+                    const uint32_t wa = *reinterpret_cast<const uint32_t *>(vc + ta * L.vc_bpt + 4 * g);
+                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(vc + tb * L.vc_bpt + 4 * g);
+                    const uint32_t wc = *reinterpret_cast<const uint32_t *>(vc + tc * L.vc_bpt + 4 * g);
+                    const uint32_t wd = *reinterpret_cast<const uint32_t *>(vc + td * L.vc_bpt + 4 * g);
+                    const uint32_t eAB = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);
+                    const uint32_t oAB = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);
+                    const uint32_t eCD = (wc & 0x0F0F0F0Fu) | ((wd << 4) & 0xF0F0F0F0u);
+                    const uint32_t oCD = ((wc >> 4) & 0x0F0F0F0Fu) | (wd & 0xF0F0F0F0u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint2 v[4];
+                        v[0] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(eAB, k, vlane_off));
+                        v[1] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(oAB, k, vlane_off));
+                        v[2] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(eCD, k, vlane_off));
+                        v[3] = lds_at<uint2>(lutV, field_offset<8, VC * 8>(oCD, k, vlane_off));
+                        const uint32_t Ah[4] = {v[0].x, v[1].x, v[2].x, v[3].x};
+                        const uint32_t Al[4] = {v[0].y, v[1].y, v[2].y, v[3].y};
+                        mma16816(O[k], Ah, b0, b1);
+                        mma16816(O[k], Al, b0, b1);
+                    }
+                    // second half: 3-bit codes of coordinates 64 + [8g, 8g + 8): 2-bit magnitudes
+                    // (half-word g) and signs (byte g); MMAs 4 .. 7
+                    const uint8_t *vc2 = pg + L.vc2_off, *vh2 = pg + L.vh2_off;
+                    const uint32_t xa = *reinterpret_cast<const uint16_t *>(vc2 + ta * L.vc2_bpt + 2 * g);
+                    const uint32_t xb = *reinterpret_cast<const uint16_t *>(vc2 + tb * L.vc2_bpt + 2 * g);
+                    const uint32_t xc = *reinterpret_cast<const uint16_t *>(vc2 + tc * L.vc2_bpt + 2 * g);
+                    const uint32_t xd = *reinterpret_cast<const uint16_t *>(vc2 + td * L.vc2_bpt + 2 * g);
+                    const uint32_t zAB = uint32_t(vh2[ta * L.vh2_bpt + g]) | (uint32_t(vh2[tb * L.vh2_bpt + g]) << 16);
+                    const uint32_t zCD = uint32_t(vh2[tc * L.vh2_bpt + g]) | (uint32_t(vh2[td * L.vh2_bpt + g]) << 16);
+                    const uint32_t fAB = (xa & 0x3333u) | ((xb << 2) & 0xCCCCu);
+                    const uint32_t gAB = ((xa >> 2) & 0x3333u) | (xb & 0xCCCCu);
+                    const uint32_t fCD = (xc & 0x3333u) | ((xd << 2) & 0xCCCCu);
+                    const uint32_t gCD = ((xc >> 2) & 0x3333u) | (xd & 0xCCCCu);
+                    const uint32_t v2off = uint32_t(lane & (kFrVC2 - 1)) * 8u;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int e0 = 2 * k, e1 = 2 * k + 1;
+                        const uint32_t z[4] = {(zAB << (15 - e0)) & 0x80008000u, (zAB << (15 - e1)) & 0x80008000u,
+                                               (zCD << (15 - e0)) & 0x80008000u, (zCD << (15 - e1)) & 0x80008000u};
+                        uint2 v[4];
+                        v[0] = lds_at<uint2>(lutV2, field_offset<4, kFrVC2 * 8>(fAB, k, v2off));
+                        v[1] = lds_at<uint2>(lutV2, field_offset<4, kFrVC2 * 8>(gAB, k, v2off));
+                        v[2] = lds_at<uint2>(lutV2, field_offset<4, kFrVC2 * 8>(fCD, k, v2off));
+                        v[3] = lds_at<uint2>(lutV2, field_offset<4, kFrVC2 * 8>(gCD, k, v2off));
+                        uint32_t Ah[4], Al[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) { Ah[r] = v[r].x ^ z[r]; Al[r] = v[r].y ^ z[r]; }
+                        mma16816(O[4 + k], Ah, b0, b1);
+                        mma16816(O[4 + k], Al, b0, b1);
+                    }
+                } else if (VB == 4) {
                     const uint8_t *vc = pg + L.vc_off;
                     const uint2 xa = *reinterpret_cast<const uint2 *>(vc + ta * 64 + 8 * g);
                     const uint2 xb = *reinterpret_cast<const uint2 *>(vc + tb * 64 + 8 * g);
@@ -604,7 +788,8 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     float *ow = oo + warp * (8 * 128);                           // [warp][8 heads][128]
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-        const int c0 = 16 * g + 2 * mt;
+        // FR: MMAs 0 .. 3 hold coordinates 8g + 2mt, + 1; 4 .. 7 the same of the second half
+        const int c0 = FR ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) : 16 * g + 2 * mt;
         ow[(2 * t) * 128 + c0] = O[mt][0] * scale_w[0];
         ow[(2 * t + 1) * 128 + c0] = O[mt][1] * scale_w[1];
         ow[(2 * t) * 128 + c0 + 1] = O[mt][2] * scale_w[0];
@@ -631,15 +816,16 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     if (timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
 }
 
-template <int KB, int VB, int NT>
+template <int KB, int VB, int NT, bool FR = false>
 size_t dec_smem(int page_bytes) {
-    constexpr int KE = key_entries<KB>(), VE = VB == 4 ? 256 : 16;
+    constexpr int KE = key_entries<KB, FR>(), VE = VB == 4 ? 256 : 16;
     // the stage area also holds the final merge: 64 + 4 x 8 x 128 floats
-    constexpr int kNS = page_stages<KB>();
+    constexpr int kNS = page_stages<KB, FR>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
-    return size_t(KE) * key_copies<KB>() * 8 + size_t(VE) * val_copies<VB>() * 8 +
-           size_t(NT) * query_ksteps<KB>() * 32 * 8 +
+    const size_t fr = FR ? size_t(key_entries2<KB, FR>()) * kFrKC2 * 8 + size_t(16) * kFrVC2 * 8 : 0;
+    return size_t(KE) * (FR ? kFrKC : key_copies<KB>()) * 8 + size_t(VE) * val_copies<VB>() * 8 + fr +
+           size_t(NT) * query_ksteps<KB, FR>() * 32 * 8 +
            stages + (2 * kNS + 1) * 8 + kNS * 4 + 4 + 64;
 }
 
@@ -648,13 +834,13 @@ size_t dec_smem(int page_bytes) {
 // (registers, shared memory and the 128-thread block).
 // The kernel only covers d = 128 with 64-token pages, so the page size (and
 // the answer) is fixed per instantiation and computed once.
-template <int KB, int VB, int NT>
+template <int KB, int VB, int NT, bool FR = false>
 int dec_resident(int page_bytes) {
     static std::atomic<int> cached{-1};
     const int c = cached.load();
     if (c >= 0) return c;
-    const size_t smem = dec_smem<KB, VB, NT>(page_bytes);
-    auto kern = dec128_kernel<KB, VB, NT>;
+    const size_t smem = dec_smem<KB, VB, NT, FR>(page_bytes);
+    auto kern = dec128_kernel<KB, VB, NT, FR>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, smem) != cudaSuccess) return 0;
@@ -662,10 +848,10 @@ int dec_resident(int page_bytes) {
     return n;
 }
 
-template <int KB, int VB, int NT>
+template <int KB, int VB, int NT, bool FR = false>
 int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
-    const size_t smem = dec_smem<KB, VB, NT>(a.L.page_bytes);
-    auto kern = dec128_kernel<KB, VB, NT>;
+    const size_t smem = dec_smem<KB, VB, NT, FR>(a.L.page_bytes);
+    auto kern = dec128_kernel<KB, VB, NT, FR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     kern<<<dim3(unsigned(n_groups), unsigned(a.n_splits)), 128, smem, st>>>(a);
@@ -686,12 +872,21 @@ uint32_t take_decode_stall() { return g_decode_stall.exchange(0); }
 bool dec128_keys_ok(const Layout &L) {
     return ((L.kbits == 2 || L.kbits == 4) && L.kqjl) || (L.kbits == 8 && !L.kqjl);
 }
+// Fractional rates the tensor-core decode covers: keys 1.5 / 2.5 bits + QJL,
+// values 3.5 bits.
+bool dec128_frac_ok(const Layout &L) {
+    return L.khalf && L.vhalf && L.kqjl && (L.ka_bits == 2 || L.ka_bits == 3) && L.va_bits == 4;
+}
 
 int dec128_resident(const Layout &L, int G) {
     if (L.d != 128 || L.P != 64 || G > 8) return 0;
-    if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return 0;
     const bool two = G > 4;
     const int pb = L.page_bytes;
+    if (dec128_frac_ok(L)) {
+        if (L.ka_bits == 3) return two ? dec_resident<3, 4, 2, true>(pb) : dec_resident<3, 4, 1, true>(pb);
+        return two ? dec_resident<2, 4, 2, true>(pb) : dec_resident<2, 4, 1, true>(pb);
+    }
+    if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return 0;
 #define TQ_DEC_RES(K, V) \
     if (L.kbits == K && L.vbits == V) return two ? dec_resident<K, V, 2>(pb) : dec_resident<K, V, 1>(pb);
     TQ_DEC_RES(2, 4) TQ_DEC_RES(2, 3) TQ_DEC_RES(4, 4) TQ_DEC_RES(4, 3) TQ_DEC_RES(8, 4) TQ_DEC_RES(8, 3)
@@ -706,7 +901,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   int64_t num_blocks, float *part_o, float *part_ml, float *logits, int64_t logits_stride,
                   uint32_t *status, cudaStream_t st) {
     if (L.d != 128 || L.P != 64 || G > 8) return -1;
-    if (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4)) return -1;
+    const bool frac = dec128_frac_ok(L);
+    if (!frac && (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4))) return -1;
     if (split_len % L.P) return -1;
     Dec128Args a;
     a.L = L;
@@ -725,6 +921,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.w = w;
     a.k_lv = kp->dev.lv;
     a.v_lv = vp->dev.lv;
+    a.k_lv2 = kp->dev.lv2;
+    a.v_lv2 = vp->dev.lv2;
     a.part_o = part_o;
     a.part_ml = part_ml;
     a.logits = logits;
@@ -732,6 +930,11 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.status = status;
     a.stall_polls = take_decode_stall();
     const bool two = G > 4;
+    if (frac) {
+        if (L.ka_bits == 3)
+            return two ? run_dec<3, 4, 2, true>(a, n_groups, st) : run_dec<3, 4, 1, true>(a, n_groups, st);
+        return two ? run_dec<2, 4, 2, true>(a, n_groups, st) : run_dec<2, 4, 1, true>(a, n_groups, st);
+    }
     if (L.kbits == 2 && L.vbits == 4) return two ? run_dec<2, 4, 2>(a, n_groups, st) : run_dec<2, 4, 1>(a, n_groups, st);
     if (L.kbits == 2 && L.vbits == 3) return two ? run_dec<2, 3, 2>(a, n_groups, st) : run_dec<2, 3, 1>(a, n_groups, st);
     if (L.kbits == 4 && L.vbits == 4) return two ? run_dec<4, 4, 2>(a, n_groups, st) : run_dec<4, 4, 1>(a, n_groups, st);
