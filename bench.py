@@ -392,6 +392,8 @@ class PresetPart:
     sequences x 8 KV heads x 8,192 tokens x d=128 bf16 (N(0,1), channels 5
     and 77 x20), 32 query heads."""
     kbits, kqjl, vbits, rotation, tag, what = 2, True, 4, 0, "", ""
+    enc_kernel, enc_launches = "tq_encode (encode_kernel: warp per vector, + qjl_gemm_kernel)", 2
+    dec_kernel = "tq_decode_attn (prep + dec128 tensor-core decode + combine)"
 
     def __init__(self, dev, batch=8, seq_len=8192, **_):
         from kv_cache_vector_07_b200 import synth, tqkv
@@ -428,9 +430,9 @@ class PresetPart:
         ex = {"bytes_per_token_and_head": self.per_tok, "codec": self.what}
         return [Op(f"{self.tag}_encode", fe, 2 * self.n * self.H, "vectors encoded", "hbm",
                    2 * self.n * self.H * self.d * 2 + self.n * self.H * self.per_tok,
-                   "tq_encode (general encoder: warp per vector)", 2 if self.kqjl else 1, flush=True, extra=ex),
+                   self.enc_kernel, self.enc_launches, flush=True, extra=ex),
                 Op(f"{self.tag}_decode", fd, self.B * self.Hq * self.L, "(query-head, key) pairs scored", "hbm",
-                   self.B * self.H * self.L * self.per_tok, "tq_decode_attn", 3, flush=True, extra=ex)]
+                   self.B * self.H * self.L * self.per_tok, self.dec_kernel, 3, flush=True, extra=ex)]
 
     def host_inputs(self):
         return {"K": self.K, "V": self.V, "Q": self.Q}
@@ -446,18 +448,22 @@ class PresetPart:
 
 class DenseRotation(PresetPart):
     kbits, kqjl, vbits, rotation, tag = 2, True, 4, 1, "dense_k3v4"
-    what = "k3v4 under the dense random rotation (encode: dense 128 x 128 product per vector)"
+    what = "k3v4 under the dense random rotation (encode: dense 128 x 128 product, four vectors per warp)"
+    enc_kernel = "tq_encode (encode_dense_kernel: dense rotation of four vectors per warp, + qjl_gemm_kernel)"
 
 
 class Fractional35(PresetPart):
     kbits, kqjl, vbits, rotation, tag = 16 | 2, True, 16 | 3, 0, "frac35"
-    what = "3.5-bit keys incl. QJL (2.5-bit Lloyd-Max + QJL) and 3.5-bit values (fractional rates, general kernels)"
+    what = "3.5-bit keys incl. QJL (2.5-bit Lloyd-Max + QJL) and 3.5-bit values (fractional rates)"
+    enc_kernel, enc_launches = "tq_encode (encode128_kernel: fused, one codebook per coordinate half)", 1
+    dec_kernel = "tq_decode_attn (prep + dec128 fractional-rate decode + combine)"
 
 
 class PolarCodes(PresetPart):
     kbits, kqjl, vbits, rotation, tag = 32, True, 32, 0, "polar"
-    what = ("PolarQuant angle codes (4-bit level-1 angles, 2-bit higher levels) for keys with QJL and for values "
-            "(general kernels)")
+    what = "PolarQuant angle codes (4-bit level-1 angles, 2-bit higher levels) for keys with QJL and for values"
+    enc_kernel = "tq_encode (encode_kernel: warp per vector, polar transform by half-plane tests, + qjl_gemm_kernel)"
+    dec_kernel = "tq_decode_attn (prep + dec128 polar decode, angle tree rebuilt per token + combine)"
 
 
 class LongCtx:

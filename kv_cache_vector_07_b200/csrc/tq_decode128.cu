@@ -86,6 +86,7 @@ struct Dec128Args {
     const float *qr, *w;           // [rows][128] from the prep kernel
     const float *k_lv, *v_lv;      // levels by stored code
     const float *k_lv2, *v_lv2;    // fractional rates: the second codebooks
+    const float *k_pt, *v_pt;      // polar codes: the angle tables (bounds, cos, sin per level)
     float *part_o;                 // [group][split][G][128]
     float *part_ml;                // [group][split][G][2]  (natural-log max, sum)
     float *logits;
@@ -162,26 +163,37 @@ __device__ __forceinline__ T lds_at(const void *base, uint32_t byte_off) {
     return *reinterpret_cast<const T *>(reinterpret_cast<const uint8_t *>(base) + byte_off);
 }
 
-template <int KB, int VB, int NT, bool FR = false>
+// Polar codes (PL, keys with QJL and values, d = 128): the unit-radius
+// reconstruction is rebuilt per token in registers, top down through the
+// angle tree (each radius the parent's times the cos / sin of the parent's
+// angle centre, the same products in the same order as polar_pair), and its
+// fp16 hi + lo pairs are the MMA operands.  Keys as for 4-bit codes (thread
+// t: pairs 16t .. 16t + 15), values as for 4-bit codes (thread g: pairs
+// 8g .. 8g + 7); no pair tables, two 132-float angle tables.
+template <int KB, int VB, int NT, bool FR = false, bool PL = false>
 __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     static_assert(KB == 2 || KB == 4 || KB == 8 || (FR && KB == 3), "key bits");
     static_assert(VB == 3 || VB == 4, "value bits");
     static_assert(!FR || ((KB == 2 || KB == 3) && VB == 4), "fractional rates: keys 1.5 / 2.5 bits, values 3.5");
+    static_assert(!PL || (KB == 4 && VB == 4 && !FR), "polar codes take the 4-bit slots");
     constexpr bool FP8 = KB == 8;                   // E4M3 keys, no QJL part
-    constexpr int kNS = page_stages<KB, FR>();
-    constexpr int KE = key_entries<KB, FR>();       // key pair-table entries (two codes)
+    constexpr int kNS = PL ? 3 : page_stages<KB, FR>();
+    constexpr int KE = PL ? 0 : key_entries<KB, FR>();   // key pair-table entries (two codes)
     constexpr int KE2 = key_entries2<KB, FR>();     // FR: second-half key pair table
-    constexpr int VE = VB == 4 ? 256 : 16;          // value pair-table entries (two codes / magnitudes)
+    constexpr int VE = PL ? 0 : (VB == 4 ? 256 : 16);    // value pair-table entries (two codes / magnitudes)
     constexpr int VE2 = FR ? 16 : 0;                // FR: second-half value magnitude pairs
     constexpr int KC = FR ? kFrKC : key_copies<KB>(), VC = val_copies<VB>();
     constexpr int NKS = query_ksteps<KB, FR>(), QK0 = qjl_kstep0<KB, FR>();
+    constexpr int PT = PL ? 2 * 136 : 0;            // PL: key and value angle tables (floats)
     extern __shared__ __align__(16) uint8_t smem[];
     uint2 *lutK = reinterpret_cast<uint2 *>(smem);                  // [KE][KC copies] {hi pair, lo pair}
     uint2 *lutK2 = lutK + KE * KC;                                  // FR: [KE2][kFrKC2]
     uint2 *lutV = lutK2 + KE2 * kFrKC2;                             // [VE][VC copies] {hi pair, lo pair}
     uint2 *lutV2 = lutV + VE * VC;                                  // FR: [VE2][kFrVC2]
     uint2 *sB = lutV2 + VE2 * kFrVC2;                               // [NT][NKS][32]
-    uint8_t *stage0 = reinterpret_cast<uint8_t *>(sB + NT * NKS * 32);
+    float *ptk = reinterpret_cast<float *>(sB + NT * NKS * 32);     // PL: key angle table, then values'
+    float *ptv = ptk + 136;
+    uint8_t *stage0 = reinterpret_cast<uint8_t *>(ptk + PT);
     const Layout &L = a.L;
     const int pbytes = L.page_bytes;
     const int stage_area = max(kNS * pbytes, (64 + 4 * 8 * 128) * 4);
@@ -213,6 +225,12 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
         const float c0 = a.k_lv[k0], c1 = a.k_lv[k1];
         const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
         lutK[i] = make_uint2(h2bits(h0, h1), h2bits(c0 - h0, c1 - h1));
+    }
+    if constexpr (PL) {
+        for (int i = tid; i < 132; i += 128) {
+            ptk[i] = a.k_pt[i];
+            ptv[i] = a.v_pt[i];
+        }
     }
     if constexpr (FR) {
         for (int i = tid; i < KE2 * kFrKC2; i += 128) {
@@ -394,7 +412,69 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
                 }
             } else {
                 const uint8_t *kcb = pg + L.kc_off;
-                if constexpr (FR) {
+                if constexpr (PL) {
+                    // tokens g, g + 8: radii at the level-2 nodes 8t .. 8t + 7 (the subtree of
+                    // level-5 node t), then per k-step the two pairs 16t + 2ks, + 1
+                    float r2[2][8];
+                    uint32_t c2w[2];                           // level-2 slots 8t .. 8t + 7
+                    uint2 c1w[2];                              // level-1 codes of pairs 16t .. 16t + 15
+#pragma unroll
+                    for (int ri = 0; ri < 2; ++ri) {
+                        const int tok = pr + g + 8 * ri;
+                        c1w[ri] = *reinterpret_cast<const uint2 *>(kcb + tok * L.kc_bpt + 8 * t);
+                        const uint4 hq = *reinterpret_cast<const uint4 *>(pg + L.kc2_off + tok * L.kc2_bpt);
+                        // slot s in word s / 16: levels 7 .. 4 (slots 48 ..) in word 3, level 3 in word 2
+                        auto fld = [](uint32_t w, int sl) { return (w >> (2 * (sl & 15))) & 3u; };
+                        // cos / sin of the centre of a level-l angle code
+                        auto cs = [&](int l, uint32_t k, int child) { return ptk[48 + 12 * (l - 2) + (child ? 8 : 4) + k]; };
+                        const float r6 = cs(7, fld(hq.w, 62), (t >> 1) & 1);
+                        const float r5 = r6 * cs(6, fld(hq.w, 60 + (t >> 1)), t & 1);
+                        const uint32_t k5 = fld(hq.w, 56 + t);
+                        float r3[4];
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const float r4 = r5 * cs(5, k5, j);
+                            const uint32_t k4 = fld(hq.w, 48 + 2 * t + j);
+                            r3[2 * j] = r4 * cs(4, k4, 0);
+                            r3[2 * j + 1] = r4 * cs(4, k4, 1);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t k3 = fld(hq.z, 32 + 4 * t + j);
+                            r2[ri][2 * j] = r3[j] * cs(3, k3, 0);
+                            r2[ri][2 * j + 1] = r3[j] * cs(3, k3, 1);
+                        }
+                        // level-2 slots 8t .. 8t + 7: word t / 2, bits 16 (t % 2) ..
+                        c2w[ri] = ((t >> 1) ? hq.y : hq.x) >> (16 * (t & 1)) & 0xFFFFu;
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t Ah[4], Al[4];
+#pragma unroll
+                        for (int ri = 0; ri < 2; ++ri) {
+                            const uint32_t k2 = (c2w[ri] >> (2 * ks)) & 3u;
+                            const float ra = r2[ri][ks] * ptk[48 + 4 + k2], rb = r2[ri][ks] * ptk[48 + 8 + k2];
+                            // level-1 codes of pairs 16t + 2ks, + 1
+                            const uint32_t cw = ks < 4 ? c1w[ri].x : c1w[ri].y;
+                            const uint32_t ka = (cw >> (8 * (ks & 3))) & 15u, kb = (cw >> (8 * (ks & 3) + 4)) & 15u;
+                            const float y0 = ra * ptk[16 + ka], y1 = ra * ptk[32 + ka];
+                            const float y2 = rb * ptk[16 + kb], y3 = rb * ptk[32 + kb];
+                            const uint32_t h01 = h2bits(y0, y1), h23 = h2bits(y2, y3);
+                            const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&h01));
+                            const float2 f23 = __half22float2(*reinterpret_cast<const __half2 *>(&h23));
+                            Ah[ri] = h01;                              // a0 (row g) / a1 (row g + 8)
+                            Ah[2 + ri] = h23;                          // a2 / a3
+                            Al[ri] = h2bits(y0 - f01.x, y1 - f01.y);
+                            Al[2 + ri] = h2bits(y2 - f23.x, y3 - f23.y);
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint2 bb = sB[(nt * NKS + ks) * 32 + lane];
+                            mma16816(accM[nt], Ah, bb.x, bb.y);
+                            mma16816(accM[nt], Al, bb.x, bb.y);
+                        }
+                    }
+                } else if constexpr (FR) {
                     // first half: KB-bit codes of coordinates 0 .. 63 (3 bits: a 2-bit magnitude
                     // array and a sign array); second half: (KB - 1)-bit codes of 64 .. 127.
                     // K-step ks covers coordinates 16 (ks % 4) + 4t .. + 3 of half ks / 4: pair
@@ -626,7 +706,58 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
             // ---------------- values: thread coordinates [16g, 16g + 16), tokens 2t, 2t+1, 2t+8, 2t+9
             {
                 const int ta = pr + 2 * t, tb = ta + 1, tc = ta + 8, td = ta + 9;
-                if constexpr (FR) {
+                if constexpr (PL) {
+                    // tokens 2t, 2t + 1, 2t + 8, 2t + 9: radii of pairs 8g .. 8g + 7 (the subtree of
+                    // level-4 node g) as fp16 hi + lo pairs per token, then regrouped per
+                    // coordinate into the V^T fragments
+                    uint32_t ph[4][8], pl[4][8];
+                    const int toks[4] = {ta, tb, tc, td};
+                    auto cs = [&](int l, uint32_t k, int child) { return ptv[48 + 12 * (l - 2) + (child ? 8 : 4) + k]; };
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int tok = toks[u];
+                        const uint32_t c1 = *reinterpret_cast<const uint32_t *>(pg + L.vc_off + tok * L.vc_bpt + 4 * g);
+                        const uint4 hq = *reinterpret_cast<const uint4 *>(pg + L.vc2_off + tok * L.vc2_bpt);
+                        // slots 48 .. 63 (levels 7 .. 4) in word 3, level 3 in word 2, the thread's
+                        // level-2 slots 4g .. 4g + 3 in word g / 4
+                        auto fld = [](uint32_t w, int sl) { return (w >> (2 * (sl & 15))) & 3u; };
+                        const uint32_t w2 = (g >> 2) ? hq.y : hq.x;
+                        const float r6 = cs(7, fld(hq.w, 62), (g >> 2) & 1);
+                        const float r5 = r6 * cs(6, fld(hq.w, 60 + (g >> 2)), (g >> 1) & 1);
+                        const float r4 = r5 * cs(5, fld(hq.w, 56 + (g >> 1)), g & 1);
+                        const uint32_t k4 = fld(hq.w, 48 + g);
+#pragma unroll
+                        for (int c3 = 0; c3 < 2; ++c3) {
+                            const float r3 = r4 * cs(4, k4, c3);
+                            const uint32_t k3 = fld(hq.z, 32 + 2 * g + c3);
+#pragma unroll
+                            for (int c2 = 0; c2 < 2; ++c2) {
+                                const float r2 = r3 * cs(3, k3, c2);
+                                const uint32_t k2 = fld(w2, 4 * g + 2 * c3 + c2);
+#pragma unroll
+                                for (int c1b = 0; c1b < 2; ++c1b) {
+                                    const int j = 4 * c3 + 2 * c2 + c1b;         // pair 8g + j
+                                    const float r1 = r2 * cs(2, k2, c1b);
+                                    const uint32_t kt = (c1 >> (4 * j)) & 15u;
+                                    const float y0 = r1 * ptv[16 + kt], y1 = r1 * ptv[32 + kt];
+                                    const uint32_t hh = h2bits(y0, y1);
+                                    const float2 hf = __half22float2(*reinterpret_cast<const __half2 *>(&hh));
+                                    ph[u][j] = hh;
+                                    pl[u][j] = h2bits(y0 - hf.x, y1 - hf.y);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {              // pair 8g + mt: coordinates 16g + 2mt, + 1
+                        const uint32_t Ah[4] = {prmt(ph[0][mt], ph[1][mt], 0x5410), prmt(ph[0][mt], ph[1][mt], 0x7632),
+                                                prmt(ph[2][mt], ph[3][mt], 0x5410), prmt(ph[2][mt], ph[3][mt], 0x7632)};
+                        const uint32_t Al[4] = {prmt(pl[0][mt], pl[1][mt], 0x5410), prmt(pl[0][mt], pl[1][mt], 0x7632),
+                                                prmt(pl[2][mt], pl[3][mt], 0x5410), prmt(pl[2][mt], pl[3][mt], 0x7632)};
+                        mma16816(O[mt], Ah, b0, b1);
+                        mma16816(O[mt], Al, b0, b1);
+                    }
+                } else if constexpr (FR) {
                     // first half: 4-bit codes of coordinates [8g, 8g + 8), word g of each token's
                     // first-half array; MMAs 0 .. 3 (rows g / g + 8: coordinates 8g + 2mt, + 1)
                     const uint8_t *vc = pg + L.vc_off;
@@ -816,16 +947,16 @@ __global__ void __launch_bounds__(128) dec128_kernel(Dec128Args a) {
     if (timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
 }
 
-template <int KB, int VB, int NT, bool FR = false>
+template <int KB, int VB, int NT, bool FR = false, bool PL = false>
 size_t dec_smem(int page_bytes) {
-    constexpr int KE = key_entries<KB, FR>(), VE = VB == 4 ? 256 : 16;
+    constexpr int KE = PL ? 0 : key_entries<KB, FR>(), VE = PL ? 0 : (VB == 4 ? 256 : 16);
     // the stage area also holds the final merge: 64 + 4 x 8 x 128 floats
-    constexpr int kNS = page_stages<KB, FR>();
+    constexpr int kNS = PL ? 3 : page_stages<KB, FR>();
     size_t stages = size_t(kNS) * page_bytes;
     if (stages < (64 + 4 * 8 * 128) * 4) stages = (64 + 4 * 8 * 128) * 4;
     const size_t fr = FR ? size_t(key_entries2<KB, FR>()) * kFrKC2 * 8 + size_t(16) * kFrVC2 * 8 : 0;
     return size_t(KE) * (FR ? kFrKC : key_copies<KB>()) * 8 + size_t(VE) * val_copies<VB>() * 8 + fr +
-           size_t(NT) * query_ksteps<KB, FR>() * 32 * 8 +
+           size_t(NT) * query_ksteps<KB, FR>() * 32 * 8 + (PL ? 2 * 136 * 4 : 0) +
            stages + (2 * kNS + 1) * 8 + kNS * 4 + 4 + 64;
 }
 
@@ -834,13 +965,13 @@ size_t dec_smem(int page_bytes) {
 // (registers, shared memory and the 128-thread block).
 // The kernel only covers d = 128 with 64-token pages, so the page size (and
 // the answer) is fixed per instantiation and computed once.
-template <int KB, int VB, int NT, bool FR = false>
+template <int KB, int VB, int NT, bool FR = false, bool PL = false>
 int dec_resident(int page_bytes) {
     static std::atomic<int> cached{-1};
     const int c = cached.load();
     if (c >= 0) return c;
-    const size_t smem = dec_smem<KB, VB, NT, FR>(page_bytes);
-    auto kern = dec128_kernel<KB, VB, NT, FR>;
+    const size_t smem = dec_smem<KB, VB, NT, FR, PL>(page_bytes);
+    auto kern = dec128_kernel<KB, VB, NT, FR, PL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 0;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, smem) != cudaSuccess) return 0;
@@ -848,10 +979,10 @@ int dec_resident(int page_bytes) {
     return n;
 }
 
-template <int KB, int VB, int NT, bool FR = false>
+template <int KB, int VB, int NT, bool FR = false, bool PL = false>
 int run_dec(const Dec128Args &a, int n_groups, cudaStream_t st) {
-    const size_t smem = dec_smem<KB, VB, NT, FR>(a.L.page_bytes);
-    auto kern = dec128_kernel<KB, VB, NT, FR>;
+    const size_t smem = dec_smem<KB, VB, NT, FR, PL>(a.L.page_bytes);
+    auto kern = dec128_kernel<KB, VB, NT, FR, PL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     kern<<<dim3(unsigned(n_groups), unsigned(a.n_splits)), 128, smem, st>>>(a);
@@ -877,11 +1008,15 @@ bool dec128_keys_ok(const Layout &L) {
 bool dec128_frac_ok(const Layout &L) {
     return L.khalf && L.vhalf && L.kqjl && (L.ka_bits == 2 || L.ka_bits == 3) && L.va_bits == 4;
 }
+// Polar codes the tensor-core decode covers: keys with QJL and values.
+bool dec128_polar_ok(const Layout &L) { return L.kpolar && L.vpolar && L.kqjl; }
 
 int dec128_resident(const Layout &L, int G) {
     if (L.d != 128 || L.P != 64 || G > 8) return 0;
     const bool two = G > 4;
     const int pb = L.page_bytes;
+    if (dec128_polar_ok(L))
+        return two ? dec_resident<4, 4, 2, false, true>(pb) : dec_resident<4, 4, 1, false, true>(pb);
     if (dec128_frac_ok(L)) {
         if (L.ka_bits == 3) return two ? dec_resident<3, 4, 2, true>(pb) : dec_resident<3, 4, 1, true>(pb);
         return two ? dec_resident<2, 4, 2, true>(pb) : dec_resident<2, 4, 1, true>(pb);
@@ -901,8 +1036,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
                   int64_t num_blocks, float *part_o, float *part_ml, float *logits, int64_t logits_stride,
                   uint32_t *status, cudaStream_t st) {
     if (L.d != 128 || L.P != 64 || G > 8) return -1;
-    const bool frac = dec128_frac_ok(L);
-    if (!frac && (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4))) return -1;
+    const bool frac = dec128_frac_ok(L), polar = dec128_polar_ok(L);
+    if (!frac && !polar && (!dec128_keys_ok(L) || !(L.vbits == 3 || L.vbits == 4))) return -1;
     if (split_len % L.P) return -1;
     Dec128Args a;
     a.L = L;
@@ -923,6 +1058,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.v_lv = vp->dev.lv;
     a.k_lv2 = kp->dev.lv2;
     a.v_lv2 = vp->dev.lv2;
+    a.k_pt = kp->dev.polar;
+    a.v_pt = vp->dev.polar;
     a.part_o = part_o;
     a.part_ml = part_ml;
     a.logits = logits;
@@ -930,6 +1067,8 @@ int launch_dec128(const tq_params *kp, const tq_params *vp, const Layout &L, con
     a.status = status;
     a.stall_polls = take_decode_stall();
     const bool two = G > 4;
+    if (polar)
+        return two ? run_dec<4, 4, 2, false, true>(a, n_groups, st) : run_dec<4, 4, 1, false, true>(a, n_groups, st);
     if (frac) {
         if (L.ka_bits == 3)
             return two ? run_dec<3, 4, 2, true>(a, n_groups, st) : run_dec<3, 4, 1, true>(a, n_groups, st);

@@ -211,6 +211,40 @@ __device__ __forceinline__ void dense_cols(const float *M, const float *vs, int 
     }
 }
 
+// dense_cols for NV vectors at once (vs: NV x D floats): each row of M is
+// read once for all of them.  The same sums in the same order as dense_cols.
+template <int D, int NV>
+__device__ __forceinline__ void dense_cols_n(const float *M, const float *vs, int lane,
+                                             float (&z)[NV][WarpVec<D>::E]) {
+    constexpr int E = WarpVec<D>::E;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < E; ++e) z[v][e] = 0.f;
+    if (lane >= WarpVec<D>::LANES) return;
+    const float *col = M + lane * E;
+#pragma unroll 2
+    for (int i = 0; i < D; ++i) {
+        float m[E];
+        if constexpr (E % 4 == 0) {
+#pragma unroll
+            for (int c = 0; c < E / 4; ++c) {
+                const float4 q = reinterpret_cast<const float4 *>(col + size_t(i) * D)[c];
+                m[4 * c] = q.x; m[4 * c + 1] = q.y; m[4 * c + 2] = q.z; m[4 * c + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) m[e] = col[size_t(i) * D + e];
+        }
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const float sv = vs[v * D + i];
+#pragma unroll
+            for (int e = 0; e < E; ++e) z[v][e] = fmaf(m[e], sv, z[v][e]);
+        }
+    }
+}
+
 // y = R x for the warp-held vector x (lane mapping of WarpVec): the dense
 // rotation through the shared buffer wbuf (D floats of this warp), else
 // H D / sqrt(D) by sign flip and butterflies.

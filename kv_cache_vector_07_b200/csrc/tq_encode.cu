@@ -43,8 +43,30 @@ struct EncodeArgs {
     int do_v;
 };
 
+// Residual of a QJL key, stored times 2^e with ||r|| 2^e in [2^10, 2^11): the
+// projection's fp16 hi + lo parts then stay normal, and its signs do not
+// depend on a positive scale.
+template <int D>
+__device__ __forceinline__ void store_resid(float *resid, const float (&r)[WarpVec<D>::E], int lane) {
+    constexpr int E = WarpVec<D>::E;
+    float rr = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) rr = fmaf(r[e], r[e], rr);
+    rr = warp_sum(rr);
+    float sc = 1.f;
+    if (rr > 0.f) {
+        const int ex = ((__float_as_int(sqrtf(rr)) >> 23) & 0xff) - 127;
+        sc = __int_as_float(min(254, max(1, 127 + 10 - ex)) << 23);
+    }
+    if (lane < WarpVec<D>::LANES) {
+        float *dst = resid + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) dst[e] = r[e] * sc;
+    }
+}
+
 template <int D, typename TIn>
-__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+__global__ void __launch_bounds__(256, D >= 512 ? 2 : 4) encode_kernel(EncodeArgs a) {
     constexpr int E = WarpVec<D>::E;
     __shared__ __align__(16) float wbuf[8][warp_buf_floats<D>()];
     // d = 1024: the transpose buffer of encode1024_t
@@ -83,24 +105,73 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
                 continue;
             }
         }
-        if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r, wbuf[threadIdx.x >> 5])) {
-            // the residual is stored times 2^e with ||r|| 2^e in [2^10, 2^11): the
-            // projection's fp16 hi + lo parts then stay normal, and its signs do
-            // not depend on a positive scale
-            float rr = 0.f;
+        if (encode_vector_warp<D>(L, P, is_v, x, page, pos, lane, r, wbuf[threadIdx.x >> 5])) store_resid<D>(a.resid + v * D, r, lane);
+    }
+}
+
+// Dense rotations (d <= 256): groups of four vectors of one kind (keys, then
+// values), rotated together so that each row of R^T is read once per group,
+// then quantized one by one.  A kernel of its own so that the others keep
+// their register budget.
+template <int D, typename TIn>
+__global__ void __launch_bounds__(256) encode_dense_kernel(EncodeArgs a) {
+    constexpr int E = WarpVec<D>::E;
+    __shared__ __align__(16) float wbuf[8][dense_buf_floats<D>()];
+    const int lane = threadIdx.x & 31;
+    const Layout &L = a.L;
+    const int64_t nvec = a.n_tokens * L.H;
+    const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    // dense rotations: groups of four vectors of one kind, rotated together so
+    // that each row of R^T is read once per group
+    const int64_t ngk = (nvec + 3) / 4, ng = a.do_v ? 2 * ngk : ngk;
+    float *wb = wbuf[threadIdx.x >> 5];
+    for (int64_t gi = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; gi < ng; gi += nwarps) {
+        const bool is_v = gi >= ngk;
+        const int64_t v0 = (is_v ? gi - ngk : gi) * 4;
+        const DevParams &P = is_v ? a.vp : a.kp;
+        float x[4][E];
+        uint8_t *page[4];
+        int pos[4];
 #pragma unroll
-            for (int e = 0; e < E; ++e) rr = fmaf(r[e], r[e], rr);
-            rr = warp_sum(rr);
-            float sc = 1.f;
-            if (rr > 0.f) {
-                const int ex = ((__float_as_int(sqrtf(rr)) >> 23) & 0xff) - 127;
-                sc = __int_as_float(min(254, max(1, 127 + 10 - ex)) << 23);
+        for (int k = 0; k < 4; ++k) {
+            const int64_t v = v0 + k;
+            page[k] = nullptr;
+            pos[k] = 0;
+            if (v < nvec) {
+                const int64_t t = v / L.H;
+                const int h = int(v - t * L.H);
+                const int slot = a.slots[t];
+                if (slot >= a.num_slots) {
+                    if (lane == 0) atomicOr(a.status, TQ_DEV_SLOT_RANGE);
+                } else if (slot >= 0) {
+                    page[k] = a.cache + (int64_t(slot / L.P) * L.H + h) * int64_t(L.page_bytes);
+                    pos[k] = slot % L.P;
+                }
             }
+            if (page[k]) load_vec<D>(reinterpret_cast<const TIn *>(is_v ? a.V : a.K) + (v0 + k) * D, lane, x[k]);
+            else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[k][e] = 0.f;
+            }
+        }
+        if (P.rot) {
+            __syncwarp();
             if (lane < WarpVec<D>::LANES) {
-                float *dst = a.resid + v * D + lane * E;
 #pragma unroll
-                for (int e = 0; e < E; ++e) dst[e] = r[e] * sc;
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int e = 0; e < E; ++e) wb[k * D + lane * E + e] = x[k][e];
             }
+            __syncwarp();
+            dense_cols_n<D, 4>(P.RdT, wb, lane, x);   // y_j = sum_i R^T[i][j] x_i
+            __syncwarp();
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (!page[k]) continue;
+            float r[E];
+            if (encode_vector_warp<D>(L, P, is_v, x[k], page[k], pos[k], lane, r, wb, P.rot != 0))
+                store_resid<D>(a.resid + (v0 + k) * D, r, lane);
         }
     }
 }
@@ -360,8 +431,18 @@ int launch_encode_d(const EncodeArgs &a, int in_dtype, const tq_params *kp, cuda
     const int64_t cap = int64_t(sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (in_dtype == TQ_DTYPE_BF16) encode_kernel<D, __nv_bfloat16><<<unsigned(blocks), 256, 0, st>>>(a);
-    else encode_kernel<D, float><<<unsigned(blocks), 256, 0, st>>>(a);
+    bool dense = false;
+    if constexpr (D <= 256) dense = a.kp.rot || (a.do_v && a.vp.rot);
+    if (dense) {
+        if constexpr (D <= 256) {
+            if (in_dtype == TQ_DTYPE_BF16) encode_dense_kernel<D, __nv_bfloat16><<<unsigned(blocks), 256, 0, st>>>(a);
+            else encode_dense_kernel<D, float><<<unsigned(blocks), 256, 0, st>>>(a);
+        }
+    } else if (in_dtype == TQ_DTYPE_BF16) {
+        encode_kernel<D, __nv_bfloat16><<<unsigned(blocks), 256, 0, st>>>(a);
+    } else {
+        encode_kernel<D, float><<<unsigned(blocks), 256, 0, st>>>(a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (a.L.kqjl && a.n_tokens > 0) {

@@ -18,6 +18,9 @@ namespace tq {
 // (64 floats at codebook_offset) for d <= 256; the codebooks alone above.
 template <int D>
 __host__ __device__ constexpr int warp_buf_floats() { return D <= 256 ? (3 * D > 2 * D + 64 ? 3 * D : 2 * D + 64) : 64; }
+// The same with room for four vectors staged for a dense rotation.
+template <int D>
+__host__ __device__ constexpr int dense_buf_floats() { return 4 * D > warp_buf_floats<D>() ? 4 * D : warp_buf_floats<D>(); }
 template <int D>
 __host__ __device__ constexpr int codebook_offset() { return D <= 256 ? 2 * D : 0; }
 
@@ -100,8 +103,12 @@ __device__ __forceinline__ void store_half_codes(uint8_t *page, int pos, int lan
 // level through shared memory (wbuf: 3 D floats of this warp: y, two radius
 // buffers, code bytes), angle codes by the bounds of P.polar, the packed
 // arrays, the fp16 norm; then y_hat top down from the centres' cos / sin and
-// r = y - y_hat into r.  Angles from atan2f; an angle within ~1e-7 (relative
-// to the radius it splits) of a bound may take either neighbour.
+// r = y - y_hat into r.  No angle is computed: "angle of (a, b) >= bound t"
+// is the half-plane test b cos t - a sin t >= 0, valid while both angles lie
+// in one half turn (level 1 folds the lower half plane onto the upper one,
+// 8 cells on); a zero pair takes the code of atan2 of its signed zeros.  An
+// angle within ~1e-7 (relative to the radius it splits) of a bound may take
+// either neighbour.
 template <int D>
 __device__ __forceinline__ bool polar_encode_warp(const Layout &L, const DevParams &P, bool is_v,
                                                   const float (&y)[WarpVec<D>::E], float n, uint16_t nh,
@@ -118,13 +125,19 @@ __device__ __forceinline__ bool polar_encode_warp(const Layout &L, const DevPara
         for (int e = 0; e < E; ++e) ys[lane * E + e] = y[e];
     }
     __syncwarp();
-    const float two_pi = 6.283185307179586f;
     for (int p = lane; p < H; p += 32) {
         const float a = ys[2 * p], b = ys[2 * p + 1];
-        float t = atan2f(b, a);
-        if (t < 0.f) t += two_pi;
-        uint32_t k = 0;
-        for (int j = 0; j < 15; ++j) k += tab[j] <= t ? 1u : 0u;
+        uint32_t k;
+        if (a == 0.f && b == 0.f) {
+            k = signbit(a) ? 8u : 0u;                         // atan2 of signed zeros: 0 or pi
+        } else {
+            const bool flip = b < 0.f || (b == 0.f && a < 0.f);   // angle in [pi, 2 pi)
+            const float a2 = flip ? -a : a, b2 = flip ? -b : b;
+            uint32_t c = 0;
+#pragma unroll
+            for (int j = 0; j < 7; ++j) c += fmaf(b2, tab[136 + 2 * j], -a2 * tab[137 + 2 * j]) >= 0.f ? 1u : 0u;
+            k = flip ? 8u + c : c;
+        }
         cb[p] = uint8_t(k);
         ra[p] = sqrtf(a * a + b * b);
     }
@@ -132,12 +145,14 @@ __device__ __forceinline__ bool polar_encode_warp(const Layout &L, const DevPara
     float *src = ra, *dst = rb;
     int slot = 0;
     for (int l = 2, nodes = H / 2; nodes >= 1; ++l, nodes >>= 1) {
-        const float *tl = tab + 48 + 12 * (l - 2);
+        const float *tcs = tab + 152 + 6 * (l - 2);
         for (int i = lane; i < nodes; i += 32) {
-            const float a = src[2 * i], b = src[2 * i + 1];
-            const float psi = atan2f(b, a);
+            const float a = src[2 * i], b = src[2 * i + 1];    // radii: the angle lies in [0, pi/2]
             uint32_t k = 0;
-            for (int j = 0; j < 3; ++j) k += tl[j] <= psi ? 1u : 0u;
+            if (a != 0.f || b != 0.f) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j) k += fmaf(b, tcs[2 * j], -a * tcs[2 * j + 1]) >= 0.f ? 1u : 0u;
+            }
             cb[H + slot + i] = uint8_t(k);
             dst[i] = sqrtf(a * a + b * b);
         }
@@ -206,10 +221,11 @@ __device__ __forceinline__ bool polar_encode_warp(const Layout &L, const DevPara
 //
 // The dense rotation (P.rot) takes y = R x through wbuf (D floats of shared
 // memory for this warp) and the norm of y; H D / sqrt(d) the norm of x.
+// With `rotated` the caller has already applied a dense rotation: x is y.
 template <int D>
 __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevParams &P, bool is_v, float (&x)[WarpVec<D>::E],
                                                    uint8_t *page, int pos, int lane, float (&r)[WarpVec<D>::E],
-                                                   float *wbuf) {
+                                                   float *wbuf, bool rotated = false) {
     constexpr int E = WarpVec<D>::E;
     const float sqrt_d = sqrtf(float(D));
     const int bits = is_v ? L.vbits : L.kbits;
@@ -218,7 +234,7 @@ __device__ __forceinline__ bool encode_vector_warp(const Layout &L, const DevPar
 #pragma unroll
         for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
     }
-    rotate_warp<D>(P, x, wbuf, lane);                   // y = R x
+    if (!rotated) rotate_warp<D>(P, x, wbuf, lane);     // y = R x
     if (P.rot) {
 #pragma unroll
         for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);

@@ -114,7 +114,8 @@ struct DevParams {
     const float *lv2, *bounds2;
     // polar codes (TQ_BITS_POLAR): level-1 bounds [0, 16), cos / sin of the
     // level-1 centres [16, 32) / [32, 48), level l >= 2 at 48 + 12 (l - 2):
-    // 3 bounds, 4 cos, 4 sin of its centres
+    // 3 bounds, 4 cos, 4 sin of its centres; cos / sin of the level-1 bounds
+    // 0 .. 6 at 136 + 2j, of the level-l bounds at 152 + 6 (l - 2) + 2j
     const float *polar;
     // d == 128 only (else null): 32 KB images of 128 x 128 operand tiles laid
     // out exactly as the tensor cores read them from shared memory (K-major,

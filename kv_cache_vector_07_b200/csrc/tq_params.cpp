@@ -425,20 +425,31 @@ extern "C" int tq_make_params_rot(int d, int bits, uint64_t seed, int rotation, 
     // level area and 32 of the bound area (the second one: fractional rates).
     std::vector<float> lv_code(64, 0.0f), bd_dev(64, 0.0f);
     // polar tables: level-1 bounds [0, 16), cos / sin of the level-1 centres
-    // [16, 32) / [32, 48); level l >= 2 at 48 + 12 (l - 2): 3 bounds, 4 cos, 4 sin
+    // [16, 32) / [32, 48); level l >= 2 at 48 + 12 (l - 2): 3 bounds, 4 cos, 4 sin;
+    // for the encoder's half-plane tests, cos / sin pairs of the level-1 bounds
+    // 0 .. 6 at 136 + 2j and of the level-l bounds at 152 + 6 (l - 2) + 2j (after
+    // the level tables, which end at 132 for d = 256)
     std::vector<float> polar_tab(256, 0.0f);
     const bool polar = bits == TQ_BITS_POLAR;
     if (polar) {
         for (int j = 0; j < L; ++j) p->h_levels[j] = lv[j];
         for (int j = 0; j < NB; ++j) p->h_bounds[j] = bd0[j];
         for (int j = 0; j < 15; ++j) polar_tab[j] = bd0[j];
+        for (int j = 0; j < 7; ++j) {
+            polar_tab[136 + 2 * j] = float(std::cos(double(bd0[j])));
+            polar_tab[137 + 2 * j] = float(std::sin(double(bd0[j])));
+        }
         for (int j = 0; j < 16; ++j) {
             polar_tab[16 + j] = float(std::cos(double(lv[j])));
             polar_tab[32 + j] = float(std::sin(double(lv[j])));
         }
         for (int l = 2; (1 << l) <= d; ++l) {
             const int b = 48 + 12 * (l - 2), li = 16 + 4 * (l - 2), bi = 15 + 3 * (l - 2);
-            for (int j = 0; j < 3; ++j) polar_tab[b + j] = bd0[bi + j];
+            for (int j = 0; j < 3; ++j) {
+                polar_tab[b + j] = bd0[bi + j];
+                polar_tab[152 + 6 * (l - 2) + 2 * j] = float(std::cos(double(bd0[bi + j])));
+                polar_tab[152 + 6 * (l - 2) + 2 * j + 1] = float(std::sin(double(bd0[bi + j])));
+            }
             for (int j = 0; j < 4; ++j) {
                 polar_tab[b + 4 + j] = float(std::cos(double(lv[li + j])));
                 polar_tab[b + 8 + j] = float(std::sin(double(lv[li + j])));
