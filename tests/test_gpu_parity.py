@@ -192,6 +192,39 @@ def test_decode_gqa_32x32k_sampled_rows():
 
 
 # ---------------------------------------------------------------------------
+# the alternative codecs at the size the bench times them: B=8 sequences x 8 KV
+# heads x 8,192 tokens, 32 query heads (dense rotation, 3.5-bit fractional
+# rates, polar codes); sampled (sequence, KV head) pairs: stored fields,
+# logits and outputs
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kbits,vbits,dense", [(2, 4, True), (2.5, 3.5, False), ("polar", "polar", False)])
+def test_alternative_codecs_bench_size_sampled(kbits, vbits, dense):
+    B, L, H, Hq, d, P = 8, 8192, 8, 32, 128, 64
+    n = B * L
+    K = synth.outlier_normal((n, H, d), seed=51, device=DEV)
+    V = synth.outlier_normal((n, H, d), seed=52, device=DEV)
+    Q = synth.normal((B, Hq, d), seed=54, device=DEV)
+    cd = Codec(d, kbits, True, vbits, seed=5, H=H, dense=dense)
+    bt, slots, nblk = synth.contiguous_block_table(B, L, P, device=DEV, shuffle_seed=53)
+    cache, flags = cd.encode(K, V, slots, nblk)
+    assert flags == 0
+    seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    logits = torch.full((B, Hq, L), float("nan"), device=DEV)
+    out = tqkv.decode_attn(cd.kp, cd.vp, cd.desc, Q, bt, seq, L, cache, logits=logits)
+    torch.cuda.synchronize()
+    cn = cache_np(cache)
+    sl = slots.cpu().numpy()
+    G = Hq // H
+    for b, kvh in [(0, 0), (7, 7), (3, 5)]:
+        idx = np.arange(b * L, (b + 1) * L)
+        Ek, Ev, exk, _, _ = cd.check_tokens(cn, sl[idx], f64(K[idx, kvh]), f64(V[idx, kvh]), kvh)
+        rows = list(range(kvh * G, kvh * G + G))
+        o_ref, lse_ref, lg_ref = O.attend(f64(Q[b, rows]), cd.Pk, Ek, cd.Pv, Ev, want_logits=True)
+        parity.check_logits(f64(logits[b, rows]), lg_ref, exk)
+        parity.check_outputs(f64(out[b, rows]), o_ref, cd.slack(Ev, lg_ref, lse_ref, o_ref))
+
+
+# ---------------------------------------------------------------------------
 # long context: B=1, Hq=32 over Hkv=4, L=262,144, 3-bit keys incl. QJL, 3-bit
 # values; one decode step and one 2,048-query prefill chunk (causal inside)
 # ---------------------------------------------------------------------------
