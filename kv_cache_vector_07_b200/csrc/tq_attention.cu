@@ -56,17 +56,21 @@ __global__ void __launch_bounds__(128) prep_kernel(PrepArgs a) {
 constexpr int kPQRows = 32;
 constexpr size_t kPQSmem = sizeof(float) * (128 * 129 + kPQRows * 128);
 
-// blockIdx.y selects which outputs j this block projects: all 128, or (with
-// few rows, so that more blocks share the work) a quarter of them, staging
-// only those rows of S; every block rotates its own rows.
+// blockIdx.y selects which outputs j this block projects: all 128 (JS = 1),
+// or (JS = 4, with few rows, so that more blocks share the work) a quarter of
+// them, staging only those rows of S; every block rotates its own rows.  All
+// 256 threads project: thread t takes output j0 + t % (128 / JS) for its
+// group of 4 (JS = 4) or 16 (JS = 1) rows.
+template <int JS>
 __global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
+    constexpr int JN = 128 / JS, NR = JN / 8;   // outputs of this block, rows per thread
     extern __shared__ float pq_smem[];
     float *sT = pq_smem;                        // [k][j], row stride 129 (bank spread)
     float *sq = pq_smem + 128 * 129;            // [32 rows][128]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = int64_t(blockIdx.x) * kPQRows;
-    const int jn = 128 / int(gridDim.y), j0 = int(blockIdx.y) * jn;
-    for (int i = tid; i < jn * 64; i += 256) {  // S[j][k] bf16 pairs -> sT[k][j]
+    const int j0 = int(blockIdx.y) * JN;
+    for (int i = tid; i < JN * 64; i += 256) {  // S[j][k] bf16 pairs -> sT[k][j]
         const int j = j0 + (i >> 6), k2 = (i & 63) * 2;
         const uint32_t pr = *reinterpret_cast<const uint32_t *>(a.kp.S + size_t(j) * 128 + k2);
         sT[k2 * 129 + j] = __uint_as_float(pr << 16);
@@ -92,20 +96,19 @@ __global__ void __launch_bounds__(256) prep_proj128_kernel(PrepArgs a) {
         }
     }
     __syncthreads();
-    const int j = tid & 127, g = tid >> 7;      // output j, rows 16 g .. 16 g + 15
-    if (j < j0 || j >= j0 + jn) return;
-    float acc[16];
+    const int j = j0 + tid % JN, g = tid / JN;  // output j, rows NR g .. NR g + NR - 1
+    float acc[NR];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+    for (int r = 0; r < NR; ++r) acc[r] = 0.f;
 #pragma unroll 4
     for (int k = 0; k < 128; ++k) {
         const float sv = sT[k * 129 + j];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = fmaf(sv, sq[(16 * g + r) * 128 + k], acc[r]);
+        for (int r = 0; r < NR; ++r) acc[r] = fmaf(sv, sq[(NR * g + r) * 128 + k], acc[r]);
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const int64_t row = r0 + 16 * g + r;
+    for (int r = 0; r < NR; ++r) {
+        const int64_t row = r0 + NR * g + r;
         if (row < a.rows) a.w[row * 128 + j] = acc[r];
     }
 }
@@ -639,12 +642,11 @@ int run_attention(const tq_params *kp, const tq_params *vp, const Layout &L, con
         const int64_t jobs = int64_t(s.n_seq) * L.H * 2 + rows;
         step_prep_kernel<D><<<unsigned((jobs + 7) / 8), 256, 0, st>>>(sa);
     } else if (D == 128 && L.kqjl && !kp->dev.rot) {
-        cudaError_t e = cudaFuncSetAttribute(prep_proj128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(kPQSmem));
-        if (e != cudaSuccess) return e;
         const unsigned rblocks = unsigned((rows + kPQRows - 1) / kPQRows);
-        const unsigned jsplit = rblocks < 64 ? 4u : 1u;      // few rows: four blocks per row tile
-        prep_proj128_kernel<<<dim3(rblocks, jsplit), 256, kPQSmem, st>>>(pa);
+        auto kern = rblocks < 64 ? prep_proj128_kernel<4> : prep_proj128_kernel<1>;   // few rows: 4 blocks per tile
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPQSmem));
+        if (e != cudaSuccess) return e;
+        kern<<<dim3(rblocks, rblocks < 64 ? 4u : 1u), 256, kPQSmem, st>>>(pa);
     } else {
         prep_kernel<D><<<unsigned((rows + 3) / 4), 128, 0, st>>>(pa);
         if (L.kqjl) {
