@@ -14,12 +14,17 @@
 //        64-feature chunk at a time; e makes the largest feature 1 <= |f| < 2
 //        and the scores are multiplied back by 2^e);
 //   Xf = [nhat c[code] | rho sqrt(pi/2)/m (2 s - 1)] per database vector,
-//        dequantized by the block's threads (two per database row, 32
+//        dequantized by the worker warps (two threads per database row, 32
 //        features each) into shared memory (128-byte swizzled K-major
 //        tiles) while the previous chunk's MMAs run.
-// Epilogue: two threads per query each read half of its 256 estimates from
-// TMEM and keep a running top-k (ties to the lower index); a merge kernel
-// combines the blocks' lists.
+// Two warp roles synchronized by mbarriers, two stages: the 16 worker warps
+// dequantize chunk g into stage g % 2 once the MMAs of chunk g - 2 are done;
+// the issuer warp loads the query chunk by TMA into the same stage, waits
+// for both operands and issues the chunk's MMAs.  At the end of a tile the
+// workers queue the next tile's first chunk, then read the tile's estimates
+// from TMEM (two threads per query, half of its 256 estimates each), keep a
+// running top-k (ties to the lower index) and hand the accumulators back;
+// a merge kernel combines the blocks' lists.
 //
 // Inside every 32-coordinate group the QJL features are in the order
 // (p, p + 16) for feature positions (2p, 2p + 1), so a pair of sign bits
@@ -37,7 +42,8 @@ namespace {
 
 constexpr int kQ = 256;                 // queries per block (two MMAs of M = 128, TMEM lanes)
 constexpr int kN = 256;                 // database vectors per tile (MMA N)
-constexpr int kThreads = 512;
+constexpr int kWorkers = 512;          // dequantize + scan (warps 0-15)
+constexpr int kThreads = kWorkers + 32; // + the TMA / MMA issuer warp (warp 16)
 constexpr int kTopK = 16;               // largest k this path takes
 constexpr int kSMs = 148;               // grid sizing (fixed, so workspace sizes do not depend on the device)
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
@@ -46,10 +52,10 @@ constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give 
 constexpr uint32_t SA = 0;                       // 2 stages x [256 x 64] fp16 (32 KB each)
 constexpr uint32_t SB = 65536;                   // 2 stages x [256 x 64] fp16 (32 KB each)
 constexpr uint32_t SLUT = SB + 65536;            // [256 code bytes][32 lane copies] half2 (32 KB)
-constexpr uint32_t STOPV = SLUT + 32768;         // [256 threads][k] scores
-constexpr uint32_t STOPI = STOPV + kThreads * kTopK * 4;   // [256 threads][k] indices (n_db < 2^31)
-constexpr uint32_t SBAR = STOPI + kThreads * kTopK * 4;
-constexpr uint32_t SM_TOTAL = SBAR + 64 + 1024;  // + slack for aligning the base
+constexpr uint32_t STOPV = SLUT + 32768;         // [512 workers][k] scores
+constexpr uint32_t STOPI = STOPV + kWorkers * kTopK * 4;   // [512 workers][k] indices (n_db < 2^31)
+constexpr uint32_t SBAR = STOPI + kWorkers * kTopK * 4;    // 8 mbarriers, then the abort flag
+constexpr uint32_t SM_TOTAL = SBAR + 128 + 1024;  // + slack for aligning the base
 static_assert(SM_TOTAL <= 232448, "shared memory");
 
 struct SearchTcArgs {
@@ -119,228 +125,290 @@ __device__ __forceinline__ void load_raw(const Rows &r, int kc, int p, uint4 &ra
     else raw.x = __ldg(reinterpret_cast<const uint32_t *>(r.ks + (kc - MSE_KC) * 8 + 4 * p));
 }
 
-// Per-block state of the scoring loop.
-struct Ctx {
+// Bounded wait that also gives up once another thread has given up; about a
+// second in all.  `quick` polls first, then polls with short naps (so that
+// waiting warps leave the issue slots to the working ones).
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag,
+                                              uint32_t quick) {
+    for (uint32_t i = 0; i < quick; ++i) {
+        if (tc05::mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *abort_flag) return false;
+    }
+    for (uint32_t i = 0; i < 4000000u; ++i) {
+        __nanosleep(32);
+        if (tc05::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    *abort_flag = 1u;
+    return false;
+}
+
+// Per-thread state of a dequantizing / scanning worker (warps 0-15).
+struct Work {
     uint8_t *sm;
-    uint64_t *bar_a, *bar_m;
-    const CUtensorMap *tmQ;
+    uint64_t *full_b, *empty, *acc_full, *acc_empty;
+    volatile uint32_t *abort_flag;
     uint32_t tmem;
-    int tid, warp, qt, qh, part;    // qh: query half (M = 128 tile) of this thread's query;
+    int tid, lane, warp, qh, part;  // qh: query half (M = 128 tile) of this thread's query;
                                     // part: feature half it dequantizes, vector half it scans
-    float *tv;                      // top-k scores, entry r of thread t at [r * 256 + t]
+    float *tv;                      // top-k scores, entry r of worker t at [r * 512 + t]
     int32_t *ti;
     const uint32_t *lut_lane;
-    uint32_t phase_a, phase_m, used_m;   // bit st: stage st's phase / MMAs outstanding
-    int a_pending;                  // thread 0: stage whose A load is not yet waited for
-    bool timeout;
-    int64_t tile;
-    int kc;
-    Rows cur, nxt;
 };
 
-// One 64-feature chunk on stage ST: prefetch the next chunk's bytes into
-// `nraw`, dequantize `raw` into shared memory, issue the MMAs, and after the
-// tile's last chunk scan its estimates.  Returns false to leave the loop.
-template <int D, int ST>
-__device__ __forceinline__ bool chunk_step(Ctx &c, const SearchTcArgs &a, const uint4 &raw, uint4 &nraw) {
-    constexpr int NKC = 2 * D / 64;
+// Waits decided per warp, so that warp-wide operations stay converged.
+__device__ __forceinline__ bool wait_w(const Work &w, uint64_t *bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, wait_or_abort(bar, parity, w.abort_flag, 64));
+}
+
+// Features [32 part, 32 part + 32) of chunk kc of row tid % 256 into stage
+// tile sB (16-byte pieces 4 part .. 4 part + 3 of the row).
+template <int D>
+__device__ __forceinline__ void dequant_chunk(const Work &w, const Rows &cur, int kc, const uint4 &raw, uint8_t *sB) {
     constexpr int MSE_KC = D / 64;
-    const int kc = c.kc;
-    const bool last = (ST == 1) && kc == NKC - 1;     // NKC is even: tiles end on stage 1
-    if (kc == 0) rows_scales<D>(c.cur);
-    if (last) {
-        rows_for<D>(a, c.tile + a.n_groups, c.tid, c.nxt);
-        load_raw<D>(c.nxt, 0, c.part, nraw);
+    uint32_t v[16];
+    if (kc < MSE_KC) {
+        const uint32_t cw[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
+            v[i] = hmul2u(w.lut_lane[byte * 32], cur.nh2);
+        }
     } else {
-        load_raw<D>(c.cur, kc + 1, c.part, nraw);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = cur.rh2 ^ ((raw.x << (15 - i)) & 0x80008000u);
     }
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc)
+        *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(w.tid & 255), uint32_t(4 * w.part + pc))) =
+            make_uint4(v[4 * pc], v[4 * pc + 1], v[4 * pc + 2], v[4 * pc + 3]);
+}
 
-    uint8_t *sA = c.sm + SA + ST * 32768;
-    uint8_t *sB = c.sm + SB + ST * 32768;
-    if ((c.used_m >> ST) & 1u) {        // the stage is free once the MMAs that read it completed
-        if (!tc05::mbar_wait_bounded(&c.bar_m[ST], (c.phase_m >> ST) & 1u, kPolls)) c.timeout = true;
-        c.phase_m ^= 1u << ST;
-        c.used_m &= ~(1u << ST);
-    }
-    if (c.tid == 0) {
-        tc05::mbar_expect_tx(&c.bar_a[ST], 32768);
-        tc05::tma_load_2d(sA, c.tmQ, kc * 64, c.qt * kQ, &c.bar_a[ST]);
-        c.a_pending = ST;
-    }
-    {
-        // features [32 part, 32 part + 32) of row tid % 256: 16-byte chunks 4 part .. 4 part + 3
-        uint32_t w[16];
-        if (kc < MSE_KC) {
-            const uint32_t cw[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t byte = __byte_perm(cw[i >> 2], 0, 0x4440 + (i & 3));
-                w[i] = hmul2u(c.lut_lane[byte * 32], c.cur.nh2);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = c.cur.rh2 ^ ((raw.x << (15 - i)) & 0x80008000u);
-        }
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
-            *reinterpret_cast<uint4 *>(sB + tc05::sw128_offset(uint32_t(c.tid & 255), uint32_t(4 * c.part + pc))) =
-                make_uint4(w[4 * pc], w[4 * pc + 1], w[4 * pc + 2], w[4 * pc + 3]);
-    }
-    tc05::fence_proxy_async_smem();
-    tc05::fence_before_sync();
-    if (__syncthreads_or(c.timeout)) return false;
-    if (c.tid == 0) {
-        if (!tc05::mbar_wait_bounded(&c.bar_a[ST], (c.phase_a >> ST) & 1u, kPolls)) c.timeout = true;
-        c.a_pending = -1;
-        tc05::fence_after_sync();
-        const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sB);
-        constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
-        // query half h: A rows [128 h, 128 h + 128) (16 KB apart), columns [256 h, 256 h + 256)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = tc05::desc_kmajor_sw128(bb + ks * 32);
-            const bool acc = (kc | ks) != 0;
-            tc05::mma_f16(c.tmem, tc05::desc_kmajor_sw128(aa + ks * 32), bd, idesc, acc);
-            tc05::mma_f16(c.tmem + 256, tc05::desc_kmajor_sw128(aa + 16384 + ks * 32), bd, idesc, acc);
-        }
-        tc05::mma_commit(&c.bar_m[ST]);
-    }
-    c.phase_a ^= 1u << ST;
-    c.used_m |= 1u << ST;
-
-    if (last) {
-        // the last commit covers every earlier MMA; consume both stages' phases
-#pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2) {
-            const int o = ST ^ s2;
-            if ((c.used_m >> o) & 1u) {
-                if (!tc05::mbar_wait_bounded(&c.bar_m[o], (c.phase_m >> o) & 1u, kPolls)) c.timeout = true;
-                c.phase_m ^= 1u << o;
-                c.used_m &= ~(1u << o);
-            }
-        }
-        tc05::fence_after_sync();
-        // estimates stay in accumulator units (2^-e of the true value) until the end
-        // this thread's vector half: columns [128 part, 128 part + 128) of its query half
-        const int64_t rem = a.n_db - (c.tile * kN + 128 * c.part);
-        const int lim = rem < 128 ? int(rem) : 128;
-        const int32_t id0 = int32_t(c.tile * kN + 128 * c.part);
-        const int K = a.k;
-        float kth = c.tv[(K - 1) * kThreads + c.tid];
+// Running top-k over this thread's 128 estimates of tile `tile` (its query,
+// vector half `part`), once the tile's MMAs are done (accumulator phase
+// `use`); then hand the accumulators back to the issuer.
+__device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, int64_t tile, int use) {
+    if (!wait_w(w, w.acc_full, uint32_t(use) & 1u)) return false;
+    tc05::fence_after_sync();
+    // estimates stay in accumulator units (2^-e of the true value) until the end
+    const int64_t rem = a.n_db - (tile * kN + 128 * w.part);
+    const int lim = rem < 128 ? int(rem) : 128;
+    const int32_t id0 = int32_t(tile * kN + 128 * w.part);
+    const int K = a.k;
+    float *tv = w.tv + w.tid;
+    int32_t *ti = w.ti + w.tid;
+    float kth = tv[(K - 1) * kWorkers];
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t r[32];
-            tc05::tmem_ld_32x32b_x32(
-                c.tmem + (uint32_t((c.warp & 3) * 32) << 16) + uint32_t(c.qh * 256 + 128 * c.part + cc * 32), r);
-            tc05::tmem_wait_ld();
+    for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tc05::tmem_ld_32x32b_x32(
+            w.tmem + (uint32_t((w.warp & 3) * 32) << 16) + uint32_t(w.qh * 256 + 128 * w.part + cc * 32), r);
+        tc05::tmem_wait_ld();
+        // the 32 estimates' maximum first: most groups hold no candidate
+        float m[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[e + 16]));
+#pragma unroll
+        for (int h = 8; h >= 1; h >>= 1)
+#pragma unroll
+            for (int e = 0; e < h; ++e) m[e] = fmaxf(m[e], m[e + h]);
+        if (m[0] > kth) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const float sv = __uint_as_float(r[e]);
                 if (sv > kth && cc * 32 + e < lim) {
                     int p = K - 1;
-                    while (p > 0 && sv > c.tv[(p - 1) * kThreads + c.tid]) {
-                        c.tv[p * kThreads + c.tid] = c.tv[(p - 1) * kThreads + c.tid];
-                        c.ti[p * kThreads + c.tid] = c.ti[(p - 1) * kThreads + c.tid];
+                    while (p > 0 && sv > tv[(p - 1) * kWorkers]) {
+                        tv[p * kWorkers] = tv[(p - 1) * kWorkers];
+                        ti[p * kWorkers] = ti[(p - 1) * kWorkers];
                         --p;
                     }
-                    c.tv[p * kThreads + c.tid] = sv;
-                    c.ti[p * kThreads + c.tid] = id0 + cc * 32 + e;
-                    kth = c.tv[(K - 1) * kThreads + c.tid];
+                    tv[p * kWorkers] = sv;
+                    ti[p * kWorkers] = id0 + cc * 32 + e;
+                    kth = tv[(K - 1) * kWorkers];
                 }
             }
         }
-        tc05::fence_before_sync();
-        if (__syncthreads_or(c.timeout)) return false;
-        tc05::fence_after_sync();
-        c.tile += a.n_groups;
-        c.kc = 0;
-        c.cur = c.nxt;
-    } else {
-        c.kc = kc + 1;
+        __syncwarp();                   // converged for the next warp-wide TMEM load
     }
+    tc05::fence_before_sync();
+    __syncwarp();
+    if (w.lane == 0) tc05::mbar_arrive(w.acc_empty);
     return true;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
+    constexpr int NKC = 2 * D / 64;                   // 64-feature chunks per tile
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_holder;
-    Ctx c;
-    c.sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint32_t *lut = reinterpret_cast<uint32_t *>(c.sm + SLUT);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(c.sm + SBAR);
-    c.bar_a = bars;
-    c.bar_m = bars + 2;
-    c.tmQ = &tmQ;
-    c.tid = threadIdx.x;
-    c.warp = c.tid >> 5;
-    c.qt = blockIdx.x;
-    c.qh = (c.tid >> 7) & 1;
-    c.part = c.tid >> 8;
-    const int grp = blockIdx.y, K = a.k;
-    c.tv = reinterpret_cast<float *>(c.sm + STOPV);
-    c.ti = reinterpret_cast<int32_t *>(c.sm + STOPI);
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *lut = reinterpret_cast<uint32_t *>(sm + SLUT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
+    uint64_t *full_a = bars;            // [2] query chunk landed (TMA)
+    uint64_t *full_b = bars + 2;        // [2] database chunk written (16 worker warps)
+    uint64_t *empty = bars + 4;         // [2] the MMAs that read the stage are done (commit)
+    uint64_t *acc_full = bars + 6;      // the tile's MMAs are done (commit)
+    uint64_t *acc_empty = bars + 7;     // the workers have read the tile's estimates (16 warps)
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + SBAR + 64);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qt = blockIdx.x, grp = blockIdx.y, K = a.k;
+    float *tv = reinterpret_cast<float *>(sm + STOPV);
+    int32_t *ti = reinterpret_cast<int32_t *>(sm + STOPI);
 
-    for (int i = c.tid; i < 256 * 32; i += kThreads) {
+    for (int i = tid; i < 256 * 32; i += kThreads) {
         const int e = i >> 5;
         lut[i] = h2pack(a.lv[e & 15], a.lv[e >> 4]);
     }
-    for (int r = 0; r < K; ++r) {
-        c.tv[r * kThreads + c.tid] = -INFINITY;
-        c.ti[r * kThreads + c.tid] = -1;
-    }
-    if (c.warp == 0) {
+    if (tid < kWorkers)
+        for (int r = 0; r < K; ++r) {
+            tv[r * kWorkers + tid] = -INFINITY;
+            ti[r * kWorkers + tid] = -1;
+        }
+    if (warp == 0) {
         tc05::tmem_alloc(&tmem_holder, 512);
         tc05::tmem_relinquish();
     }
-    if (c.tid == 0) {
-        for (int i = 0; i < 4; ++i) tc05::mbar_init(&bars[i], 1);
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc05::mbar_init(&full_a[i], 1);
+            tc05::mbar_init(&full_b[i], kWorkers / 32);
+            tc05::mbar_init(&empty[i], 1);
+        }
+        tc05::mbar_init(acc_full, 1);
+        tc05::mbar_init(acc_empty, kWorkers / 32);
+        *abort_flag = 0u;
         tc05::fence_mbar_init();
     }
     tc05::fence_before_sync();
     __syncthreads();
     tc05::fence_after_sync();
-    c.tmem = tmem_holder;
-    c.lut_lane = lut + (c.tid & 31);
-    c.phase_a = c.phase_m = c.used_m = 0;
-    c.a_pending = -1;
-    c.timeout = false;
-    c.tile = grp;
-    c.kc = 0;
+    const uint32_t tmem = tmem_holder;
+    bool timeout = false;
 
-    uint4 rawA = make_uint4(0, 0, 0, 0), rawB = rawA;
-    rows_for<D>(a, c.tile, c.tid, c.cur);
-    load_raw<D>(c.cur, 0, c.part, rawA);
-    while (c.tile < a.n_tiles) {
-        if (!chunk_step<D, 0>(c, a, rawA, rawB)) break;
-        if (!chunk_step<D, 1>(c, a, rawB, rawA)) break;
-    }
-    // after an early exit, let the copy and the MMAs still in flight finish
-    // before shared memory and TMEM are given back
-    if (c.a_pending >= 0 && !tc05::mbar_wait_bounded(&c.bar_a[c.a_pending], (c.phase_a >> c.a_pending) & 1u, kPolls))
-        c.timeout = true;
+    if (warp < kWorkers / 32) {
+        // ================= workers: dequantize each chunk, scan each tile
+        Work w;
+        w.sm = sm;
+        w.full_b = full_b;
+        w.empty = empty;
+        w.acc_full = acc_full;
+        w.acc_empty = acc_empty;
+        w.abort_flag = abort_flag;
+        w.tmem = tmem;
+        w.tid = tid;
+        w.lane = lane;
+        w.warp = warp;
+        w.qh = (tid >> 7) & 1;
+        w.part = tid >> 8;
+        w.tv = tv;
+        w.ti = ti;
+        w.lut_lane = lut + lane;
+        Rows cur, nxt;
+        uint4 raw = make_uint4(0, 0, 0, 0), nraw = raw;
+        int64_t tile = grp;
+        int used = 0;                   // tiles dequantized
+        uint32_t g = 0;                 // chunks dequantized
+        if (tile < a.n_tiles) {
+            rows_for<D>(a, tile, tid, cur);
+            load_raw<D>(cur, 0, w.part, raw);
+        }
+        while (tile < a.n_tiles && !timeout) {
+            for (int kc = 0; kc < NKC; ++kc) {
+                if (kc == 0) rows_scales<D>(cur);
+                if (kc == NKC - 1) {
+                    rows_for<D>(a, tile + a.n_groups, tid, nxt);
+                    load_raw<D>(nxt, 0, w.part, nraw);
+                } else {
+                    load_raw<D>(cur, kc + 1, w.part, nraw);
+                }
+                const int s = int(g & 1u);
+                // the stage is free once the MMAs that read it (chunk g - 2) are done
+                if (g >= 2 && !wait_w(w, &empty[s], ((g >> 1) - 1u) & 1u)) { timeout = true; break; }
+                dequant_chunk<D>(w, cur, kc, raw, sm + SB + uint32_t(s) * 32768u);
+                tc05::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc05::mbar_arrive(&full_b[s]);
+                ++g;
+                raw = nraw;
+                // the previous tile's estimates, once this tile's first chunk is queued
+                if (kc == 0 && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1)) { timeout = true; break; }
+            }
+            ++used;
+            tile += a.n_groups;
+            cur = nxt;
+        }
+        if (!timeout && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1)) timeout = true;
+    } else if (lane == 0) {
+        // ================= issuer: query chunks by TMA, the MMAs, the commits
+        uint32_t g = 0;
+        int64_t last = -1;              // last chunk whose MMAs were issued
+        int used = 0;
+        for (int64_t tile = grp; tile < a.n_tiles && !timeout; tile += a.n_groups, ++used) {
+            for (int kc = 0; kc < NKC; ++kc, ++g) {
+                const int s = int(g & 1u);
+                const uint32_t n = g >> 1;
+                if (g >= 2 && !wait_or_abort(&empty[s], (n - 1u) & 1u, abort_flag, 1u << 20)) {
+                    timeout = true;
+                    break;
+                }
+                uint8_t *sA = sm + SA + uint32_t(s) * 32768u;
+                tc05::mbar_expect_tx(&full_a[s], 32768);
+                tc05::tma_load_2d(sA, &tmQ, kc * 64, qt * kQ, &full_a[s]);
+                bool ok = true;
+                // the accumulators are free once the workers read the previous tile
+                if (kc == 0 && used > 0) ok = wait_or_abort(acc_empty, uint32_t(used - 1) & 1u, abort_flag, 1u << 20);
+                ok = ok && wait_or_abort(&full_b[s], n & 1u, abort_flag, 1u << 20);
+                // the copy completes whatever happened: wait for it before leaving
+                if (!tc05::mbar_wait_bounded(&full_a[s], n & 1u, kPolls)) ok = false;
+                if (!ok) {
+                    timeout = true;
+                    break;
+                }
+                tc05::fence_after_sync();
+                const uint32_t aa = tc05::smem_u32(sA), bb = tc05::smem_u32(sm + SB + uint32_t(s) * 32768u);
+                constexpr uint32_t idesc = tc05::idesc_f16_f32(128, 256);
+                // query half h: A rows [128 h, 128 h + 128) (16 KB apart), columns [256 h, 256 h + 256)
 #pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2)
-        if (((c.used_m >> s2) & 1u) && !tc05::mbar_wait_bounded(&c.bar_m[s2], (c.phase_m >> s2) & 1u, kPolls))
-            c.timeout = true;
-    const int q = c.qt * kQ + (c.tid & 255);            // = 256 qt + 128 qh + TMEM lane
-    if (q < a.n_q) {
-        const float qsc = a.qscale[q];
-        for (int r = 0; r < K; ++r) {
-            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + c.part) * K + r;
-            const int32_t id = c.ti[r * kThreads + c.tid];
-            a.part_v[o] = id >= 0 ? c.tv[r * kThreads + c.tid] * qsc : -INFINITY;
-            a.part_i[o] = id;
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t bd = tc05::desc_kmajor_sw128(bb + ks * 32);
+                    const bool acc = (kc | ks) != 0;
+                    tc05::mma_f16(tmem, tc05::desc_kmajor_sw128(aa + ks * 32), bd, idesc, acc);
+                    tc05::mma_f16(tmem + 256, tc05::desc_kmajor_sw128(aa + 16384 + ks * 32), bd, idesc, acc);
+                }
+                tc05::mma_commit(&empty[s]);
+                if (kc == NKC - 1) tc05::mma_commit(acc_full);
+                last = int64_t(g);
+            }
+        }
+        if (timeout) *abort_flag = 1u;
+        // every MMA issued completes before TMEM is given back
+        if (last >= 0 && !tc05::mbar_wait_bounded(&empty[last & 1], uint32_t(last >> 1) & 1u, kPolls))
+            timeout = true;
+    }
+    __syncwarp();
+
+    if (tid < kWorkers) {
+        const int q = qt * kQ + (tid & 255);            // = 256 qt + 128 qh + TMEM lane
+        const int part = tid >> 8;
+        if (q < a.n_q) {
+            const float qsc = a.qscale[q];
+            for (int r = 0; r < K; ++r) {
+                const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + part) * K + r;
+                const int32_t id = ti[r * kWorkers + tid];
+                a.part_v[o] = id >= 0 ? tv[r * kWorkers + tid] * qsc : -INFINITY;
+                a.part_i[o] = id;
+            }
         }
     }
     tc05::fence_before_sync();
     __syncthreads();
-    if (c.warp == 0) {
+    if (warp == 0) {
         tc05::fence_after_sync();
-        tc05::tmem_dealloc(c.tmem, 512);
+        tc05::tmem_dealloc(tmem, 512);
     }
-    if (c.timeout) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
+    if (timeout || *abort_flag) atomicOr(a.status, TQ_DEV_WAIT_TIMEOUT);
 }
 
 // Query features [n_q_pad][2d] fp16 = 2^-e [R q | S R q] (QJL half in the
