@@ -48,14 +48,15 @@ constexpr int kTopK = 16;               // largest k this path takes
 constexpr int kSMs = 148;               // grid sizing (fixed, so workspace sizes do not depend on the device)
 constexpr uint32_t kPolls = 1u << 20;   // about a second of polling, then give up
 
+constexpr int kStages = 2;              // operand stages (query + database chunk, 64 KB each)
+
 // shared layout (offsets from a 1024-aligned base)
-constexpr uint32_t SA = 0;                       // 2 stages x [256 x 64] fp16 (32 KB each)
-constexpr uint32_t SB = 65536;                   // 2 stages x [256 x 64] fp16 (32 KB each)
-constexpr uint32_t SLUT = SB + 65536;            // [256 code bytes][32 lane copies] half2 (32 KB)
-constexpr uint32_t STOPV = SLUT + 32768;         // [512 workers][k] scores
-constexpr uint32_t STOPI = STOPV + kWorkers * kTopK * 4;   // [512 workers][k] indices (n_db < 2^31)
-constexpr uint32_t SBAR = STOPI + kWorkers * kTopK * 4;    // 8 mbarriers, then the abort flag
-constexpr uint32_t SM_TOTAL = SBAR + 128 + 1024;  // + slack for aligning the base
+constexpr uint32_t SA = 0;                                  // stages x [256 x 64] fp16 queries (32 KB each)
+constexpr uint32_t SB = kStages * 32768;                    // stages x [256 x 64] fp16 database (32 KB each)
+constexpr uint32_t SLUT = SB + kStages * 32768;             // [256 code bytes][32 lane copies] half2 (32 KB)
+constexpr uint32_t SBAR = SLUT + 32768;                     // 3 x stages + 2 mbarriers
+constexpr uint32_t SFLAG = SBAR + 8 * (3 * kStages + 2);    // abort flag
+constexpr uint32_t SM_TOTAL = SFLAG + 16 + 1024;            // + slack for aligning the base
 static_assert(SM_TOTAL <= 232448, "shared memory");
 
 struct SearchTcArgs {
@@ -151,10 +152,33 @@ struct Work {
     uint32_t tmem;
     int tid, lane, warp, qh, part;  // qh: query half (M = 128 tile) of this thread's query;
                                     // part: feature half it dequantizes, vector half it scans
-    float *tv;                      // top-k scores, entry r of worker t at [r * 512 + t]
-    int32_t *ti;
     const uint32_t *lut_lane;
 };
+
+// A worker's running top-k in registers: kTopK scores in descending order
+// (ties: the earlier, lower index first) with their indices.  For k < kTopK
+// the first kTopK - k slots hold +inf sentinels that nothing displaces, so
+// the last slot is always the k-th best so far.
+struct TopK {
+    float v[kTopK];
+    int32_t i[kTopK];
+};
+
+// Insert (sv, id), known to beat the last slot: one bubble pass upwards.
+__device__ __forceinline__ void topk_insert(TopK &t, float sv, int32_t id) {
+    t.v[kTopK - 1] = sv;
+    t.i[kTopK - 1] = id;
+#pragma unroll
+    for (int j = kTopK - 1; j > 0; --j) {
+        const bool up = t.v[j] > t.v[j - 1];
+        const float a = t.v[j - 1], b = t.v[j];
+        const int32_t ia = t.i[j - 1], ib = t.i[j];
+        t.v[j - 1] = up ? b : a;
+        t.v[j] = up ? a : b;
+        t.i[j - 1] = up ? ib : ia;
+        t.i[j] = up ? ia : ib;
+    }
+}
 
 // Waits decided per warp, so that warp-wide operations stay converged.
 __device__ __forceinline__ bool wait_w(const Work &w, uint64_t *bar, uint32_t parity) {
@@ -187,17 +211,13 @@ __device__ __forceinline__ void dequant_chunk(const Work &w, const Rows &cur, in
 // Running top-k over this thread's 128 estimates of tile `tile` (its query,
 // vector half `part`), once the tile's MMAs are done (accumulator phase
 // `use`); then hand the accumulators back to the issuer.
-__device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, int64_t tile, int use) {
+__device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, int64_t tile, int use, TopK &top) {
     if (!wait_w(w, w.acc_full, uint32_t(use) & 1u)) return false;
     tc05::fence_after_sync();
     // estimates stay in accumulator units (2^-e of the true value) until the end
     const int64_t rem = a.n_db - (tile * kN + 128 * w.part);
     const int lim = rem < 128 ? int(rem) : 128;
     const int32_t id0 = int32_t(tile * kN + 128 * w.part);
-    const int K = a.k;
-    float *tv = w.tv + w.tid;
-    int32_t *ti = w.ti + w.tid;
-    float kth = tv[(K - 1) * kWorkers];
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
         uint32_t r[32];
@@ -212,21 +232,11 @@ __device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, 
         for (int h = 8; h >= 1; h >>= 1)
 #pragma unroll
             for (int e = 0; e < h; ++e) m[e] = fmaxf(m[e], m[e + h]);
-        if (m[0] > kth) {
+        if (m[0] > top.v[kTopK - 1]) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const float sv = __uint_as_float(r[e]);
-                if (sv > kth && cc * 32 + e < lim) {
-                    int p = K - 1;
-                    while (p > 0 && sv > tv[(p - 1) * kWorkers]) {
-                        tv[p * kWorkers] = tv[(p - 1) * kWorkers];
-                        ti[p * kWorkers] = ti[(p - 1) * kWorkers];
-                        --p;
-                    }
-                    tv[p * kWorkers] = sv;
-                    ti[p * kWorkers] = id0 + cc * 32 + e;
-                    kth = tv[(K - 1) * kWorkers];
-                }
+                if (sv > top.v[kTopK - 1] && cc * 32 + e < lim) topk_insert(top, sv, id0 + cc * 32 + e);
             }
         }
         __syncwarp();                   // converged for the next warp-wide TMEM load
@@ -246,32 +256,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t *lut = reinterpret_cast<uint32_t *>(sm + SLUT);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SBAR);
-    uint64_t *full_a = bars;            // [2] query chunk landed (TMA)
-    uint64_t *full_b = bars + 2;        // [2] database chunk written (16 worker warps)
-    uint64_t *empty = bars + 4;         // [2] the MMAs that read the stage are done (commit)
-    uint64_t *acc_full = bars + 6;      // the tile's MMAs are done (commit)
-    uint64_t *acc_empty = bars + 7;     // the workers have read the tile's estimates (16 warps)
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + SBAR + 64);
+    uint64_t *full_a = bars;                    // [stages] query chunk landed (TMA)
+    uint64_t *full_b = bars + kStages;          // [stages] database chunk written (16 worker warps)
+    uint64_t *empty = bars + 2 * kStages;       // [stages] the MMAs that read the stage are done (commit)
+    uint64_t *acc_full = bars + 3 * kStages;    // the tile's MMAs are done (commit)
+    uint64_t *acc_empty = acc_full + 1;         // the workers have read the tile's estimates (16 warps)
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + SFLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = blockIdx.x, grp = blockIdx.y, K = a.k;
-    float *tv = reinterpret_cast<float *>(sm + STOPV);
-    int32_t *ti = reinterpret_cast<int32_t *>(sm + STOPI);
 
     for (int i = tid; i < 256 * 32; i += kThreads) {
         const int e = i >> 5;
         lut[i] = h2pack(a.lv[e & 15], a.lv[e >> 4]);
     }
-    if (tid < kWorkers)
-        for (int r = 0; r < K; ++r) {
-            tv[r * kWorkers + tid] = -INFINITY;
-            ti[r * kWorkers + tid] = -1;
-        }
     if (warp == 0) {
         tc05::tmem_alloc(&tmem_holder, 512);
         tc05::tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             tc05::mbar_init(&full_a[i], 1);
             tc05::mbar_init(&full_b[i], kWorkers / 32);
             tc05::mbar_init(&empty[i], 1);
@@ -286,6 +289,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     tc05::fence_after_sync();
     const uint32_t tmem = tmem_holder;
     bool timeout = false;
+    TopK top;
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) {
+        top.v[j] = j < kTopK - K ? INFINITY : -INFINITY;
+        top.i[j] = -1;
+    }
 
     if (warp < kWorkers / 32) {
         // ================= workers: dequantize each chunk, scan each tile
@@ -302,8 +311,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
         w.warp = warp;
         w.qh = (tid >> 7) & 1;
         w.part = tid >> 8;
-        w.tv = tv;
-        w.ti = ti;
         w.lut_lane = lut + lane;
         Rows cur, nxt;
         uint4 raw = make_uint4(0, 0, 0, 0), nraw = raw;
@@ -323,9 +330,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
                 } else {
                     load_raw<D>(cur, kc + 1, w.part, nraw);
                 }
-                const int s = int(g & 1u);
-                // the stage is free once the MMAs that read it (chunk g - 2) are done
-                if (g >= 2 && !wait_w(w, &empty[s], ((g >> 1) - 1u) & 1u)) { timeout = true; break; }
+                const int s = int(g % kStages);
+                // the stage is free once the MMAs that read it (chunk g - stages) are done
+                if (g >= kStages && !wait_w(w, &empty[s], (g / kStages - 1u) & 1u)) { timeout = true; break; }
                 dequant_chunk<D>(w, cur, kc, raw, sm + SB + uint32_t(s) * 32768u);
                 tc05::fence_proxy_async_smem();
                 __syncwarp();
@@ -333,13 +340,16 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
                 ++g;
                 raw = nraw;
                 // the previous tile's estimates, once this tile's first chunk is queued
-                if (kc == 0 && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1)) { timeout = true; break; }
+                if (kc == 0 && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1, top)) {
+                    timeout = true;
+                    break;
+                }
             }
             ++used;
             tile += a.n_groups;
             cur = nxt;
         }
-        if (!timeout && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1)) timeout = true;
+        if (!timeout && used > 0 && !scan_tile(w, a, tile - a.n_groups, used - 1, top)) timeout = true;
     } else if (lane == 0) {
         // ================= issuer: query chunks by TMA, the MMAs, the commits
         uint32_t g = 0;
@@ -347,9 +357,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
         int used = 0;
         for (int64_t tile = grp; tile < a.n_tiles && !timeout; tile += a.n_groups, ++used) {
             for (int kc = 0; kc < NKC; ++kc, ++g) {
-                const int s = int(g & 1u);
-                const uint32_t n = g >> 1;
-                if (g >= 2 && !wait_or_abort(&empty[s], (n - 1u) & 1u, abort_flag, 1u << 20)) {
+                const int s = int(g % kStages);
+                const uint32_t n = g / kStages;
+                if (g >= kStages && !wait_or_abort(&empty[s], (n - 1u) & 1u, abort_flag, 1u << 20)) {
                     timeout = true;
                     break;
                 }
@@ -384,7 +394,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
         }
         if (timeout) *abort_flag = 1u;
         // every MMA issued completes before TMEM is given back
-        if (last >= 0 && !tc05::mbar_wait_bounded(&empty[last & 1], uint32_t(last >> 1) & 1u, kPolls))
+        if (last >= 0 &&
+            !tc05::mbar_wait_bounded(&empty[last % kStages], uint32_t(last / kStages) & 1u, kPolls))
             timeout = true;
     }
     __syncwarp();
@@ -394,12 +405,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
         const int part = tid >> 8;
         if (q < a.n_q) {
             const float qsc = a.qscale[q];
-            for (int r = 0; r < K; ++r) {
-                const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + part) * K + r;
-                const int32_t id = ti[r * kWorkers + tid];
-                a.part_v[o] = id >= 0 ? tv[r * kWorkers + tid] * qsc : -INFINITY;
-                a.part_i[o] = id;
-            }
+            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + part) * K - (kTopK - K);
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j)
+                if (j >= kTopK - K) {               // slot j is entry j - (kTopK - k) of the list
+                    const int32_t id = top.i[j];
+                    a.part_v[o + j] = id >= 0 ? top.v[j] * qsc : -INFINITY;
+                    a.part_i[o + j] = id;
+                }
         }
     }
     tc05::fence_before_sync();
