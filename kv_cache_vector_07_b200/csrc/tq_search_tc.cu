@@ -155,21 +155,38 @@ struct Work {
     const uint32_t *lut_lane;
 };
 
-// A worker's running top-k in registers: kTopK scores in descending order
-// (ties: the earlier, lower index first) with their indices.  For k < kTopK
-// the first kTopK - k slots hold +inf sentinels that nothing displaces, so
+// A worker's running top-k in registers: KT scores in descending order
+// (ties: the earlier, lower index first) with their indices, KT the
+// multiple of 4 at or above k.  For k < KT the first KT - k slots hold
+// +inf sentinels that nothing displaces, so
 // the last slot is always the k-th best so far.
+template <int KT>
 struct TopK {
-    float v[kTopK];
-    int32_t i[kTopK];
+    float v[KT];
+    int32_t i[KT];
 };
 
-// Insert (sv, id), known to beat the last slot: one bubble pass upwards.
-__device__ __forceinline__ void topk_insert(TopK &t, float sv, int32_t id) {
-    t.v[kTopK - 1] = sv;
-    t.i[kTopK - 1] = id;
+// r[e] for a run-time e (a select tree; registers cannot be indexed).
+__device__ __forceinline__ uint32_t pick32(const uint32_t (&r)[32], int e) {
+    uint32_t x[16];
 #pragma unroll
-    for (int j = kTopK - 1; j > 0; --j) {
+    for (int i = 0; i < 16; ++i) x[i] = (e & 16) ? r[i + 16] : r[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = (e & 8) ? x[i + 8] : x[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = (e & 4) ? x[i + 4] : x[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) x[i] = (e & 2) ? x[i + 2] : x[i];
+    return (e & 1) ? x[1] : x[0];
+}
+
+// Insert (sv, id), known to beat the last slot: one bubble pass upwards.
+template <int KT>
+__device__ __forceinline__ void topk_insert(TopK<KT> &t, float sv, int32_t id) {
+    t.v[KT - 1] = sv;
+    t.i[KT - 1] = id;
+#pragma unroll
+    for (int j = KT - 1; j > 0; --j) {
         const bool up = t.v[j] > t.v[j - 1];
         const float a = t.v[j - 1], b = t.v[j];
         const int32_t ia = t.i[j - 1], ib = t.i[j];
@@ -211,7 +228,8 @@ __device__ __forceinline__ void dequant_chunk(const Work &w, const Rows &cur, in
 // Running top-k over this thread's 128 estimates of tile `tile` (its query,
 // vector half `part`), once the tile's MMAs are done (accumulator phase
 // `use`); then hand the accumulators back to the issuer.
-__device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, int64_t tile, int use, TopK &top) {
+template <int KT>
+__device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, int64_t tile, int use, TopK<KT> &top) {
     if (!wait_w(w, w.acc_full, uint32_t(use) & 1u)) return false;
     tc05::fence_after_sync();
     // estimates stay in accumulator units (2^-e of the true value) until the end
@@ -232,11 +250,27 @@ __device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, 
         for (int h = 8; h >= 1; h >>= 1)
 #pragma unroll
             for (int e = 0; e < h; ++e) m[e] = fmaxf(m[e], m[e + h]);
-        if (m[0] > top.v[kTopK - 1]) {
+        if (KT > 12 && m[0] > top.v[KT - 1]) {
+            // 16 slots leave no registers for the select tree: one column at a time
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const float sv = __uint_as_float(r[e]);
-                if (sv > top.v[kTopK - 1] && cc * 32 + e < lim) topk_insert(top, sv, id0 + cc * 32 + e);
+                if (sv > top.v[KT - 1] && cc * 32 + e < lim) topk_insert(top, sv, id0 + cc * 32 + e);
+            }
+        } else if (m[0] > top.v[KT - 1]) {
+            // candidates against the threshold at the start of the group (it only
+            // rises), then taken in index order: the warp loops as often as its
+            // busiest lane has candidates, not once per candidate column
+            const float th = top.v[KT - 1];
+            uint32_t mask = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (__uint_as_float(r[e]) > th && cc * 32 + e < lim) mask |= 1u << e;
+            while (mask) {
+                const int e = __ffs(int(mask)) - 1;
+                mask &= mask - 1u;
+                const float sv = __uint_as_float(pick32(r, e));
+                if (sv > top.v[KT - 1]) topk_insert(top, sv, id0 + cc * 32 + e);
             }
         }
         __syncwarp();                   // converged for the next warp-wide TMEM load
@@ -247,7 +281,7 @@ __device__ __forceinline__ bool scan_tile(const Work &w, const SearchTcArgs &a, 
     return true;
 }
 
-template <int D>
+template <int D, int KT>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     constexpr int NKC = 2 * D / 64;                   // 64-feature chunks per tile
@@ -289,10 +323,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
     tc05::fence_after_sync();
     const uint32_t tmem = tmem_holder;
     bool timeout = false;
-    TopK top;
+    TopK<KT> top;
 #pragma unroll
-    for (int j = 0; j < kTopK; ++j) {
-        top.v[j] = j < kTopK - K ? INFINITY : -INFINITY;
+    for (int j = 0; j < KT; ++j) {
+        top.v[j] = j < KT - K ? INFINITY : -INFINITY;
         top.i[j] = -1;
     }
 
@@ -405,10 +439,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, SearchTcArgs a) {
         const int part = tid >> 8;
         if (q < a.n_q) {
             const float qsc = a.qscale[q];
-            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + part) * K - (kTopK - K);
+            const int64_t o = (int64_t(q) * (2 * a.n_groups) + 2 * grp + part) * K - (KT - K);
 #pragma unroll
-            for (int j = 0; j < kTopK; ++j)
-                if (j >= kTopK - K) {               // slot j is entry j - (kTopK - k) of the list
+            for (int j = 0; j < KT; ++j)
+                if (j >= KT - K) {                  // slot j is entry j - (KT - k) of the list
                     const int32_t id = top.i[j];
                     a.part_v[o + j] = id >= 0 ? top.v[j] * qsc : -INFINITY;
                     a.part_i[o + j] = id;
@@ -500,7 +534,8 @@ int run_tc(const tq_params *p, const Layout &L, const uint8_t *db, int64_t n_db,
     a.part_v = pv;
     a.part_i = pi;
     a.status = status;
-    auto kern = score_tc_kernel<D>;
+    auto kern = k <= 4 ? score_tc_kernel<D, 4> : k <= 8 ? score_tc_kernel<D, 8> : k <= 12 ? score_tc_kernel<D, 12>
+                                                                                     : score_tc_kernel<D, kTopK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SM_TOTAL));
     if (e != cudaSuccess) return e;
     kern<<<dim3(unsigned(n_qt), unsigned(n_groups)), kThreads, SM_TOTAL, st>>>(tm, a);

@@ -402,6 +402,7 @@ def test_search_million_vectors_properties():
     (128, 4, True, 3001, 130, 16, 1.0),      # tensor cores: two query tiles, ragged tails, largest k
     (256, 4, True, 1500, 5, 1, 1e5),         # tensor cores: k = 1, queries far beyond the fp16 range
     (512, 4, True, 777, 1, 3, 1e-6),         # tensor cores: one short tile, tiny query
+    (1024, 4, True, 2600, 33, 6, 1.0),       # tensor cores: d = 1024, k between 4 and 8
     (64, 3, True, 2000, 9, 7, 1.0),          # general kernel (head dim below the tensor-core tile)
     (128, 2, False, 999, 3, 20, 1.0),        # general kernel (MSE-only codes, k above 16)
 ])
