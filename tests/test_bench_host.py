@@ -108,3 +108,86 @@ def test_workload_configs(workload):
     assert workload in bench.WORKLOAD_METRICS and workload in bench.UNIT_NOTES
     assert workload in bench.SAMPLE_TEXT and workload in bench.SAMPLE_L
     json.dumps(cfg)
+
+
+class _FakeNVML:
+    """Read-only NVML stand-in: scripted SM clocks, power and throttle
+    reasons; any other attribute (a setter, a reset) is recorded as a
+    violation and fails."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+
+    def __init__(self, reasons):
+        self.calls, self.violations, self.reasons, self.n = [], [], reasons, 0
+
+    def nvmlInit(self):
+        self.calls.append("init")
+
+    def nvmlDeviceGetHandleByUUID(self, sel):
+        raise RuntimeError("no such uuid")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("handle", i)
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        self.n += 1
+        return (1965, 1965, 1800)[self.n % 3]
+
+    def nvmlDeviceGetMaxClockInfo(self, h, which):
+        return 1965
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 512_000                     # mW
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons
+
+    def __getattr__(self, name):
+        self.violations.append(name)
+        raise AttributeError(name)
+
+
+def test_clock_sampler_reads_nvml_and_changes_nothing(monkeypatch):
+    import time
+    import types
+    fake = _FakeNVML(reasons=_FakeNVML.nvmlClocksEventReasonSwPowerCap)
+    mod = types.ModuleType("pynvml")
+    for k in dir(_FakeNVML):
+        if k.startswith("nvml") or k.startswith("NVML"):
+            setattr(mod, k, getattr(fake, k))
+    mod.__getattr__ = fake.__getattr__
+    monkeypatch.setitem(sys.modules, "pynvml", mod)
+    s = bench.ClockSampler(0)
+    s.start()
+    time.sleep(0.05)
+    r = s.stop()
+    assert r["source"].startswith("nvml")
+    assert r["samples"] >= 5 and r["sm_mhz"] in (1800.0, 1965.0) and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 512.0
+    assert fake.violations == []
+
+
+def test_clock_sampler_parses_nvidia_smi_lines(tmp_path):
+    csv_path = tmp_path / "clocks.csv"
+    csv_path.write_text("0, 1965, 1965, 700.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                        "0, 1950, 1965, 810.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                        "0, 1800, 1965, 990.1, 0x0000000000000024, Not Active, Not Active, Active, Active\n"
+                        "garbage line\n")
+
+    class _Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.thread, s.nvml, s.proc, s.path, s.reasons = None, None, _Proc(), str(csv_path), set()
+    r = s.stop()
+    assert r["source"].startswith("nvidia-smi")
+    assert r["samples"] == 3 and r["sm_mhz"] == 1950.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"] and r["power_w_max"] == 990.1
+    assert not csv_path.exists()
